@@ -1,0 +1,127 @@
+"""CPU oracle for paged FP8 (E4M3) decode attention -- TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the bench's CPU-baseline /
+reference leg may import this package.  The CUDA product path never calls it
+and shares no code with it.
+
+The arithmetic lives in ``fpd_oracle.c`` (plain C, fp64, one (sequence, head)
+row at a time, the definition written out).  This module builds that file with
+gcc into ``libfpd_oracle.so`` next to it and exposes it through ctypes.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+from typing import Optional, Sequence, Tuple
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "fpd_oracle.c")
+_LIB = os.path.join(_HERE, "libfpd_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(src: str = _SRC, out: str = _LIB, extra_flags: Sequence[str] = ()) -> str:
+    """Compile the oracle with gcc (plain -O2, no fast-math: IEEE fp64)."""
+    cmd = ["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-pthread", *extra_flags,
+           "-o", out, src, "-lm"]
+    subprocess.run(cmd, check=True)
+    return out
+
+
+def _bind(lib):
+    u8p = ctypes.POINTER(ctypes.c_uint8)
+    lib.fpd_oracle_e4m3_to_f64.argtypes = [ctypes.c_uint8]
+    lib.fpd_oracle_e4m3_to_f64.restype = ctypes.c_double
+    lib.fpd_oracle_bf16_to_f64.argtypes = [ctypes.c_uint16]
+    lib.fpd_oracle_bf16_to_f64.restype = ctypes.c_double
+    vp = ctypes.c_void_p
+    ci, cd = ctypes.c_int, ctypes.c_double
+    lib.fpd_oracle_decode.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci,
+                                      cd, cd, cd, ci, vp, vp, vp, vp, ci, ci]
+    lib.fpd_oracle_decode.restype = ci
+    del u8p
+    return lib
+
+
+def load(path: Optional[str] = None):
+    """Load (building first if needed) the oracle library."""
+    global _lib
+    if path is not None:
+        return _bind(ctypes.CDLL(path))
+    with _lock:
+        if _lib is None:
+            stale = (not os.path.exists(_LIB)) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC)
+            if stale:
+                build()
+            _lib = _bind(ctypes.CDLL(_LIB))
+    return _lib
+
+
+def e4m3_to_f64(code: int, lib=None) -> float:
+    return (lib or load()).fpd_oracle_e4m3_to_f64(int(code))
+
+
+def bf16_to_f64(bits: int, lib=None) -> float:
+    return (lib or load()).fpd_oracle_bf16_to_f64(int(bits))
+
+
+def _ptr(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def decode(q, k_cache, v_cache, block_table, seq_lens, *, k_scale, v_scale, sm_scale,
+           window_left=-1, sinks=None, rows=None, threads=None, lib=None
+           ) -> Tuple[np.ndarray, np.ndarray]:
+    """fp64 decode attention.
+
+    Arrays are numpy: q uint16 (bf16 bits) [B,Hq,D]; k/v_cache uint8 E4M3 codes
+    [num_blocks, bt, Hkv, D]; block_table int32 [B, max_blocks]; seq_lens int32
+    [B]; sinks float32 [Hq] or None.  ``rows`` optionally lists flat
+    ``b * Hq + h`` rows to compute (others are left NaN).  Returns
+    (out float64 [B, Hq, D], lse float64 [B, Hq]).
+    """
+    lib = lib or load()
+    q = np.ascontiguousarray(q, dtype=np.uint16)
+    k_cache = np.ascontiguousarray(k_cache, dtype=np.uint8)
+    v_cache = np.ascontiguousarray(v_cache, dtype=np.uint8)
+    block_table = np.ascontiguousarray(block_table, dtype=np.int32)
+    seq_lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    B, Hq, D = q.shape
+    num_blocks, bt, Hkv, D2 = k_cache.shape
+    assert D2 == D and v_cache.shape == k_cache.shape
+    assert block_table.shape[0] == B and seq_lens.shape == (B,)
+    max_blocks = block_table.shape[1]
+    if sinks is not None:
+        sinks = np.ascontiguousarray(sinks, dtype=np.float32)
+        assert sinks.shape == (Hq,)
+    out = np.full((B, Hq, D), np.nan, dtype=np.float64)
+    lse = np.full((B, Hq), np.nan, dtype=np.float64)
+    rows_arr = None
+    n_rows = 0
+    if rows is not None:
+        rows_arr = np.ascontiguousarray(rows, dtype=np.int32)
+        n_rows = int(rows_arr.size)
+    if threads is None:
+        threads = os.cpu_count() or 1
+    st = lib.fpd_oracle_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                               _ptr(seq_lens), B, Hq, Hkv, D, num_blocks, bt, max_blocks,
+                               float(k_scale), float(v_scale), float(sm_scale), int(window_left),
+                               _ptr(sinks), _ptr(out), _ptr(lse), _ptr(rows_arr), n_rows,
+                               int(threads))
+    if st != 0:
+        raise ValueError(f"oracle rejected the inputs (status {st})")
+    return out, lse
+
+
+def decode_workload(wl, rows=None, threads=None, lib=None, window_left=None, sinks="keep"):
+    """Oracle on a ``workloads.Workload``."""
+    return decode(wl.q, wl.k_cache, wl.v_cache, wl.block_table, wl.seq_lens,
+                  k_scale=wl.k_scale, v_scale=wl.v_scale, sm_scale=wl.sm_scale,
+                  window_left=wl.window_left if window_left is None else window_left,
+                  sinks=wl.sinks if isinstance(sinks, str) else sinks,
+                  rows=rows, threads=threads, lib=lib)

@@ -1,0 +1,235 @@
+/*
+ * fpd_oracle.c -- the CPU oracle for paged FP8 (E4M3) decode attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the bench's
+ * CPU-baseline leg load this library; the product path never calls it.
+ * It shares no code with the CUDA kernels.
+ *
+ * What it computes, in fp64, for every sequence b and query head h.  The
+ * operation is the one the grouped-nf4-gemm solutions page
+ * "fp8-paged-attention-for-moe-serving" names (its title and summary): one
+ * decode query per sequence attending, through a block table, to a paged
+ * E4M3 K/V cache, with an optional sliding window, optional attention sinks
+ * and a caller-chosen softmax scale.
+ *
+ *   g     = Hq / Hkv, kvh = h / g            (consecutive query heads share a
+ *                                           KV head: GQA)
+ *   L     = seq_lens[b]
+ *   start = window_left >= 0 ? max(0, L - 1 - window_left) : 0
+ *           (FlashInfer's window_left, passed through by the vLLM FlashInfer
+ *            backend in the NVFP4 KV-cache gist: the query sees itself and the
+ *            window_left keys before it)
+ *   for j in [start, L):   page = block_table[b][j / bt], slot = j % bt
+ *       k_j = k_scale * e4m3(k_cache[page][slot][kvh][:])
+ *       v_j = v_scale * e4m3(v_cache[page][slot][kvh][:])
+ *       s_j = sm_scale * sum_d q[b][h][d] * k_j[d]
+ *   sigma = sinks ? sinks[h] : -inf         (a sink is a logit with no value:
+ *                                           it only enters the denominator)
+ *   m   = max(max_j s_j, sigma)
+ *   Z   = sum_j exp(s_j - m) + exp(sigma - m)
+ *   out = sum_j exp(s_j - m) / Z * v_j
+ *   lse = m + ln Z                          (natural log, sink included)
+ *
+ * Per-tensor scales: the cache writer of the gist stores x / scale, so a stored
+ * code decodes to e4m3(code) * scale.
+ *
+ * E4M3 is the OCP "e4m3fn" format (the CUDA type __nv_fp8_e4m3 named in the
+ * gist's quantisation helpers): 1 sign, 4 exponent (bias 7), 3 mantissa bits;
+ * exponent 0 is subnormal; S.1111.111 is NaN; there are no infinities.
+ *
+ * Degenerate cases: L == 0 gives out = 0 and lse = sigma (-inf without sinks).
+ * A stored NaN code inside the attended range propagates NaN (plain
+ * arithmetic); codes outside the attended range are never read.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* E4M3 (e4m3fn) code -> exact real value. */
+double fpd_oracle_e4m3_to_f64(uint8_t code)
+{
+    const int sign = code >> 7;
+    const int expo = (code >> 3) & 0xF;
+    const int mant = code & 0x7;
+    double mag;
+    if (expo == 0xF && mant == 0x7)
+        return NAN;
+    if (expo == 0)
+        mag = ldexp((double)mant / 8.0, -6);          /* subnormal: 2^-6 * m/8 */
+    else
+        mag = ldexp(1.0 + (double)mant / 8.0, expo - 7); /* normal: 2^(e-7) * (1+m/8) */
+    return sign ? -mag : mag;
+}
+
+/* bf16 bit pattern -> real value (bf16 is the top half of an IEEE binary32). */
+double fpd_oracle_bf16_to_f64(uint16_t bits)
+{
+    uint32_t u = (uint32_t)bits << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+typedef struct {
+    const uint16_t *q;
+    const uint8_t *k_cache, *v_cache;
+    const int32_t *block_table, *seq_lens;
+    int B, Hq, Hkv, D, num_blocks, bt, max_blocks;
+    double k_scale, v_scale, sm_scale;
+    int window_left;
+    const float *sinks;
+    double *out, *lse;
+    const int32_t *rows; /* list of b * Hq + h to compute, or NULL for all */
+    int n_rows;
+    int next;            /* work counter */
+    int status;
+    pthread_mutex_t mu;
+} job_t;
+
+/* Byte offset of element [page][slot][kvh][0] in a [num_blocks, bt, Hkv, D] cache. */
+static size_t cache_row(const job_t *J, int page, int slot, int kvh)
+{
+    return (((size_t)page * J->bt + slot) * J->Hkv + kvh) * (size_t)J->D;
+}
+
+static int one_row(const job_t *J, int row, double *s, double *acc)
+{
+    const int b = row / J->Hq, h = row % J->Hq;
+    const int g = J->Hq / J->Hkv;
+    const int kvh = h / g;
+    const int D = J->D;
+    const int L = J->seq_lens[b];
+    double *o = J->out + (size_t)row * D;
+    const uint16_t *qr = J->q + (size_t)row * D;
+    const double sigma = J->sinks ? (double)J->sinks[h] : -INFINITY;
+    int start, j, d;
+    double m, Z;
+
+    if (L < 0 || L > J->max_blocks * J->bt)
+        return -2;
+    start = (J->window_left >= 0) ? L - 1 - J->window_left : 0;
+    if (start < 0)
+        start = 0;
+
+    /* logits */
+    m = sigma;
+    for (j = start; j < L; ++j) {
+        const int page = J->block_table[(size_t)b * J->max_blocks + j / J->bt];
+        const uint8_t *kr;
+        double dot = 0.0;
+        if (page < 0 || page >= J->num_blocks)
+            return -3;
+        kr = J->k_cache + cache_row(J, page, j % J->bt, kvh);
+        for (d = 0; d < D; ++d)
+            dot += fpd_oracle_bf16_to_f64(qr[d]) * (J->k_scale * fpd_oracle_e4m3_to_f64(kr[d]));
+        s[j - start] = J->sm_scale * dot;
+        if (s[j - start] > m || isnan(s[j - start]))
+            m = s[j - start];
+    }
+
+    /* softmax weights, denominator and weighted sum of values */
+    for (d = 0; d < D; ++d)
+        acc[d] = 0.0;
+    Z = 0.0;
+    if (m == -INFINITY) { /* no keys and no sink */
+        for (d = 0; d < D; ++d)
+            o[d] = 0.0;
+        J->lse[row] = -INFINITY;
+        return 0;
+    }
+    for (j = start; j < L; ++j) {
+        const int page = J->block_table[(size_t)b * J->max_blocks + j / J->bt];
+        const uint8_t *vr = J->v_cache + cache_row(J, page, j % J->bt, kvh);
+        const double p = exp(s[j - start] - m);
+        Z += p;
+        for (d = 0; d < D; ++d)
+            acc[d] += p * (J->v_scale * fpd_oracle_e4m3_to_f64(vr[d]));
+    }
+    Z += exp(sigma - m);
+    for (d = 0; d < D; ++d)
+        o[d] = acc[d] / Z;
+    J->lse[row] = m + log(Z);
+    return 0;
+}
+
+static void *worker(void *arg)
+{
+    job_t *J = (job_t *)arg;
+    const int total = J->rows ? J->n_rows : J->B * J->Hq;
+    int maxL = J->max_blocks * J->bt;
+    double *s = (double *)malloc(sizeof(double) * (size_t)(maxL > 0 ? maxL : 1));
+    double *acc = (double *)malloc(sizeof(double) * (size_t)J->D);
+    for (;;) {
+        int i, row, st;
+        pthread_mutex_lock(&J->mu);
+        i = J->next++;
+        pthread_mutex_unlock(&J->mu);
+        if (i >= total)
+            break;
+        row = J->rows ? J->rows[i] : i;
+        st = one_row(J, row, s, acc);
+        if (st != 0) {
+            pthread_mutex_lock(&J->mu);
+            if (J->status == 0)
+                J->status = st;
+            pthread_mutex_unlock(&J->mu);
+        }
+    }
+    free(s);
+    free(acc);
+    return NULL;
+}
+
+/*
+ * Decode attention over the paged cache.
+ *   q            bf16 bits [B, Hq, D]
+ *   k/v_cache    E4M3 codes [num_blocks, bt, Hkv, D]
+ *   block_table  [B, max_blocks], seq_lens [B]
+ *   sinks        float [Hq] or NULL
+ *   out          double [B * Hq, D]  (only the listed rows are written)
+ *   lse          double [B * Hq]
+ *   rows/n_rows  rows (b * Hq + h) to compute; rows == NULL computes all.
+ *   n_threads    worker threads (<= 0: 1)
+ * Returns 0, -1 for bad shapes, -2 for a sequence length outside
+ * [0, max_blocks * bt], -3 for a block-table entry outside [0, num_blocks).
+ */
+int fpd_oracle_decode(const uint16_t *q, const uint8_t *k_cache, const uint8_t *v_cache,
+                      const int32_t *block_table, const int32_t *seq_lens,
+                      int B, int Hq, int Hkv, int D, int num_blocks, int bt, int max_blocks,
+                      double k_scale, double v_scale, double sm_scale, int window_left,
+                      const float *sinks, double *out, double *lse,
+                      const int32_t *rows, int n_rows, int n_threads)
+{
+    job_t J;
+    pthread_t *th;
+    int t, i;
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || D <= 0 || bt <= 0 || max_blocks < 0 ||
+        num_blocks < 0)
+        return -1;
+    if (rows) {
+        for (i = 0; i < n_rows; ++i)
+            if (rows[i] < 0 || rows[i] >= B * Hq)
+                return -1;
+    }
+    memset(&J, 0, sizeof J);
+    J.q = q; J.k_cache = k_cache; J.v_cache = v_cache;
+    J.block_table = block_table; J.seq_lens = seq_lens;
+    J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.D = D; J.num_blocks = num_blocks; J.bt = bt;
+    J.max_blocks = max_blocks;
+    J.k_scale = k_scale; J.v_scale = v_scale; J.sm_scale = sm_scale;
+    J.window_left = window_left; J.sinks = sinks; J.out = out; J.lse = lse;
+    J.rows = rows; J.n_rows = n_rows;
+    pthread_mutex_init(&J.mu, NULL);
+    if (n_threads < 1)
+        n_threads = 1;
+    th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)n_threads);
+    for (t = 0; t < n_threads; ++t)
+        pthread_create(&th[t], NULL, worker, &J);
+    for (t = 0; t < n_threads; ++t)
+        pthread_join(th[t], NULL);
+    free(th);
+    pthread_mutex_destroy(&J.mu);
+    return J.status;
+}

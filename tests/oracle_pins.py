@@ -1,0 +1,283 @@
+"""Pins that tie the CPU oracle to things other than itself.
+
+Each ``pin_*`` function takes a loaded oracle library (ctypes handle) and raises
+AssertionError when the oracle disagrees with
+
+* a library routine that computes the same thing (torch's float8_e4m3fn and
+  bfloat16 casts; torch's scaled_dot_product_attention in float64 with GQA,
+  the sink given as an extra zero-valued key whose additive mask is the sink
+  logit; scipy's logsumexp over numpy-matmul scores),
+* a closed form (K == 0 gives the mean of the attended values and lse = ln n;
+  a window of 0 keeps one key; constant value rows return that constant times
+  the non-sink probability mass; the E4M3 format's extreme values), or
+* an invariant (physical-page permutation, window >= L - 1, a -inf sink,
+  k_scale <-> sm_scale exchange, v_scale linearity, identical query rows).
+
+``tests/test_oracle_pins.py`` runs them against the oracle; the mutation test
+runs them against deliberately broken copies of the oracle and requires every
+copy to fail at least one pin.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import scipy.special
+import torch
+import torch.nn.functional as F
+
+import oracle
+from fp8_paged_decode_b200 import workloads as W
+
+
+# ---------------------------------------------------------------- helpers --
+
+def e4m3_library(codes: np.ndarray) -> np.ndarray:
+    """E4M3 codes -> float64 by torch's float8_e4m3fn cast (library routine)."""
+    t = torch.from_numpy(np.ascontiguousarray(codes, dtype=np.uint8)).view(torch.float8_e4m3fn)
+    return t.to(torch.float64).numpy()
+
+
+def bf16_library(bits: np.ndarray) -> np.ndarray:
+    t = torch.from_numpy(np.ascontiguousarray(bits, dtype=np.uint16).view(np.int16)).view(torch.bfloat16)
+    return t.to(torch.float64).numpy()
+
+
+def run(lib, wl, **kw):
+    return oracle.decode_workload(wl, lib=lib, threads=4, **kw)
+
+
+def library_attention(wl):
+    """Dense attention from the generator's per-sequence dense codes, by torch SDPA
+    (out) and scipy logsumexp (lse), in float64."""
+    assert wl.k_dense is not None
+    B, Hq, Hkv, D = wl.B, wl.Hq, wl.Hkv, wl.D
+    g = Hq // Hkv
+    out = np.zeros((B, Hq, D))
+    lse = np.zeros((B, Hq))
+    qf = bf16_library(wl.q)
+    for b in range(B):
+        L = int(wl.seq_lens[b])
+        start = max(0, L - 1 - wl.window_left) if wl.window_left >= 0 else 0
+        K = e4m3_library(wl.k_dense[b][start:L]) * wl.k_scale   # [n, Hkv, D]
+        V = e4m3_library(wl.v_dense[b][start:L]) * wl.v_scale
+        n = L - start
+        sig = None if wl.sinks is None else wl.sinks.astype(np.float64)
+        if n == 0 and sig is None:
+            out[b] = 0.0
+            lse[b] = -np.inf
+            continue
+        extra = 0 if sig is None else 1
+        Kt = torch.zeros((1, Hkv, n + extra, D), dtype=torch.float64)
+        Vt = torch.zeros((1, Hkv, n + extra, D), dtype=torch.float64)
+        Kt[0, :, :n] = torch.from_numpy(K).permute(1, 0, 2)
+        Vt[0, :, :n] = torch.from_numpy(V).permute(1, 0, 2)
+        mask = torch.zeros((1, Hq, 1, n + extra), dtype=torch.float64)
+        if sig is not None:
+            mask[0, :, 0, n] = torch.from_numpy(sig)
+        qt = torch.from_numpy(qf[b]).reshape(1, Hq, 1, D)
+        o = F.scaled_dot_product_attention(qt, Kt, Vt, attn_mask=mask, scale=wl.sm_scale,
+                                           enable_gqa=True)
+        out[b] = o[0, :, 0, :].numpy()
+        # scores by numpy matmul, lse by scipy
+        Kh = np.repeat(K, g, axis=1)                     # [n, Hq, D], head h -> kv head h // g
+        s = wl.sm_scale * np.einsum("hd,nhd->hn", qf[b], Kh)
+        if sig is not None:
+            s = np.concatenate([s, sig[:, None]], axis=1)
+        lse[b] = scipy.special.logsumexp(s, axis=1)
+    return out, lse
+
+
+def close(a, b, rtol=1e-12, atol=1e-12, what=""):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    same_inf = np.isinf(a) & np.isinf(b) & (np.sign(a) == np.sign(b))
+    ok = same_inf | (np.abs(a - b) <= atol + rtol * np.abs(b))
+    if not ok.all():
+        i = np.argwhere(~ok)[0]
+        raise AssertionError(f"{what}: mismatch at {tuple(i)}: {a[tuple(i)]!r} vs {b[tuple(i)]!r}")
+
+
+def small_cases():
+    """Small shapes covering GQA 1..16, D 64/128, page sizes 16/32/64, windows, sinks,
+    ragged lengths (1, bt-1, bt, bt+1, multi-page) and an empty sequence."""
+    return [
+        W.make_custom(B=2, Hq=8, Hkv=2, D=128, block_tokens=16, seq_lens=[37, 300], seed=0,
+                      keep_dense=True, sm_scale=1 / math.sqrt(128), name="tiny-like"),
+        W.make_custom(B=5, Hq=4, Hkv=4, D=64, block_tokens=16, seq_lens=[1, 15, 16, 17, 70],
+                      seed=11, keep_dense=True),
+        W.make_custom(B=3, Hq=16, Hkv=2, D=64, block_tokens=32, seq_lens=[200, 33, 64],
+                      window_left=40, sinks=True, sm_scale=0.125, seed=12, keep_dense=True),
+        W.make_custom(B=3, Hq=32, Hkv=2, D=128, block_tokens=64, seq_lens=[129, 5, 64],
+                      window_left=3, sinks=True, sm_scale=0.1, sigma=2.0, seed=13, keep_dense=True),
+        W.make_custom(B=2, Hq=4, Hkv=2, D=128, block_tokens=16, seq_lens=[0, 23],
+                      sinks=True, seed=14, keep_dense=True),
+    ]
+
+
+# ------------------------------------------------------------------- pins --
+
+def pin_e4m3_codes(lib):
+    codes = np.arange(256, dtype=np.uint8)
+    mine = np.array([lib.fpd_oracle_e4m3_to_f64(int(c)) for c in codes])
+    ref = e4m3_library(codes)
+    nan = np.isnan(ref)
+    assert (np.isnan(mine) == nan).all(), "NaN codes differ"
+    assert (mine[~nan] == ref[~nan]).all(), "E4M3 values differ from torch.float8_e4m3fn"
+    # format facts: only 0x7F / 0xFF are NaN; max finite 448 at 0x7E; smallest
+    # normal 2^-6 at 0x08; smallest subnormal 2^-9 at 0x01; sign symmetry.
+    assert set(np.flatnonzero(np.isnan(mine)).tolist()) == {0x7F, 0xFF}
+    assert mine[0x7E] == 448.0 and mine[0x08] == 2.0 ** -6 and mine[0x01] == 2.0 ** -9
+    assert (mine[0x80:0xFF] == -mine[0x00:0x7F]).all()
+    pos = mine[0x00:0x7F]
+    assert (np.diff(pos) > 0).all(), "positive codes must increase monotonically"
+
+
+def pin_bf16(lib):
+    rng = np.random.default_rng(7)
+    bits = np.concatenate([rng.integers(0, 1 << 16, 4000, dtype=np.uint32).astype(np.uint16),
+                           np.array([0x0000, 0x8000, 0x3F80, 0xBF80, 0x0001, 0x7F7F], np.uint16)])
+    ref = bf16_library(bits)
+    mine = np.array([lib.fpd_oracle_bf16_to_f64(int(x)) for x in bits])
+    nan = np.isnan(ref)
+    assert (np.isnan(mine) == nan).all()
+    assert (mine[~nan] == ref[~nan]).all(), "bf16 decode differs from torch.bfloat16"
+
+
+def pin_library_attention(lib, cases=None):
+    for wl in cases or small_cases():
+        out, lse = run(lib, wl)
+        ref_out, ref_lse = library_attention(wl)
+        close(out, ref_out, rtol=1e-10, atol=1e-12, what=f"out vs SDPA ({wl.name})")
+        close(lse, ref_lse, rtol=1e-12, atol=1e-12, what=f"lse vs logsumexp ({wl.name})")
+
+
+def pin_zero_keys(lib):
+    """K == 0: every logit is 0, so out = mean of attended values (times the
+    non-sink mass) and lse = ln n (or ln(n + e^sigma))."""
+    for sinks, W_ in ((False, -1), (True, 20)):
+        wl = W.make_custom(B=3, Hq=8, Hkv=2, D=64, block_tokens=16, seq_lens=[1, 50, 97],
+                           window_left=W_, sinks=sinks, seed=21, keep_dense=True)
+        wl.k_cache[:] = 0
+        out, lse = run(lib, wl)
+        for b in range(wl.B):
+            L = int(wl.seq_lens[b])
+            start = max(0, L - 1 - W_) if W_ >= 0 else 0
+            n = L - start
+            V = e4m3_library(wl.v_dense[b][start:L]) * wl.v_scale   # [n, Hkv, D]
+            for h in range(wl.Hq):
+                sig = wl.sinks[h] if sinks else -np.inf
+                Z = n + math.exp(sig)
+                close(lse[b, h], math.log(Z), what="lse, K=0")
+                close(out[b, h], V[:, h // wl.groups, :].sum(0) / Z, atol=1e-13, what="out, K=0")
+
+
+def pin_window_zero(lib):
+    """window_left = 0 keeps only the newest key: out = v_last * p, lse = logaddexp(s, sigma)."""
+    wl = W.make_custom(B=3, Hq=4, Hkv=1, D=128, block_tokens=32, seq_lens=[1, 33, 90],
+                       window_left=0, sinks=True, seed=22, keep_dense=True)
+    out, lse = run(lib, wl)
+    qf = bf16_library(wl.q)
+    for b in range(wl.B):
+        L = int(wl.seq_lens[b])
+        k = e4m3_library(wl.k_dense[b][L - 1, 0]) * wl.k_scale
+        v = e4m3_library(wl.v_dense[b][L - 1, 0]) * wl.v_scale
+        for h in range(wl.Hq):
+            s = wl.sm_scale * float(np.dot(qf[b, h], k))
+            sig = float(wl.sinks[h])
+            l_ref = np.logaddexp(s, sig)
+            close(lse[b, h], l_ref, what="lse, W=0")
+            close(out[b, h], v * math.exp(s - l_ref), atol=1e-13, what="out, W=0")
+
+
+def pin_constant_values(lib):
+    """Every value row of KV head j equal to c_j: out[h] = c_{h//g} (1 - e^(sigma - lse))."""
+    wl = W.make_custom(B=2, Hq=8, Hkv=4, D=64, block_tokens=16, seq_lens=[40, 77],
+                       window_left=30, sinks=True, seed=23)
+    consts = np.array([0x38, 0xB4, 0x41, 0x02], dtype=np.uint8)   # 1.0, -0.75, 2.25, 2^-8
+    for j in range(wl.Hkv):
+        wl.v_cache[:, :, j, :] = consts[j]
+    out, lse = run(lib, wl)
+    cval = e4m3_library(consts) * wl.v_scale
+    for b in range(wl.B):
+        for h in range(wl.Hq):
+            mass = 1.0 - math.exp(float(wl.sinks[h]) - lse[b, h])
+            close(out[b, h], np.full(wl.D, cval[h // wl.groups] * mass), rtol=1e-12, atol=1e-15,
+                  what="constant V rows")
+
+
+def pin_invariants(lib):
+    wl = W.make_custom(B=3, Hq=8, Hkv=2, D=128, block_tokens=16, seq_lens=[5, 64, 131],
+                       sinks=True, seed=24, sm_scale=0.09)
+    out, lse = run(lib, wl)
+
+    # physical page permutation (bitwise)
+    rng = np.random.default_rng(5)
+    perm = rng.permutation(wl.num_blocks)            # new position of each old page
+    inv = np.argsort(perm)
+    k2 = wl.k_cache[inv]
+    v2 = wl.v_cache[inv]
+    t2 = np.where(wl.block_table >= 0, perm[np.maximum(wl.block_table, 0)], -1).astype(np.int32)
+    o2, l2 = oracle.decode(wl.q, k2, v2, t2, wl.seq_lens, k_scale=wl.k_scale, v_scale=wl.v_scale,
+                           sm_scale=wl.sm_scale, window_left=-1, sinks=wl.sinks, lib=lib)
+    assert np.array_equal(o2, out) and np.array_equal(l2, lse), "page permutation changed the result"
+
+    # a window covering the whole sequence equals no window (bitwise)
+    for Wl in (int(wl.seq_lens.max()) - 1, int(wl.seq_lens.max()), 10 ** 6):
+        o3, l3 = run(lib, wl, window_left=Wl)
+        assert np.array_equal(o3, out) and np.array_equal(l3, lse), f"window {Wl} != no window"
+
+    # a -inf sink equals no sink
+    o4, l4 = run(lib, wl, sinks=None)
+    o5, l5 = run(lib, wl, sinks=np.full(wl.Hq, -np.inf, np.float32))
+    assert np.array_equal(o4, o5) and np.array_equal(l4, l5), "-inf sink != no sink"
+    # and a huge sink absorbs all mass
+    o6, l6 = run(lib, wl, sinks=np.full(wl.Hq, 1e4, np.float32))
+    close(l6, np.full_like(l6, 1e4), what="huge sink lse")
+    assert np.abs(o6).max() == 0.0, "huge sink must leave zero output"
+
+    # k_scale * a  <->  sm_scale * a
+    a = 1.75
+    oa, la = oracle.decode(wl.q, wl.k_cache, wl.v_cache, wl.block_table, wl.seq_lens,
+                           k_scale=wl.k_scale * a, v_scale=wl.v_scale, sm_scale=wl.sm_scale,
+                           sinks=wl.sinks, lib=lib)
+    ob, lb = oracle.decode(wl.q, wl.k_cache, wl.v_cache, wl.block_table, wl.seq_lens,
+                           k_scale=wl.k_scale, v_scale=wl.v_scale, sm_scale=wl.sm_scale * a,
+                           sinks=wl.sinks, lib=lib)
+    close(oa, ob, rtol=1e-11, atol=1e-14, what="k_scale/sm_scale exchange")
+    close(la, lb, rtol=1e-12, what="k_scale/sm_scale exchange (lse)")
+    # v_scale is linear (doubling is exact)
+    oc, lc = oracle.decode(wl.q, wl.k_cache, wl.v_cache, wl.block_table, wl.seq_lens,
+                           k_scale=wl.k_scale, v_scale=wl.v_scale * 2, sm_scale=wl.sm_scale,
+                           sinks=wl.sinks, lib=lib)
+    assert np.array_equal(oc, 2 * out) and np.array_equal(lc, lse), "v_scale not linear"
+
+    # identical query rows inside one GQA group give identical rows
+    q2 = wl.q.copy()
+    g = wl.groups
+    for j in range(wl.Hkv):
+        q2[:, j * g:(j + 1) * g, :] = q2[:, j * g:j * g + 1, :]
+    od, ld = oracle.decode(q2, wl.k_cache, wl.v_cache, wl.block_table, wl.seq_lens,
+                           k_scale=wl.k_scale, v_scale=wl.v_scale, sm_scale=wl.sm_scale,
+                           sinks=np.repeat(wl.sinks[::g], g), lib=lib)
+    for j in range(wl.Hkv):
+        for h in range(j * g, (j + 1) * g):
+            assert np.array_equal(od[:, h], od[:, j * g]) and np.array_equal(ld[:, h], ld[:, j * g])
+
+
+def pin_softmax_identity(lib):
+    """sum_j e^(s_j - lse) + e^(sigma - lse) = 1 with s_j from numpy."""
+    wl = W.make_custom(B=2, Hq=4, Hkv=2, D=64, block_tokens=16, seq_lens=[3, 45], sinks=True,
+                       sm_scale=0.3, seed=25, keep_dense=True)
+    _, lse = run(lib, wl)
+    qf = bf16_library(wl.q)
+    for b in range(wl.B):
+        K = e4m3_library(wl.k_dense[b]) * wl.k_scale
+        for h in range(wl.Hq):
+            s = wl.sm_scale * K[:, h // wl.groups, :] @ qf[b, h]
+            tot = np.exp(s - lse[b, h]).sum() + math.exp(float(wl.sinks[h]) - lse[b, h])
+            assert abs(tot - 1.0) < 1e-12, f"probabilities sum to {tot}"
+
+
+ALL_PINS = [pin_e4m3_codes, pin_bf16, pin_library_attention, pin_zero_keys, pin_window_zero,
+            pin_constant_values, pin_invariants, pin_softmax_identity]

@@ -1,0 +1,68 @@
+"""Stored oracle values and the input generator's recipe (no GPU)."""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fp8_paged_decode_b200 import workloads as W
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def test_tiny_golden_unchanged():
+    wl = W.make_workload("tiny")
+    out, lse = oracle.decode_workload(wl, threads=2)
+    rows = [l.split() for l in open(os.path.join(HERE, "golden", "tiny_oracle.txt"))
+            if not l.startswith("#")]
+    assert len(rows) == wl.B * wl.Hq
+    for r in rows:
+        b, h = int(r[0]), int(r[1])
+        vals = [float(x) for x in r[2:]]
+        o = out[b, h]
+        got = [lse[b, h], o[0], o[1], o[63], o[127], o.sum()]
+        np.testing.assert_allclose(got, vals, rtol=1e-13, atol=1e-15)
+
+
+def test_generator_recipe():
+    wl = W.make_custom(B=3, Hq=8, Hkv=2, D=64, block_tokens=16, seq_lens=[5, 40, 100],
+                       window_left=20, sinks=True, seed=9, keep_dense=True)
+    # table: every used page distinct and inside the pool, unused slots -1
+    used = []
+    for b in range(wl.B):
+        n = -(-int(wl.seq_lens[b]) // 16)
+        assert (wl.block_table[b, :n] >= 0).all() and (wl.block_table[b, n:] == -1).all()
+        used += wl.block_table[b, :n].tolist()
+    assert len(set(used)) == len(used) and max(used) < wl.num_blocks
+    # scale = amax/448 over attended values: the largest attended code is +-448
+    att = np.concatenate([wl.k_dense[b][max(0, int(L) - 21):int(L)] for b, L in enumerate(wl.seq_lens)])
+    vals = torch.from_numpy(att).view(torch.float8_e4m3fn).float().abs()
+    assert vals.max().item() == 448.0
+    # non-attended slots hold the NaN code
+    assert (wl.k_dense[2][:100 - 21] == W.E4M3_NAN_CODE).all()
+    # q is bf16 of N(0,1) samples, sinks float32 [Hq]
+    assert wl.q.dtype == np.uint16 and wl.sinks.shape == (8,)
+
+
+def test_configs_shapes():
+    wl = W.make_workload("tiny")
+    assert wl.seq_lens.tolist() == [37, 300] and wl.max_blocks == 19
+    assert wl.kv_bytes() == (37 + 300) * 2 * 128 * 2
+    for name in W.CONFIG_ORDER:
+        c = W.CONFIGS[name]
+        assert c["Hq"] % c["Hkv"] == 0
+
+
+def test_generator_deterministic():
+    a = W.make_custom(B=2, Hq=4, Hkv=2, D=64, block_tokens=16, seq_lens=[33, 7], seed=5)
+    b = W.make_custom(B=2, Hq=4, Hkv=2, D=64, block_tokens=16, seq_lens=[33, 7], seed=5)
+    assert np.array_equal(a.k_cache, b.k_cache) and np.array_equal(a.q, b.q)
+    assert np.array_equal(a.block_table, b.block_table)
+
+
+def test_lognormal_lengths():
+    wl_lens = W._draw_lens(np.random.default_rng(0), 4096, ("lognormal", 2048.0, 1.0, 1, 32768))
+    assert wl_lens.min() >= 1 and wl_lens.max() <= 32768
+    assert abs(math.log(np.median(wl_lens)) - math.log(2048)) < 0.1

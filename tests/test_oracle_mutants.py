@@ -1,0 +1,76 @@
+"""Plant plausible mistakes in copies of the oracle and check that the pins catch each.
+
+Every mutant is a textual edit of ``oracle/fpd_oracle.c`` compiled into a
+temporary library (CPU only); the shipped oracle is untouched.  A mutant that
+passes every pin would mean the pins leave that part of the oracle unchecked.
+"""
+import os
+import tempfile
+
+import pytest
+
+import oracle
+from tests import oracle_pins as P
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "fpd_oracle.c")
+
+MUTANTS = {
+    "sink dropped from denominator": [("    Z += exp(sigma - m);\n", "")],
+    "GQA head mapping h % Hkv": [("const int kvh = h / g;", "const int kvh = h % J->Hkv;")],
+    "window start off by one": [("L - 1 - J->window_left", "L - J->window_left")],
+    "E4M3 exponent bias 8": [("expo - 7", "expo - 8")],
+    "E4M3 subnormal exponent": [("(double)mant / 8.0, -6)", "(double)mant / 8.0, -7)")],
+    "E4M3 mantissa step": [("1.0 + (double)mant / 8.0", "1.0 + (double)mant / 16.0")],
+    "E4M3 sign ignored": [("return sign ? -mag : mag;", "return mag;")],
+    "cache read head-major (transposed operand)": [
+        ("(((size_t)page * J->bt + slot) * J->Hkv + kvh) * (size_t)J->D",
+         "(((size_t)page * J->Hkv + kvh) * J->bt + slot) * (size_t)J->D")],
+    "in-page slot reversed": [("j % J->bt, kvh)", "J->bt - 1 - j % J->bt, kvh)")],
+    "block table ignored": [
+        ("const int page = J->block_table[(size_t)b * J->max_blocks + j / J->bt];",
+         "const int page = (int)((size_t)b * J->max_blocks + j / J->bt) % J->num_blocks;")],
+    "wrong query row": [("const uint16_t *qr = J->q + (size_t)row * D;",
+                         "const uint16_t *qr = J->q + (size_t)(b * J->Hq + kvh) * D;")],
+    "lse without sink": [("J->lse[row] = m + log(Z);",
+                          "J->lse[row] = m + log(Z - exp(sigma - m));")],
+    "sink multiplied by sm_scale": [("(double)J->sinks[h] : -INFINITY",
+                                     "J->sm_scale * (double)J->sinks[h] : -INFINITY")],
+    "v_scale dropped": [("(J->v_scale * fpd_oracle_e4m3_to_f64(vr[d]))",
+                         "fpd_oracle_e4m3_to_f64(vr[d])")],
+    "k_scale dropped": [("(J->k_scale * fpd_oracle_e4m3_to_f64(kr[d]))",
+                         "fpd_oracle_e4m3_to_f64(kr[d])")],
+    "sm_scale dropped": [("s[j - start] = J->sm_scale * dot;", "s[j - start] = dot;")],
+    "bf16 decode shift": [("(uint32_t)bits << 16", "(uint32_t)bits << 15")],
+    "max not subtracted consistently": [("const double p = exp(s[j - start] - m);",
+                                         "const double p = exp(s[j - start]);")],
+    "last key dropped": [("for (j = start; j < L; ++j) {\n        const int page = J->block_table"
+                          "[(size_t)b * J->max_blocks + j / J->bt];\n        const uint8_t *vr",
+                          "for (j = start; j < L - 1; ++j) {\n        const int page = J->block_table"
+                          "[(size_t)b * J->max_blocks + j / J->bt];\n        const uint8_t *vr")],
+}
+
+
+@pytest.fixture(scope="module")
+def source():
+    with open(SRC) as f:
+        return f.read()
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(source, name, tmp_path):
+    text = source
+    for old, new in MUTANTS[name]:
+        assert old in text, f"mutation site missing: {old!r}"
+        text = text.replace(old, new)
+    src = tmp_path / "mutant.c"
+    src.write_text(text)
+    so = tmp_path / "libmutant.so"
+    oracle.build(str(src), str(so))
+    lib = oracle.load(str(so))
+    caught = []
+    for pin in P.ALL_PINS:
+        try:
+            pin(lib)
+        except (AssertionError, ValueError) as e:
+            caught.append(f"{pin.__name__}: {str(e)[:80]}")
+    assert caught, f"no pin catches mutant '{name}'"
