@@ -1,0 +1,465 @@
+#!/usr/bin/env python
+"""Benchmark of the paged E4M3 decode attention on B200.
+
+Metric: KV-read HBM GB/s per decode call (algorithmic K+V bytes of the attended
+tokens / call time), with % of the measured HBM peak and us/call.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl native|reference]
+
+One step = one decode call (split kernel + combine kernel) over the whole batch
+of the named synthetic workload (default: the Llama-3-8B-shaped decode, B=32,
+Hq=32, Hkv=8, D=128, 16-token pages, lengths U[1024, 8192]).  Inputs are
+resident in HBM; consecutive steps read different replicas of the KV cache so
+that the bytes of one step are not in L2 for the next (replicas x KV bytes >
+2 x L2).  Timing: CUDA events on the launching stream around exactly K steps,
+barrier + synchronize on both sides, max over ranks.  Multi-GPU (torchrun) runs
+independent replicas, one per GPU (weak scaling): the path has no exchange.
+
+`--impl reference` times the fp64 CPU oracle (on the host cores, bounded
+samples of the same workload) and prints the same JSON line with
+"impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "KV-read HBM GB/s and % of B200 peak per decode call; µs/call"
+UNIT = "GB/s"
+DEFAULT_CONFIG = "llama3_8b"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--config", default=DEFAULT_CONFIG)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--chunk-pages", type=int, default=0, help="force pages per split (tuning)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU baseline sample budget")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--json-out", default=None)
+    return ap.parse_args()
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, STREAM-style copy)"
+    return FALLBACK_HBM_GBS, "fallback 6.65 TB/s (earlier measurement on this pool)"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "fp8_paged_decode_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        if fn.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, fn), "rb") as f:
+                h.update(fn.encode())
+                h.update(f.read())
+    return h.hexdigest()
+
+
+def ncu_traffic(config_name, kv_bytes):
+    """DRAM bytes per split-kernel launch from the committed ncu summary, scaled
+    to this launch's KV bytes; None when absent or taken on other kernel code."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    if d.get("source_sha256") != kernel_source_hash():
+        return None
+    e = d.get("workloads", {}).get(config_name)
+    if not e:
+        return None
+    return int(round(e["dram_bytes_per_launch"] * kv_bytes / e["kv_bytes_per_launch"]))
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms in the background."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.fh,
+                stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"],
+                    "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max((num(r[3]) or 0) for r in rows)}
+
+
+# ------------------------------------------------------------ CPU oracle --
+
+def oracle_sample(wl, budget_s, rng_seed=0, threads=None, min_rows=1):
+    """Run the oracle on random (sequence, head) rows until about budget_s of
+    wall time is spent; returns (seconds, kv_bytes_read, rows, threads)."""
+    import numpy as np
+    import oracle
+    threads = threads or (os.cpu_count() or 1)
+    rng = np.random.default_rng(rng_seed)
+    order = rng.permutation(wl.B * wl.Hq)
+    att = wl.attended()
+    # calibrate on a few rows
+    probe = order[:max(min_rows, min(len(order), threads))]
+    t0 = time.perf_counter()
+    oracle.decode_workload(wl, rows=probe, threads=threads)
+    t_probe = time.perf_counter() - t0
+    per_row = t_probe / len(probe)
+    n = int(max(min_rows, min(len(order), budget_s / max(per_row, 1e-6))))
+    rows = order[:n]
+    t0 = time.perf_counter()
+    oracle.decode_workload(wl, rows=rows, threads=threads)
+    dt = time.perf_counter() - t0
+    kv = int(sum(int(att[r // wl.Hq]) for r in rows)) * wl.D * 2
+    return dt, kv, n, threads
+
+
+def run_reference(args):
+    """The oracle as the reference arm: every step runs it on a bounded random
+    sample of (sequence, head) rows of the same workload, using all host cores."""
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    import numpy as np
+    from fp8_paged_decode_b200 import workloads as W
+    import oracle
+    wl = W.make_workload(args.config)
+    threads = os.cpu_count() or 1
+    total_steps = args.steps + args.warmup
+    budget_s = 120.0
+    # calibrate: wall time of one parallel batch of `threads` rows
+    probe = np.arange(min(wl.B * wl.Hq, threads))
+    t0 = time.perf_counter()
+    oracle.decode_workload(wl, rows=probe, threads=threads)
+    per_row_wall = (time.perf_counter() - t0) / len(probe)
+    rows_per_step = int(budget_s / total_steps / max(per_row_wall, 1e-7))
+    rows_per_step = max(1, min(rows_per_step, wl.B * wl.Hq))
+    rng = np.random.default_rng(7)
+    att = wl.attended()
+    t_sum, kv_sum = 0.0, 0
+    for step in range(total_steps):
+        rows = rng.choice(wl.B * wl.Hq, size=rows_per_step, replace=False)
+        t0 = time.perf_counter()
+        oracle.decode_workload(wl, rows=rows, threads=min(threads, rows_per_step))
+        dt = time.perf_counter() - t0
+        if step >= args.warmup:
+            t_sum += dt
+            kv_sum += int(sum(int(att[r // wl.Hq]) for r in rows)) * wl.D * 2
+    value = kv_sum / t_sum / 1e9
+    hbm, _ = measured_peaks()
+    sample = f"{rows_per_step} random (sequence, head) rows of the workload per step"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": t_sum / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": W.describe(args.config), "sample": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": min(threads, rows_per_step),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "pct_of_peak": 100.0 * value / hbm,
+    }
+    print(json.dumps(line))
+    if args.json_out:
+        with open(args.json_out, "w") as f:
+            f.write(json.dumps(line) + "\n")
+    return 0
+
+
+# ---------------------------------------------------------------- native --
+
+def run_native(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import fp8_paged_decode_b200 as fpd
+    from fp8_paged_decode_b200 import workloads as W
+
+    ws, rank, local = dist_env()
+    assert ws == args.gpus, f"--gpus {args.gpus} but WORLD_SIZE={ws}"
+    torch.cuda.set_device(local)
+    if ws > 1:
+        dist.init_process_group("nccl", init_method="env://",
+                                timeout=__import__("datetime").timedelta(seconds=120))
+
+    def barrier():
+        if ws > 1:
+            dist.barrier()
+
+    lib = fpd.load_library()
+    wl = W.make_workload(args.config)
+    dev = torch.device("cuda", local)
+    props = torch.cuda.get_device_properties(dev)
+    l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20))
+    kv_bytes = wl.kv_bytes()
+    replicas = max(1, min(8, math.ceil(2 * l2 / kv_bytes) + (1 if kv_bytes < 4 * l2 else 0)))
+
+    q = torch.from_numpy(wl.q.view(np.int16)).view(torch.bfloat16).to(dev)
+    table = torch.from_numpy(wl.block_table).to(dev)
+    lens = torch.from_numpy(wl.seq_lens).to(dev)
+    sinks = None if wl.sinks is None else torch.from_numpy(wl.sinks).to(dev)
+    kc = [torch.from_numpy(wl.k_cache).to(dev) for _ in range(replicas)]
+    vc = [torch.from_numpy(wl.v_cache).to(dev) for _ in range(replicas)]
+    out = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((wl.B, wl.Hq), dtype=torch.float32, device=dev)
+    need = fpd.fp8_paged_decode_workspace_bytes_ex(wl.B, wl.Hq, wl.Hkv, wl.D, wl.block_tokens,
+                                                   wl.max_blocks, wl.window_left, args.chunk_pages)
+    assert need > 0
+    wsp = torch.zeros(need, dtype=torch.uint8, device=dev)
+    plan = fpd.fp8_paged_decode_plan(wl.B, wl.Hq, wl.Hkv, wl.D, wl.block_tokens, wl.max_blocks,
+                                     wl.window_left, args.chunk_pages)
+    stream = torch.cuda.current_stream(dev)
+    sh = ctypes.c_void_p(stream.cuda_stream)
+    vp = ctypes.c_void_p
+
+    def call_args(i):
+        return [vp(q.data_ptr()), vp(kc[i].data_ptr()), vp(vc[i].data_ptr()), vp(table.data_ptr()),
+                vp(lens.data_ptr()), wl.B, wl.Hq, wl.Hkv, wl.D, wl.num_blocks, wl.block_tokens,
+                wl.max_blocks, ctypes.c_float(wl.k_scale), ctypes.c_float(wl.v_scale),
+                ctypes.c_float(wl.sm_scale), wl.window_left,
+                vp(sinks.data_ptr()) if sinks is not None else None, vp(out.data_ptr()),
+                vp(lse.data_ptr()), vp(wsp.data_ptr()), ctypes.c_size_t(wsp.numel()), sh,
+                args.chunk_pages]
+
+    pre = [call_args(i) for i in range(replicas)]
+    f_prof = lib.fp8_paged_decode_attention_profiled
+    f_plain = lib.fp8_paged_decode_attention_ex
+
+    # correctness guard on this exact launch configuration (sampled rows vs oracle)
+    st = f_plain(*pre[0])
+    assert st == 0, fpd.fp8_paged_decode_status_string(st)
+    torch.cuda.synchronize()
+    guard = None
+    if rank == 0:
+        import oracle
+        rng = np.random.default_rng(0)
+        rows = rng.choice(wl.B * wl.Hq, size=min(16, wl.B * wl.Hq), replace=False)
+        ro, rl = oracle.decode_workload(wl, rows=rows)
+        o = out.float().cpu().numpy()
+        l = lse.cpu().numpy()
+        b, h = np.divmod(rows, wl.Hq)
+        err = np.abs(o[b, h] - ro[b, h])
+        ok = bool((err <= 1e-2 + 1e-2 * np.abs(ro[b, h])).all() and
+                  (np.abs(l[b, h] - rl[b, h]) <= 1e-3).all())
+        guard = {"rows_checked": int(len(rows)), "max_abs_dout": float(err.max()),
+                 "max_abs_dlse": float(np.abs(l[b, h] - rl[b, h]).max()), "ok": ok}
+        assert ok, guard
+    bits = fpd.fp8_paged_decode_check_status(wsp, clear=True)
+    assert bits == 0, f"device status {bits}"
+
+    # warm-up
+    for i in range(args.warmup):
+        st = f_plain(*pre[i % replicas])
+        assert st == 0
+    torch.cuda.synchronize()
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.25)
+    barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for i in range(K):
+        e = evs[i]
+        st = f_prof(*pre[i % replicas], vp(e[0].cuda_event), vp(e[1].cuda_event),
+                    vp(e[2].cuda_event))
+        if st != 0:
+            raise RuntimeError(fpd.fp8_paged_decode_status_string(st))
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    total_ms = start.elapsed_time(end)
+    split_ms = [evs[i][0].elapsed_time(evs[i][1]) for i in range(K)]
+    call_ms = [evs[i][0].elapsed_time(evs[i][2]) for i in range(K)]
+    combine_ms = [evs[i][1].elapsed_time(evs[i][2]) for i in range(K)]
+
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if ws > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_total_ms = float(t.item())
+    ms_per_step = max_total_ms / K
+    value = ws * kv_bytes * K / (max_total_ms / 1e3) / 1e9
+
+    # end to end through the C ABI: pinned host inputs in, results out, every step
+    e2e = None
+    if not args.no_e2e:
+        hq = torch.from_numpy(wl.q.view(np.int16)).view(torch.bfloat16).pin_memory()
+        htab = torch.from_numpy(wl.block_table).pin_memory()
+        hlen = torch.from_numpy(wl.seq_lens).pin_memory()
+        hsink = None if wl.sinks is None else torch.from_numpy(wl.sinks).pin_memory()
+        hout = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.bfloat16).pin_memory()
+        hlse = torch.empty((wl.B, wl.Hq), dtype=torch.float32).pin_memory()
+        h2d = hq.numel() * 2 + htab.numel() * 4 + hlen.numel() * 4 + (
+            hsink.numel() * 4 if hsink is not None else 0)
+        d2h = hout.numel() * 2 + hlse.numel() * 4
+        Ke = K
+        for i in range(min(args.warmup, 50)):
+            st = f_plain(*pre[i % replicas])
+        torch.cuda.synchronize()
+        barrier()
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record(stream)
+        for i in range(Ke):
+            q.copy_(hq, non_blocking=True)
+            table.copy_(htab, non_blocking=True)
+            lens.copy_(hlen, non_blocking=True)
+            if hsink is not None:
+                sinks.copy_(hsink, non_blocking=True)
+            st = f_plain(*pre[i % replicas])
+            if st != 0:
+                raise RuntimeError(fpd.fp8_paged_decode_status_string(st))
+            hout.copy_(out, non_blocking=True)
+            hlse.copy_(lse, non_blocking=True)
+        e2.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        te = torch.tensor([s2.elapsed_time(e2)], dtype=torch.float64, device=dev)
+        if ws > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = {"value": ws * kv_bytes * Ke / (float(te.item()) / 1e3) / 1e9, "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": float(te.item()) / Ke,
+               "note": "q, block_table, seq_lens, sinks H2D from pinned host and out + lse D2H "
+                       "every step; the KV cache is resident device state"}
+
+    bits = fpd.fp8_paged_decode_check_status(wsp)
+    assert bits == 0, f"device status {bits}"
+
+    hbm, peak_src = measured_peaks()
+    split_avg_ms = statistics.fmean(split_ms)
+    achieved = kv_bytes / (split_avg_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                "frac": achieved / hbm, "traffic": ncu_traffic(args.config, kv_bytes),
+                "kernel": f"fpd_split_kernel<{wl.D},{2 if wl.groups > 8 else 1}>",
+                "algorithmic_bytes_per_launch": kv_bytes,
+                "unit_bytes": f"2*D = {2 * wl.D} B per (attended token, KV head); "
+                              f"{kv_bytes // (2 * wl.D)} units per launch",
+                "kernel_avg_us": split_avg_ms * 1e3, "peak_source": peak_src}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        dt, kvb, nrows, thr = oracle_sample(wl, args.cpu_seconds)
+        cpu = {"value": kvb / dt / 1e9, "unit": UNIT, "cores": thr, "kind": "oracle",
+               "sample": f"{nrows} random (sequence, head) rows of the workload, "
+                         f"{kvb} KV bytes, {dt:.1f} s wall"}
+
+    launches_per_step = 1 + (1 if plan["max_splits"] > 1 else 0)
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "dtype_detail": "E4M3 KV converted exactly to f16; mma.sync f16 x f16 -> f32; "
+                            "softmax and reductions in f32; bf16 output",
+            "data": "synthetic",
+            "config": {"workload": W.describe(args.config), "B": wl.B, "Hq": wl.Hq,
+                       "Hkv": wl.Hkv, "D": wl.D, "block_tokens": wl.block_tokens,
+                       "kv_bytes_per_call": kv_bytes, "parallelism": f"replicas x{ws}",
+                       "l2": f"inputs larger than L2: {replicas} KV replicas rotated, "
+                             f"{replicas * kv_bytes / 2**20:.0f} MiB read per rotation vs "
+                             f"{l2 / 2**20:.0f} MiB L2",
+                       "plan": plan},
+            "us_per_call": statistics.median(call_ms) * 1e3,
+            "us_per_call_p10_p90": [float(np.percentile(call_ms, 10) * 1e3),
+                                    float(np.percentile(call_ms, 90) * 1e3)],
+            "split_kernel_us": split_avg_ms * 1e3,
+            "combine_kernel_us": statistics.fmean(combine_ms) * 1e3,
+            "pct_of_peak": 100.0 * value / hbm,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches_per_step * K, "clocks": clocks, "parity_guard": guard,
+        }
+        print(json.dumps(line))
+        if args.json_out:
+            with open(args.json_out, "w") as f:
+                f.write(json.dumps(line) + "\n")
+    if ws > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_native(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,270 @@
+"""Paged E4M3 (FP8) decode attention for B200 (sm_100a).
+
+A thin ctypes binding of ``libfp8_paged_decode.so`` (the C ABI declared in
+``include/fp8_paged_decode.h``).  The functions carry the C names and only
+marshal arguments: torch tensors become raw device pointers and the current
+CUDA stream is passed along.  Every step of the computation runs in the
+library's CUDA kernels; there is no fallback.  If the shared library is
+missing, calling any function raises immediately (build it with
+``python -m fp8_paged_decode_b200.build``).
+
+Layouts (all contiguous, on one CUDA device):
+  q            bfloat16 [B, Hq, D]
+  k_cache      uint8 or float8_e4m3fn [num_blocks, block_tokens, Hkv, D]
+  v_cache      same as k_cache
+  block_table  int32 [B, max_blocks]
+  seq_lens     int32 [B]
+  sinks        float32 [Hq] or None
+  out          bfloat16 [B, Hq, D]; lse float32 [B, Hq] (optional)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+__all__ = [
+    "FPD_OK", "FPD_ERR_INVALID_ARG", "FPD_ERR_UNSUPPORTED", "FPD_ERR_WORKSPACE_TOO_SMALL",
+    "FPD_ERR_CUDA", "FPD_DEVERR_SEQ_LEN", "FPD_DEVERR_BLOCK_TABLE", "FPD_DEVERR_TIMEOUT",
+    "FpdError", "library_path", "load_library", "fp8_paged_decode_make_plan",
+    "fp8_paged_decode_plan", "fp8_paged_decode_workspace_bytes",
+    "fp8_paged_decode_workspace_bytes_ex", "fp8_paged_decode_attention_profiled",
+    "fp8_paged_decode_attention", "fp8_paged_decode_attention_ex",
+    "fp8_paged_decode_check_status", "fp8_paged_decode_workspace_init",
+    "fp8_paged_decode_status_string", "fp8_paged_decode_version", "EXPORTED_SYMBOLS",
+]
+
+FPD_OK = 0
+FPD_ERR_INVALID_ARG = 1
+FPD_ERR_UNSUPPORTED = 2
+FPD_ERR_WORKSPACE_TOO_SMALL = 3
+FPD_ERR_CUDA = 4
+FPD_DEVERR_SEQ_LEN = 0x1
+FPD_DEVERR_BLOCK_TABLE = 0x2
+FPD_DEVERR_TIMEOUT = 0x4
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_NAME = "libfp8_paged_decode.so"
+_lock = threading.Lock()
+_lib = None
+
+# Every entry point declared in include/fp8_paged_decode.h.
+EXPORTED_SYMBOLS = (
+    "fp8_paged_decode_make_plan",
+    "fp8_paged_decode_plan",
+    "fp8_paged_decode_workspace_bytes",
+    "fp8_paged_decode_workspace_bytes_ex",
+    "fp8_paged_decode_attention",
+    "fp8_paged_decode_attention_ex",
+    "fp8_paged_decode_attention_profiled",
+    "fp8_paged_decode_check_status",
+    "fp8_paged_decode_workspace_init",
+    "fp8_paged_decode_status_string",
+    "fp8_paged_decode_version",
+)
+
+
+class FpdError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {_status_name(status)} ({status})")
+
+
+class fpd_plan(ctypes.Structure):
+    _fields_ = [("chunk_pages", ctypes.c_int), ("max_splits", ctypes.c_int),
+                ("pages_per_stage", ctypes.c_int), ("stages", ctypes.c_int),
+                ("ctas", ctypes.c_int), ("smem_bytes", ctypes.c_int),
+                ("workspace_bytes", ctypes.c_size_t)]
+
+
+def library_path() -> str:
+    return os.path.join(_PKG, _LIB_NAME)
+
+
+def _bind(lib):
+    ci, cf, cz, vp = ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_void_p
+    lib.fp8_paged_decode_make_plan.argtypes = [ci] * 10 + [ctypes.POINTER(fpd_plan)]
+    lib.fp8_paged_decode_make_plan.restype = ci
+    lib.fp8_paged_decode_plan.argtypes = [ci] * 8 + [ctypes.POINTER(fpd_plan)]
+    lib.fp8_paged_decode_plan.restype = ci
+    lib.fp8_paged_decode_workspace_bytes.argtypes = [ci] * 7
+    lib.fp8_paged_decode_workspace_bytes.restype = cz
+    lib.fp8_paged_decode_workspace_bytes_ex.argtypes = [ci] * 8
+    lib.fp8_paged_decode_workspace_bytes_ex.restype = cz
+    attn = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, cf, cf, cf, ci, vp, vp, vp, vp, cz, vp]
+    lib.fp8_paged_decode_attention.argtypes = attn
+    lib.fp8_paged_decode_attention.restype = ci
+    lib.fp8_paged_decode_attention_ex.argtypes = attn + [ci]
+    lib.fp8_paged_decode_attention_ex.restype = ci
+    lib.fp8_paged_decode_attention_profiled.argtypes = attn + [ci, vp, vp, vp]
+    lib.fp8_paged_decode_attention_profiled.restype = ci
+    lib.fp8_paged_decode_check_status.argtypes = [vp, vp, ctypes.POINTER(ci), ci]
+    lib.fp8_paged_decode_check_status.restype = ci
+    lib.fp8_paged_decode_workspace_init.argtypes = [vp, cz, vp]
+    lib.fp8_paged_decode_workspace_init.restype = ci
+    lib.fp8_paged_decode_status_string.argtypes = [ci]
+    lib.fp8_paged_decode_status_string.restype = ctypes.c_char_p
+    lib.fp8_paged_decode_version.argtypes = []
+    lib.fp8_paged_decode_version.restype = ctypes.c_char_p
+    return lib
+
+
+def load_library(path: Optional[str] = None):
+    """Load the CUDA library (no CUDA call happens at load time)."""
+    global _lib
+    with _lock:
+        if _lib is None or path is not None:
+            p = path or library_path()
+            if not os.path.exists(p):
+                raise RuntimeError(
+                    f"{p} is missing: the CUDA extension has not been built "
+                    "(python -m fp8_paged_decode_b200.build); there is no fallback path")
+            lib = _bind(ctypes.CDLL(p))
+            if path is not None:
+                return lib
+            _lib = lib
+    return _lib
+
+
+def _status_name(status: int) -> str:
+    try:
+        return load_library().fp8_paged_decode_status_string(int(status)).decode()
+    except Exception:  # noqa: BLE001 - naming only
+        return f"status {status}"
+
+
+def _check(status: int, where: str):
+    if status != FPD_OK:
+        raise FpdError(status, where)
+
+
+def fp8_paged_decode_status_string(status: int) -> str:
+    return load_library().fp8_paged_decode_status_string(int(status)).decode()
+
+
+def fp8_paged_decode_version() -> str:
+    return load_library().fp8_paged_decode_version().decode()
+
+
+def fp8_paged_decode_make_plan(B, Hq, Hkv, D, block_tokens, max_blocks, window_left, num_sms,
+                               ctas_per_sm, chunk_pages_override=0) -> dict:
+    """Host-only split planner (no CUDA call)."""
+    plan = fpd_plan()
+    st = load_library().fp8_paged_decode_make_plan(
+        int(B), int(Hq), int(Hkv), int(D), int(block_tokens), int(max_blocks), int(window_left),
+        int(num_sms), int(ctas_per_sm), int(chunk_pages_override), ctypes.byref(plan))
+    _check(st, "fp8_paged_decode_make_plan")
+    return {f: getattr(plan, f) for f, _ in fpd_plan._fields_}
+
+
+def fp8_paged_decode_plan(B, Hq, Hkv, D, block_tokens, max_blocks, window_left=-1,
+                          chunk_pages_override=0) -> dict:
+    """The plan used on the current CUDA device."""
+    plan = fpd_plan()
+    st = load_library().fp8_paged_decode_plan(
+        int(B), int(Hq), int(Hkv), int(D), int(block_tokens), int(max_blocks), int(window_left),
+        int(chunk_pages_override), ctypes.byref(plan))
+    _check(st, "fp8_paged_decode_plan")
+    return {f: getattr(plan, f) for f, _ in fpd_plan._fields_}
+
+
+def fp8_paged_decode_workspace_bytes(B, Hq, Hkv, D, block_tokens, max_blocks, window_left=-1):
+    return int(load_library().fp8_paged_decode_workspace_bytes(
+        int(B), int(Hq), int(Hkv), int(D), int(block_tokens), int(max_blocks), int(window_left)))
+
+
+def fp8_paged_decode_workspace_bytes_ex(B, Hq, Hkv, D, block_tokens, max_blocks, window_left=-1,
+                                        chunk_pages_override=0):
+    return int(load_library().fp8_paged_decode_workspace_bytes_ex(
+        int(B), int(Hq), int(Hkv), int(D), int(block_tokens), int(max_blocks), int(window_left),
+        int(chunk_pages_override)))
+
+
+def _stream_handle(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dev_ptr(t, name, dtypes, shape=None):
+    import torch
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name} must have dtype in {dtypes}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def fp8_paged_decode_attention(q, k_cache, v_cache, block_table, seq_lens, k_scale, v_scale,
+                               sm_scale, window_left=-1, sinks=None, out=None, lse=None,
+                               workspace=None, stream=None, chunk_pages_override=0,
+                               return_lse=True):
+    """Enqueue one decode call on ``stream`` (default: torch's current stream).
+
+    Allocates ``out``/``lse``/``workspace`` with torch when not given (pass them
+    in to keep a call allocation-free).  Returns ``(out, lse)``.
+    """
+    import torch
+    B, Hq, D = q.shape
+    num_blocks, bt, Hkv, D2 = k_cache.shape
+    if D2 != D:
+        raise ValueError("q and the caches disagree on head_dim")
+    max_blocks = block_table.shape[1]
+    dev = q.device
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=dev)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    need = fp8_paged_decode_workspace_bytes_ex(B, Hq, Hkv, D, bt, max_blocks, window_left,
+                                               chunk_pages_override)
+    if workspace is None:
+        if need == 0 and B > 0:
+            raise FpdError(FPD_ERR_UNSUPPORTED, "fp8_paged_decode_workspace_bytes")
+        workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)
+    kv_types = (torch.uint8, torch.float8_e4m3fn)
+    st = load_library().fp8_paged_decode_attention_ex(
+        _dev_ptr(q, "q", (torch.bfloat16,), (B, Hq, D)),
+        _dev_ptr(k_cache, "k_cache", kv_types),
+        _dev_ptr(v_cache, "v_cache", kv_types, tuple(k_cache.shape)),
+        _dev_ptr(block_table, "block_table", (torch.int32,), (B, max_blocks)),
+        _dev_ptr(seq_lens, "seq_lens", (torch.int32,), (B,)),
+        B, Hq, Hkv, D, num_blocks, bt, max_blocks,
+        float(k_scale), float(v_scale), float(sm_scale), int(window_left),
+        _dev_ptr(sinks, "sinks", (torch.float32,), (Hq,)),
+        _dev_ptr(out, "out", (torch.bfloat16,), (B, Hq, D)),
+        _dev_ptr(lse, "lse", (torch.float32,), (B, Hq)),
+        _dev_ptr(workspace, "workspace", (torch.uint8,)),
+        ctypes.c_size_t(workspace.numel()),
+        _stream_handle(stream), int(chunk_pages_override))
+    _check(st, "fp8_paged_decode_attention")
+    return out, lse
+
+
+fp8_paged_decode_attention_ex = fp8_paged_decode_attention
+
+
+def fp8_paged_decode_check_status(workspace, stream=None, clear=False) -> int:
+    """Synchronise ``stream`` and return the workspace's device status bits."""
+    import torch
+    bits = ctypes.c_int(0)
+    st = load_library().fp8_paged_decode_check_status(
+        _dev_ptr(workspace, "workspace", (torch.uint8,)), _stream_handle(stream),
+        ctypes.byref(bits), int(bool(clear)))
+    _check(st, "fp8_paged_decode_check_status")
+    return int(bits.value)
+
+
+def fp8_paged_decode_workspace_init(workspace, stream=None):
+    import torch
+    st = load_library().fp8_paged_decode_workspace_init(
+        _dev_ptr(workspace, "workspace", (torch.uint8,)), ctypes.c_size_t(workspace.numel()),
+        _stream_handle(stream))
+    _check(st, "fp8_paged_decode_workspace_init")

@@ -1,0 +1,604 @@
+// fpd_kernels.cuh -- sm_100a kernels of the paged E4M3 decode attention.
+//
+// Split kernel: one CTA per (sequence b, KV head, KV split).  Warp 4 is the
+// producer: it walks the block table and issues one TMA box per (page, K/V)
+// into a ring of shared-memory stages (128-byte swizzle, so the consumers'
+// fragment loads are bank-conflict free).  Warps 0..3 are consumers: each owns
+// 16 token rows of every 64-token stage and runs
+//   S^T = K Q^T      mma.sync m16n8k16, tokens on M, the g query heads of the
+//                    KV head on N (heads on the MMA N side, as in the "SwapsAb"
+//                    orientation of FlashInfer PR #5591, Summary),
+//   online softmax   base 2, with a lazy running max (the max moves only when
+//                    a tile exceeds it by more than 8 in the exp2 domain, the
+//                    lazy-rescale rule of the same PR's Summary),
+//   O^T += V^T P^T   mma.sync m16n8k16, head dim on M, heads on N,
+// with E4M3 -> f16 conversion in registers (exact).  The per-tensor scales
+// are folded: logits use sm_scale * k_scale, the output uses v_scale.
+// The four consumer warps are merged in shared memory at the end; a sequence
+// handled by one split writes bf16 out / lse directly (sink folded in), others
+// write fp32 partials (O / l, log2-sum-exp) that the combine kernel merges.
+//
+// Fragment layouts (PTX ISA, mma.m16n8k16 with .f16):
+//   A: a0 (row g, cols 2t..2t+1), a1 (row g+8, same), a2 (row g, cols 2t+8..),
+//      a3 (row g+8, cols 2t+8..);  B: b0 (rows 2t..2t+1, col g), b1 (rows
+//      2t+8.., col g);  C: c0,c1 (row g, cols 2t..2t+1), c2,c3 (row g+8, ...)
+//   with g = lane / 4, t = lane % 4.
+// Because q.k and P.V are sums, the head-dim index behind each fragment slot
+// may be any fixed permutation; the kernel picks the one that makes every
+// thread's shared-memory reads contiguous 16-byte vectors:
+//   QK k-step ks, slot 2t+u  -> d = t*(D/4) + 4*ks + u      (u in 0..1)
+//               slot 2t+8+u  -> d = t*(D/4) + 4*ks + 2 + u
+//   PV m-tile i, row g+8h    -> d = g*(D/8) + 2*i + h        (h in 0..1)
+#pragma once
+
+#include <cmath>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "fpd_ptx.cuh"
+
+namespace fpd {
+
+constexpr int kConsumerWarps = 4;
+constexpr int kRowsPerWarp = 16;
+constexpr int kTileTokens = kConsumerWarps * kRowsPerWarp;  // tokens per stage
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr float kLazyThreshold = 8.0f;      // log2 units
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr uint64_t kWaitLimitNs = 500000000ull;   // 0.5 s: far above any legitimate wait
+constexpr uint64_t kDrainLimitNs = 50000000ull;   // 50 ms per stage when draining after a timeout
+
+struct DecodeParams {
+  const __nv_bfloat16* q;
+  const int32_t* block_table;
+  const int32_t* seq_lens;
+  const float* sinks;
+  __nv_bfloat16* out;
+  float* lse;
+  float* part_o;     // [B, Hq, max_splits, D]
+  float* part_lse;   // [B, Hq, max_splits]   (log2 domain)
+  uint32_t* status;  // workspace header word
+  int B, Hq, Hkv, g, bt, max_blocks, num_blocks, window_left;
+  int chunk_pages, max_splits, pages_per_stage, stages;
+  float qk_scale_log2;  // sm_scale * k_scale * log2(e)
+  float v_scale;
+};
+
+// Attended page range of sequence b, shared by both kernels.
+struct SeqRange {
+  int L, start, first_page, end_page, n_splits;
+};
+
+__device__ __forceinline__ SeqRange seq_range(int L_raw, int bt, int max_blocks, int window_left,
+                                              int chunk_pages, uint32_t* status) {
+  SeqRange r;
+  int L = L_raw;
+  const int cap = max_blocks * bt;
+  if (L < 0 || L > cap) {
+    if (status) atomicOr(status, 0x1u);
+    L = L < 0 ? 0 : cap;
+  }
+  r.L = L;
+  r.start = (window_left >= 0) ? max(0, L - 1 - window_left) : 0;
+  r.first_page = r.start / bt;
+  r.end_page = (L + bt - 1) / bt;
+  const int n_pages = r.end_page - r.first_page;
+  r.n_splits = (n_pages + chunk_pages - 1) / chunk_pages;
+  return r;
+}
+
+// Byte offset inside a 1024-byte-aligned tile written by TMA with 128-byte
+// (D = 128) or 64-byte (D = 64) swizzle: 16-byte chunk index XOR line bits.
+template <int D>
+__device__ __forceinline__ uint32_t swz(uint32_t off) {
+  constexpr uint32_t mask = (D == 128) ? 7u : 3u;
+  return off ^ (((off >> 7) & mask) << 4);
+}
+
+template <int D, int NT>
+struct Consumer {
+  static constexpr int KS = D / 16;   // k-steps of the QK MMA
+  static constexpr int MT = D / 16;   // m-tiles of the PV MMA
+  static constexpr int QW = D / 4;    // contiguous q elements per thread
+
+  uint32_t qf[NT][KS][2];   // Q^T B fragments (f16x2), head = lane / 4 of n-tile
+  float cs[NT][2];          // logit scale (log2) of this thread's C columns
+  float m[NT][2];           // running max (log2 domain) of this thread's columns
+  float thr[NT][2];         // raw-accumulator threshold that triggers a rescale
+  float l[NT][2];           // partial row sums (this thread's tokens only)
+  float o[MT][NT][4];       // O^T accumulators
+
+  __device__ __forceinline__ void init(const DecodeParams& p, int b, int kvh, int lane) {
+    const int n = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int hl = nt * 8 + n;
+      float vals[QW];
+      float amax = 0.f;
+      if (hl < p.g) {
+        const __nv_bfloat16* src = p.q + ((size_t)b * p.Hq + kvh * p.g + hl) * D + t * QW;
+#pragma unroll
+        for (int i = 0; i < QW; i += 8) {
+          const uint4 raw = *reinterpret_cast<const uint4*>(src + i);
+          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float2 f = __bfloat1622float2(h2[j]);
+            vals[i + 2 * j] = f.x;
+            vals[i + 2 * j + 1] = f.y;
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < QW; ++i) amax = fmaxf(amax, fabsf(vals[i]));
+      } else {
+#pragma unroll
+        for (int i = 0; i < QW; ++i) vals[i] = 0.f;
+      }
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+      // Power-of-two prescale so the largest |q| of the head sits in [2^14, 2^15):
+      // keeps bf16 -> f16 exact for any bf16 magnitude; undone in the logit scale.
+      int e = 0;
+      if (amax > 0.f && isfinite(amax)) frexpf(amax, &e);
+      const float fac = ldexpf(1.0f, max(-126, min(126, 15 - e)));
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        qf[nt][ks][0] = pack_f16x2(vals[4 * ks] * fac, vals[4 * ks + 1] * fac);
+        qf[nt][ks][1] = pack_f16x2(vals[4 * ks + 2] * fac, vals[4 * ks + 3] * fac);
+      }
+      // this thread's C columns are heads 2t and 2t+1 of the n-tile
+      const float f0 = __shfl_sync(0xffffffffu, fac, (2 * t) * 4);
+      const float f1 = __shfl_sync(0xffffffffu, fac, (2 * t + 1) * 4);
+      cs[nt][0] = p.qk_scale_log2 / f0;
+      cs[nt][1] = p.qk_scale_log2 / f1;
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        m[nt][j] = -INFINITY;
+        thr[nt][j] = -INFINITY;
+        l[nt][j] = 0.f;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < MT; ++i)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) o[i][nt][j] = 0.f;
+  }
+
+  // One 16-row slice of a stage.  FULL: every row is inside [tok_lo, tok_hi).
+  template <bool FULL>
+  __device__ __forceinline__ void tile(const uint8_t* Kt, const uint8_t* Vt, int row0, int tok0,
+                                       int tok_lo, int tok_hi, int lane) {
+    const int n = lane >> 2, t = lane & 3;
+    // ---- K fragments: rows row0 + n and row0 + n + 8, bytes [t*D/4, (t+1)*D/4)
+    uint32_t kw[2][D / 16];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int row = row0 + n + 8 * r;
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        const uint4 v = *reinterpret_cast<const uint4*>(
+            Kt + swz<D>(row * D + t * (D / 4) + 16 * c));
+        kw[r][4 * c + 0] = v.x;
+        kw[r][4 * c + 1] = v.y;
+        kw[r][4 * c + 2] = v.z;
+        kw[r][4 * c + 3] = v.w;
+      }
+    }
+    // ---- S^T = K Q^T, two accumulation chains per n-tile
+    float s[NT][2][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int c = 0; c < 2; ++c)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) s[nt][c][j] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      uint32_t a0, a1, a2, a3;
+      e4m3x4_to_f16x2x2(kw[0][ks], a0, a2);
+      e4m3x4_to_f16x2x2(kw[1][ks], a1, a3);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+        mma_16816(s[nt][ks & 1], a0, a1, a2, a3, qf[nt][ks][0], qf[nt][ks][1]);
+    }
+    float acc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[nt][j] = s[nt][0][j] + s[nt][1][j];
+
+    bool v0 = true, v1 = true;  // rows n and n+8 inside the attended range
+    if (!FULL) {
+      const int tk0 = tok0 + n, tk1 = tok0 + n + 8;
+      v0 = tk0 >= tok_lo && tk0 < tok_hi;
+      v1 = tk1 >= tok_lo && tk1 < tok_hi;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        if (!v0) acc[nt][0] = acc[nt][1] = -INFINITY;
+        if (!v1) acc[nt][2] = acc[nt][3] = -INFINITY;
+      }
+    }
+
+    // ---- lazy running max
+    bool need = false;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+        need |= (acc[nt][j] > thr[nt][j]) || (acc[nt][j + 2] > thr[nt][j]);
+    if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          float tmax = fmaxf(acc[nt][j], acc[nt][j + 2]);
+          tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 4));
+          tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 8));
+          tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
+          const float smax = tmax * cs[nt][j];
+          if (smax > m[nt][j] + kLazyThreshold) {
+            const float alpha = fast_exp2(m[nt][j] - smax);  // 0 on the first tile
+            m[nt][j] = smax;
+            thr[nt][j] = (smax + kLazyThreshold) / cs[nt][j];
+            l[nt][j] *= alpha;
+#pragma unroll
+            for (int i = 0; i < MT; ++i) {
+              o[i][nt][j] *= alpha;
+              o[i][nt][j + 2] *= alpha;
+            }
+          }
+        }
+      }
+    }
+
+    // ---- probabilities (fp32 sums; f16 copies feed the PV MMA)
+    uint32_t pb0[NT], pb1[NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const float p0 = fast_exp2(fmaf(acc[nt][0], cs[nt][0], -m[nt][0]));
+      const float p1 = fast_exp2(fmaf(acc[nt][1], cs[nt][1], -m[nt][1]));
+      const float p2 = fast_exp2(fmaf(acc[nt][2], cs[nt][0], -m[nt][0]));
+      const float p3 = fast_exp2(fmaf(acc[nt][3], cs[nt][1], -m[nt][1]));
+      l[nt][0] += p0 + p2;
+      l[nt][1] += p1 + p3;
+      pb0[nt] = movmatrix_trans(pack_f16x2(p0, p1));   // tokens 2t..2t+1, head n
+      pb1[nt] = movmatrix_trans(pack_f16x2(p2, p3));   // tokens 2t+8..2t+9, head n
+    }
+
+    // ---- V fragments: token rows 2t, 2t+1, 2t+8, 2t+9; head-dim chunk n
+    constexpr int VB = D / 8;  // bytes of one row this thread needs
+    uint32_t va[VB / 4], vb[VB / 4], vc[VB / 4], vd[VB / 4];
+    const int rA = row0 + 2 * t;
+    if constexpr (D == 128) {
+      const uint4 A = *reinterpret_cast<const uint4*>(Vt + swz<D>((rA + 0) * D + n * VB));
+      const uint4 B = *reinterpret_cast<const uint4*>(Vt + swz<D>((rA + 1) * D + n * VB));
+      const uint4 C = *reinterpret_cast<const uint4*>(Vt + swz<D>((rA + 8) * D + n * VB));
+      const uint4 E = *reinterpret_cast<const uint4*>(Vt + swz<D>((rA + 9) * D + n * VB));
+      va[0] = A.x; va[1] = A.y; va[2] = A.z; va[3] = A.w;
+      vb[0] = B.x; vb[1] = B.y; vb[2] = B.z; vb[3] = B.w;
+      vc[0] = C.x; vc[1] = C.y; vc[2] = C.z; vc[3] = C.w;
+      vd[0] = E.x; vd[1] = E.y; vd[2] = E.z; vd[3] = E.w;
+    } else {
+      const uint2 A = *reinterpret_cast<const uint2*>(Vt + swz<D>((rA + 0) * D + n * VB));
+      const uint2 B = *reinterpret_cast<const uint2*>(Vt + swz<D>((rA + 1) * D + n * VB));
+      const uint2 C = *reinterpret_cast<const uint2*>(Vt + swz<D>((rA + 8) * D + n * VB));
+      const uint2 E = *reinterpret_cast<const uint2*>(Vt + swz<D>((rA + 9) * D + n * VB));
+      va[0] = A.x; va[1] = A.y;
+      vb[0] = B.x; vb[1] = B.y;
+      vc[0] = C.x; vc[1] = C.y;
+      vd[0] = E.x; vd[1] = E.y;
+    }
+    if (!FULL) {
+      // Zero value rows outside the range: stale bytes may hold NaN codes and
+      // 0 * NaN would poison the accumulator.
+      const int tA = tok0 + 2 * t;
+      const uint32_t mA = (tA >= tok_lo && tA < tok_hi) ? 0xffffffffu : 0u;
+      const uint32_t mB = (tA + 1 >= tok_lo && tA + 1 < tok_hi) ? 0xffffffffu : 0u;
+      const uint32_t mC = (tA + 8 >= tok_lo && tA + 8 < tok_hi) ? 0xffffffffu : 0u;
+      const uint32_t mD = (tA + 9 >= tok_lo && tA + 9 < tok_hi) ? 0xffffffffu : 0u;
+#pragma unroll
+      for (int w = 0; w < VB / 4; ++w) {
+        va[w] &= mA;
+        vb[w] &= mB;
+        vc[w] &= mC;
+        vd[w] &= mD;
+      }
+    }
+    // ---- O^T += V^T P^T
+#pragma unroll
+    for (int w = 0; w < VB / 4; ++w) {
+      const uint32_t ab_lo = prmt(va[w], vb[w], 0x5140u);  // d byte 0,1: {A,B} pairs
+      const uint32_t ab_hi = prmt(va[w], vb[w], 0x7362u);  // d byte 2,3
+      const uint32_t cd_lo = prmt(vc[w], vd[w], 0x5140u);
+      const uint32_t cd_hi = prmt(vc[w], vd[w], 0x7362u);
+      uint32_t a0, a1, a2, a3;
+      e4m3x4_to_f16x2x2(ab_lo, a0, a1);
+      e4m3x4_to_f16x2x2(cd_lo, a2, a3);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) mma_16816(o[2 * w][nt], a0, a1, a2, a3, pb0[nt], pb1[nt]);
+      e4m3x4_to_f16x2x2(ab_hi, a0, a1);
+      e4m3x4_to_f16x2x2(cd_hi, a2, a3);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+        mma_16816(o[2 * w + 1][nt], a0, a1, a2, a3, pb0[nt], pb1[nt]);
+    }
+  }
+};
+
+// Merge scratch per CTA (reuses the stage ring): [warp][head][D] O plus
+// [warp][head] (m, l).
+template <int D, int NT>
+struct MergeLayout {
+  static constexpr int H = NT * 8;
+  static constexpr int kOBytes = kConsumerWarps * H * D * 4;
+  static constexpr int kMLBytes = kConsumerWarps * H * 2 * 4;
+  static constexpr int kBytes = kOBytes + kMLBytes;
+};
+
+template <int D, int NT>
+__global__ void __launch_bounds__(kThreads)
+fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                 const DecodeParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  constexpr int kTileBytes = kTileTokens * D;
+  const int stages = p.stages;
+  int ring_bytes = stages * 2 * kTileBytes;
+  if (ring_bytes < MergeLayout<D, NT>::kBytes) ring_bytes = MergeLayout<D, NT>::kBytes;
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + ring_bytes);
+  uint64_t* empty_bar = full_bar + stages;
+
+  int bid = blockIdx.x;
+  const int kvh = bid % p.Hkv;
+  bid /= p.Hkv;
+  const int split = bid % p.max_splits;
+  const int b = bid / p.max_splits;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const SeqRange R = seq_range(p.seq_lens[b], p.bt, p.max_blocks, p.window_left, p.chunk_pages,
+                               threadIdx.x == 0 ? p.status : nullptr);
+  if (split >= (R.n_splits > 0 ? R.n_splits : 1)) return;
+  if (R.n_splits == 0) {  // empty sequence: out = 0, lse = sigma
+    for (int i = threadIdx.x; i < p.g * D; i += blockDim.x) {
+      const int h = kvh * p.g + i / D;
+      p.out[((size_t)b * p.Hq + h) * D + (i % D)] = __float2bfloat16_rn(0.f);
+    }
+    for (int i = threadIdx.x; i < p.g; i += blockDim.x) {
+      const int h = kvh * p.g + i;
+      if (p.lse) p.lse[(size_t)b * p.Hq + h] = p.sinks ? p.sinks[h] : -INFINITY;
+    }
+    return;
+  }
+  const int pb = R.first_page + split * p.chunk_pages;
+  const int pe = min(pb + p.chunk_pages, R.end_page);
+  const int tok_lo = max(R.start, pb * p.bt);
+  const int tok_hi = min(R.L, pe * p.bt);
+  const int pps = p.pages_per_stage;
+  const int n_stages = (pe - pb + pps - 1) / pps;
+  const bool single = (R.n_splits == 1);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], kConsumerWarps);
+    }
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+
+  bool timed_out = false;
+  if (warp == kConsumerWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&kmap);
+      tma_prefetch_desc(&vmap);
+    }
+    const uint64_t policy = l2_policy_evict_first();
+    const int32_t* tbl = p.block_table + (size_t)b * p.max_blocks;
+    const uint32_t page_bytes = (uint32_t)(p.bt * D);
+    int batch_base = -1;
+    int my_entry = 0;
+    for (int s = 0; s < n_stages && !timed_out; ++s) {
+      const int slot = s % stages;
+      if (s >= stages) {
+        if (!mbar_wait_bounded(&empty_bar[slot], ((s / stages) - 1) & 1, kWaitLimitNs))
+          timed_out = true;
+        timed_out = __any_sync(0xffffffffu, timed_out);
+        if (timed_out) break;
+      }
+      const int pg0 = pb + s * pps;
+      const int np = min(pps, pe - pg0);
+      // block-table entries are fetched 32 at a time by the warp's lanes
+      const int rel = pg0 - pb;
+      if ((rel & ~31) != batch_base) {
+        batch_base = rel & ~31;
+        const int idx = pb + batch_base + lane;
+        my_entry = (idx < pe) ? __ldg(tbl + idx) : 0;
+      }
+      int rows[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int e = __shfl_sync(0xffffffffu, my_entry, (rel + i) & 31);
+        const bool ok = (e >= 0 && e < p.num_blocks);
+        if (!ok && i < np && lane == 0) atomicOr(p.status, 0x2u);
+        // an invalid page is read from past the end of the pool: TMA zero-fills it
+        rows[i] = ok ? e * p.bt : p.num_blocks * p.bt;
+      }
+      if (lane == 0) {
+        uint8_t* kdst = smem + slot * 2 * kTileBytes;
+        uint8_t* vdst = kdst + kTileBytes;
+        mbar_arrive_expect_tx(&full_bar[slot], 2u * page_bytes * (uint32_t)np);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          if (i < np) {
+            tma_load_3d(kdst + i * page_bytes, &kmap, 0, kvh, rows[i], &full_bar[slot], policy);
+            tma_load_3d(vdst + i * page_bytes, &vmap, 0, kvh, rows[i], &full_bar[slot], policy);
+          }
+        }
+      }
+    }
+    if (timed_out && lane == 0) atomicOr(p.status, 0x4u);
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  Consumer<D, NT> cw;
+  cw.init(p, b, kvh, lane);
+  const int row0 = warp * kRowsPerWarp;
+  int s = 0;
+  for (; s < n_stages; ++s) {
+    const int slot = s % stages;
+    if (!mbar_wait_bounded(&full_bar[slot], (s / stages) & 1, kWaitLimitNs)) timed_out = true;
+    if (__any_sync(0xffffffffu, timed_out)) {
+      timed_out = true;
+      break;
+    }
+    const uint8_t* Kt = smem + slot * 2 * kTileBytes;
+    const uint8_t* Vt = Kt + kTileBytes;
+    const int tok0 = (pb + s * pps) * p.bt + row0;   // token of this warp's first row
+    if (tok0 + kRowsPerWarp > tok_lo && tok0 < tok_hi) {
+      if (tok0 >= tok_lo && tok0 + kRowsPerWarp <= tok_hi)
+        cw.template tile<true>(Kt, Vt, row0, tok0, tok_lo, tok_hi, lane);
+      else
+        cw.template tile<false>(Kt, Vt, row0, tok0, tok_lo, tok_hi, lane);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty_bar[slot]);
+  }
+  if (timed_out) {
+    // Let every load that may already be issued land before the ring is reused
+    // (bounded), report, and still take part in the merge barriers below so
+    // the other warps are not left waiting; the results are flagged invalid.
+    for (int r = s; r < n_stages && r < s + stages; ++r)
+      mbar_wait_bounded(&full_bar[r % stages], (r / stages) & 1, kDrainLimitNs);
+    if (lane == 0) atomicOr(p.status, 0x4u);
+  }
+
+  // ------------------------------------------------- merge the four warps
+  constexpr int H = NT * 8;
+  float* Osm = reinterpret_cast<float*>(smem);                       // [warp][H][D]
+  float* MLsm = reinterpret_cast<float*>(smem + MergeLayout<D, NT>::kOBytes);  // [warp][H][2]
+  const int n = lane >> 2, t = lane & 3;
+  named_barrier_sync(1, kConsumerWarps * 32);   // all ring reads done before reuse
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      float lsum = cw.l[nt][j];
+      lsum += __shfl_xor_sync(0xffffffffu, lsum, 4);
+      lsum += __shfl_xor_sync(0xffffffffu, lsum, 8);
+      lsum += __shfl_xor_sync(0xffffffffu, lsum, 16);
+      const int h = nt * 8 + 2 * t + j;
+      if (n == 0) {
+        MLsm[(warp * H + h) * 2 + 0] = cw.m[nt][j];
+        MLsm[(warp * H + h) * 2 + 1] = lsum;
+      }
+      // O^T column h: rows d = n*(D/8) + 2i + hh  (hh = 0 -> c0/c1, 1 -> c2/c3)
+      float* dst = Osm + ((size_t)warp * H + h) * D + n * (D / 8);
+#pragma unroll
+      for (int i = 0; i < Consumer<D, NT>::MT; ++i) {
+        dst[2 * i + 0] = cw.o[i][nt][j];
+        dst[2 * i + 1] = cw.o[i][nt][j + 2];
+      }
+    }
+  }
+  named_barrier_sync(1, kConsumerWarps * 32);
+
+  const int tid = threadIdx.x;  // 0 .. 127
+  for (int idx = tid; idx < p.g * D; idx += kConsumerWarps * 32) {
+    const int h = idx / D, d = idx % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, MLsm[(w * H + h) * 2]);
+    float Lsum = 0.f, acc = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) {
+      const float mw = MLsm[(w * H + h) * 2];
+      const float sc = (mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
+      Lsum += MLsm[(w * H + h) * 2 + 1] * sc;
+      acc += Osm[((size_t)w * H + h) * D + d] * sc;
+    }
+    const int hq = kvh * p.g + h;
+    const size_t row = (size_t)b * p.Hq + hq;
+    const float lse2 = M + __log2f(Lsum);      // log2-sum-exp of this split (no sink)
+    if (single) {
+      float Z = 1.f, Mx = lse2, wsplit = 1.f;
+      if (p.sinks) {
+        const float sg = p.sinks[hq] * kLog2e;
+        Mx = fmaxf(lse2, sg);
+        wsplit = fast_exp2(lse2 - Mx);
+        Z = wsplit + fast_exp2(sg - Mx);
+      }
+      p.out[row * D + d] = __float2bfloat16_rn(acc / Lsum * wsplit / Z * p.v_scale);
+      if (d == 0 && p.lse) p.lse[row] = (Mx + __log2f(Z)) * kLn2;
+    } else {
+      const size_t prow = row * p.max_splits + split;
+      p.part_o[prow * D + d] = acc / Lsum;
+      if (d == 0) p.part_lse[prow] = lse2;
+    }
+  }
+}
+
+struct CombineParams {
+  const int32_t* seq_lens;
+  const float* sinks;
+  const float* part_o;
+  const float* part_lse;
+  __nv_bfloat16* out;
+  float* lse;
+  int B, Hq, bt, max_blocks, window_left, chunk_pages, max_splits;
+  float v_scale;
+};
+
+// One warp per (sequence, query head) whose sequence spans several splits:
+// out = v_scale * sum_s 2^(lse_s - M) o_s / (sum_s 2^(lse_s - M) + 2^(sigma - M)).
+template <int D>
+__global__ void __launch_bounds__(256) fpd_combine_kernel(const CombineParams p) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 8 + warp;
+  if (row >= p.B * p.Hq) return;
+  const int b = row / p.Hq, h = row % p.Hq;
+  const SeqRange R = seq_range(p.seq_lens[b], p.bt, p.max_blocks, p.window_left, p.chunk_pages,
+                               nullptr);
+  const int ns = R.n_splits;
+  if (ns <= 1) return;
+  const float* pl = p.part_lse + (size_t)row * p.max_splits;
+  float M = p.sinks ? p.sinks[h] * kLog2e : -INFINITY;
+  for (int s = lane; s < ns; s += 32) M = fmaxf(M, pl[s]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  constexpr int PER = D / 32;
+  float acc[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) acc[i] = 0.f;
+  float Z = p.sinks ? fast_exp2(p.sinks[h] * kLog2e - M) : 0.f;
+  const float* po = p.part_o + (size_t)row * p.max_splits * D + lane * PER;
+  for (int s = 0; s < ns; ++s) {
+    const float w = fast_exp2(pl[s] - M);
+    Z += w;
+    if constexpr (PER == 4) {
+      const float4 v = *reinterpret_cast<const float4*>(po + (size_t)s * D);
+      acc[0] += w * v.x;
+      acc[1] += w * v.y;
+      acc[2] += w * v.z;
+      acc[3] += w * v.w;
+    } else {
+      const float2 v = *reinterpret_cast<const float2*>(po + (size_t)s * D);
+      acc[0] += w * v.x;
+      acc[1] += w * v.y;
+    }
+  }
+  const float inv = p.v_scale / Z;
+  __nv_bfloat16* dst = p.out + (size_t)row * D + lane * PER;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) dst[i] = __float2bfloat16_rn(acc[i] * inv);
+  if (lane == 0 && p.lse) p.lse[row] = (M + __log2f(Z)) * kLn2;
+}
+
+}  // namespace fpd

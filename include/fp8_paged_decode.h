@@ -1,0 +1,200 @@
+/*
+ * fp8_paged_decode.h -- C ABI of the B200 (sm_100a) paged FP8 decode attention.
+ *
+ * The operation (named by the grouped-nf4-gemm solutions page
+ * "fp8-paged-attention-for-moe-serving", title and summary): one decode query
+ * per sequence attends, through a per-sequence block table, to a paged KV cache
+ * stored as E4M3 (OCP e4m3fn) codes with per-tensor scales, with a caller-chosen
+ * softmax scale, an optional sliding window and optional per-head attention
+ * sinks.  For sequence b and query head h (GQA: g = Hq / Hkv, KV head h / g):
+ *
+ *   start = window_left >= 0 ? max(0, L_b - 1 - window_left) : 0
+ *   s_j   = sm_scale * q[b,h,:] . (k_scale * e4m3(K_b[j, h/g, :]))   j in [start, L_b)
+ *   sigma = sinks ? sinks[h] : -inf                (no value; denominator only)
+ *   out   = sum_j e^(s_j - m) v_scale e4m3(V_b[j, h/g, :]) / (sum_j e^(s_j - m) + e^(sigma - m))
+ *   lse   = m + ln(sum_j e^(s_j - m) + e^(sigma - m)),   m = max(max_j s_j, sigma)
+ *
+ * K_b[j] lives at k_cache[block_table[b][j / block_tokens]][j % block_tokens]:
+ * the FlashInfer/SGLang paged-KV convention (fish-scales-ops README, the note on
+ * paged prefill/decode APIs following those conventions; the NVFP4 KV-cache gist,
+ * vLLM FlashInfer backend section).  Per-tensor scales follow the gist's cache
+ * writer (stored code = x / scale).  window_left is FlashInfer's parameter of the
+ * same name (gist, FlashInfer backend patch).  The caller-owned workspace with a
+ * size query and no allocation on any call path follows FlashInfer PR #5591,
+ * Summary ("caller-owned workspace").
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers of the current CUDA device unless
+ *    stated otherwise; all are row-major and contiguous.  The caller owns every
+ *    buffer.  The library never allocates, frees or synchronises device memory
+ *    (fp8_paged_decode_check_status is the one call that synchronises).
+ *  - Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL = legacy
+ *    default stream) and the call returns without waiting for it.
+ *  - Calls with distinct workspaces may run concurrently.
+ *  - Host-detectable errors return a status before anything is launched.
+ *  - Data errors found on the device (sequence length outside [0, max_blocks *
+ *    block_tokens], block-table entry outside [0, num_blocks) inside the attended
+ *    range) never cause an out-of-bounds access: the length is clamped, the page
+ *    is read as zeros, and a bit is set in the workspace status word
+ *    (FPD_DEVERR_*), readable with fp8_paged_decode_check_status.
+ */
+#ifndef FP8_PAGED_DECODE_H
+#define FP8_PAGED_DECODE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FPD_OK = 0,
+    FPD_ERR_INVALID_ARG = 1,          /* null pointer, negative size, bad alignment, non-finite scale */
+    FPD_ERR_UNSUPPORTED = 2,          /* shape outside the supported set (see below) */
+    FPD_ERR_WORKSPACE_TOO_SMALL = 3,  /* workspace_bytes below the size query's answer */
+    FPD_ERR_CUDA = 4                  /* a CUDA runtime/driver call failed */
+} fpd_status;
+
+/* Device-side status bits (sticky until cleared). */
+#define FPD_DEVERR_SEQ_LEN 0x1u       /* a seq_lens entry was < 0 or > max_blocks * block_tokens (clamped) */
+#define FPD_DEVERR_BLOCK_TABLE 0x2u   /* a block-table entry in the attended range was outside [0, num_blocks) (read as zeros) */
+#define FPD_DEVERR_TIMEOUT 0x4u       /* a pipeline wait exceeded its time limit (results invalid) */
+
+/* Split plan chosen by the host planner; all fields are outputs. */
+typedef struct {
+    int chunk_pages;        /* KV pages per split (one CTA per sequence, KV head and split) */
+    int max_splits;         /* splits launched per (sequence, KV head); unused ones exit at once */
+    int pages_per_stage;    /* pages moved per pipeline stage */
+    int stages;             /* depth of the shared-memory ring */
+    int ctas;               /* grid size of the split kernel */
+    int smem_bytes;         /* dynamic shared memory per CTA */
+    size_t workspace_bytes; /* bytes this plan needs */
+} fpd_plan;
+
+/*
+ * Supported shapes: D (head_dim) in {64, 128}; g = Hq / Hkv in {1, 2, 4, 8, 16};
+ * block_tokens in {16, 32, 64}; num_blocks * block_tokens < 2^31; q, out and the
+ * caches 16-byte aligned.  Anything else returns FPD_ERR_UNSUPPORTED (or
+ * FPD_ERR_INVALID_ARG for malformed arguments); there is no fallback path.
+ */
+
+/*
+ * Host-only planner (no CUDA call): the split plan for a shape on a device with
+ * `num_sms` SMs of which `ctas_per_sm` CTAs of the split kernel fit per SM.
+ * chunk_pages_override > 0 forces the pages per split (rounded up to whole
+ * pipeline stages); 0 lets the heuristic choose.
+ * Returns FPD_OK or the validation error for the shape.
+ */
+fpd_status fp8_paged_decode_make_plan(int B, int Hq, int Hkv, int D, int block_tokens,
+                                      int max_blocks, int window_left, int num_sms,
+                                      int ctas_per_sm, int chunk_pages_override,
+                                      fpd_plan *plan);
+
+/*
+ * The plan fp8_paged_decode_attention_ex uses on the CURRENT device (its SM
+ * count and the split kernel's occupancy, queried once per device).  Returns
+ * FPD_ERR_CUDA when no device is usable.
+ */
+fpd_status fp8_paged_decode_plan(int B, int Hq, int Hkv, int D, int block_tokens, int max_blocks,
+                                 int window_left, int chunk_pages_override, fpd_plan *plan);
+
+/*
+ * Workspace bytes one fp8_paged_decode_attention call with these sizes needs on
+ * the CURRENT device (queries its SM count and the kernel occupancy once).
+ * Returns 0 for an unsupported or malformed shape, or when no device is present.
+ * The workspace holds a 256-byte header (status word) and per-split partial
+ * results; its contents between calls carry only the sticky status bits.
+ */
+size_t fp8_paged_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int block_tokens,
+                                        int max_blocks, int window_left);
+
+/* Same, for a forced split size (see fp8_paged_decode_make_plan). */
+size_t fp8_paged_decode_workspace_bytes_ex(int B, int Hq, int Hkv, int D, int block_tokens,
+                                           int max_blocks, int window_left,
+                                           int chunk_pages_override);
+
+/*
+ * Paged E4M3 decode attention (the formula at the top of this file).
+ *   q            bf16  [B, Hq, D]
+ *   k_cache      e4m3  [num_blocks, block_tokens, Hkv, D]   (token-major pages)
+ *   v_cache      e4m3  [num_blocks, block_tokens, Hkv, D]
+ *   block_table  int32 [B, max_blocks]; entry i is the physical page of the
+ *                sequence's tokens [i*block_tokens, (i+1)*block_tokens); only
+ *                the pages covering the attended range are read
+ *   seq_lens     int32 [B]; L_b, the sequence length including the new token
+ *   k_scale, v_scale   per-tensor dequantisation scales (value = code * scale)
+ *   sm_scale     softmax scale applied to q.k (sm_scale * k_scale must be > 0)
+ *   window_left  < 0: attend all L_b keys; >= 0: the newest window_left + 1
+ *   sinks        float [Hq] sink logits (same units as sm_scale * q.k), or NULL
+ *   out          bf16  [B, Hq, D] (round to nearest even)
+ *   lse          float [B, Hq] natural-log sum of exponentials including the
+ *                sink, or NULL (not written).  L_b == 0 gives out = 0 and
+ *                lse = sinks[h] (or -inf).
+ *   workspace    device buffer of at least fp8_paged_decode_workspace_bytes()
+ *                (always >= 256) bytes, 16-byte aligned.  Its first word is the
+ *                sticky device status: zero it once after allocating (or call
+ *                fp8_paged_decode_workspace_init); the rest is scratch
+ *   stream       cudaStream_t
+ * Two kernels are enqueued: the split kernel and, when some sequence spans
+ * several splits, the combine kernel.
+ */
+fpd_status fp8_paged_decode_attention(const void *q, const void *k_cache, const void *v_cache,
+                                      const int32_t *block_table, const int32_t *seq_lens,
+                                      int B, int Hq, int Hkv, int D, int num_blocks,
+                                      int block_tokens, int max_blocks, float k_scale,
+                                      float v_scale, float sm_scale, int window_left,
+                                      const float *sinks, void *out, float *lse,
+                                      void *workspace, size_t workspace_bytes, void *stream);
+
+/* Same, with a forced split size (0 = heuristic); for tests and tuning. */
+fpd_status fp8_paged_decode_attention_ex(const void *q, const void *k_cache, const void *v_cache,
+                                         const int32_t *block_table, const int32_t *seq_lens,
+                                         int B, int Hq, int Hkv, int D, int num_blocks,
+                                         int block_tokens, int max_blocks, float k_scale,
+                                         float v_scale, float sm_scale, int window_left,
+                                         const float *sinks, void *out, float *lse,
+                                         void *workspace, size_t workspace_bytes, void *stream,
+                                         int chunk_pages_override);
+
+/*
+ * Same as fp8_paged_decode_attention_ex, and additionally records the given
+ * cudaEvent_t handles (passed as void*, each may be NULL) on `stream`: one
+ * before the split kernel, one between the split and combine kernels, one after
+ * the combine kernel.  For measuring each kernel's duration with CUDA events on
+ * the stream the kernels run on; the kernels and their arguments are unchanged.
+ */
+fpd_status fp8_paged_decode_attention_profiled(const void *q, const void *k_cache,
+                                               const void *v_cache, const int32_t *block_table,
+                                               const int32_t *seq_lens, int B, int Hq, int Hkv,
+                                               int D, int num_blocks, int block_tokens,
+                                               int max_blocks, float k_scale, float v_scale,
+                                               float sm_scale, int window_left,
+                                               const float *sinks, void *out, float *lse,
+                                               void *workspace, size_t workspace_bytes,
+                                               void *stream, int chunk_pages_override,
+                                               void *event_before_split, void *event_after_split,
+                                               void *event_after_combine);
+
+/*
+ * Reads the workspace status word (FPD_DEVERR_* bits) after synchronising
+ * `stream`; clears it when `clear` is nonzero.  Writes the bits to
+ * *device_error_bits.  Needs a workspace of at least 256 bytes.
+ */
+fpd_status fp8_paged_decode_check_status(void *workspace, void *stream, int *device_error_bits,
+                                         int clear);
+
+/* Enqueue a zeroing of the workspace header (status word) on `stream`. */
+fpd_status fp8_paged_decode_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
+
+/* Human-readable name of a status code (static string). */
+const char *fp8_paged_decode_status_string(fpd_status status);
+
+/* Library version string, e.g. "0.1.0 sm_100a". */
+const char *fp8_paged_decode_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8_PAGED_DECODE_H */

@@ -1,0 +1,130 @@
+"""C-ABI library on the host (no GPU): loads, exports every declared symbol, and
+its planner / validation logic behave as documented.  No kernel is launched."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import fp8_paged_decode_b200 as fpd
+from fp8_paged_decode_b200 import build as fbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if fbuild.needs_build():
+        fbuild.build()
+    return fpd.load_library()
+
+
+def declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"\b(fp8_paged_decode_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert len(names) >= 9
+    raw = ctypes.CDLL(fpd.library_path())
+    for n in names:
+        assert hasattr(raw, n), f"{n} declared in include/ but not exported"
+    assert set(names) == set(fpd.EXPORTED_SYMBOLS)
+
+
+def test_version_and_status_strings(lib):
+    assert "sm_100a" in fpd.fp8_paged_decode_version()
+    assert fpd.fp8_paged_decode_status_string(fpd.FPD_ERR_UNSUPPORTED) == "FPD_ERR_UNSUPPORTED"
+    assert fpd.fp8_paged_decode_status_string(99) == "FPD_UNKNOWN_STATUS"
+
+
+def plan(**kw):
+    args = dict(B=32, Hq=32, Hkv=8, D=128, block_tokens=16, max_blocks=512, window_left=-1,
+                num_sms=148, ctas_per_sm=2, chunk_pages_override=0)
+    args.update(kw)
+    return fpd.fp8_paged_decode_make_plan(**args)
+
+
+def test_planner_fills_the_machine():
+    for shape in [dict(B=4, Hq=32, Hkv=8, block_tokens=64, max_blocks=2048),
+                  dict(B=32, Hq=32, Hkv=8, block_tokens=16, max_blocks=512),
+                  dict(B=256, Hq=64, Hkv=8, block_tokens=32, max_blocks=1024, window_left=4096)]:
+        p = plan(**shape)
+        assert p["ctas"] == shape["B"] * shape["Hkv"] * p["max_splits"]
+        # enough CTAs for several waves of 296 resident slots on long inputs
+        assert p["ctas"] >= 4 * 296
+        assert p["chunk_pages"] % p["pages_per_stage"] == 0
+        assert p["pages_per_stage"] * shape["block_tokens"] == 64
+
+
+def test_planner_window_caps_splits():
+    p = plan(B=64, Hq=64, Hkv=8, D=64, block_tokens=16, max_blocks=1024, window_left=128)
+    # a 129-token window spans at most 10 pages: a single split
+    assert p["max_splits"] == 1 and p["workspace_bytes"] == 256
+
+
+def test_planner_override_and_workspace():
+    p = plan(chunk_pages_override=5)
+    assert p["chunk_pages"] == 8          # rounded up to whole 4-page stages
+    assert p["max_splits"] == 512 // 8
+    ws = 256 + 32 * 32 * 64 * 128 * 4 + 32 * 32 * 64 * 4
+    assert p["workspace_bytes"] == ws
+    p1 = plan(chunk_pages_override=512)
+    assert p1["max_splits"] == 1 and p1["workspace_bytes"] == 256
+
+
+def test_planner_monotone_workspace():
+    prev = 0
+    for mb in (16, 64, 256, 1024):
+        w = plan(max_blocks=mb, chunk_pages_override=4)["workspace_bytes"]
+        assert w >= prev
+        prev = w
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(D=96), fpd.FPD_ERR_UNSUPPORTED),
+    (dict(D=256), fpd.FPD_ERR_UNSUPPORTED),
+    (dict(Hq=24, Hkv=8), fpd.FPD_ERR_UNSUPPORTED),     # g = 3
+    (dict(Hq=30, Hkv=8), fpd.FPD_ERR_INVALID_ARG),     # not a multiple
+    (dict(block_tokens=8), fpd.FPD_ERR_UNSUPPORTED),
+    (dict(block_tokens=128), fpd.FPD_ERR_UNSUPPORTED),
+    (dict(B=-1), fpd.FPD_ERR_INVALID_ARG),
+    (dict(max_blocks=0), fpd.FPD_ERR_INVALID_ARG),
+    (dict(num_sms=0), fpd.FPD_ERR_INVALID_ARG),
+    (dict(chunk_pages_override=-2), fpd.FPD_ERR_INVALID_ARG),
+])
+def test_planner_rejects(kw, status):
+    with pytest.raises(fpd.FpdError) as e:
+        plan(**kw)
+    assert e.value.status == status
+
+
+def test_attention_validates_before_any_launch(lib):
+    f = lib.fp8_paged_decode_attention
+    P = ctypes.c_void_p(4096)   # never dereferenced: validation fails first
+    args = [P, P, P, P, P, 2, 8, 2, 128, 10, 16, 4, 1.0, 1.0, 0.1, -1, None, P, None, P, 1 << 20, None]
+    bad = list(args); bad[8] = 80                       # D = 80
+    assert f(*bad) == fpd.FPD_ERR_UNSUPPORTED
+    bad = list(args); bad[0] = None                     # q == NULL
+    assert f(*bad) == fpd.FPD_ERR_INVALID_ARG
+    bad = list(args); bad[14] = 0.0                     # sm_scale * k_scale must be > 0
+    assert f(*bad) == fpd.FPD_ERR_INVALID_ARG
+    bad = list(args); bad[12] = float("nan")
+    assert f(*bad) == fpd.FPD_ERR_INVALID_ARG
+    bad = list(args); bad[0] = ctypes.c_void_p(4100)    # q not 16-byte aligned
+    assert f(*bad) == fpd.FPD_ERR_INVALID_ARG
+    bad = list(args); bad[9] = 0                        # empty pool
+    assert f(*bad) == fpd.FPD_ERR_UNSUPPORTED
+    ok = list(args); ok[5] = 0                          # B == 0: nothing to do
+    assert f(*ok) == fpd.FPD_OK
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(RuntimeError, match="no fallback"):
+        fpd.load_library(str(tmp_path / "absent.so"))
