@@ -53,8 +53,26 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU baseline sample budget")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--kernels-only", action="store_true",
+                    help="only run warm-up + K plain calls (for ncu launch lists and captures)")
     ap.add_argument("--json-out", default=None)
     return ap.parse_args()
+
+
+def whole_job_value(world_size, kv_bytes_per_call, steps, max_total_ms):
+    """Whole-job KV GB/s: every rank ran `steps` calls of `kv_bytes_per_call`; the
+    time is the maximum over ranks."""
+    return world_size * kv_bytes_per_call * steps / (max_total_ms / 1e3) / 1e9
+
+
+def max_over_ranks(value_ms, device=None):
+    """Max of a per-rank time over the process group (identity without one)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value_ms)], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
 
 
 def dist_env():
@@ -156,6 +174,37 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
                 "samples": len(rows), "power_w_max": max((num(r[3]) or 0) for r in rows)}
+
+
+class RawEvents:
+    """CUDA events created and read through the CUDA runtime directly, so that
+    events recorded inside the C library can be timed."""
+
+    def __init__(self, n):
+        from cuda.bindings import runtime as rt
+        self.rt = rt
+        self.ev = []
+        for _ in range(n):
+            err, e = rt.cudaEventCreate()
+            assert int(err) == 0, err
+            self.ev.append(e)
+
+    def handle(self, i):
+        return int(self.ev[i])
+
+    def record(self, i, stream_handle):
+        err, = self.rt.cudaEventRecord(self.ev[i], stream_handle)
+        assert int(err) == 0, err
+
+    def ms(self, i, j):
+        err, v = self.rt.cudaEventElapsedTime(self.ev[i], self.ev[j])
+        assert int(err) == 0, err
+        return float(v)
+
+    def close(self):
+        for e in self.ev:
+            self.rt.cudaEventDestroy(e)
+        self.ev = []
 
 
 # ------------------------------------------------------------ CPU oracle --
@@ -296,6 +345,21 @@ def run_native(args):
     f_prof = lib.fp8_paged_decode_attention_profiled
     f_plain = lib.fp8_paged_decode_attention_ex
 
+    if args.kernels_only:
+        for i in range(args.warmup + args.steps):
+            st = f_plain(*pre[i % replicas])
+            assert st == 0, fpd.fp8_paged_decode_status_string(st)
+        torch.cuda.synchronize()
+        assert fpd.fp8_paged_decode_check_status(wsp) == 0
+        if rank == 0:
+            print(json.dumps({"kernels_only": True, "config": args.config, "calls":
+                              args.warmup + args.steps, "launches_per_call":
+                              1 + (1 if plan["max_splits"] > 1 else 0), "plan": plan,
+                              "kv_bytes_per_call": kv_bytes, "replicas": replicas}))
+        if ws > 1:
+            dist.destroy_process_group()
+        return 0
+
     # correctness guard on this exact launch configuration (sampled rows vs oracle)
     st = f_plain(*pre[0])
     assert st == 0, fpd.fp8_paged_decode_status_string(st)
@@ -325,35 +389,31 @@ def run_native(args):
     torch.cuda.synchronize()
 
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev = RawEvents(3 * K + 2)   # per step: before split, after split, after combine; start, end
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.25)
     barrier()
     torch.cuda.synchronize()
-    start.record(stream)
+    ev.record(3 * K, stream.cuda_stream)
     for i in range(K):
-        e = evs[i]
-        st = f_prof(*pre[i % replicas], vp(e[0].cuda_event), vp(e[1].cuda_event),
-                    vp(e[2].cuda_event))
+        st = f_prof(*pre[i % replicas], vp(ev.handle(3 * i)), vp(ev.handle(3 * i + 1)),
+                    vp(ev.handle(3 * i + 2)))
         if st != 0:
             raise RuntimeError(fpd.fp8_paged_decode_status_string(st))
-    end.record(stream)
+    ev.record(3 * K + 1, stream.cuda_stream)
     torch.cuda.synchronize()
     barrier()
     clocks = sampler.stop()
-    total_ms = start.elapsed_time(end)
-    split_ms = [evs[i][0].elapsed_time(evs[i][1]) for i in range(K)]
-    call_ms = [evs[i][0].elapsed_time(evs[i][2]) for i in range(K)]
-    combine_ms = [evs[i][1].elapsed_time(evs[i][2]) for i in range(K)]
+    total_ms = ev.ms(3 * K, 3 * K + 1)
+    split_ms = [ev.ms(3 * i, 3 * i + 1) for i in range(K)]
+    call_ms = [ev.ms(3 * i, 3 * i + 2) for i in range(K)]
+    combine_ms = [ev.ms(3 * i + 1, 3 * i + 2) for i in range(K)]
+    ev.close()
 
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if ws > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_total_ms = float(t.item())
+    max_total_ms = max_over_ranks(total_ms, dev)
     ms_per_step = max_total_ms / K
-    value = ws * kv_bytes * K / (max_total_ms / 1e3) / 1e9
+    value = whole_job_value(ws, kv_bytes, K, max_total_ms)
 
     # end to end through the C ABI: pinned host inputs in, results out, every step
     e2e = None
@@ -388,12 +448,10 @@ def run_native(args):
         e2.record(stream)
         torch.cuda.synchronize()
         barrier()
-        te = torch.tensor([s2.elapsed_time(e2)], dtype=torch.float64, device=dev)
-        if ws > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e = {"value": ws * kv_bytes * Ke / (float(te.item()) / 1e3) / 1e9, "unit": UNIT,
+        te = max_over_ranks(s2.elapsed_time(e2), dev)
+        e2e = {"value": whole_job_value(ws, kv_bytes, Ke, te), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "ms_per_step": float(te.item()) / Ke,
+               "ms_per_step": te / Ke,
                "note": "q, block_table, seq_lens, sinks H2D from pinned host and out + lse D2H "
                        "every step; the KV cache is resident device state"}
 

@@ -46,6 +46,7 @@ def assert_parity(out, lse, ref_out, ref_lse, rows=None, what=""):
     assert not bad.any(), (f"{what}: {int(bad.sum())} outputs outside tolerance; worst "
                            f"|d|={err.max():.3e}")
     both_inf = np.isinf(lse) & np.isinf(ref_lse) & (np.sign(lse) == np.sign(ref_lse))
-    lerr = np.where(both_inf, 0.0, np.abs(lse - ref_lse))
+    with np.errstate(invalid="ignore"):
+        lerr = np.where(both_inf, 0.0, np.abs(lse - ref_lse))
     assert (lerr <= LSE_ATOL).all(), f"{what}: lse worst |d|={np.nanmax(lerr):.3e}"
     return float(err.max()), float(lerr.max())
