@@ -43,6 +43,7 @@ FPD_ERR_CUDA = 4
 FPD_DEVERR_SEQ_LEN = 0x1
 FPD_DEVERR_BLOCK_TABLE = 0x2
 FPD_DEVERR_TIMEOUT = 0x4
+FPD_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_NAME = "libfp8_paged_decode.so"
@@ -58,6 +59,7 @@ EXPORTED_SYMBOLS = (
     "fp8_paged_decode_attention",
     "fp8_paged_decode_attention_ex",
     "fp8_paged_decode_attention_profiled",
+    "fp8_paged_decode_attention_noalloc",
     "fp8_paged_decode_check_status",
     "fp8_paged_decode_workspace_init",
     "fp8_paged_decode_status_string",
@@ -99,6 +101,8 @@ def _bind(lib):
     lib.fp8_paged_decode_attention_ex.restype = ci
     lib.fp8_paged_decode_attention_profiled.argtypes = attn + [ci, vp, vp, vp]
     lib.fp8_paged_decode_attention_profiled.restype = ci
+    lib.fp8_paged_decode_attention_noalloc.argtypes = attn[:19] + [vp]
+    lib.fp8_paged_decode_attention_noalloc.restype = ci
     lib.fp8_paged_decode_check_status.argtypes = [vp, vp, ctypes.POINTER(ci), ci]
     lib.fp8_paged_decode_check_status.restype = ci
     lib.fp8_paged_decode_workspace_init.argtypes = [vp, cz, vp]

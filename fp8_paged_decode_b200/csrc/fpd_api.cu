@@ -408,6 +408,67 @@ fpd_status fp8_paged_decode_attention(const void* q, const void* k_cache, const 
                                        stream, 0);
 }
 
+}  // extern "C"
+
+namespace {
+
+// Scratch for fp8_paged_decode_attention_noalloc: split partials and status
+// word for callers that cannot allocate.  In host code this name is only a
+// stand-in; the device address comes from cudaGetSymbolAddress per device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[FPD_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (looked up once per
+// device, with that device current).  nullptr on failure.
+void* noalloc_scratch_address() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    g_noalloc_addr[dev] = ptr;
+  }
+  return g_noalloc_addr[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+fpd_status fp8_paged_decode_attention_noalloc(const void* q, const void* k_cache,
+                                              const void* v_cache, const int32_t* block_table,
+                                              const int32_t* seq_lens, int B, int Hq, int Hkv,
+                                              int D, int num_blocks, int bt, int max_blocks,
+                                              float k_scale, float v_scale, float sm_scale,
+                                              int window_left, const float* sinks, void* out,
+                                              float* lse, void* stream) {
+  fpd_status st = validate_shape(B, Hq, Hkv, D, bt, max_blocks);
+  if (st != FPD_OK) return st;
+  if (B == 0) return FPD_OK;
+  fpd_plan plan;
+  st = fp8_paged_decode_plan(B, Hq, Hkv, D, bt, max_blocks, window_left, 0, &plan);
+  if (st != FPD_OK) return st;
+  if (plan.workspace_bytes > FPD_NOALLOC_SCRATCH_BYTES) return FPD_ERR_WORKSPACE_TOO_SMALL;
+  void* scratch = noalloc_scratch_address();
+  if (!scratch) return FPD_ERR_CUDA;
+  // the status word must start at zero; the partials are fully rewritten
+  if (cudaMemsetAsync(scratch, 0, kHeaderBytes, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return FPD_ERR_CUDA;
+  return attention_impl(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, D, num_blocks, bt,
+                        max_blocks, k_scale, v_scale, sm_scale, window_left, sinks, out, lse,
+                        scratch, FPD_NOALLOC_SCRATCH_BYTES, stream, 0, nullptr, nullptr, nullptr);
+}
+
 fpd_status fp8_paged_decode_check_status(void* workspace, void* stream, int* device_error_bits,
                                          int clear) {
   if (!workspace || !device_error_bits) return FPD_ERR_INVALID_ARG;

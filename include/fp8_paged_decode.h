@@ -177,6 +177,49 @@ fpd_status fp8_paged_decode_attention_profiled(const void *q, const void *k_cach
                                                void *event_after_combine);
 
 /*
+ * Size of the library's static device scratch used by
+ * fp8_paged_decode_attention_noalloc: 16 MiB per GPU, held from the first use
+ * of the library on that GPU until the process exits.
+ */
+#define FPD_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+/*
+ * fp8_paged_decode_attention_noalloc -- the decode call for callers that cannot
+ * allocate device memory at all: code running where cudaMalloc is unavailable or
+ * forbidden (inside a custom allocator, a plug-in whose host owns all device
+ * memory, or a capture/replay path that must not create new allocations) and
+ * that therefore cannot provide the workspace fp8_paged_decode_attention needs.
+ * The pages describe no such entry point; it has no counterpart there.
+ *
+ * Arguments are those of fp8_paged_decode_attention without the workspace: the
+ * caller still passes every input and output.  The split partials and the status
+ * word live instead in one static device array of FPD_NOALLOC_SCRATCH_BYTES
+ * inside this library.  Behaviour:
+ *  - Nothing is allocated or freed: no cudaMalloc/cudaFree and no allocating
+ *    library routine on any call.
+ *  - A shape whose plan needs more scratch than FPD_NOALLOC_SCRATCH_BYTES is
+ *    rejected with FPD_ERR_WORKSPACE_TOO_SMALL before anything is launched.
+ *  - The first call on each device looks up the array's device address on that
+ *    device (cudaGetSymbolAddress); make that first call before any stream
+ *    capture on the device.  A failed lookup returns FPD_ERR_CUDA.
+ *  - Every call, on any stream, shares the one array, which keeps the previous
+ *    call's contents; each call zeroes the part that must start at zero (the
+ *    status word) on its own stream before its kernels.  Calls whose kernels
+ *    overlap on the GPU (different streams, no ordering between them) race on
+ *    the array and give wrong results; order them on one stream or use the
+ *    workspace entry point.
+ *  - Device status bits are kept in the shared array and are not reported.
+ */
+fpd_status fp8_paged_decode_attention_noalloc(const void *q, const void *k_cache,
+                                              const void *v_cache, const int32_t *block_table,
+                                              const int32_t *seq_lens, int B, int Hq, int Hkv,
+                                              int D, int num_blocks, int block_tokens,
+                                              int max_blocks, float k_scale, float v_scale,
+                                              float sm_scale, int window_left,
+                                              const float *sinks, void *out, float *lse,
+                                              void *stream);
+
+/*
  * Reads the workspace status word (FPD_DEVERR_* bits) after synchronising
  * `stream`; clears it when `clear` is nonzero.  Writes the bits to
  * *device_error_bits.  Needs a workspace of at least 256 bytes.
