@@ -6,7 +6,7 @@ tokens / call time), with % of the measured HBM peak and us/call.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl native|reference]
 
-One step = one decode call (split kernel + combine kernel) over the whole batch
+One step = one decode call (one persistent kernel: splits and their merge) over the whole batch
 of the named synthetic workload (default: the Llama-3-8B-shaped decode, B=32,
 Hq=32, Hkv=8, D=128, 16-token pages, lengths U[1024, 8192]).  Inputs are
 resident in HBM; consecutive steps read different replicas of the KV cache so
@@ -354,7 +354,7 @@ def run_native(args):
         if rank == 0:
             print(json.dumps({"kernels_only": True, "config": args.config, "calls":
                               args.warmup + args.steps, "launches_per_call":
-                              1 + (1 if plan["max_splits"] > 1 else 0), "plan": plan,
+                              1, "plan": plan,
                               "kv_bytes_per_call": kv_bytes, "replicas": replicas}))
         if ws > 1:
             dist.destroy_process_group()
@@ -476,7 +476,7 @@ def run_native(args):
                "sample": f"{nrows} random (sequence, head) rows of the workload, "
                          f"{kvb} KV bytes, {dt:.1f} s wall"}
 
-    launches_per_step = 1 + (1 if plan["max_splits"] > 1 else 0)
+    launches_per_step = 1   # one persistent kernel per call (split merge fused)
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": K,
@@ -496,7 +496,7 @@ def run_native(args):
             "us_per_call_p10_p90": [float(np.percentile(call_ms, 10) * 1e3),
                                     float(np.percentile(call_ms, 90) * 1e3)],
             "split_kernel_us": split_avg_ms * 1e3,
-            "combine_kernel_us": statistics.fmean(combine_ms) * 1e3,
+            "after_split_kernel_us": statistics.fmean(combine_ms) * 1e3,
             "pct_of_peak": 100.0 * value / hbm,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches_per_step * K, "clocks": clocks, "parity_guard": guard,

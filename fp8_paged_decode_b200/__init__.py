@@ -230,7 +230,9 @@ def fp8_paged_decode_attention(q, k_cache, v_cache, block_table, seq_lens, k_sca
     need = fp8_paged_decode_workspace_bytes_ex(B, Hq, Hkv, D, bt, max_blocks, window_left,
                                                chunk_pages_override)
     if workspace is None:
-        if need == 0 and B > 0:
+        if need == 0 and B > 0:   # surface the planner's own status
+            fp8_paged_decode_plan(B, Hq, Hkv, D, bt, max_blocks, window_left,
+                                  chunk_pages_override)
             raise FpdError(FPD_ERR_UNSUPPORTED, "fp8_paged_decode_workspace_bytes")
         workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)
     kv_types = (torch.uint8, torch.float8_e4m3fn)

@@ -1,6 +1,6 @@
 // fpd_api.cu -- host side of the C ABI declared in include/fp8_paged_decode.h:
-// argument validation, the split planner, TMA descriptor encoding and the two
-// kernel launches.  No call allocates or frees device memory, and only
+// argument validation, the split planner, TMA descriptor encoding and the
+// kernel launch.  No call allocates or frees device memory, and only
 // fp8_paged_decode_check_status synchronises.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -17,10 +17,10 @@
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr size_t kHeaderBytes = 256;    // status word + padding
-constexpr int kTargetWaves = 8;         // CTAs launched ~ this many waves of resident slots
-constexpr int kMinChunkTokens = 256;    // shortest KV range worth a CTA of its own
-constexpr int kRingBytesTarget = 96 * 1024;
+constexpr size_t kHeaderBytes = 256;    // status word, work counter, finished-CTA counter
+constexpr int kTargetWaves = 8;         // work items ~ this many per resident CTA slot
+constexpr int kMinChunkTokens = 256;    // shortest KV range worth its own work item
+constexpr int kOccCacheSize = 32;
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -37,85 +37,120 @@ fpd_status validate_shape(int B, int Hq, int Hkv, int D, int bt, int max_blocks)
   return FPD_OK;
 }
 
-int ring_stages(int D) {
-  const int stage_bytes = 2 * fpd::kTileTokens * D;
-  int s = kRingBytesTarget / stage_bytes;
-  return s < 2 ? 2 : (s > 8 ? 8 : s);
+int n_tiles(int g) { return g > 8 ? 2 : 1; }
+
+// Depth of the shared-memory stage ring (build-time tunable).
+#ifndef FPD_STAGES_D128_NT1
+#define FPD_STAGES_D128_NT1 3
+#endif
+#ifndef FPD_STAGES_D128_NT2
+#define FPD_STAGES_D128_NT2 4
+#endif
+#ifndef FPD_STAGES_D64
+#define FPD_STAGES_D64 6
+#endif
+int ring_stages(int D, int NT) {
+  if (D == 128) return NT == 2 ? FPD_STAGES_D128_NT2 : FPD_STAGES_D128_NT1;
+  return FPD_STAGES_D64;
 }
 
-int smem_bytes_for(int D, int g, int stages) {
-  const int NT = g > 8 ? 2 : 1;
-  int ring = stages * 2 * fpd::kTileTokens * D;
-  const int merge = fpd::kConsumerWarps * NT * 8 * D * 4 + fpd::kConsumerWarps * NT * 8 * 2 * 4;
-  if (ring < merge) ring = merge;
-  return ring + 2 * stages * 8 + 1024;  // barriers + slack for 1024-byte alignment
+int smem_bytes_for(int D, int g, int B) {
+  const int NT = n_tiles(g);
+  return fpd::smem_layout(D, NT, ring_stages(D, NT), B).total;
+}
+
+// Workspace carve-up: [header 256 B][partial O][partial lse]
+struct WsLayout {
+  size_t part_o, part_lse, total, zero_prefix;
+};
+
+WsLayout ws_layout(int B, int Hq, int Hkv, int D, int max_splits) {
+  (void)Hkv;
+  WsLayout w;
+  size_t off = kHeaderBytes;
+  w.zero_prefix = off;  // bytes that must be zero before the first call
+  w.part_o = off;
+  if (max_splits > 1) off += align_up((size_t)B * Hq * max_splits * D * sizeof(float), 256);
+  w.part_lse = off;
+  if (max_splits > 1) off += align_up((size_t)B * Hq * max_splits * sizeof(float), 256);
+  w.total = off;
+  return w;
 }
 
 // ---- per-device facts, queried once
+struct OccEntry {
+  int D, NT, smem, occ;
+};
 struct DeviceInfo {
   bool ready = false;
   int num_sms = 0;
-  int occ[2][2] = {{0, 0}, {0, 0}};  // [D==128][NT==2] CTAs per SM
+  int max_smem = 0;
+  int n_occ = 0;
+  OccEntry occ[kOccCacheSize];
 };
 std::mutex g_mu;
 DeviceInfo g_dev[kMaxDevices];
 
-template <int D, int NT>
-const void* split_kernel_ptr() {
-  return reinterpret_cast<const void*>(&fpd::fpd_split_kernel<D, NT>);
-}
-
 const void* split_kernel_for(int D, int NT) {
-  if (D == 128) return NT == 2 ? split_kernel_ptr<128, 2>() : split_kernel_ptr<128, 1>();
-  return NT == 2 ? split_kernel_ptr<64, 2>() : split_kernel_ptr<64, 1>();
+  if (D == 128)
+    return NT == 2 ? reinterpret_cast<const void*>(&fpd::fpd_split_kernel<128, 2>)
+                   : reinterpret_cast<const void*>(&fpd::fpd_split_kernel<128, 1>);
+  return NT == 2 ? reinterpret_cast<const void*>(&fpd::fpd_split_kernel<64, 2>)
+                 : reinterpret_cast<const void*>(&fpd::fpd_split_kernel<64, 1>);
 }
 
-bool device_info(int dev, DeviceInfo* out) {
-  if (dev < 0 || dev >= kMaxDevices) return false;
+bool current_device(int* dev) {
+  if (cudaGetDevice(dev) != cudaSuccess || *dev < 0 || *dev >= kMaxDevices) {
+    cudaGetLastError();
+    return false;
+  }
+  return true;
+}
+
+// SM count of the current device and the number of split-kernel CTAs that fit
+// on one SM with `smem` bytes of dynamic shared memory (0 if none).
+bool device_occupancy(int D, int NT, int smem, int* num_sms, int* ctas_per_sm) {
+  int dev = 0;
+  if (!current_device(&dev)) return false;
   std::lock_guard<std::mutex> lk(g_mu);
   DeviceInfo& di = g_dev[dev];
   if (!di.ready) {
-    int sms = 0;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    if (cudaDeviceGetAttribute(&di.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&di.max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+            cudaSuccess) {
+      cudaGetLastError();
       return false;
-    di.num_sms = sms;
-    for (int dsel = 0; dsel < 2; ++dsel) {
-      for (int nsel = 0; nsel < 2; ++nsel) {
-        const int D = dsel ? 128 : 64, NT = nsel ? 2 : 1;
-        const void* fn = split_kernel_for(D, NT);
-        const int smem = smem_bytes_for(D, NT == 2 ? 16 : 8, ring_stages(D));
-        if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-            cudaSuccess)
-          return false;
-        int occ = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, fpd::kThreads, smem) !=
-            cudaSuccess)
-          return false;
-        di.occ[dsel][nsel] = occ > 0 ? occ : 1;
-      }
     }
     di.ready = true;
   }
-  *out = di;
-  return true;
-}
-
-bool current_device_info(DeviceInfo* out, int* dev_out = nullptr) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) {
+  *num_sms = di.num_sms;
+  for (int i = 0; i < di.n_occ; ++i) {
+    const OccEntry& e = di.occ[i];
+    if (e.D == D && e.NT == NT && e.smem == smem) {
+      *ctas_per_sm = e.occ;
+      return true;
+    }
+  }
+  int occ = 0;
+  const void* fn = split_kernel_for(D, NT);
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) {
     cudaGetLastError();
     return false;
   }
-  if (dev_out) *dev_out = dev;
-  if (!device_info(dev, out)) {
-    cudaGetLastError();
-    return false;
+  const int dyn_max = di.max_smem - (int)fa.sharedSizeBytes;  // static + dynamic <= opt-in max
+  if (smem <= dyn_max) {
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn_max) !=
+            cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, fpd::kThreads, smem) !=
+            cudaSuccess) {
+      cudaGetLastError();
+      return false;
+    }
   }
+  if (di.n_occ < kOccCacheSize) di.occ[di.n_occ++] = OccEntry{D, NT, smem, occ};
+  *ctas_per_sm = occ;
   return true;
-}
-
-int ctas_per_sm_for(const DeviceInfo& di, int D, int g) {
-  return di.occ[D == 128 ? 1 : 0][g > 8 ? 1 : 0];
 }
 
 // ---- TMA descriptors
@@ -153,27 +188,27 @@ bool encode_cache_map(CUtensorMap* map, const void* base, int num_blocks, int bt
   return r == CUDA_SUCCESS;
 }
 
+// Combine launch as a programmatic dependent of the split kernel: its CTAs may
+// start while the split kernel drains and wait for it on the device.
+template <int D>
+cudaError_t launch_combine(const fpd::CombineParams& c, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(c.B * c.Hq));
+  cfg.blockDim = dim3(fpd::kCombineWarps * 32);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, fpd::fpd_combine_kernel<D>, c);
+}
+
 template <int D, int NT>
 cudaError_t launch_split(const CUtensorMap& km, const CUtensorMap& vm, const fpd::DecodeParams& p,
                          int ctas, int smem, cudaStream_t st) {
-  static bool attr_set[kMaxDevices] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < kMaxDevices && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(&fpd::fpd_split_kernel<D, NT>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
   fpd::fpd_split_kernel<D, NT><<<ctas, fpd::kThreads, smem, st>>>(km, vm, p);
-  return cudaGetLastError();
-}
-
-template <int D>
-cudaError_t launch_combine(const fpd::CombineParams& c, cudaStream_t st) {
-  const int rows = c.B * c.Hq;
-  const int blocks = (rows + 7) / 8;
-  fpd::fpd_combine_kernel<D><<<blocks, 256, 0, st>>>(c);
   return cudaGetLastError();
 }
 
@@ -194,7 +229,7 @@ const char* fp8_paged_decode_status_string(fpd_status s) {
   return "FPD_UNKNOWN_STATUS";
 }
 
-const char* fp8_paged_decode_version(void) { return "0.1.0 sm_100a"; }
+const char* fp8_paged_decode_version(void) { return "0.2.0 sm_100a"; }
 
 fpd_status fp8_paged_decode_make_plan(int B, int Hq, int Hkv, int D, int bt, int max_blocks,
                                       int window_left, int num_sms, int ctas_per_sm,
@@ -204,18 +239,19 @@ fpd_status fp8_paged_decode_make_plan(int B, int Hq, int Hkv, int D, int bt, int
   if (st != FPD_OK) return st;
   if (num_sms <= 0 || ctas_per_sm <= 0 || chunk_pages_override < 0) return FPD_ERR_INVALID_ARG;
   const int g = Hq / Hkv;
+  const int NT = n_tiles(g);
   const int pps = fpd::kTileTokens / bt;
   int pages_max = max_blocks;
   if (window_left >= 0) {
     const int64_t w = (int64_t)window_left / bt + 2;
     if (w < pages_max) pages_max = (int)w;
   }
+  const int64_t units = (int64_t)(B > 0 ? B : 1) * Hkv;
+  const int64_t slots = (int64_t)num_sms * ctas_per_sm;
   int chunk;
   if (chunk_pages_override > 0) {
     chunk = chunk_pages_override;
   } else {
-    const int64_t units = (int64_t)(B > 0 ? B : 1) * Hkv;
-    const int64_t slots = (int64_t)num_sms * ctas_per_sm;
     int64_t splits = (kTargetWaves * slots + units - 1) / units;
     if (splits < 1) splits = 1;
     chunk = (int)((pages_max + splits - 1) / splits);
@@ -224,19 +260,14 @@ fpd_status fp8_paged_decode_make_plan(int B, int Hq, int Hkv, int D, int bt, int
   }
   chunk = (chunk + pps - 1) / pps * pps;
   const int max_splits = (pages_max + chunk - 1) / chunk;
-  const int stages = ring_stages(D);
+  const int64_t items_max = units * max_splits;
   plan->chunk_pages = chunk;
   plan->max_splits = max_splits;
   plan->pages_per_stage = pps;
-  plan->stages = stages;
-  plan->ctas = (int)((int64_t)B * Hkv * max_splits);
-  plan->smem_bytes = smem_bytes_for(D, g, stages);
-  size_t ws = kHeaderBytes;
-  if (max_splits > 1) {
-    ws += align_up((size_t)B * Hq * max_splits * D * sizeof(float), 256);
-    ws += align_up((size_t)B * Hq * max_splits * sizeof(float), 256);
-  }
-  plan->workspace_bytes = ws;
+  plan->stages = ring_stages(D, NT);
+  plan->ctas = (int)(items_max < slots ? items_max : slots);
+  plan->smem_bytes = smem_bytes_for(D, g, B);
+  plan->workspace_bytes = ws_layout(B, Hq, Hkv, D, max_splits).total;
   return FPD_OK;
 }
 
@@ -245,10 +276,12 @@ fpd_status fp8_paged_decode_plan(int B, int Hq, int Hkv, int D, int bt, int max_
   if (!plan) return FPD_ERR_INVALID_ARG;
   fpd_status st = validate_shape(B, Hq, Hkv, D, bt, max_blocks);
   if (st != FPD_OK) return st;
-  DeviceInfo di;
-  if (!current_device_info(&di)) return FPD_ERR_CUDA;
-  return fp8_paged_decode_make_plan(B, Hq, Hkv, D, bt, max_blocks, window_left, di.num_sms,
-                                    ctas_per_sm_for(di, D, Hq / Hkv), chunk_pages_override, plan);
+  const int g = Hq / Hkv;
+  int sms = 0, occ = 0;
+  if (!device_occupancy(D, n_tiles(g), smem_bytes_for(D, g, B), &sms, &occ)) return FPD_ERR_CUDA;
+  if (occ <= 0) return FPD_ERR_UNSUPPORTED;  // the batch's shared-memory table does not fit
+  return fp8_paged_decode_make_plan(B, Hq, Hkv, D, bt, max_blocks, window_left, sms, occ,
+                                    chunk_pages_override, plan);
 }
 
 size_t fp8_paged_decode_workspace_bytes_ex(int B, int Hq, int Hkv, int D, int bt, int max_blocks,
@@ -301,11 +334,8 @@ static fpd_status attention_impl(const void* q, const void* k_cache, const void*
       !encode_cache_map(&vm, v_cache, num_blocks, bt, Hkv, D))
     return FPD_ERR_CUDA;
 
+  const WsLayout wl = ws_layout(B, Hq, Hkv, D, plan.max_splits);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  float* part_o = reinterpret_cast<float*>(ws + kHeaderBytes);
-  float* part_lse = reinterpret_cast<float*>(
-      ws + kHeaderBytes + align_up((size_t)B * Hq * plan.max_splits * D * sizeof(float), 256));
-
   fpd::DecodeParams p;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.block_table = block_table;
@@ -313,9 +343,10 @@ static fpd_status attention_impl(const void* q, const void* k_cache, const void*
   p.sinks = sinks;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
-  p.part_o = part_o;
-  p.part_lse = part_lse;
+  p.part_o = reinterpret_cast<float*>(ws + wl.part_o);
+  p.part_lse = reinterpret_cast<float*>(ws + wl.part_lse);
   p.status = reinterpret_cast<uint32_t*>(ws);
+  p.sched = reinterpret_cast<uint32_t*>(ws) + 1;
   p.B = B;
   p.Hq = Hq;
   p.Hkv = Hkv;
@@ -332,9 +363,9 @@ static fpd_status attention_impl(const void* q, const void* k_cache, const void*
   p.v_scale = v_scale;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e;
   if (ev0 && cudaEventRecord(static_cast<cudaEvent_t>(ev0), s) != cudaSuccess) return FPD_ERR_CUDA;
-  const int NT = g > 8 ? 2 : 1;
+  cudaError_t e;
+  const int NT = n_tiles(g);
   if (D == 128)
     e = NT == 2 ? launch_split<128, 2>(km, vm, p, plan.ctas, plan.smem_bytes, s)
                 : launch_split<128, 1>(km, vm, p, plan.ctas, plan.smem_bytes, s);
@@ -343,14 +374,13 @@ static fpd_status attention_impl(const void* q, const void* k_cache, const void*
                 : launch_split<64, 1>(km, vm, p, plan.ctas, plan.smem_bytes, s);
   if (e != cudaSuccess) return FPD_ERR_CUDA;
   if (ev1 && cudaEventRecord(static_cast<cudaEvent_t>(ev1), s) != cudaSuccess) return FPD_ERR_CUDA;
-
   if (plan.max_splits > 1) {
     fpd::CombineParams c;
     c.seq_lens = seq_lens;
     c.sinks = sinks;
-    c.part_o = part_o;
-    c.part_lse = part_lse;
-    c.out = static_cast<__nv_bfloat16*>(out);
+    c.part_o = p.part_o;
+    c.part_lse = p.part_lse;
+    c.out = p.out;
     c.lse = lse;
     c.B = B;
     c.Hq = Hq;
@@ -412,9 +442,9 @@ fpd_status fp8_paged_decode_attention(const void* q, const void* k_cache, const 
 
 namespace {
 
-// Scratch for fp8_paged_decode_attention_noalloc: split partials and status
-// word for callers that cannot allocate.  In host code this name is only a
-// stand-in; the device address comes from cudaGetSymbolAddress per device.
+// Scratch for fp8_paged_decode_attention_noalloc: split partials, work
+// counters and status word for callers that cannot allocate.  In host code this name is only
+// a stand-in; the device address comes from cudaGetSymbolAddress per device.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[FPD_NOALLOC_SCRATCH_BYTES];
 
 std::mutex g_noalloc_mu;
@@ -460,9 +490,10 @@ fpd_status fp8_paged_decode_attention_noalloc(const void* q, const void* k_cache
   if (plan.workspace_bytes > FPD_NOALLOC_SCRATCH_BYTES) return FPD_ERR_WORKSPACE_TOO_SMALL;
   void* scratch = noalloc_scratch_address();
   if (!scratch) return FPD_ERR_CUDA;
-  // the status word must start at zero; the partials are fully rewritten
-  if (cudaMemsetAsync(scratch, 0, kHeaderBytes, static_cast<cudaStream_t>(stream)) !=
-      cudaSuccess)
+  // the status word and the work counters must start at zero; the partials
+  // are fully rewritten
+  const size_t zero = ws_layout(B, Hq, Hkv, D, plan.max_splits).zero_prefix;
+  if (cudaMemsetAsync(scratch, 0, zero, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return FPD_ERR_CUDA;
   return attention_impl(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, D, num_blocks, bt,
                         max_blocks, k_scale, v_scale, sm_scale, window_left, sinks, out, lse,
@@ -487,7 +518,7 @@ fpd_status fp8_paged_decode_check_status(void* workspace, void* stream, int* dev
 
 fpd_status fp8_paged_decode_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {
   if (!workspace || workspace_bytes < kHeaderBytes) return FPD_ERR_INVALID_ARG;
-  if (cudaMemsetAsync(workspace, 0, kHeaderBytes, static_cast<cudaStream_t>(stream)) !=
+  if (cudaMemsetAsync(workspace, 0, workspace_bytes, static_cast<cudaStream_t>(stream)) !=
       cudaSuccess)
     return FPD_ERR_CUDA;
   return FPD_OK;

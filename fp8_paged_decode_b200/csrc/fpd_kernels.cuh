@@ -1,22 +1,34 @@
-// fpd_kernels.cuh -- sm_100a kernels of the paged E4M3 decode attention.
+// fpd_kernels.cuh -- the sm_100a kernel of the paged E4M3 decode attention.
 //
-// Split kernel: one CTA per (sequence b, KV head, KV split).  Warp 4 is the
-// producer: it walks the block table and issues one TMA box per (page, K/V)
-// into a ring of shared-memory stages (128-byte swizzle, so the consumers'
-// fragment loads are bank-conflict free).  Warps 0..3 are consumers: each owns
-// 16 token rows of every 64-token stage and runs
-//   S^T = K Q^T      mma.sync m16n8k16, tokens on M, the g query heads of the
-//                    KV head on N (heads on the MMA N side, as in the "SwapsAb"
-//                    orientation of FlashInfer PR #5591, Summary),
-//   online softmax   base 2, with a lazy running max (the max moves only when
-//                    a tile exceeds it by more than 8 in the exp2 domain, the
-//                    lazy-rescale rule of the same PR's Summary),
-//   O^T += V^T P^T   mma.sync m16n8k16, head dim on M, heads on N,
-// with E4M3 -> f16 conversion in registers (exact).  The per-tensor scales
-// are folded: logits use sm_scale * k_scale, the output uses v_scale.
-// The four consumer warps are merged in shared memory at the end; a sequence
-// handled by one split writes bf16 out / lse directly (sink folded in), others
-// write fp32 partials (O / l, log2-sum-exp) that the combine kernel merges.
+// One persistent kernel.  Each CTA (one or more per SM) pulls work items from
+// a global counter; an item is (sequence b, KV head, KV split) and covers up
+// to `chunk_pages` pages of that sequence's attended range.  Warp 4 is the
+// producer: for every item it publishes a small header plus the item's query
+// rows (bulk copy) in a 2-slot header ring, then streams the item's pages with
+// TMA tiled loads (one box per page of one KV head, K and V, 128-byte swizzle)
+// into a ring of shared-memory stages.  The stage ring runs straight across
+// item boundaries, so HBM reads never wait for an item to start.
+//
+// Warps 0..3 are consumers: each owns 16 token rows of every 64-token stage:
+//   S^T = K Q^T      mma.sync m16n8k16, tokens on M, the query heads of the KV
+//                    head on N (heads on the MMA N side, as in the "SwapsAb"
+//                    orientation of FlashInfer PR #5591, Summary);
+//   online softmax   base 2 with a lazy running max: the max moves only when a
+//                    tile exceeds it by more than 8 in the exp2 domain (the
+//                    lazy-rescale rule of the same PR's Summary);
+//   O^T += V^T P^T   mma.sync m16n8k16, head dim on M, heads on N;
+// with E4M3 -> f16 conversion in registers (exact) and the per-tensor scales
+// folded into the logit scale and the output.  At the end of an item the four
+// warps merge in shared memory.  An item that covers its whole sequence writes
+// bf16 out and lse (sink folded in).  Otherwise it writes an fp32 partial
+// (O / l and log2-sum-exp), and the combine kernel, launched as a programmatic
+// dependent of this one (its CTAs start during this kernel's tail and wait for
+// its completion; the FP8 paged-MLA route on the FlashInfer PR #5591 page,
+// section "Unsupported", launches its split-KV merge the same way), merges the
+// partials of every sequence
+// that spans several splits and folds in the sink.  The last CTA to leave
+// resets the work counter, so the workspace needs zeroing only once after
+// allocation.
 //
 // Fragment layouts (PTX ISA, mma.m16n8k16 with .f16):
 //   A: a0 (row g, cols 2t..2t+1), a1 (row g+8, same), a2 (row g, cols 2t+8..),
@@ -29,6 +41,10 @@
 //   QK k-step ks, slot 2t+u  -> d = t*(D/4) + 4*ks + u      (u in 0..1)
 //               slot 2t+8+u  -> d = t*(D/4) + 4*ks + 2 + u
 //   PV m-tile i, row g+8h    -> d = g*(D/8) + 2*i + h        (h in 0..1)
+//
+// Every wait (mbarrier phase, consumer-group sync) is bounded in time; on
+// expiry the kernel sets FPD_DEVERR_TIMEOUT in the status word and the warp
+// leaves, so a fault upstream can never hang the GPU.
 #pragma once
 
 #include <cmath>
@@ -45,11 +61,17 @@ constexpr int kConsumerWarps = 4;
 constexpr int kRowsPerWarp = 16;
 constexpr int kTileTokens = kConsumerWarps * kRowsPerWarp;  // tokens per stage
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
-constexpr float kLazyThreshold = 8.0f;      // log2 units
+constexpr int kHdrSlots = 2;
+constexpr int kHdrBytes = 64;                 // ItemHeader, padded
+constexpr float kLazyThreshold = 8.0f;        // log2 units
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-constexpr uint64_t kWaitLimitNs = 500000000ull;   // 0.5 s: far above any legitimate wait
-constexpr uint64_t kDrainLimitNs = 50000000ull;   // 50 ms per stage when draining after a timeout
+constexpr uint64_t kWaitLimitNs = 500000000ull;  // 0.5 s: far above any legitimate wait
+constexpr uint64_t kDrainLimitNs = 50000000ull;  // 50 ms per stage when draining
+
+constexpr uint32_t kErrSeqLen = 0x1u;
+constexpr uint32_t kErrBlockTable = 0x2u;
+constexpr uint32_t kErrTimeout = 0x4u;
 
 struct DecodeParams {
   const __nv_bfloat16* q;
@@ -58,16 +80,51 @@ struct DecodeParams {
   const float* sinks;
   __nv_bfloat16* out;
   float* lse;
-  float* part_o;     // [B, Hq, max_splits, D]
-  float* part_lse;   // [B, Hq, max_splits]   (log2 domain)
-  uint32_t* status;  // workspace header word
+  float* part_o;        // [B, Hq, max_splits, D]
+  float* part_lse;      // [B, Hq, max_splits]   (log2 domain)
+  uint32_t* status;     // workspace word 0: sticky FPD_DEVERR_* bits
+  uint32_t* sched;      // workspace words 1, 2: next work item, CTAs finished
   int B, Hq, Hkv, g, bt, max_blocks, num_blocks, window_left;
   int chunk_pages, max_splits, pages_per_stage, stages;
   float qk_scale_log2;  // sm_scale * k_scale * log2(e)
   float v_scale;
 };
 
-// Attended page range of sequence b, shared by both kernels.
+// Shared-memory carve-up (byte offsets from a 1024-byte aligned base); used by
+// the host to size the launch and by the kernel to find its buffers.
+struct SmemLayout {
+  int ring, merge, hdr, prefix, bars, total;
+};
+
+__host__ __device__ constexpr int align_to(int x, int a) { return (x + a - 1) / a * a; }
+
+__host__ __device__ inline SmemLayout smem_layout(int D, int NT, int stages, int B) {
+  SmemLayout L{};
+  const int H = NT * 8;
+  L.ring = 0;
+  L.merge = stages * 2 * kTileTokens * D;
+  const int merge_bytes = kConsumerWarps * H * (D + 4) * 4 + kConsumerWarps * H * 2 * 4;
+  L.hdr = align_to(L.merge + merge_bytes, 128);
+  const int hdr_slot = kHdrBytes + H * D * 2;
+  L.prefix = align_to(L.hdr + kHdrSlots * hdr_slot, 16);
+  L.bars = align_to(L.prefix + 4 * (B + 1), 16);
+  L.total = align_to(L.bars + (2 * stages + 2 * kHdrSlots + 1) * 8, 16) +
+            1024;  // + slack to align the base to 1024
+  return L;
+}
+
+struct ItemHeader {
+  int kind;      // 1: work item, -1: no more work
+  int b, kvh, split;
+  int ns;        // splits of this sequence (0: empty sequence)
+  int n_stages;  // pipeline stages this item consumes
+  int pb;        // first page of the item
+  int tok_lo, tok_hi;
+  int pad[7];
+};
+static_assert(sizeof(ItemHeader) == kHdrBytes, "header size");
+
+// Attended page range of a sequence.
 struct SeqRange {
   int L, start, first_page, end_page, n_splits;
 };
@@ -78,7 +135,7 @@ __device__ __forceinline__ SeqRange seq_range(int L_raw, int bt, int max_blocks,
   int L = L_raw;
   const int cap = max_blocks * bt;
   if (L < 0 || L > cap) {
-    if (status) atomicOr(status, 0x1u);
+    if (status) atomicOr(status, kErrSeqLen);
     L = L < 0 ? 0 : cap;
   }
   r.L = L;
@@ -90,12 +147,28 @@ __device__ __forceinline__ SeqRange seq_range(int L_raw, int bt, int max_blocks,
   return r;
 }
 
+// Work groups (one per split; one for an empty sequence) of a sequence.
+__device__ __forceinline__ int groups_of(int L_raw, const DecodeParams& p) {
+  const SeqRange r =
+      seq_range(L_raw, p.bt, p.max_blocks, p.window_left, p.chunk_pages, nullptr);
+  return r.n_splits > 0 ? r.n_splits : 1;
+}
+
 // Byte offset inside a 1024-byte-aligned tile written by TMA with 128-byte
 // (D = 128) or 64-byte (D = 64) swizzle: 16-byte chunk index XOR line bits.
 template <int D>
 __device__ __forceinline__ uint32_t swz(uint32_t off) {
   constexpr uint32_t mask = (D == 128) ? 7u : 3u;
   return off ^ (((off >> 7) & mask) << 4);
+}
+
+// Bounded barrier among the four consumer warps (one arrival per warp).
+__device__ __forceinline__ bool consumer_sync(uint64_t* bar, uint32_t& parity, int lane) {
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar);
+  const bool ok = mbar_wait_bounded(bar, parity, kWaitLimitNs);
+  parity ^= 1u;
+  return __all_sync(0xffffffffu, ok);
 }
 
 template <int D, int NT>
@@ -111,7 +184,9 @@ struct Consumer {
   float l[NT][2];           // partial row sums (this thread's tokens only)
   float o[MT][NT][4];       // O^T accumulators
 
-  __device__ __forceinline__ void init(const DecodeParams& p, int b, int kvh, int lane) {
+  // qtile: the item's query rows, bf16 [g][D] in shared memory.
+  __device__ __forceinline__ void init(const DecodeParams& p, const __nv_bfloat16* qtile,
+                                       int lane) {
     const int n = lane >> 2, t = lane & 3;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
@@ -119,7 +194,7 @@ struct Consumer {
       float vals[QW];
       float amax = 0.f;
       if (hl < p.g) {
-        const __nv_bfloat16* src = p.q + ((size_t)b * p.Hq + kvh * p.g + hl) * D + t * QW;
+        const __nv_bfloat16* src = qtile + hl * D + t * QW;
 #pragma unroll
         for (int i = 0; i < QW; i += 8) {
           const uint4 raw = *reinterpret_cast<const uint4*>(src + i);
@@ -212,11 +287,10 @@ struct Consumer {
 #pragma unroll
       for (int j = 0; j < 4; ++j) acc[nt][j] = s[nt][0][j] + s[nt][1][j];
 
-    bool v0 = true, v1 = true;  // rows n and n+8 inside the attended range
     if (!FULL) {
       const int tk0 = tok0 + n, tk1 = tok0 + n + 8;
-      v0 = tk0 >= tok_lo && tk0 < tok_hi;
-      v1 = tk1 >= tok_lo && tk1 < tok_hi;
+      const bool v0 = tk0 >= tok_lo && tk0 < tok_hi;
+      const bool v1 = tk1 >= tok_lo && tk1 < tok_hi;
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         if (!v0) acc[nt][0] = acc[nt][1] = -INFINITY;
@@ -330,91 +404,100 @@ struct Consumer {
   }
 };
 
-// Merge scratch per CTA (reuses the stage ring): [warp][head][D] O plus
-// [warp][head] (m, l).
-template <int D, int NT>
-struct MergeLayout {
-  static constexpr int H = NT * 8;
-  static constexpr int kOBytes = kConsumerWarps * H * D * 4;
-  static constexpr int kMLBytes = kConsumerWarps * H * 2 * 4;
-  static constexpr int kBytes = kOBytes + kMLBytes;
-};
+// ---------------------------------------------------------------- producer --
 
-template <int D, int NT>
-__global__ void __launch_bounds__(kThreads)
-fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
-                 const DecodeParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+template <int D>
+__device__ __forceinline__ void producer_loop(const CUtensorMap* kmap, const CUtensorMap* vmap,
+                                              const DecodeParams& p, uint8_t* smem,
+                                              const SmemLayout& L, const int* prefix,
+                                              int total_items, int hdr_slot_bytes,
+                                              uint64_t* full_bar, uint64_t* empty_bar,
+                                              uint64_t* hdr_full, uint64_t* hdr_empty, int lane) {
   constexpr int kTileBytes = kTileTokens * D;
   const int stages = p.stages;
-  int ring_bytes = stages * 2 * kTileBytes;
-  if (ring_bytes < MergeLayout<D, NT>::kBytes) ring_bytes = MergeLayout<D, NT>::kBytes;
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + ring_bytes);
-  uint64_t* empty_bar = full_bar + stages;
-
-  int bid = blockIdx.x;
-  const int kvh = bid % p.Hkv;
-  bid /= p.Hkv;
-  const int split = bid % p.max_splits;
-  const int b = bid / p.max_splits;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  const SeqRange R = seq_range(p.seq_lens[b], p.bt, p.max_blocks, p.window_left, p.chunk_pages,
-                               threadIdx.x == 0 ? p.status : nullptr);
-  if (split >= (R.n_splits > 0 ? R.n_splits : 1)) return;
-  if (R.n_splits == 0) {  // empty sequence: out = 0, lse = sigma
-    for (int i = threadIdx.x; i < p.g * D; i += blockDim.x) {
-      const int h = kvh * p.g + i / D;
-      p.out[((size_t)b * p.Hq + h) * D + (i % D)] = __float2bfloat16_rn(0.f);
-    }
-    for (int i = threadIdx.x; i < p.g; i += blockDim.x) {
-      const int h = kvh * p.g + i;
-      if (p.lse) p.lse[(size_t)b * p.Hq + h] = p.sinks ? p.sinks[h] : -INFINITY;
-    }
-    return;
-  }
-  const int pb = R.first_page + split * p.chunk_pages;
-  const int pe = min(pb + p.chunk_pages, R.end_page);
-  const int tok_lo = max(R.start, pb * p.bt);
-  const int tok_hi = min(R.L, pe * p.bt);
   const int pps = p.pages_per_stage;
-  const int n_stages = (pe - pb + pps - 1) / pps;
-  const bool single = (R.n_splits == 1);
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < stages; ++s) {
-      mbar_init(&full_bar[s], 1);
-      mbar_init(&empty_bar[s], kConsumerWarps);
-    }
-    fence_mbarrier_init();
+  const uint32_t page_bytes = (uint32_t)(p.bt * D);
+  const uint64_t policy = l2_policy_evict_first();
+  if (lane == 0) {
+    tma_prefetch_desc(kmap);
+    tma_prefetch_desc(vmap);
   }
-  __syncthreads();
-
-  bool timed_out = false;
-  if (warp == kConsumerWarps) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      tma_prefetch_desc(&kmap);
-      tma_prefetch_desc(&vmap);
+  int hs = 0, rs = 0;
+  uint32_t item = 0;
+  if (lane == 0) item = atomicAdd(&p.sched[0], 1u);
+  item = __shfl_sync(0xffffffffu, item, 0);
+  for (;;) {
+    const bool done = item >= (uint32_t)total_items;
+    uint32_t next = 0;
+    if (!done && lane == 0) next = atomicAdd(&p.sched[0], 1u);   // latency hidden below
+    const int hslot = hs % kHdrSlots;
+    if (hs >= kHdrSlots) {
+      const bool ok =
+          mbar_wait_bounded(&hdr_empty[hslot], ((hs / kHdrSlots) - 1) & 1, kWaitLimitNs);
+      if (!__all_sync(0xffffffffu, ok)) {
+        if (lane == 0) atomicOr(p.status, kErrTimeout);
+        return;
+      }
     }
-    const uint64_t policy = l2_policy_evict_first();
+    ItemHeader* hdr = reinterpret_cast<ItemHeader*>(smem + L.hdr + hslot * hdr_slot_bytes);
+    if (done) {
+      if (lane == 0) {
+        hdr->kind = -1;
+        mbar_arrive(&hdr_full[hslot]);
+      }
+      return;
+    }
+    // item -> (group, kv head) -> (sequence, split) by binary search of the prefix
+    const int group = (int)item / p.Hkv;
+    const int kvh = (int)item % p.Hkv;
+    int lo = 0, hi = p.B;   // largest b with prefix[b] <= group
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (prefix[mid] <= group) lo = mid; else hi = mid;
+    }
+    const int b = lo;
+    const int split = group - prefix[b];
+    const SeqRange R = seq_range(__ldg(p.seq_lens + b), p.bt, p.max_blocks, p.window_left,
+                                 p.chunk_pages, lane == 0 ? p.status : nullptr);
+    int pb = 0, pe = 0, tok_lo = 0, tok_hi = 0, n_st = 0;
+    if (R.n_splits > 0) {
+      pb = R.first_page + split * p.chunk_pages;
+      pe = min(pb + p.chunk_pages, R.end_page);
+      tok_lo = max(R.start, pb * p.bt);
+      tok_hi = min(R.L, pe * p.bt);
+      n_st = (pe - pb + pps - 1) / pps;
+    }
+    if (lane == 0) {
+      hdr->kind = 1;
+      hdr->b = b;
+      hdr->kvh = kvh;
+      hdr->split = split;
+      hdr->ns = R.n_splits;
+      hdr->n_stages = n_st;
+      hdr->pb = pb;
+      hdr->tok_lo = tok_lo;
+      hdr->tok_hi = tok_hi;
+      const uint32_t qbytes = (uint32_t)(p.g * D * 2);
+      mbar_arrive_expect_tx(&hdr_full[hslot], qbytes);
+      bulk_load(smem + L.hdr + hslot * hdr_slot_bytes + kHdrBytes,
+                p.q + ((size_t)b * p.Hq + (size_t)kvh * p.g) * D, qbytes, &hdr_full[hslot]);
+    }
+    ++hs;
+
+    // ---- stream the item's pages; block-table entries 32 at a time
     const int32_t* tbl = p.block_table + (size_t)b * p.max_blocks;
-    const uint32_t page_bytes = (uint32_t)(p.bt * D);
-    int batch_base = -1;
-    int my_entry = 0;
-    for (int s = 0; s < n_stages && !timed_out; ++s) {
-      const int slot = s % stages;
-      if (s >= stages) {
-        if (!mbar_wait_bounded(&empty_bar[slot], ((s / stages) - 1) & 1, kWaitLimitNs))
-          timed_out = true;
-        timed_out = __any_sync(0xffffffffu, timed_out);
-        if (timed_out) break;
+    int batch_base = -1, my_entry = 0;
+    for (int s = 0; s < n_st; ++s, ++rs) {
+      const int slot = rs % stages;
+      if (rs >= stages) {
+        const bool ok = mbar_wait_bounded(&empty_bar[slot], ((rs / stages) - 1) & 1, kWaitLimitNs);
+        if (!__all_sync(0xffffffffu, ok)) {
+          if (lane == 0) atomicOr(p.status, kErrTimeout);
+          return;
+        }
       }
       const int pg0 = pb + s * pps;
       const int np = min(pps, pe - pg0);
-      // block-table entries are fetched 32 at a time by the warp's lanes
       const int rel = pg0 - pb;
       if ((rel & ~31) != batch_base) {
         batch_base = rel & ~31;
@@ -426,124 +509,241 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
       for (int i = 0; i < 4; ++i) {
         const int e = __shfl_sync(0xffffffffu, my_entry, (rel + i) & 31);
         const bool ok = (e >= 0 && e < p.num_blocks);
-        if (!ok && i < np && lane == 0) atomicOr(p.status, 0x2u);
+        if (!ok && i < np && lane == 0) atomicOr(p.status, kErrBlockTable);
         // an invalid page is read from past the end of the pool: TMA zero-fills it
         rows[i] = ok ? e * p.bt : p.num_blocks * p.bt;
       }
       if (lane == 0) {
-        uint8_t* kdst = smem + slot * 2 * kTileBytes;
+        uint8_t* kdst = smem + L.ring + slot * 2 * kTileBytes;
         uint8_t* vdst = kdst + kTileBytes;
         mbar_arrive_expect_tx(&full_bar[slot], 2u * page_bytes * (uint32_t)np);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           if (i < np) {
-            tma_load_3d(kdst + i * page_bytes, &kmap, 0, kvh, rows[i], &full_bar[slot], policy);
-            tma_load_3d(vdst + i * page_bytes, &vmap, 0, kvh, rows[i], &full_bar[slot], policy);
+            tma_load_3d(kdst + i * page_bytes, kmap, 0, kvh, rows[i], &full_bar[slot], policy);
+            tma_load_3d(vdst + i * page_bytes, vmap, 0, kvh, rows[i], &full_bar[slot], policy);
           }
         }
       }
     }
-    if (timed_out && lane == 0) atomicOr(p.status, 0x4u);
+    item = __shfl_sync(0xffffffffu, next, 0);
+  }
+}
+
+// ------------------------------------------------------------------ kernel --
+
+// CTAs per SM the register budget is sized for (register cap 64K / (160 * n)).
+#ifndef FPD_MINB_D128_NT1
+#define FPD_MINB_D128_NT1 3
+#endif
+template <int D, int NT>
+struct MinBlocks {
+  static constexpr int value = (D == 128) ? (NT == 1 ? FPD_MINB_D128_NT1 : 2) : (NT == 1 ? 4 : 3);
+};
+
+template <int D, int NT>
+__global__ void __launch_bounds__(kThreads, MinBlocks<D, NT>::value)
+fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                 const DecodeParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ int warp_tot[kThreads / 32];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  constexpr int kTileBytes = kTileTokens * D;
+  constexpr int H = NT * 8;
+  const int stages = p.stages;
+  const SmemLayout L = smem_layout(D, NT, stages, p.B);
+  int* prefix = reinterpret_cast<int*>(smem + L.prefix);
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + L.bars);
+  uint64_t* empty_bar = full_bar + stages;
+  uint64_t* hdr_full = empty_bar + stages;
+  uint64_t* hdr_empty = hdr_full + kHdrSlots;
+  uint64_t* cbar = hdr_empty + kHdrSlots;
+  const int hdr_slot_bytes = kHdrBytes + H * D * 2;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  // ---- prefix over sequences of their work groups (every CTA builds its own)
+  {
+    const int per = (p.B + kThreads - 1) / kThreads;
+    const int b0 = min(p.B, tid * per), b1 = min(p.B, b0 + per);
+    int sum = 0;
+    for (int b = b0; b < b1; ++b) sum += groups_of(__ldg(p.seq_lens + b), p);
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    if (tid == 0) {
+      for (int s = 0; s < stages; ++s) {
+        mbar_init(&full_bar[s], 1);
+        mbar_init(&empty_bar[s], kConsumerWarps);
+      }
+      for (int s = 0; s < kHdrSlots; ++s) {
+        mbar_init(&hdr_full[s], 1);
+        mbar_init(&hdr_empty[s], kConsumerWarps);
+      }
+      mbar_init(cbar, kConsumerWarps);
+      fence_mbarrier_init();
+    }
+    __syncthreads();
+    int base = 0;
+    for (int w = 0; w < warp; ++w) base += warp_tot[w];
+    int run = base + incl - sum;
+    if (tid == 0) prefix[0] = 0;
+    for (int b = b0; b < b1; ++b) {
+      run += groups_of(__ldg(p.seq_lens + b), p);
+      prefix[b + 1] = run;
+    }
+    __syncthreads();
+  }
+  const int total_items = prefix[p.B] * p.Hkv;
+  pdl_launch_dependents();   // the combine kernel may be scheduled from now on
+
+  if (warp == kConsumerWarps) {
+    producer_loop<D>(&kmap, &vmap, p, smem, L, prefix, total_items, hdr_slot_bytes, full_bar,
+                     empty_bar, hdr_full, hdr_empty, lane);
     return;
   }
 
   // -------------------------------------------------------------- consumers
   Consumer<D, NT> cw;
-  cw.init(p, b, kvh, lane);
+  constexpr int OS = D + 4;                                // padded row: no bank conflicts
+  float* Osm = reinterpret_cast<float*>(smem + L.merge);   // [warp][H][OS]
+  float* MLsm = Osm + kConsumerWarps * H * OS;             // [warp][H][2]
+  const int n = lane >> 2, t = lane & 3;
   const int row0 = warp * kRowsPerWarp;
-  int s = 0;
-  for (; s < n_stages; ++s) {
-    const int slot = s % stages;
-    if (!mbar_wait_bounded(&full_bar[slot], (s / stages) & 1, kWaitLimitNs)) timed_out = true;
-    if (__any_sync(0xffffffffu, timed_out)) {
-      timed_out = true;
+  const int pps = p.pages_per_stage;
+  int hs = 0, rs = 0;
+  uint32_t cpar = 0;
+  bool alive = true;
+  for (;;) {
+    const int hslot = hs % kHdrSlots;
+    if (!__all_sync(0xffffffffu,
+                    mbar_wait_bounded(&hdr_full[hslot], (hs / kHdrSlots) & 1, kWaitLimitNs))) {
+      alive = false;
       break;
     }
-    const uint8_t* Kt = smem + slot * 2 * kTileBytes;
-    const uint8_t* Vt = Kt + kTileBytes;
-    const int tok0 = (pb + s * pps) * p.bt + row0;   // token of this warp's first row
-    if (tok0 + kRowsPerWarp > tok_lo && tok0 < tok_hi) {
-      if (tok0 >= tok_lo && tok0 + kRowsPerWarp <= tok_hi)
-        cw.template tile<true>(Kt, Vt, row0, tok0, tok_lo, tok_hi, lane);
-      else
-        cw.template tile<false>(Kt, Vt, row0, tok0, tok_lo, tok_hi, lane);
-    }
+    const uint8_t* hbase = smem + L.hdr + hslot * hdr_slot_bytes;
+    const ItemHeader hd = *reinterpret_cast<const ItemHeader*>(hbase);
+    if (hd.kind < 0) break;
+    cw.init(p, reinterpret_cast<const __nv_bfloat16*>(hbase + kHdrBytes), lane);
     __syncwarp();
-    if (lane == 0) mbar_arrive(&empty_bar[slot]);
+    if (lane == 0) mbar_arrive(&hdr_empty[hslot]);
+    ++hs;
+
+    for (int s = 0; s < hd.n_stages; ++s, ++rs) {
+      const int slot = rs % stages;
+      if (!__all_sync(0xffffffffu,
+                      mbar_wait_bounded(&full_bar[slot], (rs / stages) & 1, kWaitLimitNs))) {
+        alive = false;
+        break;
+      }
+      const uint8_t* Kt = smem + L.ring + slot * 2 * kTileBytes;
+      const uint8_t* Vt = Kt + kTileBytes;
+      const int tok0 = (hd.pb + s * pps) * p.bt + row0;   // token of this warp's first row
+      if (tok0 + kRowsPerWarp > hd.tok_lo && tok0 < hd.tok_hi) {
+        if (tok0 >= hd.tok_lo && tok0 + kRowsPerWarp <= hd.tok_hi)
+          cw.template tile<true>(Kt, Vt, row0, tok0, hd.tok_lo, hd.tok_hi, lane);
+        else
+          cw.template tile<false>(Kt, Vt, row0, tok0, hd.tok_lo, hd.tok_hi, lane);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_bar[slot]);
+    }
+    if (!alive) break;
+
+    // ---- merge the four warps of this item
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        float lsum = cw.l[nt][j];
+        lsum += __shfl_xor_sync(0xffffffffu, lsum, 4);
+        lsum += __shfl_xor_sync(0xffffffffu, lsum, 8);
+        lsum += __shfl_xor_sync(0xffffffffu, lsum, 16);
+        const int h = nt * 8 + 2 * t + j;
+        if (n == 0) {
+          MLsm[(warp * H + h) * 2 + 0] = cw.m[nt][j];
+          MLsm[(warp * H + h) * 2 + 1] = lsum;
+        }
+        // O^T column h: rows d = n*(D/8) + 2i + hh  (hh = 0 -> c0/c1, 1 -> c2/c3)
+        float* dst = Osm + ((size_t)warp * H + h) * OS + n * (D / 8);
+#pragma unroll
+        for (int i = 0; i < Consumer<D, NT>::MT; ++i) {
+          dst[2 * i + 0] = cw.o[i][nt][j];
+          dst[2 * i + 1] = cw.o[i][nt][j + 2];
+        }
+      }
+    }
+    if (!consumer_sync(cbar, cpar, lane)) {
+      alive = false;
+      break;
+    }
+    const bool single = hd.ns <= 1;
+    for (int idx = tid; idx < p.g * D; idx += kConsumerWarps * 32) {
+      const int h = idx / D, d = idx % D;
+      const int hq = hd.kvh * p.g + h;
+      const size_t row = (size_t)hd.b * p.Hq + hq;
+      if (hd.ns == 0) {  // empty sequence: out = 0, lse = sigma
+        p.out[row * D + d] = __float2bfloat16_rn(0.f);
+        if (d == 0 && p.lse) p.lse[row] = p.sinks ? p.sinks[hq] : -INFINITY;
+        continue;
+      }
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, MLsm[(w * H + h) * 2]);
+      float Lsum = 0.f, acc = 0.f;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) {
+        const float mw = MLsm[(w * H + h) * 2];
+        const float sc = (mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
+        Lsum += MLsm[(w * H + h) * 2 + 1] * sc;
+        acc += Osm[((size_t)w * H + h) * OS + d] * sc;
+      }
+      const float lse2 = M + __log2f(Lsum);   // log2-sum-exp of this split (no sink)
+      if (single) {
+        float Z = 1.f, Mx = lse2, wsplit = 1.f;
+        if (p.sinks) {
+          const float sg = p.sinks[hq] * kLog2e;
+          Mx = fmaxf(lse2, sg);
+          wsplit = fast_exp2(lse2 - Mx);
+          Z = wsplit + fast_exp2(sg - Mx);
+        }
+        p.out[row * D + d] = __float2bfloat16_rn(acc / Lsum * wsplit / Z * p.v_scale);
+        if (d == 0 && p.lse) p.lse[row] = (Mx + __log2f(Z)) * kLn2;
+      } else {
+        const size_t prow = row * p.max_splits + hd.split;
+        p.part_o[prow * D + d] = acc / Lsum;
+        if (d == 0) p.part_lse[prow] = lse2;
+      }
+    }
+    // the merge scratch is reused by the next item
+    if (!consumer_sync(cbar, cpar, lane)) {
+      alive = false;
+      break;
+    }
   }
-  if (timed_out) {
-    // Let every load that may already be issued land before the ring is reused
-    // (bounded), report, and still take part in the merge barriers below so
-    // the other warps are not left waiting; the results are flagged invalid.
-    for (int r = s; r < n_stages && r < s + stages; ++r)
+  if (!alive) {
+    // Let loads that may already be issued land before the CTA's shared memory
+    // is released (bounded), and report.
+    for (int r = rs; r < rs + stages; ++r)
       mbar_wait_bounded(&full_bar[r % stages], (r / stages) & 1, kDrainLimitNs);
-    if (lane == 0) atomicOr(p.status, 0x4u);
+    if (lane == 0) atomicOr(p.status, kErrTimeout);
+    return;
   }
-
-  // ------------------------------------------------- merge the four warps
-  constexpr int H = NT * 8;
-  float* Osm = reinterpret_cast<float*>(smem);                       // [warp][H][D]
-  float* MLsm = reinterpret_cast<float*>(smem + MergeLayout<D, NT>::kOBytes);  // [warp][H][2]
-  const int n = lane >> 2, t = lane & 3;
-  named_barrier_sync(1, kConsumerWarps * 32);   // all ring reads done before reuse
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      float lsum = cw.l[nt][j];
-      lsum += __shfl_xor_sync(0xffffffffu, lsum, 4);
-      lsum += __shfl_xor_sync(0xffffffffu, lsum, 8);
-      lsum += __shfl_xor_sync(0xffffffffu, lsum, 16);
-      const int h = nt * 8 + 2 * t + j;
-      if (n == 0) {
-        MLsm[(warp * H + h) * 2 + 0] = cw.m[nt][j];
-        MLsm[(warp * H + h) * 2 + 1] = lsum;
-      }
-      // O^T column h: rows d = n*(D/8) + 2i + hh  (hh = 0 -> c0/c1, 1 -> c2/c3)
-      float* dst = Osm + ((size_t)warp * H + h) * D + n * (D / 8);
-#pragma unroll
-      for (int i = 0; i < Consumer<D, NT>::MT; ++i) {
-        dst[2 * i + 0] = cw.o[i][nt][j];
-        dst[2 * i + 1] = cw.o[i][nt][j + 2];
-      }
-    }
-  }
-  named_barrier_sync(1, kConsumerWarps * 32);
-
-  const int tid = threadIdx.x;  // 0 .. 127
-  for (int idx = tid; idx < p.g * D; idx += kConsumerWarps * 32) {
-    const int h = idx / D, d = idx % D;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, MLsm[(w * H + h) * 2]);
-    float Lsum = 0.f, acc = 0.f;
-#pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) {
-      const float mw = MLsm[(w * H + h) * 2];
-      const float sc = (mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
-      Lsum += MLsm[(w * H + h) * 2 + 1] * sc;
-      acc += Osm[((size_t)w * H + h) * D + d] * sc;
-    }
-    const int hq = kvh * p.g + h;
-    const size_t row = (size_t)b * p.Hq + hq;
-    const float lse2 = M + __log2f(Lsum);      // log2-sum-exp of this split (no sink)
-    if (single) {
-      float Z = 1.f, Mx = lse2, wsplit = 1.f;
-      if (p.sinks) {
-        const float sg = p.sinks[hq] * kLog2e;
-        Mx = fmaxf(lse2, sg);
-        wsplit = fast_exp2(lse2 - Mx);
-        Z = wsplit + fast_exp2(sg - Mx);
-      }
-      p.out[row * D + d] = __float2bfloat16_rn(acc / Lsum * wsplit / Z * p.v_scale);
-      if (d == 0 && p.lse) p.lse[row] = (Mx + __log2f(Z)) * kLn2;
-    } else {
-      const size_t prow = row * p.max_splits + split;
-      p.part_o[prow * D + d] = acc / Lsum;
-      if (d == 0) p.part_lse[prow] = lse2;
+  // The last CTA to finish resets the work counter for the next call.
+  if (tid == 0) {
+    __threadfence();
+    if (atomicAdd(&p.sched[1], 1u) == gridDim.x - 1) {
+      atomicExch(&p.sched[0], 0u);
+      atomicExch(&p.sched[1], 0u);
     }
   }
 }
+
+// ----------------------------------------------------------------- combine --
 
 struct CombineParams {
   const int32_t* seq_lens;
@@ -556,32 +756,40 @@ struct CombineParams {
   float v_scale;
 };
 
-// One warp per (sequence, query head) whose sequence spans several splits:
-// out = v_scale * sum_s 2^(lse_s - M) o_s / (sum_s 2^(lse_s - M) + 2^(sigma - M)).
+constexpr int kCombineWarps = 4;
+
+// One CTA per (sequence, query head) row whose sequence spans several splits:
+//   out = v_scale sum_s 2^(lse_s - M) o_s / (sum_s 2^(lse_s - M) + 2^(sigma - M)),
+//   lse = (M + log2 Z) ln 2,  M = max(max_s lse_s, sigma)  (sigma in log2 units).
+// Warp w takes splits w, w + 4, ...; lanes cover the head dimension.
 template <int D>
-__global__ void __launch_bounds__(256) fpd_combine_kernel(const CombineParams p) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.x * 8 + warp;
-  if (row >= p.B * p.Hq) return;
+__global__ void __launch_bounds__(kCombineWarps * 32) fpd_combine_kernel(const CombineParams p) {
+  __shared__ float acc_sm[kCombineWarps][D];
+  __shared__ float z_sm[kCombineWarps];
+  pdl_wait_primary();
+  const int row = blockIdx.x;
   const int b = row / p.Hq, h = row % p.Hq;
   const SeqRange R = seq_range(p.seq_lens[b], p.bt, p.max_blocks, p.window_left, p.chunk_pages,
                                nullptr);
   const int ns = R.n_splits;
-  if (ns <= 1) return;
+  if (ns <= 1) return;   // written directly by the split kernel
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int PER = D / 32;
   const float* pl = p.part_lse + (size_t)row * p.max_splits;
-  float M = p.sinks ? p.sinks[h] * kLog2e : -INFINITY;
+  const float* po = p.part_o + (size_t)row * p.max_splits * D + lane * PER;
+  const float sink2 = p.sinks ? p.sinks[h] * kLog2e : -INFINITY;
+  float M = sink2;
   for (int s = lane; s < ns; s += 32) M = fmaxf(M, pl[s]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  constexpr int PER = D / 32;
   float acc[PER];
 #pragma unroll
   for (int i = 0; i < PER; ++i) acc[i] = 0.f;
-  float Z = p.sinks ? fast_exp2(p.sinks[h] * kLog2e - M) : 0.f;
-  const float* po = p.part_o + (size_t)row * p.max_splits * D + lane * PER;
-  for (int s = 0; s < ns; ++s) {
+  float z = 0.f;
+#pragma unroll 4
+  for (int s = warp; s < ns; s += kCombineWarps) {
     const float w = fast_exp2(pl[s] - M);
-    Z += w;
+    z += w;
     if constexpr (PER == 4) {
       const float4 v = *reinterpret_cast<const float4*>(po + (size_t)s * D);
       acc[0] += w * v.x;
@@ -594,11 +802,21 @@ __global__ void __launch_bounds__(256) fpd_combine_kernel(const CombineParams p)
       acc[1] += w * v.y;
     }
   }
-  const float inv = p.v_scale / Z;
-  __nv_bfloat16* dst = p.out + (size_t)row * D + lane * PER;
 #pragma unroll
-  for (int i = 0; i < PER; ++i) dst[i] = __float2bfloat16_rn(acc[i] * inv);
-  if (lane == 0 && p.lse) p.lse[row] = (M + __log2f(Z)) * kLn2;
+  for (int i = 0; i < PER; ++i) acc_sm[warp][lane * PER + i] = acc[i];
+  if (lane == 0) z_sm[warp] = z;
+  __syncthreads();
+  float Z = p.sinks ? fast_exp2(sink2 - M) : 0.f;
+#pragma unroll
+  for (int w = 0; w < kCombineWarps; ++w) Z += z_sm[w];
+  const float inv = p.v_scale / Z;
+  for (int d = threadIdx.x; d < D; d += kCombineWarps * 32) {
+    float a = 0.f;
+#pragma unroll
+    for (int w = 0; w < kCombineWarps; ++w) a += acc_sm[w][d];
+    p.out[(size_t)row * D + d] = __float2bfloat16_rn(a * inv);
+  }
+  if (threadIdx.x == 0 && p.lse) p.lse[row] = (M + __log2f(Z)) * kLn2;
 }
 
 }  // namespace fpd

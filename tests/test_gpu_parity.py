@@ -73,6 +73,24 @@ def test_forced_splits_agree(chunk):
     check(wl, chunk_pages=chunk)
 
 
+def test_workspace_reused_across_calls_and_counters_reset():
+    """The work counters live in the workspace and are reset by the kernel
+    itself: back-to-back calls on one workspace stay correct and leave those
+    words at zero."""
+    wl = W.make_custom(B=5, Hq=16, Hkv=4, D=128, block_tokens=32,
+                       seq_lens=[4000, 1, 2100, 640, 3333], sinks=True, seed=81)
+    dev = to_device(wl)
+    need = fpd.fp8_paged_decode_workspace_bytes_ex(5, 16, 4, 128, 32, wl.max_blocks, -1, 4)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    ref_out, ref_lse = oracle.decode_workload(wl)
+    for _ in range(3):
+        out, lse = run_cuda(wl, dev, chunk_pages=4, workspace=ws)
+        assert_parity(out, lse, ref_out, ref_lse, what="workspace reuse")
+    words = ws[:256].view(torch.int32).cpu().numpy()
+    assert (words[1:3] == 0).all(), "work counters not reset"
+    assert fpd.fp8_paged_decode_check_status(ws) == 0
+
+
 def test_page_permutation_bitwise():
     wl = W.make_custom(B=4, Hq=32, Hkv=8, D=128, block_tokens=16, seq_lens=[3000, 17, 555, 1024],
                        sinks=True, seed=51)
