@@ -177,12 +177,25 @@ struct Consumer {
   static constexpr int MT = D / 16;   // m-tiles of the PV MMA
   static constexpr int QW = D / 4;    // contiguous q elements per thread
 
+  uint32_t koff[D / 64];    // swizzled byte offsets of this thread's K reads (row n)
+  uint32_t voff[2];         // swizzled byte offsets of its V reads (rows 2t, 2t + 1)
   uint32_t qf[NT][KS][2];   // Q^T B fragments (f16x2), head = lane / 4 of n-tile
   float cs[NT][2];          // logit scale (log2) of this thread's C columns
   float m[NT][2];           // running max (log2 domain) of this thread's columns
   float thr[NT][2];         // raw-accumulator threshold that triggers a rescale
   float l[NT][2];           // partial row sums (this thread's tokens only)
   float o[MT][NT][4];       // O^T accumulators
+
+  // Shared-memory read offsets inside a stage tile; the same for every stage.
+  // Rows r and r + 8 share the swizzle phase (it depends on r mod 8), so the
+  // second row of each pair is the first plus 8 * D.
+  __device__ __forceinline__ void setup(int row0, int lane) {
+    const int n = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int c = 0; c < D / 64; ++c) koff[c] = swz<D>((row0 + n) * D + t * (D / 4) + 16 * c);
+    voff[0] = swz<D>((row0 + 2 * t) * D + n * (D / 8));
+    voff[1] = swz<D>((row0 + 2 * t + 1) * D + n * (D / 8));
+  }
 
   // qtile: the item's query rows, bf16 [g][D] in shared memory.
   __device__ __forceinline__ void init(const DecodeParams& p, const __nv_bfloat16* qtile,
@@ -253,11 +266,9 @@ struct Consumer {
     uint32_t kw[2][D / 16];
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
-      const int row = row0 + n + 8 * r;
 #pragma unroll
       for (int c = 0; c < D / 64; ++c) {
-        const uint4 v = *reinterpret_cast<const uint4*>(
-            Kt + swz<D>(row * D + t * (D / 4) + 16 * c));
+        const uint4 v = *reinterpret_cast<const uint4*>(Kt + koff[c] + r * 8 * D);
         kw[r][4 * c + 0] = v.x;
         kw[r][4 * c + 1] = v.y;
         kw[r][4 * c + 2] = v.z;
@@ -347,21 +358,20 @@ struct Consumer {
     // ---- V fragments: token rows 2t, 2t+1, 2t+8, 2t+9; head-dim chunk n
     constexpr int VB = D / 8;  // bytes of one row this thread needs
     uint32_t va[VB / 4], vb[VB / 4], vc[VB / 4], vd[VB / 4];
-    const int rA = row0 + 2 * t;
     if constexpr (D == 128) {
-      const uint4 A = *reinterpret_cast<const uint4*>(Vt + swz<D>((rA + 0) * D + n * VB));
-      const uint4 B = *reinterpret_cast<const uint4*>(Vt + swz<D>((rA + 1) * D + n * VB));
-      const uint4 C = *reinterpret_cast<const uint4*>(Vt + swz<D>((rA + 8) * D + n * VB));
-      const uint4 E = *reinterpret_cast<const uint4*>(Vt + swz<D>((rA + 9) * D + n * VB));
+      const uint4 A = *reinterpret_cast<const uint4*>(Vt + voff[0]);
+      const uint4 B = *reinterpret_cast<const uint4*>(Vt + voff[1]);
+      const uint4 C = *reinterpret_cast<const uint4*>(Vt + voff[0] + 8 * D);
+      const uint4 E = *reinterpret_cast<const uint4*>(Vt + voff[1] + 8 * D);
       va[0] = A.x; va[1] = A.y; va[2] = A.z; va[3] = A.w;
       vb[0] = B.x; vb[1] = B.y; vb[2] = B.z; vb[3] = B.w;
       vc[0] = C.x; vc[1] = C.y; vc[2] = C.z; vc[3] = C.w;
       vd[0] = E.x; vd[1] = E.y; vd[2] = E.z; vd[3] = E.w;
     } else {
-      const uint2 A = *reinterpret_cast<const uint2*>(Vt + swz<D>((rA + 0) * D + n * VB));
-      const uint2 B = *reinterpret_cast<const uint2*>(Vt + swz<D>((rA + 1) * D + n * VB));
-      const uint2 C = *reinterpret_cast<const uint2*>(Vt + swz<D>((rA + 8) * D + n * VB));
-      const uint2 E = *reinterpret_cast<const uint2*>(Vt + swz<D>((rA + 9) * D + n * VB));
+      const uint2 A = *reinterpret_cast<const uint2*>(Vt + voff[0]);
+      const uint2 B = *reinterpret_cast<const uint2*>(Vt + voff[1]);
+      const uint2 C = *reinterpret_cast<const uint2*>(Vt + voff[0] + 8 * D);
+      const uint2 E = *reinterpret_cast<const uint2*>(Vt + voff[1] + 8 * D);
       va[0] = A.x; va[1] = A.y;
       vb[0] = B.x; vb[1] = B.y;
       vc[0] = C.x; vc[1] = C.y;
@@ -422,14 +432,16 @@ __device__ __forceinline__ void producer_loop(const CUtensorMap* kmap, const CUt
     tma_prefetch_desc(kmap);
     tma_prefetch_desc(vmap);
   }
-  int hs = 0, rs = 0;
-  uint32_t item = 0;
-  if (lane == 0) item = atomicAdd(&p.sched[0], 1u);
-  item = __shfl_sync(0xffffffffu, item, 0);
+  int hs = 0;
+  int slot = 0, issued = 0;   // ring position and stages issued so far
+  uint32_t phase = 0;         // use count of the current slot, mod 2
+  // The first item of every CTA is its own index; later ones come from the
+  // shared counter (offset by the grid size).
+  uint32_t item = blockIdx.x;
   for (;;) {
     const bool done = item >= (uint32_t)total_items;
     uint32_t next = 0;
-    if (!done && lane == 0) next = atomicAdd(&p.sched[0], 1u);   // latency hidden below
+    if (!done && lane == 0) next = gridDim.x + atomicAdd(&p.sched[0], 1u);   // latency hidden below
     const int hslot = hs % kHdrSlots;
     if (hs >= kHdrSlots) {
       const bool ok =
@@ -487,10 +499,9 @@ __device__ __forceinline__ void producer_loop(const CUtensorMap* kmap, const CUt
     // ---- stream the item's pages; block-table entries 32 at a time
     const int32_t* tbl = p.block_table + (size_t)b * p.max_blocks;
     int batch_base = -1, my_entry = 0;
-    for (int s = 0; s < n_st; ++s, ++rs) {
-      const int slot = rs % stages;
-      if (rs >= stages) {
-        const bool ok = mbar_wait_bounded(&empty_bar[slot], ((rs / stages) - 1) & 1, kWaitLimitNs);
+    for (int s = 0; s < n_st; ++s) {
+      if (issued >= stages) {   // wait for the consumers to release the previous use
+        const bool ok = mbar_wait_bounded(&empty_bar[slot], phase ^ 1u, kWaitLimitNs);
         if (!__all_sync(0xffffffffu, ok)) {
           if (lane == 0) atomicOr(p.status, kErrTimeout);
           return;
@@ -524,6 +535,11 @@ __device__ __forceinline__ void producer_loop(const CUtensorMap* kmap, const CUt
             tma_load_3d(vdst + i * page_bytes, vmap, 0, kvh, rows[i], &full_bar[slot], policy);
           }
         }
+      }
+      ++issued;
+      if (++slot == stages) {
+        slot = 0;
+        phase ^= 1u;
       }
     }
     item = __shfl_sync(0xffffffffu, next, 0);
@@ -615,9 +631,12 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
   const int n = lane >> 2, t = lane & 3;
   const int row0 = warp * kRowsPerWarp;
   const int pps = p.pages_per_stage;
-  int hs = 0, rs = 0;
+  int hs = 0;
+  int slot = 0;             // ring position
+  uint32_t phase = 0;       // use count of the current slot, mod 2
   uint32_t cpar = 0;
   bool alive = true;
+  cw.setup(row0, lane);
   for (;;) {
     const int hslot = hs % kHdrSlots;
     if (!__all_sync(0xffffffffu,
@@ -633,10 +652,8 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
     if (lane == 0) mbar_arrive(&hdr_empty[hslot]);
     ++hs;
 
-    for (int s = 0; s < hd.n_stages; ++s, ++rs) {
-      const int slot = rs % stages;
-      if (!__all_sync(0xffffffffu,
-                      mbar_wait_bounded(&full_bar[slot], (rs / stages) & 1, kWaitLimitNs))) {
+    for (int s = 0; s < hd.n_stages; ++s) {
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full_bar[slot], phase, kWaitLimitNs))) {
         alive = false;
         break;
       }
@@ -651,6 +668,10 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty_bar[slot]);
+      if (++slot == stages) {
+        slot = 0;
+        phase ^= 1u;
+      }
     }
     if (!alive) break;
 
@@ -728,8 +749,13 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
   if (!alive) {
     // Let loads that may already be issued land before the CTA's shared memory
     // is released (bounded), and report.
-    for (int r = rs; r < rs + stages; ++r)
-      mbar_wait_bounded(&full_bar[r % stages], (r / stages) & 1, kDrainLimitNs);
+    for (int r = 0; r < stages; ++r) {
+      mbar_wait_bounded(&full_bar[slot], phase, kDrainLimitNs);
+      if (++slot == stages) {
+        slot = 0;
+        phase ^= 1u;
+      }
+    }
     if (lane == 0) atomicOr(p.status, kErrTimeout);
     return;
   }
