@@ -192,8 +192,9 @@ bool encode_cache_map(CUtensorMap* map, const void* base, int num_blocks, int bt
 // start while the split kernel drains and wait for it on the device.
 template <int D>
 cudaError_t launch_combine(const fpd::CombineParams& c, cudaStream_t st) {
+  const int rows_per_cta = fpd::kCombineWarps / c.wpr;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(c.B * c.Hq));
+  cfg.gridDim = dim3((unsigned)((c.B * c.Hq + rows_per_cta - 1) / rows_per_cta));
   cfg.blockDim = dim3(fpd::kCombineWarps * 32);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
@@ -389,6 +390,7 @@ static fpd_status attention_impl(const void* q, const void* k_cache, const void*
     c.window_left = window_left;
     c.chunk_pages = plan.chunk_pages;
     c.max_splits = plan.max_splits;
+    c.wpr = plan.max_splits <= 4 ? 1 : plan.max_splits <= 8 ? 2 : plan.max_splits <= 16 ? 4 : 8;
     c.v_scale = v_scale;
     e = D == 128 ? launch_combine<128>(c, s) : launch_combine<64>(c, s);
     if (e != cudaSuccess) return FPD_ERR_CUDA;

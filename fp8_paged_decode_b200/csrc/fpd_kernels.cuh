@@ -231,17 +231,19 @@ struct Consumer {
       // keeps bf16 -> f16 exact for any bf16 magnitude; undone in the logit scale.
       int e = 0;
       if (amax > 0.f && isfinite(amax)) frexpf(amax, &e);
-      const float fac = ldexpf(1.0f, max(-126, min(126, 15 - e)));
+      const int sh = max(-126, min(126, 15 - e));
+      const float fac = ldexpf(1.0f, sh);
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
         qf[nt][ks][0] = pack_f16x2(vals[4 * ks] * fac, vals[4 * ks + 1] * fac);
         qf[nt][ks][1] = pack_f16x2(vals[4 * ks + 2] * fac, vals[4 * ks + 3] * fac);
       }
-      // this thread's C columns are heads 2t and 2t+1 of the n-tile
-      const float f0 = __shfl_sync(0xffffffffu, fac, (2 * t) * 4);
-      const float f1 = __shfl_sync(0xffffffffu, fac, (2 * t + 1) * 4);
-      cs[nt][0] = p.qk_scale_log2 / f0;
-      cs[nt][1] = p.qk_scale_log2 / f1;
+      // this thread's C columns are heads 2t and 2t+1 of the n-tile; the
+      // prescale is a power of two, so undoing it is an exact multiply
+      const int sh0 = __shfl_sync(0xffffffffu, sh, (2 * t) * 4);
+      const int sh1 = __shfl_sync(0xffffffffu, sh, (2 * t + 1) * 4);
+      cs[nt][0] = p.qk_scale_log2 * ldexpf(1.0f, -sh0);
+      cs[nt][1] = p.qk_scale_log2 * ldexpf(1.0f, -sh1);
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         m[nt][j] = -INFINITY;
@@ -703,41 +705,53 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
       break;
     }
     const bool single = hd.ns <= 1;
-    for (int idx = tid; idx < p.g * D; idx += kConsumerWarps * 32) {
-      const int h = idx / D, d = idx % D;
-      const int hq = hd.kvh * p.g + h;
-      const size_t row = (size_t)hd.b * p.Hq + hq;
-      if (hd.ns == 0) {  // empty sequence: out = 0, lse = sigma
-        p.out[row * D + d] = __float2bfloat16_rn(0.f);
-        if (d == 0 && p.lse) p.lse[row] = p.sinks ? p.sinks[hq] : -INFINITY;
-        continue;
-      }
-      float M = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, MLsm[(w * H + h) * 2]);
-      float Lsum = 0.f, acc = 0.f;
-#pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) {
-        const float mw = MLsm[(w * H + h) * 2];
-        const float sc = (mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
-        Lsum += MLsm[(w * H + h) * 2 + 1] * sc;
-        acc += Osm[((size_t)w * H + h) * OS + d] * sc;
-      }
-      const float lse2 = M + __log2f(Lsum);   // log2-sum-exp of this split (no sink)
-      if (single) {
-        float Z = 1.f, Mx = lse2, wsplit = 1.f;
-        if (p.sinks) {
-          const float sg = p.sinks[hq] * kLog2e;
-          Mx = fmaxf(lse2, sg);
-          wsplit = fast_exp2(lse2 - Mx);
-          Z = wsplit + fast_exp2(sg - Mx);
+    {
+      // thread -> (d, first head); heads step by 128 / D.  The loop body is
+      // independent per head, so it is unrolled for overlap.
+      constexpr int HPI = kConsumerWarps * 32 / D;
+      const int d = tid % D;
+#pragma unroll 4
+      for (int h = tid / D; h < p.g; h += HPI) {
+        const int hq = hd.kvh * p.g + h;
+        const size_t row = (size_t)hd.b * p.Hq + hq;
+        if (hd.ns == 0) {  // empty sequence: out = 0, lse = sigma
+          p.out[row * D + d] = __float2bfloat16_rn(0.f);
+          if (d == 0 && p.lse) p.lse[row] = p.sinks ? p.sinks[hq] : -INFINITY;
+          continue;
         }
-        p.out[row * D + d] = __float2bfloat16_rn(acc / Lsum * wsplit / Z * p.v_scale);
-        if (d == 0 && p.lse) p.lse[row] = (Mx + __log2f(Z)) * kLn2;
-      } else {
-        const size_t prow = row * p.max_splits + hd.split;
-        p.part_o[prow * D + d] = acc / Lsum;
-        if (d == 0) p.part_lse[prow] = lse2;
+        float2 ml[kConsumerWarps];
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w)
+          ml[w] = *reinterpret_cast<const float2*>(MLsm + (w * H + h) * 2);
+        float M = ml[0].x;
+#pragma unroll
+        for (int w = 1; w < kConsumerWarps; ++w) M = fmaxf(M, ml[w].x);
+        float Lsum = 0.f, acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) {
+          const float sc = (ml[w].x == -INFINITY) ? 0.f : fast_exp2(ml[w].x - M);
+          Lsum = fmaf(ml[w].y, sc, Lsum);
+          acc = fmaf(Osm[((size_t)w * H + h) * OS + d], sc, acc);
+        }
+        const float lse2 = M + __log2f(Lsum);   // log2-sum-exp of this split (no sink)
+        if (single) {
+          float scale = p.v_scale;
+          float lse_out = lse2;
+          if (p.sinks) {
+            const float sg = p.sinks[hq] * kLog2e;
+            const float Mx = fmaxf(lse2, sg);
+            const float wsplit = fast_exp2(lse2 - Mx);
+            const float Z = wsplit + fast_exp2(sg - Mx);
+            scale *= __fdividef(wsplit, Z);
+            lse_out = Mx + __log2f(Z);
+          }
+          p.out[row * D + d] = __float2bfloat16_rn(acc * __fdividef(scale, Lsum));
+          if (d == 0 && p.lse) p.lse[row] = lse_out * kLn2;
+        } else {
+          const size_t prow = row * p.max_splits + hd.split;
+          p.part_o[prow * D + d] = __fdividef(acc, Lsum);
+          if (d == 0) p.part_lse[prow] = lse2;
+        }
       }
     }
     // the merge scratch is reused by the next item
@@ -779,70 +793,90 @@ struct CombineParams {
   __nv_bfloat16* out;
   float* lse;
   int B, Hq, bt, max_blocks, window_left, chunk_pages, max_splits;
+  int wpr;   // warps per row: 1, 2, 4 or 8
   float v_scale;
 };
 
-constexpr int kCombineWarps = 4;
+constexpr int kCombineWarps = 8;
 
-// One CTA per (sequence, query head) row whose sequence spans several splits:
+// Rows (sequence, query head) whose sequence spans several splits:
 //   out = v_scale sum_s 2^(lse_s - M) o_s / (sum_s 2^(lse_s - M) + 2^(sigma - M)),
 //   lse = (M + log2 Z) ln 2,  M = max(max_s lse_s, sigma)  (sigma in log2 units).
-// Warp w takes splits w, w + 4, ...; lanes cover the head dimension.
+// Each row gets `wpr` warps (more for long split lists); warp j of a row takes
+// splits j, j + wpr, ...; lanes cover the head dimension.
 template <int D>
 __global__ void __launch_bounds__(kCombineWarps * 32) fpd_combine_kernel(const CombineParams p) {
   __shared__ float acc_sm[kCombineWarps][D];
   __shared__ float z_sm[kCombineWarps];
   pdl_wait_primary();
-  const int row = blockIdx.x;
-  const int b = row / p.Hq, h = row % p.Hq;
-  const SeqRange R = seq_range(p.seq_lens[b], p.bt, p.max_blocks, p.window_left, p.chunk_pages,
-                               nullptr);
-  const int ns = R.n_splits;
-  if (ns <= 1) return;   // written directly by the split kernel
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wpr = p.wpr;
+  const int row = blockIdx.x * (kCombineWarps / wpr) + warp / wpr;
+  const int j = warp % wpr;
   constexpr int PER = D / 32;
-  const float* pl = p.part_lse + (size_t)row * p.max_splits;
-  const float* po = p.part_o + (size_t)row * p.max_splits * D + lane * PER;
-  const float sink2 = p.sinks ? p.sinks[h] * kLog2e : -INFINITY;
-  float M = sink2;
-  for (int s = lane; s < ns; s += 32) M = fmaxf(M, pl[s]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  int ns = 0;
+  if (row < p.B * p.Hq)
+    ns = seq_range(p.seq_lens[row / p.Hq], p.bt, p.max_blocks, p.window_left, p.chunk_pages,
+                   nullptr).n_splits;
+  const bool active = ns > 1;   // rows with one split were written by the split kernel
+  float M = -INFINITY, z = 0.f, sink2 = -INFINITY;
   float acc[PER];
 #pragma unroll
   for (int i = 0; i < PER; ++i) acc[i] = 0.f;
-  float z = 0.f;
+  if (active) {
+    const int h = row % p.Hq;
+    const float* pl = p.part_lse + (size_t)row * p.max_splits;
+    const float* po = p.part_o + (size_t)row * p.max_splits * D + lane * PER;
+    sink2 = p.sinks ? p.sinks[h] * kLog2e : -INFINITY;
+    M = sink2;
+    for (int s = lane; s < ns; s += 32) M = fmaxf(M, pl[s]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
 #pragma unroll 4
-  for (int s = warp; s < ns; s += kCombineWarps) {
-    const float w = fast_exp2(pl[s] - M);
-    z += w;
-    if constexpr (PER == 4) {
-      const float4 v = *reinterpret_cast<const float4*>(po + (size_t)s * D);
-      acc[0] += w * v.x;
-      acc[1] += w * v.y;
-      acc[2] += w * v.z;
-      acc[3] += w * v.w;
-    } else {
-      const float2 v = *reinterpret_cast<const float2*>(po + (size_t)s * D);
-      acc[0] += w * v.x;
-      acc[1] += w * v.y;
+    for (int s = j; s < ns; s += wpr) {
+      const float w = fast_exp2(pl[s] - M);
+      z += w;
+      if constexpr (PER == 4) {
+        const float4 v = *reinterpret_cast<const float4*>(po + (size_t)s * D);
+        acc[0] += w * v.x;
+        acc[1] += w * v.y;
+        acc[2] += w * v.z;
+        acc[3] += w * v.w;
+      } else {
+        const float2 v = *reinterpret_cast<const float2*>(po + (size_t)s * D);
+        acc[0] += w * v.x;
+        acc[1] += w * v.y;
+      }
     }
+  }
+  if (wpr == 1) {
+    if (active) {
+      const float Z = z + (p.sinks ? fast_exp2(sink2 - M) : 0.f);
+      const float inv = p.v_scale / Z;
+      __nv_bfloat16* dst = p.out + (size_t)row * D + lane * PER;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) dst[i] = __float2bfloat16_rn(acc[i] * inv);
+      if (lane == 0 && p.lse) p.lse[row] = (M + __log2f(Z)) * kLn2;
+    }
+    return;
   }
 #pragma unroll
   for (int i = 0; i < PER; ++i) acc_sm[warp][lane * PER + i] = acc[i];
   if (lane == 0) z_sm[warp] = z;
   __syncthreads();
-  float Z = p.sinks ? fast_exp2(sink2 - M) : 0.f;
+  if (active && j == 0) {   // the row's first warp finishes it
+    float Z = p.sinks ? fast_exp2(sink2 - M) : 0.f;
+    for (int w = warp; w < warp + wpr; ++w) Z += z_sm[w];
+    const float inv = p.v_scale / Z;
 #pragma unroll
-  for (int w = 0; w < kCombineWarps; ++w) Z += z_sm[w];
-  const float inv = p.v_scale / Z;
-  for (int d = threadIdx.x; d < D; d += kCombineWarps * 32) {
-    float a = 0.f;
-#pragma unroll
-    for (int w = 0; w < kCombineWarps; ++w) a += acc_sm[w][d];
-    p.out[(size_t)row * D + d] = __float2bfloat16_rn(a * inv);
+    for (int i = 0; i < PER; ++i) {
+      const int d = lane * PER + i;
+      float a = 0.f;
+      for (int w = warp; w < warp + wpr; ++w) a += acc_sm[w][d];
+      p.out[(size_t)row * D + d] = __float2bfloat16_rn(a * inv);
+    }
+    if (lane == 0 && p.lse) p.lse[row] = (M + __log2f(Z)) * kLn2;
   }
-  if (threadIdx.x == 0 && p.lse) p.lse[row] = (M + __log2f(Z)) * kLn2;
 }
 
 }  // namespace fpd
