@@ -517,26 +517,19 @@ __device__ __forceinline__ void producer_loop(const CUtensorMap* kmap, const CUt
         const int idx = pb + batch_base + lane;
         my_entry = (idx < pe) ? __ldg(tbl + idx) : 0;
       }
-      int rows[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int e = __shfl_sync(0xffffffffu, my_entry, (rel + i) & 31);
-        const bool ok = (e >= 0 && e < p.num_blocks);
-        if (!ok && i < np && lane == 0) atomicOr(p.status, kErrBlockTable);
+      // One lane per (page, K or V) box; the boxes are issued side by side.
+      const int e = __shfl_sync(0xffffffffu, my_entry, (rel + (lane >> 1)) & 31);
+      const bool mine = lane < 2 * np;
+      const bool ok = (e >= 0 && e < p.num_blocks);
+      if (mine && !ok && (lane & 1) == 0) atomicOr(p.status, kErrBlockTable);
+      if (lane == 0) mbar_arrive_expect_tx(&full_bar[slot], 2u * page_bytes * (uint32_t)np);
+      __syncwarp();
+      if (mine) {
         // an invalid page is read from past the end of the pool: TMA zero-fills it
-        rows[i] = ok ? e * p.bt : p.num_blocks * p.bt;
-      }
-      if (lane == 0) {
-        uint8_t* kdst = smem + L.ring + slot * 2 * kTileBytes;
-        uint8_t* vdst = kdst + kTileBytes;
-        mbar_arrive_expect_tx(&full_bar[slot], 2u * page_bytes * (uint32_t)np);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          if (i < np) {
-            tma_load_3d(kdst + i * page_bytes, kmap, 0, kvh, rows[i], &full_bar[slot], policy);
-            tma_load_3d(vdst + i * page_bytes, vmap, 0, kvh, rows[i], &full_bar[slot], policy);
-          }
-        }
+        const int row = ok ? e * p.bt : p.num_blocks * p.bt;
+        uint8_t* dst = smem + L.ring + slot * 2 * kTileBytes + (lane & 1) * kTileBytes +
+                       (lane >> 1) * page_bytes;
+        tma_load_3d(dst, (lane & 1) ? vmap : kmap, 0, kvh, row, &full_bar[slot], policy);
       }
       ++issued;
       if (++slot == stages) {
