@@ -182,8 +182,12 @@ bool encode_cache_map(CUtensorMap* map, const void* base, int num_blocks, int bt
   cuuint32_t estr[3] = {1u, 1u, 1u};
   const CUtensorMapSwizzle swz =
       D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  // No L2 promotion: each box row is one 128-byte (or 64-byte) line of one KV
+  // head, and widening it fetches the neighbouring head's line, which is
+  // often evicted before its own reader arrives (measured: 18% extra DRAM
+  // reads on the windowed, GQA-8 workload with 256-byte promotion).
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
