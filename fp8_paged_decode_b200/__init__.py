@@ -75,7 +75,8 @@ class FpdError(RuntimeError):
 
 class fpd_plan(ctypes.Structure):
     _fields_ = [("chunk_pages", ctypes.c_int), ("max_splits", ctypes.c_int),
-                ("pages_per_stage", ctypes.c_int), ("stages", ctypes.c_int),
+                ("heads_per_stage", ctypes.c_int), ("stage_tokens", ctypes.c_int),
+                ("stages", ctypes.c_int), ("header_slots", ctypes.c_int),
                 ("ctas", ctypes.c_int), ("smem_bytes", ctypes.c_int),
                 ("workspace_bytes", ctypes.c_size_t)]
 

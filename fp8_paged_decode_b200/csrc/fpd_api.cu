@@ -18,8 +18,13 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 constexpr size_t kHeaderBytes = 256;    // status word, work counter, finished-CTA counter
-constexpr int kTargetWaves = 8;         // work items ~ this many per resident CTA slot
-constexpr int kMinChunkTokens = 256;    // shortest KV range worth its own work item
+// Split heuristic, per stage shape (measured on the five synthetic workloads):
+// about this many work items per resident CTA slot, and no item below this
+// many (token, KV head) rows.  Four-head items carry a larger fixed cost (query
+// set-up of four heads, partial results of four heads), so they get fewer,
+// larger items.
+constexpr int kTargetWaves1 = 8, kMinChunkRows1 = 256;    // one KV head per stage
+constexpr int kTargetWaves4 = 5, kMinChunkRows4 = 1024;   // four KV heads per stage
 constexpr int kOccCacheSize = 32;
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -39,6 +44,10 @@ fpd_status validate_shape(int B, int Hq, int Hkv, int D, int bt, int max_blocks)
 
 int n_tiles(int g) { return g > 8 ? 2 : 1; }
 
+// KV heads per stage and work item: 4 whenever the KV heads split into groups
+// of 4 (one TMA box then covers 16 tokens of 4 heads), else 1.
+int heads_per_stage(int Hkv) { return Hkv % 4 == 0 ? 4 : 1; }
+
 // Depth of the shared-memory stage ring (build-time tunable).
 #ifndef FPD_STAGES_D128_NT1
 #define FPD_STAGES_D128_NT1 3
@@ -49,14 +58,29 @@ int n_tiles(int g) { return g > 8 ? 2 : 1; }
 #ifndef FPD_STAGES_D64
 #define FPD_STAGES_D64 6
 #endif
-int ring_stages(int D, int NT) {
+#ifndef FPD_STAGES_HB4_D128
+#define FPD_STAGES_HB4_D128 4
+#endif
+#ifndef FPD_STAGES_HB4_D64
+#define FPD_STAGES_HB4_D64 5
+#endif
+int ring_stages(int D, int NT, int HB) {
+  if (HB == 4) return D == 128 ? FPD_STAGES_HB4_D128 : FPD_STAGES_HB4_D64;
   if (D == 128) return NT == 2 ? FPD_STAGES_D128_NT2 : FPD_STAGES_D128_NT1;
   return FPD_STAGES_D64;
 }
 
-int smem_bytes_for(int D, int g, int B) {
+// Header ring depth: two slots while an item's query rows are small, one
+// otherwise, so that the stage ring keeps its shared memory.
+#ifndef FPD_HDR2_MAX_QBYTES
+#define FPD_HDR2_MAX_QBYTES 4096
+#endif
+int header_slots(int D, int g, int HB) { return HB * g * D * 2 <= FPD_HDR2_MAX_QBYTES ? 2 : 1; }
+
+int smem_bytes_for(int D, int g, int HB, int B) {
   const int NT = n_tiles(g);
-  return fpd::smem_layout(D, NT, ring_stages(D, NT), B).total;
+  return fpd::smem_layout(D, NT, HB, ring_stages(D, NT, HB), header_slots(D, g, HB), g, B)
+      .total;
 }
 
 // Workspace carve-up: [header 256 B][partial O][partial lse]
@@ -79,7 +103,7 @@ WsLayout ws_layout(int B, int Hq, int Hkv, int D, int max_splits) {
 
 // ---- per-device facts, queried once
 struct OccEntry {
-  int D, NT, smem, occ;
+  int D, NT, HB, smem, occ;
 };
 struct DeviceInfo {
   bool ready = false;
@@ -91,12 +115,17 @@ struct DeviceInfo {
 std::mutex g_mu;
 DeviceInfo g_dev[kMaxDevices];
 
-const void* split_kernel_for(int D, int NT) {
+template <int HB>
+const void* split_kernel_hb(int D, int NT) {
   if (D == 128)
-    return NT == 2 ? reinterpret_cast<const void*>(&fpd::fpd_split_kernel<128, 2>)
-                   : reinterpret_cast<const void*>(&fpd::fpd_split_kernel<128, 1>);
-  return NT == 2 ? reinterpret_cast<const void*>(&fpd::fpd_split_kernel<64, 2>)
-                 : reinterpret_cast<const void*>(&fpd::fpd_split_kernel<64, 1>);
+    return NT == 2 ? reinterpret_cast<const void*>(&fpd::fpd_split_kernel<128, 2, HB>)
+                   : reinterpret_cast<const void*>(&fpd::fpd_split_kernel<128, 1, HB>);
+  return NT == 2 ? reinterpret_cast<const void*>(&fpd::fpd_split_kernel<64, 2, HB>)
+                 : reinterpret_cast<const void*>(&fpd::fpd_split_kernel<64, 1, HB>);
+}
+
+const void* split_kernel_for(int D, int NT, int HB) {
+  return HB == 4 ? split_kernel_hb<4>(D, NT) : split_kernel_hb<1>(D, NT);
 }
 
 bool current_device(int* dev) {
@@ -109,7 +138,7 @@ bool current_device(int* dev) {
 
 // SM count of the current device and the number of split-kernel CTAs that fit
 // on one SM with `smem` bytes of dynamic shared memory (0 if none).
-bool device_occupancy(int D, int NT, int smem, int* num_sms, int* ctas_per_sm) {
+bool device_occupancy(int D, int NT, int HB, int smem, int* num_sms, int* ctas_per_sm) {
   int dev = 0;
   if (!current_device(&dev)) return false;
   std::lock_guard<std::mutex> lk(g_mu);
@@ -126,13 +155,13 @@ bool device_occupancy(int D, int NT, int smem, int* num_sms, int* ctas_per_sm) {
   *num_sms = di.num_sms;
   for (int i = 0; i < di.n_occ; ++i) {
     const OccEntry& e = di.occ[i];
-    if (e.D == D && e.NT == NT && e.smem == smem) {
+    if (e.D == D && e.NT == NT && e.HB == HB && e.smem == smem) {
       *ctas_per_sm = e.occ;
       return true;
     }
   }
   int occ = 0;
-  const void* fn = split_kernel_for(D, NT);
+  const void* fn = split_kernel_for(D, NT, HB);
   cudaFuncAttributes fa;
   if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) {
     cudaGetLastError();
@@ -148,7 +177,7 @@ bool device_occupancy(int D, int NT, int smem, int* num_sms, int* ctas_per_sm) {
       return false;
     }
   }
-  if (di.n_occ < kOccCacheSize) di.occ[di.n_occ++] = OccEntry{D, NT, smem, occ};
+  if (di.n_occ < kOccCacheSize) di.occ[di.n_occ++] = OccEntry{D, NT, HB, smem, occ};
   *ctas_per_sm = occ;
   return true;
 }
@@ -171,14 +200,26 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder() {
   return g_encode;
 }
 
-// View a [num_blocks, bt, Hkv, D] byte cache as the 3-D tensor
-// (d, kv head, token row) with box (D, 1, bt): one box = one page of one head.
-bool encode_cache_map(CUtensorMap* map, const void* base, int num_blocks, int bt, int Hkv, int D) {
+// View a [num_blocks, bt, Hkv, D] byte cache as a 3-D tensor.
+//   HB = 1: (d, kv head, token row), box (D, 1, bt): one page of one head.
+//   HB = 4: (d, token row, kv head), box (D, 16, 4): 16 tokens of 4 heads,
+//           landing head-major in shared memory (4 tiles of 16 rows).
+bool encode_cache_map(CUtensorMap* map, const void* base, int num_blocks, int bt, int Hkv, int D,
+                      int HB) {
   auto enc = encoder();
   if (!enc) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)num_blocks * bt};
-  cuuint64_t strides[2] = {(cuuint64_t)D, (cuuint64_t)Hkv * D};
-  cuuint32_t box[3] = {(cuuint32_t)D, 1u, (cuuint32_t)bt};
+  const cuuint64_t rows = (cuuint64_t)num_blocks * bt;
+  cuuint64_t dims[3], strides[2];
+  cuuint32_t box[3];
+  if (HB == 1) {
+    dims[0] = D, dims[1] = Hkv, dims[2] = rows;
+    strides[0] = D, strides[1] = (cuuint64_t)Hkv * D;
+    box[0] = D, box[1] = 1u, box[2] = bt;
+  } else {
+    dims[0] = D, dims[1] = rows, dims[2] = Hkv;
+    strides[0] = (cuuint64_t)Hkv * D, strides[1] = D;
+    box[0] = D, box[1] = fpd::kBoxTokens, box[2] = HB;
+  }
   cuuint32_t estr[3] = {1u, 1u, 1u};
   const CUtensorMapSwizzle swz =
       D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
@@ -196,10 +237,10 @@ bool encode_cache_map(CUtensorMap* map, const void* base, int num_blocks, int bt
 // start while the split kernel drains and wait for it on the device.
 template <int D>
 cudaError_t launch_combine(const fpd::CombineParams& c, cudaStream_t st) {
-  const int rows_per_cta = fpd::kCombineWarps / c.wpr;
+  const int rows_per_cta = c.rows_per_cta;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)((c.B * c.Hq + rows_per_cta - 1) / rows_per_cta));
-  cfg.blockDim = dim3(fpd::kCombineWarps * 32);
+  cfg.blockDim = dim3(c.wpr * rows_per_cta * 32);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -210,14 +251,87 @@ cudaError_t launch_combine(const fpd::CombineParams& c, cudaStream_t st) {
   return cudaLaunchKernelEx(&cfg, fpd::fpd_combine_kernel<D>, c);
 }
 
-template <int D, int NT>
+template <int D, int NT, int HB>
 cudaError_t launch_split(const CUtensorMap& km, const CUtensorMap& vm, const fpd::DecodeParams& p,
                          int ctas, int smem, cudaStream_t st) {
-  fpd::fpd_split_kernel<D, NT><<<ctas, fpd::kThreads, smem, st>>>(km, vm, p);
+  fpd::fpd_split_kernel<D, NT, HB><<<ctas, fpd::kThreads, smem, st>>>(km, vm, p);
   return cudaGetLastError();
 }
 
+template <int HB>
+cudaError_t launch_split_hb(int D, int NT, const CUtensorMap& km, const CUtensorMap& vm,
+                            const fpd::DecodeParams& p, int ctas, int smem, cudaStream_t st) {
+  if (D == 128)
+    return NT == 2 ? launch_split<128, 2, HB>(km, vm, p, ctas, smem, st)
+                   : launch_split<128, 1, HB>(km, vm, p, ctas, smem, st);
+  return NT == 2 ? launch_split<64, 2, HB>(km, vm, p, ctas, smem, st)
+                 : launch_split<64, 1, HB>(km, vm, p, ctas, smem, st);
+}
+
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// The split plan for a given stage shape (HB KV heads per stage).
+void plan_shape(int B, int Hq, int Hkv, int D, int bt, int max_blocks, int window_left,
+                int64_t slots, int chunk_pages_override, int HB, fpd_plan* plan) {
+  const int g = Hq / Hkv;
+  const int NT = n_tiles(g);
+  // with one KV head per stage a stage is 64 tokens of whole pages, and a
+  // split must be whole stages; four-head stages are 16 tokens of one page
+  const int pps = HB == 1 ? fpd::kTileTokens / bt : 1;
+  int pages_max = max_blocks;
+  if (window_left >= 0) {
+    const int64_t w = (int64_t)window_left / bt + 2;
+    if (w < pages_max) pages_max = (int)w;
+  }
+  const int64_t units = (int64_t)(B > 0 ? B : 1) * (Hkv / HB);
+  int chunk;
+  if (chunk_pages_override > 0) {
+    chunk = chunk_pages_override;
+  } else {
+    const int waves = HB == 1 ? kTargetWaves1 : kTargetWaves4;
+    const int min_rows = HB == 1 ? kMinChunkRows1 : kMinChunkRows4;
+    int64_t splits = (waves * slots + units - 1) / units;
+    if (splits < 1) splits = 1;
+    chunk = (int)((pages_max + splits - 1) / splits);
+    const int min_tokens = min_rows / HB;
+    const int min_chunk = (min_tokens + bt - 1) / bt;
+    if (chunk < min_chunk) chunk = min_chunk;
+  }
+  chunk = (chunk + pps - 1) / pps * pps;
+  const int max_splits = (pages_max + chunk - 1) / chunk;
+  const int64_t items_max = units * max_splits;
+  plan->chunk_pages = chunk;
+  plan->max_splits = max_splits;
+  plan->heads_per_stage = HB;
+  plan->stage_tokens = fpd::kTileTokens / HB;
+  plan->stages = ring_stages(D, NT, HB);
+  plan->header_slots = header_slots(D, g, HB);
+  plan->ctas = (int)(items_max < slots ? items_max : slots);
+  plan->smem_bytes = smem_bytes_for(D, g, HB, B);
+  plan->workspace_bytes = ws_layout(B, Hq, Hkv, D, max_splits).total;
+}
+
+// Validates and plans.  force_hb = 0 picks the stage shape: four KV heads per
+// stage when Hkv allows it and the four-head work items fill every CTA slot
+// at least once; otherwise (short windows over few sequences) one head per
+// stage, whose 4x more numerous items keep the machine busy.
+fpd_status plan_for(int B, int Hq, int Hkv, int D, int bt, int max_blocks, int window_left,
+                    int num_sms, int ctas_per_sm, int chunk_pages_override, int force_hb,
+                    fpd_plan* plan) {
+  if (!plan) return FPD_ERR_INVALID_ARG;
+  fpd_status st = validate_shape(B, Hq, Hkv, D, bt, max_blocks);
+  if (st != FPD_OK) return st;
+  if (num_sms <= 0 || ctas_per_sm <= 0 || chunk_pages_override < 0) return FPD_ERR_INVALID_ARG;
+  if (force_hb != 0 && force_hb != 1 && force_hb != 4) return FPD_ERR_INVALID_ARG;
+  if (force_hb == 4 && heads_per_stage(Hkv) != 4) return FPD_ERR_INVALID_ARG;
+  const int64_t slots = (int64_t)num_sms * ctas_per_sm;
+  int HB = force_hb ? force_hb : heads_per_stage(Hkv);
+  plan_shape(B, Hq, Hkv, D, bt, max_blocks, window_left, slots, chunk_pages_override, HB, plan);
+  if (force_hb == 0 && HB == 4 && chunk_pages_override == 0 &&
+      (int64_t)(B > 0 ? B : 1) * (Hkv / 4) * plan->max_splits < slots)
+    plan_shape(B, Hq, Hkv, D, bt, max_blocks, window_left, slots, 0, 1, plan);
+  return FPD_OK;
+}
 
 }  // namespace
 
@@ -239,41 +353,8 @@ const char* fp8_paged_decode_version(void) { return "0.2.0 sm_100a"; }
 fpd_status fp8_paged_decode_make_plan(int B, int Hq, int Hkv, int D, int bt, int max_blocks,
                                       int window_left, int num_sms, int ctas_per_sm,
                                       int chunk_pages_override, fpd_plan* plan) {
-  if (!plan) return FPD_ERR_INVALID_ARG;
-  fpd_status st = validate_shape(B, Hq, Hkv, D, bt, max_blocks);
-  if (st != FPD_OK) return st;
-  if (num_sms <= 0 || ctas_per_sm <= 0 || chunk_pages_override < 0) return FPD_ERR_INVALID_ARG;
-  const int g = Hq / Hkv;
-  const int NT = n_tiles(g);
-  const int pps = fpd::kTileTokens / bt;
-  int pages_max = max_blocks;
-  if (window_left >= 0) {
-    const int64_t w = (int64_t)window_left / bt + 2;
-    if (w < pages_max) pages_max = (int)w;
-  }
-  const int64_t units = (int64_t)(B > 0 ? B : 1) * Hkv;
-  const int64_t slots = (int64_t)num_sms * ctas_per_sm;
-  int chunk;
-  if (chunk_pages_override > 0) {
-    chunk = chunk_pages_override;
-  } else {
-    int64_t splits = (kTargetWaves * slots + units - 1) / units;
-    if (splits < 1) splits = 1;
-    chunk = (int)((pages_max + splits - 1) / splits);
-    const int min_chunk = (kMinChunkTokens + bt - 1) / bt;
-    if (chunk < min_chunk) chunk = min_chunk;
-  }
-  chunk = (chunk + pps - 1) / pps * pps;
-  const int max_splits = (pages_max + chunk - 1) / chunk;
-  const int64_t items_max = units * max_splits;
-  plan->chunk_pages = chunk;
-  plan->max_splits = max_splits;
-  plan->pages_per_stage = pps;
-  plan->stages = ring_stages(D, NT);
-  plan->ctas = (int)(items_max < slots ? items_max : slots);
-  plan->smem_bytes = smem_bytes_for(D, g, B);
-  plan->workspace_bytes = ws_layout(B, Hq, Hkv, D, max_splits).total;
-  return FPD_OK;
+  return plan_for(B, Hq, Hkv, D, bt, max_blocks, window_left, num_sms, ctas_per_sm,
+                  chunk_pages_override, 0, plan);
 }
 
 fpd_status fp8_paged_decode_plan(int B, int Hq, int Hkv, int D, int bt, int max_blocks,
@@ -282,11 +363,19 @@ fpd_status fp8_paged_decode_plan(int B, int Hq, int Hkv, int D, int bt, int max_
   fpd_status st = validate_shape(B, Hq, Hkv, D, bt, max_blocks);
   if (st != FPD_OK) return st;
   const int g = Hq / Hkv;
-  int sms = 0, occ = 0;
-  if (!device_occupancy(D, n_tiles(g), smem_bytes_for(D, g, B), &sms, &occ)) return FPD_ERR_CUDA;
-  if (occ <= 0) return FPD_ERR_UNSUPPORTED;  // the batch's shared-memory table does not fit
-  return fp8_paged_decode_make_plan(B, Hq, Hkv, D, bt, max_blocks, window_left, sms, occ,
-                                    chunk_pages_override, plan);
+  int HB = heads_per_stage(Hkv), force_hb = 0;
+  for (;;) {
+    int sms = 0, occ = 0;
+    if (!device_occupancy(D, n_tiles(g), HB, smem_bytes_for(D, g, HB, B), &sms, &occ))
+      return FPD_ERR_CUDA;
+    if (occ <= 0) return FPD_ERR_UNSUPPORTED;  // the batch's shared-memory table does not fit
+    st = plan_for(B, Hq, Hkv, D, bt, max_blocks, window_left, sms, occ, chunk_pages_override,
+                  force_hb, plan);
+    // the planner fell back to one head per stage: plan again with that
+    // kernel's own occupancy
+    if (st != FPD_OK || plan->heads_per_stage == HB) return st;
+    HB = force_hb = plan->heads_per_stage;
+  }
 }
 
 size_t fp8_paged_decode_workspace_bytes_ex(int B, int Hq, int Hkv, int D, int bt, int max_blocks,
@@ -335,8 +424,8 @@ static fpd_status attention_impl(const void* q, const void* k_cache, const void*
   if (!workspace || workspace_bytes < plan.workspace_bytes) return FPD_ERR_WORKSPACE_TOO_SMALL;
 
   CUtensorMap km, vm;
-  if (!encode_cache_map(&km, k_cache, num_blocks, bt, Hkv, D) ||
-      !encode_cache_map(&vm, v_cache, num_blocks, bt, Hkv, D))
+  if (!encode_cache_map(&km, k_cache, num_blocks, bt, Hkv, D, plan.heads_per_stage) ||
+      !encode_cache_map(&vm, v_cache, num_blocks, bt, Hkv, D, plan.heads_per_stage))
     return FPD_ERR_CUDA;
 
   const WsLayout wl = ws_layout(B, Hq, Hkv, D, plan.max_splits);
@@ -362,8 +451,8 @@ static fpd_status attention_impl(const void* q, const void* k_cache, const void*
   p.window_left = window_left;
   p.chunk_pages = plan.chunk_pages;
   p.max_splits = plan.max_splits;
-  p.pages_per_stage = plan.pages_per_stage;
   p.stages = plan.stages;
+  p.hdr_slots = plan.header_slots;
   p.qk_scale_log2 = qk * fpd::kLog2e;
   p.v_scale = v_scale;
 
@@ -371,12 +460,9 @@ static fpd_status attention_impl(const void* q, const void* k_cache, const void*
   if (ev0 && cudaEventRecord(static_cast<cudaEvent_t>(ev0), s) != cudaSuccess) return FPD_ERR_CUDA;
   cudaError_t e;
   const int NT = n_tiles(g);
-  if (D == 128)
-    e = NT == 2 ? launch_split<128, 2>(km, vm, p, plan.ctas, plan.smem_bytes, s)
-                : launch_split<128, 1>(km, vm, p, plan.ctas, plan.smem_bytes, s);
-  else
-    e = NT == 2 ? launch_split<64, 2>(km, vm, p, plan.ctas, plan.smem_bytes, s)
-                : launch_split<64, 1>(km, vm, p, plan.ctas, plan.smem_bytes, s);
+  e = plan.heads_per_stage == 4
+          ? launch_split_hb<4>(D, NT, km, vm, p, plan.ctas, plan.smem_bytes, s)
+          : launch_split_hb<1>(D, NT, km, vm, p, plan.ctas, plan.smem_bytes, s);
   if (e != cudaSuccess) return FPD_ERR_CUDA;
   if (ev1 && cudaEventRecord(static_cast<cudaEvent_t>(ev1), s) != cudaSuccess) return FPD_ERR_CUDA;
   if (plan.max_splits > 1) {
@@ -394,7 +480,11 @@ static fpd_status attention_impl(const void* q, const void* k_cache, const void*
     c.window_left = window_left;
     c.chunk_pages = plan.chunk_pages;
     c.max_splits = plan.max_splits;
-    c.wpr = plan.max_splits <= 4 ? 1 : plan.max_splits <= 8 ? 2 : plan.max_splits <= 16 ? 4 : 8;
+    // enough warps per row that none merges more than one batch of partials
+    // (up to 32 warps), and 8 warps per CTA at least
+    c.wpr = 1;
+    while (c.wpr < 32 && c.wpr * fpd::kCombineBatch < plan.max_splits) c.wpr *= 2;
+    c.rows_per_cta = c.wpr >= 8 ? 1 : 8 / c.wpr;
     c.v_scale = v_scale;
     e = D == 128 ? launch_combine<128>(c, s) : launch_combine<64>(c, s);
     if (e != cudaSuccess) return FPD_ERR_CUDA;

@@ -1,15 +1,24 @@
 // fpd_kernels.cuh -- the sm_100a kernel of the paged E4M3 decode attention.
 //
 // One persistent kernel.  Each CTA (one or more per SM) pulls work items from
-// a global counter; an item is (sequence b, KV head, KV split) and covers up
-// to `chunk_pages` pages of that sequence's attended range.  Warp 4 is the
-// producer: for every item it publishes a small header plus the item's query
-// rows (bulk copy) in a 2-slot header ring, then streams the item's pages with
-// TMA tiled loads (one box per page of one KV head, K and V, 128-byte swizzle)
-// into a ring of shared-memory stages.  The stage ring runs straight across
-// item boundaries, so HBM reads never wait for an item to start.
+// a global counter; an item is (sequence b, group of HB KV heads, KV split)
+// and covers up to `chunk_pages` pages of that sequence's attended range.
+// Warp 4 is the producer: for every item it publishes a small header plus the
+// item's query rows (bulk copy) in a header ring, then streams the item's KV
+// with TMA tiled loads into a ring of shared-memory stages.  The stage ring
+// runs straight across item boundaries, so HBM reads never wait for an item to
+// start.  A stage holds 64 token rows of K and of V, in one of two shapes:
 //
-// Warps 0..3 are consumers: each owns 16 token rows of every 64-token stage:
+//   HB = 4 (the KV head count is a multiple of 4): 16 tokens x 4 KV heads, one
+//     TMA box per tensor (D bytes x 16 tokens x 4 heads, 128-byte swizzle).
+//     Consumer warp w owns KV head 4j + w of the item for all of its tokens,
+//     so an item needs no merge between warps: each warp finishes its own
+//     query heads straight from registers.
+//   HB = 1: 64 tokens of one KV head, one TMA box per page and tensor; the
+//     four consumer warps split the rows 16 apiece and merge in shared memory
+//     at the end of the item.
+//
+// Per consumer warp and stage, 16 token rows of one KV head:
 //   S^T = K Q^T      mma.sync m16n8k16, tokens on M, the query heads of the KV
 //                    head on N (heads on the MMA N side, as in the "SwapsAb"
 //                    orientation of FlashInfer PR #5591, Summary);
@@ -18,17 +27,15 @@
 //                    lazy-rescale rule of the same PR's Summary);
 //   O^T += V^T P^T   mma.sync m16n8k16, head dim on M, heads on N;
 // with E4M3 -> f16 conversion in registers (exact) and the per-tensor scales
-// folded into the logit scale and the output.  At the end of an item the four
-// warps merge in shared memory.  An item that covers its whole sequence writes
-// bf16 out and lse (sink folded in).  Otherwise it writes an fp32 partial
-// (O / l and log2-sum-exp), and the combine kernel, launched as a programmatic
-// dependent of this one (its CTAs start during this kernel's tail and wait for
-// its completion; the FP8 paged-MLA route on the FlashInfer PR #5591 page,
-// section "Unsupported", launches its split-KV merge the same way), merges the
-// partials of every sequence
-// that spans several splits and folds in the sink.  The last CTA to leave
-// resets the work counter, so the workspace needs zeroing only once after
-// allocation.
+// folded into the logit scale and the output.  An item that covers its whole
+// sequence writes bf16 out and lse (sink folded in).  Otherwise it writes an
+// fp32 partial (O / l and log2-sum-exp), and the combine kernel, launched as a
+// programmatic dependent of this one (its CTAs start during this kernel's
+// tail and wait for its completion; the FP8 paged-MLA route on the FlashInfer
+// PR #5591 page, section "Unsupported", launches its split-KV merge the same
+// way), merges the partials of every sequence that spans several splits and
+// folds in the sink.  The last CTA to leave resets the work counter, so the
+// workspace needs zeroing only once after allocation.
 //
 // Fragment layouts (PTX ISA, mma.m16n8k16 with .f16):
 //   A: a0 (row g, cols 2t..2t+1), a1 (row g+8, same), a2 (row g, cols 2t+8..),
@@ -41,6 +48,8 @@
 //   QK k-step ks, slot 2t+u  -> d = t*(D/4) + 4*ks + u      (u in 0..1)
 //               slot 2t+8+u  -> d = t*(D/4) + 4*ks + 2 + u
 //   PV m-tile i, row g+8h    -> d = g*(D/8) + 2*i + h        (h in 0..1)
+// so the O^T rows a thread holds for one query head are the D/8 contiguous
+// elements starting at g*D/8.
 //
 // Every wait (mbarrier phase, consumer-group sync) is bounded in time; on
 // expiry the kernel sets FPD_DEVERR_TIMEOUT in the status word and the warp
@@ -59,10 +68,11 @@ namespace fpd {
 
 constexpr int kConsumerWarps = 4;
 constexpr int kRowsPerWarp = 16;
-constexpr int kTileTokens = kConsumerWarps * kRowsPerWarp;  // tokens per stage
+constexpr int kTileTokens = kConsumerWarps * kRowsPerWarp;  // token rows per stage and tensor
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
-constexpr int kHdrSlots = 2;
+constexpr int kMaxHdrSlots = 2;
 constexpr int kHdrBytes = 64;                 // ItemHeader, padded
+constexpr int kBoxTokens = 16;                // tokens per TMA box with HB = 4
 constexpr float kLazyThreshold = 8.0f;        // log2 units
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -85,40 +95,48 @@ struct DecodeParams {
   uint32_t* status;     // workspace word 0: sticky FPD_DEVERR_* bits
   uint32_t* sched;      // workspace words 1, 2: next work item, CTAs finished
   int B, Hq, Hkv, g, bt, max_blocks, num_blocks, window_left;
-  int chunk_pages, max_splits, pages_per_stage, stages;
+  int chunk_pages, max_splits, stages, hdr_slots;
   float qk_scale_log2;  // sm_scale * k_scale * log2(e)
   float v_scale;
 };
 
+// Bytes of one header slot: the header, then the item's query rows (HB KV
+// heads x g query heads x D, bf16).
+__host__ __device__ constexpr int hdr_slot_bytes(int D, int HB, int g) {
+  return kHdrBytes + ((HB * g * D * 2 + 15) / 16) * 16;
+}
+
 // Shared-memory carve-up (byte offsets from a 1024-byte aligned base); used by
-// the host to size the launch and by the kernel to find its buffers.
+// the host to size the launch and by the kernel to find its buffers.  Only
+// HB = 1 needs the merge buffer.
 struct SmemLayout {
   int ring, merge, hdr, prefix, bars, total;
 };
 
 __host__ __device__ constexpr int align_to(int x, int a) { return (x + a - 1) / a * a; }
 
-__host__ __device__ inline SmemLayout smem_layout(int D, int NT, int stages, int B) {
+__host__ __device__ inline SmemLayout smem_layout(int D, int NT, int HB, int stages, int hdr_slots,
+                                                  int g, int B) {
   SmemLayout L{};
   const int H = NT * 8;
   L.ring = 0;
   L.merge = stages * 2 * kTileTokens * D;
-  const int merge_bytes = kConsumerWarps * H * (D + 4) * 4 + kConsumerWarps * H * 2 * 4;
+  const int merge_bytes =
+      HB == 1 ? kConsumerWarps * H * (D + 4) * 4 + kConsumerWarps * H * 2 * 4 : 0;
   L.hdr = align_to(L.merge + merge_bytes, 128);
-  const int hdr_slot = kHdrBytes + H * D * 2;
-  L.prefix = align_to(L.hdr + kHdrSlots * hdr_slot, 16);
+  L.prefix = align_to(L.hdr + hdr_slots * hdr_slot_bytes(D, HB, g), 16);
   L.bars = align_to(L.prefix + 4 * (B + 1), 16);
-  L.total = align_to(L.bars + (2 * stages + 2 * kHdrSlots + 1) * 8, 16) +
+  L.total = align_to(L.bars + (2 * stages + 2 * kMaxHdrSlots + 1) * 8, 16) +
             1024;  // + slack to align the base to 1024
   return L;
 }
 
 struct ItemHeader {
   int kind;      // 1: work item, -1: no more work
-  int b, kvh, split;
+  int b, kvh0, split;
   int ns;        // splits of this sequence (0: empty sequence)
   int n_stages;  // pipeline stages this item consumes
-  int pb;        // first page of the item
+  int t0;        // token of the first row of the item's first stage
   int tok_lo, tok_hi;
   int pad[7];
 };
@@ -414,20 +432,90 @@ struct Consumer {
         mma_16816(o[2 * w + 1][nt], a0, a1, a2, a3, pb0[nt], pb1[nt]);
     }
   }
+  // HB = 4: this warp alone covered KV head `kvh` of the item, so its query
+  // heads are finished straight from registers.  Thread (n, t) holds, for
+  // query head nt*8 + 2t + j, the D/8 output elements starting at n*D/8.
+  __device__ __forceinline__ void finish_own(const DecodeParams& p, int b, int kvh, int split,
+                                             int ns, int lane) {
+    constexpr int E = D / 8;   // output elements per thread and query head
+    const int n = lane >> 2, t = lane & 3;
+    float lsum[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        float v = l[nt][j];
+        v += __shfl_xor_sync(0xffffffffu, v, 4);
+        v += __shfl_xor_sync(0xffffffffu, v, 8);
+        v += __shfl_xor_sync(0xffffffffu, v, 16);
+        lsum[nt][j] = v;
+      }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int hl = nt * 8 + 2 * t + j;
+        if (hl >= p.g) continue;
+        const int hq = kvh * p.g + hl;
+        const size_t row = (size_t)b * p.Hq + hq;
+        if (ns == 0) {  // empty sequence: out = 0, lse = sigma
+          uint4* dst = reinterpret_cast<uint4*>(p.out + row * D + n * E);
+#pragma unroll
+          for (int c = 0; c < E / 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+          if (n == 0 && p.lse) p.lse[row] = p.sinks ? p.sinks[hq] : -INFINITY;
+          continue;
+        }
+        const float lse2 = m[nt][j] + __log2f(lsum[nt][j]);   // log2-sum-exp, no sink
+        if (ns == 1) {
+          float scale = p.v_scale;
+          float lse_out = lse2;
+          if (p.sinks) {
+            const float sg = p.sinks[hq] * kLog2e;
+            const float Mx = fmaxf(lse2, sg);
+            const float wsplit = fast_exp2(lse2 - Mx);
+            const float Z = wsplit + fast_exp2(sg - Mx);
+            scale *= __fdividef(wsplit, Z);
+            lse_out = Mx + __log2f(Z);
+          }
+          const float inv = __fdividef(scale, lsum[nt][j]);
+          uint32_t w[MT];
+#pragma unroll
+          for (int i = 0; i < MT; ++i) w[i] = pack_bf16x2(o[i][nt][j] * inv, o[i][nt][j + 2] * inv);
+          uint4* dst = reinterpret_cast<uint4*>(p.out + row * D + n * E);
+#pragma unroll
+          for (int c = 0; c < E / 8; ++c)
+            dst[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+          if (n == 0 && p.lse) p.lse[row] = lse_out * kLn2;
+        } else {
+          const size_t prow = row * p.max_splits + split;
+          const float inv = __fdividef(1.0f, lsum[nt][j]);
+          float4* dst = reinterpret_cast<float4*>(p.part_o + prow * D + n * E);
+#pragma unroll
+          for (int c = 0; c < E / 4; ++c)
+            dst[c] = make_float4(o[2 * c][nt][j] * inv, o[2 * c][nt][j + 2] * inv,
+                                 o[2 * c + 1][nt][j] * inv, o[2 * c + 1][nt][j + 2] * inv);
+          if (n == 0) p.part_lse[prow] = lse2;
+        }
+      }
+    }
+  }
 };
 
 // ---------------------------------------------------------------- producer --
 
-template <int D>
+template <int D, int HB>
 __device__ __forceinline__ void producer_loop(const CUtensorMap* kmap, const CUtensorMap* vmap,
                                               const DecodeParams& p, uint8_t* smem,
                                               const SmemLayout& L, const int* prefix,
-                                              int total_items, int hdr_slot_bytes,
+                                              int total_items, int hslot_bytes,
                                               uint64_t* full_bar, uint64_t* empty_bar,
                                               uint64_t* hdr_full, uint64_t* hdr_empty, int lane) {
   constexpr int kTileBytes = kTileTokens * D;
+  constexpr int kStageTokens = kTileTokens / HB;   // tokens of one KV head per stage
   const int stages = p.stages;
-  const int pps = p.pages_per_stage;
+  const int n_hslots = p.hdr_slots;
+  const int groups = p.Hkv / HB;                   // KV head groups
+  const int pps = HB == 1 ? kStageTokens / p.bt : 1;   // pages per stage (HB = 1)
   const uint32_t page_bytes = (uint32_t)(p.bt * D);
   const uint64_t policy = l2_policy_evict_first();
   if (lane == 0) {
@@ -435,6 +523,8 @@ __device__ __forceinline__ void producer_loop(const CUtensorMap* kmap, const CUt
     tma_prefetch_desc(vmap);
   }
   int hs = 0;
+  int hslot = 0;
+  uint32_t hphase = 0;        // use count of the current header slot, mod 2
   int slot = 0, issued = 0;   // ring position and stages issued so far
   uint32_t phase = 0;         // use count of the current slot, mod 2
   // The first item of every CTA is its own index; later ones come from the
@@ -444,16 +534,15 @@ __device__ __forceinline__ void producer_loop(const CUtensorMap* kmap, const CUt
     const bool done = item >= (uint32_t)total_items;
     uint32_t next = 0;
     if (!done && lane == 0) next = gridDim.x + atomicAdd(&p.sched[0], 1u);   // latency hidden below
-    const int hslot = hs % kHdrSlots;
-    if (hs >= kHdrSlots) {
-      const bool ok =
-          mbar_wait_bounded(&hdr_empty[hslot], ((hs / kHdrSlots) - 1) & 1, kWaitLimitNs);
+    if (hs >= n_hslots) {
+      const bool ok = mbar_wait_bounded(&hdr_empty[hslot], hphase ^ 1u, kWaitLimitNs);
       if (!__all_sync(0xffffffffu, ok)) {
         if (lane == 0) atomicOr(p.status, kErrTimeout);
         return;
       }
     }
-    ItemHeader* hdr = reinterpret_cast<ItemHeader*>(smem + L.hdr + hslot * hdr_slot_bytes);
+    uint8_t* hbase = smem + L.hdr + hslot * hslot_bytes;
+    ItemHeader* hdr = reinterpret_cast<ItemHeader*>(hbase);
     if (done) {
       if (lane == 0) {
         hdr->kind = -1;
@@ -461,9 +550,9 @@ __device__ __forceinline__ void producer_loop(const CUtensorMap* kmap, const CUt
       }
       return;
     }
-    // item -> (group, kv head) -> (sequence, split) by binary search of the prefix
-    const int group = (int)item / p.Hkv;
-    const int kvh = (int)item % p.Hkv;
+    // item -> (group, kv head group) -> (sequence, split) by binary search
+    const int group = (int)item / groups;
+    const int kvh0 = ((int)item % groups) * HB;
     int lo = 0, hi = p.B;   // largest b with prefix[b] <= group
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
@@ -473,32 +562,42 @@ __device__ __forceinline__ void producer_loop(const CUtensorMap* kmap, const CUt
     const int split = group - prefix[b];
     const SeqRange R = seq_range(__ldg(p.seq_lens + b), p.bt, p.max_blocks, p.window_left,
                                  p.chunk_pages, lane == 0 ? p.status : nullptr);
-    int pb = 0, pe = 0, tok_lo = 0, tok_hi = 0, n_st = 0;
+    int pb = 0, pe = 0, tok_lo = 0, tok_hi = 0, t0 = 0, n_st = 0;
     if (R.n_splits > 0) {
       pb = R.first_page + split * p.chunk_pages;
       pe = min(pb + p.chunk_pages, R.end_page);
       tok_lo = max(R.start, pb * p.bt);
       tok_hi = min(R.L, pe * p.bt);
-      n_st = (pe - pb + pps - 1) / pps;
+      if (HB == 1) {   // whole pages, pps per stage
+        t0 = pb * p.bt;
+        n_st = (pe - pb + pps - 1) / pps;
+      } else {         // the 16-token blocks that touch [tok_lo, tok_hi)
+        t0 = tok_lo & ~(kBoxTokens - 1);
+        n_st = (tok_hi - t0 + kBoxTokens - 1) / kBoxTokens;
+      }
     }
     if (lane == 0) {
       hdr->kind = 1;
       hdr->b = b;
-      hdr->kvh = kvh;
+      hdr->kvh0 = kvh0;
       hdr->split = split;
       hdr->ns = R.n_splits;
       hdr->n_stages = n_st;
-      hdr->pb = pb;
+      hdr->t0 = t0;
       hdr->tok_lo = tok_lo;
       hdr->tok_hi = tok_hi;
-      const uint32_t qbytes = (uint32_t)(p.g * D * 2);
+      const uint32_t qbytes = (uint32_t)(HB * p.g * D * 2);
       mbar_arrive_expect_tx(&hdr_full[hslot], qbytes);
-      bulk_load(smem + L.hdr + hslot * hdr_slot_bytes + kHdrBytes,
-                p.q + ((size_t)b * p.Hq + (size_t)kvh * p.g) * D, qbytes, &hdr_full[hslot]);
+      bulk_load(hbase + kHdrBytes, p.q + ((size_t)b * p.Hq + (size_t)kvh0 * p.g) * D, qbytes,
+                &hdr_full[hslot]);
     }
     ++hs;
+    if (++hslot == n_hslots) {
+      hslot = 0;
+      hphase ^= 1u;
+    }
 
-    // ---- stream the item's pages; block-table entries 32 at a time
+    // ---- stream the item's KV; block-table entries 32 at a time
     const int32_t* tbl = p.block_table + (size_t)b * p.max_blocks;
     int batch_base = -1, my_entry = 0;
     for (int s = 0; s < n_st; ++s) {
@@ -509,27 +608,51 @@ __device__ __forceinline__ void producer_loop(const CUtensorMap* kmap, const CUt
           return;
         }
       }
-      const int pg0 = pb + s * pps;
-      const int np = min(pps, pe - pg0);
-      const int rel = pg0 - pb;
-      if ((rel & ~31) != batch_base) {
-        batch_base = rel & ~31;
-        const int idx = pb + batch_base + lane;
-        my_entry = (idx < pe) ? __ldg(tbl + idx) : 0;
-      }
-      // One lane per (page, K or V) box; the boxes are issued side by side.
-      const int e = __shfl_sync(0xffffffffu, my_entry, (rel + (lane >> 1)) & 31);
-      const bool mine = lane < 2 * np;
-      const bool ok = (e >= 0 && e < p.num_blocks);
-      if (mine && !ok && (lane & 1) == 0) atomicOr(p.status, kErrBlockTable);
-      if (lane == 0) mbar_arrive_expect_tx(&full_bar[slot], 2u * page_bytes * (uint32_t)np);
-      __syncwarp();
-      if (mine) {
-        // an invalid page is read from past the end of the pool: TMA zero-fills it
-        const int row = ok ? e * p.bt : p.num_blocks * p.bt;
-        uint8_t* dst = smem + L.ring + slot * 2 * kTileBytes + (lane & 1) * kTileBytes +
-                       (lane >> 1) * page_bytes;
-        tma_load_3d(dst, (lane & 1) ? vmap : kmap, 0, kvh, row, &full_bar[slot], policy);
+      uint8_t* stage = smem + L.ring + slot * 2 * kTileBytes;
+      if constexpr (HB == 1) {
+        const int pg0 = pb + s * pps;
+        const int np = min(pps, pe - pg0);
+        const int rel = pg0 - pb;
+        if ((rel & ~31) != batch_base) {
+          batch_base = rel & ~31;
+          const int idx = pb + batch_base + lane;
+          my_entry = (idx < pe) ? __ldg(tbl + idx) : 0;
+        }
+        // One lane per (page, K or V) box; the boxes are issued side by side.
+        const int e = __shfl_sync(0xffffffffu, my_entry, (rel + (lane >> 1)) & 31);
+        const bool mine = lane < 2 * np;
+        const bool ok = (e >= 0 && e < p.num_blocks);
+        if (mine && !ok && (lane & 1) == 0) atomicOr(p.status, kErrBlockTable);
+        if (lane == 0) mbar_arrive_expect_tx(&full_bar[slot], 2u * page_bytes * (uint32_t)np);
+        __syncwarp();
+        if (mine) {
+          // an invalid page is read from past the end of the pool: TMA zero-fills it
+          const int row = ok ? e * p.bt : p.num_blocks * p.bt;
+          uint8_t* dst = stage + (lane & 1) * kTileBytes + (lane >> 1) * page_bytes;
+          tma_load_3d(dst, (lane & 1) ? vmap : kmap, 0, kvh0, row, &full_bar[slot], policy);
+        }
+      } else {
+        // 16 tokens of HB heads: one box per tensor, lane 0 K and lane 1 V
+        const int tok = t0 + s * kBoxTokens;
+        const int rel = tok / p.bt - pb;
+        if ((rel & ~31) != batch_base) {
+          batch_base = rel & ~31;
+          const int idx = pb + batch_base + lane;
+          my_entry = (idx < pe) ? __ldg(tbl + idx) : 0;
+        }
+        const int e = __shfl_sync(0xffffffffu, my_entry, rel & 31);
+        const bool ok = (e >= 0 && e < p.num_blocks);
+        if (lane == 0) {
+          if (!ok) atomicOr(p.status, kErrBlockTable);
+          mbar_arrive_expect_tx(&full_bar[slot], 2u * kTileBytes);
+        }
+        __syncwarp();
+        if (lane < 2) {
+          // an invalid page is read from past the end of the pool: TMA zero-fills it
+          const int row = (ok ? e * p.bt : p.num_blocks * p.bt) + (tok - (rel + pb) * p.bt);
+          tma_load_3d(stage + lane * kTileBytes, lane ? vmap : kmap, 0, row, kvh0,
+                      &full_bar[slot], policy);
+        }
       }
       ++issued;
       if (++slot == stages) {
@@ -552,7 +675,7 @@ struct MinBlocks {
   static constexpr int value = (D == 128) ? (NT == 1 ? FPD_MINB_D128_NT1 : 2) : (NT == 1 ? 4 : 3);
 };
 
-template <int D, int NT>
+template <int D, int NT, int HB>
 __global__ void __launch_bounds__(kThreads, MinBlocks<D, NT>::value)
 fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                  const DecodeParams p) {
@@ -561,16 +684,18 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   constexpr int kTileBytes = kTileTokens * D;
+  constexpr int kStageTokens = kTileTokens / HB;
   constexpr int H = NT * 8;
   const int stages = p.stages;
-  const SmemLayout L = smem_layout(D, NT, stages, p.B);
+  const int n_hslots = p.hdr_slots;
+  const SmemLayout L = smem_layout(D, NT, HB, stages, n_hslots, p.g, p.B);
+  const int hslot_bytes = hdr_slot_bytes(D, HB, p.g);
   int* prefix = reinterpret_cast<int*>(smem + L.prefix);
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + L.bars);
   uint64_t* empty_bar = full_bar + stages;
   uint64_t* hdr_full = empty_bar + stages;
-  uint64_t* hdr_empty = hdr_full + kHdrSlots;
-  uint64_t* cbar = hdr_empty + kHdrSlots;
-  const int hdr_slot_bytes = kHdrBytes + H * D * 2;
+  uint64_t* hdr_empty = hdr_full + kMaxHdrSlots;
+  uint64_t* cbar = hdr_empty + kMaxHdrSlots;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   // ---- prefix over sequences of their work groups (every CTA builds its own)
@@ -591,7 +716,7 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
         mbar_init(&full_bar[s], 1);
         mbar_init(&empty_bar[s], kConsumerWarps);
       }
-      for (int s = 0; s < kHdrSlots; ++s) {
+      for (int s = 0; s < kMaxHdrSlots; ++s) {
         mbar_init(&hdr_full[s], 1);
         mbar_init(&hdr_empty[s], kConsumerWarps);
       }
@@ -609,52 +734,57 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
     }
     __syncthreads();
   }
-  const int total_items = prefix[p.B] * p.Hkv;
+  const int total_items = prefix[p.B] * (p.Hkv / HB);
   pdl_launch_dependents();   // the combine kernel may be scheduled from now on
 
   if (warp == kConsumerWarps) {
-    producer_loop<D>(&kmap, &vmap, p, smem, L, prefix, total_items, hdr_slot_bytes, full_bar,
-                     empty_bar, hdr_full, hdr_empty, lane);
+    producer_loop<D, HB>(&kmap, &vmap, p, smem, L, prefix, total_items, hslot_bytes, full_bar,
+                         empty_bar, hdr_full, hdr_empty, lane);
     return;
   }
 
   // -------------------------------------------------------------- consumers
   Consumer<D, NT> cw;
-  constexpr int OS = D + 4;                                // padded row: no bank conflicts
-  float* Osm = reinterpret_cast<float*>(smem + L.merge);   // [warp][H][OS]
-  float* MLsm = Osm + kConsumerWarps * H * OS;             // [warp][H][2]
   const int n = lane >> 2, t = lane & 3;
-  const int row0 = warp * kRowsPerWarp;
-  const int pps = p.pages_per_stage;
-  int hs = 0;
+  // HB = 4: this warp's KV head occupies its own 16 rows of each stage.
+  // HB = 1: this warp takes rows [16 * warp, 16 * warp + 16) of the stage.
+  const int row0 = HB == 1 ? warp * kRowsPerWarp : 0;
+  const int tile_off = HB == 1 ? 0 : warp * kRowsPerWarp * D;
+  const int tok_off = HB == 1 ? row0 : 0;
+  int hslot = 0;
+  uint32_t hphase = 0;
   int slot = 0;             // ring position
   uint32_t phase = 0;       // use count of the current slot, mod 2
   uint32_t cpar = 0;
   bool alive = true;
   cw.setup(row0, lane);
   for (;;) {
-    const int hslot = hs % kHdrSlots;
-    if (!__all_sync(0xffffffffu,
-                    mbar_wait_bounded(&hdr_full[hslot], (hs / kHdrSlots) & 1, kWaitLimitNs))) {
+    if (!__all_sync(0xffffffffu, mbar_wait_bounded(&hdr_full[hslot], hphase, kWaitLimitNs))) {
       alive = false;
       break;
     }
-    const uint8_t* hbase = smem + L.hdr + hslot * hdr_slot_bytes;
+    const uint8_t* hbase = smem + L.hdr + hslot * hslot_bytes;
     const ItemHeader hd = *reinterpret_cast<const ItemHeader*>(hbase);
     if (hd.kind < 0) break;
-    cw.init(p, reinterpret_cast<const __nv_bfloat16*>(hbase + kHdrBytes), lane);
+    cw.init(p,
+            reinterpret_cast<const __nv_bfloat16*>(hbase + kHdrBytes) +
+                (HB == 1 ? 0 : warp * p.g * D),
+            lane);
     __syncwarp();
     if (lane == 0) mbar_arrive(&hdr_empty[hslot]);
-    ++hs;
+    if (++hslot == n_hslots) {
+      hslot = 0;
+      hphase ^= 1u;
+    }
 
     for (int s = 0; s < hd.n_stages; ++s) {
       if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full_bar[slot], phase, kWaitLimitNs))) {
         alive = false;
         break;
       }
-      const uint8_t* Kt = smem + L.ring + slot * 2 * kTileBytes;
+      const uint8_t* Kt = smem + L.ring + slot * 2 * kTileBytes + tile_off;
       const uint8_t* Vt = Kt + kTileBytes;
-      const int tok0 = (hd.pb + s * pps) * p.bt + row0;   // token of this warp's first row
+      const int tok0 = hd.t0 + s * kStageTokens + tok_off;   // token of this warp's first row
       if (tok0 + kRowsPerWarp > hd.tok_lo && tok0 < hd.tok_hi) {
         if (tok0 >= hd.tok_lo && tok0 + kRowsPerWarp <= hd.tok_hi)
           cw.template tile<true>(Kt, Vt, row0, tok0, hd.tok_lo, hd.tok_hi, lane);
@@ -670,7 +800,15 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
     }
     if (!alive) break;
 
-    // ---- merge the four warps of this item
+    if constexpr (HB != 1) {
+      cw.finish_own(p, hd.b, hd.kvh0 + warp, hd.split, hd.ns, lane);
+      continue;
+    }
+
+    // ---- HB = 1: merge the four warps of this item
+    constexpr int OS = D + 4;                                // padded row: no bank conflicts
+    float* Osm = reinterpret_cast<float*>(smem + L.merge);   // [warp][H][OS]
+    float* MLsm = Osm + kConsumerWarps * H * OS;             // [warp][H][2]
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
@@ -705,7 +843,7 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
       const int d = tid % D;
 #pragma unroll 4
       for (int h = tid / D; h < p.g; h += HPI) {
-        const int hq = hd.kvh * p.g + h;
+        const int hq = hd.kvh0 * p.g + h;
         const size_t row = (size_t)hd.b * p.Hq + hq;
         if (hd.ns == 0) {  // empty sequence: out = 0, lse = sigma
           p.out[row * D + d] = __float2bfloat16_rn(0.f);
@@ -786,25 +924,28 @@ struct CombineParams {
   __nv_bfloat16* out;
   float* lse;
   int B, Hq, bt, max_blocks, window_left, chunk_pages, max_splits;
-  int wpr;   // warps per row: 1, 2, 4 or 8
+  int wpr;            // warps per row: 1, 2, 4, 8, 16 or 32
+  int rows_per_cta;   // rows per CTA (wpr * rows_per_cta <= 32)
   float v_scale;
 };
 
-constexpr int kCombineWarps = 8;
+constexpr int kCombineMaxThreads = 1024;
+constexpr int kCombineBatch = 8;   // partials a warp loads before it reduces them
 
 // Rows (sequence, query head) whose sequence spans several splits:
 //   out = v_scale sum_s 2^(lse_s - M) o_s / (sum_s 2^(lse_s - M) + 2^(sigma - M)),
 //   lse = (M + log2 Z) ln 2,  M = max(max_s lse_s, sigma)  (sigma in log2 units).
-// Each row gets `wpr` warps (more for long split lists); warp j of a row takes
-// splits j, j + wpr, ...; lanes cover the head dimension.
+// Each row gets `wpr` warps; warp j of a row takes splits j, j + wpr, ... and
+// issues the loads of kCombineBatch of them before using any, so that enough
+// partial rows are in flight; lanes cover the head dimension.
 template <int D>
-__global__ void __launch_bounds__(kCombineWarps * 32) fpd_combine_kernel(const CombineParams p) {
-  __shared__ float acc_sm[kCombineWarps][D];
-  __shared__ float z_sm[kCombineWarps];
+__global__ void __launch_bounds__(kCombineMaxThreads) fpd_combine_kernel(const CombineParams p) {
+  __shared__ float acc_sm[kCombineMaxThreads / 32][D];
+  __shared__ float z_sm[kCombineMaxThreads / 32];
   pdl_wait_primary();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int wpr = p.wpr;
-  const int row = blockIdx.x * (kCombineWarps / wpr) + warp / wpr;
+  const int row = blockIdx.x * p.rows_per_cta + warp / wpr;
   const int j = warp % wpr;
   constexpr int PER = D / 32;
   int ns = 0;
@@ -822,23 +963,37 @@ __global__ void __launch_bounds__(kCombineWarps * 32) fpd_combine_kernel(const C
     const float* po = p.part_o + (size_t)row * p.max_splits * D + lane * PER;
     sink2 = p.sinks ? p.sinks[h] * kLog2e : -INFINITY;
     M = sink2;
-    for (int s = lane; s < ns; s += 32) M = fmaxf(M, pl[s]);
+    for (int s0 = lane; s0 < ns; s0 += 32 * kCombineBatch) {
+      float v[kCombineBatch];
+#pragma unroll
+      for (int u = 0; u < kCombineBatch; ++u) v[u] = pl[min(s0 + 32 * u, ns - 1)];
+#pragma unroll
+      for (int u = 0; u < kCombineBatch; ++u) M = fmaxf(M, v[u]);
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-#pragma unroll 4
-    for (int s = j; s < ns; s += wpr) {
-      const float w = fast_exp2(pl[s] - M);
-      z += w;
-      if constexpr (PER == 4) {
-        const float4 v = *reinterpret_cast<const float4*>(po + (size_t)s * D);
-        acc[0] += w * v.x;
-        acc[1] += w * v.y;
-        acc[2] += w * v.z;
-        acc[3] += w * v.w;
-      } else {
-        const float2 v = *reinterpret_cast<const float2*>(po + (size_t)s * D);
-        acc[0] += w * v.x;
-        acc[1] += w * v.y;
+    for (int s0 = j; s0 < ns; s0 += wpr * kCombineBatch) {
+      // past the last split, re-read the last one (in bounds) and weigh it 0
+      float lv[kCombineBatch];
+      float x[kCombineBatch][PER];
+#pragma unroll
+      for (int u = 0; u < kCombineBatch; ++u) {
+        const int s = min(s0 + wpr * u, ns - 1);
+        lv[u] = pl[s];
+        if constexpr (PER == 4) {
+          const float4 t = *reinterpret_cast<const float4*>(po + (size_t)s * D);
+          x[u][0] = t.x, x[u][1] = t.y, x[u][2] = t.z, x[u][3] = t.w;
+        } else {
+          const float2 t = *reinterpret_cast<const float2*>(po + (size_t)s * D);
+          x[u][0] = t.x, x[u][1] = t.y;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kCombineBatch; ++u) {
+        const float w = s0 + wpr * u < ns ? fast_exp2(lv[u] - M) : 0.f;
+        z += w;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) acc[i] = fmaf(w, x[u][i], acc[i]);
       }
     }
   }

@@ -8,6 +8,7 @@
 
 #include <cstdint>
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
 namespace fpd {
@@ -161,6 +162,12 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 // Two floats -> f16x2 (x in the lower half), round to nearest even.
 __device__ __forceinline__ uint32_t pack_f16x2(float x, float y) {
   __half2 h = __floats2half2_rn(x, y);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Two floats -> bf16x2 (x in the lower half), round to nearest even.
+__device__ __forceinline__ uint32_t pack_bf16x2(float x, float y) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
   return *reinterpret_cast<uint32_t*>(&h);
 }
 

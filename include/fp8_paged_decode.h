@@ -63,10 +63,12 @@ typedef enum {
 
 /* Split plan chosen by the host planner; all fields are outputs. */
 typedef struct {
-    int chunk_pages;        /* KV pages per split (one CTA per sequence, KV head and split) */
-    int max_splits;         /* splits launched per (sequence, KV head); unused ones exit at once */
-    int pages_per_stage;    /* pages moved per pipeline stage */
+    int chunk_pages;        /* KV pages per split (one work item per sequence, KV head group and split) */
+    int max_splits;         /* most splits of any one sequence */
+    int heads_per_stage;    /* KV heads per pipeline stage and work item: 4 when Hkv % 4 == 0, else 1 */
+    int stage_tokens;       /* tokens per KV head and stage (heads_per_stage * stage_tokens == 64) */
     int stages;             /* depth of the shared-memory ring */
+    int header_slots;       /* depth of the work-item header ring (1 or 2) */
     int ctas;               /* grid size of the split kernel */
     int smem_bytes;         /* dynamic shared memory per CTA */
     size_t workspace_bytes; /* bytes this plan needs */
@@ -82,8 +84,8 @@ typedef struct {
 /*
  * Host-only planner (no CUDA call): the split plan for a shape on a device with
  * `num_sms` SMs of which `ctas_per_sm` CTAs of the split kernel fit per SM.
- * chunk_pages_override > 0 forces the pages per split (rounded up to whole
- * pipeline stages); 0 lets the heuristic choose.
+ * chunk_pages_override > 0 forces the pages per split (with one KV head per
+ * stage, rounded up to whole 64-token stages); 0 lets the heuristic choose.
  * Returns FPD_OK or the validation error for the shape.
  */
 fpd_status fp8_paged_decode_make_plan(int B, int Hq, int Hkv, int D, int block_tokens,

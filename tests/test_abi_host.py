@@ -58,26 +58,56 @@ def test_planner_fills_the_machine():
                   dict(B=256, Hq=64, Hkv=8, block_tokens=32, max_blocks=1024, window_left=4096)]:
         p = plan(**shape)
         # a persistent grid: one CTA per resident slot (148 SMs x 2)
-        assert p["ctas"] == min(296, shape["B"] * shape["Hkv"] * p["max_splits"]) == 296
+        # Hkv = 8: work items and stages cover KV heads in groups of 4
+        assert p["heads_per_stage"] == 4 and p["stage_tokens"] == 16
+        units = shape["B"] * shape["Hkv"] // 4
+        assert p["ctas"] == min(296, units * p["max_splits"]) == 296
         # enough work items for several per slot on long inputs
-        assert shape["B"] * shape["Hkv"] * p["max_splits"] >= 4 * 296
-        assert p["chunk_pages"] % p["pages_per_stage"] == 0
-        assert p["pages_per_stage"] * shape["block_tokens"] == 64
+        assert units * p["max_splits"] >= 4 * 296
+        # at least 256 (token, KV head) rows per work item
+        assert p["chunk_pages"] * shape["block_tokens"] * 4 >= 256
+
+
+def test_planner_one_head_per_stage():
+    # Hkv not a multiple of 4: one KV head per 64-token stage, whole stages per split
+    for bt in (16, 32, 64):
+        p = plan(Hq=16, Hkv=2, block_tokens=bt, max_blocks=8192 // bt)
+        assert p["heads_per_stage"] == 1 and p["stage_tokens"] == 64
+        assert p["chunk_pages"] * bt % 64 == 0
+        assert p["ctas"] == min(296, 32 * 2 * p["max_splits"])
+
+
+def test_planner_header_slots():
+    # two header slots while an item's query rows fit in 4 KB
+    assert plan()["header_slots"] == 2                           # 4 x 4 heads x 128 x 2 B
+    assert plan(Hq=64, Hkv=8)["header_slots"] == 1               # 4 x 8 heads
+    assert plan(Hq=64, Hkv=8, D=64)["header_slots"] == 2
+    assert plan(Hq=32, Hkv=2)["header_slots"] == 2               # 1 x 16 heads
 
 
 def test_planner_window_caps_splits():
+    # a 129-token window spans at most 10 pages: one split.  64 sequences x 2
+    # four-head groups would leave CTA slots idle, so the planner falls back to
+    # one head per stage (64 x 8 work items)
     p = plan(B=64, Hq=64, Hkv=8, D=64, block_tokens=16, max_blocks=1024, window_left=128)
-    # a 129-token window spans at most 10 pages: a single split
-    assert p["max_splits"] == 1 and p["workspace_bytes"] == 256
+    assert p["heads_per_stage"] == 1 and p["max_splits"] == 1 and p["workspace_bytes"] == 256
+    assert p["ctas"] == 296
+    # with enough sequences the four-head shape fills the machine by itself
+    p4 = plan(B=512, Hq=64, Hkv=8, D=64, block_tokens=16, max_blocks=1024, window_left=128)
+    assert p4["heads_per_stage"] == 4 and p4["max_splits"] == 1
 
 
 def test_planner_override_and_workspace():
-    p = plan(chunk_pages_override=5)
-    assert p["chunk_pages"] == 8          # rounded up to whole 4-page stages
+    # one KV head per stage: rounded up to whole 64-token (4-page) stages
+    p = plan(Hq=8, Hkv=2, chunk_pages_override=5)
+    assert p["chunk_pages"] == 8
     assert p["max_splits"] == 512 // 8
     # header + partial O + partial lse
-    ws = 256 + 32 * 32 * 64 * 128 * 4 + 32 * 32 * 64 * 4
+    ws = 256 + 32 * 8 * 64 * 128 * 4 + 32 * 8 * 64 * 4
     assert p["workspace_bytes"] == ws
+    # four KV heads per stage: 16-token stages, any page count
+    p4 = plan(chunk_pages_override=5)
+    assert p4["chunk_pages"] == 5 and p4["max_splits"] == -(-512 // 5)
     p1 = plan(chunk_pages_override=512)
     assert p1["max_splits"] == 1 and p1["workspace_bytes"] == 256
 

@@ -31,36 +31,50 @@ def test_tiny_config():
     check(W.make_workload("tiny"))
 
 
-GRID = list(itertools.product([64, 128], [1, 2, 4, 8, 16], [16, 32, 64]))
+GRID = list(itertools.product([64, 128], [1, 2, 4, 8, 16], [16, 32, 64], [2, 4]))
 
 
-@pytest.mark.parametrize("D,g,bt", GRID, ids=[f"D{d}-g{g}-bt{b}" for d, g, b in GRID])
-def test_shape_grid(D, g, bt):
-    Hkv = 2
+@pytest.mark.parametrize("D,g,bt,Hkv", GRID,
+                         ids=[f"D{d}-g{g}-bt{b}-kv{h}" for d, g, b, h in GRID])
+def test_shape_grid(D, g, bt, Hkv):
+    """Hkv = 2: one KV head per stage.  Hkv = 4: four heads per stage whenever
+    the split size is forced (the planner's own choice for so few sequences is
+    one head per stage)."""
     lens = [1, bt - 1, bt, bt + 1, 3 * bt + 5, 700]
     wl = W.make_custom(B=len(lens), Hq=g * Hkv, Hkv=Hkv, D=D, block_tokens=bt, seq_lens=lens,
-                       seed=100 + D + g + bt, sm_scale=1.0 / np.sqrt(D))
+                       seed=100 + D + g + bt + Hkv, sm_scale=1.0 / np.sqrt(D))
     check(wl)
-    check(wl, chunk_pages=64 // bt)          # one stage per split: many splits + combine
+    check(wl, chunk_pages=64 // bt)          # 64 tokens per split: many splits + combine
+    if Hkv == 4:
+        check(wl, chunk_pages=10 ** 4)       # one split per sequence: output written directly
+
+
+def test_stage_shape_choice():
+    """The shapes above really exercise both stage layouts."""
+    kw = dict(B=6, D=128, block_tokens=16, max_blocks=44, window_left=-1)
+    assert fpd.fp8_paged_decode_plan(Hq=8, Hkv=2, **kw)["heads_per_stage"] == 1
+    assert fpd.fp8_paged_decode_plan(Hq=16, Hkv=4, chunk_pages_override=4,
+                                     **kw)["heads_per_stage"] == 4
 
 
 @pytest.mark.parametrize("window,sinks", [(0, True), (5, False), (40, True), (129, True),
                                           (10 ** 6, True)])
 def test_window_and_sinks(window, sinks):
-    wl = W.make_custom(B=6, Hq=16, Hkv=2, D=128, block_tokens=16,
-                       seq_lens=[1, 2, 17, 130, 300, 1000], window_left=window, sinks=sinks,
-                       seed=7 + window, sm_scale=0.1, sigma=2.0)
-    check(wl)
-    check(wl, chunk_pages=4)
+    for Hkv in (2, 4):
+        wl = W.make_custom(B=6, Hq=8 * Hkv, Hkv=Hkv, D=128, block_tokens=16,
+                           seq_lens=[1, 2, 17, 130, 300, 1000], window_left=window, sinks=sinks,
+                           seed=7 + window + Hkv, sm_scale=0.1, sigma=2.0)
+        check(wl)
+        check(wl, chunk_pages=4)
+        check(wl, chunk_pages=10 ** 4)
 
 
-def test_empty_sequence():
-    wl = W.make_custom(B=3, Hq=8, Hkv=2, D=64, block_tokens=16, seq_lens=[0, 5, 0], sinks=True,
-                       seed=31)
-    wl_ns = W.make_custom(B=3, Hq=8, Hkv=2, D=64, block_tokens=16, seq_lens=[0, 5, 0],
-                          sinks=False, seed=31)
-    for w in (wl, wl_ns):
-        out, lse = run_cuda(w)
+@pytest.mark.parametrize("Hkv,chunk", [(2, 0), (4, 1), (4, 10 ** 4)])
+def test_empty_sequence(Hkv, chunk):
+    for sinks in (True, False):
+        w = W.make_custom(B=3, Hq=4 * Hkv, Hkv=Hkv, D=64, block_tokens=16, seq_lens=[0, 5, 0],
+                          sinks=sinks, seed=31)
+        out, lse = run_cuda(w, chunk_pages=chunk)
         ref_out, ref_lse = oracle.decode_workload(w)
         assert_parity(out, lse, ref_out, ref_lse, what="empty")
         assert (out[0] == 0).all() and (out[2] == 0).all()
