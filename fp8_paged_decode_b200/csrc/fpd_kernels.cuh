@@ -935,72 +935,104 @@ constexpr int kCombineBatch = 8;   // partials a warp loads before it reduces th
 // Rows (sequence, query head) whose sequence spans several splits:
 //   out = v_scale sum_s 2^(lse_s - M) o_s / (sum_s 2^(lse_s - M) + 2^(sigma - M)),
 //   lse = (M + log2 Z) ln 2,  M = max(max_s lse_s, sigma)  (sigma in log2 units).
-// Each row gets `wpr` warps; warp j of a row takes splits j, j + wpr, ... and
-// issues the loads of kCombineBatch of them before using any, so that enough
-// partial rows are in flight; lanes cover the head dimension.
+// Each row gets `wpr` warps; warp j of a row takes splits j, j + wpr, ...  The
+// first kCombineBatch of them are loaded together with the sequence length,
+// before the split count is known (in bounds: every row owns max_splits
+// partials; entries past the count are never used), so the whole merge costs
+// one round trip to memory.  Each warp reduces against its own maximum; the
+// row's warps are combined in shared memory.
 template <int D>
 __global__ void __launch_bounds__(kCombineMaxThreads) fpd_combine_kernel(const CombineParams p) {
-  __shared__ float acc_sm[kCombineMaxThreads / 32][D];
-  __shared__ float z_sm[kCombineMaxThreads / 32];
+  constexpr int kMaxWarps = kCombineMaxThreads / 32;
+  __shared__ float acc_sm[kMaxWarps][D];
+  __shared__ float z_sm[kMaxWarps], m_sm[kMaxWarps];
   pdl_wait_primary();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int wpr = p.wpr;
   const int row = blockIdx.x * p.rows_per_cta + warp / wpr;
   const int j = warp % wpr;
+  const bool in_range = row < p.B * p.Hq;
   constexpr int PER = D / 32;
-  int ns = 0;
-  if (row < p.B * p.Hq)
-    ns = seq_range(p.seq_lens[row / p.Hq], p.bt, p.max_blocks, p.window_left, p.chunk_pages,
-                   nullptr).n_splits;
-  const bool active = ns > 1;   // rows with one split were written by the split kernel
-  float M = -INFINITY, z = 0.f, sink2 = -INFINITY;
+  const int ms = p.max_splits;
+  const float* pl = p.part_lse + (size_t)(in_range ? row : 0) * ms;
+  const float* po = p.part_o + (size_t)(in_range ? row : 0) * ms * D + lane * PER;
+
+  // ---- one round of loads: the sequence length and this warp's first batch
+  const int L_raw = in_range ? p.seq_lens[row / p.Hq] : 0;
+  float lv[kCombineBatch];
+  float x[kCombineBatch][PER];
+#pragma unroll
+  for (int u = 0; u < kCombineBatch; ++u) {
+    const int s = j + wpr * u;
+    lv[u] = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) x[u][i] = 0.f;
+    if (in_range && s < ms) {
+      lv[u] = pl[s];
+      if constexpr (PER == 4) {
+        const float4 t = *reinterpret_cast<const float4*>(po + (size_t)s * D);
+        x[u][0] = t.x, x[u][1] = t.y, x[u][2] = t.z, x[u][3] = t.w;
+      } else {
+        const float2 t = *reinterpret_cast<const float2*>(po + (size_t)s * D);
+        x[u][0] = t.x, x[u][1] = t.y;
+      }
+    }
+  }
+  const int ns = seq_range(L_raw, p.bt, p.max_blocks, p.window_left, p.chunk_pages, nullptr)
+                     .n_splits;
+  const bool active = in_range && ns > 1;   // rows with one split were written already
+
+  // ---- this warp's splits against its own maximum m
+  float m = -INFINITY, z = 0.f;
   float acc[PER];
 #pragma unroll
   for (int i = 0; i < PER; ++i) acc[i] = 0.f;
   if (active) {
-    const int h = row % p.Hq;
-    const float* pl = p.part_lse + (size_t)row * p.max_splits;
-    const float* po = p.part_o + (size_t)row * p.max_splits * D + lane * PER;
-    sink2 = p.sinks ? p.sinks[h] * kLog2e : -INFINITY;
-    M = sink2;
-    for (int s0 = lane; s0 < ns; s0 += 32 * kCombineBatch) {
-      float v[kCombineBatch];
 #pragma unroll
-      for (int u = 0; u < kCombineBatch; ++u) v[u] = pl[min(s0 + 32 * u, ns - 1)];
+    for (int u = 0; u < kCombineBatch; ++u)
+      if (j + wpr * u < ns) m = fmaxf(m, lv[u]);
 #pragma unroll
-      for (int u = 0; u < kCombineBatch; ++u) M = fmaxf(M, v[u]);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    for (int s0 = j; s0 < ns; s0 += wpr * kCombineBatch) {
-      // past the last split, re-read the last one (in bounds) and weigh it 0
-      float lv[kCombineBatch];
-      float x[kCombineBatch][PER];
-#pragma unroll
-      for (int u = 0; u < kCombineBatch; ++u) {
-        const int s = min(s0 + wpr * u, ns - 1);
-        lv[u] = pl[s];
-        if constexpr (PER == 4) {
-          const float4 t = *reinterpret_cast<const float4*>(po + (size_t)s * D);
-          x[u][0] = t.x, x[u][1] = t.y, x[u][2] = t.z, x[u][3] = t.w;
-        } else {
-          const float2 t = *reinterpret_cast<const float2*>(po + (size_t)s * D);
-          x[u][0] = t.x, x[u][1] = t.y;
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < kCombineBatch; ++u) {
-        const float w = s0 + wpr * u < ns ? fast_exp2(lv[u] - M) : 0.f;
+    for (int u = 0; u < kCombineBatch; ++u) {
+      if (j + wpr * u < ns) {   // never touch the unused (possibly stale) entries
+        const float w = fast_exp2(lv[u] - m);
         z += w;
 #pragma unroll
         for (int i = 0; i < PER; ++i) acc[i] = fmaf(w, x[u][i], acc[i]);
       }
     }
+    // splits beyond the first batch (more than wpr * kCombineBatch of them)
+    for (int s = j + wpr * kCombineBatch; s < ns; s += wpr) {
+      const float l = pl[s];
+      float v[PER];
+      if constexpr (PER == 4) {
+        const float4 t = *reinterpret_cast<const float4*>(po + (size_t)s * D);
+        v[0] = t.x, v[1] = t.y, v[2] = t.z, v[3] = t.w;
+      } else {
+        const float2 t = *reinterpret_cast<const float2*>(po + (size_t)s * D);
+        v[0] = t.x, v[1] = t.y;
+      }
+      if (l > m) {   // rescale to the new maximum
+        const float r = fast_exp2(m - l);
+        z *= r;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) acc[i] *= r;
+        m = l;
+      }
+      const float w = fast_exp2(l - m);
+      z += w;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) acc[i] = fmaf(w, v[i], acc[i]);
+    }
   }
+
+  // ---- merge the row's warps (M = max over warps and the sink) and write
+  const float sink2 = (active && p.sinks) ? p.sinks[row % p.Hq] * kLog2e : -INFINITY;
   if (wpr == 1) {
     if (active) {
-      const float Z = z + (p.sinks ? fast_exp2(sink2 - M) : 0.f);
-      const float inv = p.v_scale / Z;
+      const float M = fmaxf(m, sink2);
+      const float r = fast_exp2(m - M);
+      const float Z = z * r + (p.sinks ? fast_exp2(sink2 - M) : 0.f);
+      const float inv = p.v_scale * r / Z;
       __nv_bfloat16* dst = p.out + (size_t)row * D + lane * PER;
 #pragma unroll
       for (int i = 0; i < PER; ++i) dst[i] = __float2bfloat16_rn(acc[i] * inv);
@@ -1010,19 +1042,34 @@ __global__ void __launch_bounds__(kCombineMaxThreads) fpd_combine_kernel(const C
   }
 #pragma unroll
   for (int i = 0; i < PER; ++i) acc_sm[warp][lane * PER + i] = acc[i];
-  if (lane == 0) z_sm[warp] = z;
+  if (lane == 0) {
+    z_sm[warp] = z;
+    m_sm[warp] = m;
+  }
   __syncthreads();
   if (active && j == 0) {   // the row's first warp finishes it
-    float Z = p.sinks ? fast_exp2(sink2 - M) : 0.f;
-    for (int w = warp; w < warp + wpr; ++w) Z += z_sm[w];
-    const float inv = p.v_scale / Z;
+    // lane w < wpr holds warp w's maximum, weight and sum
+    const float mw = lane < wpr ? m_sm[warp + lane] : -INFINITY;
+    float M = fmaxf(sink2, mw);
 #pragma unroll
-    for (int i = 0; i < PER; ++i) {
-      const int d = lane * PER + i;
-      float a = 0.f;
-      for (int w = warp; w < warp + wpr; ++w) a += acc_sm[w][d];
-      p.out[(size_t)row * D + d] = __float2bfloat16_rn(a * inv);
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float rw = mw == -INFINITY ? 0.f : fast_exp2(mw - M);   // 0: warp without a split
+    float Z = lane < wpr ? z_sm[warp + lane] * rw : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) Z += __shfl_xor_sync(0xffffffffu, Z, o);
+    if (p.sinks) Z += fast_exp2(sink2 - M);
+    const float inv = p.v_scale / Z;
+    float a[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) a[i] = 0.f;
+    for (int w = 0; w < wpr; ++w) {
+      const float r = __shfl_sync(0xffffffffu, rw, w);
+#pragma unroll
+      for (int i = 0; i < PER; ++i) a[i] = fmaf(acc_sm[warp + w][lane * PER + i], r, a[i]);
     }
+#pragma unroll
+    for (int i = 0; i < PER; ++i)
+      p.out[(size_t)row * D + lane * PER + i] = __float2bfloat16_rn(a[i] * inv);
     if (lane == 0 && p.lse) p.lse[row] = (M + __log2f(Z)) * kLn2;
   }
 }
