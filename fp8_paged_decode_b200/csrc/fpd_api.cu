@@ -251,11 +251,24 @@ cudaError_t launch_combine(const fpd::CombineParams& c, cudaStream_t st) {
   return cudaLaunchKernelEx(&cfg, fpd::fpd_combine_kernel<D>, c);
 }
 
+// The split kernel is launched as a programmatic dependent of whatever ran
+// before it in the stream: its CTAs may become resident while that kernel
+// drains, and its first instruction waits for that kernel's completion, so
+// the ordering is that of a plain launch without the launch gap.
 template <int D, int NT, int HB>
 cudaError_t launch_split(const CUtensorMap& km, const CUtensorMap& vm, const fpd::DecodeParams& p,
                          int ctas, int smem, cudaStream_t st) {
-  fpd::fpd_split_kernel<D, NT, HB><<<ctas, fpd::kThreads, smem, st>>>(km, vm, p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)ctas);
+  cfg.blockDim = dim3(fpd::kThreads);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, fpd::fpd_split_kernel<D, NT, HB>, km, vm, p);
 }
 
 template <int HB>

@@ -698,6 +698,11 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
   uint64_t* cbar = hdr_empty + kMaxHdrSlots;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
+  // The launch may be a programmatic dependent of the previous kernel in the
+  // stream (so that this grid's CTAs are resident when it finishes): nothing
+  // is read before that kernel has completed and its writes are visible.
+  pdl_wait_primary();
+
   // ---- prefix over sequences of their work groups (every CTA builds its own)
   {
     const int per = (p.B + kThreads - 1) / kThreads;
@@ -946,6 +951,7 @@ __global__ void __launch_bounds__(kCombineMaxThreads) fpd_combine_kernel(const C
   constexpr int kMaxWarps = kCombineMaxThreads / 32;
   __shared__ float acc_sm[kMaxWarps][D];
   __shared__ float z_sm[kMaxWarps], m_sm[kMaxWarps];
+  pdl_launch_dependents();   // the next call's split kernel may be scheduled
   pdl_wait_primary();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int wpr = p.wpr;
