@@ -44,6 +44,11 @@ def _bind(lib):
     lib.fpd_oracle_decode.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci,
                                       cd, cd, cd, ci, vp, vp, vp, vp, ci, ci]
     lib.fpd_oracle_decode.restype = ci
+    lib.fpd_oracle_f64_to_e4m3.argtypes = [ctypes.c_double]
+    lib.fpd_oracle_f64_to_e4m3.restype = ctypes.c_uint8
+    lib.fpd_oracle_cache_write.argtypes = [vp, vp, vp, ci, ci, ci, ctypes.c_long, ctypes.c_long,
+                                           ctypes.c_float, ctypes.c_float, vp, vp, ci, ci]
+    lib.fpd_oracle_cache_write.restype = ci
     del u8p
     return lib
 
@@ -68,6 +73,36 @@ def e4m3_to_f64(code: int, lib=None) -> float:
 
 def bf16_to_f64(bits: int, lib=None) -> float:
     return (lib or load()).fpd_oracle_bf16_to_f64(int(bits))
+
+
+def f64_to_e4m3(x: float, lib=None) -> int:
+    """Nearest E4M3 code, ties to even, saturating at +-448 (NaN -> S.1111.111)."""
+    return int((lib or load()).fpd_oracle_f64_to_e4m3(float(x)))
+
+
+def cache_write(key, value, slot_mapping, k_cache, v_cache, *, k_scale, v_scale, lib=None) -> int:
+    """FP8 KV-cache write into ``k_cache``/``v_cache`` (uint8 [num_blocks, bt, Hkv, D],
+    modified in place) of bf16 ``key``/``value`` (uint16 bits [num_tokens, Hkv, D],
+    any token stride) at ``slot_mapping`` (int64 [num_tokens], negative = skip).
+    Returns the number of out-of-range slots (skipped)."""
+    lib = lib or load()
+    assert key.dtype == np.uint16 and value.dtype == np.uint16
+    assert k_cache.dtype == np.uint8 and k_cache.flags.c_contiguous and v_cache.flags.c_contiguous
+    num_blocks, bt, Hkv, D = k_cache.shape
+    T = key.shape[0]
+    assert key.shape[1:] == (Hkv, D) and value.shape[1:] == (Hkv, D)
+    for a in (key, value):
+        assert a.strides[2] == 2 and a.strides[1] == 2 * D, "rows must be contiguous per token"
+    slot_mapping = np.ascontiguousarray(slot_mapping, dtype=np.int64)
+    assert slot_mapping.shape == (T,)
+    st = lib.fpd_oracle_cache_write(key.ctypes.data_as(ctypes.c_void_p),
+                                    value.ctypes.data_as(ctypes.c_void_p), _ptr(slot_mapping), T,
+                                    Hkv, D, key.strides[0] // 2, value.strides[0] // 2,
+                                    float(k_scale), float(v_scale), _ptr(k_cache), _ptr(v_cache),
+                                    num_blocks, bt)
+    if st < 0:
+        raise ValueError("oracle rejected the cache-write arguments")
+    return st
 
 
 def _ptr(a: Optional[np.ndarray]):

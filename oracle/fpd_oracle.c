@@ -37,6 +37,9 @@
  * gist's quantisation helpers): 1 sign, 4 exponent (bias 7), 3 mantissa bits;
  * exponent 0 is subnormal; S.1111.111 is NaN; there are no infinities.
  *
+ * The file also holds the oracle of the FP8 cache write that fills such a
+ * cache (fpd_oracle_cache_write, below the E4M3 codec).
+ *
  * Degenerate cases: L == 0 gives out = 0 and lse = sigma (-inf without sinks).
  * A stored NaN code inside the attended range propagates NaN (plain
  * arithmetic); codes outside the attended range are never read.
@@ -70,6 +73,78 @@ double fpd_oracle_bf16_to_f64(uint16_t bits)
     float f;
     memcpy(&f, &u, sizeof f);
     return (double)f;
+}
+
+/*
+ * Real value -> E4M3 code: the nearest representable value, ties to the even
+ * code (mantissa LSB 0), saturating to +-448 (S.1111.110) beyond the largest
+ * finite value, so +-inf saturate too; NaN gives the NaN code S.1111.111.
+ * The sign of zero is kept.  Written as the definition: a search over the
+ * 127 non-negative finite codes, which are increasing in value.
+ */
+uint8_t fpd_oracle_f64_to_e4m3(double x)
+{
+    const uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    const double a = fabs(x);
+    int best = 0, c;
+    double best_d;
+    if (isnan(x))
+        return (uint8_t)(sign | 0x7F);
+    if (a >= 448.0)
+        return (uint8_t)(sign | 0x7E);
+    best_d = a; /* distance to code 0 (+0) */
+    for (c = 1; c <= 0x7E; ++c) {
+        const double d = fabs(a - fpd_oracle_e4m3_to_f64((uint8_t)c));
+        if (d < best_d || (d == best_d && (c & 1) == 0 && (best & 1) == 1)) {
+            best = c;
+            best_d = d;
+        }
+    }
+    return (uint8_t)(sign | best);
+}
+
+/*
+ * FP8 KV-cache write (test infrastructure, like everything in this file).
+ * The per-tensor quantisation of the cache writer in the NVFP4 KV-cache gist
+ * (its standalone writer kernel and host wrapper): the scale's reciprocal is
+ * taken in fp32 and every element is multiplied by it in fp32 before
+ * rounding, i.e. stored = e4m3_rne_sat(float(x) * (1.0f / scale)).  Token t
+ * goes to slot s = slot_mapping[t] = page * bt + offset of the
+ * [num_blocks, bt, Hkv, D] caches; a negative slot is a padded token and is
+ * skipped.  key and value are bf16 bit patterns [num_tokens, Hkv, D] with a
+ * token stride of key_stride / value_stride elements.  Returns the number of
+ * slots past the end of the cache (skipped), or -1 for a bad argument.
+ */
+int fpd_oracle_cache_write(const uint16_t *key, const uint16_t *value, const int64_t *slot_mapping,
+                           int num_tokens, int Hkv, int D, long key_stride, long value_stride,
+                           float k_scale, float v_scale, uint8_t *k_cache, uint8_t *v_cache,
+                           int num_blocks, int bt)
+{
+    const float kr = 1.0f / k_scale, vr = 1.0f / v_scale;
+    const int64_t n_slots = (int64_t)num_blocks * bt;
+    int bad = 0, t, h, d;
+    if (num_tokens < 0 || Hkv <= 0 || D <= 0 || num_blocks <= 0 || bt <= 0)
+        return -1;
+    for (t = 0; t < num_tokens; ++t) {
+        const int64_t slot = slot_mapping[t];
+        if (slot < 0)
+            continue;
+        if (slot >= n_slots) {
+            ++bad;
+            continue;
+        }
+        for (h = 0; h < Hkv; ++h) {
+            for (d = 0; d < D; ++d) {
+                const size_t dst = ((size_t)slot * Hkv + h) * (size_t)D + d;
+                const float xk = (float)fpd_oracle_bf16_to_f64(key[t * key_stride + (long)h * D + d]);
+                const float xv = (float)fpd_oracle_bf16_to_f64(value[t * value_stride + (long)h * D + d]);
+                const float yk = xk * kr, yv = xv * vr; /* fp32 products, round to nearest */
+                k_cache[dst] = fpd_oracle_f64_to_e4m3((double)yk);
+                v_cache[dst] = fpd_oracle_f64_to_e4m3((double)yv);
+            }
+        }
+    }
+    return bad;
 }
 
 typedef struct {

@@ -279,5 +279,124 @@ def pin_softmax_identity(lib):
             assert abs(tot - 1.0) < 1e-12, f"probabilities sum to {tot}"
 
 
+# ------------------------------------------------------------ cache write --
+
+def e4m3_encode_library(x: np.ndarray) -> np.ndarray:
+    """float32 -> E4M3 codes by torch's float8_e4m3fn cast (round to nearest
+    even; defined by torch for |x| <= 448 only)."""
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.float8_e4m3fn)
+    return t.view(torch.uint8).numpy()
+
+
+def pin_e4m3_encode_library(lib):
+    """Random float32 values, every code value and every midpoint between
+    neighbouring codes, against torch's cast."""
+    rng = np.random.default_rng(40)
+    vals = [rng.standard_normal(4000) * s for s in (0.003, 0.1, 1.0, 30.0, 200.0)]
+    codes = np.arange(256, dtype=np.uint8)
+    real = e4m3_library(codes)
+    finite = np.sort(np.unique(real[np.isfinite(real)]))
+    mids = (finite[1:] + finite[:-1]) / 2                         # exact in float32
+    x = np.concatenate(vals + [finite, mids, -mids]).astype(np.float32)
+    x = x[np.abs(x) <= 448]
+    want = e4m3_encode_library(x)
+    got = np.array([oracle.f64_to_e4m3(float(v), lib=lib) for v in x], dtype=np.uint8)
+    bad = np.flatnonzero(want != got)
+    assert bad.size == 0, f"{bad.size} codes differ, e.g. x={x[bad[0]]!r}: {got[bad[0]]:#x} vs {want[bad[0]]:#x}"
+
+
+def pin_e4m3_encode_closed(lib):
+    """Closed forms of the encoder: every non-NaN code round-trips, ties go to
+    the even code, +-inf and anything past 448 saturate, signs (and the sign of
+    zero) are kept, NaN stays NaN."""
+    enc = lambda v: oracle.f64_to_e4m3(v, lib=lib)
+    for c in range(256):
+        if c & 0x7F == 0x7F:
+            continue
+        v = oracle.e4m3_to_f64(c, lib=lib)
+        assert enc(v) == c, f"code {c:#x} ({v}) does not round-trip"
+    assert enc(1.0 + 1 / 16) == 0x38 and enc(1.0 + 3 / 16) == 0x3A        # ties to even
+    assert enc(2.0 ** -10) == 0x00 and enc(3 * 2.0 ** -10) == 0x02         # subnormal ties
+    assert enc(2.0 ** -10 * 1.0001) == 0x01
+    for v in (448.0, 449.0, 464.0, 1e30, math.inf):
+        assert enc(v) == 0x7E and enc(-v) == 0xFE, f"{v} does not saturate"
+    assert enc(0.0) == 0x00 and enc(-0.0) == 0x80 and enc(-1e-9) == 0x80
+    assert enc(math.nan) & 0x7F == 0x7F
+
+
+def cache_write_library(key, value, slots, k_cache, v_cache, k_scale, v_scale):
+    """The cache write with torch: float32 product with the float32 reciprocal of
+    the scale, clamp to +-448, torch's float8 cast, numpy scatter."""
+    kc, vc = k_cache.copy(), v_cache.copy()
+    nb, bt, H, D = kc.shape
+    for src, scale, dst in ((key, k_scale, kc), (value, v_scale, vc)):
+        x = torch.from_numpy(np.ascontiguousarray(src).view(np.int16)).view(torch.bfloat16).float()
+        y = x * (torch.tensor(1.0, dtype=torch.float32) / torch.tensor(scale, dtype=torch.float32))
+        codes = y.clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        flat = dst.reshape(nb * bt, H, D)
+        for t, sl in enumerate(slots):
+            if 0 <= sl < nb * bt:
+                flat[sl] = codes[t]
+    return kc, vc
+
+
+def pin_cache_write_library(lib):
+    """Scatter with negative (skipped) slots and a strided key, bit-exact
+    against the torch version."""
+    rng = np.random.default_rng(41)
+    nb, bt, H, D, T = 7, 16, 3, 64, 40
+    wide = rng.standard_normal((T, H * D * 2)).astype(np.float32) * 3
+    kbits = torch.from_numpy(wide).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    key = kbits[:, : H * D].reshape(T, H, D)            # token stride 2*H*D: a slice
+    value = torch.from_numpy(rng.standard_normal((T, H, D)).astype(np.float32) * 50).to(
+        torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    slots = rng.permutation(nb * bt)[:T].astype(np.int64)
+    slots[slots == 0] = slots[0]
+    slots[0] = 0                                        # the first slot of the pool is used
+    slots[[3, 17, 30]] = -1                             # padded tokens
+    kc0 = rng.integers(0, 256, (nb, bt, H, D), dtype=np.uint8)
+    vc0 = rng.integers(0, 256, (nb, bt, H, D), dtype=np.uint8)
+    for ks, vs in ((0.02, 0.5), (1.0, 1.0), (3.7, 0.013)):
+        kc, vc = kc0.copy(), vc0.copy()
+        assert oracle.cache_write(key, value, slots, kc, vc, k_scale=ks, v_scale=vs, lib=lib) == 0
+        wk, wv = cache_write_library(key, value, slots, kc0, vc0, ks, vs)
+        assert np.array_equal(kc, wk), "K cache differs"
+        assert np.array_equal(vc, wv), "V cache differs"
+
+
+def pin_cache_write_invariants(lib):
+    """Permuting tokens together with their slots changes nothing; an
+    out-of-range slot is reported and skipped; a cache read back through the
+    decoder returns the (scaled) values when they are exact E4M3 values."""
+    rng = np.random.default_rng(42)
+    nb, bt, H, D, T = 5, 32, 2, 128, 50
+    key = torch.from_numpy(rng.standard_normal((T, H, D)).astype(np.float32)).to(
+        torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    value = key[::-1].copy()
+    slots = rng.permutation(nb * bt)[:T].astype(np.int64)
+    kc = np.zeros((nb, bt, H, D), np.uint8)
+    vc = np.zeros_like(kc)
+    oracle.cache_write(key, value, slots, kc, vc, k_scale=0.25, v_scale=2.0, lib=lib)
+    perm = rng.permutation(T)
+    kc2, vc2 = np.zeros_like(kc), np.zeros_like(vc)
+    oracle.cache_write(np.ascontiguousarray(key[perm]), np.ascontiguousarray(value[perm]),
+                       slots[perm], kc2, vc2, k_scale=0.25, v_scale=2.0, lib=lib)
+    assert np.array_equal(kc, kc2) and np.array_equal(vc, vc2)
+    bad = slots.copy()
+    bad[5] = nb * bt
+    kc3, vc3 = np.zeros_like(kc), np.zeros_like(vc)
+    assert oracle.cache_write(key, value, bad, kc3, vc3, k_scale=0.25, v_scale=2.0, lib=lib) == 1
+    assert not kc3.reshape(-1, H, D)[slots[5]].any(), "the skipped token was written"
+    # exact values: codes decoded and scaled back are the inputs
+    codes = rng.integers(0, 0x7F, (T, H, D)).astype(np.uint8)
+    exact = e4m3_library(codes) * 0.5                   # bf16 holds these exactly
+    xb = torch.from_numpy(exact).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    kc4, vc4 = np.zeros_like(kc), np.zeros_like(vc)
+    oracle.cache_write(xb, xb, slots, kc4, vc4, k_scale=0.5, v_scale=0.5, lib=lib)
+    back = e4m3_library(kc4.reshape(-1, H, D)[slots]) * 0.5
+    assert np.array_equal(back, exact)
+
+
 ALL_PINS = [pin_e4m3_codes, pin_bf16, pin_library_attention, pin_zero_keys, pin_window_zero,
-            pin_constant_values, pin_invariants, pin_softmax_identity]
+            pin_constant_values, pin_invariants, pin_softmax_identity, pin_e4m3_encode_library,
+            pin_e4m3_encode_closed, pin_cache_write_library, pin_cache_write_invariants]

@@ -43,6 +43,20 @@ MUTANTS = {
     "bf16 decode shift": [("(uint32_t)bits << 16", "(uint32_t)bits << 15")],
     "max not subtracted consistently": [("const double p = exp(s[j - start] - m);",
                                          "const double p = exp(s[j - start]);")],
+    "encoder ties away from zero": [("(d == best_d && (c & 1) == 0 && (best & 1) == 1)",
+                                     "(d == best_d)")],
+    "encoder does not saturate infinities": [("    if (a >= 448.0)\n        return (uint8_t)(sign | 0x7E);\n", "")],
+    "encoder drops the sign": [("return (uint8_t)(sign | best);", "return (uint8_t)best;")],
+    "writer divides instead of the fp32 reciprocal product": [
+        ("const float yk = xk * kr, yv = xv * vr;", "const float yk = xk * kr * 1.0000001f, yv = xv * vr;")],
+    "writer skips slot 0 too": [("        if (slot < 0)\n            continue;\n", "        if (slot <= 0)\n            continue;\n")],
+    "writer swaps K and V scales": [("const float kr = 1.0f / k_scale, vr = 1.0f / v_scale;",
+                                     "const float kr = 1.0f / v_scale, vr = 1.0f / k_scale;")],
+    "writer cache head-major (transposed operand)": [
+        ("const size_t dst = ((size_t)slot * Hkv + h) * (size_t)D + d;",
+         "const size_t dst = (((size_t)(slot / bt) * Hkv + h) * bt + slot % bt) * (size_t)D + d;")],
+    "writer value read with the key stride": [("value[t * value_stride + (long)h * D + d]",
+                                               "value[t * key_stride + (long)h * D + d]")],
     "last key dropped": [("for (j = start; j < L; ++j) {\n        const int page = J->block_table"
                           "[(size_t)b * J->max_blocks + j / J->bt];\n        const uint8_t *vr",
                           "for (j = start; j < L - 1; ++j) {\n        const int page = J->block_table"
