@@ -19,6 +19,14 @@ independent replicas, one per GPU (weak scaling): the path has no exchange.
 `--impl reference` times the fp64 CPU oracle (on the host cores, bounded
 samples of the same workload) and prints the same JSON line with
 "impl": "reference".
+
+`--op cache_write` instead measures the FP8 KV-cache write (bf16 K/V of new
+tokens quantised and scattered into the paged caches): HBM GB/s of its bytes
+(4 read + 2 written per element) on a prefill-sized batch larger than L2
+(`--write-tokens`, default 65536 tokens of the Llama-3-8B shape: 384 MB per
+call) and the latency of a decode-step batch (one token per sequence of the
+decode workload), timed as replays of a CUDA graph of 100 calls so that host
+launch overhead is excluded.
 """
 from __future__ import annotations
 
@@ -57,6 +65,8 @@ def parse_args():
     ap.add_argument("--kernels-only", action="store_true",
                     help="only run warm-up + K plain calls (for ncu launch lists and captures)")
     ap.add_argument("--json-out", default=None)
+    ap.add_argument("--op", default="decode", choices=["decode", "cache_write"])
+    ap.add_argument("--write-tokens", type=int, default=65536)
     return ap.parse_args()
 
 
@@ -527,10 +537,99 @@ def run_native(args):
     return 0
 
 
+def run_cache_write(args):
+    """FP8 KV-cache write: GB/s on a large batch, us on a decode-step batch (1 GPU)."""
+    import numpy as np
+    import torch
+    import fp8_paged_decode_b200 as fpd
+    from fp8_paged_decode_b200 import workloads as W
+    c = W.CONFIGS[args.config]
+    Hkv, D, bt = c["Hkv"], c["D"], c["block_tokens"]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    hbm, peak_src = measured_peaks()
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(5)
+    res = {}
+    for name, T in (("prefill", args.write_tokens), ("decode_step", c["B"])):
+        nb = 2 * ((T + bt - 1) // bt) + 8
+        key = torch.randn((T, Hkv, D), generator=gen, device=dev).to(torch.bfloat16)
+        value = torch.randn((T, Hkv, D), generator=gen, device=dev).to(torch.bfloat16)
+        perm = torch.randperm(nb * bt, generator=gen, device=dev)[:T].to(torch.int64)
+        kc = torch.zeros((nb, bt, Hkv, D), dtype=torch.uint8, device=dev)
+        vc = torch.zeros_like(kc)
+        status = torch.zeros(1, dtype=torch.int32, device=dev)
+        bytes_per = T * Hkv * D * 6
+        f = lambda: fpd.fp8_paged_decode_cache_write(key, value, perm, kc, vc, 0.02, 0.01,
+                                                     status=status, stream=stream)
+        for _ in range(args.warmup):
+            f()
+        torch.cuda.synchronize()
+        K = max(3, min(args.steps, 2000))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        graph = None
+        if name == "decode_step":   # small: replay a graph of 100 calls
+            side = torch.cuda.Stream()
+            side.wait_stream(stream)
+            with torch.cuda.stream(side):
+                graph = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(graph, stream=side):
+                    for _ in range(100):
+                        fpd.fp8_paged_decode_cache_write(key, value, perm, kc, vc, 0.02, 0.01,
+                                                         status=status, stream=side)
+            stream.wait_stream(side)
+            K = max(1, K // 100)
+            graph.replay()
+        sampler = ClockSampler(0)
+        sampler.start()
+        time.sleep(0.25)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(K):
+            if graph is not None:
+                graph.replay()
+            else:
+                f()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        clocks = sampler.stop()
+        if graph is not None:
+            K *= 100
+            del graph
+        ms = e0.elapsed_time(e1) / K
+        assert int(status.item()) == 0
+        gbs = bytes_per / (ms / 1e3) / 1e9
+        res[name] = {"tokens": T, "us_per_call": ms * 1e3, "bytes_per_call": bytes_per,
+                     "GBps": gbs, "frac_of_peak": gbs / hbm, "calls": K, "clocks": clocks,
+                     "l2": "bytes per call larger than L2 (126 MiB)" if bytes_per > 126 * 2**20
+                           else "bytes per call smaller than L2 (latency case)"}
+    line = {"metric": "FP8 KV-cache write HBM GB/s (bf16 K/V in, E4M3 pages out)",
+            "value": res["prefill"]["GBps"], "unit": "GB/s", "n_gpus": 1,
+            "steps": res["prefill"]["calls"], "warmup": args.warmup,
+            "ms_per_step": res["prefill"]["us_per_call"] / 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16->e4m3 (f32 product)",
+            "data": "synthetic",
+            "config": {"workload": f"cache write, Hkv={Hkv} D={D} block_tokens={bt} "
+                                   f"({args.config} shape), shuffled slots", "tokens": args.write_tokens},
+            "roofline": {"bound": "hbm", "achieved": res["prefill"]["GBps"], "peak": hbm,
+                         "unit": "GB/s", "frac": res["prefill"]["frac_of_peak"], "traffic": None,
+                         "kernel": "fpd_cache_write_kernel", "peak_source": peak_src,
+                         "unit_bytes": "6 B per element (bf16 K and V read, E4M3 written)"},
+            "cases": res, "gpu_launches": res["prefill"]["calls"]}
+    print(json.dumps(line))
+    if args.json_out:
+        with open(args.json_out, "w") as fo:
+            json.dump(line, fo, indent=1)
+    return 0
+
+
 def main():
     args = parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
+    if args.op == "cache_write":
+        return run_cache_write(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_native(args)

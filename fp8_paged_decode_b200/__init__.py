@@ -32,6 +32,7 @@ __all__ = [
     "fp8_paged_decode_workspace_bytes_ex", "fp8_paged_decode_attention_profiled",
     "fp8_paged_decode_attention", "fp8_paged_decode_attention_ex",
     "fp8_paged_decode_check_status", "fp8_paged_decode_workspace_init",
+    "fp8_paged_decode_cache_write",
     "fp8_paged_decode_status_string", "fp8_paged_decode_version", "EXPORTED_SYMBOLS",
 ]
 
@@ -43,6 +44,7 @@ FPD_ERR_CUDA = 4
 FPD_DEVERR_SEQ_LEN = 0x1
 FPD_DEVERR_BLOCK_TABLE = 0x2
 FPD_DEVERR_TIMEOUT = 0x4
+FPD_DEVERR_SLOT = 0x8
 FPD_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -62,6 +64,7 @@ EXPORTED_SYMBOLS = (
     "fp8_paged_decode_attention_noalloc",
     "fp8_paged_decode_check_status",
     "fp8_paged_decode_workspace_init",
+    "fp8_paged_decode_cache_write",
     "fp8_paged_decode_status_string",
     "fp8_paged_decode_version",
 )
@@ -106,6 +109,9 @@ def _bind(lib):
     lib.fp8_paged_decode_attention_noalloc.restype = ci
     lib.fp8_paged_decode_check_status.argtypes = [vp, vp, ctypes.POINTER(ci), ci]
     lib.fp8_paged_decode_check_status.restype = ci
+    lib.fp8_paged_decode_cache_write.argtypes = [vp, vp, vp, ci, ci, ci, ctypes.c_int64,
+                                                 ctypes.c_int64, cf, cf, vp, vp, ci, ci, vp, vp]
+    lib.fp8_paged_decode_cache_write.restype = ci
     lib.fp8_paged_decode_workspace_init.argtypes = [vp, cz, vp]
     lib.fp8_paged_decode_workspace_init.restype = ci
     lib.fp8_paged_decode_status_string.argtypes = [ci]
@@ -256,6 +262,35 @@ def fp8_paged_decode_attention(q, k_cache, v_cache, block_table, seq_lens, k_sca
 
 
 fp8_paged_decode_attention_ex = fp8_paged_decode_attention
+
+
+def fp8_paged_decode_cache_write(key, value, slot_mapping, k_cache, v_cache, k_scale, v_scale,
+                                 status=None, stream=None):
+    """Enqueue the FP8 KV-cache write on ``stream``: bf16 ``key``/``value``
+    [num_tokens, Hkv, D] (rows contiguous; any token stride that is a multiple
+    of 8 elements) quantised with the per-tensor scales into ``k_cache``/
+    ``v_cache`` [num_blocks, block_tokens, Hkv, D] (uint8 or float8_e4m3fn) at
+    ``slot_mapping`` (int64 [num_tokens], negative = skip).  ``status``: an
+    optional int32 CUDA tensor whose first word receives FPD_DEVERR_SLOT."""
+    import torch
+    T, Hkv, D = key.shape
+    num_blocks, bt, Hkv2, D2 = k_cache.shape
+    if (Hkv2, D2) != (Hkv, D) or tuple(value.shape) != (T, Hkv, D):
+        raise ValueError("key/value and the caches disagree on (Hkv, D)")
+    for name, t in (("key", key), ("value", value)):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be a bf16 CUDA tensor")
+        if t.stride(2) != 1 or t.stride(1) != D:
+            raise ValueError(f"{name} rows must be contiguous ([num_tokens, Hkv, D], any token stride)")
+    kv_types = (torch.uint8, torch.float8_e4m3fn)
+    st = load_library().fp8_paged_decode_cache_write(
+        ctypes.c_void_p(key.data_ptr()), ctypes.c_void_p(value.data_ptr()),
+        _dev_ptr(slot_mapping, "slot_mapping", (torch.int64,), (T,)), T, Hkv, D,
+        key.stride(0), value.stride(0), float(k_scale), float(v_scale),
+        _dev_ptr(k_cache, "k_cache", kv_types),
+        _dev_ptr(v_cache, "v_cache", kv_types, tuple(k_cache.shape)), num_blocks, bt,
+        _dev_ptr(status, "status", (torch.int32,)), _stream_handle(stream))
+    _check(st, "fp8_paged_decode_cache_write")
 
 
 def fp8_paged_decode_check_status(workspace, stream=None, clear=False) -> int:

@@ -12,6 +12,7 @@
 #include <mutex>
 
 #include "fp8_paged_decode.h"
+#include "fpd_cache_write.cuh"
 #include "fpd_kernels.cuh"
 
 namespace {
@@ -136,22 +137,41 @@ bool current_device(int* dev) {
   return true;
 }
 
-// SM count of the current device and the number of split-kernel CTAs that fit
-// on one SM with `smem` bytes of dynamic shared memory (0 if none).
-bool device_occupancy(int D, int NT, int HB, int smem, int* num_sms, int* ctas_per_sm) {
-  int dev = 0;
-  if (!current_device(&dev)) return false;
-  std::lock_guard<std::mutex> lk(g_mu);
+// The per-device facts, queried on first use (call with g_mu held).
+DeviceInfo* device_info(int dev) {
   DeviceInfo& di = g_dev[dev];
   if (!di.ready) {
     if (cudaDeviceGetAttribute(&di.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&di.max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
             cudaSuccess) {
       cudaGetLastError();
-      return false;
+      return nullptr;
     }
     di.ready = true;
   }
+  return &di;
+}
+
+// SM count of the current device.
+bool device_sm_count(int* num_sms) {
+  int dev = 0;
+  if (!current_device(&dev)) return false;
+  std::lock_guard<std::mutex> lk(g_mu);
+  const DeviceInfo* di = device_info(dev);
+  if (!di) return false;
+  *num_sms = di->num_sms;
+  return true;
+}
+
+// SM count of the current device and the number of split-kernel CTAs that fit
+// on one SM with `smem` bytes of dynamic shared memory (0 if none).
+bool device_occupancy(int D, int NT, int HB, int smem, int* num_sms, int* ctas_per_sm) {
+  int dev = 0;
+  if (!current_device(&dev)) return false;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo* dip = device_info(dev);
+  if (!dip) return false;
+  DeviceInfo& di = *dip;
   *num_sms = di.num_sms;
   for (int i = 0; i < di.n_occ; ++i) {
     const OccEntry& e = di.occ[i];
@@ -607,6 +627,51 @@ fpd_status fp8_paged_decode_attention_noalloc(const void* q, const void* k_cache
   return attention_impl(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, D, num_blocks, bt,
                         max_blocks, k_scale, v_scale, sm_scale, window_left, sinks, out, lse,
                         scratch, FPD_NOALLOC_SCRATCH_BYTES, stream, 0, nullptr, nullptr, nullptr);
+}
+
+fpd_status fp8_paged_decode_cache_write(const void* key, const void* value,
+                                        const int64_t* slot_mapping, int num_tokens, int Hkv,
+                                        int D, int64_t key_stride, int64_t value_stride,
+                                        float k_scale, float v_scale, void* k_cache,
+                                        void* v_cache, int num_blocks, int block_tokens,
+                                        uint32_t* status, void* stream) {
+  if (num_tokens < 0 || Hkv <= 0 || D <= 0 || D % 16 != 0 || num_blocks <= 0 ||
+      block_tokens <= 0)
+    return FPD_ERR_INVALID_ARG;
+  if (!(k_scale > 0.f) || !(v_scale > 0.f) || !std::isfinite(k_scale) || !std::isfinite(v_scale))
+    return FPD_ERR_INVALID_ARG;
+  if (num_tokens == 0) return FPD_OK;
+  if (!key || !value || !slot_mapping || !k_cache || !v_cache) return FPD_ERR_INVALID_ARG;
+  const int64_t row = (int64_t)Hkv * D;
+  if (key_stride < row || value_stride < row || key_stride % 8 != 0 || value_stride % 8 != 0)
+    return FPD_ERR_INVALID_ARG;
+  if (!aligned(key, 16) || !aligned(value, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+      !aligned(slot_mapping, 8) || (status && !aligned(status, 4)))
+    return FPD_ERR_INVALID_ARG;
+  if (row / fpd::kWriteElems > INT32_MAX) return FPD_ERR_UNSUPPORTED;
+  fpd::CacheWriteParams p;
+  p.key = static_cast<const __nv_bfloat16*>(key);
+  p.value = static_cast<const __nv_bfloat16*>(value);
+  p.slot_mapping = slot_mapping;
+  p.k_cache = static_cast<uint8_t*>(k_cache);
+  p.v_cache = static_cast<uint8_t*>(v_cache);
+  p.status = status;
+  p.key_stride = key_stride;
+  p.value_stride = value_stride;
+  p.n_slots = (int64_t)num_blocks * block_tokens;
+  p.num_tokens = num_tokens;
+  p.row_chunks = (int)(row / fpd::kWriteElems);
+  p.k_inv = 1.0f / k_scale;   // fp32 reciprocal, as the reference writer takes it
+  p.v_inv = 1.0f / v_scale;
+  int sms = 0;
+  if (!device_sm_count(&sms)) return FPD_ERR_CUDA;
+  const int64_t units = (int64_t)num_tokens * 2 * p.row_chunks;
+  const int64_t want = (units + fpd::kWriteThreads - 1) / fpd::kWriteThreads;
+  const int64_t cap = (int64_t)sms * 8;   // 8 CTAs of 256 threads fill an SM
+  const int grid = (int)(want < cap ? want : cap);
+  fpd::fpd_cache_write_kernel<<<grid, fpd::kWriteThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      p);
+  return cudaGetLastError() == cudaSuccess ? FPD_OK : FPD_ERR_CUDA;
 }
 
 fpd_status fp8_paged_decode_check_status(void* workspace, void* stream, int* device_error_bits,

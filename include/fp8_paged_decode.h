@@ -60,6 +60,7 @@ typedef enum {
 #define FPD_DEVERR_SEQ_LEN 0x1u       /* a seq_lens entry was < 0 or > max_blocks * block_tokens (clamped) */
 #define FPD_DEVERR_BLOCK_TABLE 0x2u   /* a block-table entry in the attended range was outside [0, num_blocks) (read as zeros) */
 #define FPD_DEVERR_TIMEOUT 0x4u       /* a pipeline wait exceeded its time limit (results invalid) */
+#define FPD_DEVERR_SLOT 0x8u          /* cache write: a slot_mapping entry was >= num_blocks * block_tokens (token skipped) */
 
 /* Split plan chosen by the host planner; all fields are outputs. */
 typedef struct {
@@ -226,6 +227,36 @@ fpd_status fp8_paged_decode_attention_noalloc(const void *q, const void *k_cache
  * `stream`; clears it when `clear` is nonzero.  Writes the bits to
  * *device_error_bits.  Needs a workspace of at least 256 bytes.
  */
+/*
+ * FP8 KV-cache write: quantise the bf16 K and V rows of new tokens with the
+ * per-tensor scales and scatter them into the paged E4M3 caches.  The
+ * quantisation is the per-tensor form of the standalone cache-writer kernel in
+ * the NVFP4 KV-cache serving gist (writer kernel and host wrapper sections):
+ *   code = e4m3_rne_satfinite(float(x) * (1.0f / scale))
+ * with the reciprocal rounded to fp32 once and the product rounded to fp32;
+ * the E4M3 rounding is to nearest, ties to even, and saturates at +-448
+ * (infinities too; NaN stays NaN).
+ *   key, value    bf16 [num_tokens, Hkv, D]; token stride key_stride /
+ *                 value_stride elements (a multiple of 8; rows contiguous);
+ *                 16-byte aligned
+ *   slot_mapping  int64 [num_tokens]: slot = page * block_tokens + offset;
+ *                 negative = padded token, skipped.  Slots must be distinct
+ *                 (two tokens on one slot race).
+ *   k_cache, v_cache  e4m3 [num_blocks, block_tokens, Hkv, D] (16-byte
+ *                 aligned), written in place at the given slots only
+ *   status        optional device word (e.g. a decode workspace's status
+ *                 word) that receives FPD_DEVERR_SLOT for a slot past the
+ *                 end of the cache; that token is skipped.  NULL: no report.
+ * Requires D % 16 == 0, k_scale and v_scale finite and > 0.  Runs on `stream`,
+ * allocates nothing, never synchronises; num_tokens == 0 is a no-op.
+ */
+fpd_status fp8_paged_decode_cache_write(const void *key, const void *value,
+                                        const int64_t *slot_mapping, int num_tokens, int Hkv,
+                                        int D, int64_t key_stride, int64_t value_stride,
+                                        float k_scale, float v_scale, void *k_cache,
+                                        void *v_cache, int num_blocks, int block_tokens,
+                                        uint32_t *status, void *stream);
+
 fpd_status fp8_paged_decode_check_status(void *workspace, void *stream, int *device_error_bits,
                                          int clear);
 
