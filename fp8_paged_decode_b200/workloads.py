@@ -58,7 +58,7 @@ class Workload:
     block_tokens: int
     num_blocks: int
     max_blocks: int
-    q: np.ndarray            # uint16 [B, Hq, D]   (bf16 bit patterns)
+    q: np.ndarray            # uint16 [B, Hq, D], or [B, q_len, Hq, D] (bf16 bit patterns)
     k_cache: np.ndarray      # uint8  [num_blocks, block_tokens, Hkv, D]
     v_cache: np.ndarray      # uint8  [num_blocks, block_tokens, Hkv, D]
     block_table: np.ndarray  # int32  [B, max_blocks]
@@ -72,16 +72,18 @@ class Workload:
     # kept only when requested (small cases) for brute-force checks.
     k_dense: Optional[List[np.ndarray]] = None
     v_dense: Optional[List[np.ndarray]] = None
+    # Query tokens per sequence (the newest q_len positions, causal).
+    q_len: int = 1
 
     @property
     def groups(self) -> int:
         return self.Hq // self.Hkv
 
     def attended(self) -> np.ndarray:
-        """Number of keys each sequence attends (window-capped)."""
+        """Number of keys each sequence's queries attend together (window-capped)."""
         L = self.seq_lens.astype(np.int64)
         if self.window_left >= 0:
-            return np.minimum(L, self.window_left + 1)
+            return np.minimum(L, self.window_left + self.q_len)
         return L
 
     def kv_bytes(self) -> int:
@@ -172,8 +174,10 @@ def make_custom(*, B: int, Hq: int, Hkv: int, D: int, block_tokens: int,
                 sm_scale: Optional[float] = None, sigma: float = 1.0, seed: int = 0,
                 spare_blocks: int = 16, max_blocks: Optional[int] = None,
                 fill: str = "nan", keep_dense: bool = False, name: str = "custom",
-                q_sigma: float = 1.0, sink_sigma: float = 1.0) -> Workload:
-    """Build one decode step of the given shape (see module docstring)."""
+                q_sigma: float = 1.0, sink_sigma: float = 1.0, q_len: int = 1) -> Workload:
+    """Build one decode step of the given shape (see module docstring).  With
+    q_len > 1 each sequence has q_len query tokens (q is [B, q_len, Hq, D]) and
+    the stored range covers every query's window."""
     assert Hq % Hkv == 0 and fill in ("nan", "data")
     lens = np.asarray(seq_lens, dtype=np.int64)
     assert lens.shape == (B,) and (lens >= 0).all()
@@ -194,12 +198,16 @@ def make_custom(*, B: int, Hq: int, Hkv: int, D: int, block_tokens: int,
         table[b, :pages[b]] = perm[off:off + pages[b]]
         off += int(pages[b])
 
-    q = _to_bf16_bits(_normal_f32(s_q, B * Hq * D, q_sigma).reshape(B, Hq, D))
+    assert q_len >= 1
+    if q_len == 1:
+        q = _to_bf16_bits(_normal_f32(s_q, B * Hq * D, q_sigma).reshape(B, Hq, D))
+    else:
+        q = _to_bf16_bits(_normal_f32(s_q, B * q_len * Hq * D, q_sigma).reshape(B, q_len, Hq, D))
     if sm_scale is None:
         sm_scale = 1.0 / math.sqrt(D)
 
     W = window_left
-    starts = np.maximum(0, lens - 1 - W) if W >= 0 else np.zeros_like(lens)
+    starts = np.maximum(0, lens - q_len - W) if W >= 0 else np.zeros_like(lens)
     n_att = lens - starts
     tot = int(n_att.sum())
     row = Hkv * D
@@ -246,7 +254,8 @@ def make_custom(*, B: int, Hq: int, Hkv: int, D: int, block_tokens: int,
                     num_blocks=num_blocks, max_blocks=max_blocks, q=q, k_cache=k_cache,
                     v_cache=v_cache, block_table=table, seq_lens=lens.astype(np.int32),
                     k_scale=k_scale, v_scale=v_scale, sm_scale=float(np.float32(sm_scale)),
-                    window_left=int(W), sinks=sinks_arr, k_dense=k_dense, v_dense=v_dense)
+                    window_left=int(W), sinks=sinks_arr, k_dense=k_dense, v_dense=v_dense,
+                    q_len=int(q_len))
 
 
 def make_workload(name: str, *, seed: Optional[int] = None, fill: str = "nan",

@@ -44,6 +44,9 @@ def _bind(lib):
     lib.fpd_oracle_decode.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci,
                                       cd, cd, cd, ci, vp, vp, vp, vp, ci, ci]
     lib.fpd_oracle_decode.restype = ci
+    lib.fpd_oracle_decode_q.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, ci,
+                                        cd, cd, cd, ci, vp, vp, vp, vp, ci, ci]
+    lib.fpd_oracle_decode_q.restype = ci
     lib.fpd_oracle_f64_to_e4m3.argtypes = [ctypes.c_double]
     lib.fpd_oracle_f64_to_e4m3.restype = ctypes.c_uint8
     lib.fpd_oracle_cache_write.argtypes = [vp, vp, vp, ci, ci, ci, ctypes.c_long, ctypes.c_long,
@@ -114,11 +117,13 @@ def decode(q, k_cache, v_cache, block_table, seq_lens, *, k_scale, v_scale, sm_s
            ) -> Tuple[np.ndarray, np.ndarray]:
     """fp64 decode attention.
 
-    Arrays are numpy: q uint16 (bf16 bits) [B,Hq,D]; k/v_cache uint8 E4M3 codes
-    [num_blocks, bt, Hkv, D]; block_table int32 [B, max_blocks]; seq_lens int32
-    [B]; sinks float32 [Hq] or None.  ``rows`` optionally lists flat
-    ``b * Hq + h`` rows to compute (others are left NaN).  Returns
-    (out float64 [B, Hq, D], lse float64 [B, Hq]).
+    Arrays are numpy: q uint16 (bf16 bits) [B,Hq,D], or [B,q_len,Hq,D] for
+    q_len query tokens per sequence (positions L - q_len .. L - 1, causal);
+    k/v_cache uint8 E4M3 codes [num_blocks, bt, Hkv, D]; block_table int32
+    [B, max_blocks]; seq_lens int32 [B]; sinks float32 [Hq] or None.  ``rows``
+    optionally lists flat ``(b * q_len + i) * Hq + h`` rows to compute (others
+    are left NaN).  Returns (out float64 [B, (q_len,) Hq, D], lse float64
+    [B, (q_len,) Hq]) with q's leading shape.
     """
     lib = lib or load()
     q = np.ascontiguousarray(q, dtype=np.uint16)
@@ -126,7 +131,12 @@ def decode(q, k_cache, v_cache, block_table, seq_lens, *, k_scale, v_scale, sm_s
     v_cache = np.ascontiguousarray(v_cache, dtype=np.uint8)
     block_table = np.ascontiguousarray(block_table, dtype=np.int32)
     seq_lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
-    B, Hq, D = q.shape
+    lead = q.shape[:-2]
+    if q.ndim == 3:
+        B, Hq, D = q.shape
+        Q = 1
+    else:
+        B, Q, Hq, D = q.shape
     num_blocks, bt, Hkv, D2 = k_cache.shape
     assert D2 == D and v_cache.shape == k_cache.shape
     assert block_table.shape[0] == B and seq_lens.shape == (B,)
@@ -134,8 +144,8 @@ def decode(q, k_cache, v_cache, block_table, seq_lens, *, k_scale, v_scale, sm_s
     if sinks is not None:
         sinks = np.ascontiguousarray(sinks, dtype=np.float32)
         assert sinks.shape == (Hq,)
-    out = np.full((B, Hq, D), np.nan, dtype=np.float64)
-    lse = np.full((B, Hq), np.nan, dtype=np.float64)
+    out = np.full(lead + (Hq, D), np.nan, dtype=np.float64)
+    lse = np.full(lead + (Hq,), np.nan, dtype=np.float64)
     rows_arr = None
     n_rows = 0
     if rows is not None:
@@ -143,11 +153,11 @@ def decode(q, k_cache, v_cache, block_table, seq_lens, *, k_scale, v_scale, sm_s
         n_rows = int(rows_arr.size)
     if threads is None:
         threads = os.cpu_count() or 1
-    st = lib.fpd_oracle_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
-                               _ptr(seq_lens), B, Hq, Hkv, D, num_blocks, bt, max_blocks,
-                               float(k_scale), float(v_scale), float(sm_scale), int(window_left),
-                               _ptr(sinks), _ptr(out), _ptr(lse), _ptr(rows_arr), n_rows,
-                               int(threads))
+    st = lib.fpd_oracle_decode_q(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                                 _ptr(seq_lens), B, Q, Hq, Hkv, D, num_blocks, bt, max_blocks,
+                                 float(k_scale), float(v_scale), float(sm_scale),
+                                 int(window_left), _ptr(sinks), _ptr(out), _ptr(lse),
+                                 _ptr(rows_arr), n_rows, int(threads))
     if st != 0:
         raise ValueError(f"oracle rejected the inputs (status {st})")
     return out, lse

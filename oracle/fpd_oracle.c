@@ -40,6 +40,12 @@
  * The file also holds the oracle of the FP8 cache write that fills such a
  * cache (fpd_oracle_cache_write, below the E4M3 codec).
  *
+ * Several query tokens per sequence (speculative / multi-token decode): the
+ * sequence's q_len newest tokens are queries.  Query i (0 <= i < q_len) sits at
+ * position p = L - q_len + i and sees the keys j in [start_i, p] (causal), with
+ * start_i = max(0, p - window_left) under a window; q, out and lse gain a
+ * q_len axis after B.  q_len = 1 is the formula above.
+ *
  * Degenerate cases: L == 0 gives out = 0 and lse = sigma (-inf without sinks).
  * A stored NaN code inside the attended range propagates NaN (plain
  * arithmetic); codes outside the attended range are never read.
@@ -151,12 +157,12 @@ typedef struct {
     const uint16_t *q;
     const uint8_t *k_cache, *v_cache;
     const int32_t *block_table, *seq_lens;
-    int B, Hq, Hkv, D, num_blocks, bt, max_blocks;
+    int B, Hq, Hkv, D, num_blocks, bt, max_blocks, q_len;
     double k_scale, v_scale, sm_scale;
     int window_left;
     const float *sinks;
     double *out, *lse;
-    const int32_t *rows; /* list of b * Hq + h to compute, or NULL for all */
+    const int32_t *rows; /* list of (b * q_len + i) * Hq + h to compute, or NULL for all */
     int n_rows;
     int next;            /* work counter */
     int status;
@@ -171,7 +177,8 @@ static size_t cache_row(const job_t *J, int page, int slot, int kvh)
 
 static int one_row(const job_t *J, int row, double *s, double *acc)
 {
-    const int b = row / J->Hq, h = row % J->Hq;
+    const int Q = J->q_len;
+    const int b = row / (Q * J->Hq), i = (row / J->Hq) % Q, h = row % J->Hq;
     const int g = J->Hq / J->Hkv;
     const int kvh = h / g;
     const int D = J->D;
@@ -179,18 +186,20 @@ static int one_row(const job_t *J, int row, double *s, double *acc)
     double *o = J->out + (size_t)row * D;
     const uint16_t *qr = J->q + (size_t)row * D;
     const double sigma = J->sinks ? (double)J->sinks[h] : -INFINITY;
-    int start, j, d;
+    int p, start, end, j, d;
     double m, Z;
 
     if (L < 0 || L > J->max_blocks * J->bt)
         return -2;
-    start = (J->window_left >= 0) ? L - 1 - J->window_left : 0;
+    p = L - Q + i;              /* the query's own position; it sees keys up to p */
+    end = p + 1 > 0 ? p + 1 : 0;
+    start = (J->window_left >= 0) ? p - J->window_left : 0;
     if (start < 0)
         start = 0;
 
     /* logits */
     m = sigma;
-    for (j = start; j < L; ++j) {
+    for (j = start; j < end; ++j) {
         const int page = J->block_table[(size_t)b * J->max_blocks + j / J->bt];
         const uint8_t *kr;
         double dot = 0.0;
@@ -214,7 +223,7 @@ static int one_row(const job_t *J, int row, double *s, double *acc)
         J->lse[row] = -INFINITY;
         return 0;
     }
-    for (j = start; j < L; ++j) {
+    for (j = start; j < end; ++j) {
         const int page = J->block_table[(size_t)b * J->max_blocks + j / J->bt];
         const uint8_t *vr = J->v_cache + cache_row(J, page, j % J->bt, kvh);
         const double p = exp(s[j - start] - m);
@@ -232,7 +241,7 @@ static int one_row(const job_t *J, int row, double *s, double *acc)
 static void *worker(void *arg)
 {
     job_t *J = (job_t *)arg;
-    const int total = J->rows ? J->n_rows : J->B * J->Hq;
+    const int total = J->rows ? J->n_rows : J->B * J->q_len * J->Hq;
     int maxL = J->max_blocks * J->bt;
     double *s = (double *)malloc(sizeof(double) * (size_t)(maxL > 0 ? maxL : 1));
     double *acc = (double *)malloc(sizeof(double) * (size_t)J->D);
@@ -258,41 +267,41 @@ static void *worker(void *arg)
 }
 
 /*
- * Decode attention over the paged cache.
- *   q            bf16 bits [B, Hq, D]
+ * Decode attention over the paged cache, q_len query tokens per sequence.
+ *   q            bf16 bits [B, q_len, Hq, D]
  *   k/v_cache    E4M3 codes [num_blocks, bt, Hkv, D]
- *   block_table  [B, max_blocks], seq_lens [B]
+ *   block_table  [B, max_blocks], seq_lens [B] (including the q_len new tokens)
  *   sinks        float [Hq] or NULL
- *   out          double [B * Hq, D]  (only the listed rows are written)
- *   lse          double [B * Hq]
- *   rows/n_rows  rows (b * Hq + h) to compute; rows == NULL computes all.
+ *   out          double [B * q_len * Hq, D]  (only the listed rows are written)
+ *   lse          double [B * q_len * Hq]
+ *   rows/n_rows  rows ((b * q_len + i) * Hq + h) to compute; NULL computes all.
  *   n_threads    worker threads (<= 0: 1)
  * Returns 0, -1 for bad shapes, -2 for a sequence length outside
  * [0, max_blocks * bt], -3 for a block-table entry outside [0, num_blocks).
  */
-int fpd_oracle_decode(const uint16_t *q, const uint8_t *k_cache, const uint8_t *v_cache,
-                      const int32_t *block_table, const int32_t *seq_lens,
-                      int B, int Hq, int Hkv, int D, int num_blocks, int bt, int max_blocks,
-                      double k_scale, double v_scale, double sm_scale, int window_left,
-                      const float *sinks, double *out, double *lse,
-                      const int32_t *rows, int n_rows, int n_threads)
+int fpd_oracle_decode_q(const uint16_t *q, const uint8_t *k_cache, const uint8_t *v_cache,
+                        const int32_t *block_table, const int32_t *seq_lens,
+                        int B, int q_len, int Hq, int Hkv, int D, int num_blocks, int bt,
+                        int max_blocks, double k_scale, double v_scale, double sm_scale,
+                        int window_left, const float *sinks, double *out, double *lse,
+                        const int32_t *rows, int n_rows, int n_threads)
 {
     job_t J;
     pthread_t *th;
     int t, i;
-    if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || D <= 0 || bt <= 0 || max_blocks < 0 ||
-        num_blocks < 0)
+    if (B < 0 || q_len < 1 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || D <= 0 || bt <= 0 ||
+        max_blocks < 0 || num_blocks < 0)
         return -1;
     if (rows) {
         for (i = 0; i < n_rows; ++i)
-            if (rows[i] < 0 || rows[i] >= B * Hq)
+            if (rows[i] < 0 || rows[i] >= B * q_len * Hq)
                 return -1;
     }
     memset(&J, 0, sizeof J);
     J.q = q; J.k_cache = k_cache; J.v_cache = v_cache;
     J.block_table = block_table; J.seq_lens = seq_lens;
     J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.D = D; J.num_blocks = num_blocks; J.bt = bt;
-    J.max_blocks = max_blocks;
+    J.max_blocks = max_blocks; J.q_len = q_len;
     J.k_scale = k_scale; J.v_scale = v_scale; J.sm_scale = sm_scale;
     J.window_left = window_left; J.sinks = sinks; J.out = out; J.lse = lse;
     J.rows = rows; J.n_rows = n_rows;
@@ -307,4 +316,17 @@ int fpd_oracle_decode(const uint16_t *q, const uint8_t *k_cache, const uint8_t *
     free(th);
     pthread_mutex_destroy(&J.mu);
     return J.status;
+}
+
+/* One query token per sequence: q bf16 bits [B, Hq, D]. */
+int fpd_oracle_decode(const uint16_t *q, const uint8_t *k_cache, const uint8_t *v_cache,
+                      const int32_t *block_table, const int32_t *seq_lens,
+                      int B, int Hq, int Hkv, int D, int num_blocks, int bt, int max_blocks,
+                      double k_scale, double v_scale, double sm_scale, int window_left,
+                      const float *sinks, double *out, double *lse,
+                      const int32_t *rows, int n_rows, int n_threads)
+{
+    return fpd_oracle_decode_q(q, k_cache, v_cache, block_table, seq_lens, B, 1, Hq, Hkv, D,
+                               num_blocks, bt, max_blocks, k_scale, v_scale, sm_scale,
+                               window_left, sinks, out, lse, rows, n_rows, n_threads);
 }

@@ -279,6 +279,74 @@ def pin_softmax_identity(lib):
             assert abs(tot - 1.0) < 1e-12, f"probabilities sum to {tot}"
 
 
+# ----------------------------------------------------- several query tokens --
+
+def pin_multi_token_library(lib):
+    """q_len queries per sequence against torch SDPA (float64, an explicit
+    causal + window mask, the sink as an extra zero-valued key) and scipy
+    logsumexp."""
+    for Q, window in ((3, -1), (4, 20), (2, 0)):
+        wl = W.make_custom(B=3, Hq=8, Hkv=2, D=64, block_tokens=16, seq_lens=[Q, 37, 90],
+                           sinks=True, window_left=window, seed=51 + Q, sm_scale=0.2,
+                           keep_dense=True, q_len=Q)
+        q = wl.q
+        out, lse = oracle.decode(q, wl.k_cache, wl.v_cache, wl.block_table, wl.seq_lens,
+                                 k_scale=wl.k_scale, v_scale=wl.v_scale, sm_scale=wl.sm_scale,
+                                 window_left=window, sinks=wl.sinks, lib=lib, threads=2)
+        qf = bf16_library(q)
+        g = wl.Hq // wl.Hkv
+        sig = wl.sinks.astype(np.float64)
+        for b in range(wl.B):
+            L = int(wl.seq_lens[b])
+            s0 = max(0, L - Q - window) if window >= 0 else 0   # first key any query sees
+            n = L - s0
+            K = e4m3_library(wl.k_dense[b][s0:L]) * wl.k_scale
+            V = e4m3_library(wl.v_dense[b][s0:L]) * wl.v_scale
+            Kt = torch.zeros((1, wl.Hkv, n + 1, wl.D), dtype=torch.float64)
+            Vt = torch.zeros_like(Kt)
+            Kt[0, :, :n] = torch.from_numpy(K).permute(1, 0, 2)
+            Vt[0, :, :n] = torch.from_numpy(V).permute(1, 0, 2)
+            mask = torch.full((1, wl.Hq, Q, n + 1), -math.inf, dtype=torch.float64)
+            for i in range(Q):
+                p = L - Q + i
+                lo = max(0, p - window) if window >= 0 else 0
+                mask[0, :, i, lo - s0:p + 1 - s0] = 0.0
+            mask[0, :, :, n] = torch.from_numpy(sig)[:, None]
+            qt = torch.from_numpy(qf[b]).permute(1, 0, 2).unsqueeze(0)   # [1, Hq, Q, D]
+            o = F.scaled_dot_product_attention(qt, Kt, Vt, attn_mask=mask, scale=wl.sm_scale,
+                                               enable_gqa=True)
+            close(out[b], o[0].permute(1, 0, 2).numpy(), rtol=1e-10, atol=1e-12,
+                  what=f"multi-token out (Q={Q}, window {window})")
+            Kh = np.repeat(K, g, axis=1)
+            sc = wl.sm_scale * np.einsum("ihd,nhd->ihn", qf[b], Kh)
+            sc = np.where(mask[0, :, :, :n].permute(1, 0, 2).numpy() == 0, sc, -np.inf)
+            sc = np.concatenate([sc, np.broadcast_to(sig[None, :, None], (Q, wl.Hq, 1))], axis=2)
+            close(lse[b], scipy.special.logsumexp(sc, axis=2), rtol=1e-12, atol=1e-12,
+                  what="multi-token lse")
+
+
+def pin_multi_token_prefix(lib):
+    """Query i of q_len equals a one-query decode of the sequence cut after
+    position L - q_len + i (what a causal query sees), with and without a
+    window."""
+    for window in (-1, 7):
+        Q = 5
+        wl = W.make_custom(B=2, Hq=4, Hkv=4, D=128, block_tokens=32, seq_lens=[50, 200],
+                           sinks=False, window_left=window, seed=53, sm_scale=0.1, q_len=Q)
+        q = wl.q
+        out, lse = oracle.decode(q, wl.k_cache, wl.v_cache, wl.block_table, wl.seq_lens,
+                                 k_scale=wl.k_scale, v_scale=wl.v_scale, sm_scale=wl.sm_scale,
+                                 window_left=window, lib=lib, threads=2)
+        for i in range(Q):
+            lens = wl.seq_lens - Q + i + 1
+            o1, l1 = oracle.decode(np.ascontiguousarray(q[:, i]), wl.k_cache, wl.v_cache,
+                                   wl.block_table, lens, k_scale=wl.k_scale,
+                                   v_scale=wl.v_scale, sm_scale=wl.sm_scale,
+                                   window_left=window, lib=lib, threads=2)
+            assert np.array_equal(out[:, i], o1) and np.array_equal(lse[:, i], l1), \
+                f"query {i} differs from the truncated single-query decode"
+
+
 # ------------------------------------------------------------ cache write --
 
 def e4m3_encode_library(x: np.ndarray) -> np.ndarray:
@@ -399,4 +467,5 @@ def pin_cache_write_invariants(lib):
 
 ALL_PINS = [pin_e4m3_codes, pin_bf16, pin_library_attention, pin_zero_keys, pin_window_zero,
             pin_constant_values, pin_invariants, pin_softmax_identity, pin_e4m3_encode_library,
-            pin_e4m3_encode_closed, pin_cache_write_library, pin_cache_write_invariants]
+            pin_e4m3_encode_closed, pin_cache_write_library, pin_cache_write_invariants,
+            pin_multi_token_library, pin_multi_token_prefix]

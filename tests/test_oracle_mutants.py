@@ -17,7 +17,9 @@ SRC = os.path.join(os.path.dirname(oracle.__file__), "fpd_oracle.c")
 MUTANTS = {
     "sink dropped from denominator": [("    Z += exp(sigma - m);\n", "")],
     "GQA head mapping h % Hkv": [("const int kvh = h / g;", "const int kvh = h % J->Hkv;")],
-    "window start off by one": [("L - 1 - J->window_left", "L - J->window_left")],
+    "window start off by one": [("p - J->window_left", "p + 1 - J->window_left")],
+    "queries not causal (all see the whole sequence)": [("p = L - Q + i;", "p = L - 1;")],
+    "query positions reversed": [("p = L - Q + i;", "p = L - 1 - i;")],
     "E4M3 exponent bias 8": [("expo - 7", "expo - 8")],
     "E4M3 subnormal exponent": [("(double)mant / 8.0, -6)", "(double)mant / 8.0, -7)")],
     "E4M3 mantissa step": [("1.0 + (double)mant / 8.0", "1.0 + (double)mant / 16.0")],
@@ -57,9 +59,9 @@ MUTANTS = {
          "const size_t dst = (((size_t)(slot / bt) * Hkv + h) * bt + slot % bt) * (size_t)D + d;")],
     "writer value read with the key stride": [("value[t * value_stride + (long)h * D + d]",
                                                "value[t * key_stride + (long)h * D + d]")],
-    "last key dropped": [("for (j = start; j < L; ++j) {\n        const int page = J->block_table"
+    "last key dropped": [("for (j = start; j < end; ++j) {\n        const int page = J->block_table"
                           "[(size_t)b * J->max_blocks + j / J->bt];\n        const uint8_t *vr",
-                          "for (j = start; j < L - 1; ++j) {\n        const int page = J->block_table"
+                          "for (j = start; j < end - 1; ++j) {\n        const int page = J->block_table"
                           "[(size_t)b * J->max_blocks + j / J->bt];\n        const uint8_t *vr")],
 }
 
