@@ -66,6 +66,8 @@ def parse_args():
                     help="only run warm-up + K plain calls (for ncu launch lists and captures)")
     ap.add_argument("--json-out", default=None)
     ap.add_argument("--op", default="decode", choices=["decode", "cache_write"])
+    ap.add_argument("--q-len", type=int, default=1,
+                    help="query tokens per sequence (speculative decode of the same workload)")
     ap.add_argument("--write-tokens", type=int, default=65536)
     return ap.parse_args()
 
@@ -220,6 +222,15 @@ class RawEvents:
 
 # ------------------------------------------------------------ CPU oracle --
 
+def rows_kv_bytes(wl, rows):
+    """The workload's algorithmic KV bytes that the given output rows stand
+    for: a sequence's K+V bytes are shared by its q_len * Hq rows, so each row
+    is credited with that share (the metric counts each KV byte once)."""
+    att = wl.attended()
+    per_seq = wl.q_len * wl.Hq
+    return sum(int(att[int(r) // per_seq]) for r in rows) * wl.Hkv * wl.D * 2 / per_seq
+
+
 def oracle_sample(wl, budget_s, rng_seed=0, threads=None, min_rows=1):
     """Run the oracle on random (sequence, head) rows until about budget_s of
     wall time is spent; returns (seconds, kv_bytes_read, rows, threads)."""
@@ -227,8 +238,7 @@ def oracle_sample(wl, budget_s, rng_seed=0, threads=None, min_rows=1):
     import oracle
     threads = threads or (os.cpu_count() or 1)
     rng = np.random.default_rng(rng_seed)
-    order = rng.permutation(wl.B * wl.Hq)
-    att = wl.attended()
+    order = rng.permutation(wl.B * wl.q_len * wl.Hq)
     # calibrate on a few rows
     probe = order[:max(min_rows, min(len(order), threads))]
     t0 = time.perf_counter()
@@ -240,8 +250,7 @@ def oracle_sample(wl, budget_s, rng_seed=0, threads=None, min_rows=1):
     t0 = time.perf_counter()
     oracle.decode_workload(wl, rows=rows, threads=threads)
     dt = time.perf_counter() - t0
-    kv = int(sum(int(att[r // wl.Hq]) for r in rows)) * wl.D * 2
-    return dt, kv, n, threads
+    return dt, rows_kv_bytes(wl, rows), n, threads
 
 
 def run_reference(args):
@@ -253,37 +262,38 @@ def run_reference(args):
     import numpy as np
     from fp8_paged_decode_b200 import workloads as W
     import oracle
-    wl = W.make_workload(args.config)
+    wl = W.make_workload(args.config, q_len=args.q_len)
     threads = os.cpu_count() or 1
     total_steps = args.steps + args.warmup
     budget_s = 120.0
     # calibrate: wall time of one parallel batch of `threads` rows
-    probe = np.arange(min(wl.B * wl.Hq, threads))
+    n_rows = wl.B * wl.q_len * wl.Hq
+    probe = np.arange(min(n_rows, threads))
     t0 = time.perf_counter()
     oracle.decode_workload(wl, rows=probe, threads=threads)
     per_row_wall = (time.perf_counter() - t0) / len(probe)
     rows_per_step = int(budget_s / total_steps / max(per_row_wall, 1e-7))
-    rows_per_step = max(1, min(rows_per_step, wl.B * wl.Hq))
+    rows_per_step = max(1, min(rows_per_step, n_rows))
     rng = np.random.default_rng(7)
-    att = wl.attended()
     t_sum, kv_sum = 0.0, 0
     for step in range(total_steps):
-        rows = rng.choice(wl.B * wl.Hq, size=rows_per_step, replace=False)
+        rows = rng.choice(n_rows, size=rows_per_step, replace=False)
         t0 = time.perf_counter()
         oracle.decode_workload(wl, rows=rows, threads=min(threads, rows_per_step))
         dt = time.perf_counter() - t0
         if step >= args.warmup:
             t_sum += dt
-            kv_sum += int(sum(int(att[r // wl.Hq]) for r in rows)) * wl.D * 2
+            kv_sum += rows_kv_bytes(wl, rows)
     value = kv_sum / t_sum / 1e9
     hbm, _ = measured_peaks()
-    sample = f"{rows_per_step} random (sequence, head) rows of the workload per step"
+    sample = (f"{rows_per_step} random (sequence, query token, head) rows of the workload per "
+              f"step, each credited with its share of the sequence's KV bytes")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": t_sum / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": W.describe(args.config), "sample": sample},
+        "config": {"workload": W.describe(args.config), "q_len": wl.q_len, "sample": sample},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": min(threads, rows_per_step),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -318,7 +328,7 @@ def run_native(args):
             dist.barrier()
 
     lib = fpd.load_library()
-    wl = W.make_workload(args.config)
+    wl = W.make_workload(args.config, q_len=args.q_len)
     dev = torch.device("cuda", local)
     props = torch.cuda.get_device_properties(dev)
     l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20))
@@ -331,21 +341,23 @@ def run_native(args):
     sinks = None if wl.sinks is None else torch.from_numpy(wl.sinks).to(dev)
     kc = [torch.from_numpy(wl.k_cache).to(dev) for _ in range(replicas)]
     vc = [torch.from_numpy(wl.v_cache).to(dev) for _ in range(replicas)]
-    out = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.bfloat16, device=dev)
-    lse = torch.empty((wl.B, wl.Hq), dtype=torch.float32, device=dev)
-    need = fpd.fp8_paged_decode_workspace_bytes_ex(wl.B, wl.Hq, wl.Hkv, wl.D, wl.block_tokens,
-                                                   wl.max_blocks, wl.window_left, args.chunk_pages)
+    lead = tuple(wl.q.shape[:-2])   # (B,) or (B, q_len)
+    out = torch.empty(lead + (wl.Hq, wl.D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(lead + (wl.Hq,), dtype=torch.float32, device=dev)
+    need = fpd.fp8_paged_decode_workspace_bytes_qlen(wl.B, wl.q_len, wl.Hq, wl.Hkv, wl.D,
+                                                     wl.block_tokens, wl.max_blocks,
+                                                     wl.window_left, args.chunk_pages)
     assert need > 0
     wsp = torch.zeros(need, dtype=torch.uint8, device=dev)
-    plan = fpd.fp8_paged_decode_plan(wl.B, wl.Hq, wl.Hkv, wl.D, wl.block_tokens, wl.max_blocks,
-                                     wl.window_left, args.chunk_pages)
+    plan = fpd.fp8_paged_decode_plan_qlen(wl.B, wl.q_len, wl.Hq, wl.Hkv, wl.D, wl.block_tokens,
+                                          wl.max_blocks, wl.window_left, args.chunk_pages)
     stream = torch.cuda.current_stream(dev)
     sh = ctypes.c_void_p(stream.cuda_stream)
     vp = ctypes.c_void_p
 
     def call_args(i):
         return [vp(q.data_ptr()), vp(kc[i].data_ptr()), vp(vc[i].data_ptr()), vp(table.data_ptr()),
-                vp(lens.data_ptr()), wl.B, wl.Hq, wl.Hkv, wl.D, wl.num_blocks, wl.block_tokens,
+                vp(lens.data_ptr()), wl.B, wl.q_len, wl.Hq, wl.Hkv, wl.D, wl.num_blocks, wl.block_tokens,
                 wl.max_blocks, ctypes.c_float(wl.k_scale), ctypes.c_float(wl.v_scale),
                 ctypes.c_float(wl.sm_scale), wl.window_left,
                 vp(sinks.data_ptr()) if sinks is not None else None, vp(out.data_ptr()),
@@ -354,7 +366,7 @@ def run_native(args):
 
     pre = [call_args(i) for i in range(replicas)]
     f_prof = lib.fp8_paged_decode_attention_profiled
-    f_plain = lib.fp8_paged_decode_attention_ex
+    f_plain = lib.fp8_paged_decode_attention_qlen
 
     if args.kernels_only:
         for i in range(args.warmup + args.steps):
@@ -379,16 +391,19 @@ def run_native(args):
     if rank == 0:
         import oracle
         rng = np.random.default_rng(0)
-        rows = rng.choice(wl.B * wl.Hq, size=min(16, wl.B * wl.Hq), replace=False)
+        n_rows = wl.B * wl.q_len * wl.Hq
+        rows = rng.choice(n_rows, size=min(16, n_rows), replace=False)
         ro, rl = oracle.decode_workload(wl, rows=rows)
-        o = out.float().cpu().numpy()
-        l = lse.cpu().numpy()
-        b, h = np.divmod(rows, wl.Hq)
-        err = np.abs(o[b, h] - ro[b, h])
-        ok = bool((err <= 1e-2 + 1e-2 * np.abs(ro[b, h])).all() and
-                  (np.abs(l[b, h] - rl[b, h]) <= 1e-3).all())
+        # rows index (sequence, query token, head) in that order
+        o = out.float().cpu().numpy().reshape(n_rows, wl.D)
+        l = lse.cpu().numpy().reshape(n_rows)
+        ro = ro.reshape(n_rows, wl.D)
+        rl = rl.reshape(n_rows)
+        err = np.abs(o[rows] - ro[rows])
+        ok = bool((err <= 1e-2 + 1e-2 * np.abs(ro[rows])).all() and
+                  (np.abs(l[rows] - rl[rows]) <= 1e-3).all())
         guard = {"rows_checked": int(len(rows)), "max_abs_dout": float(err.max()),
-                 "max_abs_dlse": float(np.abs(l[b, h] - rl[b, h]).max()), "ok": ok}
+                 "max_abs_dlse": float(np.abs(l[rows] - rl[rows]).max()), "ok": ok}
         assert ok, guard
     bits = fpd.fp8_paged_decode_check_status(wsp, clear=True)
     assert bits == 0, f"device status {bits}"
@@ -447,8 +462,8 @@ def run_native(args):
         htab = torch.from_numpy(wl.block_table).pin_memory()
         hlen = torch.from_numpy(wl.seq_lens).pin_memory()
         hsink = None if wl.sinks is None else torch.from_numpy(wl.sinks).pin_memory()
-        hout = torch.empty((wl.B, wl.Hq, wl.D), dtype=torch.bfloat16).pin_memory()
-        hlse = torch.empty((wl.B, wl.Hq), dtype=torch.float32).pin_memory()
+        hout = torch.empty(lead + (wl.Hq, wl.D), dtype=torch.bfloat16).pin_memory()
+        hlse = torch.empty(lead + (wl.Hq,), dtype=torch.float32).pin_memory()
         h2d = hq.numel() * 2 + htab.numel() * 4 + hlen.numel() * 4 + (
             hsink.numel() * 4 if hsink is not None else 0)
         d2h = hout.numel() * 2 + hlse.numel() * 4
@@ -500,8 +515,9 @@ def run_native(args):
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         dt, kvb, nrows, thr = oracle_sample(wl, args.cpu_seconds)
         cpu = {"value": kvb / dt / 1e9, "unit": UNIT, "cores": thr, "kind": "oracle",
-               "sample": f"{nrows} random (sequence, head) rows of the workload, "
-                         f"{kvb} KV bytes, {dt:.1f} s wall"}
+               "sample": f"{nrows} random (sequence, query token, head) rows of the workload, "
+                         f"{kvb:.0f} KV bytes (each row's share of its sequence), "
+                         f"{dt:.1f} s wall"}
 
     launches_per_step = 1 + (1 if plan["max_splits"] > 1 else 0)   # split (+ combine)
     if rank == 0:
@@ -512,7 +528,8 @@ def run_native(args):
             "dtype_detail": "E4M3 KV converted exactly to f16; mma.sync f16 x f16 -> f32; "
                             "softmax and reductions in f32; bf16 output",
             "data": "synthetic",
-            "config": {"workload": W.describe(args.config), "B": wl.B, "Hq": wl.Hq,
+            "config": {"workload": W.describe(args.config), "B": wl.B, "q_len": wl.q_len,
+                       "Hq": wl.Hq,
                        "Hkv": wl.Hkv, "D": wl.D, "block_tokens": wl.block_tokens,
                        "kv_bytes_per_call": kv_bytes, "parallelism": f"replicas x{ws}",
                        "l2": f"inputs larger than L2: {replicas} KV replicas rotated, "

@@ -32,7 +32,8 @@ __all__ = [
     "fp8_paged_decode_workspace_bytes_ex", "fp8_paged_decode_attention_profiled",
     "fp8_paged_decode_attention", "fp8_paged_decode_attention_ex",
     "fp8_paged_decode_check_status", "fp8_paged_decode_workspace_init",
-    "fp8_paged_decode_cache_write",
+    "fp8_paged_decode_cache_write", "fp8_paged_decode_plan_qlen",
+    "fp8_paged_decode_workspace_bytes_qlen",
     "fp8_paged_decode_status_string", "fp8_paged_decode_version", "EXPORTED_SYMBOLS",
 ]
 
@@ -65,6 +66,9 @@ EXPORTED_SYMBOLS = (
     "fp8_paged_decode_check_status",
     "fp8_paged_decode_workspace_init",
     "fp8_paged_decode_cache_write",
+    "fp8_paged_decode_attention_qlen",
+    "fp8_paged_decode_plan_qlen",
+    "fp8_paged_decode_workspace_bytes_qlen",
     "fp8_paged_decode_status_string",
     "fp8_paged_decode_version",
 )
@@ -103,9 +107,15 @@ def _bind(lib):
     lib.fp8_paged_decode_attention.restype = ci
     lib.fp8_paged_decode_attention_ex.argtypes = attn + [ci]
     lib.fp8_paged_decode_attention_ex.restype = ci
-    lib.fp8_paged_decode_attention_profiled.argtypes = attn + [ci, vp, vp, vp]
+    lib.fp8_paged_decode_attention_profiled.argtypes = attn[:6] + [ci] + attn[6:] + [ci, vp, vp, vp]
     lib.fp8_paged_decode_attention_profiled.restype = ci
     lib.fp8_paged_decode_attention_noalloc.argtypes = attn[:19] + [vp]
+    lib.fp8_paged_decode_attention_qlen.argtypes = attn[:6] + [ci] + attn[6:] + [ci]
+    lib.fp8_paged_decode_attention_qlen.restype = ci
+    lib.fp8_paged_decode_plan_qlen.argtypes = [ci] * 9 + [ctypes.POINTER(fpd_plan)]
+    lib.fp8_paged_decode_plan_qlen.restype = ci
+    lib.fp8_paged_decode_workspace_bytes_qlen.argtypes = [ci] * 9
+    lib.fp8_paged_decode_workspace_bytes_qlen.restype = cz
     lib.fp8_paged_decode_attention_noalloc.restype = ci
     lib.fp8_paged_decode_check_status.argtypes = [vp, vp, ctypes.POINTER(ci), ci]
     lib.fp8_paged_decode_check_status.restype = ci
@@ -185,6 +195,24 @@ def fp8_paged_decode_workspace_bytes(B, Hq, Hkv, D, block_tokens, max_blocks, wi
         int(B), int(Hq), int(Hkv), int(D), int(block_tokens), int(max_blocks), int(window_left)))
 
 
+def fp8_paged_decode_plan_qlen(B, q_len, Hq, Hkv, D, block_tokens, max_blocks, window_left=-1,
+                               chunk_pages_override=0) -> dict:
+    """The plan used on the current CUDA device for q_len queries per sequence."""
+    plan = fpd_plan()
+    st = load_library().fp8_paged_decode_plan_qlen(
+        int(B), int(q_len), int(Hq), int(Hkv), int(D), int(block_tokens), int(max_blocks),
+        int(window_left), int(chunk_pages_override), ctypes.byref(plan))
+    _check(st, "fp8_paged_decode_plan_qlen")
+    return {f: getattr(plan, f) for f, _ in fpd_plan._fields_}
+
+
+def fp8_paged_decode_workspace_bytes_qlen(B, q_len, Hq, Hkv, D, block_tokens, max_blocks,
+                                          window_left=-1, chunk_pages_override=0) -> int:
+    return int(load_library().fp8_paged_decode_workspace_bytes_qlen(
+        int(B), int(q_len), int(Hq), int(Hkv), int(D), int(block_tokens), int(max_blocks),
+        int(window_left), int(chunk_pages_override)))
+
+
 def fp8_paged_decode_workspace_bytes_ex(B, Hq, Hkv, D, block_tokens, max_blocks, window_left=-1,
                                         chunk_pages_override=0):
     return int(load_library().fp8_paged_decode_workspace_bytes_ex(
@@ -220,40 +248,48 @@ def fp8_paged_decode_attention(q, k_cache, v_cache, block_table, seq_lens, k_sca
                                return_lse=True):
     """Enqueue one decode call on ``stream`` (default: torch's current stream).
 
-    Allocates ``out``/``lse``/``workspace`` with torch when not given (pass them
-    in to keep a call allocation-free).  Returns ``(out, lse)``.
+    ``q`` is [B, Hq, D] (one query token per sequence) or [B, q_len, Hq, D]
+    (the q_len newest tokens of each sequence, causal); ``out``/``lse`` take
+    q's leading shape.  Allocates ``out``/``lse``/``workspace`` with torch when
+    not given (pass them in to keep a call allocation-free).  Returns
+    ``(out, lse)``.
     """
     import torch
-    B, Hq, D = q.shape
+    if q.dim() == 3:
+        B, Hq, D = q.shape
+        q_len = 1
+    else:
+        B, q_len, Hq, D = q.shape
+    lead = tuple(q.shape[:-2])
     num_blocks, bt, Hkv, D2 = k_cache.shape
     if D2 != D:
         raise ValueError("q and the caches disagree on head_dim")
     max_blocks = block_table.shape[1]
     dev = q.device
     if out is None:
-        out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=dev)
+        out = torch.empty(lead + (Hq, D), dtype=torch.bfloat16, device=dev)
     if lse is None and return_lse:
-        lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
-    need = fp8_paged_decode_workspace_bytes_ex(B, Hq, Hkv, D, bt, max_blocks, window_left,
-                                               chunk_pages_override)
+        lse = torch.empty(lead + (Hq,), dtype=torch.float32, device=dev)
+    need = fp8_paged_decode_workspace_bytes_qlen(B, q_len, Hq, Hkv, D, bt, max_blocks,
+                                                 window_left, chunk_pages_override)
     if workspace is None:
         if need == 0 and B > 0:   # surface the planner's own status
-            fp8_paged_decode_plan(B, Hq, Hkv, D, bt, max_blocks, window_left,
-                                  chunk_pages_override)
+            fp8_paged_decode_plan_qlen(B, q_len, Hq, Hkv, D, bt, max_blocks, window_left,
+                                       chunk_pages_override)
             raise FpdError(FPD_ERR_UNSUPPORTED, "fp8_paged_decode_workspace_bytes")
         workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)
     kv_types = (torch.uint8, torch.float8_e4m3fn)
-    st = load_library().fp8_paged_decode_attention_ex(
-        _dev_ptr(q, "q", (torch.bfloat16,), (B, Hq, D)),
+    st = load_library().fp8_paged_decode_attention_qlen(
+        _dev_ptr(q, "q", (torch.bfloat16,), lead + (Hq, D)),
         _dev_ptr(k_cache, "k_cache", kv_types),
         _dev_ptr(v_cache, "v_cache", kv_types, tuple(k_cache.shape)),
         _dev_ptr(block_table, "block_table", (torch.int32,), (B, max_blocks)),
         _dev_ptr(seq_lens, "seq_lens", (torch.int32,), (B,)),
-        B, Hq, Hkv, D, num_blocks, bt, max_blocks,
+        B, q_len, Hq, Hkv, D, num_blocks, bt, max_blocks,
         float(k_scale), float(v_scale), float(sm_scale), int(window_left),
         _dev_ptr(sinks, "sinks", (torch.float32,), (Hq,)),
-        _dev_ptr(out, "out", (torch.bfloat16,), (B, Hq, D)),
-        _dev_ptr(lse, "lse", (torch.float32,), (B, Hq)),
+        _dev_ptr(out, "out", (torch.bfloat16,), lead + (Hq, D)),
+        _dev_ptr(lse, "lse", (torch.float32,), lead + (Hq,)),
         _dev_ptr(workspace, "workspace", (torch.uint8,)),
         ctypes.c_size_t(workspace.numel()),
         _stream_handle(stream), int(chunk_pages_override))

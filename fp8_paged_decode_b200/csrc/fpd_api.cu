@@ -32,18 +32,22 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 bool supported_group(int g) { return g == 1 || g == 2 || g == 4 || g == 8 || g == 16; }
 
-fpd_status validate_shape(int B, int Hq, int Hkv, int D, int bt, int max_blocks) {
-  if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || bt <= 0 || max_blocks <= 0)
+// q_len query tokens per sequence: the MMA columns of a KV head are its
+// q_len * g (query token, head) pairs, at most 16 (two n-tiles).
+fpd_status validate_shape(int B, int Hq, int Hkv, int D, int bt, int max_blocks, int q_len = 1) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || bt <= 0 || max_blocks <= 0 || q_len < 1)
     return FPD_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return FPD_ERR_INVALID_ARG;
   if (!supported_group(Hq / Hkv)) return FPD_ERR_UNSUPPORTED;
+  if (q_len * (Hq / Hkv) > 16) return FPD_ERR_UNSUPPORTED;
   if (D != 64 && D != 128) return FPD_ERR_UNSUPPORTED;
   if (bt != 16 && bt != 32 && bt != 64) return FPD_ERR_UNSUPPORTED;
   if ((int64_t)max_blocks * bt > INT32_MAX) return FPD_ERR_UNSUPPORTED;
   return FPD_OK;
 }
 
-int n_tiles(int g) { return g > 8 ? 2 : 1; }
+// MMA n-tiles (8 columns each) for `cols` columns per KV head.
+int n_tiles(int cols) { return cols > 8 ? 2 : 1; }
 
 // KV heads per stage and work item: 4 whenever the KV heads split into groups
 // of 4 (one TMA box then covers 16 tokens of 4 heads), else 1.
@@ -76,11 +80,14 @@ int ring_stages(int D, int NT, int HB) {
 #ifndef FPD_HDR2_MAX_QBYTES
 #define FPD_HDR2_MAX_QBYTES 4096
 #endif
-int header_slots(int D, int g, int HB) { return HB * g * D * 2 <= FPD_HDR2_MAX_QBYTES ? 2 : 1; }
+int header_slots(int D, int cols, int HB) {
+  return HB * cols * D * 2 <= FPD_HDR2_MAX_QBYTES ? 2 : 1;
+}
 
-int smem_bytes_for(int D, int g, int HB, int B) {
-  const int NT = n_tiles(g);
-  return fpd::smem_layout(D, NT, HB, ring_stages(D, NT, HB), header_slots(D, g, HB), g, B)
+// Shared memory of the split kernel with `cols` = q_len * g columns per KV head.
+int smem_bytes_for(int D, int cols, int HB, int B) {
+  const int NT = n_tiles(cols);
+  return fpd::smem_layout(D, NT, HB, ring_stages(D, NT, HB), header_slots(D, cols, HB), cols, B)
       .total;
 }
 
@@ -104,7 +111,7 @@ WsLayout ws_layout(int B, int Hq, int Hkv, int D, int max_splits) {
 
 // ---- per-device facts, queried once
 struct OccEntry {
-  int D, NT, HB, smem, occ;
+  int D, NT, HB, mq, smem, occ;
 };
 struct DeviceInfo {
   bool ready = false;
@@ -116,17 +123,19 @@ struct DeviceInfo {
 std::mutex g_mu;
 DeviceInfo g_dev[kMaxDevices];
 
-template <int HB>
+template <int HB, bool MQ>
 const void* split_kernel_hb(int D, int NT) {
   if (D == 128)
-    return NT == 2 ? reinterpret_cast<const void*>(&fpd::fpd_split_kernel<128, 2, HB>)
-                   : reinterpret_cast<const void*>(&fpd::fpd_split_kernel<128, 1, HB>);
-  return NT == 2 ? reinterpret_cast<const void*>(&fpd::fpd_split_kernel<64, 2, HB>)
-                 : reinterpret_cast<const void*>(&fpd::fpd_split_kernel<64, 1, HB>);
+    return NT == 2 ? reinterpret_cast<const void*>(&fpd::fpd_split_kernel<128, 2, HB, MQ>)
+                   : reinterpret_cast<const void*>(&fpd::fpd_split_kernel<128, 1, HB, MQ>);
+  return NT == 2 ? reinterpret_cast<const void*>(&fpd::fpd_split_kernel<64, 2, HB, MQ>)
+                 : reinterpret_cast<const void*>(&fpd::fpd_split_kernel<64, 1, HB, MQ>);
 }
 
-const void* split_kernel_for(int D, int NT, int HB) {
-  return HB == 4 ? split_kernel_hb<4>(D, NT) : split_kernel_hb<1>(D, NT);
+// mq: the kernel for several query tokens per sequence
+const void* split_kernel_for(int D, int NT, int HB, bool mq) {
+  if (mq) return HB == 4 ? split_kernel_hb<4, true>(D, NT) : split_kernel_hb<1, true>(D, NT);
+  return HB == 4 ? split_kernel_hb<4, false>(D, NT) : split_kernel_hb<1, false>(D, NT);
 }
 
 bool current_device(int* dev) {
@@ -164,8 +173,9 @@ bool device_sm_count(int* num_sms) {
 }
 
 // SM count of the current device and the number of split-kernel CTAs that fit
-// on one SM with `smem` bytes of dynamic shared memory (0 if none).
-bool device_occupancy(int D, int NT, int HB, int smem, int* num_sms, int* ctas_per_sm) {
+// on one SM with `smem` bytes of dynamic shared memory (0 if none).  Also sets
+// the kernel's dynamic shared-memory limit, which its launch needs.
+bool device_occupancy(int D, int NT, int HB, bool mq, int smem, int* num_sms, int* ctas_per_sm) {
   int dev = 0;
   if (!current_device(&dev)) return false;
   std::lock_guard<std::mutex> lk(g_mu);
@@ -175,13 +185,13 @@ bool device_occupancy(int D, int NT, int HB, int smem, int* num_sms, int* ctas_p
   *num_sms = di.num_sms;
   for (int i = 0; i < di.n_occ; ++i) {
     const OccEntry& e = di.occ[i];
-    if (e.D == D && e.NT == NT && e.HB == HB && e.smem == smem) {
+    if (e.D == D && e.NT == NT && e.HB == HB && e.mq == (int)mq && e.smem == smem) {
       *ctas_per_sm = e.occ;
       return true;
     }
   }
   int occ = 0;
-  const void* fn = split_kernel_for(D, NT, HB);
+  const void* fn = split_kernel_for(D, NT, HB, mq);
   cudaFuncAttributes fa;
   if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) {
     cudaGetLastError();
@@ -197,7 +207,7 @@ bool device_occupancy(int D, int NT, int HB, int smem, int* num_sms, int* ctas_p
       return false;
     }
   }
-  if (di.n_occ < kOccCacheSize) di.occ[di.n_occ++] = OccEntry{D, NT, HB, smem, occ};
+  if (di.n_occ < kOccCacheSize) di.occ[di.n_occ++] = OccEntry{D, NT, HB, (int)mq, smem, occ};
   *ctas_per_sm = occ;
   return true;
 }
@@ -255,11 +265,11 @@ bool encode_cache_map(CUtensorMap* map, const void* base, int num_blocks, int bt
 
 // Combine launch as a programmatic dependent of the split kernel: its CTAs may
 // start while the split kernel drains and wait for it on the device.
-template <int D>
+template <int D, bool MQ>
 cudaError_t launch_combine(const fpd::CombineParams& c, cudaStream_t st) {
   const int rows_per_cta = c.rows_per_cta;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)((c.B * c.Hq + rows_per_cta - 1) / rows_per_cta));
+  cfg.gridDim = dim3((unsigned)((c.B * c.q_len * c.Hq + rows_per_cta - 1) / rows_per_cta));
   cfg.blockDim = dim3(c.wpr * rows_per_cta * 32);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
@@ -268,14 +278,14 @@ cudaError_t launch_combine(const fpd::CombineParams& c, cudaStream_t st) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, fpd::fpd_combine_kernel<D>, c);
+  return cudaLaunchKernelEx(&cfg, fpd::fpd_combine_kernel<D, MQ>, c);
 }
 
 // The split kernel is launched as a programmatic dependent of whatever ran
 // before it in the stream: its CTAs may become resident while that kernel
 // drains, and its first instruction waits for that kernel's completion, so
 // the ordering is that of a plain launch without the launch gap.
-template <int D, int NT, int HB>
+template <int D, int NT, int HB, bool MQ>
 cudaError_t launch_split(const CUtensorMap& km, const CUtensorMap& vm, const fpd::DecodeParams& p,
                          int ctas, int smem, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
@@ -288,32 +298,33 @@ cudaError_t launch_split(const CUtensorMap& km, const CUtensorMap& vm, const fpd
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, fpd::fpd_split_kernel<D, NT, HB>, km, vm, p);
+  return cudaLaunchKernelEx(&cfg, fpd::fpd_split_kernel<D, NT, HB, MQ>, km, vm, p);
 }
 
-template <int HB>
+template <int HB, bool MQ>
 cudaError_t launch_split_hb(int D, int NT, const CUtensorMap& km, const CUtensorMap& vm,
                             const fpd::DecodeParams& p, int ctas, int smem, cudaStream_t st) {
   if (D == 128)
-    return NT == 2 ? launch_split<128, 2, HB>(km, vm, p, ctas, smem, st)
-                   : launch_split<128, 1, HB>(km, vm, p, ctas, smem, st);
-  return NT == 2 ? launch_split<64, 2, HB>(km, vm, p, ctas, smem, st)
-                 : launch_split<64, 1, HB>(km, vm, p, ctas, smem, st);
+    return NT == 2 ? launch_split<128, 2, HB, MQ>(km, vm, p, ctas, smem, st)
+                   : launch_split<128, 1, HB, MQ>(km, vm, p, ctas, smem, st);
+  return NT == 2 ? launch_split<64, 2, HB, MQ>(km, vm, p, ctas, smem, st)
+                 : launch_split<64, 1, HB, MQ>(km, vm, p, ctas, smem, st);
 }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 // The split plan for a given stage shape (HB KV heads per stage).
-void plan_shape(int B, int Hq, int Hkv, int D, int bt, int max_blocks, int window_left,
-                int64_t slots, int chunk_pages_override, int HB, fpd_plan* plan) {
+void plan_shape(int B, int q_len, int Hq, int Hkv, int D, int bt, int max_blocks,
+                int window_left, int64_t slots, int chunk_pages_override, int HB, fpd_plan* plan) {
   const int g = Hq / Hkv;
-  const int NT = n_tiles(g);
+  const int cols = q_len * g;
+  const int NT = n_tiles(cols);
   // with one KV head per stage a stage is 64 tokens of whole pages, and a
   // split must be whole stages; four-head stages are 16 tokens of one page
   const int pps = HB == 1 ? fpd::kTileTokens / bt : 1;
   int pages_max = max_blocks;
-  if (window_left >= 0) {
-    const int64_t w = (int64_t)window_left / bt + 2;
+  if (window_left >= 0) {   // the q_len queries' windows together span window_left + q_len keys
+    const int64_t w = ((int64_t)window_left + q_len - 1) / bt + 2;
     if (w < pages_max) pages_max = (int)w;
   }
   const int64_t units = (int64_t)(B > 0 ? B : 1) * (Hkv / HB);
@@ -338,32 +349,58 @@ void plan_shape(int B, int Hq, int Hkv, int D, int bt, int max_blocks, int windo
   plan->heads_per_stage = HB;
   plan->stage_tokens = fpd::kTileTokens / HB;
   plan->stages = ring_stages(D, NT, HB);
-  plan->header_slots = header_slots(D, g, HB);
+  plan->header_slots = header_slots(D, cols, HB);
   plan->ctas = (int)(items_max < slots ? items_max : slots);
-  plan->smem_bytes = smem_bytes_for(D, g, HB, B);
-  plan->workspace_bytes = ws_layout(B, Hq, Hkv, D, max_splits).total;
+  plan->smem_bytes = smem_bytes_for(D, cols, HB, B);
+  // partial results for each of the B * q_len query tokens
+  plan->workspace_bytes = ws_layout(B * q_len, Hq, Hkv, D, max_splits).total;
 }
 
 // Validates and plans.  force_hb = 0 picks the stage shape: four KV heads per
 // stage when Hkv allows it and the four-head work items fill every CTA slot
 // at least once; otherwise (short windows over few sequences) one head per
 // stage, whose 4x more numerous items keep the machine busy.
-fpd_status plan_for(int B, int Hq, int Hkv, int D, int bt, int max_blocks, int window_left,
-                    int num_sms, int ctas_per_sm, int chunk_pages_override, int force_hb,
-                    fpd_plan* plan) {
+fpd_status plan_for(int B, int q_len, int Hq, int Hkv, int D, int bt, int max_blocks,
+                    int window_left, int num_sms, int ctas_per_sm, int chunk_pages_override,
+                    int force_hb, fpd_plan* plan) {
   if (!plan) return FPD_ERR_INVALID_ARG;
-  fpd_status st = validate_shape(B, Hq, Hkv, D, bt, max_blocks);
+  fpd_status st = validate_shape(B, Hq, Hkv, D, bt, max_blocks, q_len);
   if (st != FPD_OK) return st;
   if (num_sms <= 0 || ctas_per_sm <= 0 || chunk_pages_override < 0) return FPD_ERR_INVALID_ARG;
   if (force_hb != 0 && force_hb != 1 && force_hb != 4) return FPD_ERR_INVALID_ARG;
   if (force_hb == 4 && heads_per_stage(Hkv) != 4) return FPD_ERR_INVALID_ARG;
   const int64_t slots = (int64_t)num_sms * ctas_per_sm;
   int HB = force_hb ? force_hb : heads_per_stage(Hkv);
-  plan_shape(B, Hq, Hkv, D, bt, max_blocks, window_left, slots, chunk_pages_override, HB, plan);
+  plan_shape(B, q_len, Hq, Hkv, D, bt, max_blocks, window_left, slots, chunk_pages_override, HB,
+             plan);
   if (force_hb == 0 && HB == 4 && chunk_pages_override == 0 &&
       (int64_t)(B > 0 ? B : 1) * (Hkv / 4) * plan->max_splits < slots)
-    plan_shape(B, Hq, Hkv, D, bt, max_blocks, window_left, slots, 0, 1, plan);
+    plan_shape(B, q_len, Hq, Hkv, D, bt, max_blocks, window_left, slots, 0, 1, plan);
   return FPD_OK;
+}
+
+// The plan on the current device (its SM count and the split kernel's
+// occupancy for the chosen stage shape).
+fpd_status plan_device(int B, int q_len, int Hq, int Hkv, int D, int bt, int max_blocks,
+                       int window_left, int chunk_pages_override, fpd_plan* plan) {
+  if (!plan) return FPD_ERR_INVALID_ARG;
+  fpd_status st = validate_shape(B, Hq, Hkv, D, bt, max_blocks, q_len);
+  if (st != FPD_OK) return st;
+  const int cols = q_len * (Hq / Hkv);
+  int HB = heads_per_stage(Hkv), force_hb = 0;
+  for (;;) {
+    int sms = 0, occ = 0;
+    if (!device_occupancy(D, n_tiles(cols), HB, q_len > 1, smem_bytes_for(D, cols, HB, B), &sms,
+                          &occ))
+      return FPD_ERR_CUDA;
+    if (occ <= 0) return FPD_ERR_UNSUPPORTED;  // the batch's shared-memory table does not fit
+    st = plan_for(B, q_len, Hq, Hkv, D, bt, max_blocks, window_left, sms, occ,
+                  chunk_pages_override, force_hb, plan);
+    // the planner fell back to one head per stage: plan again with that
+    // kernel's own occupancy
+    if (st != FPD_OK || plan->heads_per_stage == HB) return st;
+    HB = force_hb = plan->heads_per_stage;
+  }
 }
 
 }  // namespace
@@ -386,29 +423,30 @@ const char* fp8_paged_decode_version(void) { return "0.2.0 sm_100a"; }
 fpd_status fp8_paged_decode_make_plan(int B, int Hq, int Hkv, int D, int bt, int max_blocks,
                                       int window_left, int num_sms, int ctas_per_sm,
                                       int chunk_pages_override, fpd_plan* plan) {
-  return plan_for(B, Hq, Hkv, D, bt, max_blocks, window_left, num_sms, ctas_per_sm,
+  return plan_for(B, 1, Hq, Hkv, D, bt, max_blocks, window_left, num_sms, ctas_per_sm,
                   chunk_pages_override, 0, plan);
 }
 
 fpd_status fp8_paged_decode_plan(int B, int Hq, int Hkv, int D, int bt, int max_blocks,
                                  int window_left, int chunk_pages_override, fpd_plan* plan) {
-  if (!plan) return FPD_ERR_INVALID_ARG;
-  fpd_status st = validate_shape(B, Hq, Hkv, D, bt, max_blocks);
-  if (st != FPD_OK) return st;
-  const int g = Hq / Hkv;
-  int HB = heads_per_stage(Hkv), force_hb = 0;
-  for (;;) {
-    int sms = 0, occ = 0;
-    if (!device_occupancy(D, n_tiles(g), HB, smem_bytes_for(D, g, HB, B), &sms, &occ))
-      return FPD_ERR_CUDA;
-    if (occ <= 0) return FPD_ERR_UNSUPPORTED;  // the batch's shared-memory table does not fit
-    st = plan_for(B, Hq, Hkv, D, bt, max_blocks, window_left, sms, occ, chunk_pages_override,
-                  force_hb, plan);
-    // the planner fell back to one head per stage: plan again with that
-    // kernel's own occupancy
-    if (st != FPD_OK || plan->heads_per_stage == HB) return st;
-    HB = force_hb = plan->heads_per_stage;
-  }
+  return plan_device(B, 1, Hq, Hkv, D, bt, max_blocks, window_left, chunk_pages_override, plan);
+}
+
+fpd_status fp8_paged_decode_plan_qlen(int B, int q_len, int Hq, int Hkv, int D, int bt,
+                                      int max_blocks, int window_left, int chunk_pages_override,
+                                      fpd_plan* plan) {
+  return plan_device(B, q_len, Hq, Hkv, D, bt, max_blocks, window_left, chunk_pages_override,
+                     plan);
+}
+
+size_t fp8_paged_decode_workspace_bytes_qlen(int B, int q_len, int Hq, int Hkv, int D, int bt,
+                                             int max_blocks, int window_left,
+                                             int chunk_pages_override) {
+  fpd_plan plan;
+  if (plan_device(B, q_len, Hq, Hkv, D, bt, max_blocks, window_left, chunk_pages_override,
+                  &plan) != FPD_OK)
+    return 0;
+  return plan.workspace_bytes;
 }
 
 size_t fp8_paged_decode_workspace_bytes_ex(int B, int Hq, int Hkv, int D, int bt, int max_blocks,
@@ -429,12 +467,12 @@ size_t fp8_paged_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int bt, i
 
 static fpd_status attention_impl(const void* q, const void* k_cache, const void* v_cache,
                                  const int32_t* block_table, const int32_t* seq_lens, int B,
-                                 int Hq, int Hkv, int D, int num_blocks, int bt, int max_blocks,
-                                 float k_scale, float v_scale, float sm_scale, int window_left,
-                                 const float* sinks, void* out, float* lse, void* workspace,
-                                 size_t workspace_bytes, void* stream, int chunk_pages_override,
-                                 void* ev0, void* ev1, void* ev2) {
-  fpd_status st = validate_shape(B, Hq, Hkv, D, bt, max_blocks);
+                                 int q_len, int Hq, int Hkv, int D, int num_blocks, int bt,
+                                 int max_blocks, float k_scale, float v_scale, float sm_scale,
+                                 int window_left, const float* sinks, void* out, float* lse,
+                                 void* workspace, size_t workspace_bytes, void* stream,
+                                 int chunk_pages_override, void* ev0, void* ev1, void* ev2) {
+  fpd_status st = validate_shape(B, Hq, Hkv, D, bt, max_blocks, q_len);
   if (st != FPD_OK) return st;
   if (num_blocks <= 0 || (int64_t)num_blocks * bt >= INT32_MAX) return FPD_ERR_UNSUPPORTED;
   if (!q || !k_cache || !v_cache || !block_table || !seq_lens || !out) return FPD_ERR_INVALID_ARG;
@@ -451,8 +489,7 @@ static fpd_status attention_impl(const void* q, const void* k_cache, const void*
 
   const int g = Hq / Hkv;
   fpd_plan plan;
-  st = fp8_paged_decode_plan(B, Hq, Hkv, D, bt, max_blocks, window_left, chunk_pages_override,
-                             &plan);
+  st = plan_device(B, q_len, Hq, Hkv, D, bt, max_blocks, window_left, chunk_pages_override, &plan);
   if (st != FPD_OK) return st;
   if (!workspace || workspace_bytes < plan.workspace_bytes) return FPD_ERR_WORKSPACE_TOO_SMALL;
 
@@ -461,7 +498,7 @@ static fpd_status attention_impl(const void* q, const void* k_cache, const void*
       !encode_cache_map(&vm, v_cache, num_blocks, bt, Hkv, D, plan.heads_per_stage))
     return FPD_ERR_CUDA;
 
-  const WsLayout wl = ws_layout(B, Hq, Hkv, D, plan.max_splits);
+  const WsLayout wl = ws_layout(B * q_len, Hq, Hkv, D, plan.max_splits);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   fpd::DecodeParams p;
   p.q = static_cast<const __nv_bfloat16*>(q);
@@ -486,16 +523,22 @@ static fpd_status attention_impl(const void* q, const void* k_cache, const void*
   p.max_splits = plan.max_splits;
   p.stages = plan.stages;
   p.hdr_slots = plan.header_slots;
+  p.q_len = q_len;
+  p.lg = __builtin_ctz((unsigned)g);
   p.qk_scale_log2 = qk * fpd::kLog2e;
   p.v_scale = v_scale;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (ev0 && cudaEventRecord(static_cast<cudaEvent_t>(ev0), s) != cudaSuccess) return FPD_ERR_CUDA;
   cudaError_t e;
-  const int NT = n_tiles(g);
-  e = plan.heads_per_stage == 4
-          ? launch_split_hb<4>(D, NT, km, vm, p, plan.ctas, plan.smem_bytes, s)
-          : launch_split_hb<1>(D, NT, km, vm, p, plan.ctas, plan.smem_bytes, s);
+  const int NT = n_tiles(q_len * g);
+  const bool mq = q_len > 1;
+  if (plan.heads_per_stage == 4)
+    e = mq ? launch_split_hb<4, true>(D, NT, km, vm, p, plan.ctas, plan.smem_bytes, s)
+           : launch_split_hb<4, false>(D, NT, km, vm, p, plan.ctas, plan.smem_bytes, s);
+  else
+    e = mq ? launch_split_hb<1, true>(D, NT, km, vm, p, plan.ctas, plan.smem_bytes, s)
+           : launch_split_hb<1, false>(D, NT, km, vm, p, plan.ctas, plan.smem_bytes, s);
   if (e != cudaSuccess) return FPD_ERR_CUDA;
   if (ev1 && cudaEventRecord(static_cast<cudaEvent_t>(ev1), s) != cudaSuccess) return FPD_ERR_CUDA;
   if (plan.max_splits > 1) {
@@ -507,6 +550,7 @@ static fpd_status attention_impl(const void* q, const void* k_cache, const void*
     c.out = p.out;
     c.lse = lse;
     c.B = B;
+    c.q_len = q_len;
     c.Hq = Hq;
     c.bt = bt;
     c.max_blocks = max_blocks;
@@ -519,7 +563,10 @@ static fpd_status attention_impl(const void* q, const void* k_cache, const void*
     while (c.wpr < 32 && c.wpr * fpd::kCombineBatch < plan.max_splits) c.wpr *= 2;
     c.rows_per_cta = c.wpr >= 8 ? 1 : 8 / c.wpr;
     c.v_scale = v_scale;
-    e = D == 128 ? launch_combine<128>(c, s) : launch_combine<64>(c, s);
+    if (mq)
+      e = D == 128 ? launch_combine<128, true>(c, s) : launch_combine<64, true>(c, s);
+    else
+      e = D == 128 ? launch_combine<128, false>(c, s) : launch_combine<64, false>(c, s);
     if (e != cudaSuccess) return FPD_ERR_CUDA;
   }
   if (ev2 && cudaEventRecord(static_cast<cudaEvent_t>(ev2), s) != cudaSuccess) return FPD_ERR_CUDA;
@@ -536,20 +583,34 @@ fpd_status fp8_paged_decode_attention_ex(const void* q, const void* k_cache, con
                                          void* out, float* lse, void* workspace,
                                          size_t workspace_bytes, void* stream,
                                          int chunk_pages_override) {
-  return attention_impl(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, D, num_blocks, bt,
+  return attention_impl(q, k_cache, v_cache, block_table, seq_lens, B, 1, Hq, Hkv, D, num_blocks, bt,
                         max_blocks, k_scale, v_scale, sm_scale, window_left, sinks, out, lse,
                         workspace, workspace_bytes, stream, chunk_pages_override, nullptr,
                         nullptr, nullptr);
 }
 
+fpd_status fp8_paged_decode_attention_qlen(const void* q, const void* k_cache,
+                                           const void* v_cache, const int32_t* block_table,
+                                           const int32_t* seq_lens, int B, int q_len, int Hq,
+                                           int Hkv, int D, int num_blocks, int bt, int max_blocks,
+                                           float k_scale, float v_scale, float sm_scale,
+                                           int window_left, const float* sinks, void* out,
+                                           float* lse, void* workspace, size_t workspace_bytes,
+                                           void* stream, int chunk_pages_override) {
+  return attention_impl(q, k_cache, v_cache, block_table, seq_lens, B, q_len, Hq, Hkv, D,
+                        num_blocks, bt, max_blocks, k_scale, v_scale, sm_scale, window_left, sinks,
+                        out, lse, workspace, workspace_bytes, stream, chunk_pages_override,
+                        nullptr, nullptr, nullptr);
+}
+
 fpd_status fp8_paged_decode_attention_profiled(
     const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
-    const int32_t* seq_lens, int B, int Hq, int Hkv, int D, int num_blocks, int bt,
+    const int32_t* seq_lens, int B, int q_len, int Hq, int Hkv, int D, int num_blocks, int bt,
     int max_blocks, float k_scale, float v_scale, float sm_scale, int window_left,
     const float* sinks, void* out, float* lse, void* workspace, size_t workspace_bytes,
     void* stream, int chunk_pages_override, void* event_before_split, void* event_after_split,
     void* event_after_combine) {
-  return attention_impl(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, D, num_blocks, bt,
+  return attention_impl(q, k_cache, v_cache, block_table, seq_lens, B, q_len, Hq, Hkv, D, num_blocks, bt,
                         max_blocks, k_scale, v_scale, sm_scale, window_left, sinks, out, lse,
                         workspace, workspace_bytes, stream, chunk_pages_override,
                         event_before_split, event_after_split, event_after_combine);
@@ -624,7 +685,7 @@ fpd_status fp8_paged_decode_attention_noalloc(const void* q, const void* k_cache
   const size_t zero = ws_layout(B, Hq, Hkv, D, plan.max_splits).zero_prefix;
   if (cudaMemsetAsync(scratch, 0, zero, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return FPD_ERR_CUDA;
-  return attention_impl(q, k_cache, v_cache, block_table, seq_lens, B, Hq, Hkv, D, num_blocks, bt,
+  return attention_impl(q, k_cache, v_cache, block_table, seq_lens, B, 1, Hq, Hkv, D, num_blocks, bt,
                         max_blocks, k_scale, v_scale, sm_scale, window_left, sinks, out, lse,
                         scratch, FPD_NOALLOC_SCRATCH_BYTES, stream, 0, nullptr, nullptr, nullptr);
 }

@@ -96,6 +96,8 @@ struct DecodeParams {
   uint32_t* sched;      // workspace words 1, 2: next work item, CTAs finished
   int B, Hq, Hkv, g, bt, max_blocks, num_blocks, window_left;
   int chunk_pages, max_splits, stages, hdr_slots;
+  int q_len;            // query tokens per sequence (columns per KV head: q_len * g)
+  int lg;               // log2(g): g is a power of two
   float qk_scale_log2;  // sm_scale * k_scale * log2(e)
   float v_scale;
 };
@@ -138,7 +140,8 @@ struct ItemHeader {
   int n_stages;  // pipeline stages this item consumes
   int t0;        // token of the first row of the item's first stage
   int tok_lo, tok_hi;
-  int pad[7];
+  int qpos0;     // position of the sequence's first query token (L - q_len)
+  int pad[6];
 };
 static_assert(sizeof(ItemHeader) == kHdrBytes, "header size");
 
@@ -147,8 +150,11 @@ struct SeqRange {
   int L, start, first_page, end_page, n_splits;
 };
 
-__device__ __forceinline__ SeqRange seq_range(int L_raw, int bt, int max_blocks, int window_left,
-                                              int chunk_pages, uint32_t* status) {
+// The union of the key ranges of the sequence's q_len queries: query i at
+// position L - q_len + i sees keys up to its own position and, under a window,
+// the window_left keys before it.
+__device__ __forceinline__ SeqRange seq_range(int L_raw, int q_len, int bt, int max_blocks,
+                                              int window_left, int chunk_pages, uint32_t* status) {
   SeqRange r;
   int L = L_raw;
   const int cap = max_blocks * bt;
@@ -157,7 +163,7 @@ __device__ __forceinline__ SeqRange seq_range(int L_raw, int bt, int max_blocks,
     L = L < 0 ? 0 : cap;
   }
   r.L = L;
-  r.start = (window_left >= 0) ? max(0, L - 1 - window_left) : 0;
+  r.start = (window_left >= 0) ? max(0, L - q_len - window_left) : 0;
   r.first_page = r.start / bt;
   r.end_page = (L + bt - 1) / bt;
   const int n_pages = r.end_page - r.first_page;
@@ -166,9 +172,9 @@ __device__ __forceinline__ SeqRange seq_range(int L_raw, int bt, int max_blocks,
 }
 
 // Work groups (one per split; one for an empty sequence) of a sequence.
-__device__ __forceinline__ int groups_of(int L_raw, const DecodeParams& p) {
+__device__ __forceinline__ int groups_of(int L_raw, int q_len, const DecodeParams& p) {
   const SeqRange r =
-      seq_range(L_raw, p.bt, p.max_blocks, p.window_left, p.chunk_pages, nullptr);
+      seq_range(L_raw, q_len, p.bt, p.max_blocks, p.window_left, p.chunk_pages, nullptr);
   return r.n_splits > 0 ? r.n_splits : 1;
 }
 
@@ -189,7 +195,18 @@ __device__ __forceinline__ bool consumer_sync(uint64_t* bar, uint32_t& parity, i
   return __all_sync(0xffffffffu, ok);
 }
 
-template <int D, int NT>
+// Key ranges of a boundary tile's columns.  With several queries per sequence
+// column c of the MMA N side is query position qpos0 + c / g (head c % g); it
+// sees the item's tokens [tok_lo, tok_hi) up to its own position and, under a
+// window, from `window` tokens before it.  Columns c >= ncols are padding and
+// keep the item's range.  With one query every column has the item's range.
+struct TileMask {
+  int tok_lo, tok_hi, qpos0, window, lg, ncols;
+};
+
+// MQ: several query tokens per sequence (columns are (position, head) pairs
+// with per-column key ranges); otherwise one query and columns are heads.
+template <int D, int NT, bool MQ>
 struct Consumer {
   static constexpr int KS = D / 16;   // k-steps of the QK MMA
   static constexpr int MT = D / 16;   // m-tiles of the PV MMA
@@ -215,17 +232,20 @@ struct Consumer {
     voff[1] = swz<D>((row0 + 2 * t + 1) * D + n * (D / 8));
   }
 
-  // qtile: the item's query rows, bf16 [g][D] in shared memory.
-  __device__ __forceinline__ void init(const DecodeParams& p, const __nv_bfloat16* qtile,
-                                       int lane) {
+  // qbase: the item's query rows in shared memory, bf16 [position][rows_per_pos][D];
+  // column c (query position c / g, head c % g) is row
+  // (c / g) * rows_per_pos + w_off + c % g.
+  __device__ __forceinline__ void init(const DecodeParams& p, const __nv_bfloat16* qbase,
+                                       int rows_per_pos, int w_off, int lane) {
     const int n = lane >> 2, t = lane & 3;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      const int hl = nt * 8 + n;
+      const int c = nt * 8 + n;
       float vals[QW];
       float amax = 0.f;
-      if (hl < p.g) {
-        const __nv_bfloat16* src = qtile + hl * D + t * QW;
+      if (c < (MQ ? p.q_len * p.g : p.g)) {
+        const int qrow = MQ ? (c >> p.lg) * rows_per_pos + w_off + (c & (p.g - 1)) : w_off + c;
+        const __nv_bfloat16* src = qbase + qrow * D + t * QW;
 #pragma unroll
         for (int i = 0; i < QW; i += 8) {
           const uint4 raw = *reinterpret_cast<const uint4*>(src + i);
@@ -256,7 +276,7 @@ struct Consumer {
         qf[nt][ks][0] = pack_f16x2(vals[4 * ks] * fac, vals[4 * ks + 1] * fac);
         qf[nt][ks][1] = pack_f16x2(vals[4 * ks + 2] * fac, vals[4 * ks + 3] * fac);
       }
-      // this thread's C columns are heads 2t and 2t+1 of the n-tile; the
+      // this thread's C columns are columns 2t and 2t+1 of the n-tile; the
       // prescale is a power of two, so undoing it is an exact multiply
       const int sh0 = __shfl_sync(0xffffffffu, sh, (2 * t) * 4);
       const int sh1 = __shfl_sync(0xffffffffu, sh, (2 * t + 1) * 4);
@@ -277,10 +297,11 @@ struct Consumer {
         for (int j = 0; j < 4; ++j) o[i][nt][j] = 0.f;
   }
 
-  // One 16-row slice of a stage.  FULL: every row is inside [tok_lo, tok_hi).
+  // One 16-row slice of a stage.  FULL: every row is inside every column's
+  // range; otherwise rows are masked per column (mk).
   template <bool FULL>
   __device__ __forceinline__ void tile(const uint8_t* Kt, const uint8_t* Vt, int row0, int tok0,
-                                       int tok_lo, int tok_hi, int lane) {
+                                       const TileMask& mk, int lane) {
     const int n = lane >> 2, t = lane & 3;
     // ---- K fragments: rows row0 + n and row0 + n + 8, bytes [t*D/4, (t+1)*D/4)
     uint32_t kw[2][D / 16];
@@ -318,10 +339,27 @@ struct Consumer {
 #pragma unroll
       for (int j = 0; j < 4; ++j) acc[nt][j] = s[nt][0][j] + s[nt][1][j];
 
-    if (!FULL) {
+    if constexpr (!FULL && MQ) {
       const int tk0 = tok0 + n, tk1 = tok0 + n + 8;
-      const bool v0 = tk0 >= tok_lo && tk0 < tok_hi;
-      const bool v1 = tk1 >= tok_lo && tk1 < tok_hi;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int c = nt * 8 + 2 * t + j;
+          int lo = mk.tok_lo, hi = mk.tok_hi;
+          if (c < mk.ncols) {
+            const int pos = mk.qpos0 + (c >> mk.lg);   // this column's query position
+            hi = min(hi, pos + 1);
+            if (mk.window >= 0) lo = max(lo, pos - mk.window);
+          }
+          if (!(tk0 >= lo && tk0 < hi)) acc[nt][j] = -INFINITY;
+          if (!(tk1 >= lo && tk1 < hi)) acc[nt][j + 2] = -INFINITY;
+        }
+      }
+    } else if constexpr (!FULL) {
+      const int tk0 = tok0 + n, tk1 = tok0 + n + 8;
+      const bool v0 = tk0 >= mk.tok_lo && tk0 < mk.tok_hi;
+      const bool v1 = tk1 >= mk.tok_lo && tk1 < mk.tok_hi;
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         if (!v0) acc[nt][0] = acc[nt][1] = -INFINITY;
@@ -365,10 +403,14 @@ struct Consumer {
     uint32_t pb0[NT], pb1[NT];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      const float p0 = fast_exp2(fmaf(acc[nt][0], cs[nt][0], -m[nt][0]));
-      const float p1 = fast_exp2(fmaf(acc[nt][1], cs[nt][1], -m[nt][1]));
-      const float p2 = fast_exp2(fmaf(acc[nt][2], cs[nt][0], -m[nt][0]));
-      const float p3 = fast_exp2(fmaf(acc[nt][3], cs[nt][1], -m[nt][1]));
+      float p0 = fast_exp2(fmaf(acc[nt][0], cs[nt][0], -m[nt][0]));
+      float p1 = fast_exp2(fmaf(acc[nt][1], cs[nt][1], -m[nt][1]));
+      float p2 = fast_exp2(fmaf(acc[nt][2], cs[nt][0], -m[nt][0]));
+      float p3 = fast_exp2(fmaf(acc[nt][3], cs[nt][1], -m[nt][1]));
+      if (!FULL && MQ) {   // a column with no key yet: every logit and its max are -inf
+        if (m[nt][0] == -INFINITY) p0 = p2 = 0.f;
+        if (m[nt][1] == -INFINITY) p1 = p3 = 0.f;
+      }
       l[nt][0] += p0 + p2;
       l[nt][1] += p1 + p3;
       pb0[nt] = movmatrix_trans(pack_f16x2(p0, p1));   // tokens 2t..2t+1, head n
@@ -398,8 +440,9 @@ struct Consumer {
       vd[0] = E.x; vd[1] = E.y;
     }
     if (!FULL) {
-      // Zero value rows outside the range: stale bytes may hold NaN codes and
-      // 0 * NaN would poison the accumulator.
+      // Zero value rows outside the item's range: stale bytes may hold NaN
+      // codes and 0 * NaN would poison the accumulator.
+      const int tok_lo = mk.tok_lo, tok_hi = mk.tok_hi;
       const int tA = tok0 + 2 * t;
       const uint32_t mA = (tA >= tok_lo && tA < tok_hi) ? 0xffffffffu : 0u;
       const uint32_t mB = (tA + 1 >= tok_lo && tA + 1 < tok_hi) ? 0xffffffffu : 0u;
@@ -454,14 +497,17 @@ struct Consumer {
     for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
-        const int hl = nt * 8 + 2 * t + j;
-        if (hl >= p.g) continue;
-        const int hq = kvh * p.g + hl;
-        const size_t row = (size_t)b * p.Hq + hq;
-        if (ns == 0) {  // empty sequence: out = 0, lse = sigma
+        const int c = nt * 8 + 2 * t + j;   // column: query position c / g, head c % g
+        if (c >= (MQ ? p.q_len * p.g : p.g)) continue;
+        const int hq = kvh * p.g + (MQ ? c & (p.g - 1) : c);
+        const size_t row = MQ ? ((size_t)b * p.q_len + (c >> p.lg)) * p.Hq + hq
+                              : (size_t)b * p.Hq + hq;
+        // false: this query saw no key in the item (only possible with MQ)
+        const bool keys = !MQ || lsum[nt][j] > 0.f;
+        if (ns == 0 || (ns == 1 && !keys)) {  // no key at all: out = 0, lse = sigma
           uint4* dst = reinterpret_cast<uint4*>(p.out + row * D + n * E);
 #pragma unroll
-          for (int c = 0; c < E / 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+          for (int k = 0; k < E / 8; ++k) dst[k] = make_uint4(0u, 0u, 0u, 0u);
           if (n == 0 && p.lse) p.lse[row] = p.sinks ? p.sinks[hq] : -INFINITY;
           continue;
         }
@@ -483,18 +529,18 @@ struct Consumer {
           for (int i = 0; i < MT; ++i) w[i] = pack_bf16x2(o[i][nt][j] * inv, o[i][nt][j + 2] * inv);
           uint4* dst = reinterpret_cast<uint4*>(p.out + row * D + n * E);
 #pragma unroll
-          for (int c = 0; c < E / 8; ++c)
-            dst[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+          for (int k = 0; k < E / 8; ++k)
+            dst[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
           if (n == 0 && p.lse) p.lse[row] = lse_out * kLn2;
         } else {
           const size_t prow = row * p.max_splits + split;
-          const float inv = __fdividef(1.0f, lsum[nt][j]);
+          const float inv = keys ? __fdividef(1.0f, lsum[nt][j]) : 0.f;   // no key: O = 0
           float4* dst = reinterpret_cast<float4*>(p.part_o + prow * D + n * E);
 #pragma unroll
-          for (int c = 0; c < E / 4; ++c)
-            dst[c] = make_float4(o[2 * c][nt][j] * inv, o[2 * c][nt][j + 2] * inv,
-                                 o[2 * c + 1][nt][j] * inv, o[2 * c + 1][nt][j + 2] * inv);
-          if (n == 0) p.part_lse[prow] = lse2;
+          for (int k = 0; k < E / 4; ++k)
+            dst[k] = make_float4(o[2 * k][nt][j] * inv, o[2 * k][nt][j + 2] * inv,
+                                 o[2 * k + 1][nt][j] * inv, o[2 * k + 1][nt][j + 2] * inv);
+          if (n == 0) p.part_lse[prow] = keys ? lse2 : -INFINITY;
         }
       }
     }
@@ -503,7 +549,7 @@ struct Consumer {
 
 // ---------------------------------------------------------------- producer --
 
-template <int D, int HB>
+template <int D, int HB, bool MQ>
 __device__ __forceinline__ void producer_loop(const CUtensorMap* kmap, const CUtensorMap* vmap,
                                               const DecodeParams& p, uint8_t* smem,
                                               const SmemLayout& L, const int* prefix,
@@ -514,6 +560,7 @@ __device__ __forceinline__ void producer_loop(const CUtensorMap* kmap, const CUt
   constexpr int kStageTokens = kTileTokens / HB;   // tokens of one KV head per stage
   const int stages = p.stages;
   const int n_hslots = p.hdr_slots;
+  const int QL = MQ ? p.q_len : 1;                 // query tokens per sequence
   const int groups = p.Hkv / HB;                   // KV head groups
   const int pps = HB == 1 ? kStageTokens / p.bt : 1;   // pages per stage (HB = 1)
   const uint32_t page_bytes = (uint32_t)(p.bt * D);
@@ -560,7 +607,8 @@ __device__ __forceinline__ void producer_loop(const CUtensorMap* kmap, const CUt
     }
     const int b = lo;
     const int split = group - prefix[b];
-    const SeqRange R = seq_range(__ldg(p.seq_lens + b), p.bt, p.max_blocks, p.window_left,
+    const SeqRange R = seq_range(__ldg(p.seq_lens + b), QL, p.bt, p.max_blocks,
+                                 p.window_left,
                                  p.chunk_pages, lane == 0 ? p.status : nullptr);
     int pb = 0, pe = 0, tok_lo = 0, tok_hi = 0, t0 = 0, n_st = 0;
     if (R.n_splits > 0) {
@@ -586,10 +634,15 @@ __device__ __forceinline__ void producer_loop(const CUtensorMap* kmap, const CUt
       hdr->t0 = t0;
       hdr->tok_lo = tok_lo;
       hdr->tok_hi = tok_hi;
+      hdr->qpos0 = R.L - QL;
+      // the query rows of the item's KV heads, one copy per query position:
+      // [position][HB * g][D] in the slot
       const uint32_t qbytes = (uint32_t)(HB * p.g * D * 2);
-      mbar_arrive_expect_tx(&hdr_full[hslot], qbytes);
-      bulk_load(hbase + kHdrBytes, p.q + ((size_t)b * p.Hq + (size_t)kvh0 * p.g) * D, qbytes,
-                &hdr_full[hslot]);
+      mbar_arrive_expect_tx(&hdr_full[hslot], qbytes * (uint32_t)QL);
+      for (int i = 0; i < QL; ++i)
+        bulk_load(hbase + kHdrBytes + (size_t)i * qbytes,
+                  p.q + (((size_t)b * QL + i) * p.Hq + (size_t)kvh0 * p.g) * D, qbytes,
+                  &hdr_full[hslot]);
     }
     ++hs;
     if (++hslot == n_hslots) {
@@ -675,7 +728,7 @@ struct MinBlocks {
   static constexpr int value = (D == 128) ? (NT == 1 ? FPD_MINB_D128_NT1 : 2) : (NT == 1 ? 4 : 3);
 };
 
-template <int D, int NT, int HB>
+template <int D, int NT, int HB, bool MQ>
 __global__ void __launch_bounds__(kThreads, MinBlocks<D, NT>::value)
 fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                  const DecodeParams p) {
@@ -688,8 +741,10 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
   constexpr int H = NT * 8;
   const int stages = p.stages;
   const int n_hslots = p.hdr_slots;
-  const SmemLayout L = smem_layout(D, NT, HB, stages, n_hslots, p.g, p.B);
-  const int hslot_bytes = hdr_slot_bytes(D, HB, p.g);
+  // a header slot holds q_len * g query rows per KV head
+  const int QL = MQ ? p.q_len : 1;   // query tokens per sequence
+  const SmemLayout L = smem_layout(D, NT, HB, stages, n_hslots, QL * p.g, p.B);
+  const int hslot_bytes = hdr_slot_bytes(D, HB, QL * p.g);
   int* prefix = reinterpret_cast<int*>(smem + L.prefix);
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + L.bars);
   uint64_t* empty_bar = full_bar + stages;
@@ -708,7 +763,7 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
     const int per = (p.B + kThreads - 1) / kThreads;
     const int b0 = min(p.B, tid * per), b1 = min(p.B, b0 + per);
     int sum = 0;
-    for (int b = b0; b < b1; ++b) sum += groups_of(__ldg(p.seq_lens + b), p);
+    for (int b = b0; b < b1; ++b) sum += groups_of(__ldg(p.seq_lens + b), QL, p);
     int incl = sum;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -734,7 +789,7 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
     int run = base + incl - sum;
     if (tid == 0) prefix[0] = 0;
     for (int b = b0; b < b1; ++b) {
-      run += groups_of(__ldg(p.seq_lens + b), p);
+      run += groups_of(__ldg(p.seq_lens + b), QL, p);
       prefix[b + 1] = run;
     }
     __syncthreads();
@@ -743,13 +798,13 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
   pdl_launch_dependents();   // the combine kernel may be scheduled from now on
 
   if (warp == kConsumerWarps) {
-    producer_loop<D, HB>(&kmap, &vmap, p, smem, L, prefix, total_items, hslot_bytes, full_bar,
+    producer_loop<D, HB, MQ>(&kmap, &vmap, p, smem, L, prefix, total_items, hslot_bytes, full_bar,
                          empty_bar, hdr_full, hdr_empty, lane);
     return;
   }
 
   // -------------------------------------------------------------- consumers
-  Consumer<D, NT> cw;
+  Consumer<D, NT, MQ> cw;
   const int n = lane >> 2, t = lane & 3;
   // HB = 4: this warp's KV head occupies its own 16 rows of each stage.
   // HB = 1: this warp takes rows [16 * warp, 16 * warp + 16) of the stage.
@@ -771,10 +826,16 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
     const uint8_t* hbase = smem + L.hdr + hslot * hslot_bytes;
     const ItemHeader hd = *reinterpret_cast<const ItemHeader*>(hbase);
     if (hd.kind < 0) break;
-    cw.init(p,
-            reinterpret_cast<const __nv_bfloat16*>(hbase + kHdrBytes) +
-                (HB == 1 ? 0 : warp * p.g * D),
-            lane);
+    cw.init(p, reinterpret_cast<const __nv_bfloat16*>(hbase + kHdrBytes), HB * p.g,
+            HB == 1 ? 0 : warp * p.g, lane);
+    // Tiles inside every column's range skip the masks: past the newest key
+    // the first query sees, and at or after the oldest key the last query
+    // sees (window).  With one query per sequence that is [tok_lo, tok_hi).
+    const TileMask mk{hd.tok_lo, hd.tok_hi, hd.qpos0, p.window_left, p.lg, QL * p.g};
+    const int full_lo = MQ && p.window_left >= 0
+                            ? max(hd.tok_lo, hd.qpos0 + QL - 1 - p.window_left)
+                            : hd.tok_lo;
+    const int full_hi = MQ ? min(hd.tok_hi, hd.qpos0 + 1) : hd.tok_hi;
     __syncwarp();
     if (lane == 0) mbar_arrive(&hdr_empty[hslot]);
     if (++hslot == n_hslots) {
@@ -791,10 +852,10 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
       const uint8_t* Vt = Kt + kTileBytes;
       const int tok0 = hd.t0 + s * kStageTokens + tok_off;   // token of this warp's first row
       if (tok0 + kRowsPerWarp > hd.tok_lo && tok0 < hd.tok_hi) {
-        if (tok0 >= hd.tok_lo && tok0 + kRowsPerWarp <= hd.tok_hi)
-          cw.template tile<true>(Kt, Vt, row0, tok0, hd.tok_lo, hd.tok_hi, lane);
+        if (tok0 >= full_lo && tok0 + kRowsPerWarp <= full_hi)
+          cw.template tile<true>(Kt, Vt, row0, tok0, mk, lane);
         else
-          cw.template tile<false>(Kt, Vt, row0, tok0, hd.tok_lo, hd.tok_hi, lane);
+          cw.template tile<false>(Kt, Vt, row0, tok0, mk, lane);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty_bar[slot]);
@@ -830,7 +891,7 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
         // O^T column h: rows d = n*(D/8) + 2i + hh  (hh = 0 -> c0/c1, 1 -> c2/c3)
         float* dst = Osm + ((size_t)warp * H + h) * OS + n * (D / 8);
 #pragma unroll
-        for (int i = 0; i < Consumer<D, NT>::MT; ++i) {
+        for (int i = 0; i < Consumer<D, NT, MQ>::MT; ++i) {
           dst[2 * i + 0] = cw.o[i][nt][j];
           dst[2 * i + 1] = cw.o[i][nt][j + 2];
         }
@@ -847,9 +908,11 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
       constexpr int HPI = kConsumerWarps * 32 / D;
       const int d = tid % D;
 #pragma unroll 4
-      for (int h = tid / D; h < p.g; h += HPI) {
-        const int hq = hd.kvh0 * p.g + h;
-        const size_t row = (size_t)hd.b * p.Hq + hq;
+      for (int h = tid / D; h < (MQ ? p.q_len * p.g : p.g); h += HPI) {
+        // column h: query position h / g, head h % g
+        const int hq = hd.kvh0 * p.g + (MQ ? h & (p.g - 1) : h);
+        const size_t row = MQ ? ((size_t)hd.b * p.q_len + (h >> p.lg)) * p.Hq + hq
+                              : (size_t)hd.b * p.Hq + hq;
         if (hd.ns == 0) {  // empty sequence: out = 0, lse = sigma
           p.out[row * D + d] = __float2bfloat16_rn(0.f);
           if (d == 0 && p.lse) p.lse[row] = p.sinks ? p.sinks[hq] : -INFINITY;
@@ -870,6 +933,17 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
           acc = fmaf(Osm[((size_t)w * H + h) * OS + d], sc, acc);
         }
         const float lse2 = M + __log2f(Lsum);   // log2-sum-exp of this split (no sink)
+        if (MQ && !(Lsum > 0.f)) {   // this query saw no key in the item
+          if (single) {
+            p.out[row * D + d] = __float2bfloat16_rn(0.f);
+            if (d == 0 && p.lse) p.lse[row] = p.sinks ? p.sinks[hq] : -INFINITY;
+          } else {
+            const size_t prow = row * p.max_splits + hd.split;
+            p.part_o[prow * D + d] = 0.f;
+            if (d == 0) p.part_lse[prow] = -INFINITY;
+          }
+          continue;
+        }
         if (single) {
           float scale = p.v_scale;
           float lse_out = lse2;
@@ -928,7 +1002,7 @@ struct CombineParams {
   const float* part_lse;
   __nv_bfloat16* out;
   float* lse;
-  int B, Hq, bt, max_blocks, window_left, chunk_pages, max_splits;
+  int B, q_len, Hq, bt, max_blocks, window_left, chunk_pages, max_splits;
   int wpr;            // warps per row: 1, 2, 4, 8, 16 or 32
   int rows_per_cta;   // rows per CTA (wpr * rows_per_cta <= 32)
   float v_scale;
@@ -937,7 +1011,7 @@ struct CombineParams {
 constexpr int kCombineMaxThreads = 1024;
 constexpr int kCombineBatch = 8;   // partials a warp loads before it reduces them
 
-// Rows (sequence, query head) whose sequence spans several splits:
+// Rows (sequence, query token, query head) whose sequence spans several splits:
 //   out = v_scale sum_s 2^(lse_s - M) o_s / (sum_s 2^(lse_s - M) + 2^(sigma - M)),
 //   lse = (M + log2 Z) ln 2,  M = max(max_s lse_s, sigma)  (sigma in log2 units).
 // Each row gets `wpr` warps; warp j of a row takes splits j, j + wpr, ...  The
@@ -945,8 +1019,9 @@ constexpr int kCombineBatch = 8;   // partials a warp loads before it reduces th
 // before the split count is known (in bounds: every row owns max_splits
 // partials; entries past the count are never used), so the whole merge costs
 // one round trip to memory.  Each warp reduces against its own maximum; the
-// row's warps are combined in shared memory.
-template <int D>
+// row's warps are combined in shared memory.  MQ: several queries per
+// sequence, where a split may hold no key of a query (its lse is -inf).
+template <int D, bool MQ>
 __global__ void __launch_bounds__(kCombineMaxThreads) fpd_combine_kernel(const CombineParams p) {
   constexpr int kMaxWarps = kCombineMaxThreads / 32;
   __shared__ float acc_sm[kMaxWarps][D];
@@ -957,14 +1032,15 @@ __global__ void __launch_bounds__(kCombineMaxThreads) fpd_combine_kernel(const C
   const int wpr = p.wpr;
   const int row = blockIdx.x * p.rows_per_cta + warp / wpr;
   const int j = warp % wpr;
-  const bool in_range = row < p.B * p.Hq;
+  const int QL = MQ ? p.q_len : 1;   // query tokens per sequence
+  const bool in_range = row < p.B * QL * p.Hq;
   constexpr int PER = D / 32;
   const int ms = p.max_splits;
   const float* pl = p.part_lse + (size_t)(in_range ? row : 0) * ms;
   const float* po = p.part_o + (size_t)(in_range ? row : 0) * ms * D + lane * PER;
 
   // ---- one round of loads: the sequence length and this warp's first batch
-  const int L_raw = in_range ? p.seq_lens[row / p.Hq] : 0;
+  const int L_raw = in_range ? p.seq_lens[row / (QL * p.Hq)] : 0;
   float lv[kCombineBatch];
   float x[kCombineBatch][PER];
 #pragma unroll
@@ -984,8 +1060,9 @@ __global__ void __launch_bounds__(kCombineMaxThreads) fpd_combine_kernel(const C
       }
     }
   }
-  const int ns = seq_range(L_raw, p.bt, p.max_blocks, p.window_left, p.chunk_pages, nullptr)
-                     .n_splits;
+  const int ns =
+      seq_range(L_raw, QL, p.bt, p.max_blocks, p.window_left, p.chunk_pages, nullptr)
+          .n_splits;
   const bool active = in_range && ns > 1;   // rows with one split were written already
 
   // ---- this warp's splits against its own maximum m
@@ -999,7 +1076,8 @@ __global__ void __launch_bounds__(kCombineMaxThreads) fpd_combine_kernel(const C
       if (j + wpr * u < ns) m = fmaxf(m, lv[u]);
 #pragma unroll
     for (int u = 0; u < kCombineBatch; ++u) {
-      if (j + wpr * u < ns) {   // never touch the unused (possibly stale) entries
+      // never touch unused (possibly stale) entries; -inf: no key of the query there
+      if (j + wpr * u < ns && (!MQ || lv[u] != -INFINITY)) {
         const float w = fast_exp2(lv[u] - m);
         z += w;
 #pragma unroll
@@ -1017,7 +1095,8 @@ __global__ void __launch_bounds__(kCombineMaxThreads) fpd_combine_kernel(const C
         const float2 t = *reinterpret_cast<const float2*>(po + (size_t)s * D);
         v[0] = t.x, v[1] = t.y;
       }
-      if (l > m) {   // rescale to the new maximum
+      if (MQ && l == -INFINITY) continue;   // the query saw no key in this split
+      if (l > m) {   // rescale to the new maximum (m = -inf: r = 0)
         const float r = fast_exp2(m - l);
         z *= r;
 #pragma unroll

@@ -91,8 +91,8 @@ class Workload:
         return int(self.attended().sum()) * self.Hkv * self.D * 2
 
     def io_bytes(self) -> int:
-        """q in, out and lse out: B*Hq*(2D + 2D + 4) bytes."""
-        return self.B * self.Hq * (2 * self.D + 2 * self.D + 4)
+        """q in, out and lse out: B*q_len*Hq*(2D + 2D + 4) bytes."""
+        return self.B * self.q_len * self.Hq * (2 * self.D + 2 * self.D + 4)
 
 
 # The five synthetic workloads (shapes, distributions and scales as specified
@@ -259,9 +259,11 @@ def make_custom(*, B: int, Hq: int, Hkv: int, D: int, block_tokens: int,
 
 
 def make_workload(name: str, *, seed: Optional[int] = None, fill: str = "nan",
-                  keep_dense: bool = False, B: Optional[int] = None) -> Workload:
+                  keep_dense: bool = False, B: Optional[int] = None,
+                  q_len: int = 1) -> Workload:
     """One of the five named workloads.  ``B`` may shrink the batch (keeps the
-    first B sequences' length draws)."""
+    first B sequences' length draws); ``q_len`` > 1 gives each sequence that
+    many query tokens (speculative decode of the same shape)."""
     c = CONFIGS[name]
     s = c["seed"] if seed is None else seed
     rng = np.random.default_rng(np.random.SeedSequence([s, 0x5EED]))
@@ -281,4 +283,4 @@ def make_workload(name: str, *, seed: Optional[int] = None, fill: str = "nan",
     return make_custom(B=nb, Hq=c["Hq"], Hkv=c["Hkv"], D=c["D"], block_tokens=bt,
                        seq_lens=lens, window_left=c["window_left"], sinks=c["sinks"],
                        sm_scale=c["sm_scale"], sigma=c["sigma"], seed=s, fill=fill,
-                       keep_dense=keep_dense, max_blocks=max_blocks, name=name)
+                       keep_dense=keep_dense, max_blocks=max_blocks, name=name, q_len=q_len)

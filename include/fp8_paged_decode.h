@@ -161,7 +161,39 @@ fpd_status fp8_paged_decode_attention_ex(const void *q, const void *k_cache, con
                                          int chunk_pages_override);
 
 /*
- * Same as fp8_paged_decode_attention_ex, and additionally records the given
+ * Several query tokens per sequence (speculative / multi-token decode): each
+ * sequence's q_len newest tokens are queries.  Query i sits at position
+ * p = seq_lens[b] - q_len + i, attends causally to the keys up to p and, with
+ * window_left >= 0, only to the window_left keys before p as well; sinks
+ * enter every query's denominator.  A query with p < 0 sees no key (out = 0,
+ * lse = its sink, or -inf).  q_len = 1 is fp8_paged_decode_attention_ex.
+ * (Multi-token decode rows as routed on the FlashInfer PR #5591 page,
+ * "Unsupported" section; MTP decode in the NVFP4 KV-cache serving gist.)
+ *   q    bf16 [B, q_len, Hq, D];  out bf16 [B, q_len, Hq, D];  lse f32 [B, q_len, Hq]
+ *   other arguments as in fp8_paged_decode_attention_ex; seq_lens include the
+ *   q_len new tokens, whose K/V must already be in the cache.
+ * Supported: q_len >= 1 with q_len * (Hq / Hkv) <= 16 (else
+ * FPD_ERR_UNSUPPORTED).  Size the workspace with the _qlen query below.
+ */
+fpd_status fp8_paged_decode_attention_qlen(const void *q, const void *k_cache, const void *v_cache,
+                                           const int32_t *block_table, const int32_t *seq_lens,
+                                           int B, int q_len, int Hq, int Hkv, int D,
+                                           int num_blocks, int block_tokens, int max_blocks,
+                                           float k_scale, float v_scale, float sm_scale,
+                                           int window_left, const float *sinks, void *out,
+                                           float *lse, void *workspace, size_t workspace_bytes,
+                                           void *stream, int chunk_pages_override);
+
+/* The plan and the workspace bytes for q_len query tokens per sequence. */
+fpd_status fp8_paged_decode_plan_qlen(int B, int q_len, int Hq, int Hkv, int D, int block_tokens,
+                                      int max_blocks, int window_left, int chunk_pages_override,
+                                      fpd_plan *plan);
+size_t fp8_paged_decode_workspace_bytes_qlen(int B, int q_len, int Hq, int Hkv, int D,
+                                             int block_tokens, int max_blocks, int window_left,
+                                             int chunk_pages_override);
+
+/*
+ * Same as fp8_paged_decode_attention_qlen, and additionally records the given
  * cudaEvent_t handles (passed as void*, each may be NULL) on `stream`: one
  * before the split kernel, one between the split and combine kernels, one after
  * the combine kernel.  For measuring each kernel's duration with CUDA events on
@@ -169,7 +201,7 @@ fpd_status fp8_paged_decode_attention_ex(const void *q, const void *k_cache, con
  */
 fpd_status fp8_paged_decode_attention_profiled(const void *q, const void *k_cache,
                                                const void *v_cache, const int32_t *block_table,
-                                               const int32_t *seq_lens, int B, int Hq, int Hkv,
+                                               const int32_t *seq_lens, int B, int q_len, int Hq, int Hkv,
                                                int D, int num_blocks, int block_tokens,
                                                int max_blocks, float k_scale, float v_scale,
                                                float sm_scale, int window_left,
