@@ -28,6 +28,7 @@ __all__ = [
     "FPD_OK", "FPD_ERR_INVALID_ARG", "FPD_ERR_UNSUPPORTED", "FPD_ERR_WORKSPACE_TOO_SMALL",
     "FPD_ERR_CUDA", "FPD_DEVERR_SEQ_LEN", "FPD_DEVERR_BLOCK_TABLE", "FPD_DEVERR_TIMEOUT",
     "FpdError", "library_path", "load_library", "fp8_paged_decode_make_plan",
+    "fp8_paged_decode_make_plan_qlen", "FPD_MAX_Q_LEN",
     "fp8_paged_decode_plan", "fp8_paged_decode_workspace_bytes",
     "fp8_paged_decode_workspace_bytes_ex", "fp8_paged_decode_attention_profiled",
     "fp8_paged_decode_attention", "fp8_paged_decode_attention_ex",
@@ -47,6 +48,7 @@ FPD_DEVERR_BLOCK_TABLE = 0x2
 FPD_DEVERR_TIMEOUT = 0x4
 FPD_DEVERR_SLOT = 0x8
 FPD_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
+FPD_MAX_Q_LEN = 64
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_NAME = "libfp8_paged_decode.so"
@@ -56,6 +58,7 @@ _lib = None
 # Every entry point declared in include/fp8_paged_decode.h.
 EXPORTED_SYMBOLS = (
     "fp8_paged_decode_make_plan",
+    "fp8_paged_decode_make_plan_qlen",
     "fp8_paged_decode_plan",
     "fp8_paged_decode_workspace_bytes",
     "fp8_paged_decode_workspace_bytes_ex",
@@ -85,7 +88,8 @@ class fpd_plan(ctypes.Structure):
                 ("heads_per_stage", ctypes.c_int), ("stage_tokens", ctypes.c_int),
                 ("stages", ctypes.c_int), ("header_slots", ctypes.c_int),
                 ("ctas", ctypes.c_int), ("smem_bytes", ctypes.c_int),
-                ("workspace_bytes", ctypes.c_size_t)]
+                ("workspace_bytes", ctypes.c_size_t), ("q_per_item", ctypes.c_int),
+                ("q_chunks", ctypes.c_int)]
 
 
 def library_path() -> str:
@@ -96,6 +100,8 @@ def _bind(lib):
     ci, cf, cz, vp = ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_void_p
     lib.fp8_paged_decode_make_plan.argtypes = [ci] * 10 + [ctypes.POINTER(fpd_plan)]
     lib.fp8_paged_decode_make_plan.restype = ci
+    lib.fp8_paged_decode_make_plan_qlen.argtypes = [ci] * 11 + [ctypes.POINTER(fpd_plan)]
+    lib.fp8_paged_decode_make_plan_qlen.restype = ci
     lib.fp8_paged_decode_plan.argtypes = [ci] * 8 + [ctypes.POINTER(fpd_plan)]
     lib.fp8_paged_decode_plan.restype = ci
     lib.fp8_paged_decode_workspace_bytes.argtypes = [ci] * 7
@@ -176,6 +182,18 @@ def fp8_paged_decode_make_plan(B, Hq, Hkv, D, block_tokens, max_blocks, window_l
         int(B), int(Hq), int(Hkv), int(D), int(block_tokens), int(max_blocks), int(window_left),
         int(num_sms), int(ctas_per_sm), int(chunk_pages_override), ctypes.byref(plan))
     _check(st, "fp8_paged_decode_make_plan")
+    return {f: getattr(plan, f) for f, _ in fpd_plan._fields_}
+
+
+def fp8_paged_decode_make_plan_qlen(B, q_len, Hq, Hkv, D, block_tokens, max_blocks, window_left,
+                                    num_sms, ctas_per_sm, chunk_pages_override=0) -> dict:
+    """Host-only split planner for q_len query tokens per sequence (no CUDA call)."""
+    plan = fpd_plan()
+    st = load_library().fp8_paged_decode_make_plan_qlen(
+        int(B), int(q_len), int(Hq), int(Hkv), int(D), int(block_tokens), int(max_blocks),
+        int(window_left), int(num_sms), int(ctas_per_sm), int(chunk_pages_override),
+        ctypes.byref(plan))
+    _check(st, "fp8_paged_decode_make_plan_qlen")
     return {f: getattr(plan, f) for f, _ in fpd_plan._fields_}
 
 

@@ -32,14 +32,13 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 bool supported_group(int g) { return g == 1 || g == 2 || g == 4 || g == 8 || g == 16; }
 
-// q_len query tokens per sequence: the MMA columns of a KV head are its
-// q_len * g (query token, head) pairs, at most 16 (two n-tiles).
+// q_len query tokens per sequence, 1 .. FPD_MAX_Q_LEN.
 fpd_status validate_shape(int B, int Hq, int Hkv, int D, int bt, int max_blocks, int q_len = 1) {
   if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || bt <= 0 || max_blocks <= 0 || q_len < 1)
     return FPD_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return FPD_ERR_INVALID_ARG;
   if (!supported_group(Hq / Hkv)) return FPD_ERR_UNSUPPORTED;
-  if (q_len * (Hq / Hkv) > 16) return FPD_ERR_UNSUPPORTED;
+  if (q_len > FPD_MAX_Q_LEN) return FPD_ERR_UNSUPPORTED;
   if (D != 64 && D != 128) return FPD_ERR_UNSUPPORTED;
   if (bt != 16 && bt != 32 && bt != 64) return FPD_ERR_UNSUPPORTED;
   if ((int64_t)max_blocks * bt > INT32_MAX) return FPD_ERR_UNSUPPORTED;
@@ -48,6 +47,23 @@ fpd_status validate_shape(int B, int Hq, int Hkv, int D, int bt, int max_blocks,
 
 // MMA n-tiles (8 columns each) for `cols` columns per KV head.
 int n_tiles(int cols) { return cols > 8 ? 2 : 1; }
+
+// Query positions per work item with q_len queries per sequence: a work item's
+// MMA columns are its positions x the g query heads of a KV head, at most
+// FPD_MQ_COLS (8: one n-tile, 16: two).  A sequence's queries are cut into
+// ceil(q_len / P) chunks of near-equal size; each chunk is its own work item
+// over the same KV range (g = 16 always takes one position per item).
+#ifndef FPD_MQ_COLS
+#define FPD_MQ_COLS 16
+#endif
+int q_per_item(int q_len, int g) {
+  if (q_len <= 1) return 1;
+  int P = FPD_MQ_COLS / g;
+  if (P < 1) P = 1;
+  if (P >= q_len) return q_len;
+  const int chunks = (q_len + P - 1) / P;
+  return (q_len + chunks - 1) / chunks;
+}
 
 // KV heads per stage and work item: 4 whenever the KV heads split into groups
 // of 4 (one TMA box then covers 16 tokens of 4 heads), else 1.
@@ -317,7 +333,9 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 void plan_shape(int B, int q_len, int Hq, int Hkv, int D, int bt, int max_blocks,
                 int window_left, int64_t slots, int chunk_pages_override, int HB, fpd_plan* plan) {
   const int g = Hq / Hkv;
-  const int cols = q_len * g;
+  const int qp = q_per_item(q_len, g);
+  const int q_chunks = (q_len + qp - 1) / qp;
+  const int cols = qp * g;   // MMA columns of a work item
   const int NT = n_tiles(cols);
   // with one KV head per stage a stage is 64 tokens of whole pages, and a
   // split must be whole stages; four-head stages are 16 tokens of one page
@@ -327,7 +345,7 @@ void plan_shape(int B, int q_len, int Hq, int Hkv, int D, int bt, int max_blocks
     const int64_t w = ((int64_t)window_left + q_len - 1) / bt + 2;
     if (w < pages_max) pages_max = (int)w;
   }
-  const int64_t units = (int64_t)(B > 0 ? B : 1) * (Hkv / HB);
+  const int64_t units = (int64_t)(B > 0 ? B : 1) * (Hkv / HB) * q_chunks;
   int chunk;
   if (chunk_pages_override > 0) {
     chunk = chunk_pages_override;
@@ -354,6 +372,8 @@ void plan_shape(int B, int q_len, int Hq, int Hkv, int D, int bt, int max_blocks
   plan->smem_bytes = smem_bytes_for(D, cols, HB, B);
   // partial results for each of the B * q_len query tokens
   plan->workspace_bytes = ws_layout(B * q_len, Hq, Hkv, D, max_splits).total;
+  plan->q_per_item = qp;
+  plan->q_chunks = q_chunks;
 }
 
 // Validates and plans.  force_hb = 0 picks the stage shape: four KV heads per
@@ -374,7 +394,7 @@ fpd_status plan_for(int B, int q_len, int Hq, int Hkv, int D, int bt, int max_bl
   plan_shape(B, q_len, Hq, Hkv, D, bt, max_blocks, window_left, slots, chunk_pages_override, HB,
              plan);
   if (force_hb == 0 && HB == 4 && chunk_pages_override == 0 &&
-      (int64_t)(B > 0 ? B : 1) * (Hkv / 4) * plan->max_splits < slots)
+      (int64_t)(B > 0 ? B : 1) * (Hkv / 4) * plan->q_chunks * plan->max_splits < slots)
     plan_shape(B, q_len, Hq, Hkv, D, bt, max_blocks, window_left, slots, 0, 1, plan);
   return FPD_OK;
 }
@@ -386,7 +406,7 @@ fpd_status plan_device(int B, int q_len, int Hq, int Hkv, int D, int bt, int max
   if (!plan) return FPD_ERR_INVALID_ARG;
   fpd_status st = validate_shape(B, Hq, Hkv, D, bt, max_blocks, q_len);
   if (st != FPD_OK) return st;
-  const int cols = q_len * (Hq / Hkv);
+  const int cols = q_per_item(q_len, Hq / Hkv) * (Hq / Hkv);   // MMA columns of a work item
   int HB = heads_per_stage(Hkv), force_hb = 0;
   for (;;) {
     int sms = 0, occ = 0;
@@ -424,6 +444,14 @@ fpd_status fp8_paged_decode_make_plan(int B, int Hq, int Hkv, int D, int bt, int
                                       int window_left, int num_sms, int ctas_per_sm,
                                       int chunk_pages_override, fpd_plan* plan) {
   return plan_for(B, 1, Hq, Hkv, D, bt, max_blocks, window_left, num_sms, ctas_per_sm,
+                  chunk_pages_override, 0, plan);
+}
+
+fpd_status fp8_paged_decode_make_plan_qlen(int B, int q_len, int Hq, int Hkv, int D, int bt,
+                                           int max_blocks, int window_left, int num_sms,
+                                           int ctas_per_sm, int chunk_pages_override,
+                                           fpd_plan* plan) {
+  return plan_for(B, q_len, Hq, Hkv, D, bt, max_blocks, window_left, num_sms, ctas_per_sm,
                   chunk_pages_override, 0, plan);
 }
 
@@ -524,6 +552,8 @@ static fpd_status attention_impl(const void* q, const void* k_cache, const void*
   p.stages = plan.stages;
   p.hdr_slots = plan.header_slots;
   p.q_len = q_len;
+  p.q_per_item = plan.q_per_item;
+  p.q_chunks = plan.q_chunks;
   p.lg = __builtin_ctz((unsigned)g);
   p.qk_scale_log2 = qk * fpd::kLog2e;
   p.v_scale = v_scale;
@@ -531,7 +561,7 @@ static fpd_status attention_impl(const void* q, const void* k_cache, const void*
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (ev0 && cudaEventRecord(static_cast<cudaEvent_t>(ev0), s) != cudaSuccess) return FPD_ERR_CUDA;
   cudaError_t e;
-  const int NT = n_tiles(q_len * g);
+  const int NT = n_tiles(plan.q_per_item * g);
   const bool mq = q_len > 1;
   if (plan.heads_per_stage == 4)
     e = mq ? launch_split_hb<4, true>(D, NT, km, vm, p, plan.ctas, plan.smem_bytes, s)

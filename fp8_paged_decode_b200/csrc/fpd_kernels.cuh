@@ -96,7 +96,9 @@ struct DecodeParams {
   uint32_t* sched;      // workspace words 1, 2: next work item, CTAs finished
   int B, Hq, Hkv, g, bt, max_blocks, num_blocks, window_left;
   int chunk_pages, max_splits, stages, hdr_slots;
-  int q_len;            // query tokens per sequence (columns per KV head: q_len * g)
+  int q_len;            // query tokens per sequence
+  int q_per_item;       // query positions per work item (its columns: q_per_item * g <= 16)
+  int q_chunks;         // work items per (sequence, split, KV head group): ceil(q_len / q_per_item)
   int lg;               // log2(g): g is a power of two
   float qk_scale_log2;  // sm_scale * k_scale * log2(e)
   float v_scale;
@@ -140,8 +142,10 @@ struct ItemHeader {
   int n_stages;  // pipeline stages this item consumes
   int t0;        // token of the first row of the item's first stage
   int tok_lo, tok_hi;
-  int qpos0;     // position of the sequence's first query token (L - q_len)
-  int pad[6];
+  int qpos0;     // position of the item's first query token
+  int qrow0;     // index of that query among the sequence's q_len queries
+  int npos;      // query positions of the item (its columns: npos * g)
+  int pad[4];
 };
 static_assert(sizeof(ItemHeader) == kHdrBytes, "header size");
 
@@ -236,14 +240,14 @@ struct Consumer {
   // column c (query position c / g, head c % g) is row
   // (c / g) * rows_per_pos + w_off + c % g.
   __device__ __forceinline__ void init(const DecodeParams& p, const __nv_bfloat16* qbase,
-                                       int rows_per_pos, int w_off, int lane) {
+                                       int rows_per_pos, int w_off, int ncols, int lane) {
     const int n = lane >> 2, t = lane & 3;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const int c = nt * 8 + n;
       float vals[QW];
       float amax = 0.f;
-      if (c < (MQ ? p.q_len * p.g : p.g)) {
+      if (c < (MQ ? ncols : p.g)) {
         const int qrow = MQ ? (c >> p.lg) * rows_per_pos + w_off + (c & (p.g - 1)) : w_off + c;
         const __nv_bfloat16* src = qbase + qrow * D + t * QW;
 #pragma unroll
@@ -477,9 +481,10 @@ struct Consumer {
   }
   // HB = 4: this warp alone covered KV head `kvh` of the item, so its query
   // heads are finished straight from registers.  Thread (n, t) holds, for
-  // query head nt*8 + 2t + j, the D/8 output elements starting at n*D/8.
+  // column nt*8 + 2t + j, the D/8 output elements starting at n*D/8.  The
+  // item's columns are queries qrow0 .. qrow0 + ncols / g - 1 of the sequence.
   __device__ __forceinline__ void finish_own(const DecodeParams& p, int b, int kvh, int split,
-                                             int ns, int lane) {
+                                             int ns, int qrow0, int ncols, int lane) {
     constexpr int E = D / 8;   // output elements per thread and query head
     const int n = lane >> 2, t = lane & 3;
     float lsum[NT][2];
@@ -498,9 +503,9 @@ struct Consumer {
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         const int c = nt * 8 + 2 * t + j;   // column: query position c / g, head c % g
-        if (c >= (MQ ? p.q_len * p.g : p.g)) continue;
+        if (c >= (MQ ? ncols : p.g)) continue;
         const int hq = kvh * p.g + (MQ ? c & (p.g - 1) : c);
-        const size_t row = MQ ? ((size_t)b * p.q_len + (c >> p.lg)) * p.Hq + hq
+        const size_t row = MQ ? ((size_t)b * p.q_len + qrow0 + (c >> p.lg)) * p.Hq + hq
                               : (size_t)b * p.Hq + hq;
         // false: this query saw no key in the item (only possible with MQ)
         const bool keys = !MQ || lsum[nt][j] > 0.f;
@@ -561,6 +566,7 @@ __device__ __forceinline__ void producer_loop(const CUtensorMap* kmap, const CUt
   const int stages = p.stages;
   const int n_hslots = p.hdr_slots;
   const int QL = MQ ? p.q_len : 1;                 // query tokens per sequence
+  const int QC = MQ ? p.q_chunks : 1;              // query chunks per (group, KV head group)
   const int groups = p.Hkv / HB;                   // KV head groups
   const int pps = HB == 1 ? kStageTokens / p.bt : 1;   // pages per stage (HB = 1)
   const uint32_t page_bytes = (uint32_t)(p.bt * D);
@@ -597,9 +603,13 @@ __device__ __forceinline__ void producer_loop(const CUtensorMap* kmap, const CUt
       }
       return;
     }
-    // item -> (group, kv head group) -> (sequence, split) by binary search
-    const int group = (int)item / groups;
-    const int kvh0 = ((int)item % groups) * HB;
+    // item -> (group, kv head group, query chunk) -> (sequence, split) by
+    // binary search.  The query chunks of one KV range are consecutive items,
+    // so they run at about the same time and share the pages in L2.
+    const int unit = MQ ? (int)item / QC : (int)item;
+    const int qc = MQ ? (int)item - unit * QC : 0;
+    const int group = unit / groups;
+    const int kvh0 = (unit % groups) * HB;
     int lo = 0, hi = p.B;   // largest b with prefix[b] <= group
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
@@ -634,14 +644,18 @@ __device__ __forceinline__ void producer_loop(const CUtensorMap* kmap, const CUt
       hdr->t0 = t0;
       hdr->tok_lo = tok_lo;
       hdr->tok_hi = tok_hi;
-      hdr->qpos0 = R.L - QL;
+      const int qrow0 = MQ ? qc * p.q_per_item : 0;
+      const int npos = MQ ? min(p.q_per_item, QL - qrow0) : 1;
+      hdr->qpos0 = R.L - QL + qrow0;
+      hdr->qrow0 = qrow0;
+      hdr->npos = npos;
       // the query rows of the item's KV heads, one copy per query position:
       // [position][HB * g][D] in the slot
       const uint32_t qbytes = (uint32_t)(HB * p.g * D * 2);
-      mbar_arrive_expect_tx(&hdr_full[hslot], qbytes * (uint32_t)QL);
-      for (int i = 0; i < QL; ++i)
+      mbar_arrive_expect_tx(&hdr_full[hslot], qbytes * (uint32_t)npos);
+      for (int i = 0; i < npos; ++i)
         bulk_load(hbase + kHdrBytes + (size_t)i * qbytes,
-                  p.q + (((size_t)b * QL + i) * p.Hq + (size_t)kvh0 * p.g) * D, qbytes,
+                  p.q + (((size_t)b * QL + qrow0 + i) * p.Hq + (size_t)kvh0 * p.g) * D, qbytes,
                   &hdr_full[hslot]);
     }
     ++hs;
@@ -743,8 +757,9 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
   const int n_hslots = p.hdr_slots;
   // a header slot holds q_len * g query rows per KV head
   const int QL = MQ ? p.q_len : 1;   // query tokens per sequence
-  const SmemLayout L = smem_layout(D, NT, HB, stages, n_hslots, QL * p.g, p.B);
-  const int hslot_bytes = hdr_slot_bytes(D, HB, QL * p.g);
+  const int QP = MQ ? p.q_per_item : 1;   // query positions per item
+  const SmemLayout L = smem_layout(D, NT, HB, stages, n_hslots, QP * p.g, p.B);
+  const int hslot_bytes = hdr_slot_bytes(D, HB, QP * p.g);
   int* prefix = reinterpret_cast<int*>(smem + L.prefix);
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + L.bars);
   uint64_t* empty_bar = full_bar + stages;
@@ -794,7 +809,7 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
     }
     __syncthreads();
   }
-  const int total_items = prefix[p.B] * (p.Hkv / HB);
+  const int total_items = prefix[p.B] * (p.Hkv / HB) * (MQ ? p.q_chunks : 1);
   pdl_launch_dependents();   // the combine kernel may be scheduled from now on
 
   if (warp == kConsumerWarps) {
@@ -826,14 +841,15 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
     const uint8_t* hbase = smem + L.hdr + hslot * hslot_bytes;
     const ItemHeader hd = *reinterpret_cast<const ItemHeader*>(hbase);
     if (hd.kind < 0) break;
+    const int ncols = MQ ? hd.npos * p.g : p.g;   // the item's columns per KV head
     cw.init(p, reinterpret_cast<const __nv_bfloat16*>(hbase + kHdrBytes), HB * p.g,
-            HB == 1 ? 0 : warp * p.g, lane);
+            HB == 1 ? 0 : warp * p.g, ncols, lane);
     // Tiles inside every column's range skip the masks: past the newest key
     // the first query sees, and at or after the oldest key the last query
     // sees (window).  With one query per sequence that is [tok_lo, tok_hi).
-    const TileMask mk{hd.tok_lo, hd.tok_hi, hd.qpos0, p.window_left, p.lg, QL * p.g};
+    const TileMask mk{hd.tok_lo, hd.tok_hi, hd.qpos0, p.window_left, p.lg, ncols};
     const int full_lo = MQ && p.window_left >= 0
-                            ? max(hd.tok_lo, hd.qpos0 + QL - 1 - p.window_left)
+                            ? max(hd.tok_lo, hd.qpos0 + hd.npos - 1 - p.window_left)
                             : hd.tok_lo;
     const int full_hi = MQ ? min(hd.tok_hi, hd.qpos0 + 1) : hd.tok_hi;
     __syncwarp();
@@ -867,7 +883,7 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
     if (!alive) break;
 
     if constexpr (HB != 1) {
-      cw.finish_own(p, hd.b, hd.kvh0 + warp, hd.split, hd.ns, lane);
+      cw.finish_own(p, hd.b, hd.kvh0 + warp, hd.split, hd.ns, hd.qrow0, ncols, lane);
       continue;
     }
 
@@ -908,10 +924,10 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
       constexpr int HPI = kConsumerWarps * 32 / D;
       const int d = tid % D;
 #pragma unroll 4
-      for (int h = tid / D; h < (MQ ? p.q_len * p.g : p.g); h += HPI) {
-        // column h: query position h / g, head h % g
+      for (int h = tid / D; h < ncols; h += HPI) {
+        // column h: query qrow0 + h / g of the sequence, head h % g
         const int hq = hd.kvh0 * p.g + (MQ ? h & (p.g - 1) : h);
-        const size_t row = MQ ? ((size_t)hd.b * p.q_len + (h >> p.lg)) * p.Hq + hq
+        const size_t row = MQ ? ((size_t)hd.b * QL + hd.qrow0 + (h >> p.lg)) * p.Hq + hq
                               : (size_t)hd.b * p.Hq + hq;
         if (hd.ns == 0) {  // empty sequence: out = 0, lse = sigma
           p.out[row * D + d] = __float2bfloat16_rn(0.f);

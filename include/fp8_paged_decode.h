@@ -73,6 +73,8 @@ typedef struct {
     int ctas;               /* grid size of the split kernel */
     int smem_bytes;         /* dynamic shared memory per CTA */
     size_t workspace_bytes; /* bytes this plan needs */
+    int q_per_item;         /* query positions per work item (1 with one query per sequence) */
+    int q_chunks;           /* work items per sequence, KV head group and split: ceil(q_len / q_per_item) */
 } fpd_plan;
 
 /*
@@ -93,6 +95,13 @@ fpd_status fp8_paged_decode_make_plan(int B, int Hq, int Hkv, int D, int block_t
                                       int max_blocks, int window_left, int num_sms,
                                       int ctas_per_sm, int chunk_pages_override,
                                       fpd_plan *plan);
+
+/* The host-only planner for q_len query tokens per sequence (see
+ * fp8_paged_decode_attention_qlen); q_len = 1 is fp8_paged_decode_make_plan. */
+fpd_status fp8_paged_decode_make_plan_qlen(int B, int q_len, int Hq, int Hkv, int D,
+                                           int block_tokens, int max_blocks, int window_left,
+                                           int num_sms, int ctas_per_sm,
+                                           int chunk_pages_override, fpd_plan *plan);
 
 /*
  * The plan fp8_paged_decode_attention_ex uses on the CURRENT device (its SM
@@ -172,9 +181,13 @@ fpd_status fp8_paged_decode_attention_ex(const void *q, const void *k_cache, con
  *   q    bf16 [B, q_len, Hq, D];  out bf16 [B, q_len, Hq, D];  lse f32 [B, q_len, Hq]
  *   other arguments as in fp8_paged_decode_attention_ex; seq_lens include the
  *   q_len new tokens, whose K/V must already be in the cache.
- * Supported: q_len >= 1 with q_len * (Hq / Hkv) <= 16 (else
- * FPD_ERR_UNSUPPORTED).  Size the workspace with the _qlen query below.
+ * Supported: 1 <= q_len <= FPD_MAX_Q_LEN (else FPD_ERR_UNSUPPORTED), any
+ * supported g.  A work item covers the KV range of one split for up to 16 / g
+ * of the sequence's queries (at least one); longer query runs are cut into
+ * several items over the same pages, which then mostly come from L2.  Size the
+ * workspace with the _qlen query below.
  */
+#define FPD_MAX_Q_LEN 64
 fpd_status fp8_paged_decode_attention_qlen(const void *q, const void *k_cache, const void *v_cache,
                                            const int32_t *block_table, const int32_t *seq_lens,
                                            int B, int q_len, int Hq, int Hkv, int D,

@@ -120,6 +120,47 @@ def test_planner_monotone_workspace():
         prev = w
 
 
+def plan_q(q_len, **kw):
+    args = dict(B=32, q_len=q_len, Hq=32, Hkv=8, D=128, block_tokens=16, max_blocks=512,
+                window_left=-1, num_sms=148, ctas_per_sm=2, chunk_pages_override=0)
+    args.update(kw)
+    return fpd.fp8_paged_decode_make_plan_qlen(**args)
+
+
+@pytest.mark.parametrize("g,q_len,per_item,chunks", [
+    (4, 1, 1, 1), (4, 2, 2, 1), (4, 4, 4, 1),      # up to 16 columns: one item per KV range
+    (4, 5, 3, 2), (4, 8, 4, 2),                    # near-equal chunks of <= 4 positions
+    (8, 2, 2, 1), (8, 3, 2, 2), (8, 8, 2, 4),
+    (16, 1, 1, 1), (16, 4, 1, 4),                  # one position per item
+    (1, 16, 16, 1), (1, 17, 9, 2), (2, 64, 8, 8),
+])
+def test_planner_query_chunks(g, q_len, per_item, chunks):
+    p = plan_q(q_len, Hq=8 * g)
+    assert (p["q_per_item"], p["q_chunks"]) == (per_item, chunks)
+    assert p["q_per_item"] * g <= 16 or p["q_per_item"] == 1
+    # the partials cover every (sequence, query, head) row
+    n_rows = 32 * q_len * 8 * g
+    if p["max_splits"] > 1:
+        assert p["workspace_bytes"] == 256 + n_rows * p["max_splits"] * (128 * 4 + 4)
+    # more work items per KV range: no more splits than with one query
+    assert p["max_splits"] <= plan(Hq=8 * g)["max_splits"]
+
+
+def test_planner_q_len_one_is_the_single_query_plan():
+    for shape in [dict(), dict(Hq=64, window_left=4096, block_tokens=32, max_blocks=1024),
+                  dict(Hq=16, Hkv=2)]:
+        assert plan_q(1, **shape) == plan(**shape)
+
+
+def test_planner_q_len_limits():
+    assert plan_q(fpd.FPD_MAX_Q_LEN)["q_chunks"] == fpd.FPD_MAX_Q_LEN * 4 // 16
+    for q_len, status in ((fpd.FPD_MAX_Q_LEN + 1, fpd.FPD_ERR_UNSUPPORTED),
+                          (0, fpd.FPD_ERR_INVALID_ARG)):
+        with pytest.raises(fpd.FpdError) as e:
+            plan_q(q_len)
+        assert e.value.status == status
+
+
 @pytest.mark.parametrize("kw,status", [
     (dict(D=96), fpd.FPD_ERR_UNSUPPORTED),
     (dict(D=256), fpd.FPD_ERR_UNSUPPORTED),

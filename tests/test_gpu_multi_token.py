@@ -46,6 +46,25 @@ def test_grid(gq, Hkv, D, bt):
         check(wl, chunk_pages=1)      # four-head stages, one page per split
 
 
+# more than 16 columns: a sequence's queries are cut into several work items
+GQC = [(1, 17), (2, 9), (4, 5), (4, 8), (8, 3), (8, 8), (16, 2), (16, 3)]
+GRIDC = list(itertools.product(GQC, [2, 4], [64, 128]))
+
+
+@pytest.mark.parametrize("gq,Hkv,D", GRIDC,
+                         ids=[f"g{g}-q{q}-kv{h}-D{d}" for (g, q), h, d in GRIDC])
+def test_query_chunks(gq, Hkv, D):
+    g, Q = gq
+    lens = [1, Q - 1, Q, 2 * Q + 1, 37, 300, 700]
+    wl = W.make_custom(B=len(lens), Hq=g * Hkv, Hkv=Hkv, D=D, block_tokens=16, seq_lens=lens,
+                       seed=500 + g + Q + Hkv + D, sm_scale=1.0 / np.sqrt(D), sinks=True,
+                       q_len=Q)
+    check(wl)
+    check(wl, chunk_pages=2)
+    wl.window_left = 20
+    check(wl, what=f"{wl.name} q_len={Q} window 20")
+
+
 @pytest.mark.parametrize("window", [0, 3, 40, 129, 10 ** 6])
 def test_windows(window):
     for Hkv, Q in ((2, 4), (4, 3)):
@@ -71,9 +90,10 @@ def test_one_query_matches_the_single_query_entry_bitwise():
     assert np.array_equal(a_lse, b_lse[:, 0].cpu().numpy())
 
 
-def test_unsupported_column_count():
-    wl = W.make_custom(B=2, Hq=16, Hkv=2, D=128, block_tokens=16, seq_lens=[40, 50], seed=62,
-                       q_len=3)                       # 3 x 8 = 24 columns
+def test_unsupported_q_len():
+    Q = fpd.FPD_MAX_Q_LEN + 1
+    wl = W.make_custom(B=2, Hq=4, Hkv=2, D=64, block_tokens=16, seq_lens=[70, 80], seed=62,
+                       q_len=Q)
     dev = to_device(wl)
     with pytest.raises(fpd.FpdError) as e:
         fpd.fp8_paged_decode_attention(dev["q"], dev["k_cache"], dev["v_cache"],
