@@ -47,11 +47,18 @@ def _bind(lib):
     lib.fpd_oracle_decode_q.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, ci,
                                         cd, cd, cd, ci, vp, vp, vp, vp, ci, ci]
     lib.fpd_oracle_decode_q.restype = ci
+    lib.fpd_oracle_decode_x.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, ci,
+                                        cd, cd, cd, ci, vp, vp, vp, vp, ci, ci, ci, ci]
+    lib.fpd_oracle_decode_x.restype = ci
+    lib.fpd_oracle_f16_to_f64.argtypes = [ctypes.c_uint16]
+    lib.fpd_oracle_f16_to_f64.restype = ctypes.c_double
     lib.fpd_oracle_f64_to_e4m3.argtypes = [ctypes.c_double]
     lib.fpd_oracle_f64_to_e4m3.restype = ctypes.c_uint8
     lib.fpd_oracle_cache_write.argtypes = [vp, vp, vp, ci, ci, ci, ctypes.c_long, ctypes.c_long,
                                            ctypes.c_float, ctypes.c_float, vp, vp, ci, ci]
     lib.fpd_oracle_cache_write.restype = ci
+    lib.fpd_oracle_cache_write_x.argtypes = lib.fpd_oracle_cache_write.argtypes + [ci]
+    lib.fpd_oracle_cache_write_x.restype = ci
     del u8p
     return lib
 
@@ -78,31 +85,42 @@ def bf16_to_f64(bits: int, lib=None) -> float:
     return (lib or load()).fpd_oracle_bf16_to_f64(int(bits))
 
 
+def f16_to_f64(bits: int, lib=None) -> float:
+    return (lib or load()).fpd_oracle_f16_to_f64(int(bits))
+
+
 def f64_to_e4m3(x: float, lib=None) -> int:
     """Nearest E4M3 code, ties to even, saturating at +-448 (NaN -> S.1111.111)."""
     return int((lib or load()).fpd_oracle_f64_to_e4m3(float(x)))
 
 
-def cache_write(key, value, slot_mapping, k_cache, v_cache, *, k_scale, v_scale, lib=None) -> int:
+def cache_write(key, value, slot_mapping, k_cache, v_cache, *, k_scale, v_scale, lib=None,
+                kv_layout="NHD") -> int:
     """FP8 KV-cache write into ``k_cache``/``v_cache`` (uint8 [num_blocks, bt, Hkv, D],
-    modified in place) of bf16 ``key``/``value`` (uint16 bits [num_tokens, Hkv, D],
-    any token stride) at ``slot_mapping`` (int64 [num_tokens], negative = skip).
-    Returns the number of out-of-range slots (skipped)."""
+    or [num_blocks, Hkv, bt, D] with ``kv_layout="HND"``; modified in place) of
+    bf16 ``key``/``value`` (uint16 bits [num_tokens, Hkv, D], any token stride) at
+    ``slot_mapping`` (int64 [num_tokens], negative = skip).  Returns the number
+    of out-of-range slots (skipped)."""
     lib = lib or load()
     assert key.dtype == np.uint16 and value.dtype == np.uint16
     assert k_cache.dtype == np.uint8 and k_cache.flags.c_contiguous and v_cache.flags.c_contiguous
-    num_blocks, bt, Hkv, D = k_cache.shape
+    assert kv_layout in ("NHD", "HND")
+    if kv_layout == "HND":
+        num_blocks, Hkv, bt, D = k_cache.shape
+    else:
+        num_blocks, bt, Hkv, D = k_cache.shape
     T = key.shape[0]
     assert key.shape[1:] == (Hkv, D) and value.shape[1:] == (Hkv, D)
     for a in (key, value):
         assert a.strides[2] == 2 and a.strides[1] == 2 * D, "rows must be contiguous per token"
     slot_mapping = np.ascontiguousarray(slot_mapping, dtype=np.int64)
     assert slot_mapping.shape == (T,)
-    st = lib.fpd_oracle_cache_write(key.ctypes.data_as(ctypes.c_void_p),
-                                    value.ctypes.data_as(ctypes.c_void_p), _ptr(slot_mapping), T,
-                                    Hkv, D, key.strides[0] // 2, value.strides[0] // 2,
-                                    float(k_scale), float(v_scale), _ptr(k_cache), _ptr(v_cache),
-                                    num_blocks, bt)
+    st = lib.fpd_oracle_cache_write_x(key.ctypes.data_as(ctypes.c_void_p),
+                                      value.ctypes.data_as(ctypes.c_void_p), _ptr(slot_mapping),
+                                      T, Hkv, D, key.strides[0] // 2, value.strides[0] // 2,
+                                      float(k_scale), float(v_scale), _ptr(k_cache),
+                                      _ptr(v_cache), num_blocks, bt,
+                                      1 if kv_layout == "HND" else 0)
     if st < 0:
         raise ValueError("oracle rejected the cache-write arguments")
     return st
@@ -113,13 +131,14 @@ def _ptr(a: Optional[np.ndarray]):
 
 
 def decode(q, k_cache, v_cache, block_table, seq_lens, *, k_scale, v_scale, sm_scale,
-           window_left=-1, sinks=None, rows=None, threads=None, lib=None
-           ) -> Tuple[np.ndarray, np.ndarray]:
+           window_left=-1, sinks=None, rows=None, threads=None, lib=None, q_dtype="bf16",
+           kv_layout="NHD") -> Tuple[np.ndarray, np.ndarray]:
     """fp64 decode attention.
 
-    Arrays are numpy: q uint16 (bf16 bits) [B,Hq,D], or [B,q_len,Hq,D] for
-    q_len query tokens per sequence (positions L - q_len .. L - 1, causal);
-    k/v_cache uint8 E4M3 codes [num_blocks, bt, Hkv, D]; block_table int32
+    Arrays are numpy: q uint16 (bf16 bits, or fp16 bits with ``q_dtype="f16"``)
+    [B,Hq,D], or [B,q_len,Hq,D] for q_len query tokens per sequence (positions
+    L - q_len .. L - 1, causal); k/v_cache uint8 E4M3 codes
+    [num_blocks, bt, Hkv, D] (``kv_layout="HND"``: [num_blocks, Hkv, bt, D]); block_table int32
     [B, max_blocks]; seq_lens int32 [B]; sinks float32 [Hq] or None.  ``rows``
     optionally lists flat ``(b * q_len + i) * Hq + h`` rows to compute (others
     are left NaN).  Returns (out float64 [B, (q_len,) Hq, D], lse float64
@@ -137,7 +156,11 @@ def decode(q, k_cache, v_cache, block_table, seq_lens, *, k_scale, v_scale, sm_s
         Q = 1
     else:
         B, Q, Hq, D = q.shape
-    num_blocks, bt, Hkv, D2 = k_cache.shape
+    assert q_dtype in ("bf16", "f16") and kv_layout in ("NHD", "HND")
+    if kv_layout == "HND":
+        num_blocks, Hkv, bt, D2 = k_cache.shape
+    else:
+        num_blocks, bt, Hkv, D2 = k_cache.shape
     assert D2 == D and v_cache.shape == k_cache.shape
     assert block_table.shape[0] == B and seq_lens.shape == (B,)
     max_blocks = block_table.shape[1]
@@ -153,11 +176,12 @@ def decode(q, k_cache, v_cache, block_table, seq_lens, *, k_scale, v_scale, sm_s
         n_rows = int(rows_arr.size)
     if threads is None:
         threads = os.cpu_count() or 1
-    st = lib.fpd_oracle_decode_q(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+    st = lib.fpd_oracle_decode_x(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
                                  _ptr(seq_lens), B, Q, Hq, Hkv, D, num_blocks, bt, max_blocks,
                                  float(k_scale), float(v_scale), float(sm_scale),
                                  int(window_left), _ptr(sinks), _ptr(out), _ptr(lse),
-                                 _ptr(rows_arr), n_rows, int(threads))
+                                 _ptr(rows_arr), n_rows, int(threads),
+                                 1 if q_dtype == "f16" else 0, 1 if kv_layout == "HND" else 0)
     if st != 0:
         raise ValueError(f"oracle rejected the inputs (status {st})")
     return out, lse

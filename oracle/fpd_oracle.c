@@ -46,6 +46,12 @@
  * start_i = max(0, p - window_left) under a window; q, out and lse gain a
  * q_len axis after B.  q_len = 1 is the formula above.
  *
+ * Interface variants (the layouts and forms the gist's FlashInfer backend and
+ * cache writer use): the query may be IEEE fp16 instead of bf16, and the
+ * pages may be head-major, [num_blocks, Hkv, bt, D] ("HND"), instead of
+ * token-major [num_blocks, bt, Hkv, D] ("NHD"); only the addressing of
+ * element [page][slot][kvh][d] changes.
+ *
  * Degenerate cases: L == 0 gives out = 0 and lse = sigma (-inf without sinks).
  * A stored NaN code inside the attended range propagates NaN (plain
  * arithmetic); codes outside the attended range are never read.
@@ -79,6 +85,29 @@ double fpd_oracle_bf16_to_f64(uint16_t bits)
     float f;
     memcpy(&f, &u, sizeof f);
     return (double)f;
+}
+
+/* IEEE binary16 bit pattern -> real value: 1 sign, 5 exponent (bias 15), 10
+ * mantissa bits; exponent 0 is subnormal (2^-14 * m / 1024); exponent 31 is
+ * inf (m = 0) or NaN. */
+double fpd_oracle_f16_to_f64(uint16_t bits)
+{
+    const int s = bits >> 15, e = (bits >> 10) & 0x1F, m = bits & 0x3FF;
+    const double sign = s ? -1.0 : 1.0;
+    if (e == 0x1F)
+        return m ? NAN : sign * INFINITY;
+    if (e == 0)
+        return sign * ldexp((double)m / 1024.0, -14);
+    return sign * ldexp(1.0 + (double)m / 1024.0, e - 15);
+}
+
+/* Byte offset of element [page][slot][kvh][0]: token-major pages
+ * [num_blocks, bt, Hkv, D], or head-major [num_blocks, Hkv, bt, D] (hnd). */
+static size_t page_row(int hnd, int page, int slot, int kvh, int bt, int Hkv, int D)
+{
+    if (hnd)
+        return (((size_t)page * Hkv + kvh) * bt + slot) * (size_t)D;
+    return (((size_t)page * bt + slot) * Hkv + kvh) * (size_t)D;
 }
 
 /*
@@ -118,13 +147,14 @@ uint8_t fpd_oracle_f64_to_e4m3(double x)
  * goes to slot s = slot_mapping[t] = page * bt + offset of the
  * [num_blocks, bt, Hkv, D] caches; a negative slot is a padded token and is
  * skipped.  key and value are bf16 bit patterns [num_tokens, Hkv, D] with a
- * token stride of key_stride / value_stride elements.  Returns the number of
- * slots past the end of the cache (skipped), or -1 for a bad argument.
+ * token stride of key_stride / value_stride elements.  hnd selects head-major
+ * pages [num_blocks, Hkv, bt, D].  Returns the number of slots past the end of
+ * the cache (skipped), or -1 for a bad argument.
  */
-int fpd_oracle_cache_write(const uint16_t *key, const uint16_t *value, const int64_t *slot_mapping,
-                           int num_tokens, int Hkv, int D, long key_stride, long value_stride,
-                           float k_scale, float v_scale, uint8_t *k_cache, uint8_t *v_cache,
-                           int num_blocks, int bt)
+int fpd_oracle_cache_write_x(const uint16_t *key, const uint16_t *value,
+                             const int64_t *slot_mapping, int num_tokens, int Hkv, int D,
+                             long key_stride, long value_stride, float k_scale, float v_scale,
+                             uint8_t *k_cache, uint8_t *v_cache, int num_blocks, int bt, int hnd)
 {
     const float kr = 1.0f / k_scale, vr = 1.0f / v_scale;
     const int64_t n_slots = (int64_t)num_blocks * bt;
@@ -141,7 +171,8 @@ int fpd_oracle_cache_write(const uint16_t *key, const uint16_t *value, const int
         }
         for (h = 0; h < Hkv; ++h) {
             for (d = 0; d < D; ++d) {
-                const size_t dst = ((size_t)slot * Hkv + h) * (size_t)D + d;
+                const size_t dst =
+                    page_row(hnd, (int)(slot / bt), (int)(slot % bt), h, bt, Hkv, D) + d;
                 const float xk = (float)fpd_oracle_bf16_to_f64(key[t * key_stride + (long)h * D + d]);
                 const float xv = (float)fpd_oracle_bf16_to_f64(value[t * value_stride + (long)h * D + d]);
                 const float yk = xk * kr, yv = xv * vr; /* fp32 products, round to nearest */
@@ -153,6 +184,17 @@ int fpd_oracle_cache_write(const uint16_t *key, const uint16_t *value, const int
     return bad;
 }
 
+/* Token-major pages (the default layout). */
+int fpd_oracle_cache_write(const uint16_t *key, const uint16_t *value, const int64_t *slot_mapping,
+                           int num_tokens, int Hkv, int D, long key_stride, long value_stride,
+                           float k_scale, float v_scale, uint8_t *k_cache, uint8_t *v_cache,
+                           int num_blocks, int bt)
+{
+    return fpd_oracle_cache_write_x(key, value, slot_mapping, num_tokens, Hkv, D, key_stride,
+                                    value_stride, k_scale, v_scale, k_cache, v_cache,
+                                    num_blocks, bt, 0);
+}
+
 typedef struct {
     const uint16_t *q;
     const uint8_t *k_cache, *v_cache;
@@ -160,6 +202,8 @@ typedef struct {
     int B, Hq, Hkv, D, num_blocks, bt, max_blocks, q_len;
     double k_scale, v_scale, sm_scale;
     int window_left;
+    int q_f16;           /* q holds IEEE fp16 bit patterns instead of bf16 */
+    int kv_hnd;          /* head-major pages [num_blocks, Hkv, bt, D] */
     const float *sinks;
     double *out, *lse;
     const int32_t *rows; /* list of (b * q_len + i) * Hq + h to compute, or NULL for all */
@@ -169,10 +213,15 @@ typedef struct {
     pthread_mutex_t mu;
 } job_t;
 
-/* Byte offset of element [page][slot][kvh][0] in a [num_blocks, bt, Hkv, D] cache. */
+/* Byte offset of element [page][slot][kvh][0] in the job's cache layout. */
 static size_t cache_row(const job_t *J, int page, int slot, int kvh)
 {
-    return (((size_t)page * J->bt + slot) * J->Hkv + kvh) * (size_t)J->D;
+    return page_row(J->kv_hnd, page, slot, kvh, J->bt, J->Hkv, J->D);
+}
+
+static double q_value(const job_t *J, uint16_t bits)
+{
+    return J->q_f16 ? fpd_oracle_f16_to_f64(bits) : fpd_oracle_bf16_to_f64(bits);
 }
 
 static int one_row(const job_t *J, int row, double *s, double *acc)
@@ -207,7 +256,7 @@ static int one_row(const job_t *J, int row, double *s, double *acc)
             return -3;
         kr = J->k_cache + cache_row(J, page, j % J->bt, kvh);
         for (d = 0; d < D; ++d)
-            dot += fpd_oracle_bf16_to_f64(qr[d]) * (J->k_scale * fpd_oracle_e4m3_to_f64(kr[d]));
+            dot += q_value(J, qr[d]) * (J->k_scale * fpd_oracle_e4m3_to_f64(kr[d]));
         s[j - start] = J->sm_scale * dot;
         if (s[j - start] > m || isnan(s[j - start]))
             m = s[j - start];
@@ -276,15 +325,17 @@ static void *worker(void *arg)
  *   lse          double [B * q_len * Hq]
  *   rows/n_rows  rows ((b * q_len + i) * Hq + h) to compute; NULL computes all.
  *   n_threads    worker threads (<= 0: 1)
+ *   q_f16        q holds IEEE fp16 bit patterns instead of bf16
+ *   kv_hnd       the caches are head-major [num_blocks, Hkv, bt, D]
  * Returns 0, -1 for bad shapes, -2 for a sequence length outside
  * [0, max_blocks * bt], -3 for a block-table entry outside [0, num_blocks).
  */
-int fpd_oracle_decode_q(const uint16_t *q, const uint8_t *k_cache, const uint8_t *v_cache,
+int fpd_oracle_decode_x(const uint16_t *q, const uint8_t *k_cache, const uint8_t *v_cache,
                         const int32_t *block_table, const int32_t *seq_lens,
                         int B, int q_len, int Hq, int Hkv, int D, int num_blocks, int bt,
                         int max_blocks, double k_scale, double v_scale, double sm_scale,
                         int window_left, const float *sinks, double *out, double *lse,
-                        const int32_t *rows, int n_rows, int n_threads)
+                        const int32_t *rows, int n_rows, int n_threads, int q_f16, int kv_hnd)
 {
     job_t J;
     pthread_t *th;
@@ -304,6 +355,7 @@ int fpd_oracle_decode_q(const uint16_t *q, const uint8_t *k_cache, const uint8_t
     J.max_blocks = max_blocks; J.q_len = q_len;
     J.k_scale = k_scale; J.v_scale = v_scale; J.sm_scale = sm_scale;
     J.window_left = window_left; J.sinks = sinks; J.out = out; J.lse = lse;
+    J.q_f16 = q_f16; J.kv_hnd = kv_hnd;
     J.rows = rows; J.n_rows = n_rows;
     pthread_mutex_init(&J.mu, NULL);
     if (n_threads < 1)
@@ -316,6 +368,19 @@ int fpd_oracle_decode_q(const uint16_t *q, const uint8_t *k_cache, const uint8_t
     free(th);
     pthread_mutex_destroy(&J.mu);
     return J.status;
+}
+
+/* bf16 q, token-major pages. */
+int fpd_oracle_decode_q(const uint16_t *q, const uint8_t *k_cache, const uint8_t *v_cache,
+                        const int32_t *block_table, const int32_t *seq_lens,
+                        int B, int q_len, int Hq, int Hkv, int D, int num_blocks, int bt,
+                        int max_blocks, double k_scale, double v_scale, double sm_scale,
+                        int window_left, const float *sinks, double *out, double *lse,
+                        const int32_t *rows, int n_rows, int n_threads)
+{
+    return fpd_oracle_decode_x(q, k_cache, v_cache, block_table, seq_lens, B, q_len, Hq, Hkv,
+                               D, num_blocks, bt, max_blocks, k_scale, v_scale, sm_scale,
+                               window_left, sinks, out, lse, rows, n_rows, n_threads, 0, 0);
 }
 
 /* One query token per sequence: q bf16 bits [B, Hq, D]. */

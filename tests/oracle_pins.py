@@ -43,19 +43,25 @@ def bf16_library(bits: np.ndarray) -> np.ndarray:
     return t.to(torch.float64).numpy()
 
 
+def f16_library(bits: np.ndarray) -> np.ndarray:
+    """IEEE fp16 bit patterns -> float64 by numpy's float16 (library routine)."""
+    return np.ascontiguousarray(bits, dtype=np.uint16).view(np.float16).astype(np.float64)
+
+
 def run(lib, wl, **kw):
     return oracle.decode_workload(wl, lib=lib, threads=4, **kw)
 
 
-def library_attention(wl):
+def library_attention(wl, qf=None):
     """Dense attention from the generator's per-sequence dense codes, by torch SDPA
-    (out) and scipy logsumexp (lse), in float64."""
+    (out) and scipy logsumexp (lse), in float64.  qf: the query values (default:
+    wl.q decoded as bf16)."""
     assert wl.k_dense is not None
     B, Hq, Hkv, D = wl.B, wl.Hq, wl.Hkv, wl.D
     g = Hq // Hkv
     out = np.zeros((B, Hq, D))
     lse = np.zeros((B, Hq))
-    qf = bf16_library(wl.q)
+    qf = bf16_library(wl.q) if qf is None else qf
     for b in range(B):
         L = int(wl.seq_lens[b])
         start = max(0, L - 1 - wl.window_left) if wl.window_left >= 0 else 0
@@ -465,7 +471,79 @@ def pin_cache_write_invariants(lib):
     assert np.array_equal(back, exact)
 
 
+# ---------------------------------------------------- interface variants --
+
+def pin_f16_codes(lib):
+    """All 65536 fp16 bit patterns against numpy's float16 (NaN as NaN)."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    want = f16_library(bits)
+    got = np.array([lib.fpd_oracle_f16_to_f64(int(b)) for b in bits])
+    nan = np.isnan(want)
+    assert np.array_equal(np.isnan(got), nan), "fp16 NaN patterns differ"
+    assert np.array_equal(got[~nan], want[~nan]), "fp16 decode differs from numpy float16"
+
+
+def pin_f16_query_library(lib):
+    """An fp16 query against torch SDPA / scipy logsumexp on the same values."""
+    for wl in small_cases()[:4]:
+        rng = np.random.default_rng(61)
+        q16 = (rng.standard_normal(wl.q.shape) * 3.0).astype(np.float16)
+        q16.reshape(-1)[::7] *= np.float16(1e-3)         # small and subnormal-range values
+        bits = q16.view(np.uint16)
+        out, lse = oracle.decode(bits, wl.k_cache, wl.v_cache, wl.block_table, wl.seq_lens,
+                                 k_scale=wl.k_scale, v_scale=wl.v_scale, sm_scale=wl.sm_scale,
+                                 window_left=wl.window_left, sinks=wl.sinks, lib=lib, threads=2,
+                                 q_dtype="f16")
+        ref_out, ref_lse = library_attention(wl, qf=f16_library(bits))
+        close(out, ref_out, rtol=1e-10, atol=1e-12, what=f"{wl.name} fp16-q out")
+        close(lse, ref_lse, rtol=1e-12, atol=1e-12, what=f"{wl.name} fp16-q lse")
+
+
+def to_hnd(cache: np.ndarray) -> np.ndarray:
+    """[num_blocks, bt, Hkv, D] -> [num_blocks, Hkv, bt, D] (numpy transpose)."""
+    return np.ascontiguousarray(cache.transpose(0, 2, 1, 3))
+
+
+def pin_hnd_layout(lib):
+    """Head-major pages hold the same elements at other addresses: decoding the
+    transposed caches as HND equals the token-major decode bitwise, for one and
+    several queries; and the cache write into HND pages equals the token-major
+    write transposed."""
+    cases = small_cases()
+    cases.append(W.make_custom(B=3, Hq=8, Hkv=4, D=64, block_tokens=32, seq_lens=[3, 40, 99],
+                               sinks=True, window_left=10, seed=62, q_len=3))
+    for wl in cases:
+        kw = dict(k_scale=wl.k_scale, v_scale=wl.v_scale, sm_scale=wl.sm_scale,
+                  window_left=wl.window_left, sinks=wl.sinks, lib=lib, threads=2)
+        o1, l1 = oracle.decode(wl.q, wl.k_cache, wl.v_cache, wl.block_table, wl.seq_lens, **kw)
+        o2, l2 = oracle.decode(wl.q, to_hnd(wl.k_cache), to_hnd(wl.v_cache), wl.block_table,
+                               wl.seq_lens, kv_layout="HND", **kw)
+        assert np.array_equal(o1, o2, equal_nan=True) and np.array_equal(l1, l2, equal_nan=True), \
+            f"{wl.name}: HND decode differs from the token-major decode"
+    rng = np.random.default_rng(63)
+    T, Hkv, D, bt, nb = 40, 2, 64, 16, 4
+    key = bf16_bits_of(rng.standard_normal((T, Hkv, D)))
+    value = bf16_bits_of(rng.standard_normal((T, Hkv, D)))
+    slots = rng.permutation(nb * bt)[:T].astype(np.int64)
+    slots[::9] = -1
+    kc = rng.integers(0, 256, (nb, bt, Hkv, D), dtype=np.uint8)
+    vc = rng.integers(0, 256, (nb, bt, Hkv, D), dtype=np.uint8)
+    kh, vh = to_hnd(kc), to_hnd(vc)
+    oracle.cache_write(key, value, slots, kc, vc, k_scale=0.02, v_scale=0.01, lib=lib)
+    oracle.cache_write(key, value, slots, kh, vh, k_scale=0.02, v_scale=0.01, lib=lib,
+                       kv_layout="HND")
+    assert np.array_equal(kh, to_hnd(kc)) and np.array_equal(vh, to_hnd(vc)), \
+        "HND cache write differs from the token-major write"
+
+
+def bf16_bits_of(x: np.ndarray) -> np.ndarray:
+    """float -> bf16 bit patterns by torch's bfloat16 cast (round to nearest even)."""
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
 ALL_PINS = [pin_e4m3_codes, pin_bf16, pin_library_attention, pin_zero_keys, pin_window_zero,
             pin_constant_values, pin_invariants, pin_softmax_identity, pin_e4m3_encode_library,
             pin_e4m3_encode_closed, pin_cache_write_library, pin_cache_write_invariants,
-            pin_multi_token_library, pin_multi_token_prefix]
+            pin_multi_token_library, pin_multi_token_prefix, pin_f16_codes,
+            pin_f16_query_library, pin_hnd_layout]

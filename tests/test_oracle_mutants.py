@@ -25,8 +25,15 @@ MUTANTS = {
     "E4M3 mantissa step": [("1.0 + (double)mant / 8.0", "1.0 + (double)mant / 16.0")],
     "E4M3 sign ignored": [("return sign ? -mag : mag;", "return mag;")],
     "cache read head-major (transposed operand)": [
-        ("(((size_t)page * J->bt + slot) * J->Hkv + kvh) * (size_t)J->D",
-         "(((size_t)page * J->Hkv + kvh) * J->bt + slot) * (size_t)J->D")],
+        ("return page_row(J->kv_hnd, page", "return page_row(!J->kv_hnd, page")],
+    "HND pages addressed token-major": [
+        ("        return (((size_t)page * Hkv + kvh) * bt + slot) * (size_t)D;\n",
+         "        return (((size_t)page * bt + slot) * Hkv + kvh) * (size_t)D;\n")],
+    "fp16 exponent bias 16": [("(1.0 + (double)m / 1024.0, e - 15)",
+                               "(1.0 + (double)m / 1024.0, e - 16)")],
+    "fp16 subnormal scale": [("ldexp((double)m / 1024.0, -14)", "ldexp((double)m / 1024.0, -15)")],
+    "fp16 query decoded as bf16": [("return J->q_f16 ? fpd_oracle_f16_to_f64(bits) :",
+                                    "return 0 ? fpd_oracle_f16_to_f64(bits) :")],
     "in-page slot reversed": [("j % J->bt, kvh)", "J->bt - 1 - j % J->bt, kvh)")],
     "block table ignored": [
         ("const int page = J->block_table[(size_t)b * J->max_blocks + j / J->bt];",
@@ -55,8 +62,7 @@ MUTANTS = {
     "writer swaps K and V scales": [("const float kr = 1.0f / k_scale, vr = 1.0f / v_scale;",
                                      "const float kr = 1.0f / v_scale, vr = 1.0f / k_scale;")],
     "writer cache head-major (transposed operand)": [
-        ("const size_t dst = ((size_t)slot * Hkv + h) * (size_t)D + d;",
-         "const size_t dst = (((size_t)(slot / bt) * Hkv + h) * bt + slot % bt) * (size_t)D + d;")],
+        ("page_row(hnd, (int)(slot / bt)", "page_row(!hnd, (int)(slot / bt)")],
     "writer value read with the key stride": [("value[t * value_stride + (long)h * D + d]",
                                                "value[t * key_stride + (long)h * D + d]")],
     "last key dropped": [("for (j = start; j < end; ++j) {\n        const int page = J->block_table"
