@@ -28,7 +28,8 @@ __all__ = [
     "FPD_OK", "FPD_ERR_INVALID_ARG", "FPD_ERR_UNSUPPORTED", "FPD_ERR_WORKSPACE_TOO_SMALL",
     "FPD_ERR_CUDA", "FPD_DEVERR_SEQ_LEN", "FPD_DEVERR_BLOCK_TABLE", "FPD_DEVERR_TIMEOUT",
     "FpdError", "library_path", "load_library", "fp8_paged_decode_make_plan",
-    "fp8_paged_decode_make_plan_qlen", "FPD_MAX_Q_LEN",
+    "fp8_paged_decode_make_plan_qlen", "FPD_MAX_Q_LEN", "FPD_KV_NHD", "FPD_KV_HND",
+    "FPD_Q_BF16", "FPD_Q_F16", "fpd_decode_args", "fp8_paged_decode_cache_write_layout",
     "fp8_paged_decode_plan", "fp8_paged_decode_workspace_bytes",
     "fp8_paged_decode_workspace_bytes_ex", "fp8_paged_decode_attention_profiled",
     "fp8_paged_decode_attention", "fp8_paged_decode_attention_ex",
@@ -49,6 +50,10 @@ FPD_DEVERR_TIMEOUT = 0x4
 FPD_DEVERR_SLOT = 0x8
 FPD_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 FPD_MAX_Q_LEN = 64
+FPD_KV_NHD = 0
+FPD_KV_HND = 1
+FPD_Q_BF16 = 0
+FPD_Q_F16 = 1
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_NAME = "libfp8_paged_decode.so"
@@ -70,6 +75,8 @@ EXPORTED_SYMBOLS = (
     "fp8_paged_decode_workspace_init",
     "fp8_paged_decode_cache_write",
     "fp8_paged_decode_attention_qlen",
+    "fp8_paged_decode_attention_args",
+    "fp8_paged_decode_cache_write_layout",
     "fp8_paged_decode_plan_qlen",
     "fp8_paged_decode_workspace_bytes_qlen",
     "fp8_paged_decode_status_string",
@@ -90,6 +97,24 @@ class fpd_plan(ctypes.Structure):
                 ("ctas", ctypes.c_int), ("smem_bytes", ctypes.c_int),
                 ("workspace_bytes", ctypes.c_size_t), ("q_per_item", ctypes.c_int),
                 ("q_chunks", ctypes.c_int)]
+
+
+class fpd_decode_args(ctypes.Structure):
+    """Mirror of the C struct fpd_decode_args (field order and types)."""
+    _fields_ = [("q", ctypes.c_void_p), ("q_dtype", ctypes.c_int),
+                ("q_token_stride", ctypes.c_int64),
+                ("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p),
+                ("kv_layout", ctypes.c_int),
+                ("block_table", ctypes.c_void_p), ("seq_lens", ctypes.c_void_p),
+                ("B", ctypes.c_int), ("q_len", ctypes.c_int), ("Hq", ctypes.c_int),
+                ("Hkv", ctypes.c_int), ("D", ctypes.c_int), ("num_blocks", ctypes.c_int),
+                ("block_tokens", ctypes.c_int), ("max_blocks", ctypes.c_int),
+                ("k_scale", ctypes.c_float), ("v_scale", ctypes.c_float),
+                ("k_scale_dev", ctypes.c_void_p), ("v_scale_dev", ctypes.c_void_p),
+                ("sm_scale", ctypes.c_float), ("window_left", ctypes.c_int),
+                ("sinks", ctypes.c_void_p), ("out", ctypes.c_void_p),
+                ("out_token_stride", ctypes.c_int64), ("lse", ctypes.c_void_p),
+                ("chunk_pages_override", ctypes.c_int)]
 
 
 def library_path() -> str:
@@ -118,6 +143,8 @@ def _bind(lib):
     lib.fp8_paged_decode_attention_noalloc.argtypes = attn[:19] + [vp]
     lib.fp8_paged_decode_attention_qlen.argtypes = attn[:6] + [ci] + attn[6:] + [ci]
     lib.fp8_paged_decode_attention_qlen.restype = ci
+    lib.fp8_paged_decode_attention_args.argtypes = [ctypes.POINTER(fpd_decode_args), vp, cz, vp]
+    lib.fp8_paged_decode_attention_args.restype = ci
     lib.fp8_paged_decode_plan_qlen.argtypes = [ci] * 9 + [ctypes.POINTER(fpd_plan)]
     lib.fp8_paged_decode_plan_qlen.restype = ci
     lib.fp8_paged_decode_workspace_bytes_qlen.argtypes = [ci] * 9
@@ -128,6 +155,9 @@ def _bind(lib):
     lib.fp8_paged_decode_cache_write.argtypes = [vp, vp, vp, ci, ci, ci, ctypes.c_int64,
                                                  ctypes.c_int64, cf, cf, vp, vp, ci, ci, vp, vp]
     lib.fp8_paged_decode_cache_write.restype = ci
+    lib.fp8_paged_decode_cache_write_layout.argtypes = (
+        lib.fp8_paged_decode_cache_write.argtypes[:14] + [ci, vp, vp])
+    lib.fp8_paged_decode_cache_write_layout.restype = ci
     lib.fp8_paged_decode_workspace_init.argtypes = [vp, cz, vp]
     lib.fp8_paged_decode_workspace_init.restype = ci
     lib.fp8_paged_decode_status_string.argtypes = [ci]
@@ -260,17 +290,51 @@ def _dev_ptr(t, name, dtypes, shape=None):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _token_rows(t, name, lead, Hq, D):
+    """Element stride between consecutive query tokens of a [*lead, Hq, D] view
+    whose (Hq, D) rows are contiguous; raises otherwise."""
+    if tuple(t.shape) != tuple(lead) + (Hq, D):
+        raise ValueError(f"{name} must have shape {tuple(lead) + (Hq, D)}, got {tuple(t.shape)}")
+    if (D > 1 and t.stride(-1) != 1) or (Hq > 1 and t.stride(-2) != D):
+        raise ValueError(f"{name} must have contiguous [Hq, D] rows")
+    if len(lead) == 1:
+        return t.stride(0) if lead[0] > 1 else Hq * D
+    B, Q = lead
+    if Q == 1:
+        return t.stride(0) if B > 1 else Hq * D
+    tok = t.stride(1)
+    if B > 1 and t.stride(0) != Q * tok:
+        raise ValueError(f"{name}: the query tokens of all sequences must be equally spaced")
+    return tok
+
+
+def _scale_arg(x, name):
+    """(host value, device pointer) of a scale given as a number or a CUDA tensor."""
+    import torch
+    if isinstance(x, torch.Tensor):
+        if not x.is_cuda or x.dtype != torch.float32 or x.numel() != 1:
+            raise TypeError(f"{name} as a tensor must be one float32 on the GPU")
+        return 1.0, ctypes.c_void_p(x.data_ptr())
+    return float(x), None
+
+
 def fp8_paged_decode_attention(q, k_cache, v_cache, block_table, seq_lens, k_scale, v_scale,
                                sm_scale, window_left=-1, sinks=None, out=None, lse=None,
                                workspace=None, stream=None, chunk_pages_override=0,
-                               return_lse=True):
+                               return_lse=True, kv_layout="NHD"):
     """Enqueue one decode call on ``stream`` (default: torch's current stream).
 
     ``q`` is [B, Hq, D] (one query token per sequence) or [B, q_len, Hq, D]
-    (the q_len newest tokens of each sequence, causal); ``out``/``lse`` take
-    q's leading shape.  Allocates ``out``/``lse``/``workspace`` with torch when
-    not given (pass them in to keep a call allocation-free).  Returns
-    ``(out, lse)``.
+    (the q_len newest tokens of each sequence, causal), bf16 or fp16; its
+    [Hq, D] rows must be contiguous, the tokens may be spaced further apart
+    (a slice of a fused QKV buffer).  ``out`` (bf16, q's shape, same rule) and
+    ``lse`` (float32, contiguous) are allocated when not given.  The caches are
+    E4M3 (uint8 or float8_e4m3fn) [num_blocks, block_tokens, Hkv, D], or
+    [num_blocks, Hkv, block_tokens, D] with ``kv_layout="HND"``.  ``k_scale`` /
+    ``v_scale`` are numbers or one-element float32 CUDA tensors (read on the
+    GPU when the call runs, e.g. for CUDA-graph replay with new scales).
+    Allocates ``out``/``lse``/``workspace`` with torch when not given (pass
+    them in to keep a call allocation-free).  Returns ``(out, lse)``.
     """
     import torch
     if q.dim() == 3:
@@ -279,7 +343,12 @@ def fp8_paged_decode_attention(q, k_cache, v_cache, block_table, seq_lens, k_sca
     else:
         B, q_len, Hq, D = q.shape
     lead = tuple(q.shape[:-2])
-    num_blocks, bt, Hkv, D2 = k_cache.shape
+    if kv_layout not in ("NHD", "HND"):
+        raise ValueError("kv_layout must be 'NHD' or 'HND'")
+    if kv_layout == "HND":
+        num_blocks, Hkv, bt, D2 = k_cache.shape
+    else:
+        num_blocks, bt, Hkv, D2 = k_cache.shape
     if D2 != D:
         raise ValueError("q and the caches disagree on head_dim")
     max_blocks = block_table.shape[1]
@@ -296,21 +365,39 @@ def fp8_paged_decode_attention(q, k_cache, v_cache, block_table, seq_lens, k_sca
                                        chunk_pages_override)
             raise FpdError(FPD_ERR_UNSUPPORTED, "fp8_paged_decode_workspace_bytes")
         workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)
+    for name, t in (("q", q), ("out", out)):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda:
+            raise TypeError(f"{name} must be a CUDA tensor")
+    if q.dtype not in (torch.bfloat16, torch.float16):
+        raise TypeError("q must be bf16 or fp16")
+    if out.dtype != torch.bfloat16:
+        raise TypeError("out must be bf16")
+    a = fpd_decode_args()
+    a.q = q.data_ptr()
+    a.q_dtype = FPD_Q_F16 if q.dtype == torch.float16 else FPD_Q_BF16
+    a.q_token_stride = _token_rows(q, "q", lead, Hq, D)
     kv_types = (torch.uint8, torch.float8_e4m3fn)
-    st = load_library().fp8_paged_decode_attention_qlen(
-        _dev_ptr(q, "q", (torch.bfloat16,), lead + (Hq, D)),
-        _dev_ptr(k_cache, "k_cache", kv_types),
-        _dev_ptr(v_cache, "v_cache", kv_types, tuple(k_cache.shape)),
-        _dev_ptr(block_table, "block_table", (torch.int32,), (B, max_blocks)),
-        _dev_ptr(seq_lens, "seq_lens", (torch.int32,), (B,)),
-        B, q_len, Hq, Hkv, D, num_blocks, bt, max_blocks,
-        float(k_scale), float(v_scale), float(sm_scale), int(window_left),
-        _dev_ptr(sinks, "sinks", (torch.float32,), (Hq,)),
-        _dev_ptr(out, "out", (torch.bfloat16,), lead + (Hq, D)),
-        _dev_ptr(lse, "lse", (torch.float32,), lead + (Hq,)),
-        _dev_ptr(workspace, "workspace", (torch.uint8,)),
-        ctypes.c_size_t(workspace.numel()),
-        _stream_handle(stream), int(chunk_pages_override))
+    a.k_cache = _dev_ptr(k_cache, "k_cache", kv_types).value
+    a.v_cache = _dev_ptr(v_cache, "v_cache", kv_types, tuple(k_cache.shape)).value
+    a.kv_layout = FPD_KV_HND if kv_layout == "HND" else FPD_KV_NHD
+    a.block_table = _dev_ptr(block_table, "block_table", (torch.int32,), (B, max_blocks)).value
+    a.seq_lens = _dev_ptr(seq_lens, "seq_lens", (torch.int32,), (B,)).value
+    a.B, a.q_len, a.Hq, a.Hkv, a.D = B, q_len, Hq, Hkv, D
+    a.num_blocks, a.block_tokens, a.max_blocks = num_blocks, bt, max_blocks
+    a.k_scale, a.k_scale_dev = _scale_arg(k_scale, "k_scale")
+    a.v_scale, a.v_scale_dev = _scale_arg(v_scale, "v_scale")
+    a.sm_scale = float(sm_scale)
+    a.window_left = int(window_left)
+    sp = _dev_ptr(sinks, "sinks", (torch.float32,), (Hq,))
+    a.sinks = sp.value if sp is not None else None
+    a.out = out.data_ptr()
+    a.out_token_stride = _token_rows(out, "out", lead, Hq, D)
+    lp = _dev_ptr(lse, "lse", (torch.float32,), lead + (Hq,))
+    a.lse = lp.value if lp is not None else None
+    a.chunk_pages_override = int(chunk_pages_override)
+    st = load_library().fp8_paged_decode_attention_args(
+        ctypes.byref(a), _dev_ptr(workspace, "workspace", (torch.uint8,)),
+        ctypes.c_size_t(workspace.numel()), _stream_handle(stream))
     _check(st, "fp8_paged_decode_attention")
     return out, lse
 
@@ -319,16 +406,22 @@ fp8_paged_decode_attention_ex = fp8_paged_decode_attention
 
 
 def fp8_paged_decode_cache_write(key, value, slot_mapping, k_cache, v_cache, k_scale, v_scale,
-                                 status=None, stream=None):
+                                 status=None, stream=None, kv_layout="NHD"):
     """Enqueue the FP8 KV-cache write on ``stream``: bf16 ``key``/``value``
     [num_tokens, Hkv, D] (rows contiguous; any token stride that is a multiple
     of 8 elements) quantised with the per-tensor scales into ``k_cache``/
-    ``v_cache`` [num_blocks, block_tokens, Hkv, D] (uint8 or float8_e4m3fn) at
+    ``v_cache`` [num_blocks, block_tokens, Hkv, D] (or [num_blocks, Hkv,
+    block_tokens, D] with ``kv_layout="HND"``; uint8 or float8_e4m3fn) at
     ``slot_mapping`` (int64 [num_tokens], negative = skip).  ``status``: an
     optional int32 CUDA tensor whose first word receives FPD_DEVERR_SLOT."""
     import torch
     T, Hkv, D = key.shape
-    num_blocks, bt, Hkv2, D2 = k_cache.shape
+    if kv_layout not in ("NHD", "HND"):
+        raise ValueError("kv_layout must be 'NHD' or 'HND'")
+    if kv_layout == "HND":
+        num_blocks, Hkv2, bt, D2 = k_cache.shape
+    else:
+        num_blocks, bt, Hkv2, D2 = k_cache.shape
     if (Hkv2, D2) != (Hkv, D) or tuple(value.shape) != (T, Hkv, D):
         raise ValueError("key/value and the caches disagree on (Hkv, D)")
     for name, t in (("key", key), ("value", value)):
@@ -337,12 +430,13 @@ def fp8_paged_decode_cache_write(key, value, slot_mapping, k_cache, v_cache, k_s
         if t.stride(2) != 1 or t.stride(1) != D:
             raise ValueError(f"{name} rows must be contiguous ([num_tokens, Hkv, D], any token stride)")
     kv_types = (torch.uint8, torch.float8_e4m3fn)
-    st = load_library().fp8_paged_decode_cache_write(
+    st = load_library().fp8_paged_decode_cache_write_layout(
         ctypes.c_void_p(key.data_ptr()), ctypes.c_void_p(value.data_ptr()),
         _dev_ptr(slot_mapping, "slot_mapping", (torch.int64,), (T,)), T, Hkv, D,
         key.stride(0), value.stride(0), float(k_scale), float(v_scale),
         _dev_ptr(k_cache, "k_cache", kv_types),
         _dev_ptr(v_cache, "v_cache", kv_types, tuple(k_cache.shape)), num_blocks, bt,
+        FPD_KV_HND if kv_layout == "HND" else FPD_KV_NHD,
         _dev_ptr(status, "status", (torch.int32,)), _stream_handle(stream))
     _check(st, "fp8_paged_decode_cache_write")
 

@@ -246,18 +246,28 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder() {
   return g_encode;
 }
 
-// View a [num_blocks, bt, Hkv, D] byte cache as a 3-D tensor.
+// View a byte cache as a tensor for TMA.
+// Token-major pages [num_blocks, bt, Hkv, D], 3-D:
 //   HB = 1: (d, kv head, token row), box (D, 1, bt): one page of one head.
 //   HB = 4: (d, token row, kv head), box (D, 16, 4): 16 tokens of 4 heads,
 //           landing head-major in shared memory (4 tiles of 16 rows).
+// Head-major pages [num_blocks, Hkv, bt, D] (hnd), 4-D (d, slot, kv head, page):
+//   HB = 1: box (D, bt, 1, 1); HB = 4: box (D, 16, 4, 1).  Both land in shared
+//   memory exactly as the token-major boxes do.
 bool encode_cache_map(CUtensorMap* map, const void* base, int num_blocks, int bt, int Hkv, int D,
-                      int HB) {
+                      int HB, bool hnd) {
   auto enc = encoder();
   if (!enc) return false;
   const cuuint64_t rows = (cuuint64_t)num_blocks * bt;
-  cuuint64_t dims[3], strides[2];
-  cuuint32_t box[3];
-  if (HB == 1) {
+  cuuint64_t dims[4], strides[3];
+  cuuint32_t box[4];
+  cuuint32_t rank = 3;
+  if (hnd) {
+    rank = 4;
+    dims[0] = D, dims[1] = bt, dims[2] = Hkv, dims[3] = num_blocks;
+    strides[0] = D, strides[1] = (cuuint64_t)bt * D, strides[2] = (cuuint64_t)Hkv * bt * D;
+    box[0] = D, box[1] = HB == 1 ? bt : fpd::kBoxTokens, box[2] = HB, box[3] = 1u;
+  } else if (HB == 1) {
     dims[0] = D, dims[1] = Hkv, dims[2] = rows;
     strides[0] = D, strides[1] = (cuuint64_t)Hkv * D;
     box[0] = D, box[1] = 1u, box[2] = bt;
@@ -266,14 +276,14 @@ bool encode_cache_map(CUtensorMap* map, const void* base, int num_blocks, int bt
     strides[0] = (cuuint64_t)Hkv * D, strides[1] = D;
     box[0] = D, box[1] = fpd::kBoxTokens, box[2] = HB;
   }
-  cuuint32_t estr[3] = {1u, 1u, 1u};
+  cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
   const CUtensorMapSwizzle swz =
       D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   // No L2 promotion: each box row is one 128-byte (or 64-byte) line of one KV
   // head, and widening it fetches the neighbouring head's line, which is
   // often evicted before its own reader arrives (measured: 18% extra DRAM
   // reads on the windowed, GQA-8 workload with 256-byte promotion).
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides,
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, const_cast<void*>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -493,48 +503,97 @@ size_t fp8_paged_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int bt, i
 
 }  // extern "C"
 
-static fpd_status attention_impl(const void* q, const void* k_cache, const void* v_cache,
-                                 const int32_t* block_table, const int32_t* seq_lens, int B,
-                                 int q_len, int Hq, int Hkv, int D, int num_blocks, int bt,
-                                 int max_blocks, float k_scale, float v_scale, float sm_scale,
-                                 int window_left, const float* sinks, void* out, float* lse,
-                                 void* workspace, size_t workspace_bytes, void* stream,
-                                 int chunk_pages_override, void* ev0, void* ev1, void* ev2) {
+// The descriptor of a token-major, bf16, contiguous call.
+static fpd_decode_args plain_args(const void* q, const void* k_cache, const void* v_cache,
+                           const int32_t* block_table, const int32_t* seq_lens, int B, int q_len,
+                           int Hq, int Hkv, int D, int num_blocks, int bt, int max_blocks,
+                           float k_scale, float v_scale, float sm_scale, int window_left,
+                           const float* sinks, void* out, float* lse, int chunk_pages_override) {
+  fpd_decode_args a;
+  std::memset(&a, 0, sizeof a);
+  a.q = q;
+  a.q_dtype = FPD_Q_BF16;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+  a.kv_layout = FPD_KV_NHD;
+  a.block_table = block_table;
+  a.seq_lens = seq_lens;
+  a.B = B;
+  a.q_len = q_len;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.D = D;
+  a.num_blocks = num_blocks;
+  a.block_tokens = bt;
+  a.max_blocks = max_blocks;
+  a.k_scale = k_scale;
+  a.v_scale = v_scale;
+  a.sm_scale = sm_scale;
+  a.window_left = window_left;
+  a.sinks = sinks;
+  a.out = out;
+  a.lse = lse;
+  a.chunk_pages_override = chunk_pages_override;
+  return a;
+}
+
+static fpd_status attention_impl(const fpd_decode_args& a, void* workspace,
+                                 size_t workspace_bytes, void* stream, void* ev0, void* ev1,
+                                 void* ev2) {
+  const int B = a.B, q_len = a.q_len, Hq = a.Hq, Hkv = a.Hkv, D = a.D, bt = a.block_tokens;
+  const int max_blocks = a.max_blocks, num_blocks = a.num_blocks, window_left = a.window_left;
   fpd_status st = validate_shape(B, Hq, Hkv, D, bt, max_blocks, q_len);
   if (st != FPD_OK) return st;
   if (num_blocks <= 0 || (int64_t)num_blocks * bt >= INT32_MAX) return FPD_ERR_UNSUPPORTED;
-  if (!q || !k_cache || !v_cache || !block_table || !seq_lens || !out) return FPD_ERR_INVALID_ARG;
-  if (!aligned(q, 16) || !aligned(out, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
-      !aligned(block_table, 4) || !aligned(seq_lens, 4) || (lse && !aligned(lse, 4)) ||
-      (sinks && !aligned(sinks, 4)) || (workspace && !aligned(workspace, 16)))
+  if (!a.q || !a.k_cache || !a.v_cache || !a.block_table || !a.seq_lens || !a.out)
     return FPD_ERR_INVALID_ARG;
-  if (!std::isfinite(k_scale) || !std::isfinite(v_scale) || !std::isfinite(sm_scale))
+  if (a.q_dtype != FPD_Q_BF16 && a.q_dtype != FPD_Q_F16) return FPD_ERR_INVALID_ARG;
+  if (a.kv_layout != FPD_KV_NHD && a.kv_layout != FPD_KV_HND) return FPD_ERR_INVALID_ARG;
+  const int64_t row = (int64_t)Hq * D;
+  const int64_t q_stride = a.q_token_stride ? a.q_token_stride : row;
+  const int64_t o_stride = a.out_token_stride ? a.out_token_stride : row;
+  // 16-byte rows: the query rows are bulk-copied and the outputs stored 16 bytes at a time
+  if (q_stride < row || o_stride < row || q_stride % 8 != 0 || o_stride % 8 != 0)
     return FPD_ERR_INVALID_ARG;
-  const float qk = sm_scale * k_scale;
-  if (!(qk > 0.f) || !std::isfinite(qk * fpd::kLog2e)) return FPD_ERR_INVALID_ARG;
-  if (chunk_pages_override < 0) return FPD_ERR_INVALID_ARG;
+  if (!aligned(a.q, 16) || !aligned(a.out, 16) || !aligned(a.k_cache, 16) ||
+      !aligned(a.v_cache, 16) || !aligned(a.block_table, 4) || !aligned(a.seq_lens, 4) ||
+      (a.lse && !aligned(a.lse, 4)) || (a.sinks && !aligned(a.sinks, 4)) ||
+      (a.k_scale_dev && !aligned(a.k_scale_dev, 4)) ||
+      (a.v_scale_dev && !aligned(a.v_scale_dev, 4)) || (workspace && !aligned(workspace, 16)))
+    return FPD_ERR_INVALID_ARG;
+  if (!std::isfinite(a.sm_scale) || !(a.sm_scale > 0.f) ||
+      !std::isfinite(a.sm_scale * fpd::kLog2e))
+    return FPD_ERR_INVALID_ARG;
+  const float qk = a.sm_scale * a.k_scale;
+  if (!a.k_scale_dev && (!std::isfinite(a.k_scale) || !(qk > 0.f) ||
+                         !std::isfinite(qk * fpd::kLog2e)))
+    return FPD_ERR_INVALID_ARG;
+  if (!a.v_scale_dev && !std::isfinite(a.v_scale)) return FPD_ERR_INVALID_ARG;
+  if (a.chunk_pages_override < 0) return FPD_ERR_INVALID_ARG;
   if (B == 0) return FPD_OK;
 
   const int g = Hq / Hkv;
   fpd_plan plan;
-  st = plan_device(B, q_len, Hq, Hkv, D, bt, max_blocks, window_left, chunk_pages_override, &plan);
+  st = plan_device(B, q_len, Hq, Hkv, D, bt, max_blocks, window_left, a.chunk_pages_override,
+                   &plan);
   if (st != FPD_OK) return st;
   if (!workspace || workspace_bytes < plan.workspace_bytes) return FPD_ERR_WORKSPACE_TOO_SMALL;
 
+  const bool hnd = a.kv_layout == FPD_KV_HND;
   CUtensorMap km, vm;
-  if (!encode_cache_map(&km, k_cache, num_blocks, bt, Hkv, D, plan.heads_per_stage) ||
-      !encode_cache_map(&vm, v_cache, num_blocks, bt, Hkv, D, plan.heads_per_stage))
+  if (!encode_cache_map(&km, a.k_cache, num_blocks, bt, Hkv, D, plan.heads_per_stage, hnd) ||
+      !encode_cache_map(&vm, a.v_cache, num_blocks, bt, Hkv, D, plan.heads_per_stage, hnd))
     return FPD_ERR_CUDA;
 
   const WsLayout wl = ws_layout(B * q_len, Hq, Hkv, D, plan.max_splits);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   fpd::DecodeParams p;
-  p.q = static_cast<const __nv_bfloat16*>(q);
-  p.block_table = block_table;
-  p.seq_lens = seq_lens;
-  p.sinks = sinks;
-  p.out = static_cast<__nv_bfloat16*>(out);
-  p.lse = lse;
+  p.q = static_cast<const __nv_bfloat16*>(a.q);
+  p.block_table = a.block_table;
+  p.seq_lens = a.seq_lens;
+  p.sinks = a.sinks;
+  p.out = static_cast<__nv_bfloat16*>(a.out);
+  p.lse = a.lse;
   p.part_o = reinterpret_cast<float*>(ws + wl.part_o);
   p.part_lse = reinterpret_cast<float*>(ws + wl.part_lse);
   p.status = reinterpret_cast<uint32_t*>(ws);
@@ -556,7 +615,14 @@ static fpd_status attention_impl(const void* q, const void* k_cache, const void*
   p.q_chunks = plan.q_chunks;
   p.lg = __builtin_ctz((unsigned)g);
   p.qk_scale_log2 = qk * fpd::kLog2e;
-  p.v_scale = v_scale;
+  p.v_scale = a.v_scale;
+  p.q_tok_stride = q_stride;
+  p.out_tok_stride = o_stride;
+  p.k_scale_dev = a.k_scale_dev;
+  p.v_scale_dev = a.v_scale_dev;
+  p.sm_scale_log2 = a.sm_scale * fpd::kLog2e;
+  p.q_f16 = a.q_dtype == FPD_Q_F16;
+  p.kv_hnd = hnd;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (ev0 && cudaEventRecord(static_cast<cudaEvent_t>(ev0), s) != cudaSuccess) return FPD_ERR_CUDA;
@@ -573,12 +639,12 @@ static fpd_status attention_impl(const void* q, const void* k_cache, const void*
   if (ev1 && cudaEventRecord(static_cast<cudaEvent_t>(ev1), s) != cudaSuccess) return FPD_ERR_CUDA;
   if (plan.max_splits > 1) {
     fpd::CombineParams c;
-    c.seq_lens = seq_lens;
-    c.sinks = sinks;
+    c.seq_lens = a.seq_lens;
+    c.sinks = a.sinks;
     c.part_o = p.part_o;
     c.part_lse = p.part_lse;
     c.out = p.out;
-    c.lse = lse;
+    c.lse = a.lse;
     c.B = B;
     c.q_len = q_len;
     c.Hq = Hq;
@@ -592,7 +658,9 @@ static fpd_status attention_impl(const void* q, const void* k_cache, const void*
     c.wpr = 1;
     while (c.wpr < 32 && c.wpr * fpd::kCombineBatch < plan.max_splits) c.wpr *= 2;
     c.rows_per_cta = c.wpr >= 8 ? 1 : 8 / c.wpr;
-    c.v_scale = v_scale;
+    c.v_scale = a.v_scale;
+    c.v_scale_dev = a.v_scale_dev;
+    c.out_tok_stride = o_stride;
     if (mq)
       e = D == 128 ? launch_combine<128, true>(c, s) : launch_combine<64, true>(c, s);
     else
@@ -613,10 +681,10 @@ fpd_status fp8_paged_decode_attention_ex(const void* q, const void* k_cache, con
                                          void* out, float* lse, void* workspace,
                                          size_t workspace_bytes, void* stream,
                                          int chunk_pages_override) {
-  return attention_impl(q, k_cache, v_cache, block_table, seq_lens, B, 1, Hq, Hkv, D, num_blocks, bt,
-                        max_blocks, k_scale, v_scale, sm_scale, window_left, sinks, out, lse,
-                        workspace, workspace_bytes, stream, chunk_pages_override, nullptr,
-                        nullptr, nullptr);
+  return attention_impl(plain_args(q, k_cache, v_cache, block_table, seq_lens, B, 1, Hq, Hkv, D,
+                                   num_blocks, bt, max_blocks, k_scale, v_scale, sm_scale,
+                                   window_left, sinks, out, lse, chunk_pages_override),
+                        workspace, workspace_bytes, stream, nullptr, nullptr, nullptr);
 }
 
 fpd_status fp8_paged_decode_attention_qlen(const void* q, const void* k_cache,
@@ -627,10 +695,16 @@ fpd_status fp8_paged_decode_attention_qlen(const void* q, const void* k_cache,
                                            int window_left, const float* sinks, void* out,
                                            float* lse, void* workspace, size_t workspace_bytes,
                                            void* stream, int chunk_pages_override) {
-  return attention_impl(q, k_cache, v_cache, block_table, seq_lens, B, q_len, Hq, Hkv, D,
-                        num_blocks, bt, max_blocks, k_scale, v_scale, sm_scale, window_left, sinks,
-                        out, lse, workspace, workspace_bytes, stream, chunk_pages_override,
-                        nullptr, nullptr, nullptr);
+  return attention_impl(plain_args(q, k_cache, v_cache, block_table, seq_lens, B, q_len, Hq,
+                                   Hkv, D, num_blocks, bt, max_blocks, k_scale, v_scale, sm_scale,
+                                   window_left, sinks, out, lse, chunk_pages_override),
+                        workspace, workspace_bytes, stream, nullptr, nullptr, nullptr);
+}
+
+fpd_status fp8_paged_decode_attention_args(const fpd_decode_args* args, void* workspace,
+                                           size_t workspace_bytes, void* stream) {
+  if (!args) return FPD_ERR_INVALID_ARG;
+  return attention_impl(*args, workspace, workspace_bytes, stream, nullptr, nullptr, nullptr);
 }
 
 fpd_status fp8_paged_decode_attention_profiled(
@@ -640,10 +714,11 @@ fpd_status fp8_paged_decode_attention_profiled(
     const float* sinks, void* out, float* lse, void* workspace, size_t workspace_bytes,
     void* stream, int chunk_pages_override, void* event_before_split, void* event_after_split,
     void* event_after_combine) {
-  return attention_impl(q, k_cache, v_cache, block_table, seq_lens, B, q_len, Hq, Hkv, D, num_blocks, bt,
-                        max_blocks, k_scale, v_scale, sm_scale, window_left, sinks, out, lse,
-                        workspace, workspace_bytes, stream, chunk_pages_override,
-                        event_before_split, event_after_split, event_after_combine);
+  return attention_impl(plain_args(q, k_cache, v_cache, block_table, seq_lens, B, q_len, Hq,
+                                   Hkv, D, num_blocks, bt, max_blocks, k_scale, v_scale, sm_scale,
+                                   window_left, sinks, out, lse, chunk_pages_override),
+                        workspace, workspace_bytes, stream, event_before_split,
+                        event_after_split, event_after_combine);
 }
 
 fpd_status fp8_paged_decode_attention(const void* q, const void* k_cache, const void* v_cache,
@@ -715,20 +790,25 @@ fpd_status fp8_paged_decode_attention_noalloc(const void* q, const void* k_cache
   const size_t zero = ws_layout(B, Hq, Hkv, D, plan.max_splits).zero_prefix;
   if (cudaMemsetAsync(scratch, 0, zero, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return FPD_ERR_CUDA;
-  return attention_impl(q, k_cache, v_cache, block_table, seq_lens, B, 1, Hq, Hkv, D, num_blocks, bt,
-                        max_blocks, k_scale, v_scale, sm_scale, window_left, sinks, out, lse,
-                        scratch, FPD_NOALLOC_SCRATCH_BYTES, stream, 0, nullptr, nullptr, nullptr);
+  return attention_impl(plain_args(q, k_cache, v_cache, block_table, seq_lens, B, 1, Hq, Hkv, D,
+                                   num_blocks, bt, max_blocks, k_scale, v_scale, sm_scale,
+                                   window_left, sinks, out, lse, 0),
+                        scratch, FPD_NOALLOC_SCRATCH_BYTES, stream, nullptr, nullptr, nullptr);
 }
 
-fpd_status fp8_paged_decode_cache_write(const void* key, const void* value,
-                                        const int64_t* slot_mapping, int num_tokens, int Hkv,
-                                        int D, int64_t key_stride, int64_t value_stride,
-                                        float k_scale, float v_scale, void* k_cache,
-                                        void* v_cache, int num_blocks, int block_tokens,
-                                        uint32_t* status, void* stream) {
+fpd_status fp8_paged_decode_cache_write_layout(const void* key, const void* value,
+                                               const int64_t* slot_mapping, int num_tokens,
+                                               int Hkv, int D, int64_t key_stride,
+                                               int64_t value_stride, float k_scale,
+                                               float v_scale, void* k_cache, void* v_cache,
+                                               int num_blocks, int block_tokens, int kv_layout,
+                                               uint32_t* status, void* stream) {
   if (num_tokens < 0 || Hkv <= 0 || D <= 0 || D % 16 != 0 || num_blocks <= 0 ||
       block_tokens <= 0)
     return FPD_ERR_INVALID_ARG;
+  if (kv_layout != FPD_KV_NHD && kv_layout != FPD_KV_HND) return FPD_ERR_INVALID_ARG;
+  if (kv_layout == FPD_KV_HND && (int64_t)num_blocks * block_tokens >= INT32_MAX)
+    return FPD_ERR_UNSUPPORTED;
   if (!(k_scale > 0.f) || !(v_scale > 0.f) || !std::isfinite(k_scale) || !std::isfinite(v_scale))
     return FPD_ERR_INVALID_ARG;
   if (num_tokens == 0) return FPD_OK;
@@ -754,6 +834,9 @@ fpd_status fp8_paged_decode_cache_write(const void* key, const void* value,
   p.row_chunks = (int)(row / fpd::kWriteElems);
   p.k_inv = 1.0f / k_scale;   // fp32 reciprocal, as the reference writer takes it
   p.v_inv = 1.0f / v_scale;
+  p.hnd = kv_layout == FPD_KV_HND;
+  p.bt = block_tokens;
+  p.head_chunks = D / fpd::kWriteElems;
   int sms = 0;
   if (!device_sm_count(&sms)) return FPD_ERR_CUDA;
   const int64_t units = (int64_t)num_tokens * 2 * p.row_chunks;
@@ -763,6 +846,18 @@ fpd_status fp8_paged_decode_cache_write(const void* key, const void* value,
   fpd::fpd_cache_write_kernel<<<grid, fpd::kWriteThreads, 0, static_cast<cudaStream_t>(stream)>>>(
       p);
   return cudaGetLastError() == cudaSuccess ? FPD_OK : FPD_ERR_CUDA;
+}
+
+fpd_status fp8_paged_decode_cache_write(const void* key, const void* value,
+                                        const int64_t* slot_mapping, int num_tokens, int Hkv,
+                                        int D, int64_t key_stride, int64_t value_stride,
+                                        float k_scale, float v_scale, void* k_cache,
+                                        void* v_cache, int num_blocks, int block_tokens,
+                                        uint32_t* status, void* stream) {
+  return fp8_paged_decode_cache_write_layout(key, value, slot_mapping, num_tokens, Hkv, D,
+                                             key_stride, value_stride, k_scale, v_scale, k_cache,
+                                             v_cache, num_blocks, block_tokens, FPD_KV_NHD,
+                                             status, stream);
 }
 
 fpd_status fp8_paged_decode_check_status(void* workspace, void* stream, int* device_error_bits,

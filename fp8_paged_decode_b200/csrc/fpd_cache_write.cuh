@@ -11,7 +11,9 @@
 //
 // Layout: key/value [num_tokens, Hkv, D] bf16 with a token stride (elements);
 // caches [num_blocks, block_tokens, Hkv, D] E4M3, so the Hkv * D elements of
-// one token form one contiguous row on both sides.  One thread converts 16
+// one token form one contiguous row on both sides; or head-major caches
+// [num_blocks, Hkv, block_tokens, D] (the gist writer's HND layout), where each
+// 16-element chunk still lands contiguously inside one head's row.  One thread converts 16
 // consecutive elements: two 16-byte loads, one 16-byte store, so a warp reads
 // 1 KB and writes 512 B of one row contiguously.  The op is HBM-bound:
 // 6 bytes per element (4 read, 2 written).
@@ -40,6 +42,9 @@ struct CacheWriteParams {
   int num_tokens;
   int row_chunks;          // Hkv * D / 16
   float k_inv, v_inv;      // 1 / k_scale, 1 / v_scale, rounded to fp32 on the host
+  int hnd;                 // head-major pages [num_blocks, Hkv, bt, D] (else token-major)
+  int bt;                  // tokens per page (head-major pages)
+  int head_chunks;         // D / 16
 };
 
 // Eight bf16 (a 16-byte vector) times `inv`, as four e4m3x2 pairs packed into
@@ -80,8 +85,17 @@ __global__ void __launch_bounds__(kWriteThreads) fpd_cache_write_kernel(const Ca
     const uint4 b = __ldcs(reinterpret_cast<const uint4*>(src) + 1);
     const float inv = is_v ? p.v_inv : p.k_inv;
     const uint2 lo = quantise8(a, inv), hi = quantise8(b, inv);
-    uint8_t* dst = (is_v ? p.v_cache : p.k_cache) +
-                   (slot * p.row_chunks + c) * kWriteElems;
+    uint8_t* base = is_v ? p.v_cache : p.k_cache;
+    uint8_t* dst;
+    if (p.hnd) {   // [page][kv head][in-page slot][d]; slots fit in 32 bits here
+      const int s32 = (int)slot;
+      const int page = s32 / p.bt, off = s32 - page * p.bt;
+      const int h = c / p.head_chunks, part = c - h * p.head_chunks;
+      const int Hkv = p.row_chunks / p.head_chunks;
+      dst = base + ((((int64_t)page * Hkv + h) * p.bt + off) * p.head_chunks + part) * kWriteElems;
+    } else {       // [slot][kv head][d]: a token's row is contiguous
+      dst = base + (slot * p.row_chunks + c) * kWriteElems;
+    }
     *reinterpret_cast<uint4*>(dst) = make_uint4(lo.x, lo.y, hi.x, hi.y);
   }
 }

@@ -102,6 +102,14 @@ struct DecodeParams {
   int lg;               // log2(g): g is a power of two
   float qk_scale_log2;  // sm_scale * k_scale * log2(e)
   float v_scale;
+  // interface variants
+  int64_t q_tok_stride;       // elements between consecutive query tokens (>= Hq * D)
+  int64_t out_tok_stride;     // elements between consecutive output tokens
+  const float* k_scale_dev;   // device scales, read after the grid dependency
+  const float* v_scale_dev;   //   resolves; nullptr: the host values above
+  float sm_scale_log2;        // sm_scale * log2(e), for a device k_scale
+  int q_f16;                  // the query is fp16 (else bf16)
+  int kv_hnd;                 // pages are [num_blocks, Hkv, bt, D] (else [.., bt, Hkv, D])
 };
 
 // Bytes of one header slot: the header, then the item's query rows (HB KV
@@ -239,8 +247,10 @@ struct Consumer {
   // qbase: the item's query rows in shared memory, bf16 [position][rows_per_pos][D];
   // column c (query position c / g, head c % g) is row
   // (c / g) * rows_per_pos + w_off + c % g.
-  __device__ __forceinline__ void init(const DecodeParams& p, const __nv_bfloat16* qbase,
-                                       int rows_per_pos, int w_off, int ncols, int lane) {
+  // qk_scale: the logit scale in the log2 domain (sm_scale * k_scale * log2 e).
+  __device__ __forceinline__ void init(const DecodeParams& p, float qk_scale,
+                                       const __nv_bfloat16* qbase, int rows_per_pos, int w_off,
+                                       int ncols, int lane) {
     const int n = lane >> 2, t = lane & 3;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
@@ -250,15 +260,29 @@ struct Consumer {
       if (c < (MQ ? ncols : p.g)) {
         const int qrow = MQ ? (c >> p.lg) * rows_per_pos + w_off + (c & (p.g - 1)) : w_off + c;
         const __nv_bfloat16* src = qbase + qrow * D + t * QW;
+        if (p.q_f16) {   // fp16 query: the same 16-bit rows, another decoding
 #pragma unroll
-        for (int i = 0; i < QW; i += 8) {
-          const uint4 raw = *reinterpret_cast<const uint4*>(src + i);
-          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+          for (int i = 0; i < QW; i += 8) {
+            const uint4 raw = *reinterpret_cast<const uint4*>(src + i);
+            const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float2 f = __bfloat1622float2(h2[j]);
-            vals[i + 2 * j] = f.x;
-            vals[i + 2 * j + 1] = f.y;
+            for (int j = 0; j < 4; ++j) {
+              const float2 f = __half22float2(h2[j]);
+              vals[i + 2 * j] = f.x;
+              vals[i + 2 * j + 1] = f.y;
+            }
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < QW; i += 8) {
+            const uint4 raw = *reinterpret_cast<const uint4*>(src + i);
+            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float2 f = __bfloat1622float2(h2[j]);
+              vals[i + 2 * j] = f.x;
+              vals[i + 2 * j + 1] = f.y;
+            }
           }
         }
 #pragma unroll
@@ -270,7 +294,8 @@ struct Consumer {
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
       // Power-of-two prescale so the largest |q| of the head sits in [2^14, 2^15):
-      // keeps bf16 -> f16 exact for any bf16 magnitude; undone in the logit scale.
+      // keeps bf16 -> f16 exact for any bf16 magnitude (and fp16 exact, down to
+      // 2^-24 of the largest element); undone in the logit scale.
       int e = 0;
       if (amax > 0.f && isfinite(amax)) frexpf(amax, &e);
       const int sh = max(-126, min(126, 15 - e));
@@ -284,8 +309,8 @@ struct Consumer {
       // prescale is a power of two, so undoing it is an exact multiply
       const int sh0 = __shfl_sync(0xffffffffu, sh, (2 * t) * 4);
       const int sh1 = __shfl_sync(0xffffffffu, sh, (2 * t + 1) * 4);
-      cs[nt][0] = p.qk_scale_log2 * ldexpf(1.0f, -sh0);
-      cs[nt][1] = p.qk_scale_log2 * ldexpf(1.0f, -sh1);
+      cs[nt][0] = qk_scale * ldexpf(1.0f, -sh0);
+      cs[nt][1] = qk_scale * ldexpf(1.0f, -sh1);
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         m[nt][j] = -INFINITY;
@@ -483,8 +508,8 @@ struct Consumer {
   // heads are finished straight from registers.  Thread (n, t) holds, for
   // column nt*8 + 2t + j, the D/8 output elements starting at n*D/8.  The
   // item's columns are queries qrow0 .. qrow0 + ncols / g - 1 of the sequence.
-  __device__ __forceinline__ void finish_own(const DecodeParams& p, int b, int kvh, int split,
-                                             int ns, int qrow0, int ncols, int lane) {
+  __device__ __forceinline__ void finish_own(const DecodeParams& p, float v_scale, int b, int kvh,
+                                             int split, int ns, int qrow0, int ncols, int lane) {
     constexpr int E = D / 8;   // output elements per thread and query head
     const int n = lane >> 2, t = lane & 3;
     float lsum[NT][2];
@@ -505,12 +530,13 @@ struct Consumer {
         const int c = nt * 8 + 2 * t + j;   // column: query position c / g, head c % g
         if (c >= (MQ ? ncols : p.g)) continue;
         const int hq = kvh * p.g + (MQ ? c & (p.g - 1) : c);
-        const size_t row = MQ ? ((size_t)b * p.q_len + qrow0 + (c >> p.lg)) * p.Hq + hq
-                              : (size_t)b * p.Hq + hq;
+        const size_t tok = MQ ? (size_t)b * p.q_len + qrow0 + (c >> p.lg) : (size_t)b;
+        const size_t row = tok * p.Hq + hq;
+        __nv_bfloat16* const orow = p.out + tok * p.out_tok_stride + (size_t)hq * D;
         // false: this query saw no key in the item (only possible with MQ)
         const bool keys = !MQ || lsum[nt][j] > 0.f;
         if (ns == 0 || (ns == 1 && !keys)) {  // no key at all: out = 0, lse = sigma
-          uint4* dst = reinterpret_cast<uint4*>(p.out + row * D + n * E);
+          uint4* dst = reinterpret_cast<uint4*>(orow + n * E);
 #pragma unroll
           for (int k = 0; k < E / 8; ++k) dst[k] = make_uint4(0u, 0u, 0u, 0u);
           if (n == 0 && p.lse) p.lse[row] = p.sinks ? p.sinks[hq] : -INFINITY;
@@ -518,7 +544,7 @@ struct Consumer {
         }
         const float lse2 = m[nt][j] + __log2f(lsum[nt][j]);   // log2-sum-exp, no sink
         if (ns == 1) {
-          float scale = p.v_scale;
+          float scale = v_scale;
           float lse_out = lse2;
           if (p.sinks) {
             const float sg = p.sinks[hq] * kLog2e;
@@ -532,7 +558,7 @@ struct Consumer {
           uint32_t w[MT];
 #pragma unroll
           for (int i = 0; i < MT; ++i) w[i] = pack_bf16x2(o[i][nt][j] * inv, o[i][nt][j + 2] * inv);
-          uint4* dst = reinterpret_cast<uint4*>(p.out + row * D + n * E);
+          uint4* dst = reinterpret_cast<uint4*>(orow + n * E);
 #pragma unroll
           for (int k = 0; k < E / 8; ++k)
             dst[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
@@ -655,8 +681,8 @@ __device__ __forceinline__ void producer_loop(const CUtensorMap* kmap, const CUt
       mbar_arrive_expect_tx(&hdr_full[hslot], qbytes * (uint32_t)npos);
       for (int i = 0; i < npos; ++i)
         bulk_load(hbase + kHdrBytes + (size_t)i * qbytes,
-                  p.q + (((size_t)b * QL + qrow0 + i) * p.Hq + (size_t)kvh0 * p.g) * D, qbytes,
-                  &hdr_full[hslot]);
+                  p.q + ((size_t)b * QL + qrow0 + i) * p.q_tok_stride + (size_t)kvh0 * p.g * D,
+                  qbytes, &hdr_full[hslot]);
     }
     ++hs;
     if (++hslot == n_hslots) {
@@ -694,9 +720,13 @@ __device__ __forceinline__ void producer_loop(const CUtensorMap* kmap, const CUt
         __syncwarp();
         if (mine) {
           // an invalid page is read from past the end of the pool: TMA zero-fills it
-          const int row = ok ? e * p.bt : p.num_blocks * p.bt;
           uint8_t* dst = stage + (lane & 1) * kTileBytes + (lane >> 1) * page_bytes;
-          tma_load_3d(dst, (lane & 1) ? vmap : kmap, 0, kvh0, row, &full_bar[slot], policy);
+          const CUtensorMap* map = (lane & 1) ? vmap : kmap;
+          if (p.kv_hnd)   // (d, slot, kv head, page)
+            tma_load_4d(dst, map, 0, 0, kvh0, ok ? e : p.num_blocks, &full_bar[slot], policy);
+          else            // (d, kv head, token row)
+            tma_load_3d(dst, map, 0, kvh0, ok ? e * p.bt : p.num_blocks * p.bt, &full_bar[slot],
+                        policy);
         }
       } else {
         // 16 tokens of HB heads: one box per tensor, lane 0 K and lane 1 V
@@ -716,9 +746,15 @@ __device__ __forceinline__ void producer_loop(const CUtensorMap* kmap, const CUt
         __syncwarp();
         if (lane < 2) {
           // an invalid page is read from past the end of the pool: TMA zero-fills it
-          const int row = (ok ? e * p.bt : p.num_blocks * p.bt) + (tok - (rel + pb) * p.bt);
-          tma_load_3d(stage + lane * kTileBytes, lane ? vmap : kmap, 0, row, kvh0,
-                      &full_bar[slot], policy);
+          const int in_page = tok - (rel + pb) * p.bt;   // first slot of the block in its page
+          const CUtensorMap* map = lane ? vmap : kmap;
+          if (p.kv_hnd)   // (d, slot, kv head, page)
+            tma_load_4d(stage + lane * kTileBytes, map, 0, in_page, kvh0, ok ? e : p.num_blocks,
+                        &full_bar[slot], policy);
+          else            // (d, token row, kv head)
+            tma_load_3d(stage + lane * kTileBytes, map, 0,
+                        (ok ? e * p.bt : p.num_blocks * p.bt) + in_page, kvh0, &full_bar[slot],
+                        policy);
         }
       }
       ++issued;
@@ -819,6 +855,10 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
   }
 
   // -------------------------------------------------------------- consumers
+  // scales: host values, or device words (readable now: the grid dependency
+  // has resolved)
+  const float qk_scale = p.k_scale_dev ? p.sm_scale_log2 * *p.k_scale_dev : p.qk_scale_log2;
+  const float v_scale = p.v_scale_dev ? *p.v_scale_dev : p.v_scale;
   Consumer<D, NT, MQ> cw;
   const int n = lane >> 2, t = lane & 3;
   // HB = 4: this warp's KV head occupies its own 16 rows of each stage.
@@ -842,7 +882,7 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
     const ItemHeader hd = *reinterpret_cast<const ItemHeader*>(hbase);
     if (hd.kind < 0) break;
     const int ncols = MQ ? hd.npos * p.g : p.g;   // the item's columns per KV head
-    cw.init(p, reinterpret_cast<const __nv_bfloat16*>(hbase + kHdrBytes), HB * p.g,
+    cw.init(p, qk_scale, reinterpret_cast<const __nv_bfloat16*>(hbase + kHdrBytes), HB * p.g,
             HB == 1 ? 0 : warp * p.g, ncols, lane);
     // Tiles inside every column's range skip the masks: past the newest key
     // the first query sees, and at or after the oldest key the last query
@@ -883,7 +923,7 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
     if (!alive) break;
 
     if constexpr (HB != 1) {
-      cw.finish_own(p, hd.b, hd.kvh0 + warp, hd.split, hd.ns, hd.qrow0, ncols, lane);
+      cw.finish_own(p, v_scale, hd.b, hd.kvh0 + warp, hd.split, hd.ns, hd.qrow0, ncols, lane);
       continue;
     }
 
@@ -927,10 +967,11 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
       for (int h = tid / D; h < ncols; h += HPI) {
         // column h: query qrow0 + h / g of the sequence, head h % g
         const int hq = hd.kvh0 * p.g + (MQ ? h & (p.g - 1) : h);
-        const size_t row = MQ ? ((size_t)hd.b * QL + hd.qrow0 + (h >> p.lg)) * p.Hq + hq
-                              : (size_t)hd.b * p.Hq + hq;
+        const size_t tok = MQ ? (size_t)hd.b * QL + hd.qrow0 + (h >> p.lg) : (size_t)hd.b;
+        const size_t row = tok * p.Hq + hq;
+        __nv_bfloat16* const orow = p.out + tok * p.out_tok_stride + (size_t)hq * D;
         if (hd.ns == 0) {  // empty sequence: out = 0, lse = sigma
-          p.out[row * D + d] = __float2bfloat16_rn(0.f);
+          orow[d] = __float2bfloat16_rn(0.f);
           if (d == 0 && p.lse) p.lse[row] = p.sinks ? p.sinks[hq] : -INFINITY;
           continue;
         }
@@ -951,7 +992,7 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
         const float lse2 = M + __log2f(Lsum);   // log2-sum-exp of this split (no sink)
         if (MQ && !(Lsum > 0.f)) {   // this query saw no key in the item
           if (single) {
-            p.out[row * D + d] = __float2bfloat16_rn(0.f);
+            orow[d] = __float2bfloat16_rn(0.f);
             if (d == 0 && p.lse) p.lse[row] = p.sinks ? p.sinks[hq] : -INFINITY;
           } else {
             const size_t prow = row * p.max_splits + hd.split;
@@ -961,7 +1002,7 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
           continue;
         }
         if (single) {
-          float scale = p.v_scale;
+          float scale = v_scale;
           float lse_out = lse2;
           if (p.sinks) {
             const float sg = p.sinks[hq] * kLog2e;
@@ -971,7 +1012,7 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
             scale *= __fdividef(wsplit, Z);
             lse_out = Mx + __log2f(Z);
           }
-          p.out[row * D + d] = __float2bfloat16_rn(acc * __fdividef(scale, Lsum));
+          orow[d] = __float2bfloat16_rn(acc * __fdividef(scale, Lsum));
           if (d == 0 && p.lse) p.lse[row] = lse_out * kLn2;
         } else {
           const size_t prow = row * p.max_splits + hd.split;
@@ -1022,6 +1063,8 @@ struct CombineParams {
   int wpr;            // warps per row: 1, 2, 4, 8, 16 or 32
   int rows_per_cta;   // rows per CTA (wpr * rows_per_cta <= 32)
   float v_scale;
+  const float* v_scale_dev;   // device v_scale or nullptr
+  int64_t out_tok_stride;     // elements between consecutive output tokens
 };
 
 constexpr int kCombineMaxThreads = 1024;
@@ -1055,8 +1098,9 @@ __global__ void __launch_bounds__(kCombineMaxThreads) fpd_combine_kernel(const C
   const float* pl = p.part_lse + (size_t)(in_range ? row : 0) * ms;
   const float* po = p.part_o + (size_t)(in_range ? row : 0) * ms * D + lane * PER;
 
-  // ---- one round of loads: the sequence length and this warp's first batch
+  // ---- one round of loads: the sequence length, v_scale and this warp's first batch
   const int L_raw = in_range ? p.seq_lens[row / (QL * p.Hq)] : 0;
+  const float v_scale = p.v_scale_dev ? *p.v_scale_dev : p.v_scale;
   float lv[kCombineBatch];
   float x[kCombineBatch][PER];
 #pragma unroll
@@ -1127,14 +1171,16 @@ __global__ void __launch_bounds__(kCombineMaxThreads) fpd_combine_kernel(const C
   }
 
   // ---- merge the row's warps (M = max over warps and the sink) and write
-  const float sink2 = (active && p.sinks) ? p.sinks[row % p.Hq] * kLog2e : -INFINITY;
+  const int hq = row % p.Hq;
+  const float sink2 = (active && p.sinks) ? p.sinks[hq] * kLog2e : -INFINITY;
+  __nv_bfloat16* const orow = p.out + (size_t)(row / p.Hq) * p.out_tok_stride + (size_t)hq * D;
   if (wpr == 1) {
     if (active) {
       const float M = fmaxf(m, sink2);
       const float r = fast_exp2(m - M);
       const float Z = z * r + (p.sinks ? fast_exp2(sink2 - M) : 0.f);
-      const float inv = p.v_scale * r / Z;
-      __nv_bfloat16* dst = p.out + (size_t)row * D + lane * PER;
+      const float inv = v_scale * r / Z;
+      __nv_bfloat16* dst = orow + lane * PER;
 #pragma unroll
       for (int i = 0; i < PER; ++i) dst[i] = __float2bfloat16_rn(acc[i] * inv);
       if (lane == 0 && p.lse) p.lse[row] = (M + __log2f(Z)) * kLn2;
@@ -1159,7 +1205,7 @@ __global__ void __launch_bounds__(kCombineMaxThreads) fpd_combine_kernel(const C
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) Z += __shfl_xor_sync(0xffffffffu, Z, o);
     if (p.sinks) Z += fast_exp2(sink2 - M);
-    const float inv = p.v_scale / Z;
+    const float inv = v_scale / Z;
     float a[PER];
 #pragma unroll
     for (int i = 0; i < PER; ++i) a[i] = 0.f;
@@ -1170,7 +1216,7 @@ __global__ void __launch_bounds__(kCombineMaxThreads) fpd_combine_kernel(const C
     }
 #pragma unroll
     for (int i = 0; i < PER; ++i)
-      p.out[(size_t)row * D + lane * PER + i] = __float2bfloat16_rn(a[i] * inv);
+      orow[lane * PER + i] = __float2bfloat16_rn(a[i] * inv);
     if (lane == 0 && p.lse) p.lse[row] = (M + __log2f(Z)) * kLn2;
   }
 }

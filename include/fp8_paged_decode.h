@@ -206,6 +206,61 @@ size_t fp8_paged_decode_workspace_bytes_qlen(int B, int q_len, int Hq, int Hkv, 
                                              int chunk_pages_override);
 
 /*
+ * Interface variants: the general decode call, described by a struct.
+ * The layouts and forms are the ones the pages' serving stack uses: the
+ * FlashInfer backend of the NVFP4 KV-cache serving gist takes the query in the
+ * model dtype (bf16 or fp16), pages in token-major (NHD) or head-major (HND)
+ * order (its cache writer writes both), and a query/output that may be a slice
+ * of a wider buffer (the fused QKV projection); per-tensor scales kept in
+ * device memory let one captured CUDA graph be replayed with new scales.
+ */
+#define FPD_KV_NHD 0   /* pages [num_blocks, block_tokens, Hkv, D] (token-major) */
+#define FPD_KV_HND 1   /* pages [num_blocks, Hkv, block_tokens, D] (head-major) */
+#define FPD_Q_BF16 0
+#define FPD_Q_F16  1
+
+typedef struct {
+    /* query token t = b * q_len + i, head h, element d is at
+     * q[t * q_token_stride + h * D + d]; q_token_stride = 0 means Hq * D.
+     * Nonzero strides must be >= Hq * D and a multiple of 8 (16 bytes). */
+    const void *q;
+    int q_dtype;                 /* FPD_Q_BF16 or FPD_Q_F16 */
+    int64_t q_token_stride;      /* elements */
+    const void *k_cache;         /* e4m3 pages in kv_layout order */
+    const void *v_cache;
+    int kv_layout;               /* FPD_KV_NHD or FPD_KV_HND */
+    const int32_t *block_table;  /* [B, max_blocks] */
+    const int32_t *seq_lens;     /* [B], including the q_len new tokens */
+    int B, q_len, Hq, Hkv, D, num_blocks, block_tokens, max_blocks;
+    float k_scale, v_scale;      /* host scales, used when the device ones are NULL */
+    const float *k_scale_dev;    /* device float or NULL; read by the kernels */
+    const float *v_scale_dev;    /* device float or NULL */
+    float sm_scale;
+    int window_left;             /* < 0: no window */
+    const float *sinks;          /* [Hq] f32 or NULL */
+    /* out is bf16; token t, head h, element d at out[t * out_token_stride + h * D + d];
+     * 0 means Hq * D; nonzero: >= Hq * D and a multiple of 8. */
+    void *out;
+    int64_t out_token_stride;    /* elements */
+    float *lse;                  /* [B, q_len, Hq] contiguous, or NULL */
+    int chunk_pages_override;    /* 0: heuristic */
+} fpd_decode_args;
+
+/*
+ * The decode call for any combination of the variants above.  q_len, masks,
+ * sinks and the workspace are as in fp8_paged_decode_attention_qlen (size the
+ * workspace with fp8_paged_decode_workspace_bytes_qlen: the variants do not
+ * change it).  Device scales are read on the GPU after the work queued before
+ * this call on `stream` has completed, so a kernel earlier in the stream may
+ * write them; their validity (finite, > 0) is the caller's: a bad device scale
+ * gives NaN or infinite outputs, not an error.  Host scales are validated as in
+ * the other calls.  Returns FPD_ERR_INVALID_ARG for a bad stride, dtype or
+ * layout code, and the errors of fp8_paged_decode_attention otherwise.
+ */
+fpd_status fp8_paged_decode_attention_args(const fpd_decode_args *args, void *workspace,
+                                           size_t workspace_bytes, void *stream);
+
+/*
  * Same as fp8_paged_decode_attention_qlen, and additionally records the given
  * cudaEvent_t handles (passed as void*, each may be NULL) on `stream`: one
  * before the split kernel, one between the split and combine kernels, one after
@@ -268,11 +323,6 @@ fpd_status fp8_paged_decode_attention_noalloc(const void *q, const void *k_cache
                                               void *stream);
 
 /*
- * Reads the workspace status word (FPD_DEVERR_* bits) after synchronising
- * `stream`; clears it when `clear` is nonzero.  Writes the bits to
- * *device_error_bits.  Needs a workspace of at least 256 bytes.
- */
-/*
  * FP8 KV-cache write: quantise the bf16 K and V rows of new tokens with the
  * per-tensor scales and scatter them into the paged E4M3 caches.  The
  * quantisation is the per-tensor form of the standalone cache-writer kernel in
@@ -302,6 +352,24 @@ fpd_status fp8_paged_decode_cache_write(const void *key, const void *value,
                                         void *v_cache, int num_blocks, int block_tokens,
                                         uint32_t *status, void *stream);
 
+/*
+ * The cache write into pages of either layout (kv_layout FPD_KV_NHD or
+ * FPD_KV_HND); fp8_paged_decode_cache_write is kv_layout = FPD_KV_NHD.  Head-
+ * major pages need num_blocks * block_tokens < 2^31.
+ */
+fpd_status fp8_paged_decode_cache_write_layout(const void *key, const void *value,
+                                               const int64_t *slot_mapping, int num_tokens,
+                                               int Hkv, int D, int64_t key_stride,
+                                               int64_t value_stride, float k_scale,
+                                               float v_scale, void *k_cache, void *v_cache,
+                                               int num_blocks, int block_tokens, int kv_layout,
+                                               uint32_t *status, void *stream);
+
+/*
+ * Reads the workspace status word (FPD_DEVERR_* bits) after synchronising
+ * `stream`; clears it when `clear` is nonzero.  Writes the bits to
+ * *device_error_bits.  Needs a workspace of at least 256 bytes.
+ */
 fpd_status fp8_paged_decode_check_status(void *workspace, void *stream, int *device_error_bits,
                                          int clear);
 

@@ -202,3 +202,47 @@ def test_attention_validates_before_any_launch(lib):
 def test_missing_library_fails_loudly(tmp_path):
     with pytest.raises(RuntimeError, match="no fallback"):
         fpd.load_library(str(tmp_path / "absent.so"))
+
+
+def base_args(**kw):
+    P = 4096   # never dereferenced: validation fails first (or B == 0 returns early)
+    a = fpd.fpd_decode_args()
+    a.q = a.k_cache = a.v_cache = a.block_table = a.seq_lens = a.out = P
+    a.B, a.q_len, a.Hq, a.Hkv, a.D = 2, 1, 8, 2, 128
+    a.num_blocks, a.block_tokens, a.max_blocks = 10, 16, 4
+    a.k_scale = a.v_scale = 1.0
+    a.sm_scale = 0.1
+    a.window_left = -1
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("field,value", [
+    ("q_token_stride", 7), ("q_token_stride", 8 * 128 - 8), ("out_token_stride", 1028),
+    ("q_dtype", 2), ("kv_layout", 2), ("sm_scale", 0.0), ("chunk_pages_override", -1),
+    ("k_scale", float("inf")),
+])
+def test_args_entry_validates_each_field(lib, field, value):
+    """Each field of the descriptor reaches its check (the C and Python struct
+    layouts agree); no CUDA call is made before these checks."""
+    f = lib.fp8_paged_decode_attention_args
+    ws = ctypes.c_void_p(4096)
+    assert f(ctypes.byref(base_args(**{field: value})), ws, 1 << 20, None) == \
+        fpd.FPD_ERR_INVALID_ARG
+    # a device k_scale lifts the host k_scale check
+    if field == "k_scale":
+        a = base_args(k_scale=float("inf"), k_scale_dev=4096, B=0)
+        assert f(ctypes.byref(a), ws, 1 << 20, None) == fpd.FPD_OK
+
+
+def test_args_entry_accepts_the_variants(lib):
+    f = lib.fp8_paged_decode_attention_args
+    ws = ctypes.c_void_p(4096)
+    for kw in (dict(), dict(q_dtype=fpd.FPD_Q_F16), dict(kv_layout=fpd.FPD_KV_HND),
+               dict(q_token_stride=8 * 128 + 8 * 3 * 128, out_token_stride=8 * 128 + 64),
+               dict(q_len=5)):
+        assert f(ctypes.byref(base_args(B=0, **kw)), ws, 1 << 20, None) == fpd.FPD_OK
+    assert f(None, ws, 1 << 20, None) == fpd.FPD_ERR_INVALID_ARG
+    # misaligned q base stays rejected through the descriptor
+    assert f(ctypes.byref(base_args(q=4100)), ws, 1 << 20, None) == fpd.FPD_ERR_INVALID_ARG
