@@ -104,20 +104,29 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, "fallback 6.65 TB/s (earlier measurement on this pool)"
 
 
+# The sources the E4M3 split and combine kernels and their launch are built
+# from; the ncu traffic record is valid only for this exact code.
+KERNEL_SOURCES = ("fpd_api.cu", "fpd_kernels.cuh", "fpd_ptx.cuh")
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "fp8_paged_decode_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
-        if fn.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, fn), "rb") as f:
-                h.update(fn.encode())
-                h.update(f.read())
+    for fn in KERNEL_SOURCES:
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(fn.encode())
+            h.update(f.read())
     return h.hexdigest()
 
 
-def ncu_traffic(config_name, kv_bytes):
+def traffic_key(config_name, q_len):
+    return config_name if q_len == 1 else f"{config_name}/q{q_len}"
+
+
+def ncu_traffic(config_name, kv_bytes, plan=None, q_len=1):
     """DRAM bytes per split-kernel launch from the committed ncu summary, scaled
-    to this launch's KV bytes; None when absent or taken on other kernel code."""
+    to this launch's KV bytes; None when absent, taken on other kernel code or
+    recorded for another launch plan."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
@@ -125,8 +134,10 @@ def ncu_traffic(config_name, kv_bytes):
         d = json.load(f)
     if d.get("source_sha256") != kernel_source_hash():
         return None
-    e = d.get("workloads", {}).get(config_name)
+    e = d.get("workloads", {}).get(traffic_key(config_name, q_len))
     if not e:
+        return None
+    if plan is not None and e.get("plan") is not None and e["plan"] != plan:
         return None
     return int(round(e["dram_bytes_per_launch"] * kv_bytes / e["kv_bytes_per_launch"]))
 
@@ -502,7 +513,7 @@ def run_native(args):
     split_avg_ms = statistics.fmean(split_ms)
     achieved = kv_bytes / (split_avg_ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                "frac": achieved / hbm, "traffic": ncu_traffic(args.config, kv_bytes),
+                "frac": achieved / hbm, "traffic": ncu_traffic(args.config, kv_bytes, plan, wl.q_len),
                 "kernel": f"fpd_split_kernel<{wl.D},{2 if wl.groups > 8 else 1}>",
                 "algorithmic_bytes_per_launch": kv_bytes,
                 "unit_bytes": f"2*D = {2 * wl.D} B per (attended token, KV head); "
