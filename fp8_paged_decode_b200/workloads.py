@@ -74,6 +74,11 @@ class Workload:
     v_dense: Optional[List[np.ndarray]] = None
     # Query tokens per sequence (the newest q_len positions, causal).
     q_len: int = 1
+    # "e4m3" (k_cache / v_cache) or "nvfp4": then kv_cache holds the pages,
+    # uint8 [num_blocks, page_bytes], each [K data | K scales | V data | V scales]
+    # with data [Hkv][bt][D/2] (E2M1 pairs) and scales [Hkv][bt][D/16] (E4M3).
+    kv_format: str = "e4m3"
+    kv_cache: Optional[np.ndarray] = None
 
     @property
     def groups(self) -> int:
@@ -87,8 +92,10 @@ class Workload:
         return L
 
     def kv_bytes(self) -> int:
-        """Algorithmic K+V bytes one decode call must read."""
-        return int(self.attended().sum()) * self.Hkv * self.D * 2
+        """Algorithmic K+V bytes one decode call must read (NVFP4: the E2M1 data
+        and the E4M3 block scales, D/2 + D/16 bytes per token and head and side)."""
+        per = self.D if self.kv_format == "e4m3" else self.D // 2 + self.D // 16
+        return int(self.attended().sum()) * self.Hkv * per * 2
 
     def io_bytes(self) -> int:
         """q in, out and lse out: B*q_len*Hq*(2D + 2D + 4) bytes."""
@@ -284,3 +291,121 @@ def make_workload(name: str, *, seed: Optional[int] = None, fill: str = "nan",
                        seq_lens=lens, window_left=c["window_left"], sinks=c["sinks"],
                        sm_scale=c["sm_scale"], sigma=c["sigma"], seed=s, fill=fill,
                        keep_dense=keep_dense, max_blocks=max_blocks, name=name, q_len=q_len)
+
+
+# ------------------------------------------------------------------ NVFP4 --
+
+# Magnitude distribution of the synthetic E2M1 codes (values 0, 0.5, 1, 1.5,
+# 2, 3, 4, 6): a bell shape like block-scaled normal data, in 1/128 steps.
+NVFP4_CODE_WEIGHTS = (12, 22, 22, 19, 17, 18, 12, 6)
+E4M3_SF_EXPONENTS = (5, 6, 7, 8)   # block scales 0.25 .. 3.75
+
+
+def _nibble_lut() -> np.ndarray:
+    """Random byte -> E2M1 code: bits 0..6 pick the magnitude by the weights,
+    bit 7 the sign."""
+    mag = np.repeat(np.arange(8, dtype=np.uint8), NVFP4_CODE_WEIGHTS)
+    assert mag.size == 128
+    lut = np.empty(256, dtype=np.uint8)
+    lut[:128] = mag
+    lut[128:] = mag | 0x8
+    return lut
+
+
+def _random_nvfp4_bytes(rng: np.random.Generator, n: int) -> np.ndarray:
+    """n bytes of two independent synthetic E2M1 codes each."""
+    lut = _nibble_lut()
+    r = rng.integers(0, 1 << 16, size=n, dtype=np.uint16)
+    return (lut[r & 0xFF] | (lut[r >> 8] << 4)).astype(np.uint8)
+
+
+def _random_sf_codes(rng: np.random.Generator, n: int) -> np.ndarray:
+    e = rng.choice(np.asarray(E4M3_SF_EXPONENTS, dtype=np.uint8), size=n)
+    m = rng.integers(0, 8, size=n, dtype=np.uint8)
+    return ((e << 3) | m).astype(np.uint8)
+
+
+def nvfp4_page_bytes(Hkv: int, bt: int, D: int) -> int:
+    return 2 * Hkv * bt * (D // 2 + D // 16)
+
+
+def make_custom_nvfp4(*, B: int, Hq: int, Hkv: int, D: int, block_tokens: int,
+                      seq_lens: Sequence[int], window_left: int = -1, sinks: bool = False,
+                      sm_scale: Optional[float] = None, seed: int = 0, spare_blocks: int = 16,
+                      max_blocks: Optional[int] = None, name: str = "custom-nvfp4",
+                      q_sigma: float = 1.0, sink_sigma: float = 1.0, q_len: int = 1,
+                      k_scale: float = 0.2, v_scale: float = 0.2) -> Workload:
+    """One decode step over NVFP4 pages (head-major, the page layout of
+    ``Workload.kv_cache``).  The E2M1 codes follow ``NVFP4_CODE_WEIGHTS`` with
+    random signs and the block scales are E4M3 values 0.25 .. 3.75; no
+    quantisation arithmetic is involved.  Every block scale of a slot the decode
+    must not read (before the window, past seq_len, spare pages) is the E4M3 NaN
+    code, so a leak shows up as NaN."""
+    assert Hq % Hkv == 0 and D % 16 == 0
+    lens = np.asarray(seq_lens, dtype=np.int64)
+    assert lens.shape == (B,) and (lens >= 0).all()
+    bt = block_tokens
+    root = np.random.SeedSequence([seed, 0xF4])
+    s_perm, s_q, s_data, s_sf, s_sink = root.spawn(5)
+    pages = -(-lens // bt)
+    if max_blocks is None:
+        max_blocks = int(max(1, pages.max() if B else 1))
+    assert (pages <= max_blocks).all()
+    num_blocks = max(int(pages.sum()) + spare_blocks, 1)
+    perm = np.random.default_rng(s_perm).permutation(num_blocks).astype(np.int32)
+    table = np.full((B, max_blocks), -1, dtype=np.int32)
+    off = 0
+    for b in range(B):
+        table[b, :pages[b]] = perm[off:off + pages[b]]
+        off += int(pages[b])
+    shape = (B, Hq, D) if q_len == 1 else (B, q_len, Hq, D)
+    q = _to_bf16_bits(_normal_f32(s_q, int(np.prod(shape)), q_sigma).reshape(shape))
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(D)
+
+    data_b, sf_b = Hkv * bt * D // 2, Hkv * bt * D // 16
+    page_bytes = 2 * (data_b + sf_b)
+    kv = np.empty((num_blocks, page_bytes), dtype=np.uint8)
+    rd, rs = np.random.default_rng(s_data), np.random.default_rng(s_sf)
+    for side in range(2):
+        base = side * (data_b + sf_b)
+        kv[:, base:base + data_b] = _random_nvfp4_bytes(rd, num_blocks * data_b).reshape(
+            num_blocks, data_b)
+        kv[:, base + data_b:base + data_b + sf_b] = _random_sf_codes(
+            rs, num_blocks * sf_b).reshape(num_blocks, sf_b)
+    # slots the decode must not read: NaN block scales
+    W = int(window_left)
+    starts = np.maximum(0, lens - q_len - W) if W >= 0 else np.zeros_like(lens)
+    valid = np.zeros((num_blocks, bt), dtype=bool)
+    for b in range(B):
+        j = np.arange(starts[b], lens[b], dtype=np.int64)
+        valid[table[b, j // bt], j % bt] = True
+    for side in range(2):
+        base = side * (data_b + sf_b) + data_b
+        sf = kv[:, base:base + sf_b].reshape(num_blocks, Hkv, bt, D // 16)
+        sf[np.broadcast_to(~valid[:, None, :, None], sf.shape)] = E4M3_NAN_CODE
+    sinks_arr = _normal_f32(s_sink, Hq, sink_sigma) if sinks else None
+    return Workload(name=name, seed=seed, B=B, Hq=Hq, Hkv=Hkv, D=D, block_tokens=bt,
+                    num_blocks=num_blocks, max_blocks=max_blocks, q=q, k_cache=None,
+                    v_cache=None, block_table=table, seq_lens=lens.astype(np.int32),
+                    k_scale=float(np.float32(k_scale)), v_scale=float(np.float32(v_scale)),
+                    sm_scale=float(np.float32(sm_scale)), window_left=W, sinks=sinks_arr,
+                    q_len=int(q_len), kv_format="nvfp4", kv_cache=kv)
+
+
+def make_workload_nvfp4(name: str, *, seed: Optional[int] = None, B: Optional[int] = None,
+                        q_len: int = 1) -> Workload:
+    """A named workload's shape, lengths, window and sinks over NVFP4 pages."""
+    c = CONFIGS[name]
+    s = c["seed"] if seed is None else seed
+    rng = np.random.default_rng(np.random.SeedSequence([s, 0x5EED]))
+    lens = _draw_lens(rng, c["B"], c["lens"])
+    nb = c["B"] if B is None else B
+    lens = lens[:nb]
+    bt = c["block_tokens"]
+    spec = c["lens"]
+    max_len = max(spec[1]) if spec[0] == "fixed" else (spec[2] if spec[0] == "uniform" else spec[4])
+    return make_custom_nvfp4(B=nb, Hq=c["Hq"], Hkv=c["Hkv"], D=c["D"], block_tokens=bt,
+                             seq_lens=lens, window_left=c["window_left"], sinks=c["sinks"],
+                             sm_scale=c["sm_scale"], seed=s, max_blocks=-(-max_len // bt),
+                             name=name + "-nvfp4", q_len=q_len)

@@ -52,6 +52,14 @@
  * token-major [num_blocks, bt, Hkv, D] ("NHD"); only the addressing of
  * element [page][slot][kvh][d] changes.
  *
+ * NVFP4 pages (the format of the NVFP4 KV-cache serving gist, its cache writer
+ * and the FlashInfer paged reader it routes to): each K or V element is an
+ * E2M1 code (4 bits; element 2i of a row in the low nibble of byte i) times
+ * the E4M3 scale of its block of 16 elements, times the per-tensor scale:
+ *   k_j[d] = k_scale * e2m1(code) * e4m3(sf[d / 16])
+ * Pages are head-major; a page holds a data region [Hkv][bt][D/2] and a
+ * scale region [Hkv][bt][D/16] per side, at caller-given page strides.
+ *
  * Degenerate cases: L == 0 gives out = 0 and lse = sigma (-inf without sinks).
  * A stored NaN code inside the attended range propagates NaN (plain
  * arithmetic); codes outside the attended range are never read.
@@ -99,6 +107,40 @@ double fpd_oracle_f16_to_f64(uint16_t bits)
     if (e == 0)
         return sign * ldexp((double)m / 1024.0, -14);
     return sign * ldexp(1.0 + (double)m / 1024.0, e - 15);
+}
+
+/* E2M1 code (low 4 bits) -> real value: 1 sign, 2 exponent (bias 1), 1
+ * mantissa bit; exponent 0 is subnormal (0 or 0.5).  Values 0, 0.5, 1, 1.5,
+ * 2, 3, 4, 6 and their negatives; no inf or NaN. */
+double fpd_oracle_e2m1_to_f64(uint8_t code)
+{
+    const int s = (code >> 3) & 1, e = (code >> 1) & 3, m = code & 1;
+    const double mag = e == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return s ? -mag : mag;
+}
+
+/* Real value -> E2M1 code: nearest value, ties to the even code, saturating
+ * at +-6; the sign of zero is kept.  A search over the 8 codes, which are
+ * increasing in value.  (NaN has no E2M1 code; it gives +0 here.) */
+uint8_t fpd_oracle_f64_to_e2m1(double x)
+{
+    const uint8_t sign = signbit(x) ? 0x8 : 0x0;
+    const double a = fabs(x);
+    int best = 0, c;
+    double best_d;
+    if (isnan(x))
+        return 0;
+    if (a >= 6.0)
+        return (uint8_t)(sign | 0x7);
+    best_d = a;
+    for (c = 1; c <= 7; ++c) {
+        const double d = fabs(a - fpd_oracle_e2m1_to_f64((uint8_t)c));
+        if (d < best_d || (d == best_d && (c & 1) == 0 && (best & 1) == 1)) {
+            best = c;
+            best_d = d;
+        }
+    }
+    return (uint8_t)(sign | best);
 }
 
 /* Byte offset of element [page][slot][kvh][0]: token-major pages
@@ -204,6 +246,9 @@ typedef struct {
     int window_left;
     int q_f16;           /* q holds IEEE fp16 bit patterns instead of bf16 */
     int kv_hnd;          /* head-major pages [num_blocks, Hkv, bt, D] */
+    int nvfp4;           /* NVFP4 pages: k_cache/v_cache hold the E2M1 data */
+    const uint8_t *k_sf, *v_sf;           /* NVFP4 block scales (E4M3) */
+    long data_page_stride, sf_page_stride; /* NVFP4 bytes between pages */
     const float *sinks;
     double *out, *lse;
     const int32_t *rows; /* list of (b * q_len + i) * Hq + h to compute, or NULL for all */
@@ -217,6 +262,19 @@ typedef struct {
 static size_t cache_row(const job_t *J, int page, int slot, int kvh)
 {
     return page_row(J->kv_hnd, page, slot, kvh, J->bt, J->Hkv, J->D);
+}
+
+/* NVFP4 element [page][slot][kvh][d] of one side without the per-tensor scale:
+ * data [page][kvh][slot][D/2] (two codes per byte, even d low), block scales
+ * [page][kvh][slot][D/16]. */
+static double nvfp4_elem(const job_t *J, const uint8_t *data, const uint8_t *sf, int page,
+                         int slot, int kvh, int d)
+{
+    const size_t row = (size_t)kvh * J->bt + slot;
+    const uint8_t byte = data[(size_t)page * J->data_page_stride + row * (J->D / 2) + d / 2];
+    const uint8_t code = (d & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 0xF);
+    const uint8_t sfc = sf[(size_t)page * J->sf_page_stride + row * (J->D / 16) + d / 16];
+    return fpd_oracle_e2m1_to_f64(code) * fpd_oracle_e4m3_to_f64(sfc);
 }
 
 static double q_value(const job_t *J, uint16_t bits)
@@ -254,9 +312,15 @@ static int one_row(const job_t *J, int row, double *s, double *acc)
         double dot = 0.0;
         if (page < 0 || page >= J->num_blocks)
             return -3;
+        if (J->nvfp4) {
+            for (d = 0; d < D; ++d)
+                dot += q_value(J, qr[d]) *
+                       (J->k_scale * nvfp4_elem(J, J->k_cache, J->k_sf, page, j % J->bt, kvh, d));
+        } else {
         kr = J->k_cache + cache_row(J, page, j % J->bt, kvh);
         for (d = 0; d < D; ++d)
             dot += q_value(J, qr[d]) * (J->k_scale * fpd_oracle_e4m3_to_f64(kr[d]));
+        }
         s[j - start] = J->sm_scale * dot;
         if (s[j - start] > m || isnan(s[j - start]))
             m = s[j - start];
@@ -277,8 +341,14 @@ static int one_row(const job_t *J, int row, double *s, double *acc)
         const uint8_t *vr = J->v_cache + cache_row(J, page, j % J->bt, kvh);
         const double p = exp(s[j - start] - m);
         Z += p;
+        if (J->nvfp4) {
+            for (d = 0; d < D; ++d)
+                acc[d] += p * (J->v_scale *
+                               nvfp4_elem(J, J->v_cache, J->v_sf, page, j % J->bt, kvh, d));
+        } else {
         for (d = 0; d < D; ++d)
             acc[d] += p * (J->v_scale * fpd_oracle_e4m3_to_f64(vr[d]));
+        }
     }
     Z += exp(sigma - m);
     for (d = 0; d < D; ++d)
@@ -368,6 +438,127 @@ int fpd_oracle_decode_x(const uint16_t *q, const uint8_t *k_cache, const uint8_t
     free(th);
     pthread_mutex_destroy(&J.mu);
     return J.status;
+}
+
+/*
+ * Decode over NVFP4 pages (head-major).  k_data / v_data: E2M1 codes,
+ * [page][kvh][slot][D/2] bytes at data_page_stride bytes per page; k_sf / v_sf:
+ * E4M3 block scales [page][kvh][slot][D/16] at sf_page_stride bytes per page
+ * (the writer's page [K data | K scales | V data | V scales] is four such
+ * pointers with one stride).  Everything else as fpd_oracle_decode_x.
+ */
+int fpd_oracle_decode_nvfp4(const uint16_t *q, const uint8_t *k_data, const uint8_t *k_sf,
+                            const uint8_t *v_data, const uint8_t *v_sf, long data_page_stride,
+                            long sf_page_stride, const int32_t *block_table,
+                            const int32_t *seq_lens, int B, int q_len, int Hq, int Hkv, int D,
+                            int num_blocks, int bt, int max_blocks, double k_scale,
+                            double v_scale, double sm_scale, int window_left,
+                            const float *sinks, double *out, double *lse, const int32_t *rows,
+                            int n_rows, int n_threads, int q_f16)
+{
+    job_t J;
+    pthread_t *th;
+    int t, i;
+    if (B < 0 || q_len < 1 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || D <= 0 || D % 16 != 0 ||
+        bt <= 0 || max_blocks < 0 || num_blocks < 0 || data_page_stride <= 0 ||
+        sf_page_stride <= 0)
+        return -1;
+    if (rows) {
+        for (i = 0; i < n_rows; ++i)
+            if (rows[i] < 0 || rows[i] >= B * q_len * Hq)
+                return -1;
+    }
+    memset(&J, 0, sizeof J);
+    J.q = q; J.k_cache = k_data; J.v_cache = v_data; J.k_sf = k_sf; J.v_sf = v_sf;
+    J.nvfp4 = 1; J.kv_hnd = 1;
+    J.data_page_stride = data_page_stride; J.sf_page_stride = sf_page_stride;
+    J.block_table = block_table; J.seq_lens = seq_lens;
+    J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.D = D; J.num_blocks = num_blocks; J.bt = bt;
+    J.max_blocks = max_blocks; J.q_len = q_len;
+    J.k_scale = k_scale; J.v_scale = v_scale; J.sm_scale = sm_scale;
+    J.window_left = window_left; J.sinks = sinks; J.out = out; J.lse = lse;
+    J.q_f16 = q_f16;
+    J.rows = rows; J.n_rows = n_rows;
+    pthread_mutex_init(&J.mu, NULL);
+    if (n_threads < 1)
+        n_threads = 1;
+    th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)n_threads);
+    for (t = 0; t < n_threads; ++t)
+        pthread_create(&th[t], NULL, worker, &J);
+    for (t = 0; t < n_threads; ++t)
+        pthread_join(th[t], NULL);
+    free(th);
+    pthread_mutex_destroy(&J.mu);
+    return J.status;
+}
+
+/*
+ * NVFP4 KV-cache write: the per-block quantisation of the gist's NVFP4 cache
+ * writer (its writer kernel and quantisation helper), with the reciprocals
+ * taken exactly in fp32 where the gist uses approximate ones:
+ *   gs    = 1 / scale                         (the per-tensor "global" scale)
+ *   sf    = e4m3_rne_sat((amax16 * (1/6)) * gs)   amax16 = max |x| of 16 elements
+ *   osc   = sf == 0 ? 0 : 1 / (e4m3(sf) * (1 / gs))
+ *   code  = e2m1_rne_sat(x * osc)
+ * every product and reciprocal rounded to fp32.  Token t goes to slot
+ * s = slot_mapping[t] (page s / bt, in-page slot s % bt); negative slots are
+ * skipped, slots past the end counted and skipped.  Layout as in
+ * fpd_oracle_decode_nvfp4.  Returns the count of out-of-range slots, or -1.
+ */
+int fpd_oracle_cache_write_nvfp4(const uint16_t *key, const uint16_t *value,
+                                 const int64_t *slot_mapping, int num_tokens, int Hkv, int D,
+                                 long key_stride, long value_stride, float k_scale,
+                                 float v_scale, uint8_t *k_data, uint8_t *k_sf, uint8_t *v_data,
+                                 uint8_t *v_sf, long data_page_stride, long sf_page_stride,
+                                 int num_blocks, int bt)
+{
+    const int64_t n_slots = (int64_t)num_blocks * bt;
+    int bad = 0, t, side, h, blk, i;
+    if (num_tokens < 0 || Hkv <= 0 || D <= 0 || D % 16 != 0 || num_blocks <= 0 || bt <= 0)
+        return -1;
+    for (t = 0; t < num_tokens; ++t) {
+        const int64_t slot = slot_mapping[t];
+        int page, off;
+        if (slot < 0)
+            continue;
+        if (slot >= n_slots) {
+            ++bad;
+            continue;
+        }
+        page = (int)(slot / bt);
+        off = (int)(slot % bt);
+        for (side = 0; side < 2; ++side) {
+            const uint16_t *src = side ? value + t * value_stride : key + t * key_stride;
+            const float gs = 1.0f / (side ? v_scale : k_scale);
+            uint8_t *data = side ? v_data : k_data;
+            uint8_t *sf = side ? v_sf : k_sf;
+            for (h = 0; h < Hkv; ++h) {
+                const size_t row = (size_t)h * bt + off;
+                for (blk = 0; blk < D / 16; ++blk) {
+                    float x[16], amax = 0.0f, sf_f, sf_v, osc;
+                    uint8_t sfc, codes[16];
+                    for (i = 0; i < 16; ++i) {
+                        x[i] = (float)fpd_oracle_bf16_to_f64(src[(long)h * D + blk * 16 + i]);
+                        if (fabsf(x[i]) > amax)
+                            amax = fabsf(x[i]);
+                    }
+                    sf_f = (amax * (1.0f / 6.0f)) * gs;
+                    sfc = fpd_oracle_f64_to_e4m3((double)sf_f);
+                    sf_v = (float)fpd_oracle_e4m3_to_f64(sfc);
+                    osc = sf_v == 0.0f ? 0.0f : 1.0f / (sf_v * (1.0f / gs));
+                    for (i = 0; i < 16; ++i) {
+                        const float y = x[i] * osc;
+                        codes[i] = fpd_oracle_f64_to_e2m1((double)y);
+                    }
+                    for (i = 0; i < 8; ++i)
+                        data[(size_t)page * data_page_stride + row * (D / 2) + blk * 8 + i] =
+                            (uint8_t)(codes[2 * i] | (codes[2 * i + 1] << 4));
+                    sf[(size_t)page * sf_page_stride + row * (D / 16) + blk] = sfc;
+                }
+            }
+        }
+    }
+    return bad;
 }
 
 /* bf16 q, token-major pages. */

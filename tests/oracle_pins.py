@@ -98,7 +98,8 @@ def close(a, b, rtol=1e-12, atol=1e-12, what=""):
     a = np.asarray(a, dtype=np.float64)
     b = np.asarray(b, dtype=np.float64)
     same_inf = np.isinf(a) & np.isinf(b) & (np.sign(a) == np.sign(b))
-    ok = same_inf | (np.abs(a - b) <= atol + rtol * np.abs(b))
+    with np.errstate(invalid="ignore"):
+        ok = same_inf | (np.abs(a - b) <= atol + rtol * np.abs(b))
     if not ok.all():
         i = np.argwhere(~ok)[0]
         raise AssertionError(f"{what}: mismatch at {tuple(i)}: {a[tuple(i)]!r} vs {b[tuple(i)]!r}")
@@ -542,8 +543,238 @@ def bf16_bits_of(x: np.ndarray) -> np.ndarray:
     return t.view(torch.int16).numpy().view(np.uint16)
 
 
+# ------------------------------------------------------------------ NVFP4 --
+
+def e2m1_library(codes: np.ndarray) -> np.ndarray:
+    """E2M1 codes (low 4 bits) -> float64 by ml_dtypes' float4_e2m1fn (library)."""
+    import ml_dtypes
+    return np.ascontiguousarray(codes, dtype=np.uint8).view(ml_dtypes.float4_e2m1fn) \
+        .astype(np.float64)
+
+
+def nvfp4_dense(wl, side):
+    """Dense [num_blocks, Hkv, bt, D] real values (without the per-tensor scale)
+    of one side of an NVFP4 workload's pages, by numpy views of the page bytes,
+    ml_dtypes' E2M1 and torch's E4M3 decoding."""
+    lay = oracle.nvfp4_page_layout(wl.Hkv, wl.block_tokens, wl.D)
+    nb, Hkv, bt, D = wl.num_blocks, wl.Hkv, wl.block_tokens, wl.D
+    d0 = lay["k_data" if side == 0 else "v_data"]
+    s0 = lay["k_sf" if side == 0 else "v_sf"]
+    data = wl.kv_cache[:, d0:d0 + Hkv * bt * D // 2].reshape(nb, Hkv, bt, D // 2)
+    sf = wl.kv_cache[:, s0:s0 + Hkv * bt * D // 16].reshape(nb, Hkv, bt, D // 16)
+    codes = np.empty((nb, Hkv, bt, D), dtype=np.uint8)
+    codes[..., 0::2] = data & 0xF
+    codes[..., 1::2] = data >> 4
+    return e2m1_library(codes) * np.repeat(e4m3_library(sf), 16, axis=-1)
+
+
+def nvfp4_cases():
+    return [
+        W.make_custom_nvfp4(B=3, Hq=8, Hkv=2, D=64, block_tokens=16, seq_lens=[1, 40, 100],
+                            sinks=True, seed=71),
+        W.make_custom_nvfp4(B=2, Hq=16, Hkv=4, D=128, block_tokens=32, seq_lens=[70, 129],
+                            window_left=50, sinks=True, seed=72, sm_scale=0.1, q_len=3),
+        W.make_custom_nvfp4(B=2, Hq=4, Hkv=4, D=128, block_tokens=64, seq_lens=[0, 200],
+                            seed=73),
+    ]
+
+
+def pin_e2m1_codes(lib):
+    """All 16 E2M1 codes against ml_dtypes."""
+    codes = np.arange(16, dtype=np.uint8)
+    got = np.array([lib.fpd_oracle_e2m1_to_f64(int(c)) for c in codes])
+    want = e2m1_library(codes)
+    assert np.array_equal(got, want) and np.array_equal(np.signbit(got), np.signbit(want)), \
+        "E2M1 decode differs from ml_dtypes"
+
+
+def pin_e2m1_encode_library(lib):
+    """Nearest-even, saturating E2M1 encoding against ml_dtypes' cast, on ties,
+    overflow, tiny values and random values of both signs."""
+    import ml_dtypes
+    rng = np.random.default_rng(74)
+    ties = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    x = np.concatenate([ties, -ties, [0.0, -0.0, 6.0, 6.5, 7.0, 1e9, -1e9, np.inf, -np.inf,
+                                      1e-30, -1e-30], rng.standard_normal(4000) * 3,
+                        rng.uniform(-8, 8, 4000)])
+    got = np.array([lib.fpd_oracle_f64_to_e2m1(float(v)) for v in x], dtype=np.uint8)
+    want = x.astype(ml_dtypes.float4_e2m1fn).view(np.uint8) & 0xF
+    assert np.array_equal(got, want), \
+        f"E2M1 encode differs at {x[np.argmax(got != want)]!r}"
+
+
+def pin_nvfp4_decode_library(lib):
+    """NVFP4 decode against torch SDPA and scipy logsumexp on the pages'
+    values decoded by numpy views, ml_dtypes and torch (float64)."""
+    for wl in nvfp4_cases():
+        out, lse = oracle.decode_nvfp4_workload(wl, lib=lib, threads=2)
+        Kd, Vd = nvfp4_dense(wl, 0), nvfp4_dense(wl, 1)
+        Q = wl.q_len
+        qf = bf16_library(wl.q).reshape(wl.B, Q, wl.Hq, wl.D)
+        g = wl.Hq // wl.Hkv
+        sig = wl.sinks.astype(np.float64) if wl.sinks is not None else None
+        ro = np.zeros((wl.B, Q, wl.Hq, wl.D))
+        rl = np.zeros((wl.B, Q, wl.Hq))
+        for b in range(wl.B):
+            L = int(wl.seq_lens[b])
+            j = np.arange(L)
+            pages = wl.block_table[b, j // wl.block_tokens]
+            K = Kd[pages, :, j % wl.block_tokens] * wl.k_scale    # [L, Hkv, D]
+            V = Vd[pages, :, j % wl.block_tokens] * wl.v_scale
+            for i in range(Q):
+                p = L - Q + i
+                lo = max(0, p - wl.window_left) if wl.window_left >= 0 else 0
+                n = max(0, p + 1 - lo)
+                Kt = torch.zeros((1, wl.Hkv, n + 1, wl.D), dtype=torch.float64)
+                Vt = torch.zeros_like(Kt)
+                if n:
+                    Kt[0, :, :n] = torch.from_numpy(K[lo:p + 1]).permute(1, 0, 2)
+                    Vt[0, :, :n] = torch.from_numpy(V[lo:p + 1]).permute(1, 0, 2)
+                mask = torch.zeros((1, wl.Hq, 1, n + 1), dtype=torch.float64)
+                mask[0, :, 0, n] = torch.from_numpy(sig) if sig is not None else -math.inf
+                if n == 0 and sig is None:
+                    ro[b, i] = 0.0
+                    rl[b, i] = -np.inf
+                    continue
+                qt = torch.from_numpy(qf[b, i]).reshape(1, wl.Hq, 1, wl.D)
+                o = F.scaled_dot_product_attention(qt, Kt, Vt, attn_mask=mask,
+                                                   scale=wl.sm_scale, enable_gqa=True)
+                ro[b, i] = o[0, :, 0].numpy()
+                sc = wl.sm_scale * np.einsum("hd,nhd->hn", qf[b, i],
+                                             np.repeat(K[lo:p + 1], g, axis=1))
+                if sig is not None:
+                    sc = np.concatenate([sc, sig[:, None]], axis=1)
+                rl[b, i] = scipy.special.logsumexp(sc, axis=1)
+        close(out.reshape(ro.shape), ro, rtol=1e-10, atol=1e-12, what=f"{wl.name} NVFP4 out")
+        close(lse.reshape(rl.shape), rl, rtol=1e-12, atol=1e-12, what=f"{wl.name} NVFP4 lse")
+
+
+def pin_nvfp4_page_strides(lib):
+    """The four page regions as separate arrays (their own page strides) give
+    the bits of the combined page layout."""
+    for wl in nvfp4_cases():
+        lay = oracle.nvfp4_page_layout(wl.Hkv, wl.block_tokens, wl.D)
+        nb, shp = wl.num_blocks, (wl.num_blocks, wl.Hkv, wl.block_tokens)
+        db, sb = wl.Hkv * wl.block_tokens * wl.D // 2, wl.Hkv * wl.block_tokens * wl.D // 16
+        reg = tuple(np.ascontiguousarray(wl.kv_cache[:, lay[k]:lay[k] + n]).reshape(shp + (n // (shp[1] * shp[2]),))
+                    for k, n in (("k_data", db), ("k_sf", sb), ("v_data", db), ("v_sf", sb)))
+        kw = dict(Hkv=wl.Hkv, block_tokens=wl.block_tokens, k_scale=wl.k_scale,
+                  v_scale=wl.v_scale, sm_scale=wl.sm_scale, window_left=wl.window_left,
+                  sinks=wl.sinks, lib=lib, threads=2)
+        o1, l1 = oracle.decode_nvfp4(wl.q, wl.kv_cache, wl.block_table, wl.seq_lens, **kw)
+        o2, l2 = oracle.decode_nvfp4(wl.q, None, wl.block_table, wl.seq_lens, regions=reg, **kw)
+        assert np.array_equal(o1, o2, equal_nan=True) and np.array_equal(l1, l2, equal_nan=True), \
+            "separate page regions differ from the combined page"
+        del nb
+
+
+def nvfp4_writer_library(key_bits, value_bits, k_scale, v_scale):
+    """The writer's codes by library roundings: torch's E4M3 cast for the block
+    scale, ml_dtypes' E2M1 cast for the elements, numpy float32 products."""
+    import ml_dtypes
+    T, Hkv, D = key_bits.shape
+    res = []
+    for bits, scale in ((key_bits, k_scale), (value_bits, v_scale)):
+        x = bf16_library(bits).astype(np.float32).reshape(T, Hkv, D // 16, 16)
+        gs = np.float32(1.0) / np.float32(scale)
+        amax = np.abs(x).max(axis=-1)
+        sf_f = (amax * (np.float32(1.0) / np.float32(6.0))) * gs
+        sfc = torch.from_numpy(sf_f.astype(np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        sfv = e4m3_library(sfc).astype(np.float32)
+        with np.errstate(divide="ignore"):
+            osc = np.where(sfv == 0, np.float32(0),
+                           np.float32(1.0) / (sfv * (np.float32(1.0) / gs))).astype(np.float32)
+        y = (x * osc[..., None]).astype(np.float32)
+        codes = y.astype(np.float64).astype(ml_dtypes.float4_e2m1fn).view(np.uint8) & 0xF
+        res.append((codes.reshape(T, Hkv, D), sfc))
+    return res
+
+
+def pin_nvfp4_writer_library(lib):
+    """The NVFP4 cache writer's codes and block scales against the same
+    recipe computed with library roundings; slots land in the page layout."""
+    rng = np.random.default_rng(75)
+    for Hkv, D, bt, T in ((2, 64, 16, 40), (4, 128, 32, 70)):
+        x = rng.standard_normal((2, T, Hkv, D)).astype(np.float32) * 2
+        x[:, ::7, :, :16] *= 1e-3
+        x[:, 3, 0, 16:32] = 0.0                          # an all-zero block
+        kb, vb = (torch.from_numpy(x[i]).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+                  for i in range(2))
+        nb = T // bt + 3
+        lay = oracle.nvfp4_page_layout(Hkv, bt, D)
+        kv = np.zeros((nb, lay["page_bytes"]), dtype=np.uint8)
+        slots = rng.permutation(nb * bt)[:T].astype(np.int64)
+        slots[::5] = -1
+        ks, vs = 0.05, 0.03
+        assert oracle.cache_write_nvfp4(kb, vb, slots, kv, block_tokens=bt, k_scale=ks,
+                                        v_scale=vs, lib=lib) == 0
+        (kc, ksf), (vc, vsf) = nvfp4_writer_library(kb, vb, np.float32(ks), np.float32(vs))
+        for side, (codes, sfc) in enumerate(((kc, ksf), (vc, vsf))):
+            d0 = lay["k_data" if side == 0 else "v_data"]
+            s0 = lay["k_sf" if side == 0 else "v_sf"]
+            data = kv[:, d0:d0 + Hkv * bt * D // 2].reshape(nb, Hkv, bt, D // 2)
+            sf = kv[:, s0:s0 + Hkv * bt * D // 16].reshape(nb, Hkv, bt, D // 16)
+            for t in range(T):
+                if slots[t] < 0:
+                    continue
+                pg, off = divmod(int(slots[t]), bt)
+                got = np.empty((Hkv, D), dtype=np.uint8)
+                got[:, 0::2] = data[pg, :, off] & 0xF
+                got[:, 1::2] = data[pg, :, off] >> 4
+                assert np.array_equal(got, codes[t]), f"side {side} token {t}: codes differ"
+                assert np.array_equal(sf[pg, :, off], sfc[t]), f"side {side} token {t}: scales differ"
+
+
+def pin_nvfp4_round_trip(lib):
+    """Closed forms of the write -> decode round trip: values c * s * k_scale
+    with c an E2M1 value, max |c| = 6 per block, s a power of two and k_scale a
+    power of two come back exactly; an all-zero block gives scale code 0; on
+    random data every element is within one block step (scale * k_scale) of
+    its input."""
+    rng = np.random.default_rng(76)
+    Hkv, D, bt, T = 2, 64, 16, 20
+    vals = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], dtype=np.float64)
+    c = vals[rng.integers(0, 8, (T, Hkv, D // 16, 16))] * rng.choice([-1.0, 1.0], (T, Hkv, D // 16, 16))
+    c[..., 0] = 6.0
+    s = 2.0 ** rng.integers(-4, 5, (T, Hkv, D // 16, 1))
+    k_scale = 0.125
+    x = (c * s * k_scale).reshape(T, Hkv, D)
+    x[0, 1, :16] = 0.0
+    bits = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(bf16_library(bits), x)
+    nb = T // bt + 2
+    lay = oracle.nvfp4_page_layout(Hkv, bt, D)
+    kv = np.zeros((nb, lay["page_bytes"]), dtype=np.uint8)
+    slots = np.arange(T, dtype=np.int64)
+    oracle.cache_write_nvfp4(bits, bits, slots, kv, block_tokens=bt, k_scale=k_scale,
+                             v_scale=k_scale, lib=lib)
+    wl = W.Workload(name="rt", seed=0, B=1, Hq=Hkv, Hkv=Hkv, D=D, block_tokens=bt, num_blocks=nb,
+                    max_blocks=nb, q=np.zeros((1, Hkv, D), np.uint16), k_cache=None, v_cache=None,
+                    block_table=np.arange(nb, dtype=np.int32)[None], seq_lens=np.array([T], np.int32),
+                    k_scale=k_scale, v_scale=k_scale, sm_scale=1.0, window_left=-1, sinks=None,
+                    kv_format="nvfp4", kv_cache=kv)
+    dense = nvfp4_dense(wl, 0).transpose(0, 2, 1, 3).reshape(nb * bt, Hkv, D)[:T] * k_scale
+    assert np.array_equal(dense, x), "exactly representable blocks do not round-trip"
+    sf = kv[:, lay["k_sf"]:lay["k_sf"] + Hkv * bt * D // 16].reshape(nb, Hkv, bt, D // 16)
+    assert sf[0, 1, 0, 0] == 0, "an all-zero block must get scale code 0"
+    # random data: within one block step
+    y = rng.standard_normal((T, Hkv, D)).astype(np.float32)
+    yb = torch.from_numpy(y).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    kv2 = np.zeros_like(kv)
+    oracle.cache_write_nvfp4(yb, yb, slots, kv2, block_tokens=bt, k_scale=0.02, v_scale=0.02,
+                             lib=lib)
+    wl.kv_cache, wl.k_scale = kv2, 0.02
+    d2 = nvfp4_dense(wl, 0).transpose(0, 2, 1, 3).reshape(nb * bt, Hkv, D)[:T] * 0.02
+    sf2 = kv2[:, lay["k_sf"]:lay["k_sf"] + Hkv * bt * D // 16].reshape(nb, Hkv, bt, D // 16)
+    step = np.repeat(e4m3_library(sf2).transpose(0, 2, 1, 3).reshape(nb * bt, Hkv, D // 16)[:T],
+                     16, axis=-1) * 0.02
+    assert (np.abs(d2 - bf16_library(yb)) <= step + 1e-12).all(), "round-trip error above one step"
+
+
 ALL_PINS = [pin_e4m3_codes, pin_bf16, pin_library_attention, pin_zero_keys, pin_window_zero,
             pin_constant_values, pin_invariants, pin_softmax_identity, pin_e4m3_encode_library,
             pin_e4m3_encode_closed, pin_cache_write_library, pin_cache_write_invariants,
             pin_multi_token_library, pin_multi_token_prefix, pin_f16_codes,
-            pin_f16_query_library, pin_hnd_layout]
+            pin_f16_query_library, pin_hnd_layout, pin_e2m1_codes, pin_e2m1_encode_library,
+            pin_nvfp4_decode_library, pin_nvfp4_page_strides, pin_nvfp4_writer_library,
+            pin_nvfp4_round_trip]

@@ -32,6 +32,18 @@ MUTANTS = {
     "fp16 exponent bias 16": [("(1.0 + (double)m / 1024.0, e - 15)",
                                "(1.0 + (double)m / 1024.0, e - 16)")],
     "fp16 subnormal scale": [("ldexp((double)m / 1024.0, -14)", "ldexp((double)m / 1024.0, -15)")],
+    "NVFP4 nibble order swapped": [
+        ("(d & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 0xF)",
+         "(d & 1) ? (uint8_t)(byte & 0xF) : (uint8_t)(byte >> 4)")],
+    "NVFP4 scale of the neighbouring block": [("row * (J->D / 16) + d / 16]",
+                                               "row * (J->D / 16) + ((d / 16) ^ 1)]")],
+    "E2M1 subnormal value": [("e == 0 ? 0.5 * m :", "e == 0 ? 0.25 * m :")],
+    "E2M1 exponent bias 2": [("ldexp(1.0 + 0.5 * m, e - 1)", "ldexp(1.0 + 0.5 * m, e - 2)")],
+    "NVFP4 writer amax / 8": [("sf_f = (amax * (1.0f / 6.0f)) * gs;", "sf_f = (amax * (1.0f / 8.0f)) * gs;")],
+    "NVFP4 writer ignores the block scale": [
+        ("osc = sf_v == 0.0f ? 0.0f : 1.0f / (sf_v * (1.0f / gs));", "osc = sf_v == 0.0f ? 0.0f : gs;")],
+    "NVFP4 writer nibbles swapped": [("(uint8_t)(codes[2 * i] | (codes[2 * i + 1] << 4))",
+                                      "(uint8_t)(codes[2 * i + 1] | (codes[2 * i] << 4))")],
     "fp16 query decoded as bf16": [("return J->q_f16 ? fpd_oracle_f16_to_f64(bits) :",
                                     "return 0 ? fpd_oracle_f16_to_f64(bits) :")],
     "in-page slot reversed": [("j % J->bt, kvh)", "J->bt - 1 - j % J->bt, kvh)")],
