@@ -30,6 +30,8 @@ __all__ = [
     "FpdError", "library_path", "load_library", "fp8_paged_decode_make_plan",
     "fp8_paged_decode_make_plan_qlen", "FPD_MAX_Q_LEN", "FPD_KV_NHD", "FPD_KV_HND",
     "FPD_Q_BF16", "FPD_Q_F16", "fpd_decode_args", "fp8_paged_decode_cache_write_layout",
+    "FPD_KV_E4M3", "FPD_KV_NVFP4", "nvfp4_page_layout", "fp8_paged_decode_attention_nvfp4",
+    "fp8_paged_decode_cache_write_nvfp4", "fp8_paged_decode_workspace_bytes_args",
     "fp8_paged_decode_plan", "fp8_paged_decode_workspace_bytes",
     "fp8_paged_decode_workspace_bytes_ex", "fp8_paged_decode_attention_profiled",
     "fp8_paged_decode_attention", "fp8_paged_decode_attention_ex",
@@ -54,6 +56,8 @@ FPD_KV_NHD = 0
 FPD_KV_HND = 1
 FPD_Q_BF16 = 0
 FPD_Q_F16 = 1
+FPD_KV_E4M3 = 0
+FPD_KV_NVFP4 = 1
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_NAME = "libfp8_paged_decode.so"
@@ -76,7 +80,11 @@ EXPORTED_SYMBOLS = (
     "fp8_paged_decode_cache_write",
     "fp8_paged_decode_attention_qlen",
     "fp8_paged_decode_attention_args",
+    "fp8_paged_decode_attention_args_profiled",
+    "fp8_paged_decode_plan_args",
+    "fp8_paged_decode_workspace_bytes_args",
     "fp8_paged_decode_cache_write_layout",
+    "fp8_paged_decode_cache_write_nvfp4",
     "fp8_paged_decode_plan_qlen",
     "fp8_paged_decode_workspace_bytes_qlen",
     "fp8_paged_decode_status_string",
@@ -114,7 +122,9 @@ class fpd_decode_args(ctypes.Structure):
                 ("sm_scale", ctypes.c_float), ("window_left", ctypes.c_int),
                 ("sinks", ctypes.c_void_p), ("out", ctypes.c_void_p),
                 ("out_token_stride", ctypes.c_int64), ("lse", ctypes.c_void_p),
-                ("chunk_pages_override", ctypes.c_int)]
+                ("chunk_pages_override", ctypes.c_int), ("kv_format", ctypes.c_int),
+                ("k_scales", ctypes.c_void_p), ("v_scales", ctypes.c_void_p),
+                ("kv_page_stride", ctypes.c_int64), ("sf_page_stride", ctypes.c_int64)]
 
 
 def library_path() -> str:
@@ -145,6 +155,18 @@ def _bind(lib):
     lib.fp8_paged_decode_attention_qlen.restype = ci
     lib.fp8_paged_decode_attention_args.argtypes = [ctypes.POINTER(fpd_decode_args), vp, cz, vp]
     lib.fp8_paged_decode_attention_args.restype = ci
+    lib.fp8_paged_decode_attention_args_profiled.argtypes = [ctypes.POINTER(fpd_decode_args), vp,
+                                                             cz, vp, vp, vp, vp]
+    lib.fp8_paged_decode_attention_args_profiled.restype = ci
+    lib.fp8_paged_decode_plan_args.argtypes = [ctypes.POINTER(fpd_decode_args),
+                                               ctypes.POINTER(fpd_plan)]
+    lib.fp8_paged_decode_plan_args.restype = ci
+    lib.fp8_paged_decode_workspace_bytes_args.argtypes = [ctypes.POINTER(fpd_decode_args)]
+    lib.fp8_paged_decode_workspace_bytes_args.restype = cz
+    i64 = ctypes.c_int64
+    lib.fp8_paged_decode_cache_write_nvfp4.argtypes = [vp, vp, vp, ci, ci, ci, i64, i64, cf, cf,
+                                                       vp, vp, vp, vp, i64, i64, ci, ci, vp, vp]
+    lib.fp8_paged_decode_cache_write_nvfp4.restype = ci
     lib.fp8_paged_decode_plan_qlen.argtypes = [ci] * 9 + [ctypes.POINTER(fpd_plan)]
     lib.fp8_paged_decode_plan_qlen.restype = ci
     lib.fp8_paged_decode_workspace_bytes_qlen.argtypes = [ci] * 9
@@ -458,3 +480,121 @@ def fp8_paged_decode_workspace_init(workspace, stream=None):
         _dev_ptr(workspace, "workspace", (torch.uint8,)), ctypes.c_size_t(workspace.numel()),
         _stream_handle(stream))
     _check(st, "fp8_paged_decode_workspace_init")
+
+
+# ------------------------------------------------------------------ NVFP4 --
+
+def nvfp4_page_layout(Hkv: int, block_tokens: int, D: int) -> dict:
+    """Byte offsets inside one NVFP4 page [K data | K scales | V data | V scales]
+    (data [Hkv][bt][D/2], scales [Hkv][bt][D/16] per side) and the page size."""
+    data = Hkv * block_tokens * D // 2
+    sf = Hkv * block_tokens * D // 16
+    return dict(k_data=0, k_sf=data, v_data=data + sf, v_sf=2 * data + sf,
+                page_bytes=2 * (data + sf))
+
+
+def _nvfp4_pointers(kv_pages, Hkv, block_tokens, D):
+    import torch
+    lay = nvfp4_page_layout(Hkv, block_tokens, D)
+    if not isinstance(kv_pages, torch.Tensor) or not kv_pages.is_cuda or kv_pages.dtype != torch.uint8:
+        raise TypeError("kv_pages must be a uint8 CUDA tensor")
+    if kv_pages.dim() != 2 or kv_pages.shape[1] != lay["page_bytes"] or not kv_pages.is_contiguous():
+        raise ValueError(f"kv_pages must be contiguous [num_blocks, {lay['page_bytes']}]")
+    base = kv_pages.data_ptr()
+    return {k: base + lay[k] for k in ("k_data", "k_sf", "v_data", "v_sf")}, lay["page_bytes"]
+
+
+def fp8_paged_decode_attention_nvfp4(q, kv_pages, block_table, seq_lens, k_scale, v_scale,
+                                     sm_scale, *, Hkv, block_tokens, window_left=-1, sinks=None,
+                                     out=None, lse=None, workspace=None, stream=None,
+                                     chunk_pages_override=0, return_lse=True):
+    """Decode over NVFP4 pages: ``kv_pages`` uint8 [num_blocks, page_bytes], each
+    page [K data | K scales | V data | V scales] (``nvfp4_page_layout``; head-major
+    E2M1 pairs, element 2i in the low nibble, and one E4M3 scale per 16
+    elements).  An element is e2m1(code) * e4m3(block scale) * k_scale
+    (v_scale).  q, out, lse, scales and the rest as ``fp8_paged_decode_attention``."""
+    import torch
+    if q.dim() == 3:
+        B, Hq, D = q.shape
+        q_len = 1
+    else:
+        B, q_len, Hq, D = q.shape
+    lead = tuple(q.shape[:-2])
+    ptrs, page_bytes = _nvfp4_pointers(kv_pages, Hkv, block_tokens, D)
+    num_blocks = kv_pages.shape[0]
+    max_blocks = block_table.shape[1]
+    dev = q.device
+    if out is None:
+        out = torch.empty(lead + (Hq, D), dtype=torch.bfloat16, device=dev)
+    if lse is None and return_lse:
+        lse = torch.empty(lead + (Hq,), dtype=torch.float32, device=dev)
+    if q.dtype not in (torch.bfloat16, torch.float16) or out.dtype != torch.bfloat16:
+        raise TypeError("q must be bf16 or fp16 and out bf16")
+    a = fpd_decode_args()
+    a.q = q.data_ptr()
+    a.q_dtype = FPD_Q_F16 if q.dtype == torch.float16 else FPD_Q_BF16
+    a.q_token_stride = _token_rows(q, "q", lead, Hq, D)
+    a.k_cache, a.v_cache = ptrs["k_data"], ptrs["v_data"]
+    a.k_scales, a.v_scales = ptrs["k_sf"], ptrs["v_sf"]
+    a.kv_page_stride = a.sf_page_stride = page_bytes
+    a.kv_format = FPD_KV_NVFP4
+    a.kv_layout = FPD_KV_HND
+    a.block_table = _dev_ptr(block_table, "block_table", (torch.int32,), (B, max_blocks)).value
+    a.seq_lens = _dev_ptr(seq_lens, "seq_lens", (torch.int32,), (B,)).value
+    a.B, a.q_len, a.Hq, a.Hkv, a.D = B, q_len, Hq, Hkv, D
+    a.num_blocks, a.block_tokens, a.max_blocks = num_blocks, block_tokens, max_blocks
+    a.k_scale, a.k_scale_dev = _scale_arg(k_scale, "k_scale")
+    a.v_scale, a.v_scale_dev = _scale_arg(v_scale, "v_scale")
+    a.sm_scale = float(sm_scale)
+    a.window_left = int(window_left)
+    sp = _dev_ptr(sinks, "sinks", (torch.float32,), (Hq,))
+    a.sinks = sp.value if sp is not None else None
+    a.out = out.data_ptr()
+    a.out_token_stride = _token_rows(out, "out", lead, Hq, D)
+    lp = _dev_ptr(lse, "lse", (torch.float32,), lead + (Hq,))
+    a.lse = lp.value if lp is not None else None
+    a.chunk_pages_override = int(chunk_pages_override)
+    lib = load_library()
+    if workspace is None:
+        need = int(lib.fp8_paged_decode_workspace_bytes_args(ctypes.byref(a)))
+        if need == 0 and B > 0:
+            plan = fpd_plan()
+            _check(lib.fp8_paged_decode_plan_args(ctypes.byref(a), ctypes.byref(plan)),
+                   "fp8_paged_decode_plan_args")
+            raise FpdError(FPD_ERR_UNSUPPORTED, "fp8_paged_decode_workspace_bytes_args")
+        workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)
+    st = lib.fp8_paged_decode_attention_args(
+        ctypes.byref(a), _dev_ptr(workspace, "workspace", (torch.uint8,)),
+        ctypes.c_size_t(workspace.numel()), _stream_handle(stream))
+    _check(st, "fp8_paged_decode_attention_nvfp4")
+    return out, lse
+
+
+def fp8_paged_decode_workspace_bytes_args(args) -> int:
+    return int(load_library().fp8_paged_decode_workspace_bytes_args(ctypes.byref(args)))
+
+
+def fp8_paged_decode_cache_write_nvfp4(key, value, slot_mapping, kv_pages, k_scale, v_scale, *,
+                                       block_tokens, status=None, stream=None):
+    """Enqueue the NVFP4 KV-cache write: bf16 ``key``/``value`` [num_tokens, Hkv,
+    D] (rows contiguous, token stride a multiple of 8) quantised per 16-element
+    block into ``kv_pages`` (uint8 [num_blocks, page_bytes], ``nvfp4_page_layout``)
+    at ``slot_mapping`` (int64, negative = skip)."""
+    import torch
+    T, Hkv, D = key.shape
+    if tuple(value.shape) != (T, Hkv, D):
+        raise ValueError("key and value disagree on shape")
+    for name, t in (("key", key), ("value", value)):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be a bf16 CUDA tensor")
+        if t.stride(2) != 1 or t.stride(1) != D:
+            raise ValueError(f"{name} rows must be contiguous")
+    ptrs, page_bytes = _nvfp4_pointers(kv_pages, Hkv, block_tokens, D)
+    vp = ctypes.c_void_p
+    st = load_library().fp8_paged_decode_cache_write_nvfp4(
+        vp(key.data_ptr()), vp(value.data_ptr()),
+        _dev_ptr(slot_mapping, "slot_mapping", (torch.int64,), (T,)), T, Hkv, D, key.stride(0),
+        value.stride(0), float(k_scale), float(v_scale), vp(ptrs["k_data"]), vp(ptrs["k_sf"]),
+        vp(ptrs["v_data"]), vp(ptrs["v_sf"]), page_bytes, page_bytes, kv_pages.shape[0],
+        block_tokens, _dev_ptr(status, "status", (torch.int32,)), _stream_handle(stream))
+    _check(st, "fp8_paged_decode_cache_write_nvfp4")

@@ -85,10 +85,20 @@ int heads_per_stage(int Hkv) { return Hkv % 4 == 0 ? 4 : 1; }
 #ifndef FPD_STAGES_HB4_D64
 #define FPD_STAGES_HB4_D64 5
 #endif
-int ring_stages(int D, int NT, int HB) {
-  if (HB == 4) return D == 128 ? FPD_STAGES_HB4_D128 : FPD_STAGES_HB4_D64;
-  if (D == 128) return NT == 2 ? FPD_STAGES_D128_NT2 : FPD_STAGES_D128_NT1;
-  return FPD_STAGES_D64;
+// NVFP4 stages are 72 D bytes instead of 128 D: the ring keeps about the same
+// bytes in flight with 16 / 9 as many stages.
+#ifndef FPD_FP4_STAGES_NUM
+#define FPD_FP4_STAGES_NUM 16
+#endif
+#ifndef FPD_FP4_STAGES_DEN
+#define FPD_FP4_STAGES_DEN 9
+#endif
+int ring_stages(int D, int NT, int HB, bool fp4 = false) {
+  int s;
+  if (HB == 4) s = D == 128 ? FPD_STAGES_HB4_D128 : FPD_STAGES_HB4_D64;
+  else if (D == 128) s = NT == 2 ? FPD_STAGES_D128_NT2 : FPD_STAGES_D128_NT1;
+  else s = FPD_STAGES_D64;
+  return fp4 ? s * FPD_FP4_STAGES_NUM / FPD_FP4_STAGES_DEN : s;
 }
 
 // Header ring depth: two slots while an item's query rows are small, one
@@ -101,9 +111,10 @@ int header_slots(int D, int cols, int HB) {
 }
 
 // Shared memory of the split kernel with `cols` = q_len * g columns per KV head.
-int smem_bytes_for(int D, int cols, int HB, int B) {
+int smem_bytes_for(int D, int cols, int HB, int B, bool fp4 = false) {
   const int NT = n_tiles(cols);
-  return fpd::smem_layout(D, NT, HB, ring_stages(D, NT, HB), header_slots(D, cols, HB), cols, B)
+  return fpd::smem_layout(D, NT, HB, ring_stages(D, NT, HB, fp4), header_slots(D, cols, HB), cols,
+                          B, fp4)
       .total;
 }
 
@@ -127,7 +138,7 @@ WsLayout ws_layout(int B, int Hq, int Hkv, int D, int max_splits) {
 
 // ---- per-device facts, queried once
 struct OccEntry {
-  int D, NT, HB, mq, smem, occ;
+  int D, NT, HB, mq, fp4, smem, occ;
 };
 struct DeviceInfo {
   bool ready = false;
@@ -139,19 +150,24 @@ struct DeviceInfo {
 std::mutex g_mu;
 DeviceInfo g_dev[kMaxDevices];
 
-template <int HB, bool MQ>
-const void* split_kernel_hb(int D, int NT) {
-  if (D == 128)
-    return NT == 2 ? reinterpret_cast<const void*>(&fpd::fpd_split_kernel<128, 2, HB, MQ>)
-                   : reinterpret_cast<const void*>(&fpd::fpd_split_kernel<128, 1, HB, MQ>);
-  return NT == 2 ? reinterpret_cast<const void*>(&fpd::fpd_split_kernel<64, 2, HB, MQ>)
-                 : reinterpret_cast<const void*>(&fpd::fpd_split_kernel<64, 1, HB, MQ>);
+template <int D, int NT, int HB, bool MQ>
+const void* split_kernel_ptr(bool fp4) {
+  return fp4 ? reinterpret_cast<const void*>(&fpd::fpd_split_kernel_nvfp4<D, NT, HB, MQ>)
+             : reinterpret_cast<const void*>(&fpd::fpd_split_kernel<D, NT, HB, MQ>);
 }
 
-// mq: the kernel for several query tokens per sequence
-const void* split_kernel_for(int D, int NT, int HB, bool mq) {
-  if (mq) return HB == 4 ? split_kernel_hb<4, true>(D, NT) : split_kernel_hb<1, true>(D, NT);
-  return HB == 4 ? split_kernel_hb<4, false>(D, NT) : split_kernel_hb<1, false>(D, NT);
+template <int HB, bool MQ>
+const void* split_kernel_hb(int D, int NT, bool fp4) {
+  if (D == 128)
+    return NT == 2 ? split_kernel_ptr<128, 2, HB, MQ>(fp4) : split_kernel_ptr<128, 1, HB, MQ>(fp4);
+  return NT == 2 ? split_kernel_ptr<64, 2, HB, MQ>(fp4) : split_kernel_ptr<64, 1, HB, MQ>(fp4);
+}
+
+// mq: the kernel for several query tokens per sequence; fp4: over NVFP4 pages
+const void* split_kernel_for(int D, int NT, int HB, bool mq, bool fp4) {
+  if (mq)
+    return HB == 4 ? split_kernel_hb<4, true>(D, NT, fp4) : split_kernel_hb<1, true>(D, NT, fp4);
+  return HB == 4 ? split_kernel_hb<4, false>(D, NT, fp4) : split_kernel_hb<1, false>(D, NT, fp4);
 }
 
 bool current_device(int* dev) {
@@ -191,7 +207,8 @@ bool device_sm_count(int* num_sms) {
 // SM count of the current device and the number of split-kernel CTAs that fit
 // on one SM with `smem` bytes of dynamic shared memory (0 if none).  Also sets
 // the kernel's dynamic shared-memory limit, which its launch needs.
-bool device_occupancy(int D, int NT, int HB, bool mq, int smem, int* num_sms, int* ctas_per_sm) {
+bool device_occupancy(int D, int NT, int HB, bool mq, bool fp4, int smem, int* num_sms,
+                      int* ctas_per_sm) {
   int dev = 0;
   if (!current_device(&dev)) return false;
   std::lock_guard<std::mutex> lk(g_mu);
@@ -201,13 +218,14 @@ bool device_occupancy(int D, int NT, int HB, bool mq, int smem, int* num_sms, in
   *num_sms = di.num_sms;
   for (int i = 0; i < di.n_occ; ++i) {
     const OccEntry& e = di.occ[i];
-    if (e.D == D && e.NT == NT && e.HB == HB && e.mq == (int)mq && e.smem == smem) {
+    if (e.D == D && e.NT == NT && e.HB == HB && e.mq == (int)mq && e.fp4 == (int)fp4 &&
+        e.smem == smem) {
       *ctas_per_sm = e.occ;
       return true;
     }
   }
   int occ = 0;
-  const void* fn = split_kernel_for(D, NT, HB, mq);
+  const void* fn = split_kernel_for(D, NT, HB, mq, fp4);
   cudaFuncAttributes fa;
   if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) {
     cudaGetLastError();
@@ -223,7 +241,8 @@ bool device_occupancy(int D, int NT, int HB, bool mq, int smem, int* num_sms, in
       return false;
     }
   }
-  if (di.n_occ < kOccCacheSize) di.occ[di.n_occ++] = OccEntry{D, NT, HB, (int)mq, smem, occ};
+  if (di.n_occ < kOccCacheSize)
+    di.occ[di.n_occ++] = OccEntry{D, NT, HB, (int)mq, (int)fp4, smem, occ};
   *ctas_per_sm = occ;
   return true;
 }
@@ -289,6 +308,38 @@ bool encode_cache_map(CUtensorMap* map, const void* base, int num_blocks, int bt
   return r == CUDA_SUCCESS;
 }
 
+// TMA views of NVFP4 pages (head-major, no swizzle: the rows are read by
+// plain 8- and 16-byte loads).
+//   data:   (d pair, slot, kv head, page), strides (D/2, bt*D/2, data stride);
+//           box (D/2, 16, 4, 1) with four heads per stage, (D/2, bt, 1, 1) with one.
+//   scales: (the D bytes of 16 tokens' block scales, 16-token group, kv head,
+//           page), strides (D, bt*D/16, scale stride); box (D, 1, 4, 1) or
+//           (D, bt/16, 1, 1).
+// Each box lands in shared memory as rows [head][token][bytes], like the
+// E4M3 tiles.
+bool encode_nvfp4_map(CUtensorMap* map, const void* base, int num_blocks, int bt, int Hkv, int D,
+                      int HB, int64_t page_stride, bool scales) {
+  auto enc = encoder();
+  if (!enc) return false;
+  cuuint64_t dims[4], strides[3];
+  cuuint32_t box[4];
+  if (!scales) {
+    dims[0] = D / 2, dims[1] = bt, dims[2] = Hkv, dims[3] = num_blocks;
+    strides[0] = D / 2, strides[1] = (cuuint64_t)bt * (D / 2);
+    box[0] = D / 2, box[1] = HB == 1 ? bt : fpd::kBoxTokens, box[2] = HB, box[3] = 1u;
+  } else {
+    dims[0] = D, dims[1] = bt / fpd::kBoxTokens, dims[2] = Hkv, dims[3] = num_blocks;
+    strides[0] = D, strides[1] = (cuuint64_t)bt * (D / 16);
+    box[0] = D, box[1] = HB == 1 ? bt / fpd::kBoxTokens : 1u, box[2] = HB, box[3] = 1u;
+  }
+  strides[2] = (cuuint64_t)page_stride;
+  cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // Combine launch as a programmatic dependent of the split kernel: its CTAs may
 // start while the split kernel drains and wait for it on the device.
 template <int D, bool MQ>
@@ -337,11 +388,40 @@ cudaError_t launch_split_hb(int D, int NT, const CUtensorMap& km, const CUtensor
                  : launch_split<64, 1, HB, MQ>(km, vm, p, ctas, smem, st);
 }
 
+// The NVFP4 split kernel, launched like the E4M3 one (programmatic dependent).
+template <int D, int NT, int HB, bool MQ>
+cudaError_t launch_split_nvfp4(const CUtensorMap (&maps)[4], const fpd::DecodeParams& p, int ctas,
+                               int smem, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)ctas);
+  cfg.blockDim = dim3(fpd::kThreads);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, fpd::fpd_split_kernel_nvfp4<D, NT, HB, MQ>, maps[0], maps[1],
+                            maps[2], maps[3], p);
+}
+
+template <int HB, bool MQ>
+cudaError_t launch_split_nvfp4_hb(int D, int NT, const CUtensorMap (&maps)[4],
+                                  const fpd::DecodeParams& p, int ctas, int smem, cudaStream_t st) {
+  if (D == 128)
+    return NT == 2 ? launch_split_nvfp4<128, 2, HB, MQ>(maps, p, ctas, smem, st)
+                   : launch_split_nvfp4<128, 1, HB, MQ>(maps, p, ctas, smem, st);
+  return NT == 2 ? launch_split_nvfp4<64, 2, HB, MQ>(maps, p, ctas, smem, st)
+                 : launch_split_nvfp4<64, 1, HB, MQ>(maps, p, ctas, smem, st);
+}
+
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 // The split plan for a given stage shape (HB KV heads per stage).
 void plan_shape(int B, int q_len, int Hq, int Hkv, int D, int bt, int max_blocks,
-                int window_left, int64_t slots, int chunk_pages_override, int HB, fpd_plan* plan) {
+                int window_left, int64_t slots, int chunk_pages_override, int HB, fpd_plan* plan,
+                bool fp4 = false) {
   const int g = Hq / Hkv;
   const int qp = q_per_item(q_len, g);
   const int q_chunks = (q_len + qp - 1) / qp;
@@ -376,10 +456,10 @@ void plan_shape(int B, int q_len, int Hq, int Hkv, int D, int bt, int max_blocks
   plan->max_splits = max_splits;
   plan->heads_per_stage = HB;
   plan->stage_tokens = fpd::kTileTokens / HB;
-  plan->stages = ring_stages(D, NT, HB);
+  plan->stages = ring_stages(D, NT, HB, fp4);
   plan->header_slots = header_slots(D, cols, HB);
   plan->ctas = (int)(items_max < slots ? items_max : slots);
-  plan->smem_bytes = smem_bytes_for(D, cols, HB, B);
+  plan->smem_bytes = smem_bytes_for(D, cols, HB, B, fp4);
   // partial results for each of the B * q_len query tokens
   plan->workspace_bytes = ws_layout(B * q_len, Hq, Hkv, D, max_splits).total;
   plan->q_per_item = qp;
@@ -392,7 +472,7 @@ void plan_shape(int B, int q_len, int Hq, int Hkv, int D, int bt, int max_blocks
 // stage, whose 4x more numerous items keep the machine busy.
 fpd_status plan_for(int B, int q_len, int Hq, int Hkv, int D, int bt, int max_blocks,
                     int window_left, int num_sms, int ctas_per_sm, int chunk_pages_override,
-                    int force_hb, fpd_plan* plan) {
+                    int force_hb, fpd_plan* plan, bool fp4 = false) {
   if (!plan) return FPD_ERR_INVALID_ARG;
   fpd_status st = validate_shape(B, Hq, Hkv, D, bt, max_blocks, q_len);
   if (st != FPD_OK) return st;
@@ -402,17 +482,18 @@ fpd_status plan_for(int B, int q_len, int Hq, int Hkv, int D, int bt, int max_bl
   const int64_t slots = (int64_t)num_sms * ctas_per_sm;
   int HB = force_hb ? force_hb : heads_per_stage(Hkv);
   plan_shape(B, q_len, Hq, Hkv, D, bt, max_blocks, window_left, slots, chunk_pages_override, HB,
-             plan);
+             plan, fp4);
   if (force_hb == 0 && HB == 4 && chunk_pages_override == 0 &&
       (int64_t)(B > 0 ? B : 1) * (Hkv / 4) * plan->q_chunks * plan->max_splits < slots)
-    plan_shape(B, q_len, Hq, Hkv, D, bt, max_blocks, window_left, slots, 0, 1, plan);
+    plan_shape(B, q_len, Hq, Hkv, D, bt, max_blocks, window_left, slots, 0, 1, plan, fp4);
   return FPD_OK;
 }
 
 // The plan on the current device (its SM count and the split kernel's
 // occupancy for the chosen stage shape).
 fpd_status plan_device(int B, int q_len, int Hq, int Hkv, int D, int bt, int max_blocks,
-                       int window_left, int chunk_pages_override, fpd_plan* plan) {
+                       int window_left, int chunk_pages_override, fpd_plan* plan,
+                       bool fp4 = false) {
   if (!plan) return FPD_ERR_INVALID_ARG;
   fpd_status st = validate_shape(B, Hq, Hkv, D, bt, max_blocks, q_len);
   if (st != FPD_OK) return st;
@@ -420,12 +501,12 @@ fpd_status plan_device(int B, int q_len, int Hq, int Hkv, int D, int bt, int max
   int HB = heads_per_stage(Hkv), force_hb = 0;
   for (;;) {
     int sms = 0, occ = 0;
-    if (!device_occupancy(D, n_tiles(cols), HB, q_len > 1, smem_bytes_for(D, cols, HB, B), &sms,
-                          &occ))
+    if (!device_occupancy(D, n_tiles(cols), HB, q_len > 1, fp4,
+                          smem_bytes_for(D, cols, HB, B, fp4), &sms, &occ))
       return FPD_ERR_CUDA;
     if (occ <= 0) return FPD_ERR_UNSUPPORTED;  // the batch's shared-memory table does not fit
     st = plan_for(B, q_len, Hq, Hkv, D, bt, max_blocks, window_left, sms, occ,
-                  chunk_pages_override, force_hb, plan);
+                  chunk_pages_override, force_hb, plan, fp4);
     // the planner fell back to one head per stage: plan again with that
     // kernel's own occupancy
     if (st != FPD_OK || plan->heads_per_stage == HB) return st;
@@ -549,6 +630,20 @@ static fpd_status attention_impl(const fpd_decode_args& a, void* workspace,
     return FPD_ERR_INVALID_ARG;
   if (a.q_dtype != FPD_Q_BF16 && a.q_dtype != FPD_Q_F16) return FPD_ERR_INVALID_ARG;
   if (a.kv_layout != FPD_KV_NHD && a.kv_layout != FPD_KV_HND) return FPD_ERR_INVALID_ARG;
+  if (a.kv_format != FPD_KV_E4M3 && a.kv_format != FPD_KV_NVFP4) return FPD_ERR_INVALID_ARG;
+  const bool fp4 = a.kv_format == FPD_KV_NVFP4;
+  // NVFP4 pages: head-major, data and scale regions at their own page strides
+  const int64_t fp4_data = (int64_t)Hkv * bt * (D / 2), fp4_sf = (int64_t)Hkv * bt * (D / 16);
+  const int64_t data_stride = a.kv_page_stride ? a.kv_page_stride : fp4_data;
+  const int64_t sf_stride = a.sf_page_stride ? a.sf_page_stride : fp4_sf;
+  if (fp4) {
+    if (a.kv_layout != FPD_KV_HND) return FPD_ERR_UNSUPPORTED;
+    if (!a.k_scales || !a.v_scales || !aligned(a.k_scales, 16) || !aligned(a.v_scales, 16))
+      return FPD_ERR_INVALID_ARG;
+    if (data_stride < fp4_data || sf_stride < fp4_sf || data_stride % 16 != 0 ||
+        sf_stride % 16 != 0)
+      return FPD_ERR_INVALID_ARG;
+  }
   const int64_t row = (int64_t)Hq * D;
   const int64_t q_stride = a.q_token_stride ? a.q_token_stride : row;
   const int64_t o_stride = a.out_token_stride ? a.out_token_stride : row;
@@ -575,15 +670,25 @@ static fpd_status attention_impl(const fpd_decode_args& a, void* workspace,
   const int g = Hq / Hkv;
   fpd_plan plan;
   st = plan_device(B, q_len, Hq, Hkv, D, bt, max_blocks, window_left, a.chunk_pages_override,
-                   &plan);
+                   &plan, fp4);
   if (st != FPD_OK) return st;
   if (!workspace || workspace_bytes < plan.workspace_bytes) return FPD_ERR_WORKSPACE_TOO_SMALL;
 
   const bool hnd = a.kv_layout == FPD_KV_HND;
-  CUtensorMap km, vm;
-  if (!encode_cache_map(&km, a.k_cache, num_blocks, bt, Hkv, D, plan.heads_per_stage, hnd) ||
-      !encode_cache_map(&vm, a.v_cache, num_blocks, bt, Hkv, D, plan.heads_per_stage, hnd))
+  CUtensorMap km, vm, maps4[4];
+  if (fp4) {   // K data, K scales, V data, V scales
+    const int HBp = plan.heads_per_stage;
+    if (!encode_nvfp4_map(&maps4[0], a.k_cache, num_blocks, bt, Hkv, D, HBp, data_stride, false) ||
+        !encode_nvfp4_map(&maps4[1], a.k_scales, num_blocks, bt, Hkv, D, HBp, sf_stride, true) ||
+        !encode_nvfp4_map(&maps4[2], a.v_cache, num_blocks, bt, Hkv, D, HBp, data_stride, false) ||
+        !encode_nvfp4_map(&maps4[3], a.v_scales, num_blocks, bt, Hkv, D, HBp, sf_stride, true))
+      return FPD_ERR_CUDA;
+  } else if (!encode_cache_map(&km, a.k_cache, num_blocks, bt, Hkv, D, plan.heads_per_stage,
+                               hnd) ||
+             !encode_cache_map(&vm, a.v_cache, num_blocks, bt, Hkv, D, plan.heads_per_stage,
+                               hnd)) {
     return FPD_ERR_CUDA;
+  }
 
   const WsLayout wl = ws_layout(B * q_len, Hq, Hkv, D, plan.max_splits);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -629,12 +734,19 @@ static fpd_status attention_impl(const fpd_decode_args& a, void* workspace,
   cudaError_t e;
   const int NT = n_tiles(plan.q_per_item * g);
   const bool mq = q_len > 1;
-  if (plan.heads_per_stage == 4)
-    e = mq ? launch_split_hb<4, true>(D, NT, km, vm, p, plan.ctas, plan.smem_bytes, s)
-           : launch_split_hb<4, false>(D, NT, km, vm, p, plan.ctas, plan.smem_bytes, s);
+  const int ctas = plan.ctas, smem = plan.smem_bytes;
+  if (fp4 && plan.heads_per_stage == 4)
+    e = mq ? launch_split_nvfp4_hb<4, true>(D, NT, maps4, p, ctas, smem, s)
+           : launch_split_nvfp4_hb<4, false>(D, NT, maps4, p, ctas, smem, s);
+  else if (fp4)
+    e = mq ? launch_split_nvfp4_hb<1, true>(D, NT, maps4, p, ctas, smem, s)
+           : launch_split_nvfp4_hb<1, false>(D, NT, maps4, p, ctas, smem, s);
+  else if (plan.heads_per_stage == 4)
+    e = mq ? launch_split_hb<4, true>(D, NT, km, vm, p, ctas, smem, s)
+           : launch_split_hb<4, false>(D, NT, km, vm, p, ctas, smem, s);
   else
-    e = mq ? launch_split_hb<1, true>(D, NT, km, vm, p, plan.ctas, plan.smem_bytes, s)
-           : launch_split_hb<1, false>(D, NT, km, vm, p, plan.ctas, plan.smem_bytes, s);
+    e = mq ? launch_split_hb<1, true>(D, NT, km, vm, p, ctas, smem, s)
+           : launch_split_hb<1, false>(D, NT, km, vm, p, ctas, smem, s);
   if (e != cudaSuccess) return FPD_ERR_CUDA;
   if (ev1 && cudaEventRecord(static_cast<cudaEvent_t>(ev1), s) != cudaSuccess) return FPD_ERR_CUDA;
   if (plan.max_splits > 1) {
@@ -705,6 +817,31 @@ fpd_status fp8_paged_decode_attention_args(const fpd_decode_args* args, void* wo
                                            size_t workspace_bytes, void* stream) {
   if (!args) return FPD_ERR_INVALID_ARG;
   return attention_impl(*args, workspace, workspace_bytes, stream, nullptr, nullptr, nullptr);
+}
+
+fpd_status fp8_paged_decode_attention_args_profiled(const fpd_decode_args* args, void* workspace,
+                                                    size_t workspace_bytes, void* stream,
+                                                    void* event_before_split,
+                                                    void* event_after_split,
+                                                    void* event_after_combine) {
+  if (!args) return FPD_ERR_INVALID_ARG;
+  return attention_impl(*args, workspace, workspace_bytes, stream, event_before_split,
+                        event_after_split, event_after_combine);
+}
+
+fpd_status fp8_paged_decode_plan_args(const fpd_decode_args* args, fpd_plan* plan) {
+  if (!args || !plan) return FPD_ERR_INVALID_ARG;
+  if (args->kv_format != FPD_KV_E4M3 && args->kv_format != FPD_KV_NVFP4)
+    return FPD_ERR_INVALID_ARG;
+  return plan_device(args->B, args->q_len, args->Hq, args->Hkv, args->D, args->block_tokens,
+                     args->max_blocks, args->window_left, args->chunk_pages_override, plan,
+                     args->kv_format == FPD_KV_NVFP4);
+}
+
+size_t fp8_paged_decode_workspace_bytes_args(const fpd_decode_args* args) {
+  fpd_plan plan;
+  if (fp8_paged_decode_plan_args(args, &plan) != FPD_OK) return 0;
+  return plan.workspace_bytes;
 }
 
 fpd_status fp8_paged_decode_attention_profiled(
@@ -845,6 +982,69 @@ fpd_status fp8_paged_decode_cache_write_layout(const void* key, const void* valu
   const int grid = (int)(want < cap ? want : cap);
   fpd::fpd_cache_write_kernel<<<grid, fpd::kWriteThreads, 0, static_cast<cudaStream_t>(stream)>>>(
       p);
+  return cudaGetLastError() == cudaSuccess ? FPD_OK : FPD_ERR_CUDA;
+}
+
+fpd_status fp8_paged_decode_cache_write_nvfp4(const void* key, const void* value,
+                                              const int64_t* slot_mapping, int num_tokens,
+                                              int Hkv, int D, int64_t key_stride,
+                                              int64_t value_stride, float k_scale, float v_scale,
+                                              void* k_data, void* k_sf, void* v_data, void* v_sf,
+                                              int64_t data_page_stride, int64_t sf_page_stride,
+                                              int num_blocks, int block_tokens, uint32_t* status,
+                                              void* stream) {
+  if (num_tokens < 0 || Hkv <= 0 || D <= 0 || D % 16 != 0 || num_blocks <= 0 ||
+      block_tokens <= 0)
+    return FPD_ERR_INVALID_ARG;
+  if ((int64_t)num_blocks * block_tokens >= INT32_MAX) return FPD_ERR_UNSUPPORTED;
+  if (!(k_scale > 0.f) || !(v_scale > 0.f) || !std::isfinite(k_scale) || !std::isfinite(v_scale))
+    return FPD_ERR_INVALID_ARG;
+  if (num_tokens == 0) return FPD_OK;
+  if (!key || !value || !slot_mapping || !k_data || !k_sf || !v_data || !v_sf)
+    return FPD_ERR_INVALID_ARG;
+  const int64_t row = (int64_t)Hkv * D;
+  const int64_t data_b = (int64_t)Hkv * block_tokens * (D / 2);
+  const int64_t sf_b = (int64_t)Hkv * block_tokens * (D / 16);
+  const int64_t ds = data_page_stride ? data_page_stride : data_b;
+  const int64_t ss = sf_page_stride ? sf_page_stride : sf_b;
+  if (key_stride < row || value_stride < row || key_stride % 8 != 0 || value_stride % 8 != 0 ||
+      ds < data_b || ss < sf_b || ds % 16 != 0 || ss % 16 != 0)
+    return FPD_ERR_INVALID_ARG;
+  if (!aligned(key, 16) || !aligned(value, 16) || !aligned(k_data, 16) || !aligned(k_sf, 16) ||
+      !aligned(v_data, 16) || !aligned(v_sf, 16) || !aligned(slot_mapping, 8) ||
+      (status && !aligned(status, 4)))
+    return FPD_ERR_INVALID_ARG;
+  if (row / 16 > INT32_MAX) return FPD_ERR_UNSUPPORTED;
+  fpd::CacheWriteFp4Params p;
+  p.key = static_cast<const __nv_bfloat16*>(key);
+  p.value = static_cast<const __nv_bfloat16*>(value);
+  p.slot_mapping = slot_mapping;
+  p.k_data = static_cast<uint8_t*>(k_data);
+  p.k_sf = static_cast<uint8_t*>(k_sf);
+  p.v_data = static_cast<uint8_t*>(v_data);
+  p.v_sf = static_cast<uint8_t*>(v_sf);
+  p.status = status;
+  p.key_stride = key_stride;
+  p.value_stride = value_stride;
+  p.data_page_stride = ds;
+  p.sf_page_stride = ss;
+  p.n_slots = (int64_t)num_blocks * block_tokens;
+  p.num_tokens = num_tokens;
+  p.D = D;
+  p.bt = block_tokens;
+  p.blocks = (int)(row / 16);
+  p.k_gs = 1.0f / k_scale;   // the per-tensor "global" scale, fp32
+  p.v_gs = 1.0f / v_scale;
+  p.k_rgs = 1.0f / p.k_gs;
+  p.v_rgs = 1.0f / p.v_gs;
+  int sms = 0;
+  if (!device_sm_count(&sms)) return FPD_ERR_CUDA;
+  const int64_t units = (int64_t)num_tokens * 2 * p.blocks;
+  const int64_t want = (units + fpd::kWriteThreads - 1) / fpd::kWriteThreads;
+  const int64_t cap = (int64_t)sms * 8;
+  const int grid = (int)(want < cap ? want : cap);
+  fpd::fpd_cache_write_nvfp4_kernel<<<grid, fpd::kWriteThreads, 0,
+                                      static_cast<cudaStream_t>(stream)>>>(p);
   return cudaGetLastError() == cudaSuccess ? FPD_OK : FPD_ERR_CUDA;
 }
 

@@ -100,4 +100,104 @@ __global__ void __launch_bounds__(kWriteThreads) fpd_cache_write_kernel(const Ca
   }
 }
 
+// ------------------------------------------------------------------ NVFP4 --
+//
+// NVFP4 cache write: the block recipe of the gist's NVFP4 cache writer (writer
+// kernel and quantisation helper) with exact fp32 reciprocals: per 16
+// consecutive elements of a token's head row
+//   sf   = e4m3_rne_sat((amax * (1/6)) * gs)        gs = 1 / scale
+//   osc  = sf == 0 ? 0 : 1 / (e4m3(sf) * (1 / gs))
+//   code = e2m1_rne_sat(x * osc)                    (element 2i in the low nibble)
+// into head-major pages: data [page][kv head][slot][D/2], scales
+// [page][kv head][slot][D/16], each region at its own page stride.  One thread
+// per 16-element block: two 16-byte loads, one 8-byte and one 1-byte store.
+
+struct CacheWriteFp4Params {
+  const __nv_bfloat16* key;
+  const __nv_bfloat16* value;
+  const int64_t* slot_mapping;
+  uint8_t* k_data;
+  uint8_t* k_sf;
+  uint8_t* v_data;
+  uint8_t* v_sf;
+  uint32_t* status;
+  int64_t key_stride, value_stride;         // elements between tokens
+  int64_t data_page_stride, sf_page_stride;  // bytes between pages
+  int64_t n_slots;
+  int num_tokens, D, bt;
+  int blocks;                               // Hkv * D / 16 per token and side
+  float k_gs, v_gs;                         // 1 / k_scale, 1 / v_scale (fp32)
+  float k_rgs, v_rgs;                       // 1 / gs (fp32)
+};
+
+// Two floats -> one byte of two E2M1 codes (lo in the low nibble), round to
+// nearest even, saturating at +-6.
+__device__ __forceinline__ uint32_t f32x2_to_e2m1x2(float lo, float hi) {
+  uint16_t r;
+  asm("{\n\t.reg .b8 b;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b, %1, %2;\n\t"
+      "cvt.u16.u8 %0, b;\n\t}"
+      : "=h"(r)
+      : "f"(hi), "f"(lo));
+  return r;
+}
+
+__global__ void __launch_bounds__(kWriteThreads) fpd_cache_write_nvfp4_kernel(
+    const CacheWriteFp4Params p) {
+  constexpr float kInv6 = 1.0f / 6.0f;
+  const int64_t per_token = 2LL * p.blocks;
+  const int64_t units = (int64_t)p.num_tokens * per_token;
+  const int hb = p.D / 16;   // blocks per head row
+  for (int64_t u = (int64_t)blockIdx.x * kWriteThreads + threadIdx.x; u < units;
+       u += (int64_t)gridDim.x * kWriteThreads) {
+    const int t = (int)(u / per_token);
+    const int r = (int)(u - (int64_t)t * per_token);
+    const bool is_v = r >= p.blocks;
+    const int blk = is_v ? r - p.blocks : r;
+    const int64_t slot = __ldg(p.slot_mapping + t);
+    if (slot < 0) continue;   // padded token
+    if (slot >= p.n_slots) {
+      if (p.status && blk == 0 && !is_v) atomicOr(p.status, kErrSlot);
+      continue;
+    }
+    const __nv_bfloat16* src =
+        (is_v ? p.value + (int64_t)t * p.value_stride : p.key + (int64_t)t * p.key_stride) +
+        blk * 16;
+    const uint4 a = __ldcs(reinterpret_cast<const uint4*>(src));
+    const uint4 b = __ldcs(reinterpret_cast<const uint4*>(src) + 1);
+    float x[16];
+    const __nv_bfloat162* ha = reinterpret_cast<const __nv_bfloat162*>(&a);
+    const __nv_bfloat162* hb2 = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 fa = __bfloat1622float2(ha[j]);
+      const float2 fb = __bfloat1622float2(hb2[j]);
+      x[2 * j] = fa.x, x[2 * j + 1] = fa.y;
+      x[8 + 2 * j] = fb.x, x[8 + 2 * j + 1] = fb.y;
+    }
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
+    const float gs = is_v ? p.v_gs : p.k_gs;
+    const float rgs = is_v ? p.v_rgs : p.k_rgs;
+    const float sf_f = __fmul_rn(__fmul_rn(amax, kInv6), gs);
+    const uint32_t sfc = f32x4_to_e4m3x4(sf_f, 0.f, 0.f, 0.f) & 0xFFu;
+    const float sf_v = __half2float(__ushort_as_half(
+        (unsigned short)(e4m3x2_to_f16x2((uint16_t)sfc) & 0xFFFFu)));
+    const float osc = sf_v == 0.f ? 0.f : __frcp_rn(__fmul_rn(sf_v, rgs));
+    uint32_t w[2] = {0u, 0u};
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      w[i / 4] |= f32x2_to_e2m1x2(__fmul_rn(x[2 * i], osc), __fmul_rn(x[2 * i + 1], osc))
+                  << (8 * (i % 4));
+    const int page = (int)(slot / p.bt), off = (int)(slot - (int64_t)page * p.bt);
+    const int h = blk / hb, j = blk - h * hb;
+    const int64_t row = (int64_t)h * p.bt + off;
+    uint8_t* data = (is_v ? p.v_data : p.k_data) + (int64_t)page * p.data_page_stride +
+                    row * (p.D / 2) + j * 8;
+    *reinterpret_cast<uint2*>(data) = make_uint2(w[0], w[1]);
+    (is_v ? p.v_sf : p.k_sf)[(int64_t)page * p.sf_page_stride + row * hb + j] = (uint8_t)sfc;
+  }
+}
+
 }  // namespace fpd

@@ -127,12 +127,37 @@ struct SmemLayout {
 
 __host__ __device__ constexpr int align_to(int x, int a) { return (x + a - 1) / a * a; }
 
+// NVFP4 stage: four regions [K data | K scales | V data | V scales] holding
+// kTileTokens rows each; a row is D / 2 bytes of E2M1 pairs and D / 16 block
+// scales.  Every TMA destination in shared memory must sit on a 128-byte
+// boundary, so the scale region is 512 bytes even where its rows need only
+// 256, and with one head per stage each page's scales start a slot of
+// fp4_sf_pitch bytes.
+__host__ __device__ constexpr int fp4_data_bytes(int D) { return kTileTokens * D / 2; }
+__host__ __device__ constexpr int fp4_sf_bytes(int D) {
+  return kTileTokens * D / 16 > 512 ? kTileTokens * D / 16 : 512;
+}
+__host__ __device__ constexpr int fp4_sf_pitch(int bt, int D) {
+  return bt * D / 16 > 128 ? bt * D / 16 : 128;
+}
+
+// Bytes the TMA boxes of one NVFP4 stage deliver (without the padding).
+__host__ __device__ constexpr int fp4_stage_payload(int D) {
+  return 2 * kTileTokens * (D / 2 + D / 16);
+}
+
+// Bytes of one ring stage: kTileTokens rows of K and of V.  E4M3 rows are D
+// bytes; NVFP4 stages are laid out as above.
+__host__ __device__ constexpr int stage_bytes(int D, bool fp4) {
+  return fp4 ? 2 * (fp4_data_bytes(D) + fp4_sf_bytes(D)) : 2 * kTileTokens * D;
+}
+
 __host__ __device__ inline SmemLayout smem_layout(int D, int NT, int HB, int stages, int hdr_slots,
-                                                  int g, int B) {
+                                                  int g, int B, bool fp4 = false) {
   SmemLayout L{};
   const int H = NT * 8;
   L.ring = 0;
-  L.merge = stages * 2 * kTileTokens * D;
+  L.merge = stages * stage_bytes(D, fp4);
   const int merge_bytes =
       HB == 1 ? kConsumerWarps * H * (D + 4) * 4 + kConsumerWarps * H * 2 * 4 : 0;
   L.hdr = align_to(L.merge + merge_bytes, 128);
@@ -218,7 +243,10 @@ struct TileMask {
 
 // MQ: several query tokens per sequence (columns are (position, head) pairs
 // with per-column key ranges); otherwise one query and columns are heads.
-template <int D, int NT, bool MQ>
+// FP4: the stage holds NVFP4 rows (E2M1 pairs and E4M3 block scales, no
+// swizzle; the warp's 16 rows start at the pointers passed to tile());
+// otherwise E4M3 rows in the swizzled TMA layout.
+template <int D, int NT, bool MQ, bool FP4 = false>
 struct Consumer {
   static constexpr int KS = D / 16;   // k-steps of the QK MMA
   static constexpr int MT = D / 16;   // m-tiles of the PV MMA
@@ -328,12 +356,91 @@ struct Consumer {
 
   // One 16-row slice of a stage.  FULL: every row is inside every column's
   // range; otherwise rows are masked per column (mk).
+  // NVFP4 K fragments of rows n and n + 8 (this thread's elements
+  // [t*D/4, (t+1)*D/4) of each, D/8 bytes of E2M1 pairs) as f16x2 words in the
+  // E4M3 path's order: word 2ks = elements 4ks, 4ks+1; word 2ks+1 = 4ks+2, 4ks+3.
+  // Each value is the E2M1 code times its block's E4M3 scale, exact in f16.
+  __device__ __forceinline__ void fp4_k_frags(const uint8_t* Kd, const uint8_t* Ks, int lane,
+                                              uint32_t (&kh)[2][D / 8]) {
+    const int n = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int row = n + 8 * r;
+      uint32_t w[D / 32];
+      if constexpr (D == 128) {
+        const uint4 v = *reinterpret_cast<const uint4*>(Kd + row * (D / 2) + t * 16);
+        w[0] = v.x, w[1] = v.y, w[2] = v.z, w[3] = v.w;
+      } else {
+        const uint2 v = *reinterpret_cast<const uint2*>(Kd + row * (D / 2) + t * 8);
+        w[0] = v.x, w[1] = v.y;
+      }
+      // block scales of this thread's elements: D/64 blocks of 16
+      uint32_t sc[D / 64];
+      if constexpr (D == 128) {
+        const uint32_t s2 = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(Ks + row * (D / 16) + 2 * t));
+        sc[0] = prmt(s2, s2, 0x1010u);
+        sc[1] = prmt(s2, s2, 0x3232u);
+      } else {
+        const uint32_t s2 = e4m3x2_to_f16x2((uint16_t)Ks[row * (D / 16) + t]);
+        sc[0] = prmt(s2, s2, 0x1010u);
+      }
+#pragma unroll
+      for (int i = 0; i < D / 32; ++i) {
+        uint32_t h[4];
+        e2m1x8_to_f16x2x4(w[i], h);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) kh[r][4 * i + j] = hmul2(h[j], sc[(4 * i + j) / 8]);
+      }
+    }
+  }
+
+  // NVFP4 V rows 2t, 2t+1, 2t+8, 2t+9, this thread's elements [n*D/8, (n+1)*D/8)
+  // (D/16 bytes each, one block scale), as f16x2 words (word i = elements 2i,
+  // 2i+1), rows outside [tok_lo, tok_hi) zeroed when not FULL.
+  template <bool FULL>
+  __device__ __forceinline__ void fp4_v_rows(const uint8_t* Vd, const uint8_t* Vs, int tok0,
+                                             const TileMask& mk, int lane,
+                                             uint32_t (&vh)[4][D / 16]) {
+    const int n = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int row = 2 * t + (r & 1) + 8 * (r >> 1);
+      uint32_t w[D / 64];
+      if constexpr (D == 128) {
+        const uint2 v = *reinterpret_cast<const uint2*>(Vd + row * (D / 2) + n * 8);
+        w[0] = v.x, w[1] = v.y;
+      } else {
+        w[0] = *reinterpret_cast<const uint32_t*>(Vd + row * (D / 2) + n * 4);
+      }
+      const uint8_t sfc = Vs[row * (D / 16) + (D == 128 ? n : n / 2)];
+      const uint32_t s2 = e4m3x2_to_f16x2((uint16_t)sfc);
+      const uint32_t sc = prmt(s2, s2, 0x1010u);
+      uint32_t mask = 0xffffffffu;
+      if (!FULL) {
+        const int tk = tok0 + row;
+        mask = (tk >= mk.tok_lo && tk < mk.tok_hi) ? 0xffffffffu : 0u;
+      }
+#pragma unroll
+      for (int i = 0; i < D / 64; ++i) {
+        uint32_t h[4];
+        e2m1x8_to_f16x2x4(w[i], h);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) vh[r][4 * i + j] = hmul2(h[j], sc) & mask;
+      }
+    }
+  }
+
   template <bool FULL>
   __device__ __forceinline__ void tile(const uint8_t* Kt, const uint8_t* Vt, int row0, int tok0,
-                                       const TileMask& mk, int lane) {
+                                       const TileMask& mk, int lane,
+                                       const uint8_t* Ks = nullptr, const uint8_t* Vs = nullptr) {
     const int n = lane >> 2, t = lane & 3;
     // ---- K fragments: rows row0 + n and row0 + n + 8, bytes [t*D/4, (t+1)*D/4)
-    uint32_t kw[2][D / 16];
+    uint32_t kw[2][FP4 ? 1 : D / 16];
+    uint32_t kh[2][FP4 ? D / 8 : 1];
+    if constexpr (FP4) {
+      fp4_k_frags(Kt, Ks, lane, kh);
+    } else {
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
 #pragma unroll
@@ -344,6 +451,7 @@ struct Consumer {
         kw[r][4 * c + 2] = v.z;
         kw[r][4 * c + 3] = v.w;
       }
+    }
     }
     // ---- S^T = K Q^T, two accumulation chains per n-tile
     float s[NT][2][4];
@@ -356,8 +464,13 @@ struct Consumer {
 #pragma unroll
     for (int ks = 0; ks < KS; ++ks) {
       uint32_t a0, a1, a2, a3;
-      e4m3x4_to_f16x2x2(kw[0][ks], a0, a2);
-      e4m3x4_to_f16x2x2(kw[1][ks], a1, a3);
+      if constexpr (FP4) {
+        a0 = kh[0][2 * ks], a2 = kh[0][2 * ks + 1];
+        a1 = kh[1][2 * ks], a3 = kh[1][2 * ks + 1];
+      } else {
+        e4m3x4_to_f16x2x2(kw[0][ks], a0, a2);
+        e4m3x4_to_f16x2x2(kw[1][ks], a1, a3);
+      }
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
         mma_16816(s[nt][ks & 1], a0, a1, a2, a3, qf[nt][ks][0], qf[nt][ks][1]);
@@ -446,6 +559,22 @@ struct Consumer {
       pb1[nt] = movmatrix_trans(pack_f16x2(p2, p3));   // tokens 2t+8..2t+9, head n
     }
 
+    if constexpr (FP4) {
+      // ---- O^T += V^T P^T from NVFP4 rows: m-tile i takes element 2i (M row n)
+      // and 2i+1 (M row n + 8) of this thread's chunk, tokens paired by prmt
+      uint32_t vh[4][D / 16];
+      fp4_v_rows<FULL>(Vt, Vs, tok0, mk, lane, vh);
+#pragma unroll
+      for (int i = 0; i < MT; ++i) {
+        const uint32_t a0 = prmt(vh[0][i], vh[1][i], 0x5410u);   // (A, B) element 2i
+        const uint32_t a1 = prmt(vh[0][i], vh[1][i], 0x7632u);   // (A, B) element 2i+1
+        const uint32_t a2 = prmt(vh[2][i], vh[3][i], 0x5410u);
+        const uint32_t a3 = prmt(vh[2][i], vh[3][i], 0x7632u);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) mma_16816(o[i][nt], a0, a1, a2, a3, pb0[nt], pb1[nt]);
+      }
+      return;
+    } else {
     // ---- V fragments: token rows 2t, 2t+1, 2t+8, 2t+9; head-dim chunk n
     constexpr int VB = D / 8;  // bytes of one row this thread needs
     uint32_t va[VB / 4], vb[VB / 4], vc[VB / 4], vd[VB / 4];
@@ -502,6 +631,7 @@ struct Consumer {
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
         mma_16816(o[2 * w + 1][nt], a0, a1, a2, a3, pb0[nt], pb1[nt]);
+    }
     }
   }
   // HB = 4: this warp alone covered KV head `kvh` of the item, so its query
@@ -580,14 +710,20 @@ struct Consumer {
 
 // ---------------------------------------------------------------- producer --
 
-template <int D, int HB, bool MQ>
+// FP4: NVFP4 pages, four tensors per stage (kmap / vmap the E2M1 data, ksmap /
+// vsmap the block scales); otherwise E4M3 pages (kmap / vmap).
+template <int D, int HB, bool MQ, bool FP4>
 __device__ __forceinline__ void producer_loop(const CUtensorMap* kmap, const CUtensorMap* vmap,
+                                              const CUtensorMap* ksmap, const CUtensorMap* vsmap,
                                               const DecodeParams& p, uint8_t* smem,
                                               const SmemLayout& L, const int* prefix,
                                               int total_items, int hslot_bytes,
                                               uint64_t* full_bar, uint64_t* empty_bar,
                                               uint64_t* hdr_full, uint64_t* hdr_empty, int lane) {
   constexpr int kTileBytes = kTileTokens * D;
+  constexpr int kStage = stage_bytes(D, FP4);
+  constexpr int kDataBytes = fp4_data_bytes(D);   // NVFP4 regions of a stage
+  constexpr int kSfBytes = fp4_sf_bytes(D);
   constexpr int kStageTokens = kTileTokens / HB;   // tokens of one KV head per stage
   const int stages = p.stages;
   const int n_hslots = p.hdr_slots;
@@ -600,6 +736,10 @@ __device__ __forceinline__ void producer_loop(const CUtensorMap* kmap, const CUt
   if (lane == 0) {
     tma_prefetch_desc(kmap);
     tma_prefetch_desc(vmap);
+    if constexpr (FP4) {
+      tma_prefetch_desc(ksmap);
+      tma_prefetch_desc(vsmap);
+    }
   }
   int hs = 0;
   int hslot = 0;
@@ -701,8 +841,67 @@ __device__ __forceinline__ void producer_loop(const CUtensorMap* kmap, const CUt
           return;
         }
       }
-      uint8_t* stage = smem + L.ring + slot * 2 * kTileBytes;
-      if constexpr (HB == 1) {
+      uint8_t* stage = smem + L.ring + slot * kStage;
+      if constexpr (FP4 && HB == 1) {
+        // NVFP4, one head: per page four boxes (K data, K scales, V data, V
+        // scales), lane 4q + r for page q of the stage
+        const int pg0 = pb + s * pps;
+        const int np = min(pps, pe - pg0);
+        const int rel = pg0 - pb;
+        if ((rel & ~31) != batch_base) {
+          batch_base = rel & ~31;
+          const int idx = pb + batch_base + lane;
+          my_entry = (idx < pe) ? __ldg(tbl + idx) : 0;
+        }
+        const int e = __shfl_sync(0xffffffffu, my_entry, (rel + (lane >> 2)) & 31);
+        const bool mine = lane < 4 * np;
+        const bool ok = (e >= 0 && e < p.num_blocks);
+        if (mine && !ok && (lane & 3) == 0) atomicOr(p.status, kErrBlockTable);
+        if (lane == 0)
+          mbar_arrive_expect_tx(&full_bar[slot],
+                                (uint32_t)(np * p.bt * (D / 2 + D / 16) * 2));
+        __syncwarp();
+        if (mine) {
+          // an invalid page is read from past the end of the pool: TMA zero-fills it
+          const int page = ok ? e : p.num_blocks;
+          const int q = lane >> 2, r = lane & 3;
+          if (r == 0 || r == 2)   // data: (d pair, slot, kv head, page)
+            tma_load_4d(stage + (r == 0 ? 0 : kDataBytes + kSfBytes) + q * p.bt * (D / 2),
+                        r == 0 ? kmap : vmap, 0, 0, kvh0, page, &full_bar[slot], policy);
+          else                    // scales: (16-token group scales, group, kv head, page)
+            tma_load_4d(stage + (r == 1 ? kDataBytes : 2 * kDataBytes + kSfBytes) +
+                            q * fp4_sf_pitch(p.bt, D),
+                        r == 1 ? ksmap : vsmap, 0, 0, kvh0, page, &full_bar[slot], policy);
+        }
+      } else if constexpr (FP4) {
+        // NVFP4, 16 tokens of 4 heads: lanes 0..3 load K data, K scales, V
+        // data, V scales of the block
+        const int tok = t0 + s * kBoxTokens;
+        const int rel = tok / p.bt - pb;
+        if ((rel & ~31) != batch_base) {
+          batch_base = rel & ~31;
+          const int idx = pb + batch_base + lane;
+          my_entry = (idx < pe) ? __ldg(tbl + idx) : 0;
+        }
+        const int e = __shfl_sync(0xffffffffu, my_entry, rel & 31);
+        const bool ok = (e >= 0 && e < p.num_blocks);
+        if (lane == 0) {
+          if (!ok) atomicOr(p.status, kErrBlockTable);
+          mbar_arrive_expect_tx(&full_bar[slot], (uint32_t)fp4_stage_payload(D));
+        }
+        __syncwarp();
+        if (lane < 4) {
+          const int page = ok ? e : p.num_blocks;
+          const int in_page = tok - (rel + pb) * p.bt;   // first slot of the block in its page
+          if (lane == 0 || lane == 2)
+            tma_load_4d(stage + (lane == 0 ? 0 : kDataBytes + kSfBytes), lane == 0 ? kmap : vmap,
+                        0, in_page, kvh0, page, &full_bar[slot], policy);
+          else
+            tma_load_4d(stage + (lane == 1 ? kDataBytes : 2 * kDataBytes + kSfBytes),
+                        lane == 1 ? ksmap : vsmap, 0, in_page / kBoxTokens, kvh0, page,
+                        &full_bar[slot], policy);
+        }
+      } else if constexpr (HB == 1) {
         const int pg0 = pb + s * pps;
         const int np = min(pps, pe - pg0);
         const int rel = pg0 - pb;
@@ -778,15 +977,20 @@ struct MinBlocks {
   static constexpr int value = (D == 128) ? (NT == 1 ? FPD_MINB_D128_NT1 : 2) : (NT == 1 ? 4 : 3);
 };
 
-template <int D, int NT, int HB, bool MQ>
-__global__ void __launch_bounds__(kThreads, MinBlocks<D, NT>::value)
-fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
-                 const DecodeParams p) {
+// The split kernel's body.  FP4: NVFP4 pages (kmap / vmap the E2M1 data,
+// ksmap / vsmap the block scales); otherwise E4M3 pages (kmap / vmap).
+template <int D, int NT, int HB, bool MQ, bool FP4>
+__device__ __forceinline__ void split_body(const CUtensorMap* kmap, const CUtensorMap* vmap,
+                                           const CUtensorMap* ksmap, const CUtensorMap* vsmap,
+                                           const DecodeParams& p) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ int warp_tot[kThreads / 32];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   constexpr int kTileBytes = kTileTokens * D;
+  constexpr int kStage = stage_bytes(D, FP4);
+  constexpr int kDataBytes = fp4_data_bytes(D);   // NVFP4 regions of a stage
+  constexpr int kSfBytes = fp4_sf_bytes(D);
   constexpr int kStageTokens = kTileTokens / HB;
   constexpr int H = NT * 8;
   const int stages = p.stages;
@@ -794,7 +998,7 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
   // a header slot holds q_len * g query rows per KV head
   const int QL = MQ ? p.q_len : 1;   // query tokens per sequence
   const int QP = MQ ? p.q_per_item : 1;   // query positions per item
-  const SmemLayout L = smem_layout(D, NT, HB, stages, n_hslots, QP * p.g, p.B);
+  const SmemLayout L = smem_layout(D, NT, HB, stages, n_hslots, QP * p.g, p.B, FP4);
   const int hslot_bytes = hdr_slot_bytes(D, HB, QP * p.g);
   int* prefix = reinterpret_cast<int*>(smem + L.prefix);
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + L.bars);
@@ -849,8 +1053,8 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
   pdl_launch_dependents();   // the combine kernel may be scheduled from now on
 
   if (warp == kConsumerWarps) {
-    producer_loop<D, HB, MQ>(&kmap, &vmap, p, smem, L, prefix, total_items, hslot_bytes, full_bar,
-                         empty_bar, hdr_full, hdr_empty, lane);
+    producer_loop<D, HB, MQ, FP4>(kmap, vmap, ksmap, vsmap, p, smem, L, prefix, total_items,
+                                  hslot_bytes, full_bar, empty_bar, hdr_full, hdr_empty, lane);
     return;
   }
 
@@ -859,13 +1063,16 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
   // has resolved)
   const float qk_scale = p.k_scale_dev ? p.sm_scale_log2 * *p.k_scale_dev : p.qk_scale_log2;
   const float v_scale = p.v_scale_dev ? *p.v_scale_dev : p.v_scale;
-  Consumer<D, NT, MQ> cw;
+  Consumer<D, NT, MQ, FP4> cw;
   const int n = lane >> 2, t = lane & 3;
   // HB = 4: this warp's KV head occupies its own 16 rows of each stage.
   // HB = 1: this warp takes rows [16 * warp, 16 * warp + 16) of the stage.
   const int row0 = HB == 1 ? warp * kRowsPerWarp : 0;
   const int tile_off = HB == 1 ? 0 : warp * kRowsPerWarp * D;
   const int tok_off = HB == 1 ? row0 : 0;
+  const int sf_off = HB == 1 ? (warp * kRowsPerWarp / p.bt) * fp4_sf_pitch(p.bt, D) +
+                                   (warp * kRowsPerWarp % p.bt) * (D / 16)
+                             : warp * kRowsPerWarp * (D / 16);
   int hslot = 0;
   uint32_t hphase = 0;
   int slot = 0;             // ring position
@@ -904,14 +1111,23 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
         alive = false;
         break;
       }
-      const uint8_t* Kt = smem + L.ring + slot * 2 * kTileBytes + tile_off;
-      const uint8_t* Vt = Kt + kTileBytes;
+      const uint8_t* st = smem + L.ring + slot * kStage;
+      // E4M3: the swizzled K and V tiles; NVFP4: the warp's 16 rows of the
+      // four regions (rows 16 * warp onward, for either stage shape)
+      const uint8_t* Kt = FP4 ? st + warp * kRowsPerWarp * (D / 2) : st + tile_off;
+      const uint8_t* Vt =
+          FP4 ? st + kDataBytes + kSfBytes + warp * kRowsPerWarp * (D / 2) : Kt + kTileBytes;
+      // (the scale rows of this warp: head `warp` with four heads per stage;
+      // with one head, rows 16 * warp of the stage, in page slot
+      // 16 * warp / bt at its row 16 * warp % bt)
+      const uint8_t* Ks = FP4 ? st + kDataBytes + sf_off : nullptr;
+      const uint8_t* Vs = FP4 ? st + 2 * kDataBytes + kSfBytes + sf_off : nullptr;
       const int tok0 = hd.t0 + s * kStageTokens + tok_off;   // token of this warp's first row
       if (tok0 + kRowsPerWarp > hd.tok_lo && tok0 < hd.tok_hi) {
         if (tok0 >= full_lo && tok0 + kRowsPerWarp <= full_hi)
-          cw.template tile<true>(Kt, Vt, row0, tok0, mk, lane);
+          cw.template tile<true>(Kt, Vt, row0, tok0, mk, lane, Ks, Vs);
         else
-          cw.template tile<false>(Kt, Vt, row0, tok0, mk, lane);
+          cw.template tile<false>(Kt, Vt, row0, tok0, mk, lane, Ks, Vs);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty_bar[slot]);
@@ -947,7 +1163,7 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
         // O^T column h: rows d = n*(D/8) + 2i + hh  (hh = 0 -> c0/c1, 1 -> c2/c3)
         float* dst = Osm + ((size_t)warp * H + h) * OS + n * (D / 8);
 #pragma unroll
-        for (int i = 0; i < Consumer<D, NT, MQ>::MT; ++i) {
+        for (int i = 0; i < Consumer<D, NT, MQ, FP4>::MT; ++i) {
           dst[2 * i + 0] = cw.o[i][nt][j];
           dst[2 * i + 1] = cw.o[i][nt][j + 2];
         }
@@ -1048,6 +1264,24 @@ fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
       atomicExch(&p.sched[1], 0u);
     }
   }
+}
+
+template <int D, int NT, int HB, bool MQ>
+__global__ void __launch_bounds__(kThreads, MinBlocks<D, NT>::value)
+fpd_split_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                 const DecodeParams p) {
+  split_body<D, NT, HB, MQ, false>(&kmap, &vmap, nullptr, nullptr, p);
+}
+
+// The split kernel over NVFP4 pages: TMA views of the K and V data (E2M1
+// pairs) and of their block scales.
+template <int D, int NT, int HB, bool MQ>
+__global__ void __launch_bounds__(kThreads, MinBlocks<D, NT>::value)
+fpd_split_kernel_nvfp4(const __grid_constant__ CUtensorMap kdata,
+                       const __grid_constant__ CUtensorMap ksf,
+                       const __grid_constant__ CUtensorMap vdata,
+                       const __grid_constant__ CUtensorMap vsf, const DecodeParams p) {
+  split_body<D, NT, HB, MQ, true>(&kdata, &vdata, &ksf, &vsf, p);
 }
 
 // ----------------------------------------------------------------- combine --

@@ -151,6 +151,34 @@ __device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t x, uint32_t& lo, uint
       : "r"(x));
 }
 
+// Two E4M3 bytes -> f16x2 (the lower byte into the lower half); exact.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t x) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(x));
+  return r;
+}
+
+// Eight E2M1 codes (4 bytes, the lower nibble of each byte first) -> four
+// f16x2: h[j] = the two codes of byte j (lower nibble into the lower half).
+// Every E2M1 value is exact in f16.
+__device__ __forceinline__ void e2m1x8_to_f16x2x4(uint32_t x, uint32_t (&h)[4]) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+      : "r"(x));
+}
+
+// f16x2 product, round to nearest even (exact for E2M1 x E4M3 values).
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
 // Four floats -> four E4M3 bytes (x0 in the lowest byte), round to nearest
 // even, saturating to +-448.
 __device__ __forceinline__ uint32_t f32x4_to_e4m3x4(float x0, float x1, float x2, float x3) {

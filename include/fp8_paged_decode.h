@@ -218,6 +218,8 @@ size_t fp8_paged_decode_workspace_bytes_qlen(int B, int q_len, int Hq, int Hkv, 
 #define FPD_KV_HND 1   /* pages [num_blocks, Hkv, block_tokens, D] (head-major) */
 #define FPD_Q_BF16 0
 #define FPD_Q_F16  1
+#define FPD_KV_E4M3  0   /* E4M3 codes, one byte per element */
+#define FPD_KV_NVFP4 1   /* E2M1 codes with an E4M3 scale per 16 elements */
 
 typedef struct {
     /* query token t = b * q_len + i, head h, element d is at
@@ -244,6 +246,20 @@ typedef struct {
     int64_t out_token_stride;    /* elements */
     float *lse;                  /* [B, q_len, Hq] contiguous, or NULL */
     int chunk_pages_override;    /* 0: heuristic */
+    /* Page format.  FPD_KV_NVFP4 (head-major pages only): k_cache / v_cache
+     * point at the E2M1 data of page 0, [Hkv][bt][D/2] bytes per page (element
+     * 2i of a row in the low nibble of byte i), and k_scales / v_scales at its
+     * E4M3 block scales, [Hkv][bt][D/16] bytes per page (one per 16 elements);
+     * consecutive pages are kv_page_stride (data) and sf_page_stride (scales)
+     * bytes apart, 0 meaning packed.  An element's value is
+     * e2m1(code) * e4m3(block scale) * k_scale (v_scale).  The writer's page
+     * [K data | K scales | V data | V scales] is four such pointers with one
+     * stride.  Strides must be multiples of 16. */
+    int kv_format;               /* FPD_KV_E4M3 or FPD_KV_NVFP4 */
+    const void *k_scales;
+    const void *v_scales;
+    int64_t kv_page_stride;
+    int64_t sf_page_stride;
 } fpd_decode_args;
 
 /*
@@ -259,6 +275,22 @@ typedef struct {
  */
 fpd_status fp8_paged_decode_attention_args(const fpd_decode_args *args, void *workspace,
                                            size_t workspace_bytes, void *stream);
+
+/* fp8_paged_decode_attention_args that also records the given cudaEvent_t
+ * handles (void*, each may be NULL) on `stream` before the split kernel,
+ * between the two kernels and after the combine kernel, as
+ * fp8_paged_decode_attention_profiled does. */
+fpd_status fp8_paged_decode_attention_args_profiled(const fpd_decode_args *args, void *workspace,
+                                                    size_t workspace_bytes, void *stream,
+                                                    void *event_before_split,
+                                                    void *event_after_split,
+                                                    void *event_after_combine);
+
+/* The plan and the workspace bytes of a descriptor's call on the current
+ * device (the page format changes the kernel's shared memory and so the
+ * plan).  workspace_bytes_args returns 0 for an invalid descriptor. */
+fpd_status fp8_paged_decode_plan_args(const fpd_decode_args *args, fpd_plan *plan);
+size_t fp8_paged_decode_workspace_bytes_args(const fpd_decode_args *args);
 
 /*
  * Same as fp8_paged_decode_attention_qlen, and additionally records the given
@@ -364,6 +396,33 @@ fpd_status fp8_paged_decode_cache_write_layout(const void *key, const void *valu
                                                float v_scale, void *k_cache, void *v_cache,
                                                int num_blocks, int block_tokens, int kv_layout,
                                                uint32_t *status, void *stream);
+
+/*
+ * NVFP4 KV-cache write: the block quantisation of the NVFP4 KV-cache serving
+ * gist's cache writer (its writer kernel and quantisation helper), with the
+ * reciprocals taken exactly in fp32 where the gist uses approximate ones.  For
+ * each 16 consecutive elements x of a token's K (V) head row, with
+ * gs = 1 / k_scale (1 / v_scale):
+ *   scale = e4m3_rne_satfinite((max|x| * (1/6)) * gs)
+ *   code  = e2m1_rne_satfinite(x * (1 / (scale * (1 / gs))))   (0 if scale == 0)
+ * every product and reciprocal rounded to fp32.  Codes go to the data region
+ * and scales to the scale region of head-major NVFP4 pages (see
+ * fpd_decode_args: data [Hkv][bt][D/2] bytes, element 2i in the low nibble;
+ * scales [Hkv][bt][D/16]), at the given page strides (0 = packed).
+ *   key, value, slot_mapping, status: as in fp8_paged_decode_cache_write
+ *   k_data, k_sf, v_data, v_sf: 16-byte aligned device pointers to page 0
+ * Requires D % 16 == 0, num_blocks * block_tokens < 2^31, strides multiples of
+ * 16 and at least the packed region sizes, scales finite and > 0.  NaN inputs
+ * give unspecified codes.  Runs on `stream`, allocates nothing.
+ */
+fpd_status fp8_paged_decode_cache_write_nvfp4(const void *key, const void *value,
+                                              const int64_t *slot_mapping, int num_tokens,
+                                              int Hkv, int D, int64_t key_stride,
+                                              int64_t value_stride, float k_scale, float v_scale,
+                                              void *k_data, void *k_sf, void *v_data, void *v_sf,
+                                              int64_t data_page_stride, int64_t sf_page_stride,
+                                              int num_blocks, int block_tokens, uint32_t *status,
+                                              void *stream);
 
 /*
  * Reads the workspace status word (FPD_DEVERR_* bits) after synchronising
