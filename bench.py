@@ -66,6 +66,8 @@ def parse_args():
                     help="only run warm-up + K plain calls (for ncu launch lists and captures)")
     ap.add_argument("--json-out", default=None)
     ap.add_argument("--op", default="decode", choices=["decode", "cache_write"])
+    ap.add_argument("--kv-format", default="e4m3", choices=["e4m3", "nvfp4"],
+                    help="page format: E4M3 (token-major) or NVFP4 (head-major) pages")
     ap.add_argument("--q-len", type=int, default=1,
                     help="query tokens per sequence (speculative decode of the same workload)")
     ap.add_argument("--write-tokens", type=int, default=65536)
@@ -119,11 +121,12 @@ def kernel_source_hash():
     return h.hexdigest()
 
 
-def traffic_key(config_name, q_len):
-    return config_name if q_len == 1 else f"{config_name}/q{q_len}"
+def traffic_key(config_name, q_len, kv_format="e4m3"):
+    key = config_name if q_len == 1 else f"{config_name}/q{q_len}"
+    return key if kv_format == "e4m3" else f"{key}/{kv_format}"
 
 
-def ncu_traffic(config_name, kv_bytes, plan=None, q_len=1):
+def ncu_traffic(config_name, kv_bytes, plan=None, q_len=1, kv_format="e4m3"):
     """DRAM bytes per split-kernel launch from the committed ncu summary, scaled
     to this launch's KV bytes; None when absent, taken on other kernel code or
     recorded for another launch plan."""
@@ -134,7 +137,7 @@ def ncu_traffic(config_name, kv_bytes, plan=None, q_len=1):
         d = json.load(f)
     if d.get("source_sha256") != kernel_source_hash():
         return None
-    e = d.get("workloads", {}).get(traffic_key(config_name, q_len))
+    e = d.get("workloads", {}).get(traffic_key(config_name, q_len, kv_format))
     if not e:
         return None
     if plan is not None and e.get("plan") is not None and e["plan"] != plan:
@@ -233,13 +236,29 @@ class RawEvents:
 
 # ------------------------------------------------------------ CPU oracle --
 
+def make_wl(args):
+    from fp8_paged_decode_b200 import workloads as W
+    if args.kv_format == "nvfp4":
+        return W.make_workload_nvfp4(args.config, q_len=args.q_len)
+    return W.make_workload(args.config, q_len=args.q_len)
+
+
+def oracle_rows(wl, rows, threads=None):
+    import oracle
+    if wl.kv_format == "nvfp4":
+        return oracle.decode_nvfp4_workload(wl, rows=rows, threads=threads)
+    return oracle.decode_workload(wl, rows=rows, threads=threads)
+
+
 def rows_kv_bytes(wl, rows):
     """The workload's algorithmic KV bytes that the given output rows stand
     for: a sequence's K+V bytes are shared by its q_len * Hq rows, so each row
     is credited with that share (the metric counts each KV byte once)."""
-    att = wl.attended()
+    import numpy as np
+    att = wl.attended().astype(np.float64)
     per_seq = wl.q_len * wl.Hq
-    return sum(int(att[int(r) // per_seq]) for r in rows) * wl.Hkv * wl.D * 2 / per_seq
+    seq_bytes = att / max(att.sum(), 1.0) * wl.kv_bytes()
+    return sum(float(seq_bytes[int(r) // per_seq]) for r in rows) / per_seq
 
 
 def oracle_sample(wl, budget_s, rng_seed=0, threads=None, min_rows=1):
@@ -253,13 +272,13 @@ def oracle_sample(wl, budget_s, rng_seed=0, threads=None, min_rows=1):
     # calibrate on a few rows
     probe = order[:max(min_rows, min(len(order), threads))]
     t0 = time.perf_counter()
-    oracle.decode_workload(wl, rows=probe, threads=threads)
+    oracle_rows(wl, probe, threads=threads)
     t_probe = time.perf_counter() - t0
     per_row = t_probe / len(probe)
     n = int(max(min_rows, min(len(order), budget_s / max(per_row, 1e-6))))
     rows = order[:n]
     t0 = time.perf_counter()
-    oracle.decode_workload(wl, rows=rows, threads=threads)
+    oracle_rows(wl, rows, threads=threads)
     dt = time.perf_counter() - t0
     return dt, rows_kv_bytes(wl, rows), n, threads
 
@@ -273,7 +292,7 @@ def run_reference(args):
     import numpy as np
     from fp8_paged_decode_b200 import workloads as W
     import oracle
-    wl = W.make_workload(args.config, q_len=args.q_len)
+    wl = make_wl(args)
     threads = os.cpu_count() or 1
     total_steps = args.steps + args.warmup
     budget_s = 120.0
@@ -281,7 +300,7 @@ def run_reference(args):
     n_rows = wl.B * wl.q_len * wl.Hq
     probe = np.arange(min(n_rows, threads))
     t0 = time.perf_counter()
-    oracle.decode_workload(wl, rows=probe, threads=threads)
+    oracle_rows(wl, probe, threads=threads)
     per_row_wall = (time.perf_counter() - t0) / len(probe)
     rows_per_step = int(budget_s / total_steps / max(per_row_wall, 1e-7))
     rows_per_step = max(1, min(rows_per_step, n_rows))
@@ -290,7 +309,7 @@ def run_reference(args):
     for step in range(total_steps):
         rows = rng.choice(n_rows, size=rows_per_step, replace=False)
         t0 = time.perf_counter()
-        oracle.decode_workload(wl, rows=rows, threads=min(threads, rows_per_step))
+        oracle_rows(wl, rows, threads=min(threads, rows_per_step))
         dt = time.perf_counter() - t0
         if step >= args.warmup:
             t_sum += dt
@@ -304,7 +323,8 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": t_sum / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": W.describe(args.config), "q_len": wl.q_len, "sample": sample},
+        "config": {"workload": W.describe(args.config), "q_len": wl.q_len,
+                   "kv_format": wl.kv_format, "sample": sample},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": min(threads, rows_per_step),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -339,7 +359,7 @@ def run_native(args):
             dist.barrier()
 
     lib = fpd.load_library()
-    wl = W.make_workload(args.config, q_len=args.q_len)
+    wl = make_wl(args)
     dev = torch.device("cuda", local)
     props = torch.cuda.get_device_properties(dev)
     l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20))
@@ -350,38 +370,65 @@ def run_native(args):
     table = torch.from_numpy(wl.block_table).to(dev)
     lens = torch.from_numpy(wl.seq_lens).to(dev)
     sinks = None if wl.sinks is None else torch.from_numpy(wl.sinks).to(dev)
-    kc = [torch.from_numpy(wl.k_cache).to(dev) for _ in range(replicas)]
-    vc = [torch.from_numpy(wl.v_cache).to(dev) for _ in range(replicas)]
+    nvfp4 = wl.kv_format == "nvfp4"
+    if nvfp4:   # one tensor of pages [K data | K scales | V data | V scales] per replica
+        kc = [torch.from_numpy(wl.kv_cache).to(dev) for _ in range(replicas)]
+        vc = kc
+    else:
+        kc = [torch.from_numpy(wl.k_cache).to(dev) for _ in range(replicas)]
+        vc = [torch.from_numpy(wl.v_cache).to(dev) for _ in range(replicas)]
     lead = tuple(wl.q.shape[:-2])   # (B,) or (B, q_len)
     out = torch.empty(lead + (wl.Hq, wl.D), dtype=torch.bfloat16, device=dev)
     lse = torch.empty(lead + (wl.Hq,), dtype=torch.float32, device=dev)
-    need = fpd.fp8_paged_decode_workspace_bytes_qlen(wl.B, wl.q_len, wl.Hq, wl.Hkv, wl.D,
-                                                     wl.block_tokens, wl.max_blocks,
-                                                     wl.window_left, args.chunk_pages)
-    assert need > 0
-    wsp = torch.zeros(need, dtype=torch.uint8, device=dev)
-    plan = fpd.fp8_paged_decode_plan_qlen(wl.B, wl.q_len, wl.Hq, wl.Hkv, wl.D, wl.block_tokens,
-                                          wl.max_blocks, wl.window_left, args.chunk_pages)
     stream = torch.cuda.current_stream(dev)
     sh = ctypes.c_void_p(stream.cuda_stream)
     vp = ctypes.c_void_p
 
-    def call_args(i):
-        return [vp(q.data_ptr()), vp(kc[i].data_ptr()), vp(vc[i].data_ptr()), vp(table.data_ptr()),
-                vp(lens.data_ptr()), wl.B, wl.q_len, wl.Hq, wl.Hkv, wl.D, wl.num_blocks, wl.block_tokens,
-                wl.max_blocks, ctypes.c_float(wl.k_scale), ctypes.c_float(wl.v_scale),
-                ctypes.c_float(wl.sm_scale), wl.window_left,
-                vp(sinks.data_ptr()) if sinks is not None else None, vp(out.data_ptr()),
-                vp(lse.data_ptr()), vp(wsp.data_ptr()), ctypes.c_size_t(wsp.numel()), sh,
-                args.chunk_pages]
+    def descriptor(i):
+        """The call on replica i, as the C ABI's descriptor."""
+        a = fpd.fpd_decode_args()
+        a.q, a.q_dtype = q.data_ptr(), fpd.FPD_Q_BF16
+        if nvfp4:
+            lay = fpd.nvfp4_page_layout(wl.Hkv, wl.block_tokens, wl.D)
+            base = kc[i].data_ptr()
+            a.k_cache, a.v_cache = base + lay["k_data"], base + lay["v_data"]
+            a.k_scales, a.v_scales = base + lay["k_sf"], base + lay["v_sf"]
+            a.kv_page_stride = a.sf_page_stride = lay["page_bytes"]
+            a.kv_format, a.kv_layout = fpd.FPD_KV_NVFP4, fpd.FPD_KV_HND
+        else:
+            a.k_cache, a.v_cache = kc[i].data_ptr(), vc[i].data_ptr()
+            a.kv_format, a.kv_layout = fpd.FPD_KV_E4M3, fpd.FPD_KV_NHD
+        a.block_table, a.seq_lens = table.data_ptr(), lens.data_ptr()
+        a.B, a.q_len, a.Hq, a.Hkv, a.D = wl.B, wl.q_len, wl.Hq, wl.Hkv, wl.D
+        a.num_blocks, a.block_tokens, a.max_blocks = wl.num_blocks, wl.block_tokens, wl.max_blocks
+        a.k_scale, a.v_scale, a.sm_scale = wl.k_scale, wl.v_scale, wl.sm_scale
+        a.window_left = wl.window_left
+        a.sinks = sinks.data_ptr() if sinks is not None else None
+        a.out, a.lse = out.data_ptr(), lse.data_ptr()
+        a.chunk_pages_override = args.chunk_pages
+        return a
 
-    pre = [call_args(i) for i in range(replicas)]
-    f_prof = lib.fp8_paged_decode_attention_profiled
-    f_plain = lib.fp8_paged_decode_attention_qlen
+    descs = [descriptor(i) for i in range(replicas)]
+    refs = [ctypes.byref(d) for d in descs]
+    need = fpd.fp8_paged_decode_workspace_bytes_args(descs[0])
+    assert need > 0
+    wsp = torch.zeros(need, dtype=torch.uint8, device=dev)
+    plan_s = fpd.fpd_plan()
+    assert lib.fp8_paged_decode_plan_args(refs[0], ctypes.byref(plan_s)) == 0
+    plan = {f: getattr(plan_s, f) for f, _ in fpd.fpd_plan._fields_}
+    ws_ptr, ws_n = vp(wsp.data_ptr()), ctypes.c_size_t(wsp.numel())
+    f_args = lib.fp8_paged_decode_attention_args
+    f_args_prof = lib.fp8_paged_decode_attention_args_profiled
+
+    def f_plain(i):
+        return f_args(refs[i % replicas], ws_ptr, ws_n, sh)
+
+    def f_prof(i, e0, e1, e2):
+        return f_args_prof(refs[i % replicas], ws_ptr, ws_n, sh, e0, e1, e2)
 
     if args.kernels_only:
         for i in range(args.warmup + args.steps):
-            st = f_plain(*pre[i % replicas])
+            st = f_plain(i)
             assert st == 0, fpd.fp8_paged_decode_status_string(st)
         torch.cuda.synchronize()
         assert fpd.fp8_paged_decode_check_status(wsp) == 0
@@ -395,7 +442,7 @@ def run_native(args):
         return 0
 
     # correctness guard on this exact launch configuration (sampled rows vs oracle)
-    st = f_plain(*pre[0])
+    st = f_plain(0)
     assert st == 0, fpd.fp8_paged_decode_status_string(st)
     torch.cuda.synchronize()
     guard = None
@@ -404,7 +451,7 @@ def run_native(args):
         rng = np.random.default_rng(0)
         n_rows = wl.B * wl.q_len * wl.Hq
         rows = rng.choice(n_rows, size=min(16, n_rows), replace=False)
-        ro, rl = oracle.decode_workload(wl, rows=rows)
+        ro, rl = oracle_rows(wl, rows)
         # rows index (sequence, query token, head) in that order
         o = out.float().cpu().numpy().reshape(n_rows, wl.D)
         l = lse.cpu().numpy().reshape(n_rows)
@@ -421,7 +468,7 @@ def run_native(args):
 
     # warm-up
     for i in range(args.warmup):
-        st = f_plain(*pre[i % replicas])
+        st = f_plain(i)
         assert st == 0
     torch.cuda.synchronize()
 
@@ -436,7 +483,7 @@ def run_native(args):
     torch.cuda.synchronize()
     ev.record(0, stream.cuda_stream)
     for i in range(K):
-        st = f_plain(*pre[i % replicas])
+        st = f_plain(i)
         if st != 0:
             raise RuntimeError(fpd.fp8_paged_decode_status_string(st))
     ev.record(1, stream.cuda_stream)
@@ -452,7 +499,7 @@ def run_native(args):
     evr = RawEvents(3 * Kr)
     torch.cuda.synchronize()
     for i in range(Kr):
-        st = f_prof(*pre[i % replicas], vp(evr.handle(3 * i)), vp(evr.handle(3 * i + 1)),
+        st = f_prof(i, vp(evr.handle(3 * i)), vp(evr.handle(3 * i + 1)),
                     vp(evr.handle(3 * i + 2)))
         if st != 0:
             raise RuntimeError(fpd.fp8_paged_decode_status_string(st))
@@ -480,7 +527,7 @@ def run_native(args):
         d2h = hout.numel() * 2 + hlse.numel() * 4
         Ke = K
         for i in range(min(args.warmup, 50)):
-            st = f_plain(*pre[i % replicas])
+            st = f_plain(i)
         torch.cuda.synchronize()
         barrier()
         s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -491,7 +538,7 @@ def run_native(args):
             lens.copy_(hlen, non_blocking=True)
             if hsink is not None:
                 sinks.copy_(hsink, non_blocking=True)
-            st = f_plain(*pre[i % replicas])
+            st = f_plain(i)
             if st != 0:
                 raise RuntimeError(fpd.fp8_paged_decode_status_string(st))
             hout.copy_(out, non_blocking=True)
@@ -513,7 +560,8 @@ def run_native(args):
     split_avg_ms = statistics.fmean(split_ms)
     achieved = kv_bytes / (split_avg_ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                "frac": achieved / hbm, "traffic": ncu_traffic(args.config, kv_bytes, plan, wl.q_len),
+                "frac": achieved / hbm, "traffic": ncu_traffic(args.config, kv_bytes, plan, wl.q_len,
+                                                  wl.kv_format),
                 "kernel": f"fpd_split_kernel<{wl.D},{2 if wl.groups > 8 else 1}>",
                 "algorithmic_bytes_per_launch": kv_bytes,
                 "unit_bytes": f"2*D = {2 * wl.D} B per (attended token, KV head); "
@@ -536,10 +584,13 @@ def run_native(args):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-            "dtype_detail": "E4M3 KV converted exactly to f16; mma.sync f16 x f16 -> f32; "
+            "dtype_detail": ("E4M3 KV" if not nvfp4 else
+                             "NVFP4 KV (E2M1 x E4M3 block scale)") +
+                            " converted exactly to f16; mma.sync f16 x f16 -> f32; "
                             "softmax and reductions in f32; bf16 output",
             "data": "synthetic",
             "config": {"workload": W.describe(args.config), "B": wl.B, "q_len": wl.q_len,
+                       "kv_format": wl.kv_format,
                        "Hq": wl.Hq,
                        "Hkv": wl.Hkv, "D": wl.D, "block_tokens": wl.block_tokens,
                        "kv_bytes_per_call": kv_bytes, "parallelism": f"replicas x{ws}",
