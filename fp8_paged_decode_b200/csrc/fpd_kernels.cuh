@@ -394,38 +394,61 @@ struct Consumer {
     }
   }
 
-  // NVFP4 V rows 2t, 2t+1, 2t+8, 2t+9, this thread's elements [n*D/8, (n+1)*D/8)
-  // (D/16 bytes each, one block scale), as f16x2 words (word i = elements 2i,
-  // 2i+1), rows outside [tok_lo, tok_hi) zeroed when not FULL.
+  // NVFP4 V for the PV MMA: token pairs (2t, 2t+1) and (2t+8, 2t+9), this
+  // thread's elements [n*D/8, (n+1)*D/8) (D/16 bytes and one block scale per
+  // row).  vp[pr][e] = f16x2(element e of the pair's first token, of its
+  // second token), scaled, and zeroed for tokens outside [tok_lo, tok_hi)
+  // when not FULL.  The two tokens' codes are interleaved nibble by nibble
+  // before the conversion, so one cvt gives the MMA's token pair directly.
+  // Lanes alternate which token of a pair they load first so that every load
+  // spreads over all the banks (rows 0, 2, 4, 6 alone would share half).
   template <bool FULL>
-  __device__ __forceinline__ void fp4_v_rows(const uint8_t* Vd, const uint8_t* Vs, int tok0,
-                                             const TileMask& mk, int lane,
-                                             uint32_t (&vh)[4][D / 16]) {
+  __device__ __forceinline__ void fp4_v_pairs(const uint8_t* Vd, const uint8_t* Vs, int tok0,
+                                              const TileMask& mk, int lane,
+                                              uint32_t (&vp)[2][D / 8]) {
     const int n = lane >> 2, t = lane & 3;
+    const int swap = D == 128 ? (t & 1) : (t >> 1);
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int row = 2 * t + (r & 1) + 8 * (r >> 1);
-      uint32_t w[D / 64];
+    for (int pr = 0; pr < 2; ++pr) {
+      const int rowA = 2 * t + 8 * pr;
+      const int r0 = rowA + swap, r1 = rowA + 1 - swap;
+      uint32_t x[D / 64], y[D / 64], wa[D / 64], wb[D / 64];
       if constexpr (D == 128) {
-        const uint2 v = *reinterpret_cast<const uint2*>(Vd + row * (D / 2) + n * 8);
-        w[0] = v.x, w[1] = v.y;
+        const uint2 u = *reinterpret_cast<const uint2*>(Vd + r0 * (D / 2) + n * 8);
+        const uint2 v = *reinterpret_cast<const uint2*>(Vd + r1 * (D / 2) + n * 8);
+        x[0] = u.x, x[1] = u.y, y[0] = v.x, y[1] = v.y;
       } else {
-        w[0] = *reinterpret_cast<const uint32_t*>(Vd + row * (D / 2) + n * 4);
+        x[0] = *reinterpret_cast<const uint32_t*>(Vd + r0 * (D / 2) + n * 4);
+        y[0] = *reinterpret_cast<const uint32_t*>(Vd + r1 * (D / 2) + n * 4);
       }
-      const uint8_t sfc = Vs[row * (D / 16) + (D == 128 ? n : n / 2)];
-      const uint32_t s2 = e4m3x2_to_f16x2((uint16_t)sfc);
-      const uint32_t sc = prmt(s2, s2, 0x1010u);
+#pragma unroll
+      for (int w = 0; w < D / 64; ++w) {
+        wa[w] = swap ? y[w] : x[w];
+        wb[w] = swap ? x[w] : y[w];
+      }
+      const int blk = D == 128 ? n : n / 2;   // the block of this thread's elements
+      const uint16_t sab = (uint16_t)(Vs[rowA * (D / 16) + blk] |
+                                      (Vs[(rowA + 1) * (D / 16) + blk] << 8));
+      const uint32_t sc = e4m3x2_to_f16x2(sab);   // (scale of token A, of token B)
       uint32_t mask = 0xffffffffu;
       if (!FULL) {
-        const int tk = tok0 + row;
-        mask = (tk >= mk.tok_lo && tk < mk.tok_hi) ? 0xffffffffu : 0u;
+        const int ta = tok0 + rowA;
+        mask = ((ta >= mk.tok_lo && ta < mk.tok_hi) ? 0x0000ffffu : 0u) |
+               ((ta + 1 >= mk.tok_lo && ta + 1 < mk.tok_hi) ? 0xffff0000u : 0u);
       }
 #pragma unroll
-      for (int i = 0; i < D / 64; ++i) {
-        uint32_t h[4];
-        e2m1x8_to_f16x2x4(w[i], h);
+      for (int w = 0; w < D / 64; ++w) {
+        // byte j of lo: element 8w+2j of A (low nibble) and of B; hi: 8w+2j+1
+        const uint32_t lo = (wa[w] & 0x0F0F0F0Fu) | ((wb[w] << 4) & 0xF0F0F0F0u);
+        const uint32_t hi = ((wa[w] >> 4) & 0x0F0F0F0Fu) | (wb[w] & 0xF0F0F0F0u);
+        uint32_t L[4], H[4];
+        e2m1x8_to_f16x2x4(lo, L);
+        e2m1x8_to_f16x2x4(hi, H);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) vh[r][4 * i + j] = hmul2(h[j], sc) & mask;
+        for (int k = 0; k < 4; ++k) {
+          vp[pr][8 * w + 2 * k] = hmul2(L[k], sc) & mask;
+          vp[pr][8 * w + 2 * k + 1] = hmul2(H[k], sc) & mask;
+        }
       }
     }
   }
@@ -561,17 +584,15 @@ struct Consumer {
 
     if constexpr (FP4) {
       // ---- O^T += V^T P^T from NVFP4 rows: m-tile i takes element 2i (M row n)
-      // and 2i+1 (M row n + 8) of this thread's chunk, tokens paired by prmt
-      uint32_t vh[4][D / 16];
-      fp4_v_rows<FULL>(Vt, Vs, tok0, mk, lane, vh);
+      // and 2i+1 (M row n + 8) of this thread's chunk for both token pairs
+      uint32_t vp[2][D / 8];
+      fp4_v_pairs<FULL>(Vt, Vs, tok0, mk, lane, vp);
 #pragma unroll
       for (int i = 0; i < MT; ++i) {
-        const uint32_t a0 = prmt(vh[0][i], vh[1][i], 0x5410u);   // (A, B) element 2i
-        const uint32_t a1 = prmt(vh[0][i], vh[1][i], 0x7632u);   // (A, B) element 2i+1
-        const uint32_t a2 = prmt(vh[2][i], vh[3][i], 0x5410u);
-        const uint32_t a3 = prmt(vh[2][i], vh[3][i], 0x7632u);
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) mma_16816(o[i][nt], a0, a1, a2, a3, pb0[nt], pb1[nt]);
+        for (int nt = 0; nt < NT; ++nt)
+          mma_16816(o[i][nt], vp[0][2 * i], vp[0][2 * i + 1], vp[1][2 * i], vp[1][2 * i + 1],
+                    pb0[nt], pb1[nt]);
       }
       return;
     } else {
