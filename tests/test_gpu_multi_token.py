@@ -116,3 +116,17 @@ def test_llama_shape_speculative():
     qi, hi = np.divmod(rest, wl.Hq)
     assert_parity(out[bi, qi, hi][None], lse[bi, qi, hi][None], ref_out[bi, qi, hi][None],
                   ref_lse[bi, qi, hi][None], what="llama shape q_len=4")
+
+
+@pytest.mark.parametrize("g,Hkv", [(1, 4), (16, 1)])
+def test_max_q_len(g, Hkv):
+    """q_len at its limit: 64 queries per sequence (4 items of 16 positions for
+    g = 1, 64 one-position items for g = 16)."""
+    Q = fpd.FPD_MAX_Q_LEN
+    lens = [Q - 10, Q, 200, 1000]
+    wl = W.make_custom(B=len(lens), Hq=g * Hkv, Hkv=Hkv, D=64, block_tokens=16, seq_lens=lens,
+                       seed=700 + g, sm_scale=0.125, sinks=True, q_len=Q)
+    check(wl)
+    check(wl, chunk_pages=3)
+    wl.window_left = 30
+    check(wl, what=f"q_len {Q} window 30")

@@ -237,3 +237,86 @@ def test_write_then_decode():
     assert np.array_equal(pg.cpu().numpy(), want)
     wl.kv_cache, wl.k_scale, wl.v_scale = want, float(np.float32(ks)), float(np.float32(vs))
     check(wl, what="write then decode")
+
+
+def test_graph_capture_device_scales_no_allocation():
+    """NVFP4 decode captured in a CUDA graph with device scales: nothing is
+    allocated during capture, and replays after new scale values use them."""
+    wl = W.make_custom_nvfp4(B=4, Hq=32, Hkv=8, D=128, block_tokens=16,
+                             seq_lens=[2000, 10, 700, 4000], sinks=True, seed=640)
+    d = dev_inputs(wl)
+    ks = torch.tensor([wl.k_scale], dtype=torch.float32, device="cuda")
+    vs = torch.tensor([wl.v_scale], dtype=torch.float32, device="cuda")
+    out = torch.empty((4, 32, 128), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((4, 32), dtype=torch.float32, device="cuda")
+    ws = torch.zeros(64 << 20, dtype=torch.uint8, device="cuda")
+
+    def call():
+        fpd.fp8_paged_decode_attention_nvfp4(d["q"], d["kv"], d["table"], d["lens"], ks, vs,
+                                             wl.sm_scale, Hkv=8, block_tokens=16,
+                                             sinks=d["sinks"], out=out, lse=lse, workspace=ws)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        call()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        before = torch.cuda.memory_allocated()
+        call()
+        after = torch.cuda.memory_allocated()
+    assert after == before
+    for kx, vx in ((wl.k_scale, wl.v_scale), (wl.k_scale * 1.5, wl.v_scale * 0.5)):
+        ks.fill_(kx)
+        vs.fill_(vx)
+        out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        ro, rl = oracle.decode_nvfp4(wl.q, wl.kv_cache, wl.block_table, wl.seq_lens, Hkv=8,
+                                     block_tokens=16, k_scale=np.float32(kx),
+                                     v_scale=np.float32(vx), sm_scale=wl.sm_scale,
+                                     sinks=wl.sinks)
+        assert_parity(out.float().cpu().numpy().astype(np.float64),
+                      lse.cpu().numpy().astype(np.float64), ro, rl, what=f"replay {kx}, {vx}")
+
+
+def test_page_permutation_bitwise_and_repeat():
+    """Moving pages to other physical slots (and the table with them) changes no
+    bit of the result; two identical calls give identical bits."""
+    wl = W.make_custom_nvfp4(B=5, Hq=16, Hkv=4, D=128, block_tokens=32,
+                             seq_lens=[33, 500, 1, 1024, 77], sinks=True, seed=641)
+    out1, lse1 = run_nvfp4(wl, chunk=2)
+    out1b, lse1b = run_nvfp4(wl, chunk=2)
+    assert torch.equal(out1, out1b) and torch.equal(lse1, lse1b)
+    perm = np.random.default_rng(642).permutation(wl.num_blocks)
+    inv = np.argsort(perm)
+    wl2 = W.make_custom_nvfp4(B=5, Hq=16, Hkv=4, D=128, block_tokens=32,
+                              seq_lens=[33, 500, 1, 1024, 77], sinks=True, seed=641)
+    wl2.kv_cache = np.ascontiguousarray(wl.kv_cache[inv])       # page p moves to slot perm[p]
+    table = wl.block_table.copy()
+    table[table >= 0] = perm[table[table >= 0]]
+    wl2.block_table = table
+    out2, lse2 = run_nvfp4(wl2, chunk=2)
+    assert torch.equal(out1, out2) and torch.equal(lse1, lse2)
+
+
+def test_cache_write_strided_key_value():
+    """key and value as slices of a fused [T, (Hq + 2 Hkv) * D] projection."""
+    rng = np.random.default_rng(643)
+    T, Hq, Hkv, D, bt = 50, 16, 4, 128, 16
+    fused = torch.from_numpy(rng.standard_normal((T, (Hq + 2 * Hkv) * D)).astype(np.float32)) \
+        .to(torch.bfloat16).cuda()
+    key = fused[:, Hq * D:(Hq + Hkv) * D].view(T, Hkv, D)
+    value = fused[:, (Hq + Hkv) * D:].view(T, Hkv, D)
+    nb = T // bt + 2
+    lay = fpd.nvfp4_page_layout(Hkv, bt, D)
+    pg = torch.zeros((nb, lay["page_bytes"]), dtype=torch.uint8, device="cuda")
+    slots = rng.permutation(nb * bt)[:T].astype(np.int64)
+    fpd.fp8_paged_decode_cache_write_nvfp4(key, value, torch.from_numpy(slots).cuda(), pg, 0.05,
+                                           0.02, block_tokens=bt)
+    torch.cuda.synchronize()
+    kb = fused.cpu().view(torch.int16).numpy().view(np.uint16)
+    want = np.zeros((nb, lay["page_bytes"]), dtype=np.uint8)
+    oracle.cache_write_nvfp4(np.ascontiguousarray(kb[:, Hq * D:(Hq + Hkv) * D]).reshape(T, Hkv, D),
+                             np.ascontiguousarray(kb[:, (Hq + Hkv) * D:]).reshape(T, Hkv, D),
+                             slots, want, block_tokens=bt, k_scale=0.05, v_scale=0.02)
+    assert np.array_equal(pg.cpu().numpy(), want)
