@@ -106,9 +106,10 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, "fallback 6.65 TB/s (earlier measurement on this pool)"
 
 
-# The sources the E4M3 split and combine kernels and their launch are built
-# from; the ncu traffic record is valid only for this exact code.
-KERNEL_SOURCES = ("fpd_api.cu", "fpd_kernels.cuh", "fpd_ptx.cuh")
+# The device code of the split and combine kernels; the ncu traffic record is
+# valid only for this exact code and, per workload, for the launch plan it
+# records (checked in ncu_traffic).
+KERNEL_SOURCES = ("fpd_kernels.cuh", "fpd_ptx.cuh")
 
 
 def kernel_source_hash():
