@@ -418,6 +418,10 @@ cudaError_t launch_split_nvfp4_hb(int D, int NT, const CUtensorMap (&maps)[4],
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+#ifndef FPD_SINGLE_SPLIT_STAGES
+#define FPD_SINGLE_SPLIT_STAGES 6
+#endif
+
 // The split plan for a given stage shape (HB KV heads per stage).
 void plan_shape(int B, int q_len, int Hq, int Hkv, int D, int bt, int max_blocks,
                 int window_left, int64_t slots, int chunk_pages_override, int HB, fpd_plan* plan,
@@ -450,6 +454,16 @@ void plan_shape(int B, int q_len, int Hq, int Hkv, int D, int bt, int max_blocks
     if (chunk < min_chunk) chunk = min_chunk;
   }
   chunk = (chunk + pps - 1) / pps * pps;
+  // A call too small to fill the machine whose longest item is only a few
+  // stages runs one split per sequence: no combine launch, and the serial
+  // chain of a few stages is shorter than a second kernel (tiny batches).
+  if (chunk_pages_override == 0) {
+    const int64_t stage_tokens = fpd::kTileTokens / HB;
+    const int64_t longest = ((int64_t)pages_max * bt + stage_tokens - 1) / stage_tokens;
+    const int64_t splits_now = (pages_max + chunk - 1) / chunk;
+    if (longest <= FPD_SINGLE_SPLIT_STAGES && units * splits_now < slots)
+      chunk = (pages_max + pps - 1) / pps * pps;
+  }
   const int max_splits = (pages_max + chunk - 1) / chunk;
   const int64_t items_max = units * max_splits;
   plan->chunk_pages = chunk;

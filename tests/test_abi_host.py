@@ -246,3 +246,17 @@ def test_args_entry_accepts_the_variants(lib):
     assert f(None, ws, 1 << 20, None) == fpd.FPD_ERR_INVALID_ARG
     # misaligned q base stays rejected through the descriptor
     assert f(ctypes.byref(base_args(q=4100)), ws, 1 << 20, None) == fpd.FPD_ERR_INVALID_ARG
+
+
+def test_planner_single_split_for_tiny_calls():
+    """A call that cannot fill the machine and whose longest item is a few
+    stages gets one split (no combine launch); longer ones keep splitting."""
+    p = plan(B=2, Hq=8, Hkv=2, block_tokens=16, max_blocks=19)      # <= 304 tokens, 5 stages
+    assert p["max_splits"] == 1 and p["workspace_bytes"] == 256
+    p = plan(B=2, Hq=8, Hkv=2, block_tokens=16, max_blocks=40)      # 640 tokens, 10 stages
+    assert p["max_splits"] > 1
+    p = plan(B=2, Hq=32, Hkv=8, block_tokens=16, max_blocks=6)      # four-head stages: 6 stages
+    assert p["max_splits"] == 1
+    # overriding the split size still wins
+    assert plan(B=2, Hq=8, Hkv=2, block_tokens=16, max_blocks=19,
+                chunk_pages_override=4)["max_splits"] == 5
