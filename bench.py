@@ -62,6 +62,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU baseline sample budget")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="skip the CUDA-graph replay timing (L2 flushed before each replay)")
     ap.add_argument("--kernels-only", action="store_true",
                     help="only run warm-up + K plain calls (for ncu launch lists and captures)")
     ap.add_argument("--json-out", default=None)
@@ -514,6 +516,43 @@ def run_native(args):
     ms_per_step = max_total_ms / K
     value = whole_job_value(ws, kv_bytes, K, max_total_ms)
 
+    # One call captured in a CUDA graph, replayed with the L2 flushed before each
+    # replay (a write of 2x L2 bytes); median and p10/p90 of the replays.
+    graph = None
+    if not args.no_graph:
+        flush = torch.empty(2 * l2 // 4 + 1, dtype=torch.float32, device=dev)
+        gstream = torch.cuda.Stream(dev)
+        gstream.wait_stream(stream)
+        gh = vp(gstream.cuda_stream)
+        with torch.cuda.stream(gstream):
+            for _ in range(3):
+                assert f_args(refs[0], ws_ptr, ws_n, gh) == 0
+        torch.cuda.synchronize()
+        cg = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(cg, stream=gstream):
+            st = f_args(refs[0], ws_ptr, ws_n, gh)
+        assert st == 0, fpd.fp8_paged_decode_status_string(st)
+        n_rep, n_warm = 1000, 100
+        e_a = [torch.cuda.Event(enable_timing=True) for _ in range(n_rep)]
+        e_b = [torch.cuda.Event(enable_timing=True) for _ in range(n_rep)]
+        with torch.cuda.stream(gstream):
+            for i in range(n_warm):
+                flush.fill_(float(i))
+                cg.replay()
+            for i in range(n_rep):
+                flush.fill_(float(i))
+                e_a[i].record(gstream)
+                cg.replay()
+                e_b[i].record(gstream)
+        torch.cuda.synchronize()
+        tr = sorted(e_a[i].elapsed_time(e_b[i]) * 1e3 for i in range(n_rep))
+        graph = {"median_us": tr[n_rep // 2], "p10_us": tr[n_rep // 10],
+                 "p90_us": tr[(9 * n_rep) // 10], "replays": n_rep, "warmup_replays": n_warm,
+                 "l2_flush_bytes": int(flush.numel() * 4),
+                 "kv_gbs_at_median": kv_bytes / tr[n_rep // 2] / 1e3}
+        del cg
+        assert fpd.fp8_paged_decode_check_status(wsp, clear=True) == 0
+
     # end to end through the C ABI: pinned host inputs in, results out, every step
     e2e = None
     if not args.no_e2e:
@@ -607,6 +646,7 @@ def run_native(args):
             "pct_of_peak": 100.0 * value / hbm,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches_per_step * K, "clocks": clocks, "parity_guard": guard,
+            "graph_replay_cold_l2": graph,
         }
         print(json.dumps(line))
         if args.json_out:
