@@ -30,7 +30,8 @@ __all__ = [
     "FpdError", "library_path", "load_library", "fp8_paged_decode_make_plan",
     "fp8_paged_decode_make_plan_qlen", "FPD_MAX_Q_LEN", "FPD_KV_NHD", "FPD_KV_HND",
     "FPD_Q_BF16", "FPD_Q_F16", "fpd_decode_args", "fp8_paged_decode_cache_write_layout",
-    "FPD_KV_E4M3", "FPD_KV_NVFP4", "nvfp4_page_layout", "fp8_paged_decode_attention_nvfp4",
+    "FPD_KV_E4M3", "FPD_KV_NVFP4", "FPD_OUT_BF16", "FPD_OUT_F32", "fp8_paged_decode_cp_merge",
+    "nvfp4_page_layout", "fp8_paged_decode_attention_nvfp4",
     "fp8_paged_decode_cache_write_nvfp4", "fp8_paged_decode_workspace_bytes_args",
     "fp8_paged_decode_plan", "fp8_paged_decode_workspace_bytes",
     "fp8_paged_decode_workspace_bytes_ex", "fp8_paged_decode_attention_profiled",
@@ -58,6 +59,8 @@ FPD_Q_BF16 = 0
 FPD_Q_F16 = 1
 FPD_KV_E4M3 = 0
 FPD_KV_NVFP4 = 1
+FPD_OUT_BF16 = 0
+FPD_OUT_F32 = 1
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_NAME = "libfp8_paged_decode.so"
@@ -87,6 +90,7 @@ EXPORTED_SYMBOLS = (
     "fp8_paged_decode_cache_write_nvfp4",
     "fp8_paged_decode_plan_qlen",
     "fp8_paged_decode_workspace_bytes_qlen",
+    "fp8_paged_decode_cp_merge",
     "fp8_paged_decode_status_string",
     "fp8_paged_decode_version",
 )
@@ -124,7 +128,8 @@ class fpd_decode_args(ctypes.Structure):
                 ("out_token_stride", ctypes.c_int64), ("lse", ctypes.c_void_p),
                 ("chunk_pages_override", ctypes.c_int), ("kv_format", ctypes.c_int),
                 ("k_scales", ctypes.c_void_p), ("v_scales", ctypes.c_void_p),
-                ("kv_page_stride", ctypes.c_int64), ("sf_page_stride", ctypes.c_int64)]
+                ("kv_page_stride", ctypes.c_int64), ("sf_page_stride", ctypes.c_int64),
+                ("out_dtype", ctypes.c_int)]
 
 
 def library_path() -> str:
@@ -167,6 +172,8 @@ def _bind(lib):
     lib.fp8_paged_decode_cache_write_nvfp4.argtypes = [vp, vp, vp, ci, ci, ci, i64, i64, cf, cf,
                                                        vp, vp, vp, vp, i64, i64, ci, ci, vp, vp]
     lib.fp8_paged_decode_cache_write_nvfp4.restype = ci
+    lib.fp8_paged_decode_cp_merge.argtypes = [vp, ci, i64, i64, ci, ci, vp, vp, i64, vp, vp]
+    lib.fp8_paged_decode_cp_merge.restype = ci
     lib.fp8_paged_decode_plan_qlen.argtypes = [ci] * 9 + [ctypes.POINTER(fpd_plan)]
     lib.fp8_paged_decode_plan_qlen.restype = ci
     lib.fp8_paged_decode_workspace_bytes_qlen.argtypes = [ci] * 9
@@ -343,14 +350,16 @@ def _scale_arg(x, name):
 def fp8_paged_decode_attention(q, k_cache, v_cache, block_table, seq_lens, k_scale, v_scale,
                                sm_scale, window_left=-1, sinks=None, out=None, lse=None,
                                workspace=None, stream=None, chunk_pages_override=0,
-                               return_lse=True, kv_layout="NHD"):
+                               return_lse=True, kv_layout="NHD", out_dtype="bf16"):
     """Enqueue one decode call on ``stream`` (default: torch's current stream).
 
     ``q`` is [B, Hq, D] (one query token per sequence) or [B, q_len, Hq, D]
     (the q_len newest tokens of each sequence, causal), bf16 or fp16; its
     [Hq, D] rows must be contiguous, the tokens may be spaced further apart
-    (a slice of a fused QKV buffer).  ``out`` (bf16, q's shape, same rule) and
-    ``lse`` (float32, contiguous) are allocated when not given.  The caches are
+    (a slice of a fused QKV buffer).  ``out`` (q's shape, same rule; bf16, or
+    float32 for the partial result of a context-parallel rank) and ``lse``
+    (float32, contiguous) are allocated when not given, ``out`` with
+    ``out_dtype`` ("bf16" or "f32").  The caches are
     E4M3 (uint8 or float8_e4m3fn) [num_blocks, block_tokens, Hkv, D], or
     [num_blocks, Hkv, block_tokens, D] with ``kv_layout="HND"``.  ``k_scale`` /
     ``v_scale`` are numbers or one-element float32 CUDA tensors (read on the
@@ -375,25 +384,12 @@ def fp8_paged_decode_attention(q, k_cache, v_cache, block_table, seq_lens, k_sca
         raise ValueError("q and the caches disagree on head_dim")
     max_blocks = block_table.shape[1]
     dev = q.device
-    if out is None:
-        out = torch.empty(lead + (Hq, D), dtype=torch.bfloat16, device=dev)
-    if lse is None and return_lse:
-        lse = torch.empty(lead + (Hq,), dtype=torch.float32, device=dev)
-    need = fp8_paged_decode_workspace_bytes_qlen(B, q_len, Hq, Hkv, D, bt, max_blocks,
-                                                 window_left, chunk_pages_override)
-    if workspace is None:
-        if need == 0 and B > 0:   # surface the planner's own status
-            fp8_paged_decode_plan_qlen(B, q_len, Hq, Hkv, D, bt, max_blocks, window_left,
-                                       chunk_pages_override)
-            raise FpdError(FPD_ERR_UNSUPPORTED, "fp8_paged_decode_workspace_bytes")
-        workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)
+    out, lse = _alloc_outputs(out, lse, lead, Hq, D, dev, out_dtype, return_lse)
     for name, t in (("q", q), ("out", out)):
         if not isinstance(t, torch.Tensor) or not t.is_cuda:
             raise TypeError(f"{name} must be a CUDA tensor")
     if q.dtype not in (torch.bfloat16, torch.float16):
         raise TypeError("q must be bf16 or fp16")
-    if out.dtype != torch.bfloat16:
-        raise TypeError("out must be bf16")
     a = fpd_decode_args()
     a.q = q.data_ptr()
     a.q_dtype = FPD_Q_F16 if q.dtype == torch.float16 else FPD_Q_BF16
@@ -417,11 +413,48 @@ def fp8_paged_decode_attention(q, k_cache, v_cache, block_table, seq_lens, k_sca
     lp = _dev_ptr(lse, "lse", (torch.float32,), lead + (Hq,))
     a.lse = lp.value if lp is not None else None
     a.chunk_pages_override = int(chunk_pages_override)
-    st = load_library().fp8_paged_decode_attention_args(
+    a.out_dtype = _out_code(out)
+    _run_args(a, workspace, dev, stream, "fp8_paged_decode_attention")
+    return out, lse
+
+
+def _alloc_outputs(out, lse, lead, Hq, D, dev, out_dtype, return_lse):
+    import torch
+    if out_dtype not in ("bf16", "f32"):
+        raise ValueError("out_dtype must be 'bf16' or 'f32'")
+    if out is None:
+        dt = torch.float32 if out_dtype == "f32" else torch.bfloat16
+        out = torch.empty(lead + (Hq, D), dtype=dt, device=dev)
+    if lse is None and return_lse:
+        lse = torch.empty(lead + (Hq,), dtype=torch.float32, device=dev)
+    return out, lse
+
+
+def _out_code(out):
+    import torch
+    if out.dtype == torch.bfloat16:
+        return FPD_OUT_BF16
+    if out.dtype == torch.float32:
+        return FPD_OUT_F32
+    raise TypeError("out must be bf16 or float32")
+
+
+def _run_args(a, workspace, dev, stream, where):
+    """Run a filled descriptor; allocates the workspace it needs when none is given."""
+    import torch
+    lib = load_library()
+    if workspace is None:
+        need = int(lib.fp8_paged_decode_workspace_bytes_args(ctypes.byref(a)))
+        if need == 0 and a.B > 0:   # surface the planner's own status
+            plan = fpd_plan()
+            _check(lib.fp8_paged_decode_plan_args(ctypes.byref(a), ctypes.byref(plan)),
+                   "fp8_paged_decode_plan_args")
+            raise FpdError(FPD_ERR_UNSUPPORTED, "fp8_paged_decode_workspace_bytes_args")
+        workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)
+    st = lib.fp8_paged_decode_attention_args(
         ctypes.byref(a), _dev_ptr(workspace, "workspace", (torch.uint8,)),
         ctypes.c_size_t(workspace.numel()), _stream_handle(stream))
-    _check(st, "fp8_paged_decode_attention")
-    return out, lse
+    _check(st, where)
 
 
 fp8_paged_decode_attention_ex = fp8_paged_decode_attention
@@ -507,7 +540,7 @@ def _nvfp4_pointers(kv_pages, Hkv, block_tokens, D):
 def fp8_paged_decode_attention_nvfp4(q, kv_pages, block_table, seq_lens, k_scale, v_scale,
                                      sm_scale, *, Hkv, block_tokens, window_left=-1, sinks=None,
                                      out=None, lse=None, workspace=None, stream=None,
-                                     chunk_pages_override=0, return_lse=True):
+                                     chunk_pages_override=0, return_lse=True, out_dtype="bf16"):
     """Decode over NVFP4 pages: ``kv_pages`` uint8 [num_blocks, page_bytes], each
     page [K data | K scales | V data | V scales] (``nvfp4_page_layout``; head-major
     E2M1 pairs, element 2i in the low nibble, and one E4M3 scale per 16
@@ -524,12 +557,9 @@ def fp8_paged_decode_attention_nvfp4(q, kv_pages, block_table, seq_lens, k_scale
     num_blocks = kv_pages.shape[0]
     max_blocks = block_table.shape[1]
     dev = q.device
-    if out is None:
-        out = torch.empty(lead + (Hq, D), dtype=torch.bfloat16, device=dev)
-    if lse is None and return_lse:
-        lse = torch.empty(lead + (Hq,), dtype=torch.float32, device=dev)
-    if q.dtype not in (torch.bfloat16, torch.float16) or out.dtype != torch.bfloat16:
-        raise TypeError("q must be bf16 or fp16 and out bf16")
+    out, lse = _alloc_outputs(out, lse, lead, Hq, D, dev, out_dtype, return_lse)
+    if q.dtype not in (torch.bfloat16, torch.float16):
+        raise TypeError("q must be bf16 or fp16")
     a = fpd_decode_args()
     a.q = q.data_ptr()
     a.q_dtype = FPD_Q_F16 if q.dtype == torch.float16 else FPD_Q_BF16
@@ -554,24 +584,40 @@ def fp8_paged_decode_attention_nvfp4(q, kv_pages, block_table, seq_lens, k_scale
     lp = _dev_ptr(lse, "lse", (torch.float32,), lead + (Hq,))
     a.lse = lp.value if lp is not None else None
     a.chunk_pages_override = int(chunk_pages_override)
-    lib = load_library()
-    if workspace is None:
-        need = int(lib.fp8_paged_decode_workspace_bytes_args(ctypes.byref(a)))
-        if need == 0 and B > 0:
-            plan = fpd_plan()
-            _check(lib.fp8_paged_decode_plan_args(ctypes.byref(a), ctypes.byref(plan)),
-                   "fp8_paged_decode_plan_args")
-            raise FpdError(FPD_ERR_UNSUPPORTED, "fp8_paged_decode_workspace_bytes_args")
-        workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)
-    st = lib.fp8_paged_decode_attention_args(
-        ctypes.byref(a), _dev_ptr(workspace, "workspace", (torch.uint8,)),
-        ctypes.c_size_t(workspace.numel()), _stream_handle(stream))
-    _check(st, "fp8_paged_decode_attention_nvfp4")
+    a.out_dtype = _out_code(out)
+    _run_args(a, workspace, dev, stream, "fp8_paged_decode_attention_nvfp4")
     return out, lse
 
 
 def fp8_paged_decode_workspace_bytes_args(args) -> int:
     return int(load_library().fp8_paged_decode_workspace_bytes_args(ctypes.byref(args)))
+
+
+def fp8_paged_decode_cp_merge(partials, out, lse=None, sinks=None, stream=None):
+    """Enqueue the context-parallel merge: ``partials`` float32 [R, block_floats],
+    rank r's row holding its f32 decode output [rows, D] followed by its lse
+    [rows] (``cp.partial_views`` lays a buffer out so), rows = out.numel() / D;
+    ``out`` bf16 [B, Hq, D] or [B, q_len, Hq, D] ([Hq, D] rows contiguous),
+    ``lse`` float32 of out's leading shape or None, ``sinks`` float32 [Hq] or
+    None.  Returns ``(out, lse)``."""
+    import torch
+    if out.dim() not in (3, 4) or out.dtype != torch.bfloat16:
+        raise TypeError("out must be bf16 [B, Hq, D] or [B, q_len, Hq, D]")
+    Hq, D = out.shape[-2], out.shape[-1]
+    lead = tuple(out.shape[:-2])
+    rows = out.numel() // D
+    if partials.dim() != 2:
+        raise ValueError("partials must be [R, block_floats]")
+    R, block = partials.shape
+    pp = _dev_ptr(partials, "partials", (torch.float32,))
+    lp = _dev_ptr(lse, "lse", (torch.float32,), lead + (Hq,))
+    sp = _dev_ptr(sinks, "sinks", (torch.float32,), (Hq,))
+    st = load_library().fp8_paged_decode_cp_merge(
+        pp, int(R), int(block), int(rows), int(Hq), int(D), sp,
+        ctypes.c_void_p(out.data_ptr()), _token_rows(out, "out", lead, Hq, D), lp,
+        _stream_handle(stream))
+    _check(st, "fp8_paged_decode_cp_merge")
+    return out, lse
 
 
 def fp8_paged_decode_cache_write_nvfp4(key, value, slot_mapping, kv_pages, k_scale, v_scale, *,

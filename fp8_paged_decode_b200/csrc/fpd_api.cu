@@ -13,6 +13,7 @@
 
 #include "fp8_paged_decode.h"
 #include "fpd_cache_write.cuh"
+#include "fpd_cp_merge.cuh"
 #include "fpd_kernels.cuh"
 
 namespace {
@@ -123,15 +124,17 @@ struct WsLayout {
   size_t part_o, part_lse, total, zero_prefix;
 };
 
-WsLayout ws_layout(int B, int Hq, int Hkv, int D, int max_splits) {
+// f32_out: every row goes through the combine, so partials exist for one split too.
+WsLayout ws_layout(int B, int Hq, int Hkv, int D, int max_splits, bool f32_out = false) {
   (void)Hkv;
   WsLayout w;
   size_t off = kHeaderBytes;
   w.zero_prefix = off;  // bytes that must be zero before the first call
+  const bool parts = max_splits > 1 || f32_out;
   w.part_o = off;
-  if (max_splits > 1) off += align_up((size_t)B * Hq * max_splits * D * sizeof(float), 256);
+  if (parts) off += align_up((size_t)B * Hq * max_splits * D * sizeof(float), 256);
   w.part_lse = off;
-  if (max_splits > 1) off += align_up((size_t)B * Hq * max_splits * sizeof(float), 256);
+  if (parts) off += align_up((size_t)B * Hq * max_splits * sizeof(float), 256);
   w.total = off;
   return w;
 }
@@ -632,6 +635,19 @@ static fpd_decode_args plain_args(const void* q, const void* k_cache, const void
   return a;
 }
 
+// The plan of a descriptor's call: its page format sets the kernel, and an
+// f32 output keeps a partial for every row.
+static fpd_status plan_args_impl(const fpd_decode_args& a, fpd_plan* plan) {
+  if (a.kv_format != FPD_KV_E4M3 && a.kv_format != FPD_KV_NVFP4) return FPD_ERR_INVALID_ARG;
+  if (a.out_dtype != FPD_OUT_BF16 && a.out_dtype != FPD_OUT_F32) return FPD_ERR_INVALID_ARG;
+  const fpd_status st =
+      plan_device(a.B, a.q_len, a.Hq, a.Hkv, a.D, a.block_tokens, a.max_blocks, a.window_left,
+                  a.chunk_pages_override, plan, a.kv_format == FPD_KV_NVFP4);
+  if (st == FPD_OK && a.out_dtype == FPD_OUT_F32)
+    plan->workspace_bytes = ws_layout(a.B * a.q_len, a.Hq, a.Hkv, a.D, plan->max_splits, true).total;
+  return st;
+}
+
 static fpd_status attention_impl(const fpd_decode_args& a, void* workspace,
                                  size_t workspace_bytes, void* stream, void* ev0, void* ev1,
                                  void* ev2) {
@@ -645,7 +661,9 @@ static fpd_status attention_impl(const fpd_decode_args& a, void* workspace,
   if (a.q_dtype != FPD_Q_BF16 && a.q_dtype != FPD_Q_F16) return FPD_ERR_INVALID_ARG;
   if (a.kv_layout != FPD_KV_NHD && a.kv_layout != FPD_KV_HND) return FPD_ERR_INVALID_ARG;
   if (a.kv_format != FPD_KV_E4M3 && a.kv_format != FPD_KV_NVFP4) return FPD_ERR_INVALID_ARG;
+  if (a.out_dtype != FPD_OUT_BF16 && a.out_dtype != FPD_OUT_F32) return FPD_ERR_INVALID_ARG;
   const bool fp4 = a.kv_format == FPD_KV_NVFP4;
+  const bool f32_out = a.out_dtype == FPD_OUT_F32;
   // NVFP4 pages: head-major, data and scale regions at their own page strides
   const int64_t fp4_data = (int64_t)Hkv * bt * (D / 2), fp4_sf = (int64_t)Hkv * bt * (D / 16);
   const int64_t data_stride = a.kv_page_stride ? a.kv_page_stride : fp4_data;
@@ -683,8 +701,7 @@ static fpd_status attention_impl(const fpd_decode_args& a, void* workspace,
 
   const int g = Hq / Hkv;
   fpd_plan plan;
-  st = plan_device(B, q_len, Hq, Hkv, D, bt, max_blocks, window_left, a.chunk_pages_override,
-                   &plan, fp4);
+  st = plan_args_impl(a, &plan);
   if (st != FPD_OK) return st;
   if (!workspace || workspace_bytes < plan.workspace_bytes) return FPD_ERR_WORKSPACE_TOO_SMALL;
 
@@ -704,7 +721,7 @@ static fpd_status attention_impl(const fpd_decode_args& a, void* workspace,
     return FPD_ERR_CUDA;
   }
 
-  const WsLayout wl = ws_layout(B * q_len, Hq, Hkv, D, plan.max_splits);
+  const WsLayout wl = ws_layout(B * q_len, Hq, Hkv, D, plan.max_splits, f32_out);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   fpd::DecodeParams p;
   p.q = static_cast<const __nv_bfloat16*>(a.q);
@@ -742,6 +759,7 @@ static fpd_status attention_impl(const fpd_decode_args& a, void* workspace,
   p.sm_scale_log2 = a.sm_scale * fpd::kLog2e;
   p.q_f16 = a.q_dtype == FPD_Q_F16;
   p.kv_hnd = hnd;
+  p.out_f32 = f32_out ? static_cast<float*>(a.out) : nullptr;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (ev0 && cudaEventRecord(static_cast<cudaEvent_t>(ev0), s) != cudaSuccess) return FPD_ERR_CUDA;
@@ -763,13 +781,14 @@ static fpd_status attention_impl(const fpd_decode_args& a, void* workspace,
            : launch_split_hb<1, false>(D, NT, km, vm, p, ctas, smem, s);
   if (e != cudaSuccess) return FPD_ERR_CUDA;
   if (ev1 && cudaEventRecord(static_cast<cudaEvent_t>(ev1), s) != cudaSuccess) return FPD_ERR_CUDA;
-  if (plan.max_splits > 1) {
+  if (plan.max_splits > 1 || f32_out) {
     fpd::CombineParams c;
     c.seq_lens = a.seq_lens;
     c.sinks = a.sinks;
     c.part_o = p.part_o;
     c.part_lse = p.part_lse;
     c.out = p.out;
+    c.out_f32 = p.out_f32;
     c.lse = a.lse;
     c.B = B;
     c.q_len = q_len;
@@ -845,11 +864,7 @@ fpd_status fp8_paged_decode_attention_args_profiled(const fpd_decode_args* args,
 
 fpd_status fp8_paged_decode_plan_args(const fpd_decode_args* args, fpd_plan* plan) {
   if (!args || !plan) return FPD_ERR_INVALID_ARG;
-  if (args->kv_format != FPD_KV_E4M3 && args->kv_format != FPD_KV_NVFP4)
-    return FPD_ERR_INVALID_ARG;
-  return plan_device(args->B, args->q_len, args->Hq, args->Hkv, args->D, args->block_tokens,
-                     args->max_blocks, args->window_left, args->chunk_pages_override, plan,
-                     args->kv_format == FPD_KV_NVFP4);
+  return plan_args_impl(*args, plan);
 }
 
 size_t fp8_paged_decode_workspace_bytes_args(const fpd_decode_args* args) {
@@ -996,6 +1011,38 @@ fpd_status fp8_paged_decode_cache_write_layout(const void* key, const void* valu
   const int grid = (int)(want < cap ? want : cap);
   fpd::fpd_cache_write_kernel<<<grid, fpd::kWriteThreads, 0, static_cast<cudaStream_t>(stream)>>>(
       p);
+  return cudaGetLastError() == cudaSuccess ? FPD_OK : FPD_ERR_CUDA;
+}
+
+fpd_status fp8_paged_decode_cp_merge(const float* partials, int R, int64_t block_floats,
+                                     int64_t rows, int Hq, int D, const float* sinks, void* out,
+                                     int64_t out_token_stride, float* lse, void* stream) {
+  if (R < 1 || Hq < 1 || rows < 0 || rows % Hq != 0) return FPD_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FPD_ERR_UNSUPPORTED;
+  if (block_floats < rows * (D + 1) || block_floats % 4 != 0) return FPD_ERR_INVALID_ARG;
+  const int64_t o_stride = out_token_stride ? out_token_stride : (int64_t)Hq * D;
+  if (o_stride < (int64_t)Hq * D || o_stride % 8 != 0) return FPD_ERR_INVALID_ARG;
+  if (!partials || !out || !aligned(partials, 16) || !aligned(out, 16) ||
+      (lse && !aligned(lse, 4)) || (sinks && !aligned(sinks, 4)))
+    return FPD_ERR_INVALID_ARG;
+  if (rows == 0) return FPD_OK;
+  const int64_t grid = (rows + fpd::kCpMergeWarps - 1) / fpd::kCpMergeWarps;
+  if (grid > INT32_MAX) return FPD_ERR_UNSUPPORTED;
+  fpd::CpMergeParams p;
+  p.partials = partials;
+  p.sinks = sinks;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.block = block_floats;
+  p.rows = rows;
+  p.out_tok_stride = o_stride;
+  p.R = R;
+  p.Hq = Hq;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (D == 128)
+    fpd::fpd_cp_merge_kernel<128><<<(int)grid, fpd::kCpMergeWarps * 32, 0, s>>>(p);
+  else
+    fpd::fpd_cp_merge_kernel<64><<<(int)grid, fpd::kCpMergeWarps * 32, 0, s>>>(p);
   return cudaGetLastError() == cudaSuccess ? FPD_OK : FPD_ERR_CUDA;
 }
 

@@ -110,6 +110,9 @@ struct DecodeParams {
   float sm_scale_log2;        // sm_scale * log2(e), for a device k_scale
   int q_f16;                  // the query is fp16 (else bf16)
   int kv_hnd;                 // pages are [num_blocks, Hkv, bt, D] (else [.., bt, Hkv, D])
+  // f32 output (same element strides as `out`): every row, one split or
+  // several, leaves its partial in the workspace and the combine writes it
+  float* out_f32;
 };
 
 // Bytes of one header slot: the header, then the item's query rows (HB KV
@@ -686,7 +689,9 @@ struct Consumer {
         __nv_bfloat16* const orow = p.out + tok * p.out_tok_stride + (size_t)hq * D;
         // false: this query saw no key in the item (only possible with MQ)
         const bool keys = !MQ || lsum[nt][j] > 0.f;
-        if (ns == 0 || (ns == 1 && !keys)) {  // no key at all: out = 0, lse = sigma
+        const bool one = ns == 1 && !p.out_f32;   // finished here, not by the combine
+        if (ns == 0 || (one && !keys)) {  // no key at all: out = 0, lse = sigma
+          if (p.out_f32) continue;        // the combine writes the row
           uint4* dst = reinterpret_cast<uint4*>(orow + n * E);
 #pragma unroll
           for (int k = 0; k < E / 8; ++k) dst[k] = make_uint4(0u, 0u, 0u, 0u);
@@ -694,7 +699,7 @@ struct Consumer {
           continue;
         }
         const float lse2 = m[nt][j] + __log2f(lsum[nt][j]);   // log2-sum-exp, no sink
-        if (ns == 1) {
+        if (one) {
           float scale = v_scale;
           float lse_out = lse2;
           if (p.sinks) {
@@ -1194,7 +1199,7 @@ __device__ __forceinline__ void split_body(const CUtensorMap* kmap, const CUtens
       alive = false;
       break;
     }
-    const bool single = hd.ns <= 1;
+    const bool single = hd.ns <= 1 && !p.out_f32;   // else the combine finishes the rows
     {
       // thread -> (d, first head); heads step by 128 / D.  The loop body is
       // independent per head, so it is unrolled for overlap.
@@ -1208,6 +1213,7 @@ __device__ __forceinline__ void split_body(const CUtensorMap* kmap, const CUtens
         const size_t row = tok * p.Hq + hq;
         __nv_bfloat16* const orow = p.out + tok * p.out_tok_stride + (size_t)hq * D;
         if (hd.ns == 0) {  // empty sequence: out = 0, lse = sigma
+          if (p.out_f32) continue;   // the combine writes the row
           orow[d] = __float2bfloat16_rn(0.f);
           if (d == 0 && p.lse) p.lse[row] = p.sinks ? p.sinks[hq] : -INFINITY;
           continue;
@@ -1313,6 +1319,7 @@ struct CombineParams {
   const float* part_o;
   const float* part_lse;
   __nv_bfloat16* out;
+  float* out_f32;     // non-null: f32 output, and every row is merged here
   float* lse;
   int B, q_len, Hq, bt, max_blocks, window_left, chunk_pages, max_splits;
   int wpr;            // warps per row: 1, 2, 4, 8, 16 or 32
@@ -1321,6 +1328,22 @@ struct CombineParams {
   const float* v_scale_dev;   // device v_scale or nullptr
   int64_t out_tok_stride;     // elements between consecutive output tokens
 };
+
+// One lane's PER consecutive output elements, x[i] * inv, as bf16 or f32.
+template <int PER>
+__device__ __forceinline__ void store_out_row(const CombineParams& p, size_t off, const float* x,
+                                              float inv) {
+  if (p.out_f32) {
+    float* dst = p.out_f32 + off;
+#pragma unroll
+    for (int i = 0; i < PER; i += 2)
+      *reinterpret_cast<float2*>(dst + i) = make_float2(x[i] * inv, x[i + 1] * inv);
+  } else {
+    __nv_bfloat16* dst = p.out + off;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) dst[i] = __float2bfloat16_rn(x[i] * inv);
+  }
+}
 
 constexpr int kCombineMaxThreads = 1024;
 constexpr int kCombineBatch = 8;   // partials a warp loads before it reduces them
@@ -1378,7 +1401,8 @@ __global__ void __launch_bounds__(kCombineMaxThreads) fpd_combine_kernel(const C
   const int ns =
       seq_range(L_raw, QL, p.bt, p.max_blocks, p.window_left, p.chunk_pages, nullptr)
           .n_splits;
-  const bool active = in_range && ns > 1;   // rows with one split were written already
+  // rows with one split were written by the split kernel, unless the output is f32
+  const bool active = in_range && (ns > 1 || p.out_f32);
 
   // ---- this warp's splits against its own maximum m
   float m = -INFINITY, z = 0.f;
@@ -1428,17 +1452,18 @@ __global__ void __launch_bounds__(kCombineMaxThreads) fpd_combine_kernel(const C
   // ---- merge the row's warps (M = max over warps and the sink) and write
   const int hq = row % p.Hq;
   const float sink2 = (active && p.sinks) ? p.sinks[hq] * kLog2e : -INFINITY;
-  __nv_bfloat16* const orow = p.out + (size_t)(row / p.Hq) * p.out_tok_stride + (size_t)hq * D;
+  // this lane's PER output elements of the row
+  const size_t ooff = (size_t)(row / p.Hq) * p.out_tok_stride + (size_t)hq * D + lane * PER;
   if (wpr == 1) {
     if (active) {
       const float M = fmaxf(m, sink2);
       const float r = fast_exp2(m - M);
       const float Z = z * r + (p.sinks ? fast_exp2(sink2 - M) : 0.f);
-      const float inv = v_scale * r / Z;
-      __nv_bfloat16* dst = orow + lane * PER;
-#pragma unroll
-      for (int i = 0; i < PER; ++i) dst[i] = __float2bfloat16_rn(acc[i] * inv);
-      if (lane == 0 && p.lse) p.lse[row] = (M + __log2f(Z)) * kLn2;
+      // false only for an f32 row with no key and no sink: out = 0, lse = -inf
+      const bool any = Z > 0.f;
+      const float inv = any ? v_scale * r / Z : 0.f;
+      store_out_row<PER>(p, ooff, acc, inv);
+      if (lane == 0 && p.lse) p.lse[row] = any ? (M + __log2f(Z)) * kLn2 : -INFINITY;
     }
     return;
   }
@@ -1460,7 +1485,8 @@ __global__ void __launch_bounds__(kCombineMaxThreads) fpd_combine_kernel(const C
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) Z += __shfl_xor_sync(0xffffffffu, Z, o);
     if (p.sinks) Z += fast_exp2(sink2 - M);
-    const float inv = v_scale / Z;
+    const bool any = Z > 0.f;   // as above
+    const float inv = any ? v_scale / Z : 0.f;
     float a[PER];
 #pragma unroll
     for (int i = 0; i < PER; ++i) a[i] = 0.f;
@@ -1469,10 +1495,8 @@ __global__ void __launch_bounds__(kCombineMaxThreads) fpd_combine_kernel(const C
 #pragma unroll
       for (int i = 0; i < PER; ++i) a[i] = fmaf(acc_sm[warp + w][lane * PER + i], r, a[i]);
     }
-#pragma unroll
-    for (int i = 0; i < PER; ++i)
-      orow[lane * PER + i] = __float2bfloat16_rn(a[i] * inv);
-    if (lane == 0 && p.lse) p.lse[row] = (M + __log2f(Z)) * kLn2;
+    store_out_row<PER>(p, ooff, a, inv);
+    if (lane == 0 && p.lse) p.lse[row] = any ? (M + __log2f(Z)) * kLn2 : -INFINITY;
   }
 }
 

@@ -220,6 +220,8 @@ size_t fp8_paged_decode_workspace_bytes_qlen(int B, int q_len, int Hq, int Hkv, 
 #define FPD_Q_F16  1
 #define FPD_KV_E4M3  0   /* E4M3 codes, one byte per element */
 #define FPD_KV_NVFP4 1   /* E2M1 codes with an E4M3 scale per 16 elements */
+#define FPD_OUT_BF16 0   /* out is bf16 */
+#define FPD_OUT_F32  1   /* out is f32: the (O, lse) partial of a context-parallel rank */
 
 typedef struct {
     /* query token t = b * q_len + i, head h, element d is at
@@ -260,6 +262,13 @@ typedef struct {
     const void *v_scales;
     int64_t kv_page_stride;
     int64_t sf_page_stride;
+    /* Output type.  FPD_OUT_F32: out is f32 with the same element strides
+     * (nonzero out_token_stride a multiple of 8, out 16-byte aligned); every
+     * row is then finished by the combine kernel, so the workspace holds one
+     * partial per row even when no sequence is split: size it with
+     * fp8_paged_decode_workspace_bytes_args.  A row with no key and no sink
+     * gets out = 0 and lse = -inf, which fp8_paged_decode_cp_merge skips. */
+    int out_dtype;               /* FPD_OUT_BF16 or FPD_OUT_F32 */
 } fpd_decode_args;
 
 /*
@@ -288,7 +297,8 @@ fpd_status fp8_paged_decode_attention_args_profiled(const fpd_decode_args *args,
 
 /* The plan and the workspace bytes of a descriptor's call on the current
  * device (the page format changes the kernel's shared memory and so the
- * plan).  workspace_bytes_args returns 0 for an invalid descriptor. */
+ * plan, and an f32 output needs the partials even for one split).
+ * workspace_bytes_args returns 0 for an invalid descriptor. */
 fpd_status fp8_paged_decode_plan_args(const fpd_decode_args *args, fpd_plan *plan);
 size_t fp8_paged_decode_workspace_bytes_args(const fpd_decode_args *args);
 
@@ -423,6 +433,42 @@ fpd_status fp8_paged_decode_cache_write_nvfp4(const void *key, const void *value
                                               int64_t data_page_stride, int64_t sf_page_stride,
                                               int num_blocks, int block_tokens, uint32_t *status,
                                               void *stream);
+
+/*
+ * Context-parallel decode: the merge.  When each of R ranks holds part of
+ * every sequence's KV pages, each computes the decode over its own keys with
+ * no sinks and an f32 output (fpd_decode_args.out_dtype = FPD_OUT_F32), the
+ * ranks exchange those (O_r, lse_r) partials (an all-gather), and this call
+ * folds them into the attention over all keys:
+ *   out = sum_r e^(lse_r - M) O_r / Z,   lse = M + ln Z,
+ *   Z = sum_r e^(lse_r - M) + e^(sigma - M),   M = max(max_r lse_r, sigma),
+ * sigma = sinks[h] (absent: -inf).  This is the split-KV merge of partial O
+ * and LSE of FlashInfer PR #5591 (Summary: the workspace's partial_O /
+ * partial_lse and its split merge), with ranks in place of splits; that page
+ * lists decode context parallelism (DCP) as unsupported ("Unsupported"
+ * section), so the partition of the keys is the caller's.
+ *   partials     f32, R blocks of block_floats floats, one per rank in any
+ *                order: a block's first rows * D floats are O_r [rows][D],
+ *                the next rows floats lse_r [rows] (natural log, -inf for a
+ *                rank with no key of the row), the rest padding.  rows =
+ *                B * q_len * Hq, a row being (token, head) with the head
+ *                innermost.  An all-gather of each rank's [O | lse | pad]
+ *                buffer produces this layout.
+ *   block_floats >= rows * (D + 1), a multiple of 4 (16-byte blocks).
+ *   sinks        f32 [Hq] or NULL.
+ *   out          bf16; row (t, h) at out[t * out_token_stride + h * D];
+ *                out_token_stride 0 means Hq * D.
+ *   lse          f32 [rows] or NULL.
+ * R >= 1, Hq >= 1, D in {64, 128}, rows >= 0 a multiple of Hq; partials and
+ * out 16-byte aligned, out_token_stride a multiple of 8 and >= Hq * D.  A row that
+ * no rank and no sink covers gets out = 0 and lse = -inf.  The call enqueues
+ * one kernel and does not synchronise.  Errors: FPD_ERR_INVALID_ARG (null
+ * pointer, bad alignment, stride or count), FPD_ERR_UNSUPPORTED (D),
+ * FPD_ERR_CUDA (launch failure).  Nothing is written on error.
+ */
+fpd_status fp8_paged_decode_cp_merge(const float *partials, int R, int64_t block_floats,
+                                     int64_t rows, int Hq, int D, const float *sinks, void *out,
+                                     int64_t out_token_stride, float *lse, void *stream);
 
 /*
  * Reads the workspace status word (FPD_DEVERR_* bits) after synchronising

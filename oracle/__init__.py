@@ -50,6 +50,8 @@ def _bind(lib):
     lib.fpd_oracle_decode_x.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, ci,
                                         cd, cd, cd, ci, vp, vp, vp, vp, ci, ci, ci, ci]
     lib.fpd_oracle_decode_x.restype = ci
+    lib.fpd_oracle_merge.argtypes = [vp, vp, ci, ctypes.c_long, ci, ci, vp, vp, vp]
+    lib.fpd_oracle_merge.restype = None
     lib.fpd_oracle_f16_to_f64.argtypes = [ctypes.c_uint16]
     lib.fpd_oracle_f16_to_f64.restype = ctypes.c_double
     lib.fpd_oracle_e2m1_to_f64.argtypes = [ctypes.c_uint8]
@@ -317,3 +319,23 @@ def cache_write_nvfp4(key, value, slot_mapping, kv_cache, *, block_tokens, k_sca
     if st < 0:
         raise ValueError("oracle rejected the NVFP4 cache-write arguments")
     return st
+
+
+def merge(o_parts, lse_parts, Hq: int, sinks=None, lib=None):
+    """The merge of R partial results of disjoint key sets (``fpd_oracle_merge``):
+    ``o_parts`` [R, *lead, Hq, D] and ``lse_parts`` [R, *lead, Hq] (natural log,
+    -inf for a part with no key), ``sinks`` [Hq] or None.  Returns fp64
+    (out [*lead, Hq, D], lse [*lead, Hq])."""
+    lib = lib or load()
+    o = np.ascontiguousarray(o_parts, dtype=np.float64)
+    l = np.ascontiguousarray(lse_parts, dtype=np.float64)
+    R, D = o.shape[0], o.shape[-1]
+    lead = o.shape[1:-1]
+    rows = int(np.prod(lead))
+    if l.shape != (R,) + tuple(lead) or lead[-1] != Hq:
+        raise ValueError("o_parts / lse_parts shapes disagree")
+    s = None if sinks is None else np.ascontiguousarray(sinks, dtype=np.float32)
+    out = np.zeros(tuple(lead) + (D,), dtype=np.float64)
+    lse = np.zeros(tuple(lead), dtype=np.float64)
+    lib.fpd_oracle_merge(_ptr(o), _ptr(l), R, rows, D, Hq, _ptr(s), _ptr(out), _ptr(lse))
+    return out, lse

@@ -38,7 +38,9 @@
  * exponent 0 is subnormal; S.1111.111 is NaN; there are no infinities.
  *
  * The file also holds the oracle of the FP8 cache write that fills such a
- * cache (fpd_oracle_cache_write, below the E4M3 codec).
+ * cache (fpd_oracle_cache_write, below the E4M3 codec), and the merge of
+ * partial results over disjoint key sets that context-parallel decode needs
+ * (fpd_oracle_merge, at the end).
  *
  * Several query tokens per sequence (speculative / multi-token decode): the
  * sequence's q_len newest tokens are queries.  Query i (0 <= i < q_len) sits at
@@ -585,4 +587,51 @@ int fpd_oracle_decode(const uint16_t *q, const uint8_t *k_cache, const uint8_t *
     return fpd_oracle_decode_q(q, k_cache, v_cache, block_table, seq_lens, B, 1, Hq, Hkv, D,
                                num_blocks, bt, max_blocks, k_scale, v_scale, sm_scale,
                                window_left, sinks, out, lse, rows, n_rows, n_threads);
+}
+
+/*
+ * The merge of partial results (context-parallel decode).  When the keys of a
+ * row are split into R disjoint parts, part r giving the attention over its
+ * own keys without a sink, O_r = sum_{j in r} e^(s_j - m_r) v_j / Z_r and
+ * lse_r = m_r + ln Z_r, the attention over all keys follows from the split-KV
+ * merge of partial O and LSE (FlashInfer PR #5591, Summary), since
+ * e^(lse_r) = sum_{j in r} e^(s_j):
+ *   M   = max(max_r lse_r, sigma)
+ *   Z   = sum_r e^(lse_r - M) + e^(sigma - M)
+ *   out = sum_r e^(lse_r - M) O_r / Z,   lse = M + ln Z
+ * A part with no key (lse_r = -inf) weighs nothing; with no part and no sink
+ * out = 0 and lse = -inf, as in the decode.
+ *   o_parts [R][rows][D], lse_parts [R][rows]; row = (token, head), head
+ *   innermost, so its sink is sinks[row % Hq].
+ */
+void fpd_oracle_merge(const double *o_parts, const double *lse_parts, int R, long rows, int D,
+                      int Hq, const float *sinks, double *out, double *lse)
+{
+    long row;
+    int r, d;
+    for (row = 0; row < rows; ++row) {
+        const double sigma = sinks ? (double)sinks[row % Hq] : -INFINITY;
+        double M = sigma, Z = 0.0;
+        double *o = out + (size_t)row * D;
+        for (r = 0; r < R; ++r)
+            if (lse_parts[(size_t)r * rows + row] > M)
+                M = lse_parts[(size_t)r * rows + row];
+        for (d = 0; d < D; ++d)
+            o[d] = 0.0;
+        if (M == -INFINITY) {
+            lse[row] = -INFINITY;
+            continue;
+        }
+        for (r = 0; r < R; ++r) {
+            const double l = lse_parts[(size_t)r * rows + row];
+            const double w = l == -INFINITY ? 0.0 : exp(l - M);
+            Z += w;
+            for (d = 0; d < D; ++d)
+                o[d] += w * o_parts[((size_t)r * rows + row) * D + d];
+        }
+        Z += exp(sigma - M);
+        for (d = 0; d < D; ++d)
+            o[d] /= Z;
+        lse[row] = M + log(Z);
+    }
 }

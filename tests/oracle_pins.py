@@ -771,10 +771,45 @@ def pin_nvfp4_round_trip(lib):
     assert (np.abs(d2 - bf16_library(yb)) <= step + 1e-12).all(), "round-trip error above one step"
 
 
+def _page_split(table, lens, bt, parts, r):
+    """Part r of `parts` of every sequence's pages: a contiguous run of whole pages."""
+    pages = -(-lens // bt)
+    t = np.zeros_like(table)
+    l = np.zeros_like(lens)
+    for b in range(len(lens)):
+        p0, p1 = r * pages[b] // parts, (r + 1) * pages[b] // parts
+        t[b, :p1 - p0] = table[b, p0:p1]
+        l[b] = max(0, min(p1 * bt, lens[b]) - p0 * bt)
+    return t, l
+
+
+def pin_merge_library(lib):
+    """The merge of partial results over disjoint key sets (context-parallel
+    decode): the oracle's decodes of each part's keys, without the sink,
+    merged with the sink, equal dense attention over all keys by torch SDPA
+    and scipy logsumexp.  Parts from 1 to 5, some of them empty."""
+    for wl in small_cases():
+        if wl.window_left >= 0:
+            continue   # windows and positions are not part of the merge
+        for parts in (1, 2, 3, 5):
+            o_p, l_p = [], []
+            for r in range(parts):
+                t, l = _page_split(wl.block_table, wl.seq_lens, wl.block_tokens, parts, r)
+                o, ls = oracle.decode(wl.q, wl.k_cache, wl.v_cache, t, l, k_scale=wl.k_scale,
+                                      v_scale=wl.v_scale, sm_scale=wl.sm_scale, sinks=None,
+                                      threads=4, lib=lib)
+                o_p.append(o)
+                l_p.append(ls)
+            out, lse = oracle.merge(np.stack(o_p), np.stack(l_p), wl.Hq, wl.sinks, lib=lib)
+            ref_out, ref_lse = library_attention(wl)
+            close(out, ref_out, rtol=1e-10, atol=1e-12, what=f"merged out ({wl.name}, {parts})")
+            close(lse, ref_lse, rtol=1e-12, atol=1e-12, what=f"merged lse ({wl.name}, {parts})")
+
+
 ALL_PINS = [pin_e4m3_codes, pin_bf16, pin_library_attention, pin_zero_keys, pin_window_zero,
             pin_constant_values, pin_invariants, pin_softmax_identity, pin_e4m3_encode_library,
             pin_e4m3_encode_closed, pin_cache_write_library, pin_cache_write_invariants,
             pin_multi_token_library, pin_multi_token_prefix, pin_f16_codes,
             pin_f16_query_library, pin_hnd_layout, pin_e2m1_codes, pin_e2m1_encode_library,
             pin_nvfp4_decode_library, pin_nvfp4_page_strides, pin_nvfp4_writer_library,
-            pin_nvfp4_round_trip]
+            pin_nvfp4_round_trip, pin_merge_library]

@@ -77,6 +77,12 @@ MUTANTS = {
         ("page_row(hnd, (int)(slot / bt)", "page_row(!hnd, (int)(slot / bt)")],
     "writer value read with the key stride": [("value[t * value_stride + (long)h * D + d]",
                                                "value[t * key_stride + (long)h * D + d]")],
+    "merge drops the sink": [("        Z += exp(sigma - M);\n        for (d = 0; d < D; ++d)\n            o[d] /= Z;",
+                              "        for (d = 0; d < D; ++d)\n            o[d] /= Z;")],
+    "merge weights parts equally": [("const double w = l == -INFINITY ? 0.0 : exp(l - M);",
+                                     "const double w = l == -INFINITY ? 0.0 : 1.0;")],
+    "merge lse without the maximum": [("lse[row] = M + log(Z);", "lse[row] = log(Z);")],
+    "merge sink of the wrong head": [("(double)sinks[row % Hq]", "(double)sinks[(row + 1) % Hq]")],
     "last key dropped": [("for (j = start; j < end; ++j) {\n        const int page = J->block_table"
                           "[(size_t)b * J->max_blocks + j / J->bt];\n        const uint8_t *vr",
                           "for (j = start; j < end - 1; ++j) {\n        const int page = J->block_table"
