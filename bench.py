@@ -67,7 +67,10 @@ def parse_args():
     ap.add_argument("--kernels-only", action="store_true",
                     help="only run warm-up + K plain calls (for ncu launch lists and captures)")
     ap.add_argument("--json-out", default=None)
-    ap.add_argument("--op", default="decode", choices=["decode", "cache_write"])
+    ap.add_argument("--op", default="decode", choices=["decode", "cache_write", "cp"])
+    ap.add_argument("--cp-ranks", type=int, default=8,
+                    help="--op cp on one process: the context-parallel width whose rank "
+                         "step is timed (under torchrun the world size is the width)")
     ap.add_argument("--kv-format", default="e4m3", choices=["e4m3", "nvfp4"],
                     help="page format: E4M3 (token-major) or NVFP4 (head-major) pages")
     ap.add_argument("--q-len", type=int, default=1,
@@ -744,12 +747,194 @@ def run_cache_write(args):
     return 0
 
 
+def run_cp(args):
+    """Context-parallel decode of one workload over R ranks: each rank decodes
+    its contiguous page share of every sequence into an f32 partial, the
+    partials are all-gathered over NCCL, and each rank merges them.  Under
+    torchrun (R = world size) every step runs all three, timed per step on
+    each rank, max over ranks.  On one process the step of the rank with the
+    most keys of an R-way partition is timed (its decode and the merge of R
+    partials computed beforehand) and the exchange is not run.  L2 is evicted
+    (a 256 MiB read) before each timed step, outside the timed events."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import fp8_paged_decode_b200 as fpd
+    from fp8_paged_decode_b200 import cp
+    from fp8_paged_decode_b200 import workloads as W
+
+    ws, rank, local = dist_env()
+    assert ws == args.gpus, f"--gpus {args.gpus} but WORLD_SIZE={ws}"
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        dist.init_process_group("nccl", init_method="env://", device_id=dev,
+                                timeout=__import__("datetime").timedelta(seconds=120))
+    R = ws if ws > 1 else args.cp_ranks
+    if args.kv_format != "e4m3" or args.q_len != 1:
+        raise SystemExit("--op cp: E4M3 pages and one query per sequence")
+    wl = make_wl(args)
+    if wl.window_left >= 0:
+        raise SystemExit(f"--op cp: {args.config} has a sliding window, which context-parallel "
+                         "decode does not take")
+    B, Hq, D, bt = wl.B, wl.Hq, wl.D, wl.block_tokens
+    q = torch.from_numpy(wl.q.view(np.int16)).view(torch.bfloat16).to(dev)
+    kc = torch.from_numpy(wl.k_cache).to(dev)
+    vc = torch.from_numpy(wl.v_cache).to(dev)
+    sinks = None if wl.sinks is None else torch.from_numpy(wl.sinks).to(dev)
+    shards = [cp.cp_shard(wl.block_table, wl.seq_lens, R, r, bt) for r in range(R)]
+    keys = [int(l.astype(np.int64).sum()) for _, l in shards]
+    me = rank if ws > 1 else int(np.argmax(keys))
+    rows = B * Hq
+    blk = cp.partial_block_floats(rows, D)
+    partial = torch.zeros(blk, dtype=torch.float32, device=dev)
+    gathered = torch.zeros((R, blk), dtype=torch.float32, device=dev)
+    out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    lib = fpd.load_library()
+    stream = torch.cuda.current_stream(dev)
+    sh = ctypes.c_void_p(stream.cuda_stream)
+    vp = ctypes.c_void_p
+
+    def descriptor(table, lens, buf):
+        """The f32 partial decode of one rank's keys into `buf`, as the C ABI's descriptor."""
+        a = fpd.fpd_decode_args()
+        a.q, a.q_dtype = q.data_ptr(), fpd.FPD_Q_BF16
+        a.k_cache, a.v_cache = kc.data_ptr(), vc.data_ptr()
+        a.kv_format, a.kv_layout = fpd.FPD_KV_E4M3, fpd.FPD_KV_NHD
+        a.block_table, a.seq_lens = table.data_ptr(), lens.data_ptr()
+        a.B, a.q_len, a.Hq, a.Hkv, a.D = B, 1, Hq, wl.Hkv, D
+        a.num_blocks, a.block_tokens, a.max_blocks = wl.num_blocks, bt, table.shape[1]
+        a.k_scale, a.v_scale, a.sm_scale = wl.k_scale, wl.v_scale, wl.sm_scale
+        a.window_left, a.sinks = -1, None
+        a.out, a.lse = buf.data_ptr(), buf.data_ptr() + rows * D * 4
+        a.out_dtype = fpd.FPD_OUT_F32
+        a.chunk_pages_override = args.chunk_pages
+        return a
+
+    dev_shards = [(torch.from_numpy(t).to(dev), torch.from_numpy(l).to(dev)) for t, l in shards]
+    descs = [descriptor(*dev_shards[r], gathered[r]) for r in range(R)]
+    mine = descriptor(*dev_shards[me], partial)
+    need = max(fpd.fp8_paged_decode_workspace_bytes_args(d) for d in descs)
+    assert need > 0
+    wsp = torch.zeros(need, dtype=torch.uint8, device=dev)
+    ws_ptr, ws_n = vp(wsp.data_ptr()), ctypes.c_size_t(wsp.numel())
+    f_dec = lib.fp8_paged_decode_attention_args
+    merge_args = (vp(gathered.data_ptr()), R, blk, rows, Hq, D,
+                  vp(sinks.data_ptr()) if sinks is not None else None, vp(out.data_ptr()), 0,
+                  vp(lse.data_ptr()), sh)
+    if ws == 1:   # every rank's partial, once: the merge's input
+        for d in descs:
+            assert f_dec(ctypes.byref(d), ws_ptr, ws_n, sh) == 0
+    mine_ref = ctypes.byref(mine)
+
+    def step():
+        st = f_dec(mine_ref, ws_ptr, ws_n, sh)
+        if ws > 1:
+            cp.cp_exchange(partial, None, gathered)
+        st |= lib.fp8_paged_decode_cp_merge(*merge_args)
+        assert st == 0
+
+    # L2 is evicted by reading a 256 MiB buffer (a reduction), which leaves no
+    # dirty lines whose write-back would compete with the timed reads
+    flush_buf = torch.ones(256 * 2 ** 20, dtype=torch.uint8, device=dev)
+    flush = lambda: torch.amax(flush_buf)
+    K = max(1, min(args.steps, 2000))
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.25)
+    torch.cuda.synchronize()
+    # the timed steps: two events around each step, L2 flushed before it
+    pairs = [(ev(), ev()) for _ in range(K)]
+    for e0, e1 in pairs:
+        flush()
+        e0.record(stream)
+        step()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    total_ms = float(sum(e0.elapsed_time(e1) for e0, e1 in pairs))
+    mx = max_over_ranks(total_ms, dev) if ws > 1 else total_ms
+    ms = mx / K
+    # breakdown (untimed for the line's value): the rank's decode alone, the merge alone
+    dec = [(ev(), ev()) for _ in range(min(K, 200))]
+    for e0, e1 in dec:
+        flush()
+        e0.record(stream)
+        assert f_dec(mine_ref, ws_ptr, ws_n, sh) == 0
+        e1.record(stream)
+    # the merge alone: a CUDA graph of 100 launches, replayed 10 times
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    graph = torch.cuda.CUDAGraph()
+    side_args = merge_args[:-1] + (ctypes.c_void_p(side.cuda_stream),)
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            for _ in range(100):
+                lib.fp8_paged_decode_cp_merge(*side_args)
+    stream.wait_stream(side)
+    graph.replay()
+    m0, m1 = ev(), ev()
+    m0.record(stream)
+    for _ in range(10):
+        graph.replay()
+    m1.record(stream)
+    torch.cuda.synchronize()
+    del graph
+    dec_ms = float(np.median([e0.elapsed_time(e1) for e0, e1 in dec]))
+    merge_ms = m0.elapsed_time(m1) / 1000
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    row_kv = wl.Hkv * D * 2   # K and V bytes of one token
+    all_bytes = int(wl.seq_lens.astype(np.int64).sum()) * row_kv
+    my_bytes = keys[me] * row_kv
+    gbs = all_bytes / (ms / 1e3) / 1e9
+    hbm, peak_src = measured_peaks()
+    line = {
+        "metric": "context-parallel decode: KV GB/s over all ranks' keys per step; us/step",
+        "value": gbs, "unit": "GB/s", "n_gpus": ws, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms, "us_per_step": ms * 1e3, "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "cp_ranks": R,
+        "exchange": ("nccl all_gather_into_tensor of the f32 partials" if ws > 1 else
+                     "not run: one GPU; the timed step is one rank's decode and merge"),
+        "us_alone": {"partial_decode_median_cold_l2": dec_ms * 1e3,
+                     "merge_graph_replay": merge_ms * 1e3},
+        "rank_kv_bytes": my_bytes, "all_kv_bytes": all_bytes,
+        "partial_decode_frac_of_peak": my_bytes / (dec_ms / 1e3) / 1e9 / hbm,
+        "peak_source": peak_src,
+        "exchange_bytes_per_rank": blk * 4,
+        "config": {"workload": f"{W.describe(args.config)}; keys split into {R} "
+                               "contiguous page runs per sequence",
+                   "l2": "evicted (a 256 MiB read) before each timed step"},
+        "clocks": clocks,
+        "gpu_launches": K * 3,   # split, combine and merge kernels per step
+    }
+    print(json.dumps(line))
+    if args.json_out:
+        with open(args.json_out, "w") as fo:
+            json.dump(line, fo, indent=1)
+    return 0
+
+
 def main():
     args = parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.op == "cache_write":
         return run_cache_write(args)
+    if args.op == "cp":
+        return run_cp(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_native(args)

@@ -108,7 +108,7 @@ class fpd_plan(ctypes.Structure):
                 ("stages", ctypes.c_int), ("header_slots", ctypes.c_int),
                 ("ctas", ctypes.c_int), ("smem_bytes", ctypes.c_int),
                 ("workspace_bytes", ctypes.c_size_t), ("q_per_item", ctypes.c_int),
-                ("q_chunks", ctypes.c_int)]
+                ("q_chunks", ctypes.c_int), ("adapt_chunk_pages", ctypes.c_int)]
 
 
 class fpd_decode_args(ctypes.Structure):

@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -27,6 +28,7 @@ constexpr size_t kHeaderBytes = 256;    // status word, work counter, finished-C
 // larger items.
 constexpr int kTargetWaves1 = 8, kMinChunkRows1 = 256;    // one KV head per stage
 constexpr int kTargetWaves4 = 5, kMinChunkRows4 = 1024;   // four KV heads per stage
+constexpr int kMinItemTokens = 48;   // shortest split when a call cannot fill the machine
 constexpr int kOccCacheSize = 32;
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -427,8 +429,8 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 
 // The split plan for a given stage shape (HB KV heads per stage).
 void plan_shape(int B, int q_len, int Hq, int Hkv, int D, int bt, int max_blocks,
-                int window_left, int64_t slots, int chunk_pages_override, int HB, fpd_plan* plan,
-                bool fp4 = false) {
+                int window_left, int num_sms, int64_t slots, int chunk_pages_override, int HB,
+                fpd_plan* plan, bool fp4 = false) {
   const int g = Hq / Hkv;
   const int qp = q_per_item(q_len, g);
   const int q_chunks = (q_len + qp - 1) / qp;
@@ -443,20 +445,43 @@ void plan_shape(int B, int q_len, int Hq, int Hkv, int D, int bt, int max_blocks
     if (w < pages_max) pages_max = (int)w;
   }
   const int64_t units = (int64_t)(B > 0 ? B : 1) * (Hkv / HB) * q_chunks;
-  int chunk;
+  const auto round_pps = [pps](int64_t c) { return (int)((c + pps - 1) / pps * pps); };
+  const auto splits_at = [pages_max](int c) { return (int64_t)((pages_max + c - 1) / c); };
+  int chunk, adapt = 0;
+  int64_t grid_items = 0;   // items the grid is sized for (0: those of `chunk`)
   if (chunk_pages_override > 0) {
-    chunk = chunk_pages_override;
+    chunk = round_pps(chunk_pages_override);
   } else {
     const int waves = HB == 1 ? kTargetWaves1 : kTargetWaves4;
     const int min_rows = HB == 1 ? kMinChunkRows1 : kMinChunkRows4;
     int64_t splits = (waves * slots + units - 1) / units;
     if (splits < 1) splits = 1;
-    chunk = (int)((pages_max + splits - 1) / splits);
-    const int min_tokens = min_rows / HB;
-    const int min_chunk = (min_tokens + bt - 1) / bt;
-    if (chunk < min_chunk) chunk = min_chunk;
+    chunk = round_pps((pages_max + splits - 1) / splits);
+    const int min_chunk = round_pps(((int64_t)min_rows / HB + bt - 1) / bt);
+    if (chunk < min_chunk) {
+      // Too few pages for `waves` rounds of items of the minimum size.  Such
+      // calls run best as about two items per SM in one round (measured on
+      // uniform batches): items of equal size fill every SM alike.
+      chunk = min_chunk;
+      const int64_t target = 2 * (int64_t)num_sms;
+      const int one_round = round_pps((pages_max + (target + units - 1) / units - 1) /
+                                      ((target + units - 1) / units));
+      const int floor_chunk = round_pps((kMinItemTokens + bt - 1) / bt);
+      const int64_t items_min = units * splits_at(chunk);
+      if (items_min <= target) {
+        // under-filled: split finer, down to items of a few stages, unless
+        // the call needs no split at all (then no combine runs)
+        if (splits_at(chunk) > 1) chunk = std::max(one_round, floor_chunk);
+      } else if (2 * items_min <= 5 * slots && one_round > chunk) {
+        // between one and 2.5 rounds: larger items in one round, taken by
+        // the kernel only if the sequences turn out to be of about equal
+        // length (it sees the lengths; the plan does not); the grid is
+        // sized for those items
+        adapt = one_round;
+        grid_items = units * splits_at(adapt);
+      }
+    }
   }
-  chunk = (chunk + pps - 1) / pps * pps;
   // A call too small to fill the machine whose longest item is only a few
   // stages runs one split per sequence: no combine launch, and the serial
   // chain of a few stages is shorter than a second kernel (tiny batches).
@@ -468,8 +493,9 @@ void plan_shape(int B, int q_len, int Hq, int Hkv, int D, int bt, int max_blocks
       chunk = (pages_max + pps - 1) / pps * pps;
   }
   const int max_splits = (pages_max + chunk - 1) / chunk;
-  const int64_t items_max = units * max_splits;
+  const int64_t items_max = grid_items > 0 ? grid_items : units * max_splits;
   plan->chunk_pages = chunk;
+  plan->adapt_chunk_pages = adapt;
   plan->max_splits = max_splits;
   plan->heads_per_stage = HB;
   plan->stage_tokens = fpd::kTileTokens / HB;
@@ -483,26 +509,21 @@ void plan_shape(int B, int q_len, int Hq, int Hkv, int D, int bt, int max_blocks
   plan->q_chunks = q_chunks;
 }
 
-// Validates and plans.  force_hb = 0 picks the stage shape: four KV heads per
-// stage when Hkv allows it and the four-head work items fill every CTA slot
-// at least once; otherwise (short windows over few sequences) one head per
-// stage, whose 4x more numerous items keep the machine busy.
+// Validates and plans.  The stage shape is four KV heads per stage whenever
+// Hkv allows it, also when the four-head items of a call leave CTA slots idle
+// (short windows, few sequences): one-head items of the same keys were slower
+// on every such shape measured, since each item pays its set-up and epilogue.
 fpd_status plan_for(int B, int q_len, int Hq, int Hkv, int D, int bt, int max_blocks,
                     int window_left, int num_sms, int ctas_per_sm, int chunk_pages_override,
-                    int force_hb, fpd_plan* plan, bool fp4 = false) {
+                    fpd_plan* plan, bool fp4 = false) {
   if (!plan) return FPD_ERR_INVALID_ARG;
   fpd_status st = validate_shape(B, Hq, Hkv, D, bt, max_blocks, q_len);
   if (st != FPD_OK) return st;
   if (num_sms <= 0 || ctas_per_sm <= 0 || chunk_pages_override < 0) return FPD_ERR_INVALID_ARG;
-  if (force_hb != 0 && force_hb != 1 && force_hb != 4) return FPD_ERR_INVALID_ARG;
-  if (force_hb == 4 && heads_per_stage(Hkv) != 4) return FPD_ERR_INVALID_ARG;
   const int64_t slots = (int64_t)num_sms * ctas_per_sm;
-  int HB = force_hb ? force_hb : heads_per_stage(Hkv);
-  plan_shape(B, q_len, Hq, Hkv, D, bt, max_blocks, window_left, slots, chunk_pages_override, HB,
-             plan, fp4);
-  if (force_hb == 0 && HB == 4 && chunk_pages_override == 0 &&
-      (int64_t)(B > 0 ? B : 1) * (Hkv / 4) * plan->q_chunks * plan->max_splits < slots)
-    plan_shape(B, q_len, Hq, Hkv, D, bt, max_blocks, window_left, slots, 0, 1, plan, fp4);
+  const int HB = heads_per_stage(Hkv);
+  plan_shape(B, q_len, Hq, Hkv, D, bt, max_blocks, window_left, num_sms, slots,
+             chunk_pages_override, HB, plan, fp4);
   return FPD_OK;
 }
 
@@ -515,20 +536,14 @@ fpd_status plan_device(int B, int q_len, int Hq, int Hkv, int D, int bt, int max
   fpd_status st = validate_shape(B, Hq, Hkv, D, bt, max_blocks, q_len);
   if (st != FPD_OK) return st;
   const int cols = q_per_item(q_len, Hq / Hkv) * (Hq / Hkv);   // MMA columns of a work item
-  int HB = heads_per_stage(Hkv), force_hb = 0;
-  for (;;) {
-    int sms = 0, occ = 0;
-    if (!device_occupancy(D, n_tiles(cols), HB, q_len > 1, fp4,
-                          smem_bytes_for(D, cols, HB, B, fp4), &sms, &occ))
-      return FPD_ERR_CUDA;
-    if (occ <= 0) return FPD_ERR_UNSUPPORTED;  // the batch's shared-memory table does not fit
-    st = plan_for(B, q_len, Hq, Hkv, D, bt, max_blocks, window_left, sms, occ,
-                  chunk_pages_override, force_hb, plan, fp4);
-    // the planner fell back to one head per stage: plan again with that
-    // kernel's own occupancy
-    if (st != FPD_OK || plan->heads_per_stage == HB) return st;
-    HB = force_hb = plan->heads_per_stage;
-  }
+  const int HB = heads_per_stage(Hkv);
+  int sms = 0, occ = 0;
+  if (!device_occupancy(D, n_tiles(cols), HB, q_len > 1, fp4, smem_bytes_for(D, cols, HB, B, fp4),
+                        &sms, &occ))
+    return FPD_ERR_CUDA;
+  if (occ <= 0) return FPD_ERR_UNSUPPORTED;  // the batch's shared-memory table does not fit
+  return plan_for(B, q_len, Hq, Hkv, D, bt, max_blocks, window_left, sms, occ,
+                  chunk_pages_override, plan, fp4);
 }
 
 }  // namespace
@@ -552,7 +567,7 @@ fpd_status fp8_paged_decode_make_plan(int B, int Hq, int Hkv, int D, int bt, int
                                       int window_left, int num_sms, int ctas_per_sm,
                                       int chunk_pages_override, fpd_plan* plan) {
   return plan_for(B, 1, Hq, Hkv, D, bt, max_blocks, window_left, num_sms, ctas_per_sm,
-                  chunk_pages_override, 0, plan);
+                  chunk_pages_override, plan);
 }
 
 fpd_status fp8_paged_decode_make_plan_qlen(int B, int q_len, int Hq, int Hkv, int D, int bt,
@@ -560,7 +575,7 @@ fpd_status fp8_paged_decode_make_plan_qlen(int B, int q_len, int Hq, int Hkv, in
                                            int ctas_per_sm, int chunk_pages_override,
                                            fpd_plan* plan) {
   return plan_for(B, q_len, Hq, Hkv, D, bt, max_blocks, window_left, num_sms, ctas_per_sm,
-                  chunk_pages_override, 0, plan);
+                  chunk_pages_override, plan);
 }
 
 fpd_status fp8_paged_decode_plan(int B, int Hq, int Hkv, int D, int bt, int max_blocks,
@@ -760,6 +775,7 @@ static fpd_status attention_impl(const fpd_decode_args& a, void* workspace,
   p.q_f16 = a.q_dtype == FPD_Q_F16;
   p.kv_hnd = hnd;
   p.out_f32 = f32_out ? static_cast<float*>(a.out) : nullptr;
+  p.adapt_chunk = plan.adapt_chunk_pages;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (ev0 && cudaEventRecord(static_cast<cudaEvent_t>(ev0), s) != cudaSuccess) return FPD_ERR_CUDA;
@@ -796,7 +812,7 @@ static fpd_status attention_impl(const fpd_decode_args& a, void* workspace,
     c.bt = bt;
     c.max_blocks = max_blocks;
     c.window_left = window_left;
-    c.chunk_pages = plan.chunk_pages;
+    c.chunk_word = p.sched + 2;
     c.max_splits = plan.max_splits;
     // enough warps per row that none merges more than one batch of partials
     // (up to 32 warps), and 8 warps per CTA at least

@@ -12,9 +12,10 @@
 //
 // One warp per row; each lane owns D / 32 consecutive elements and reads
 // them from every rank with one 8- or 16-byte load, so a row's R partial rows
-// are read once, coalesced.  The op reads R * (D + 1) * 4 bytes and writes
-// 2 * D (+ 4) bytes per row: HBM-bound, and for decode-sized calls (a few
-// hundred rows) a single wave of latency.
+// are read once, coalesced, eight ranks per round trip to memory.  The op
+// reads R * (D + 1) * 4 bytes and writes 2 * D (+ 4) bytes per row: HBM-bound
+// in principle, and for decode-sized calls (a few hundred rows, partials that
+// the exchange has just written to L2) one or two round trips of latency.
 #pragma once
 
 #include <cstdint>
@@ -40,49 +41,63 @@ struct CpMergeParams {
 template <int D>
 __global__ void __launch_bounds__(kCpMergeWarps * 32) fpd_cp_merge_kernel(const CpMergeParams p) {
   constexpr int PER = D / 32;
+  constexpr int kBatch = 8;   // ranks whose partials are loaded together
   constexpr float kL2e = 1.4426950408889634f;
   const int lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * kCpMergeWarps + (threadIdx.x >> 5);
   if (row >= p.rows) return;
   const float* lse_r = p.partials + p.rows * D + row;         // rank r: lse_r[r * block]
   const float* o_r = p.partials + row * D + lane * PER;       // rank r: o_r[r * block + i]
-
-  // the largest partial lse (lanes take ranks lane, lane + 32, ...)
-  float mx = -INFINITY;
-  for (int r = lane; r < p.R; r += 32) mx = fmaxf(mx, lse_r[(int64_t)r * p.block]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   const int hq = (int)(row % p.Hq);
   const float sg = p.sinks ? p.sinks[hq] : -INFINITY;
-  const float M = fmaxf(mx, sg);
 
+  // Running maximum m, sum z and weighted sum acc over the ranks; each batch
+  // of kBatch ranks costs one round trip to memory (all of them for R <= 8).
+  float m = -INFINITY, z = 0.f;
   float acc[PER];
 #pragma unroll
   for (int i = 0; i < PER; ++i) acc[i] = 0.f;
-  float Z = 0.f;
-  if (mx != -INFINITY) {
-#pragma unroll 4
-    for (int r = 0; r < p.R; ++r) {
-      const int64_t off = (int64_t)r * p.block;
-      const float l = lse_r[off];   // the same address in every lane
-      float v[PER];
-      if constexpr (PER == 4) {
-        const float4 t = *reinterpret_cast<const float4*>(o_r + off);
-        v[0] = t.x, v[1] = t.y, v[2] = t.z, v[3] = t.w;
-      } else {
-        const float2 t = *reinterpret_cast<const float2*>(o_r + off);
-        v[0] = t.x, v[1] = t.y;
-      }
-      if (l == -INFINITY) continue;   // the rank holds no key of this row
-      const float w = fast_exp2((l - M) * kL2e);
-      Z += w;
+  for (int r0 = 0; r0 < p.R; r0 += kBatch) {
+    float lv[kBatch];
+    float x[kBatch][PER];
 #pragma unroll
-      for (int i = 0; i < PER; ++i) acc[i] = fmaf(w, v[i], acc[i]);
+    for (int u = 0; u < kBatch; ++u) {
+      lv[u] = -INFINITY;
+      if (r0 + u < p.R) {
+        const int64_t off = (int64_t)(r0 + u) * p.block;
+        lv[u] = lse_r[off];   // the same address in every lane
+        if constexpr (PER == 4) {
+          const float4 t = *reinterpret_cast<const float4*>(o_r + off);
+          x[u][0] = t.x, x[u][1] = t.y, x[u][2] = t.z, x[u][3] = t.w;
+        } else {
+          const float2 t = *reinterpret_cast<const float2*>(o_r + off);
+          x[u][0] = t.x, x[u][1] = t.y;
+        }
+      }
+    }
+    float mb = m;
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) mb = fmaxf(mb, lv[u]);
+    if (mb == -INFINITY) continue;   // no rank of this batch holds a key of the row
+    const float sc = m == -INFINITY ? 0.f : fast_exp2((m - mb) * kL2e);
+    z *= sc;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) acc[i] *= sc;
+    m = mb;
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      if (lv[u] == -INFINITY) continue;   // a rank without a key of this row (or past R)
+      const float w = fast_exp2((lv[u] - m) * kL2e);
+      z += w;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) acc[i] = fmaf(w, x[u][i], acc[i]);
     }
   }
-  if (p.sinks && sg != -INFINITY) Z += fast_exp2((sg - M) * kL2e);
+  const float M = fmaxf(m, sg);
+  const float rr = m == -INFINITY ? 0.f : fast_exp2((m - M) * kL2e);
+  const float Z = z * rr + (sg == -INFINITY ? 0.f : fast_exp2((sg - M) * kL2e));
   const bool any = Z > 0.f;   // false: no rank and no sink covers the row
-  const float inv = any ? 1.0f / Z : 0.f;
+  const float inv = any ? rr / Z : 0.f;
   const int64_t tok = row / p.Hq;
   __nv_bfloat16* dst = p.out + tok * p.out_tok_stride + (int64_t)hq * D + lane * PER;
 #pragma unroll

@@ -93,7 +93,8 @@ struct DecodeParams {
   float* part_o;        // [B, Hq, max_splits, D]
   float* part_lse;      // [B, Hq, max_splits]   (log2 domain)
   uint32_t* status;     // workspace word 0: sticky FPD_DEVERR_* bits
-  uint32_t* sched;      // workspace words 1, 2: next work item, CTAs finished
+  uint32_t* sched;      // workspace words 1, 2: next work item, CTAs finished;
+                        // word 3: the split size the call used (for the combine)
   int B, Hq, Hkv, g, bt, max_blocks, num_blocks, window_left;
   int chunk_pages, max_splits, stages, hdr_slots;
   int q_len;            // query tokens per sequence
@@ -113,6 +114,9 @@ struct DecodeParams {
   // f32 output (same element strides as `out`): every row, one split or
   // several, leaves its partial in the workspace and the combine writes it
   float* out_f32;
+  // > 0: the split size to take instead of chunk_pages when the sequences
+  // are of about equal length and chunk_pages gives more items than the grid
+  int adapt_chunk;
 };
 
 // Bytes of one header slot: the header, then the item's query rows (HB KV
@@ -211,11 +215,51 @@ __device__ __forceinline__ SeqRange seq_range(int L_raw, int q_len, int bt, int 
   return r;
 }
 
-// Work groups (one per split; one for an empty sequence) of a sequence.
-__device__ __forceinline__ int groups_of(int L_raw, int q_len, const DecodeParams& p) {
-  const SeqRange r =
-      seq_range(L_raw, q_len, p.bt, p.max_blocks, p.window_left, p.chunk_pages, nullptr);
+// Work groups (one per split; one for an empty sequence) of a sequence at
+// split size `chunk` pages.
+__device__ __forceinline__ int groups_of(int L_raw, int q_len, const DecodeParams& p, int chunk) {
+  const SeqRange r = seq_range(L_raw, q_len, p.bt, p.max_blocks, p.window_left, chunk, nullptr);
   return r.n_splits > 0 ? r.n_splits : 1;
+}
+
+// Prefix over the sequences of their work groups at split size `chunk`
+// (every CTA builds its own: prefix[b] groups come before sequence b).  Every
+// thread of the block takes part; returns the most groups of one sequence.
+// red: 2 * kThreads / 32 ints of shared memory.
+__device__ __forceinline__ int build_prefix(const DecodeParams& p, int q_len, int chunk,
+                                            int* prefix, int* red) {
+  constexpr int kWarps = kThreads / 32;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int per = (p.B + kThreads - 1) / kThreads;
+  const int b0 = min(p.B, tid * per), b1 = min(p.B, b0 + per);
+  int sum = 0, mx = 0;
+  for (int b = b0; b < b1; ++b) {
+    const int g = groups_of(__ldg(p.seq_lens + b), q_len, p, chunk);
+    sum += g;
+    mx = max(mx, g);
+  }
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  __syncthreads();   // an earlier pass has finished reading red
+  if (lane == 31) red[warp] = incl;
+  if (lane == 0) red[kWarps + warp] = mx;
+  __syncthreads();
+  int run = incl - sum;
+  for (int w = 0; w < warp; ++w) run += red[w];
+  if (tid == 0) prefix[0] = 0;
+  for (int b = b0; b < b1; ++b) {
+    run += groups_of(__ldg(p.seq_lens + b), q_len, p, chunk);
+    prefix[b + 1] = run;
+  }
+  int most = 0;
+  for (int w = 0; w < kWarps; ++w) most = max(most, red[kWarps + w]);
+  __syncthreads();   // the prefix is complete
+  return most;
 }
 
 // Byte offset inside a 1024-byte-aligned tile written by TMA with 128-byte
@@ -743,7 +787,7 @@ __device__ __forceinline__ void producer_loop(const CUtensorMap* kmap, const CUt
                                               const CUtensorMap* ksmap, const CUtensorMap* vsmap,
                                               const DecodeParams& p, uint8_t* smem,
                                               const SmemLayout& L, const int* prefix,
-                                              int total_items, int hslot_bytes,
+                                              int chunk, int total_items, int hslot_bytes,
                                               uint64_t* full_bar, uint64_t* empty_bar,
                                               uint64_t* hdr_full, uint64_t* hdr_empty, int lane) {
   constexpr int kTileBytes = kTileTokens * D;
@@ -810,12 +854,11 @@ __device__ __forceinline__ void producer_loop(const CUtensorMap* kmap, const CUt
     const int b = lo;
     const int split = group - prefix[b];
     const SeqRange R = seq_range(__ldg(p.seq_lens + b), QL, p.bt, p.max_blocks,
-                                 p.window_left,
-                                 p.chunk_pages, lane == 0 ? p.status : nullptr);
+                                 p.window_left, chunk, lane == 0 ? p.status : nullptr);
     int pb = 0, pe = 0, tok_lo = 0, tok_hi = 0, t0 = 0, n_st = 0;
     if (R.n_splits > 0) {
-      pb = R.first_page + split * p.chunk_pages;
-      pe = min(pb + p.chunk_pages, R.end_page);
+      pb = R.first_page + split * chunk;
+      pe = min(pb + chunk, R.end_page);
       tok_lo = max(R.start, pb * p.bt);
       tok_hi = min(R.L, pe * p.bt);
       if (HB == 1) {   // whole pages, pps per stage
@@ -1010,7 +1053,7 @@ __device__ __forceinline__ void split_body(const CUtensorMap* kmap, const CUtens
                                            const CUtensorMap* ksmap, const CUtensorMap* vsmap,
                                            const DecodeParams& p) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ int warp_tot[kThreads / 32];
+  __shared__ int warp_tot[2 * (kThreads / 32)];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   constexpr int kTileBytes = kTileTokens * D;
@@ -1039,48 +1082,45 @@ __device__ __forceinline__ void split_body(const CUtensorMap* kmap, const CUtens
   // is read before that kernel has completed and its writes are visible.
   pdl_wait_primary();
 
-  // ---- prefix over sequences of their work groups (every CTA builds its own)
+  if (tid == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], kConsumerWarps);
+    }
+    for (int s = 0; s < kMaxHdrSlots; ++s) {
+      mbar_init(&hdr_full[s], 1);
+      mbar_init(&hdr_empty[s], kConsumerWarps);
+    }
+    mbar_init(cbar, kConsumerWarps);
+    fence_mbarrier_init();   // visible to the block after build_prefix's barriers
+  }
+
+  // ---- the split size and the prefix over sequences of their work groups.
+  // The plan may offer a larger split size for calls of a few rounds of
+  // items: taken when the sequences are of about equal length (the longest
+  // one's groups times B within 4/3 of all groups), since then its items, one
+  // round of about two per SM, fill every SM alike; otherwise the plan's size
+  // runs over the grid, sized for the larger items.  Every CTA reaches the
+  // same choice from the same lengths.
+  const int G = (p.Hkv / HB) * (MQ ? p.q_chunks : 1);   // items per work group
+  int chunk = p.chunk_pages;
   {
-    const int per = (p.B + kThreads - 1) / kThreads;
-    const int b0 = min(p.B, tid * per), b1 = min(p.B, b0 + per);
-    int sum = 0;
-    for (int b = b0; b < b1; ++b) sum += groups_of(__ldg(p.seq_lens + b), QL, p);
-    int incl = sum;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
+    const int most = build_prefix(p, QL, chunk, prefix, warp_tot);
+    const int64_t groups = prefix[p.B];
+    if (p.adapt_chunk > 0 && groups * G > (int64_t)gridDim.x &&
+        4 * groups >= 3 * (int64_t)p.B * most) {
+      chunk = p.adapt_chunk;
+      build_prefix(p, QL, chunk, prefix, warp_tot);
     }
-    if (lane == 31) warp_tot[warp] = incl;
-    if (tid == 0) {
-      for (int s = 0; s < stages; ++s) {
-        mbar_init(&full_bar[s], 1);
-        mbar_init(&empty_bar[s], kConsumerWarps);
-      }
-      for (int s = 0; s < kMaxHdrSlots; ++s) {
-        mbar_init(&hdr_full[s], 1);
-        mbar_init(&hdr_empty[s], kConsumerWarps);
-      }
-      mbar_init(cbar, kConsumerWarps);
-      fence_mbarrier_init();
-    }
-    __syncthreads();
-    int base = 0;
-    for (int w = 0; w < warp; ++w) base += warp_tot[w];
-    int run = base + incl - sum;
-    if (tid == 0) prefix[0] = 0;
-    for (int b = b0; b < b1; ++b) {
-      run += groups_of(__ldg(p.seq_lens + b), QL, p);
-      prefix[b + 1] = run;
-    }
-    __syncthreads();
+    if (blockIdx.x == 0 && tid == 0) p.sched[2] = (uint32_t)chunk;
   }
   const int total_items = prefix[p.B] * (p.Hkv / HB) * (MQ ? p.q_chunks : 1);
   pdl_launch_dependents();   // the combine kernel may be scheduled from now on
 
   if (warp == kConsumerWarps) {
-    producer_loop<D, HB, MQ, FP4>(kmap, vmap, ksmap, vsmap, p, smem, L, prefix, total_items,
-                                  hslot_bytes, full_bar, empty_bar, hdr_full, hdr_empty, lane);
+    producer_loop<D, HB, MQ, FP4>(kmap, vmap, ksmap, vsmap, p, smem, L, prefix, chunk,
+                                  total_items, hslot_bytes, full_bar, empty_bar, hdr_full,
+                                  hdr_empty, lane);
     return;
   }
 
@@ -1321,7 +1361,8 @@ struct CombineParams {
   __nv_bfloat16* out;
   float* out_f32;     // non-null: f32 output, and every row is merged here
   float* lse;
-  int B, q_len, Hq, bt, max_blocks, window_left, chunk_pages, max_splits;
+  int B, q_len, Hq, bt, max_blocks, window_left, max_splits;
+  const uint32_t* chunk_word;   // the split size the split kernel used (workspace word 3)
   int wpr;            // warps per row: 1, 2, 4, 8, 16 or 32
   int rows_per_cta;   // rows per CTA (wpr * rows_per_cta <= 32)
   float v_scale;
@@ -1378,6 +1419,7 @@ __global__ void __launch_bounds__(kCombineMaxThreads) fpd_combine_kernel(const C
 
   // ---- one round of loads: the sequence length, v_scale and this warp's first batch
   const int L_raw = in_range ? p.seq_lens[row / (QL * p.Hq)] : 0;
+  const int chunk = (int)*p.chunk_word;
   const float v_scale = p.v_scale_dev ? *p.v_scale_dev : p.v_scale;
   float lv[kCombineBatch];
   float x[kCombineBatch][PER];
@@ -1399,7 +1441,7 @@ __global__ void __launch_bounds__(kCombineMaxThreads) fpd_combine_kernel(const C
     }
   }
   const int ns =
-      seq_range(L_raw, QL, p.bt, p.max_blocks, p.window_left, p.chunk_pages, nullptr)
+      seq_range(L_raw, QL, p.bt, p.max_blocks, p.window_left, chunk, nullptr)
           .n_splits;
   // rows with one split were written by the split kernel, unless the output is f32
   const bool active = in_range && (ns > 1 || p.out_f32);

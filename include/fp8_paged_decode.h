@@ -75,6 +75,9 @@ typedef struct {
     size_t workspace_bytes; /* bytes this plan needs */
     int q_per_item;         /* query positions per work item (1 with one query per sequence) */
     int q_chunks;           /* work items per sequence, KV head group and split: ceil(q_len / q_per_item) */
+    int adapt_chunk_pages;  /* 0, or the larger split size the kernel takes instead of chunk_pages
+                               when the sequences are of about equal length (the grid is then
+                               sized for its items); max_splits and the workspace follow chunk_pages */
 } fpd_plan;
 
 /*
@@ -87,8 +90,8 @@ typedef struct {
 /*
  * Host-only planner (no CUDA call): the split plan for a shape on a device with
  * `num_sms` SMs of which `ctas_per_sm` CTAs of the split kernel fit per SM.
- * chunk_pages_override > 0 forces the pages per split (with one KV head per
- * stage, rounded up to whole 64-token stages); 0 lets the heuristic choose.
+ * chunk_pages_override > 0 forces the pages per split (rounded up to whole
+ * 64-token stages when a stage holds one KV head); 0 lets the heuristic choose.
  * Returns FPD_OK or the validation error for the shape.
  */
 fpd_status fp8_paged_decode_make_plan(int B, int Hq, int Hkv, int D, int block_tokens,

@@ -87,11 +87,11 @@ def test_planner_header_slots():
 
 def test_planner_window_caps_splits():
     # a 129-token window spans at most 10 pages: one split.  64 sequences x 2
-    # four-head groups would leave CTA slots idle, so the planner falls back to
-    # one head per stage (64 x 8 work items)
+    # four-head groups leave CTA slots idle, and the planner keeps four heads
+    # per stage all the same (128 work items, no combine)
     p = plan(B=64, Hq=64, Hkv=8, D=64, block_tokens=16, max_blocks=1024, window_left=128)
-    assert p["heads_per_stage"] == 1 and p["max_splits"] == 1 and p["workspace_bytes"] == 256
-    assert p["ctas"] == 296
+    assert p["heads_per_stage"] == 4 and p["max_splits"] == 1 and p["workspace_bytes"] == 256
+    assert p["ctas"] == 128
     # with enough sequences the four-head shape fills the machine by itself
     p4 = plan(B=512, Hq=64, Hkv=8, D=64, block_tokens=16, max_blocks=1024, window_left=128)
     assert p4["heads_per_stage"] == 4 and p4["max_splits"] == 1
