@@ -260,3 +260,36 @@ def test_planner_single_split_for_tiny_calls():
     # overriding the split size still wins
     assert plan(B=2, Hq=8, Hkv=2, block_tokens=16, max_blocks=19,
                 chunk_pages_override=4)["max_splits"] == 5
+
+
+def test_planner_underfilled_calls_split_finer():
+    """A call whose minimum-size items cannot fill the machine splits down to
+    items of about 48 tokens (two items per SM at most); one that needs no
+    split keeps a single one, so no combine kernel runs."""
+    p = plan(B=1, max_blocks=256, ctas_per_sm=3)            # one 4096-token sequence
+    assert p["chunk_pages"] == 3 and p["adapt_chunk_pages"] == 0
+    assert p["max_splits"] == 86 and p["ctas"] == 2 * 86    # two four-head groups
+    p = plan(B=1, block_tokens=64, max_blocks=64, ctas_per_sm=3)
+    assert p["chunk_pages"] == 1                             # 64-token pages: one page
+    p = plan(B=64, Hq=64, Hkv=8, D=64, max_blocks=1024, window_left=128, ctas_per_sm=3)
+    assert p["max_splits"] == 1 and p["ctas"] == 128
+
+
+def test_planner_offers_one_round_split_size():
+    """Between one and 2.5 rounds of minimum-size items: the plan keeps the
+    minimum split (max_splits, workspace) and offers a larger one for one round
+    of about two items per SM, with the grid sized for it."""
+    p = plan(B=4, block_tokens=64, max_blocks=256, ctas_per_sm=3)   # 4 x 16384 tokens
+    assert p["chunk_pages"] == 4 and p["max_splits"] == 64        # 512 items: 1.15 rounds
+    assert p["adapt_chunk_pages"] == 7 and p["ctas"] == 8 * 37    # 296 items
+    # one KV head per stage: whole 64-token stages (4 pages)
+    p = plan(B=8, Hq=8, Hkv=2, max_blocks=1024, ctas_per_sm=3)
+    assert p["heads_per_stage"] == 1 and p["adapt_chunk_pages"] == 56
+    assert p["ctas"] == 16 * 19
+    # many rounds (Llama-3-8B-shaped, long context): the queue balances them
+    for kw in (dict(), dict(B=4, block_tokens=64, max_blocks=2048)):
+        p = plan(ctas_per_sm=3, **kw)
+        assert p["adapt_chunk_pages"] == 0 and p["ctas"] == 444
+    # a forced split size is used as given
+    p = plan(B=4, block_tokens=64, max_blocks=256, ctas_per_sm=3, chunk_pages_override=4)
+    assert p["adapt_chunk_pages"] == 0 and p["ctas"] == 444

@@ -37,9 +37,7 @@ GRID = list(itertools.product([64, 128], [1, 2, 4, 8, 16], [16, 32, 64], [2, 4])
 @pytest.mark.parametrize("D,g,bt,Hkv", GRID,
                          ids=[f"D{d}-g{g}-bt{b}-kv{h}" for d, g, b, h in GRID])
 def test_shape_grid(D, g, bt, Hkv):
-    """Hkv = 2: one KV head per stage.  Hkv = 4: four heads per stage whenever
-    the split size is forced (the planner's own choice for so few sequences is
-    one head per stage)."""
+    """Hkv = 2: one KV head per stage.  Hkv = 4: four heads per stage."""
     lens = [1, bt - 1, bt, bt + 1, 3 * bt + 5, 700]
     wl = W.make_custom(B=len(lens), Hq=g * Hkv, Hkv=Hkv, D=D, block_tokens=bt, seq_lens=lens,
                        seed=100 + D + g + bt + Hkv, sm_scale=1.0 / np.sqrt(D))
