@@ -224,8 +224,10 @@ __device__ __forceinline__ int groups_of(int L_raw, int q_len, const DecodeParam
 
 // Prefix over the sequences of their work groups at split size `chunk`
 // (every CTA builds its own: prefix[b] groups come before sequence b).  Every
-// thread of the block takes part; returns the most groups of one sequence.
+// thread of the block takes part.  MOST: also return the most groups of one
+// sequence.  AGAIN: an earlier pass may still be reading `red`.
 // red: 2 * kThreads / 32 ints of shared memory.
+template <bool MOST, bool AGAIN>
 __device__ __forceinline__ int build_prefix(const DecodeParams& p, int q_len, int chunk,
                                             int* prefix, int* red) {
   constexpr int kWarps = kThreads / 32;
@@ -236,18 +238,18 @@ __device__ __forceinline__ int build_prefix(const DecodeParams& p, int q_len, in
   for (int b = b0; b < b1; ++b) {
     const int g = groups_of(__ldg(p.seq_lens + b), q_len, p, chunk);
     sum += g;
-    mx = max(mx, g);
+    if (MOST) mx = max(mx, g);
   }
   int incl = sum;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const int v = __shfl_up_sync(0xffffffffu, incl, o);
     if (lane >= o) incl += v;
-    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (MOST) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   }
-  __syncthreads();   // an earlier pass has finished reading red
+  if (AGAIN) __syncthreads();
   if (lane == 31) red[warp] = incl;
-  if (lane == 0) red[kWarps + warp] = mx;
+  if (MOST && lane == 0) red[kWarps + warp] = mx;
   __syncthreads();
   int run = incl - sum;
   for (int w = 0; w < warp; ++w) run += red[w];
@@ -257,7 +259,8 @@ __device__ __forceinline__ int build_prefix(const DecodeParams& p, int q_len, in
     prefix[b + 1] = run;
   }
   int most = 0;
-  for (int w = 0; w < kWarps; ++w) most = max(most, red[kWarps + w]);
+  if (MOST)
+    for (int w = 0; w < kWarps; ++w) most = max(most, red[kWarps + w]);
   __syncthreads();   // the prefix is complete
   return most;
 }
@@ -1104,16 +1107,17 @@ __device__ __forceinline__ void split_body(const CUtensorMap* kmap, const CUtens
   // same choice from the same lengths.
   const int G = (p.Hkv / HB) * (MQ ? p.q_chunks : 1);   // items per work group
   int chunk = p.chunk_pages;
-  {
-    const int most = build_prefix(p, QL, chunk, prefix, warp_tot);
+  if (p.adapt_chunk > 0) {
+    const int most = build_prefix<true, false>(p, QL, chunk, prefix, warp_tot);
     const int64_t groups = prefix[p.B];
-    if (p.adapt_chunk > 0 && groups * G > (int64_t)gridDim.x &&
-        4 * groups >= 3 * (int64_t)p.B * most) {
+    if (groups * G > (int64_t)gridDim.x && 4 * groups >= 3 * (int64_t)p.B * most) {
       chunk = p.adapt_chunk;
-      build_prefix(p, QL, chunk, prefix, warp_tot);
+      build_prefix<false, true>(p, QL, chunk, prefix, warp_tot);
     }
-    if (blockIdx.x == 0 && tid == 0) p.sched[2] = (uint32_t)chunk;
+  } else {
+    build_prefix<false, false>(p, QL, chunk, prefix, warp_tot);
   }
+  if (blockIdx.x == 0 && tid == 0) p.sched[2] = (uint32_t)chunk;
   const int total_items = prefix[p.B] * (p.Hkv / HB) * (MQ ? p.q_chunks : 1);
   pdl_launch_dependents();   // the combine kernel may be scheduled from now on
 
