@@ -32,6 +32,7 @@ from __future__ import annotations
 
 import argparse
 import ctypes
+import ctypes.util
 import hashlib
 import json
 import math
@@ -115,6 +116,31 @@ def measured_peaks():
 # valid only for this exact code and, per workload, for the launch plan it
 # records (checked in ncu_traffic).
 KERNEL_SOURCES = ("fpd_kernels.cuh", "fpd_ptx.cuh")
+
+
+def cudart():
+    """The CUDA runtime library that torch loads (for raw async copies and event
+    calls from the host loop)."""
+    import torch
+    cands = [os.path.join(os.path.dirname(torch.__file__), "..", "nvidia", "cuda_runtime", "lib",
+                          "libcudart.so.12")]
+    found = ctypes.util.find_library("cudart")
+    if found:
+        cands.append(found)
+    for c in cands:
+        if os.path.exists(c) or not os.path.isabs(c):
+            try:
+                rt = ctypes.CDLL(c)
+                break
+            except OSError:
+                continue
+    else:
+        raise RuntimeError("no CUDA runtime library found for the end-to-end loop")
+    vp = ctypes.c_void_p
+    rt.cudaMemcpyAsync.argtypes = [vp, vp, ctypes.c_size_t, ctypes.c_int, vp]
+    rt.cudaEventRecord.argtypes = [vp, vp]
+    rt.cudaStreamWaitEvent.argtypes = [vp, vp, ctypes.c_uint]
+    return rt
 
 
 def kernel_source_hash():
@@ -390,10 +416,12 @@ def run_native(args):
     sh = ctypes.c_void_p(stream.cuda_stream)
     vp = ctypes.c_void_p
 
-    def descriptor(i):
-        """The call on replica i, as the C ABI's descriptor."""
+    def descriptor(i, io=None):
+        """The call on replica i, as the C ABI's descriptor; io: other device
+        buffers for (q, table, lens, sinks, out, lse)."""
+        q_, table_, lens_, sinks_, out_, lse_ = io or (q, table, lens, sinks, out, lse)
         a = fpd.fpd_decode_args()
-        a.q, a.q_dtype = q.data_ptr(), fpd.FPD_Q_BF16
+        a.q, a.q_dtype = q_.data_ptr(), fpd.FPD_Q_BF16
         if nvfp4:
             lay = fpd.nvfp4_page_layout(wl.Hkv, wl.block_tokens, wl.D)
             base = kc[i].data_ptr()
@@ -404,13 +432,13 @@ def run_native(args):
         else:
             a.k_cache, a.v_cache = kc[i].data_ptr(), vc[i].data_ptr()
             a.kv_format, a.kv_layout = fpd.FPD_KV_E4M3, fpd.FPD_KV_NHD
-        a.block_table, a.seq_lens = table.data_ptr(), lens.data_ptr()
+        a.block_table, a.seq_lens = table_.data_ptr(), lens_.data_ptr()
         a.B, a.q_len, a.Hq, a.Hkv, a.D = wl.B, wl.q_len, wl.Hq, wl.Hkv, wl.D
         a.num_blocks, a.block_tokens, a.max_blocks = wl.num_blocks, wl.block_tokens, wl.max_blocks
         a.k_scale, a.v_scale, a.sm_scale = wl.k_scale, wl.v_scale, wl.sm_scale
         a.window_left = wl.window_left
-        a.sinks = sinks.data_ptr() if sinks is not None else None
-        a.out, a.lse = out.data_ptr(), lse.data_ptr()
+        a.sinks = sinks_.data_ptr() if sinks_ is not None else None
+        a.out, a.lse = out_.data_ptr(), lse_.data_ptr()
         a.chunk_pages_override = args.chunk_pages
         return a
 
@@ -556,45 +584,135 @@ def run_native(args):
         del cg
         assert fpd.fp8_paged_decode_check_status(wsp, clear=True) == 0
 
-    # end to end through the C ABI: pinned host inputs in, results out, every step
+    # End to end through the C ABI: every step copies its inputs from pinned host
+    # memory and reads its result back.  Pipelined as a serving loop would run
+    # it: two sets of device inputs and outputs, the host-to-device copies on
+    # one side stream and the reads on another, so that step i's copies
+    # overlap the kernels of steps i - 1 and i + 1.  The serial form (copies
+    # and kernels one after another on one stream) is timed too.
     e2e = None
     if not args.no_e2e:
-        hq = torch.from_numpy(wl.q.view(np.int16)).view(torch.bfloat16).pin_memory()
-        htab = torch.from_numpy(wl.block_table).pin_memory()
-        hlen = torch.from_numpy(wl.seq_lens).pin_memory()
-        hsink = None if wl.sinks is None else torch.from_numpy(wl.sinks).pin_memory()
-        hout = torch.empty(lead + (wl.Hq, wl.D), dtype=torch.bfloat16).pin_memory()
-        hlse = torch.empty(lead + (wl.Hq,), dtype=torch.float32).pin_memory()
-        h2d = hq.numel() * 2 + htab.numel() * 4 + hlen.numel() * 4 + (
-            hsink.numel() * 4 if hsink is not None else 0)
-        d2h = hout.numel() * 2 + hlse.numel() * 4
+        # a step's inputs (q, block table, lengths, sinks) sit in one buffer and
+        # its results (out, lse) in another, on both sides: one copy each way
+        def packed(tensors, pinned):
+            offs, total = [], 0
+            for t in tensors:
+                offs.append(total)
+                total += (t.numel() * t.element_size() + 255) // 256 * 256
+            buf = (torch.empty(total, dtype=torch.uint8).pin_memory() if pinned else
+                   torch.empty(total, dtype=torch.uint8, device=dev))
+            views = [buf[o:o + t.numel() * t.element_size()].view(t.dtype).view(t.shape)
+                     for o, t in zip(offs, tensors)]
+            return buf, views
+        src = [torch.from_numpy(wl.q.view(np.int16)).view(torch.bfloat16),
+               torch.from_numpy(wl.block_table), torch.from_numpy(wl.seq_lens)]
+        if wl.sinks is not None:
+            src.append(torch.from_numpy(wl.sinks))
+        h_inbuf, h_inv = packed(src, True)
+        for v, t in zip(h_inv, src):
+            v.copy_(t)
+        res = [out, lse]
+        h_outbuf = [packed(res, True) for _ in range(2)]
+        d_in = [packed(src, False) for _ in range(2)]
+        d_out = [packed(res, False) for _ in range(2)]
+        h2d = h_inbuf.numel()
+        d2h = h_outbuf[0][0].numel()
+        io = []
+        for j in range(2):
+            v = d_in[j][1]
+            io.append((v[0], v[1], v[2], v[3] if wl.sinks is not None else None,
+                       d_out[j][1][0], d_out[j][1][1]))
+        edescs = [[descriptor(i, io[j]) for j in range(2)] for i in range(replicas)]
+        erefs = [[ctypes.byref(d) for d in row] for row in edescs]
+        # copies, event records and waits go straight to the CUDA runtime, so
+        # that the host side of a step costs a few microseconds
+        rt = cudart()
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        h_in, h_out = vp(s_in.cuda_stream), vp(s_out.cuda_stream)
+        evs = [[torch.cuda.Event() for _ in range(2)] for _ in range(3)]
+        for row in evs:   # every buffer starts free (this also creates the events)
+            for e in row:
+                e.record(stream)
+        torch.cuda.synchronize()
+        ev_in, ev_k, ev_out = [[vp(e.cuda_event) for e in row] for row in evs]
+
+        def copies(j):
+            return ([(vp(d_in[j][0].data_ptr()), vp(h_inbuf.data_ptr()), h2d)],
+                    [(vp(h_outbuf[j][0].data_ptr()), vp(d_out[j][0].data_ptr()), d2h)])
+        cps = [copies(0), copies(1)]
+        H2D, D2H = 1, 2
+
+        def e2e_step(i):   # returns the OR of the runtime's error codes
+            j = i % 2
+            ins, outs = cps[j]
+            err = rt.cudaStreamWaitEvent(h_in, ev_k[j], 0)   # step i - 2 has read these inputs
+            for d, h, n in ins:
+                err |= rt.cudaMemcpyAsync(d, h, n, H2D, h_in)
+            err |= rt.cudaEventRecord(ev_in[j], h_in)
+            err |= rt.cudaStreamWaitEvent(sh, ev_in[j], 0)
+            err |= rt.cudaStreamWaitEvent(sh, ev_out[j], 0)   # step i - 2's results have left
+            st = f_args(erefs[i % replicas][j], ws_ptr, ws_n, sh)
+            if st != 0:
+                raise RuntimeError(fpd.fp8_paged_decode_status_string(st))
+            err |= rt.cudaEventRecord(ev_k[j], sh)
+            err |= rt.cudaStreamWaitEvent(h_out, ev_k[j], 0)
+            for h, d, n in outs:
+                err |= rt.cudaMemcpyAsync(h, d, n, D2H, h_out)
+            return err | rt.cudaEventRecord(ev_out[j], h_out)
+
+        def serial_step(i):
+            ins, outs = cps[0]
+            err = 0
+            for d, h, n in ins:
+                err |= rt.cudaMemcpyAsync(d, h, n, H2D, sh)
+            st = f_args(erefs[i % replicas][0], ws_ptr, ws_n, sh)
+            if st != 0:
+                raise RuntimeError(fpd.fp8_paged_decode_status_string(st))
+            for h, d, n in outs:
+                err |= rt.cudaMemcpyAsync(h, d, n, D2H, sh)
+            return err
+
         Ke = K
         for i in range(min(args.warmup, 50)):
-            st = f_plain(i)
+            assert e2e_step(i) == 0, "CUDA runtime error in the end-to-end loop"
         torch.cuda.synchronize()
         barrier()
         s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s2.record(stream)
+        s_in.wait_event(s2)
+        err = 0
         for i in range(Ke):
-            q.copy_(hq, non_blocking=True)
-            table.copy_(htab, non_blocking=True)
-            lens.copy_(hlen, non_blocking=True)
-            if hsink is not None:
-                sinks.copy_(hsink, non_blocking=True)
-            st = f_plain(i)
-            if st != 0:
-                raise RuntimeError(fpd.fp8_paged_decode_status_string(st))
-            hout.copy_(out, non_blocking=True)
-            hlse.copy_(lse, non_blocking=True)
+            err |= e2e_step(i)
+        stream.wait_stream(s_out)
         e2.record(stream)
         torch.cuda.synchronize()
         barrier()
         te = max_over_ranks(s2.elapsed_time(e2), dev)
+        assert err == 0, "CUDA runtime error in the end-to-end loop"
+        # the last step's result must be what the device computed
+        last = (Ke - 1) % 2
+        assert torch.equal(h_outbuf[last][0], d_out[last][0].cpu())
+        # serial: copies and the call back to back on one stream
+        Ks = min(Ke, 2000)
+        s3, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s3.record(stream)
+        for i in range(Ks):
+            err |= serial_step(i)
+        e3.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ts = max_over_ranks(s3.elapsed_time(e3), dev)
+        assert err == 0, "CUDA runtime error in the end-to-end loop"
         e2e = {"value": whole_job_value(ws, kv_bytes, Ke, te), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": te / Ke,
-               "note": "q, block_table, seq_lens, sinks H2D from pinned host and out + lse D2H "
-                       "every step; the KV cache is resident device state"}
+               "serial": {"value": whole_job_value(ws, kv_bytes, Ks, ts),
+                          "ms_per_step": ts / Ks},
+               "note": "every step: q, block_table, seq_lens (and sinks) in one pinned host "
+                       "buffer copied to the device, out and lse read back in one copy; "
+                       "double-buffered on two side streams so that a step's copies overlap "
+                       "the neighbouring steps' kernels ('serial': all on one stream); the KV "
+                       "cache is resident device state"}
 
     bits = fpd.fp8_paged_decode_check_status(wsp)
     assert bits == 0, f"device status {bits}"
