@@ -69,6 +69,9 @@ def parse_args():
                     help="only run warm-up + K plain calls (for ncu launch lists and captures)")
     ap.add_argument("--json-out", default=None)
     ap.add_argument("--op", default="decode", choices=["decode", "cache_write", "cp"])
+    ap.add_argument("--cp-fused", action="store_true",
+                    help="--op cp: the exchange fused into the decode (peer-memory stores and "
+                         "flags) instead of an NCCL all-gather")
     ap.add_argument("--cp-ranks", type=int, default=8,
                     help="--op cp on one process: the context-parallel width whose rank "
                          "step is timed (under torchrun the world size is the width)")
@@ -873,7 +876,7 @@ def run_cp(args):
     each rank, max over ranks.  On one process the step of the rank with the
     most keys of an R-way partition is timed (its decode and the merge of R
     partials computed beforehand) and the exchange is not run.  L2 is evicted
-    (a 256 MiB read) before each timed step, outside the timed events."""
+    (a 1 GiB read) before each timed step, outside the timed events."""
     import numpy as np
     import torch
     import torch.distributed as dist
@@ -954,13 +957,61 @@ def run_cp(args):
         st |= lib.fp8_paged_decode_cp_merge(*merge_args)
         assert st == 0
 
-    # L2 is evicted by reading a 256 MiB buffer (a reduction), which leaves no
+    if args.cp_fused:
+        # the exchange fused into the decode: the rank's combine kernel stores
+        # its rows into every rank's gather buffer and raises its flag there;
+        # the merge waits for the R flags.  One process: the other ranks'
+        # slots are filled once, and their flags are raised (a fill, before
+        # the timed events) each step.
+        ex = cp.CpExchange(B, Hq, D) if ws > 1 else cp.CpExchange.local(R, B, Hq, D)
+        fused = []
+        for r in range(R if ws == 1 else 1):
+            rr = r if ws == 1 else rank
+            a = descriptor(*dev_shards[rr], partial)
+            a.out, a.lse = None, None
+            fused.append(a)
+        fstatus = torch.zeros(1, dtype=torch.int32, device=dev)
+        flags_me, gather_me = ex.flags(me), ex.gather(me)
+        fsh = ctypes.c_void_p(stream.cuda_stream)
+
+        ex.next_epoch()
+        for r, a in enumerate(fused):
+            (a.cp_gather, a.cp_flags, a.cp_ranks, a.cp_rank, a.cp_epoch,
+             a.cp_block_floats) = ex.publish_fields(r if ws == 1 else rank)
+        if ws == 1:
+            for a in fused:
+                assert f_dec(ctypes.byref(a), ws_ptr, ws_n, fsh) == 0
+        mine_f = fused[me] if ws == 1 else fused[0]
+        mine_f_ref = ctypes.byref(mine_f)
+        margs = [ctypes.c_void_p(gather_me.data_ptr()), R, blk, rows, Hq, D,
+                 ctypes.c_void_p(sinks.data_ptr()) if sinks is not None else None,
+                 ctypes.c_void_p(out.data_ptr()), 0, ctypes.c_void_p(lse.data_ptr()),
+                 ctypes.c_void_p(flags_me.data_ptr()), ctypes.c_uint32(0),
+                 ctypes.c_uint64(1_000_000_000), ctypes.c_void_p(fstatus.data_ptr()), fsh]
+        f_merge_wait = lib.fp8_paged_decode_cp_merge_wait
+
+        def pre_step():   # untimed: a new epoch; one process: every rank's flag raised
+            mine_f.cp_epoch = ex.next_epoch()
+            margs[11] = ctypes.c_uint32(ex.epoch)
+            if ws == 1:
+                flags_me.fill_(ex.epoch)
+
+        def step():
+            st = f_dec(mine_f_ref, ws_ptr, ws_n, fsh)
+            st |= f_merge_wait(*margs)
+            assert st == 0
+    else:
+        def pre_step():
+            pass
+
+    # L2 is evicted by reading a 1 GiB buffer (a reduction), which leaves no
     # dirty lines whose write-back would compete with the timed reads
-    flush_buf = torch.ones(256 * 2 ** 20, dtype=torch.uint8, device=dev)
+    flush_buf = torch.ones(1024 * 2 ** 20, dtype=torch.uint8, device=dev)   # the host stays ahead
     flush = lambda: torch.amax(flush_buf)
     K = max(1, min(args.steps, 2000))
     ev = lambda: torch.cuda.Event(enable_timing=True)
     for _ in range(args.warmup):
+        pre_step()
         step()
     torch.cuda.synchronize()
     if ws > 1:
@@ -973,6 +1024,7 @@ def run_cp(args):
     pairs = [(ev(), ev()) for _ in range(K)]
     for e0, e1 in pairs:
         flush()
+        pre_step()
         e0.record(stream)
         step()
         e1.record(stream)
@@ -988,6 +1040,28 @@ def run_cp(args):
         e0.record(stream)
         assert f_dec(mine_ref, ws_ptr, ws_n, sh) == 0
         e1.record(stream)
+    fused_alone = {}
+    if args.cp_fused:
+        assert int(fstatus.item()) == 0, "a rank's flag did not arrive"
+        # the publishing decode alone, then the waiting merge alone (flags set)
+        pub = [(ev(), ev()) for _ in range(min(K, 200))]
+        for e0, e1 in pub:
+            flush()
+            pre_step()
+            e0.record(stream)
+            assert f_dec(mine_f_ref, ws_ptr, ws_n, fsh) == 0
+            e1.record(stream)
+        mw = [(ev(), ev()) for _ in range(min(K, 200))]
+        for e0, e1 in mw:
+            flush()
+            e0.record(stream)
+            assert f_merge_wait(*margs) == 0
+            e1.record(stream)
+        torch.cuda.synchronize()
+        fused_alone = {
+            "publishing_decode_median_cold_l2": float(np.median([a.elapsed_time(b) for a, b in pub])) * 1e3,
+            "waiting_merge_median_cold_l2": float(np.median([a.elapsed_time(b) for a, b in mw])) * 1e3}
+        ex.close()
     # the merge alone: a CUDA graph of 100 launches, replayed 10 times
     side = torch.cuda.Stream(dev)
     side.wait_stream(stream)
@@ -1024,17 +1098,21 @@ def run_cp(args):
         "ms_per_step": ms, "us_per_step": ms * 1e3, "higher_is_better": True,
         "scaling": "strong", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "cp_ranks": R,
-        "exchange": ("nccl all_gather_into_tensor of the f32 partials" if ws > 1 else
+        "exchange": (("fused: the combine kernel stores the rows into every rank's gather "
+                      "buffer over peer memory and raises a flag; the merge waits for the flags"
+                      + ("" if ws > 1 else " (one GPU: the other ranks' slots and flags are "
+                         "set outside the timed step)")) if args.cp_fused else
+                     "nccl all_gather_into_tensor of the f32 partials" if ws > 1 else
                      "not run: one GPU; the timed step is one rank's decode and merge"),
         "us_alone": {"partial_decode_median_cold_l2": dec_ms * 1e3,
-                     "merge_graph_replay": merge_ms * 1e3},
+                     "merge_graph_replay": merge_ms * 1e3, **fused_alone},
         "rank_kv_bytes": my_bytes, "all_kv_bytes": all_bytes,
         "partial_decode_frac_of_peak": my_bytes / (dec_ms / 1e3) / 1e9 / hbm,
         "peak_source": peak_src,
         "exchange_bytes_per_rank": blk * 4,
         "config": {"workload": f"{W.describe(args.config)}; keys split into {R} "
                                "contiguous page runs per sequence",
-                   "l2": "evicted (a 256 MiB read) before each timed step"},
+                   "l2": "evicted (a 1 GiB read) before each timed step"},
         "clocks": clocks,
         "gpu_launches": K * 3,   # split, combine and merge kernels per step
     }

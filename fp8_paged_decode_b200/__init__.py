@@ -31,6 +31,7 @@ __all__ = [
     "fp8_paged_decode_make_plan_qlen", "FPD_MAX_Q_LEN", "FPD_KV_NHD", "FPD_KV_HND",
     "FPD_Q_BF16", "FPD_Q_F16", "fpd_decode_args", "fp8_paged_decode_cache_write_layout",
     "FPD_KV_E4M3", "FPD_KV_NVFP4", "FPD_OUT_BF16", "FPD_OUT_F32", "fp8_paged_decode_cp_merge",
+    "fp8_paged_decode_cp_merge_wait",
     "nvfp4_page_layout", "fp8_paged_decode_attention_nvfp4",
     "fp8_paged_decode_cache_write_nvfp4", "fp8_paged_decode_workspace_bytes_args",
     "fp8_paged_decode_plan", "fp8_paged_decode_workspace_bytes",
@@ -91,6 +92,7 @@ EXPORTED_SYMBOLS = (
     "fp8_paged_decode_plan_qlen",
     "fp8_paged_decode_workspace_bytes_qlen",
     "fp8_paged_decode_cp_merge",
+    "fp8_paged_decode_cp_merge_wait",
     "fp8_paged_decode_status_string",
     "fp8_paged_decode_version",
 )
@@ -129,7 +131,10 @@ class fpd_decode_args(ctypes.Structure):
                 ("chunk_pages_override", ctypes.c_int), ("kv_format", ctypes.c_int),
                 ("k_scales", ctypes.c_void_p), ("v_scales", ctypes.c_void_p),
                 ("kv_page_stride", ctypes.c_int64), ("sf_page_stride", ctypes.c_int64),
-                ("out_dtype", ctypes.c_int)]
+                ("out_dtype", ctypes.c_int),
+                ("cp_gather", ctypes.c_void_p), ("cp_flags", ctypes.c_void_p),
+                ("cp_ranks", ctypes.c_int), ("cp_rank", ctypes.c_int),
+                ("cp_epoch", ctypes.c_uint32), ("cp_block_floats", ctypes.c_int64)]
 
 
 def library_path() -> str:
@@ -174,6 +179,9 @@ def _bind(lib):
     lib.fp8_paged_decode_cache_write_nvfp4.restype = ci
     lib.fp8_paged_decode_cp_merge.argtypes = [vp, ci, i64, i64, ci, ci, vp, vp, i64, vp, vp]
     lib.fp8_paged_decode_cp_merge.restype = ci
+    lib.fp8_paged_decode_cp_merge_wait.argtypes = [vp, ci, i64, i64, ci, ci, vp, vp, i64, vp, vp,
+                                                   ctypes.c_uint32, ctypes.c_uint64, vp, vp]
+    lib.fp8_paged_decode_cp_merge_wait.restype = ci
     lib.fp8_paged_decode_plan_qlen.argtypes = [ci] * 9 + [ctypes.POINTER(fpd_plan)]
     lib.fp8_paged_decode_plan_qlen.restype = ci
     lib.fp8_paged_decode_workspace_bytes_qlen.argtypes = [ci] * 9
@@ -350,7 +358,8 @@ def _scale_arg(x, name):
 def fp8_paged_decode_attention(q, k_cache, v_cache, block_table, seq_lens, k_scale, v_scale,
                                sm_scale, window_left=-1, sinks=None, out=None, lse=None,
                                workspace=None, stream=None, chunk_pages_override=0,
-                               return_lse=True, kv_layout="NHD", out_dtype="bf16"):
+                               return_lse=True, kv_layout="NHD", out_dtype="bf16",
+                               cp_publish=None):
     """Enqueue one decode call on ``stream`` (default: torch's current stream).
 
     ``q`` is [B, Hq, D] (one query token per sequence) or [B, q_len, Hq, D]
@@ -359,7 +368,11 @@ def fp8_paged_decode_attention(q, k_cache, v_cache, block_table, seq_lens, k_sca
     (a slice of a fused QKV buffer).  ``out`` (q's shape, same rule; bf16, or
     float32 for the partial result of a context-parallel rank) and ``lse``
     (float32, contiguous) are allocated when not given, ``out`` with
-    ``out_dtype`` ("bf16" or "f32").  The caches are
+    ``out_dtype`` ("bf16" or "f32").  ``cp_publish``: the descriptor's
+    (cp_gather, cp_flags, cp_ranks, cp_rank, cp_epoch, cp_block_floats) for a
+    context-parallel rank whose rows go to every rank's gather buffer (see
+    ``cp.CpExchange``); out and lse are then neither allocated nor written and
+    (None, None) is returned.  The caches are
     E4M3 (uint8 or float8_e4m3fn) [num_blocks, block_tokens, Hkv, D], or
     [num_blocks, Hkv, block_tokens, D] with ``kv_layout="HND"``.  ``k_scale`` /
     ``v_scale`` are numbers or one-element float32 CUDA tensors (read on the
@@ -384,8 +397,11 @@ def fp8_paged_decode_attention(q, k_cache, v_cache, block_table, seq_lens, k_sca
         raise ValueError("q and the caches disagree on head_dim")
     max_blocks = block_table.shape[1]
     dev = q.device
-    out, lse = _alloc_outputs(out, lse, lead, Hq, D, dev, out_dtype, return_lse)
-    for name, t in (("q", q), ("out", out)):
+    if cp_publish is not None:
+        out, lse, out_dtype = None, None, "f32"
+    else:
+        out, lse = _alloc_outputs(out, lse, lead, Hq, D, dev, out_dtype, return_lse)
+    for name, t in (("q", q),) + ((("out", out),) if out is not None else ()):
         if not isinstance(t, torch.Tensor) or not t.is_cuda:
             raise TypeError(f"{name} must be a CUDA tensor")
     if q.dtype not in (torch.bfloat16, torch.float16):
@@ -408,12 +424,17 @@ def fp8_paged_decode_attention(q, k_cache, v_cache, block_table, seq_lens, k_sca
     a.window_left = int(window_left)
     sp = _dev_ptr(sinks, "sinks", (torch.float32,), (Hq,))
     a.sinks = sp.value if sp is not None else None
-    a.out = out.data_ptr()
-    a.out_token_stride = _token_rows(out, "out", lead, Hq, D)
-    lp = _dev_ptr(lse, "lse", (torch.float32,), lead + (Hq,))
-    a.lse = lp.value if lp is not None else None
+    if cp_publish is not None:
+        (a.cp_gather, a.cp_flags, a.cp_ranks, a.cp_rank, a.cp_epoch,
+         a.cp_block_floats) = cp_publish
+        a.out_dtype = FPD_OUT_F32
+    else:
+        a.out = out.data_ptr()
+        a.out_token_stride = _token_rows(out, "out", lead, Hq, D)
+        lp = _dev_ptr(lse, "lse", (torch.float32,), lead + (Hq,))
+        a.lse = lp.value if lp is not None else None
+        a.out_dtype = _out_code(out)
     a.chunk_pages_override = int(chunk_pages_override)
-    a.out_dtype = _out_code(out)
     _run_args(a, workspace, dev, stream, "fp8_paged_decode_attention")
     return out, lse
 
@@ -591,6 +612,34 @@ def fp8_paged_decode_attention_nvfp4(q, kv_pages, block_table, seq_lens, k_scale
 
 def fp8_paged_decode_workspace_bytes_args(args) -> int:
     return int(load_library().fp8_paged_decode_workspace_bytes_args(ctypes.byref(args)))
+
+
+def fp8_paged_decode_cp_merge_wait(gather, flags, epoch, out, lse=None, sinks=None,
+                                   timeout_ns=1_000_000_000, status=None, stream=None):
+    """The merge of a fused exchange: waits (at most ``timeout_ns`` of GPU time)
+    until ``flags`` (uint32 CUDA tensor [R], this rank's flag words) all equal
+    ``epoch``, then merges ``gather`` (float32 [R, block_floats], the slots the
+    ranks' publishing decode calls filled) like ``fp8_paged_decode_cp_merge``.
+    A timeout or-s FPD_DEVERR_TIMEOUT into ``status`` (int32 CUDA tensor) and
+    leaves ``out`` unwritten."""
+    import torch
+    if out.dim() not in (3, 4) or out.dtype != torch.bfloat16:
+        raise TypeError("out must be bf16 [B, Hq, D] or [B, q_len, Hq, D]")
+    Hq, D = out.shape[-2], out.shape[-1]
+    lead = tuple(out.shape[:-2])
+    R, block = gather.shape
+    if flags.dtype not in (torch.int32, torch.uint32) or flags.numel() != R:
+        raise ValueError("flags must be R 32-bit words")
+    st = load_library().fp8_paged_decode_cp_merge_wait(
+        _dev_ptr(gather, "gather", (torch.float32,)), int(R), int(block), int(out.numel() // D),
+        int(Hq), int(D), _dev_ptr(sinks, "sinks", (torch.float32,), (Hq,)),
+        ctypes.c_void_p(out.data_ptr()), _token_rows(out, "out", lead, Hq, D),
+        _dev_ptr(lse, "lse", (torch.float32,), lead + (Hq,)),
+        _dev_ptr(flags, "flags", (torch.int32, torch.uint32)), ctypes.c_uint32(int(epoch)),
+        ctypes.c_uint64(int(timeout_ns)), _dev_ptr(status, "status", (torch.int32,)),
+        _stream_handle(stream))
+    _check(st, "fp8_paged_decode_cp_merge_wait")
+    return out, lse
 
 
 def fp8_paged_decode_cp_merge(partials, out, lse=None, sinks=None, stream=None):

@@ -18,6 +18,12 @@ its own last key.
 
 The per-rank buffer is [O (rows * D) | lse (rows) | pad to 4 floats] f32, rows =
 B * Hq, so an all-gather of it is already the merge's [R, block] input.
+
+``CpExchange`` and ``fp8_paged_decode_attention_cp_fused`` fuse the exchange
+into the decode instead: each rank's combine kernel stores its rows straight
+into every rank's gather buffer (peer memory mapped with CUDA IPC) and raises a
+flag there, and each rank's merge waits for the flags; no collective runs on
+the data path.
 """
 from __future__ import annotations
 
@@ -120,3 +126,201 @@ def fp8_paged_decode_attention_cp(q, k_cache, v_cache, block_table, seq_lens, k_
     if lse is None:
         lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
     return fpd.fp8_paged_decode_cp_merge(gathered, out, lse, sinks)
+
+
+# ------------------------------------------------------------ fused exchange --
+
+def _cudart():
+    import ctypes
+    import ctypes.util
+    import os
+    import torch
+    cands = [os.path.join(os.path.dirname(torch.__file__), "..", "nvidia", "cuda_runtime", "lib",
+                          "libcudart.so.12")]
+    found = ctypes.util.find_library("cudart")
+    if found:
+        cands.append(found)
+    for c in cands:
+        try:
+            rt = ctypes.CDLL(c)
+            break
+        except OSError:
+            continue
+    else:
+        raise RuntimeError("no CUDA runtime library found")
+
+    class Handle(ctypes.Structure):
+        _fields_ = [("reserved", ctypes.c_char * 64)]
+    vp = ctypes.c_void_p
+    rt.cudaMalloc.argtypes = [ctypes.POINTER(vp), ctypes.c_size_t]
+    rt.cudaFree.argtypes = [vp]
+    rt.cudaMemset.argtypes = [vp, ctypes.c_int, ctypes.c_size_t]
+    rt.cudaIpcGetMemHandle.argtypes = [ctypes.POINTER(Handle), vp]
+    rt.cudaIpcOpenMemHandle.argtypes = [ctypes.POINTER(vp), Handle, ctypes.c_uint]
+    rt.cudaIpcCloseMemHandle.argtypes = [vp]
+    rt.Handle = Handle
+    return rt
+
+
+class CpExchange:
+    """The buffers of the exchange fused into the decode (``cp_gather`` /
+    ``cp_flags`` of the decode descriptor) for one process group, one process
+    per GPU.
+
+    Every rank owns one device allocation (cudaMalloc): its gather buffer, R
+    slots of ``partial_block_floats(B * Hq, D)`` floats, followed by R flag
+    words.  The ranks exchange CUDA IPC handles of their allocations once (a
+    gather of small host objects over the process group), so each rank holds
+    device pointers to every rank's buffer; its combine kernel stores its rows
+    straight into slot ``rank`` of all of them over NVLink and raises its flag
+    there, and its merge waits for the R flags of its own buffer.
+
+    ``CpExchange.local(R, ...)`` makes R such buffers in one process, standing
+    in for R ranks on one GPU (the publishing calls then run one after another,
+    and every flag is set before any merge waits on it)."""
+
+    def __init__(self, B, Hq, D, group=None, _local_ranks=None):
+        import ctypes
+        import torch
+        self.B, self.Hq, self.D = B, Hq, D
+        self.block = partial_block_floats(B * Hq, D)
+        self._rt = _cudart()
+        self._opened = []
+        self._own = []
+        if _local_ranks is not None:
+            self.R, self.rank = _local_ranks, 0
+            bases = [self._alloc() for _ in range(self.R)]
+            self._own = list(bases)
+        else:
+            import torch.distributed as dist
+            self.R = dist.get_world_size(group)
+            self.rank = dist.get_rank(group)
+            mine = self._alloc()
+            self._own = [mine]
+            h = self._rt.Handle()
+            self._check(self._rt.cudaIpcGetMemHandle(ctypes.byref(h), ctypes.c_void_p(mine)))
+            handles = [None] * self.R
+            dist.all_gather_object(handles, bytes(h.reserved), group=group)
+            bases = []
+            for r, hb in enumerate(handles):
+                if r == self.rank:
+                    bases.append(mine)
+                    continue
+                hr = self._rt.Handle()
+                ctypes.memmove(hr.reserved, hb, 64)
+                p = ctypes.c_void_p()
+                self._check(self._rt.cudaIpcOpenMemHandle(ctypes.byref(p), hr, 1))
+                self._opened.append(p.value)
+                bases.append(p.value)
+        self.bases = bases
+        dev = torch.device("cuda", torch.cuda.current_device())
+        self.gather_ptrs = torch.tensor(bases, dtype=torch.int64, device=dev)
+        self.flag_ptrs = torch.tensor([b + self.R * self.block * 4 for b in bases],
+                                      dtype=torch.int64, device=dev)
+        self.epoch = 0
+
+    @classmethod
+    def local(cls, R, B, Hq, D):
+        return cls(B, Hq, D, _local_ranks=R)
+
+    def _check(self, err):
+        if err != 0:
+            raise RuntimeError(f"CUDA runtime error {err} in the context-parallel exchange")
+
+    def _alloc(self):
+        import ctypes
+        nbytes = self.R_bytes()
+        p = ctypes.c_void_p()
+        self._check(self._rt.cudaMalloc(ctypes.byref(p), nbytes))
+        self._check(self._rt.cudaMemset(p, 0, nbytes))
+        return p.value
+
+    def R_bytes(self):
+        """Bytes of one rank's allocation: R gather slots, then R flag words."""
+        return self.R * self.block * 4 + ((self.R * 4 + 255) // 256) * 256
+
+    def gather(self, r=None):
+        """Rank r's gather buffer as float32 [R, block] (this process's rank by default)."""
+        import torch
+        base = self.bases[self.rank if r is None else r]
+        return _borrowed(base, (self.R, self.block), torch.float32)
+
+    def flags(self, r=None):
+        import torch
+        base = self.bases[self.rank if r is None else r] + self.R * self.block * 4
+        return _borrowed(base, (self.R,), torch.int32)
+
+    def next_epoch(self):
+        self.epoch = self.epoch % 0xFFFFFFFF + 1   # never 0
+        return self.epoch
+
+    def publish_fields(self, rank=None):
+        """(cp_gather, cp_flags, cp_ranks, cp_rank, cp_epoch, cp_block_floats) of
+        this rank's publishing decode call at the current epoch."""
+        return (self.gather_ptrs.data_ptr(), self.flag_ptrs.data_ptr(), self.R,
+                self.rank if rank is None else rank, self.epoch, self.block)
+
+    def close(self):
+        import ctypes
+        for p in self._opened:
+            self._rt.cudaIpcCloseMemHandle(ctypes.c_void_p(p))
+        for p in self._own:
+            self._rt.cudaFree(ctypes.c_void_p(p))
+        self._opened, self._own = [], []
+
+
+class _CudaArray:
+    """Raw device memory described by the CUDA array interface (not owned)."""
+
+    def __init__(self, ptr, shape, typestr):
+        self.__cuda_array_interface__ = {"shape": tuple(shape), "typestr": typestr,
+                                         "data": (int(ptr), False), "version": 3,
+                                         "strides": None}
+
+
+def _borrowed(ptr, shape, dtype):
+    """A torch tensor over device memory that torch neither owns nor frees."""
+    import torch
+    typestr = {torch.float32: "<f4", torch.int32: "<i4"}[dtype]
+    return torch.as_tensor(_CudaArray(ptr, shape, typestr), device="cuda")
+
+
+def fp8_paged_decode_attention_cp_fused(q, k_cache, v_cache, block_table, seq_lens, k_scale,
+                                        v_scale, sm_scale, *, exchange, sinks=None, out=None,
+                                        lse=None, workspace=None, timeout_ns=1_000_000_000,
+                                        status=None, rank=None, publish=True, merge=True,
+                                        kv_layout="NHD", chunk_pages_override=0):
+    """One rank's context-parallel decode with the exchange fused into it, on
+    torch's current stream: the decode over this rank's keys (``block_table`` /
+    ``seq_lens``, as ``fp8_paged_decode_attention_cp``) stores its f32 rows
+    into every rank's gather buffer of ``exchange`` (a ``CpExchange``) and
+    raises its flag there; the merge then waits for all ranks' flags of the
+    current ``exchange.epoch`` (call ``exchange.next_epoch()`` once per step,
+    on every rank, before this) and folds the slots and the sinks together.
+    ``rank`` (default: the exchange's) and ``publish`` / ``merge`` let one
+    process stand in for several ranks.  A flag that does not arrive within
+    ``timeout_ns`` or-s FPD_DEVERR_TIMEOUT into ``status`` (int32 CUDA tensor)
+    and leaves ``out`` unwritten.  Returns ``(out, lse)``."""
+    import torch
+    import fp8_paged_decode_b200 as fpd
+    if q.dim() != 3:
+        raise ValueError("context-parallel decode takes one query token per sequence: q [B, Hq, D]")
+    if exchange.epoch == 0:
+        raise ValueError("call exchange.next_epoch() before the step")
+    B, Hq, D = q.shape
+    r = exchange.rank if rank is None else rank
+    if publish:
+        fpd.fp8_paged_decode_attention(q, k_cache, v_cache, block_table, seq_lens, k_scale,
+                                       v_scale, sm_scale, window_left=-1, sinks=None,
+                                       workspace=workspace, kv_layout=kv_layout,
+                                       chunk_pages_override=chunk_pages_override,
+                                       cp_publish=exchange.publish_fields(r))
+    if not merge:
+        return None, None
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    return fpd.fp8_paged_decode_cp_merge_wait(exchange.gather(r), exchange.flags(r),
+                                              exchange.epoch, out, lse, sinks,
+                                              timeout_ns=timeout_ns, status=status)

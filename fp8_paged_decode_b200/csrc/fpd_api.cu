@@ -671,7 +671,8 @@ static fpd_status attention_impl(const fpd_decode_args& a, void* workspace,
   fpd_status st = validate_shape(B, Hq, Hkv, D, bt, max_blocks, q_len);
   if (st != FPD_OK) return st;
   if (num_blocks <= 0 || (int64_t)num_blocks * bt >= INT32_MAX) return FPD_ERR_UNSUPPORTED;
-  if (!a.q || !a.k_cache || !a.v_cache || !a.block_table || !a.seq_lens || !a.out)
+  if (!a.q || !a.k_cache || !a.v_cache || !a.block_table || !a.seq_lens ||
+      (!a.out && a.cp_ranks <= 0))
     return FPD_ERR_INVALID_ARG;
   if (a.q_dtype != FPD_Q_BF16 && a.q_dtype != FPD_Q_F16) return FPD_ERR_INVALID_ARG;
   if (a.kv_layout != FPD_KV_NHD && a.kv_layout != FPD_KV_HND) return FPD_ERR_INVALID_ARG;
@@ -679,6 +680,16 @@ static fpd_status attention_impl(const fpd_decode_args& a, void* workspace,
   if (a.out_dtype != FPD_OUT_BF16 && a.out_dtype != FPD_OUT_F32) return FPD_ERR_INVALID_ARG;
   const bool fp4 = a.kv_format == FPD_KV_NVFP4;
   const bool f32_out = a.out_dtype == FPD_OUT_F32;
+  const bool cp_pub = a.cp_ranks > 0;
+  if (a.cp_ranks < 0) return FPD_ERR_INVALID_ARG;
+  if (cp_pub) {   // the fused context-parallel exchange
+    if (!f32_out || q_len != 1 || !a.cp_gather || !a.cp_flags || a.cp_rank < 0 ||
+        a.cp_rank >= a.cp_ranks || a.cp_epoch == 0 || !aligned(a.cp_gather, 8) ||
+        !aligned(a.cp_flags, 8) || a.cp_block_floats % 4 != 0 ||
+        a.cp_block_floats < (int64_t)B * Hq * (D + 1) ||
+        (a.out_token_stride != 0 && a.out_token_stride != (int64_t)Hq * D))
+      return FPD_ERR_INVALID_ARG;
+  }
   // NVFP4 pages: head-major, data and scale regions at their own page strides
   const int64_t fp4_data = (int64_t)Hkv * bt * (D / 2), fp4_sf = (int64_t)Hkv * bt * (D / 16);
   const int64_t data_stride = a.kv_page_stride ? a.kv_page_stride : fp4_data;
@@ -697,7 +708,7 @@ static fpd_status attention_impl(const fpd_decode_args& a, void* workspace,
   // 16-byte rows: the query rows are bulk-copied and the outputs stored 16 bytes at a time
   if (q_stride < row || o_stride < row || q_stride % 8 != 0 || o_stride % 8 != 0)
     return FPD_ERR_INVALID_ARG;
-  if (!aligned(a.q, 16) || !aligned(a.out, 16) || !aligned(a.k_cache, 16) ||
+  if (!aligned(a.q, 16) || (a.out && !aligned(a.out, 16)) || !aligned(a.k_cache, 16) ||
       !aligned(a.v_cache, 16) || !aligned(a.block_table, 4) || !aligned(a.seq_lens, 4) ||
       (a.lse && !aligned(a.lse, 4)) || (a.sinks && !aligned(a.sinks, 4)) ||
       (a.k_scale_dev && !aligned(a.k_scale_dev, 4)) ||
@@ -774,7 +785,7 @@ static fpd_status attention_impl(const fpd_decode_args& a, void* workspace,
   p.sm_scale_log2 = a.sm_scale * fpd::kLog2e;
   p.q_f16 = a.q_dtype == FPD_Q_F16;
   p.kv_hnd = hnd;
-  p.out_f32 = f32_out ? static_cast<float*>(a.out) : nullptr;
+  p.combine_all = f32_out;
   p.adapt_chunk = plan.adapt_chunk_pages;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -804,7 +815,15 @@ static fpd_status attention_impl(const fpd_decode_args& a, void* workspace,
     c.part_o = p.part_o;
     c.part_lse = p.part_lse;
     c.out = p.out;
-    c.out_f32 = p.out_f32;
+    c.out_f32 = f32_out && !cp_pub ? static_cast<float*>(a.out) : nullptr;
+    c.cp_ranks = cp_pub ? a.cp_ranks : 0;
+    c.cp_rank = a.cp_rank;
+    c.cp_gather = a.cp_gather;
+    c.cp_flags = a.cp_flags;
+    c.cp_done = reinterpret_cast<uint32_t*>(ws) + 4;
+    c.cp_block = a.cp_block_floats;
+    c.cp_rows = (int64_t)B * Hq;
+    c.cp_epoch = a.cp_epoch;
     c.lse = a.lse;
     c.B = B;
     c.q_len = q_len;
@@ -1030,16 +1049,19 @@ fpd_status fp8_paged_decode_cache_write_layout(const void* key, const void* valu
   return cudaGetLastError() == cudaSuccess ? FPD_OK : FPD_ERR_CUDA;
 }
 
-fpd_status fp8_paged_decode_cp_merge(const float* partials, int R, int64_t block_floats,
-                                     int64_t rows, int Hq, int D, const float* sinks, void* out,
-                                     int64_t out_token_stride, float* lse, void* stream) {
+static fpd_status cp_merge_impl(const float* partials, int R, int64_t block_floats, int64_t rows,
+                                int Hq, int D, const float* sinks, void* out,
+                                int64_t out_token_stride, float* lse, const uint32_t* flags,
+                                uint32_t epoch, uint64_t timeout_ns, uint32_t* status,
+                                void* stream) {
   if (R < 1 || Hq < 1 || rows < 0 || rows % Hq != 0) return FPD_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return FPD_ERR_UNSUPPORTED;
   if (block_floats < rows * (D + 1) || block_floats % 4 != 0) return FPD_ERR_INVALID_ARG;
   const int64_t o_stride = out_token_stride ? out_token_stride : (int64_t)Hq * D;
   if (o_stride < (int64_t)Hq * D || o_stride % 8 != 0) return FPD_ERR_INVALID_ARG;
   if (!partials || !out || !aligned(partials, 16) || !aligned(out, 16) ||
-      (lse && !aligned(lse, 4)) || (sinks && !aligned(sinks, 4)))
+      (lse && !aligned(lse, 4)) || (sinks && !aligned(sinks, 4)) ||
+      (flags && !aligned(flags, 4)) || (status && !aligned(status, 4)))
     return FPD_ERR_INVALID_ARG;
   if (rows == 0) return FPD_OK;
   const int64_t grid = (rows + fpd::kCpMergeWarps - 1) / fpd::kCpMergeWarps;
@@ -1054,12 +1076,37 @@ fpd_status fp8_paged_decode_cp_merge(const float* partials, int R, int64_t block
   p.out_tok_stride = o_stride;
   p.R = R;
   p.Hq = Hq;
+  p.flags = flags;
+  p.epoch = epoch;
+  p.timeout_ns = timeout_ns;
+  p.status = status;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (D == 128)
-    fpd::fpd_cp_merge_kernel<128><<<(int)grid, fpd::kCpMergeWarps * 32, 0, s>>>(p);
-  else
-    fpd::fpd_cp_merge_kernel<64><<<(int)grid, fpd::kCpMergeWarps * 32, 0, s>>>(p);
+  const dim3 g((unsigned)grid), b(fpd::kCpMergeWarps * 32);
+  if (flags) {
+    if (D == 128) fpd::fpd_cp_merge_kernel<128, true><<<g, b, 0, s>>>(p);
+    else fpd::fpd_cp_merge_kernel<64, true><<<g, b, 0, s>>>(p);
+  } else {
+    if (D == 128) fpd::fpd_cp_merge_kernel<128, false><<<g, b, 0, s>>>(p);
+    else fpd::fpd_cp_merge_kernel<64, false><<<g, b, 0, s>>>(p);
+  }
   return cudaGetLastError() == cudaSuccess ? FPD_OK : FPD_ERR_CUDA;
+}
+
+fpd_status fp8_paged_decode_cp_merge(const float* partials, int R, int64_t block_floats,
+                                     int64_t rows, int Hq, int D, const float* sinks, void* out,
+                                     int64_t out_token_stride, float* lse, void* stream) {
+  return cp_merge_impl(partials, R, block_floats, rows, Hq, D, sinks, out, out_token_stride, lse,
+                       nullptr, 0, 0, nullptr, stream);
+}
+
+fpd_status fp8_paged_decode_cp_merge_wait(const float* gather, int R, int64_t block_floats,
+                                          int64_t rows, int Hq, int D, const float* sinks,
+                                          void* out, int64_t out_token_stride, float* lse,
+                                          const uint32_t* flags, uint32_t epoch,
+                                          uint64_t timeout_ns, uint32_t* status, void* stream) {
+  if (!flags || epoch == 0 || timeout_ns == 0) return FPD_ERR_INVALID_ARG;
+  return cp_merge_impl(gather, R, block_floats, rows, Hq, D, sinks, out, out_token_stride, lse,
+                       flags, epoch, timeout_ns, status, stream);
 }
 
 fpd_status fp8_paged_decode_cache_write_nvfp4(const void* key, const void* value,

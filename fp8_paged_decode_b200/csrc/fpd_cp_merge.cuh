@@ -10,6 +10,10 @@
 // where sigma is the head's sink logit (-inf without sinks); a sink adds to
 // the denominator only, so the ranks' partials carry none.
 //
+// With the exchange fused into the ranks' combine kernels (they store their
+// rows straight into every rank's gather buffer over NVLink and raise a flag
+// there), the merge first waits for the R flags.
+//
 // One warp per row; each lane owns D / 32 consecutive elements and reads
 // them from every rank with one 8- or 16-byte load, so a row's R partial rows
 // are read once, coalesced, eight ranks per round trip to memory.  The op
@@ -25,7 +29,8 @@
 
 namespace fpd {
 
-constexpr int kCpMergeWarps = 8;   // rows per CTA
+constexpr int kCpMergeWarps = 8;          // rows per CTA
+constexpr uint32_t kCpErrTimeout = 0x4u;  // a rank's flag did not arrive in time
 
 struct CpMergeParams {
   const float* partials;    // R blocks of `block` floats: [rows][D] O, then [rows] lse
@@ -36,13 +41,47 @@ struct CpMergeParams {
   int64_t rows;
   int64_t out_tok_stride;   // elements between consecutive tokens of `out`
   int R, Hq;
+  // WAIT: the partials arrive from the ranks' combine kernels; flags[r]
+  // reaches `epoch` once rank r's rows are all in place.
+  const uint32_t* flags;
+  uint32_t epoch;
+  uint64_t timeout_ns;
+  uint32_t* status;         // kCpErrTimeout is or-ed in when a flag does not arrive
 };
 
-template <int D>
+// WAIT: first wait for every rank's flag (one thread per CTA, acquire loads at
+// system scope, bounded by timeout_ns of the GPU's global timer); a CTA that
+// gives up records kCpErrTimeout and writes nothing.
+template <int D, bool WAIT>
 __global__ void __launch_bounds__(kCpMergeWarps * 32) fpd_cp_merge_kernel(const CpMergeParams p) {
   constexpr int PER = D / 32;
   constexpr int kBatch = 8;   // ranks whose partials are loaded together
   constexpr float kL2e = 1.4426950408889634f;
+  if constexpr (WAIT) {
+    __shared__ int arrived;
+    if (threadIdx.x < 32) {   // warp 0: lane r polls rank r's flags (r, r + 32, ...)
+      const int lane0 = threadIdx.x;
+      const uint64_t t0 = global_timer_ns();
+      bool ok = true;
+      for (uint32_t spins = 0;; ++spins) {
+        // acquire loads: once a lane sees its flag, the rows behind it are visible
+        bool mine = true;
+        for (int r = lane0; r < p.R; r += 32) mine &= ld_acquire_sys(p.flags + r) == p.epoch;
+        if (__all_sync(0xffffffffu, mine)) break;
+        if (spins >= (1u << 30) || global_timer_ns() - t0 > p.timeout_ns) {
+          ok = false;
+          break;
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (lane0 == 0) {
+        if (!ok && p.status) atomicOr(p.status, kCpErrTimeout);
+        arrived = ok;
+      }
+    }
+    __syncthreads();
+    if (!arrived) return;
+  }
   const int lane = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * kCpMergeWarps + (threadIdx.x >> 5);
   if (row >= p.rows) return;

@@ -111,9 +111,10 @@ struct DecodeParams {
   float sm_scale_log2;        // sm_scale * log2(e), for a device k_scale
   int q_f16;                  // the query is fp16 (else bf16)
   int kv_hnd;                 // pages are [num_blocks, Hkv, bt, D] (else [.., bt, Hkv, D])
-  // f32 output (same element strides as `out`): every row, one split or
-  // several, leaves its partial in the workspace and the combine writes it
-  float* out_f32;
+  // nonzero: every row, one split or several, leaves its partial in the
+  // workspace and the combine writes it (f32 output, context-parallel
+  // publishing)
+  int combine_all;
   // > 0: the split size to take instead of chunk_pages when the sequences
   // are of about equal length and chunk_pages gives more items than the grid
   int adapt_chunk;
@@ -736,9 +737,9 @@ struct Consumer {
         __nv_bfloat16* const orow = p.out + tok * p.out_tok_stride + (size_t)hq * D;
         // false: this query saw no key in the item (only possible with MQ)
         const bool keys = !MQ || lsum[nt][j] > 0.f;
-        const bool one = ns == 1 && !p.out_f32;   // finished here, not by the combine
+        const bool one = ns == 1 && !p.combine_all;   // finished here, not by the combine
         if (ns == 0 || (one && !keys)) {  // no key at all: out = 0, lse = sigma
-          if (p.out_f32) continue;        // the combine writes the row
+          if (p.combine_all) continue;    // the combine writes the row
           uint4* dst = reinterpret_cast<uint4*>(orow + n * E);
 #pragma unroll
           for (int k = 0; k < E / 8; ++k) dst[k] = make_uint4(0u, 0u, 0u, 0u);
@@ -1243,7 +1244,7 @@ __device__ __forceinline__ void split_body(const CUtensorMap* kmap, const CUtens
       alive = false;
       break;
     }
-    const bool single = hd.ns <= 1 && !p.out_f32;   // else the combine finishes the rows
+    const bool single = hd.ns <= 1 && !p.combine_all;   // else the combine finishes the rows
     {
       // thread -> (d, first head); heads step by 128 / D.  The loop body is
       // independent per head, so it is unrolled for overlap.
@@ -1257,7 +1258,7 @@ __device__ __forceinline__ void split_body(const CUtensorMap* kmap, const CUtens
         const size_t row = tok * p.Hq + hq;
         __nv_bfloat16* const orow = p.out + tok * p.out_tok_stride + (size_t)hq * D;
         if (hd.ns == 0) {  // empty sequence: out = 0, lse = sigma
-          if (p.out_f32) continue;   // the combine writes the row
+          if (p.combine_all) continue;   // the combine writes the row
           orow[d] = __float2bfloat16_rn(0.f);
           if (d == 0 && p.lse) p.lse[row] = p.sinks ? p.sinks[hq] : -INFINITY;
           continue;
@@ -1372,13 +1373,63 @@ struct CombineParams {
   float v_scale;
   const float* v_scale_dev;   // device v_scale or nullptr
   int64_t out_tok_stride;     // elements between consecutive output tokens
+  // Context-parallel publishing (cp_ranks > 0): every f32 row goes to slot
+  // cp_rank of each rank's gather buffer (cp_gather[r] + cp_rank * cp_block:
+  // [cp_rows][D] O, then [cp_rows] lse), and once the whole grid has stored
+  // its rows, word cp_rank of each rank's flags is set to cp_epoch.
+  float* const* cp_gather;    // device array [cp_ranks] of gather buffers
+  uint32_t* const* cp_flags;  // device array [cp_ranks] of flag arrays [cp_ranks]
+  uint32_t* cp_done;          // CTAs that finished publishing (zero between calls)
+  int64_t cp_block, cp_rows;
+  int cp_ranks, cp_rank;
+  uint32_t cp_epoch;
 };
 
-// One lane's PER consecutive output elements, x[i] * inv, as bf16 or f32.
+// A row's lse (natural log): to `lse` if given, or to every rank's gather buffer.
+template <int D>
+__device__ __forceinline__ void store_lse(const CombineParams& p, int row, float v) {
+  if (p.cp_ranks > 0) {
+    for (int r = 0; r < p.cp_ranks; ++r)
+      p.cp_gather[r][p.cp_rank * p.cp_block + p.cp_rows * D + row] = v;
+  } else if (p.lse) {
+    p.lse[row] = v;
+  }
+}
+
+// Context-parallel publishing: once every CTA of the grid has stored its rows
+// into all ranks' gather buffers, the last one raises this rank's flag at each
+// rank.  Each CTA releases its stores at GPU scope into the count; the last
+// one, having seen every count, fences at system scope before the flags, so a
+// rank that reads a flag with acquire semantics sees all the rows (release is
+// cumulative).  One system-scope fence per grid.  Every thread of the CTA
+// calls this.
+__device__ __forceinline__ void cp_publish_done(const CombineParams& p) {
+  if (p.cp_ranks <= 0) return;
+  __syncthreads();   // this CTA's rows are stored
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(p.cp_done, 1u) == gridDim.x - 1) {   // the grid's last CTA
+      __threadfence_system();   // one fence orders every row before all the flags
+      *p.cp_done = 0u;          // for the next call
+      for (int r = 0; r < p.cp_ranks; ++r)
+        st_relaxed_sys(p.cp_flags[r] + p.cp_rank, p.cp_epoch);
+    }
+  }
+}
+
+// One lane's PER consecutive output elements, x[i] * inv: bf16, f32, or f32
+// into every rank's gather buffer.
 template <int PER>
 __device__ __forceinline__ void store_out_row(const CombineParams& p, size_t off, const float* x,
                                               float inv) {
-  if (p.out_f32) {
+  if (p.cp_ranks > 0) {
+    for (int r = 0; r < p.cp_ranks; ++r) {
+      float* dst = p.cp_gather[r] + p.cp_rank * p.cp_block + off;
+#pragma unroll
+      for (int i = 0; i < PER; i += 2)
+        *reinterpret_cast<float2*>(dst + i) = make_float2(x[i] * inv, x[i + 1] * inv);
+    }
+  } else if (p.out_f32) {
     float* dst = p.out_f32 + off;
 #pragma unroll
     for (int i = 0; i < PER; i += 2)
@@ -1448,7 +1499,7 @@ __global__ void __launch_bounds__(kCombineMaxThreads) fpd_combine_kernel(const C
       seq_range(L_raw, QL, p.bt, p.max_blocks, p.window_left, chunk, nullptr)
           .n_splits;
   // rows with one split were written by the split kernel, unless the output is f32
-  const bool active = in_range && (ns > 1 || p.out_f32);
+  const bool active = in_range && (ns > 1 || p.out_f32 || p.cp_ranks > 0);
 
   // ---- this warp's splits against its own maximum m
   float m = -INFINITY, z = 0.f;
@@ -1509,8 +1560,9 @@ __global__ void __launch_bounds__(kCombineMaxThreads) fpd_combine_kernel(const C
       const bool any = Z > 0.f;
       const float inv = any ? v_scale * r / Z : 0.f;
       store_out_row<PER>(p, ooff, acc, inv);
-      if (lane == 0 && p.lse) p.lse[row] = any ? (M + __log2f(Z)) * kLn2 : -INFINITY;
+      if (lane == 0) store_lse<D>(p, row, any ? (M + __log2f(Z)) * kLn2 : -INFINITY);
     }
+    cp_publish_done(p);
     return;
   }
 #pragma unroll
@@ -1542,8 +1594,9 @@ __global__ void __launch_bounds__(kCombineMaxThreads) fpd_combine_kernel(const C
       for (int i = 0; i < PER; ++i) a[i] = fmaf(acc_sm[warp + w][lane * PER + i], r, a[i]);
     }
     store_out_row<PER>(p, ooff, a, inv);
-    if (lane == 0 && p.lse) p.lse[row] = any ? (M + __log2f(Z)) * kLn2 : -INFINITY;
+    if (lane == 0) store_lse<D>(p, row, any ? (M + __log2f(Z)) * kLn2 : -INFINITY);
   }
+  cp_publish_done(p);
 }
 
 }  // namespace fpd

@@ -272,6 +272,23 @@ typedef struct {
      * fp8_paged_decode_workspace_bytes_args.  A row with no key and no sink
      * gets out = 0 and lse = -inf, which fp8_paged_decode_cp_merge skips. */
     int out_dtype;               /* FPD_OUT_BF16 or FPD_OUT_F32 */
+    /* Context-parallel publishing (cp_ranks > 0): the exchange of the ranks'
+     * partials fused into this call.  Needs out_dtype = FPD_OUT_F32, q_len = 1
+     * and contiguous out rows (out_token_stride 0 or Hq * D); `out` and `lse`
+     * are not written.  The combine kernel stores every row's f32 O and lse
+     * straight into slot cp_rank of each rank r's gather buffer cp_gather[r]
+     * (cp_block_floats floats per slot: [B*Hq][D] O, then [B*Hq] lse; the
+     * fp8_paged_decode_cp_merge layout) over peer memory (NVLink), and when
+     * the whole grid has stored its rows it sets word cp_rank of each rank's
+     * flag array cp_flags[r] to cp_epoch (a release store at system scope).
+     * cp_gather and cp_flags are device arrays of cp_ranks device pointers
+     * (peer pointers from CUDA IPC or another mapping).  Workspace word 4
+     * counts the finished CTAs and must be zero between calls (it is reset). */
+    float *const *cp_gather;
+    uint32_t *const *cp_flags;
+    int cp_ranks, cp_rank;
+    uint32_t cp_epoch;
+    int64_t cp_block_floats;
 } fpd_decode_args;
 
 /*
@@ -472,6 +489,24 @@ fpd_status fp8_paged_decode_cache_write_nvfp4(const void *key, const void *value
 fpd_status fp8_paged_decode_cp_merge(const float *partials, int R, int64_t block_floats,
                                      int64_t rows, int Hq, int D, const float *sinks, void *out,
                                      int64_t out_token_stride, float *lse, void *stream);
+
+/*
+ * The merge of a fused exchange: `gather` is this rank's gather buffer, whose
+ * R slots the ranks' decode calls fill (fpd_decode_args.cp_gather), and
+ * flags[r] (this rank's flag array, device memory) reaches `epoch` once rank
+ * r's slot is complete.  Each CTA first waits for all R flags (acquire loads at
+ * system scope) for at most timeout_ns nanoseconds of the GPU's global timer;
+ * a CTA that gives up or-s FPD_DEVERR_TIMEOUT into *status (device word, may
+ * be NULL) and writes nothing.  The other arguments and errors are those of
+ * fp8_paged_decode_cp_merge; epoch 0, timeout 0 or a NULL flags pointer is
+ * FPD_ERR_INVALID_ARG.  Epochs must change from call to call (the flags keep
+ * the last one).
+ */
+fpd_status fp8_paged_decode_cp_merge_wait(const float *gather, int R, int64_t block_floats,
+                                          int64_t rows, int Hq, int D, const float *sinks,
+                                          void *out, int64_t out_token_stride, float *lse,
+                                          const uint32_t *flags, uint32_t epoch,
+                                          uint64_t timeout_ns, uint32_t *status, void *stream);
 
 /*
  * Reads the workspace status word (FPD_DEVERR_* bits) after synchronising

@@ -229,3 +229,162 @@ def test_rank_call_rejects_several_queries():
     q = torch.zeros((1, 2, 8, 128), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(ValueError):
         cp.fp8_paged_decode_attention_cp(q, None, None, None, None, 1.0, 1.0, 0.1)
+
+
+# ---------------------------------------------------------- fused exchange --
+
+def _fused_step(wl, dev, ex, R, ranks_publishing=None):
+    """One step of R ranks on one GPU: every rank's publishing decode (one after
+    another), then every rank's waiting merge.  Returns the R (out, lse)."""
+    ex.next_epoch()
+    for r in (range(R) if ranks_publishing is None else ranks_publishing):
+        t_r, l_r = cp.cp_shard(wl.block_table, wl.seq_lens, R, r, wl.block_tokens)
+        cp.fp8_paged_decode_attention_cp_fused(
+            dev["q"], dev["k_cache"], dev["v_cache"], torch.from_numpy(t_r).cuda(),
+            torch.from_numpy(l_r).cuda(), wl.k_scale, wl.v_scale, wl.sm_scale, exchange=ex,
+            rank=r, merge=False)
+    return [cp.fp8_paged_decode_attention_cp_fused(
+                dev["q"], None, None, None, None, wl.k_scale, wl.v_scale, wl.sm_scale,
+                exchange=ex, rank=r, sinks=dev["sinks"], publish=False)
+            for r in range(R)]
+
+
+@pytest.mark.parametrize("case", [0, 2, 3, 5])
+def test_fused_exchange_vs_oracle(case):
+    """Each rank's combine kernel stores its rows into every rank's gather
+    buffer and raises its flag there; each rank's merge waits for the flags.
+    All ranks agree bitwise, with each other and with the unfused path."""
+    Hq, Hkv, D, bt, lens, sinks, R = CP_CASES[case]
+    B = len(lens)
+    wl = W.make_custom(B=B, Hq=Hq, Hkv=Hkv, D=D, block_tokens=bt, seq_lens=lens, sinks=sinks,
+                       seed=300 + case)
+    dev = to_device(wl)
+    ex = cp.CpExchange.local(R, B, Hq, D)
+    try:
+        res = _fused_step(wl, dev, ex, R)
+        torch.cuda.synchronize()
+        flags = ex.flags(0).cpu()
+        assert (flags == ex.epoch).all()
+        # the unfused path: f32 partials, then the merge of the gathered rows
+        gathered = torch.zeros((R, cp.partial_block_floats(B * Hq, D)), dtype=torch.float32,
+                               device="cuda")
+        for r in range(R):
+            t_r, l_r = cp.cp_shard(wl.block_table, wl.seq_lens, R, r, bt)
+            o_v, l_v = cp.partial_views(gathered[r], (B,), Hq, D)
+            _decode_f32(wl, dev, table=torch.from_numpy(t_r).cuda(),
+                        lens=torch.from_numpy(l_r).cuda(), sinks=None, out=o_v, lse=l_v)
+        ref = fpd.fp8_paged_decode_cp_merge(gathered, torch.empty_like(res[0][0]),
+                                            torch.empty_like(res[0][1]), dev["sinks"])
+        torch.cuda.synchronize()
+        for o, l in res:
+            assert torch.equal(o, ref[0]) and torch.equal(l, ref[1])
+        ro, rl = oracle.decode_workload(wl)
+        assert_parity(res[0][0].float().cpu().numpy().astype(np.float64),
+                      res[0][1].cpu().numpy().astype(np.float64), ro, rl,
+                      what=f"fused exchange, case {case}, {R} ranks")
+    finally:
+        ex.close()
+
+
+def test_fused_exchange_consecutive_steps():
+    """The flags keep the last epoch and the finished-CTA counter resets itself:
+    a second step with another query is right too."""
+    wl = W.make_custom(B=3, Hq=32, Hkv=8, D=128, block_tokens=16, seq_lens=[40, 3000, 7000],
+                       sinks=True, seed=51)
+    dev = to_device(wl)
+    ex = cp.CpExchange.local(4, 3, 32, 128)
+    try:
+        ws = None
+        for step in range(3):
+            wl.q = W.make_custom(B=3, Hq=32, Hkv=8, D=128, block_tokens=16,
+                                 seq_lens=[40, 3000, 7000], seed=60 + step).q
+            dev["q"] = torch.from_numpy(wl.q.view(np.int16)).view(torch.bfloat16).cuda()
+            out, lse = _fused_step(wl, dev, ex, 4)[2]
+            torch.cuda.synchronize()
+            ro, rl = oracle.decode_workload(wl)
+            assert_parity(out.float().cpu().numpy().astype(np.float64),
+                          lse.cpu().numpy().astype(np.float64), ro, rl, what=f"step {step}")
+        assert ex.epoch == 3
+    finally:
+        ex.close()
+
+
+def test_fused_exchange_missing_rank_times_out():
+    """A rank whose flag never arrives: the merge's bounded wait gives up,
+    records FPD_DEVERR_TIMEOUT and writes nothing; the GPU stays usable."""
+    wl = W.make_custom(B=2, Hq=8, Hkv=2, D=128, block_tokens=16, seq_lens=[100, 300], seed=71)
+    dev = to_device(wl)
+    ex = cp.CpExchange.local(2, 2, 8, 128)
+    try:
+        ex.next_epoch()
+        t_r, l_r = cp.cp_shard(wl.block_table, wl.seq_lens, 2, 0, 16)
+        cp.fp8_paged_decode_attention_cp_fused(
+            dev["q"], dev["k_cache"], dev["v_cache"], torch.from_numpy(t_r).cuda(),
+            torch.from_numpy(l_r).cuda(), wl.k_scale, wl.v_scale, wl.sm_scale, exchange=ex,
+            rank=0, merge=False)   # rank 1 never publishes
+        out = torch.full((2, 8, 128), 7.0, dtype=torch.bfloat16, device="cuda")
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        cp.fp8_paged_decode_attention_cp_fused(
+            dev["q"], None, None, None, None, wl.k_scale, wl.v_scale, wl.sm_scale, exchange=ex,
+            rank=0, publish=False, out=out, timeout_ns=2_000_000, status=status)
+        torch.cuda.synchronize()
+        assert int(status.item()) & fpd.FPD_DEVERR_TIMEOUT
+        assert (out == 7.0).all()
+        # the context is fine: an ordinary call still works
+        o, l = fpd.fp8_paged_decode_attention(dev["q"], dev["k_cache"], dev["v_cache"],
+                                              dev["block_table"], dev["seq_lens"], wl.k_scale,
+                                              wl.v_scale, wl.sm_scale)
+        torch.cuda.synchronize()
+        ro, rl = oracle.decode_workload(wl)
+        assert_parity(o.float().cpu().numpy().astype(np.float64),
+                      l.cpu().numpy().astype(np.float64), ro, rl, what="after the timeout")
+    finally:
+        ex.close()
+
+
+def test_fused_exchange_rejects_bad_descriptors():
+    wl = W.make_custom(B=2, Hq=8, Hkv=2, D=128, block_tokens=16, seq_lens=[100, 300], seed=72)
+    dev = to_device(wl)
+    ex = cp.CpExchange.local(2, 2, 8, 128)
+    try:
+        ex.next_epoch()
+        g, f, R, _, e, blk = ex.publish_fields(0)
+        for fields in ((g, f, R, 2, e, blk),          # rank out of range
+                       (g, f, R, 0, 0, blk),          # epoch 0
+                       (g, f, R, 0, e, blk - 4),      # slot too small
+                       (0, f, R, 0, e, blk)):         # no gather pointers
+            with pytest.raises(fpd.FpdError) as err:
+                fpd.fp8_paged_decode_attention(dev["q"], dev["k_cache"], dev["v_cache"],
+                                               dev["block_table"], dev["seq_lens"], wl.k_scale,
+                                               wl.v_scale, wl.sm_scale, cp_publish=fields)
+            assert err.value.status == fpd.FPD_ERR_INVALID_ARG
+    finally:
+        ex.close()
+
+
+def test_fused_exchange_through_a_process_group():
+    """The distributed constructor (IPC handles gathered over the group) with
+    one rank, and the fused call through it."""
+    import torch.distributed as dist
+    wl = W.make_custom(B=4, Hq=32, Hkv=8, D=128, block_tokens=16, seq_lens=[3, 800, 2500, 4096],
+                       sinks=True, seed=43)
+    dev = to_device(wl)
+    store = dist.TCPStore("127.0.0.1", _free_port(), 1, True,
+                          timeout=datetime.timedelta(seconds=60))
+    dist.init_process_group("gloo", store=store, rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        ex = cp.CpExchange(4, 32, 128)
+        try:
+            ex.next_epoch()
+            out, lse = cp.fp8_paged_decode_attention_cp_fused(
+                dev["q"], dev["k_cache"], dev["v_cache"], dev["block_table"], dev["seq_lens"],
+                wl.k_scale, wl.v_scale, wl.sm_scale, exchange=ex, sinks=dev["sinks"])
+            torch.cuda.synchronize()
+        finally:
+            ex.close()
+    finally:
+        dist.destroy_process_group()
+    ro, rl = oracle.decode_workload(wl)
+    assert_parity(out.float().cpu().numpy().astype(np.float64),
+                  lse.cpu().numpy().astype(np.float64), ro, rl, what="one-rank exchange")
