@@ -118,8 +118,13 @@ fpd_status fp8_paged_decode_plan(int B, int Hq, int Hkv, int D, int block_tokens
  * Workspace bytes one fp8_paged_decode_attention call with these sizes needs on
  * the CURRENT device (queries its SM count and the kernel occupancy once).
  * Returns 0 for an unsupported or malformed shape, or when no device is present.
- * The workspace holds a 256-byte header (status word) and per-split partial
- * results; its contents between calls carry only the sticky status bits.
+ * The workspace holds a 256-byte header and per-split partial results.  Header
+ * words: 0 the sticky FPD_DEVERR_* status bits; 1 and 2 the work counter and
+ * the finished-CTA count (reset by the kernel itself); 3 the split size
+ * (pages) the last call used; 4 the publishing CTA count of the fused
+ * context-parallel exchange (reset by the kernel).  Zero the header once
+ * before the first call (fp8_paged_decode_workspace_init); between calls it
+ * carries only the status bits and word 3.
  */
 size_t fp8_paged_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int block_tokens,
                                         int max_blocks, int window_left);
