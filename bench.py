@@ -971,30 +971,39 @@ def run_cp(args):
             a.out, a.lse = None, None
             fused.append(a)
         fstatus = torch.zeros(1, dtype=torch.int32, device=dev)
-        flags_me, gather_me = ex.flags(me), ex.gather(me)
         fsh = ctypes.c_void_p(stream.cuda_stream)
 
-        ex.next_epoch()
-        for r, a in enumerate(fused):
+        def set_fields(a, r):
             (a.cp_gather, a.cp_flags, a.cp_ranks, a.cp_rank, a.cp_epoch,
-             a.cp_block_floats) = ex.publish_fields(r if ws == 1 else rank)
-        if ws == 1:
-            for a in fused:
-                assert f_dec(ctypes.byref(a), ws_ptr, ws_n, fsh) == 0
+             a.cp_block_floats) = ex.publish_fields(r)
+
+        # this rank's gather buffer and flags, per epoch parity
+        views = {}
+        for _ in range(2):
+            ex.next_epoch()
+            views[ex.epoch & 1] = (ex.gather(me), ex.flags(me))
+            for r, a in enumerate(fused):
+                set_fields(a, r if ws == 1 else rank)
+            if ws == 1:   # every rank's slots of both buffers hold its partial
+                for a in fused:
+                    assert f_dec(ctypes.byref(a), ws_ptr, ws_n, fsh) == 0
         mine_f = fused[me] if ws == 1 else fused[0]
         mine_f_ref = ctypes.byref(mine_f)
-        margs = [ctypes.c_void_p(gather_me.data_ptr()), R, blk, rows, Hq, D,
+        margs = [None, R, blk, rows, Hq, D,
                  ctypes.c_void_p(sinks.data_ptr()) if sinks is not None else None,
                  ctypes.c_void_p(out.data_ptr()), 0, ctypes.c_void_p(lse.data_ptr()),
-                 ctypes.c_void_p(flags_me.data_ptr()), ctypes.c_uint32(0),
-                 ctypes.c_uint64(1_000_000_000), ctypes.c_void_p(fstatus.data_ptr()), fsh]
+                 None, None, ctypes.c_uint64(1_000_000_000), ctypes.c_void_p(fstatus.data_ptr()),
+                 fsh]
         f_merge_wait = lib.fp8_paged_decode_cp_merge_wait
 
         def pre_step():   # untimed: a new epoch; one process: every rank's flag raised
-            mine_f.cp_epoch = ex.next_epoch()
-            margs[11] = ctypes.c_uint32(ex.epoch)
+            e = ex.next_epoch()
+            set_fields(mine_f, me if ws == 1 else rank)
+            g, fl = views[e & 1]
+            margs[0], margs[10], margs[11] = (ctypes.c_void_p(g.data_ptr()),
+                                              ctypes.c_void_p(fl.data_ptr()), ctypes.c_uint32(e))
             if ws == 1:
-                flags_me.fill_(ex.epoch)
+                fl.fill_(e)
 
         def step():
             st = f_dec(mine_f_ref, ws_ptr, ws_n, fsh)

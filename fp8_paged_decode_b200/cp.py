@@ -167,13 +167,17 @@ class CpExchange:
     ``cp_flags`` of the decode descriptor) for one process group, one process
     per GPU.
 
-    Every rank owns one device allocation (cudaMalloc): its gather buffer, R
-    slots of ``partial_block_floats(B * Hq, D)`` floats, followed by R flag
-    words.  The ranks exchange CUDA IPC handles of their allocations once (a
-    gather of small host objects over the process group), so each rank holds
-    device pointers to every rank's buffer; its combine kernel stores its rows
-    straight into slot ``rank`` of all of them over NVLink and raises its flag
-    there, and its merge waits for the R flags of its own buffer.
+    Every rank owns one device allocation (cudaMalloc): two gather buffers of
+    R slots of ``partial_block_floats(B * Hq, D)`` floats, then two arrays of R
+    flag words.  The ranks exchange CUDA IPC handles of their allocations once
+    (a gather of small host objects over the process group), so each rank
+    holds device pointers to every rank's buffers; its combine kernel stores
+    its rows straight into slot ``rank`` of all of them over NVLink and raises
+    its flag there, and its merge waits for the R flags of its own buffer.
+    Steps alternate between the two buffers by the parity of the epoch: a rank
+    may publish step k + 1 while a slower rank still merges step k, but not
+    step k + 2, whose merge waits for that rank's step k + 1, which its stream
+    runs after its merge of step k.
 
     ``CpExchange.local(R, ...)`` makes R such buffers in one process, standing
     in for R ranks on one GPU (the publishing calls then run one after another,
@@ -214,9 +218,11 @@ class CpExchange:
                 bases.append(p.value)
         self.bases = bases
         dev = torch.device("cuda", torch.cuda.current_device())
-        self.gather_ptrs = torch.tensor(bases, dtype=torch.int64, device=dev)
-        self.flag_ptrs = torch.tensor([b + self.R * self.block * 4 for b in bases],
-                                      dtype=torch.int64, device=dev)
+        # per parity: every rank's gather buffer and flag array
+        self.gather_ptrs = [torch.tensor([self._gather_at(b, par) for b in bases],
+                                         dtype=torch.int64, device=dev) for par in (0, 1)]
+        self.flag_ptrs = [torch.tensor([self._flags_at(b, par) for b in bases],
+                                       dtype=torch.int64, device=dev) for par in (0, 1)]
         self.epoch = 0
 
     @classmethod
@@ -235,20 +241,33 @@ class CpExchange:
         self._check(self._rt.cudaMemset(p, 0, nbytes))
         return p.value
 
+    def _flag_stride(self):
+        return (self.R * 4 + 255) // 256 * 256
+
     def R_bytes(self):
-        """Bytes of one rank's allocation: R gather slots, then R flag words."""
-        return self.R * self.block * 4 + ((self.R * 4 + 255) // 256) * 256
+        """Bytes of one rank's allocation: two gather buffers of R slots, then
+        two arrays of R flag words."""
+        return 2 * self.R * self.block * 4 + 2 * self._flag_stride()
+
+    def _gather_at(self, base, parity):
+        return base + parity * self.R * self.block * 4
+
+    def _flags_at(self, base, parity):
+        return base + 2 * self.R * self.block * 4 + parity * self._flag_stride()
 
     def gather(self, r=None):
-        """Rank r's gather buffer as float32 [R, block] (this process's rank by default)."""
+        """Rank r's gather buffer of the current epoch, float32 [R, block]
+        (this process's rank by default)."""
         import torch
         base = self.bases[self.rank if r is None else r]
-        return _borrowed(base, (self.R, self.block), torch.float32)
+        return _borrowed(self._gather_at(base, self.epoch & 1), (self.R, self.block),
+                         torch.float32)
 
     def flags(self, r=None):
+        """Rank r's flag words of the current epoch, int32 [R]."""
         import torch
-        base = self.bases[self.rank if r is None else r] + self.R * self.block * 4
-        return _borrowed(base, (self.R,), torch.int32)
+        base = self.bases[self.rank if r is None else r]
+        return _borrowed(self._flags_at(base, self.epoch & 1), (self.R,), torch.int32)
 
     def next_epoch(self):
         self.epoch = self.epoch % 0xFFFFFFFF + 1   # never 0
@@ -257,7 +276,8 @@ class CpExchange:
     def publish_fields(self, rank=None):
         """(cp_gather, cp_flags, cp_ranks, cp_rank, cp_epoch, cp_block_floats) of
         this rank's publishing decode call at the current epoch."""
-        return (self.gather_ptrs.data_ptr(), self.flag_ptrs.data_ptr(), self.R,
+        par = self.epoch & 1
+        return (self.gather_ptrs[par].data_ptr(), self.flag_ptrs[par].data_ptr(), self.R,
                 self.rank if rank is None else rank, self.epoch, self.block)
 
     def close(self):

@@ -285,10 +285,14 @@ typedef struct {
      * (cp_block_floats floats per slot: [B*Hq][D] O, then [B*Hq] lse; the
      * fp8_paged_decode_cp_merge layout) over peer memory (NVLink), and when
      * the whole grid has stored its rows it sets word cp_rank of each rank's
-     * flag array cp_flags[r] to cp_epoch (a release store at system scope).
+     * flag array cp_flags[r] to cp_epoch (one system-scope fence, then the
+     * flag stores).
      * cp_gather and cp_flags are device arrays of cp_ranks device pointers
      * (peer pointers from CUDA IPC or another mapping).  Workspace word 4
-     * counts the finished CTAs and must be zero between calls (it is reset). */
+     * counts the finished CTAs and must be zero between calls (it is reset).
+     * A slot must not be rewritten while its rank may still merge it: alternate
+     * two sets of gather buffers and flags by the parity of the epoch (a rank
+     * can run at most one step ahead of another). */
     float *const *cp_gather;
     uint32_t *const *cp_flags;
     int cp_ranks, cp_rank;
