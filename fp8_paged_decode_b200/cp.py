@@ -270,8 +270,16 @@ class CpExchange:
         return _borrowed(self._flags_at(base, self.epoch & 1), (self.R,), torch.int32)
 
     def next_epoch(self):
-        self.epoch = self.epoch % 0xFFFFFFFF + 1   # never 0
+        """Advance to the next step: epochs run 1, 2, ..., 2**32 - 2 and wrap to 1,
+        so they are never 0 and their parity always alternates."""
+        self.epoch = self.epoch % 0xFFFFFFFE + 1
         return self.epoch
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
 
     def publish_fields(self, rank=None):
         """(cp_gather, cp_flags, cp_ranks, cp_rank, cp_epoch, cp_block_floats) of

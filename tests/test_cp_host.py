@@ -165,3 +165,17 @@ def test_two_gloo_ranks_exchange_and_merge():
         assert p.exitcode == 0
     for rank, err_o, err_l in res:
         assert err_o < 1e-5 and err_l < 1e-5, (rank, err_o, err_l)
+
+
+def test_exchange_epochs_alternate_parity_and_skip_zero():
+    """The fused exchange alternates its two buffers by the epoch's parity: the
+    epoch sequence must never hit 0 (the flags' initial value) and must keep
+    alternating across the wrap."""
+    ex = cp.CpExchange.__new__(cp.CpExchange)   # host logic only, no buffers
+    ex.epoch = 0
+    seen = [ex.next_epoch() for _ in range(4)]
+    assert seen == [1, 2, 3, 4]
+    ex.epoch = 0xFFFFFFFD
+    seq = [ex.next_epoch() for _ in range(4)]
+    assert seq == [0xFFFFFFFE, 1, 2, 3]
+    assert all((a ^ b) & 1 for a, b in zip([0xFFFFFFFD] + seq, seq))
