@@ -146,13 +146,28 @@ def cudart():
     return rt
 
 
+def _code_lines(text):
+    """The source without // comments and blank lines (a line holding a string
+    literal keeps its text after //), so that comment edits keep the hash."""
+    out = []
+    for line in text.splitlines():
+        if '"' not in line and "//" in line:
+            line = line[:line.index("//")]
+        line = line.rstrip()
+        if line:
+            out.append(line)
+    return "\n".join(out)
+
+
 def kernel_source_hash():
+    """sha256 of the split kernel's device code (fpd_kernels.cuh, fpd_ptx.cuh)
+    without comments: the key of the committed DRAM-traffic record."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "fp8_paged_decode_b200", "csrc")
     for fn in KERNEL_SOURCES:
-        with open(os.path.join(csrc, fn), "rb") as f:
+        with open(os.path.join(csrc, fn), encoding="utf-8") as f:
             h.update(fn.encode())
-            h.update(f.read())
+            h.update(_code_lines(f.read()).encode())
     return h.hexdigest()
 
 

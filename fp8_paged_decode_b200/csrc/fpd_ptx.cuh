@@ -92,8 +92,8 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
-// 3-D tiled load of one box into shared memory, completing on `bar`
-// (no multicast).  Out-of-range boxes are filled with zeros by the hardware.
+// 3-D tiled load of one box into this CTA's shared memory, completing on
+// `bar`.  Out-of-range boxes are filled with zeros by the hardware.
 __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* map, int c0, int c1,
                                             int c2, uint64_t* bar, uint64_t policy) {
   asm volatile(

@@ -66,3 +66,13 @@ def test_lognormal_lengths():
     wl_lens = W._draw_lens(np.random.default_rng(0), 4096, ("lognormal", 2048.0, 1.0, 1, 32768))
     assert wl_lens.min() >= 1 and wl_lens.max() <= 32768
     assert abs(math.log(np.median(wl_lens)) - math.log(2048)) < 0.1
+
+
+def test_kernel_hash_ignores_comments_only():
+    """The traffic record is keyed by the kernels' code without comments: a
+    comment edit keeps the key, a code edit changes it."""
+    import bench
+    src = 'int a = 1;  // one\n// a comment line\n\nasm("x // y");\nint b = 2;\n'
+    assert bench._code_lines(src) == 'int a = 1;\nasm("x // y");\nint b = 2;'
+    assert bench._code_lines(src.replace("// one", "// uno")) == bench._code_lines(src)
+    assert bench._code_lines(src.replace("b = 2", "b = 3")) != bench._code_lines(src)
