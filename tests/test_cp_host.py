@@ -179,3 +179,18 @@ def test_exchange_epochs_alternate_parity_and_skip_zero():
     seq = [ex.next_epoch() for _ in range(4)]
     assert seq == [0xFFFFFFFE, 1, 2, 3]
     assert all((a ^ b) & 1 for a, b in zip([0xFFFFFFFD] + seq, seq))
+
+
+def test_rank_calls_reject_bad_input_before_any_device_work():
+    q4 = torch.zeros((1, 2, 8, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        cp.fp8_paged_decode_attention_cp(q4, None, None, None, None, 1.0, 1.0, 0.1)
+    ex = cp.CpExchange.__new__(cp.CpExchange)
+    ex.epoch, ex.rank = 0, 0
+    with pytest.raises(ValueError):
+        cp.fp8_paged_decode_attention_cp_fused(q4, None, None, None, None, 1.0, 1.0, 0.1,
+                                               exchange=ex)
+    q3 = torch.zeros((1, 8, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):   # no epoch started
+        cp.fp8_paged_decode_attention_cp_fused(q3, None, None, None, None, 1.0, 1.0, 0.1,
+                                               exchange=ex)
