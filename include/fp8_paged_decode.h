@@ -37,6 +37,13 @@
  *    range) never cause an out-of-bounds access: the length is clamped, the page
  *    is read as zeros, and a bit is set in the workspace status word
  *    (FPD_DEVERR_*), readable with fp8_paged_decode_check_status.
+ *
+ * Beyond the single-query E4M3 call: several query tokens per sequence
+ * (_qlen), a descriptor form with fp16 queries, head-major pages, token
+ * strides, device scales, NVFP4 pages and an f32 output (_args), the FP8 and
+ * NVFP4 cache writers, and context-parallel decode (the f32 partial of a rank,
+ * the merge of R ranks' partials, and the exchange fused into the decode with
+ * a merge that waits for the ranks' flags).
  */
 #ifndef FP8_PAGED_DECODE_H
 #define FP8_PAGED_DECODE_H
@@ -59,7 +66,8 @@ typedef enum {
 /* Device-side status bits (sticky until cleared). */
 #define FPD_DEVERR_SEQ_LEN 0x1u       /* a seq_lens entry was < 0 or > max_blocks * block_tokens (clamped) */
 #define FPD_DEVERR_BLOCK_TABLE 0x2u   /* a block-table entry in the attended range was outside [0, num_blocks) (read as zeros) */
-#define FPD_DEVERR_TIMEOUT 0x4u       /* a pipeline wait exceeded its time limit (results invalid) */
+#define FPD_DEVERR_TIMEOUT 0x4u       /* a pipeline wait, or a context-parallel merge's wait for a
+                                         rank's flag, exceeded its time limit (results invalid) */
 #define FPD_DEVERR_SLOT 0x8u          /* cache write: a slot_mapping entry was >= num_blocks * block_tokens (token skipped) */
 
 /* Split plan chosen by the host planner; all fields are outputs. */
