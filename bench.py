@@ -32,7 +32,6 @@ from __future__ import annotations
 
 import argparse
 import ctypes
-import ctypes.util
 import hashlib
 import json
 import math
@@ -122,28 +121,10 @@ KERNEL_SOURCES = ("fpd_kernels.cuh", "fpd_ptx.cuh")
 
 
 def cudart():
-    """The CUDA runtime library that torch loads (for raw async copies and event
-    calls from the host loop)."""
-    import torch
-    cands = [os.path.join(os.path.dirname(torch.__file__), "..", "nvidia", "cuda_runtime", "lib",
-                          "libcudart.so.12")]
-    found = ctypes.util.find_library("cudart")
-    if found:
-        cands.append(found)
-    for c in cands:
-        if os.path.exists(c) or not os.path.isabs(c):
-            try:
-                rt = ctypes.CDLL(c)
-                break
-            except OSError:
-                continue
-    else:
-        raise RuntimeError("no CUDA runtime library found for the end-to-end loop")
-    vp = ctypes.c_void_p
-    rt.cudaMemcpyAsync.argtypes = [vp, vp, ctypes.c_size_t, ctypes.c_int, vp]
-    rt.cudaEventRecord.argtypes = [vp, vp]
-    rt.cudaStreamWaitEvent.argtypes = [vp, vp, ctypes.c_uint]
-    return rt
+    """The CUDA runtime library torch loads (raw async copies and event calls
+    for the end-to-end host loop)."""
+    from fp8_paged_decode_b200 import cp
+    return cp._cudart()
 
 
 def _code_lines(text):

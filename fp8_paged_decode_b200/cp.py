@@ -131,6 +131,9 @@ def fp8_paged_decode_attention_cp(q, k_cache, v_cache, block_table, seq_lens, k_
 # ------------------------------------------------------------ fused exchange --
 
 def _cudart():
+    """The CUDA runtime library that torch loads, with the prototypes the
+    context-parallel exchange and the benchmark's host loop use: device
+    allocation, IPC handles, async copies and event calls."""
     import ctypes
     import ctypes.util
     import os
@@ -158,6 +161,9 @@ def _cudart():
     rt.cudaIpcGetMemHandle.argtypes = [ctypes.POINTER(Handle), vp]
     rt.cudaIpcOpenMemHandle.argtypes = [ctypes.POINTER(vp), Handle, ctypes.c_uint]
     rt.cudaIpcCloseMemHandle.argtypes = [vp]
+    rt.cudaMemcpyAsync.argtypes = [vp, vp, ctypes.c_size_t, ctypes.c_int, vp]
+    rt.cudaEventRecord.argtypes = [vp, vp]
+    rt.cudaStreamWaitEvent.argtypes = [vp, vp, ctypes.c_uint]
     rt.Handle = Handle
     return rt
 
@@ -289,12 +295,14 @@ class CpExchange:
                 self.rank if rank is None else rank, self.epoch, self.block)
 
     def close(self):
+        """Unmap the peers' buffers and free this rank's (after the device work
+        that uses them has finished); the exchange is unusable afterwards."""
         import ctypes
         for p in self._opened:
             self._rt.cudaIpcCloseMemHandle(ctypes.c_void_p(p))
         for p in self._own:
             self._rt.cudaFree(ctypes.c_void_p(p))
-        self._opened, self._own = [], []
+        self._opened, self._own, self.bases = [], [], []
 
 
 class _CudaArray:
