@@ -293,3 +293,34 @@ def test_planner_offers_one_round_split_size():
     # a forced split size is used as given
     p = plan(B=4, block_tokens=64, max_blocks=256, ctas_per_sm=3, chunk_pages_override=4)
     assert p["adapt_chunk_pages"] == 0 and p["ctas"] == 444
+
+
+def test_ctypes_structs_match_the_c_header(tmp_path):
+    """The Python mirrors of fpd_plan and fpd_decode_args have the C layout:
+    every field's offset and the struct sizes, as a C compiler sees the header."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "fp8_paged_decode.h"',
+             "int main(void) {"]
+    for cname, cls in (("fpd_plan", fpd.fpd_plan), ("fpd_decode_args", fpd.fpd_decode_args)):
+        lines.append(f'printf("{cname} size %zu\\n", sizeof({cname}));')
+        for f, _ in cls._fields_:
+            lines.append(f'printf("{cname} {f} %zu\\n", offsetof({cname}, {f}));')
+    lines += ["return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run([cc, "-I", os.path.join(root, "include"), "-o", str(exe), str(src)], check=True)
+    seen = {}
+    for line in subprocess.run([str(exe)], check=True, capture_output=True,
+                               text=True).stdout.splitlines():
+        name, field, value = line.split()
+        seen[(name, field)] = int(value)
+    for cname, cls in (("fpd_plan", fpd.fpd_plan), ("fpd_decode_args", fpd.fpd_decode_args)):
+        assert seen[(cname, "size")] == ctypes.sizeof(cls), cname
+        for f, _ in cls._fields_:
+            assert seen[(cname, f)] == getattr(cls, f).offset, (cname, f)
