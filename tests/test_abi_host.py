@@ -324,3 +324,39 @@ def test_ctypes_structs_match_the_c_header(tmp_path):
         assert seen[(cname, "size")] == ctypes.sizeof(cls), cname
         for f, _ in cls._fields_:
             assert seen[(cname, f)] == getattr(cls, f).offset, (cname, f)
+
+
+def test_binding_arguments_match_the_header():
+    """Every entry point's ctypes argtypes matches its C prototype: as many
+    arguments, pointers where the header has pointers, and scalars of the
+    header's size and kind (a wrong one would shift or garble later ones)."""
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    with open(os.path.join(root, "include", "fp8_paged_decode.h")) as f:
+        text = re.sub(r"/\*.*?\*/", " ", f.read(), flags=re.S)   # drop comments
+    protos = dict(
+        (m.group(1), m.group(2))
+        for m in re.finditer(r"\b(fp8_paged_decode_\w+)\s*\(([^;{}]*?)\)\s*;", text))
+    lib = fpd.load_library()
+    # C parameter type -> (is a pointer, size in bytes, is a float)
+    scalar = {"int": (4, False), "fpd_status": (4, False), "float": (4, True),
+              "size_t": (8, False), "int64_t": (8, False), "uint32_t": (4, False),
+              "uint64_t": (8, False)}
+    checked = 0
+    for name in fpd.EXPORTED_SYMBOLS:
+        params = protos[name].strip()
+        plist = [] if params in ("", "void") else [x.strip() for x in params.split(",")]
+        argtypes = getattr(lib, name).argtypes
+        assert argtypes is not None, name
+        assert len(argtypes) == len(plist), (name, len(argtypes), len(plist))
+        for decl, at in zip(plist, argtypes):
+            is_ptr = "*" in decl
+            py_ptr = at in (ctypes.c_void_p, ctypes.c_char_p) or hasattr(at, "_type_") and \
+                isinstance(getattr(at, "_type_", None), type)
+            assert is_ptr == py_ptr, (name, decl, at)
+            if not is_ptr:
+                ctype = decl.rsplit(None, 1)[0].replace("const", "").strip()
+                size, is_float = scalar[ctype]
+                assert ctypes.sizeof(at) == size, (name, decl, at)
+                assert (at in (ctypes.c_float, ctypes.c_double)) == is_float, (name, decl, at)
+        checked += 1
+    assert checked == len(fpd.EXPORTED_SYMBOLS)
