@@ -360,3 +360,40 @@ def test_binding_arguments_match_the_header():
                 assert (at in (ctypes.c_float, ctypes.c_double)) == is_float, (name, decl, at)
         checked += 1
     assert checked == len(fpd.EXPORTED_SYMBOLS)
+
+
+def test_planner_invariants_on_random_shapes():
+    """For many random supported shapes and machine sizes, the plan is
+    self-consistent: splits cover every page, whole stages with one head per
+    stage, a grid within the resident slots, a larger offered split size only
+    with fewer items, and a workspace that holds every partial."""
+    import numpy as np
+    rng = np.random.default_rng(2024)
+    for _ in range(3000):
+        Hkv = int(rng.choice([1, 2, 4, 8, 16]))
+        g = int(rng.choice([1, 2, 4, 8, 16]))
+        D = int(rng.choice([64, 128]))
+        bt = int(rng.choice([16, 32, 64]))
+        B = int(rng.integers(1, 300))
+        q_len = int(rng.choice([1, 1, 1, 2, 3, 4, 8]))
+        max_blocks = int(rng.integers(1, 3000))
+        window = int(rng.choice([-1, -1, 0, 5, 128, 4096]))
+        sms, occ = int(rng.choice([132, 148, 160])), int(rng.integers(1, 4))
+        p = fpd.fp8_paged_decode_make_plan_qlen(B, q_len, g * Hkv, Hkv, D, bt, max_blocks,
+                                                window, sms, occ)
+        HB = p["heads_per_stage"]
+        assert HB == (4 if Hkv % 4 == 0 else 1)
+        pages = max_blocks if window < 0 else min(max_blocks, (window + q_len - 1) // bt + 2)
+        assert p["chunk_pages"] >= 1 and p["max_splits"] == -(-pages // p["chunk_pages"])
+        if HB == 1:
+            assert p["chunk_pages"] % (64 // bt) == 0
+        units = B * (Hkv // HB) * p["q_chunks"]
+        assert 1 <= p["ctas"] <= sms * occ
+        assert p["ctas"] <= units * p["max_splits"]
+        a = p["adapt_chunk_pages"]
+        if a:
+            assert a > p["chunk_pages"] and (HB == 4 or a % (64 // bt) == 0)
+            assert p["ctas"] == min(sms * occ, units * -(-pages // a))
+        parts = B * q_len * g * Hkv * p["max_splits"] if p["max_splits"] > 1 else 0
+        assert p["workspace_bytes"] >= 256 + parts * (D + 1) * 4
+        assert p["q_per_item"] * g <= 16 or p["q_per_item"] == 1
