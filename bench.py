@@ -8,8 +8,11 @@ tokens / call time), with % of the measured HBM peak and us/call.
 
 One step = one decode call (the persistent split kernel and, when a sequence spans
 several splits, the combine kernel) over the whole batch
-of the named synthetic workload (default: the Llama-3-8B-shaped decode, B=32,
-Hq=32, Hkv=8, D=128, 16-token pages, lengths U[1024, 8192]).  Inputs are
+of the named synthetic workload (default: the large mixed batch, B=256, Hq=64,
+Hkv=8, D=128, 32-token pages, lognormal lengths of median 2048, window 4096,
+sinks: the largest single-GPU workload).  The same run then measures the other
+four workloads the same way and adds them to the line under "per_config"
+(long context, Llama-3-8B-shaped, sliding window + sinks, tiny).  Inputs are
 resident in HBM; consecutive steps read different replicas of the KV cache so
 that the bytes of one step are not in L2 for the next (replicas x KV bytes >
 2 x L2).  Timing: CUDA events on the launching stream around exactly K steps,
@@ -47,7 +50,9 @@ sys.path.insert(0, ROOT)
 
 METRIC = "KV-read HBM GB/s and % of B200 peak per decode call; µs/call"
 UNIT = "GB/s"
-DEFAULT_CONFIG = "llama3_8b"
+DEFAULT_CONFIG = "large_mixed"
+# measured beside the default workload in the same run (per_config)
+PER_CONFIG_DEFAULT = ("tiny", "llama3_8b", "swa_sinks", "long_context")
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -57,6 +62,10 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--config", default=DEFAULT_CONFIG)
+    ap.add_argument("--per-config", default="",
+                    help="comma-separated workloads measured after the headline one in the same "
+                         "run ('none': only the headline; default: every other workload when "
+                         "the headline is the default E4M3 single-query decode)")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--chunk-pages", type=int, default=0, help="force pages per split (tuning)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -370,13 +379,39 @@ def run_reference(args):
 
 # ---------------------------------------------------------------- native --
 
+def per_config_names(args):
+    """Workloads measured beside the headline one, in the same run: every other
+    configuration when the headline is the default E4M3 single-query decode."""
+    if args.per_config == "none":
+        return []
+    if args.per_config:
+        names = [n for n in args.per_config.split(",") if n]
+    elif args.config == DEFAULT_CONFIG and args.q_len == 1 and args.kv_format == "e4m3":
+        names = list(PER_CONFIG_DEFAULT)
+    else:
+        names = []
+    return [n for n in names if n != args.config]
+
+
+def per_config_entry(line):
+    """The figures of one workload's line that the per-configuration table keeps."""
+    rf = line["roofline"]
+    return {"workload": line["config"]["workload"], "kv_bytes_per_call":
+            line["config"]["kv_bytes_per_call"], "us_per_call": line["us_per_call"],
+            "kv_gbs": line["value"], "pct_of_peak": line["pct_of_peak"],
+            "split_kernel_us": line["split_kernel_us"],
+            "combine_kernel_us": line["combine_kernel_us"],
+            "roofline_frac": rf["frac"], "roofline_traffic": rf["traffic"],
+            "graph_replay_cold_l2": line["graph_replay_cold_l2"], "e2e": line["e2e"],
+            "parity_guard": line["parity_guard"], "clocks": line["clocks"],
+            "steps": line["steps"], "plan": line["config"]["plan"]}
+
+
 def run_native(args):
-    import numpy as np
     import torch
     import torch.distributed as dist
 
     import fp8_paged_decode_b200 as fpd
-    from fp8_paged_decode_b200 import workloads as W
 
     ws, rank, local = dist_env()
     assert ws == args.gpus, f"--gpus {args.gpus} but WORLD_SIZE={ws}"
@@ -390,6 +425,42 @@ def run_native(args):
             dist.barrier()
 
     lib = fpd.load_library()
+    line = measure_native(args, lib, ws, rank, local, barrier)
+    if line is not None and not args.kernels_only:
+        others = per_config_names(args)
+        if others:
+            # every other workload in the same run, the same way (no CPU
+            # baseline: that is quoted once, on the headline workload)
+            table = {args.config: per_config_entry(line)} if rank == 0 else None
+            for name in others:
+                sub_args = argparse.Namespace(**{**vars(args), "config": name,
+                                                 "no_cpu_baseline": True})
+                sub = measure_native(sub_args, lib, ws, rank, local, barrier)
+                if rank == 0:
+                    table[name] = per_config_entry(sub)
+                torch.cuda.empty_cache()
+            if rank == 0:
+                line["per_config"] = table
+        if rank == 0:
+            print(json.dumps(line))
+            if args.json_out:
+                with open(args.json_out, "w") as f:
+                    f.write(json.dumps(line) + "\n")
+    if ws > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def measure_native(args, lib, ws, rank, local, barrier):
+    """One workload: warm-up, K timed calls, the per-kernel event pass, the
+    cold-L2 graph replay and the end-to-end loop.  Returns rank 0's JSON line
+    (a dict; None on other ranks and for --kernels-only)."""
+    import numpy as np
+    import torch
+
+    import fp8_paged_decode_b200 as fpd
+    from fp8_paged_decode_b200 import workloads as W
+
     wl = make_wl(args)
     dev = torch.device("cuda", local)
     props = torch.cuda.get_device_properties(dev)
@@ -470,9 +541,7 @@ def run_native(args):
                               args.warmup + args.steps, "launches_per_call":
                               1 + (1 if plan["max_splits"] > 1 else 0), "plan": plan,
                               "kv_bytes_per_call": kv_bytes, "replicas": replicas}))
-        if ws > 1:
-            dist.destroy_process_group()
-        return 0
+        return None
 
     # correctness guard on this exact launch configuration (sampled rows vs oracle)
     st = f_plain(0)
@@ -768,13 +837,8 @@ def run_native(args):
             "gpu_launches": launches_per_step * K, "clocks": clocks, "parity_guard": guard,
             "graph_replay_cold_l2": graph,
         }
-        print(json.dumps(line))
-        if args.json_out:
-            with open(args.json_out, "w") as f:
-                f.write(json.dumps(line) + "\n")
-    if ws > 1:
-        dist.destroy_process_group()
-    return 0
+        return line
+    return None
 
 
 def run_cache_write(args):

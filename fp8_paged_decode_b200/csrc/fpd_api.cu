@@ -663,9 +663,12 @@ static fpd_status plan_args_impl(const fpd_decode_args& a, fpd_plan* plan) {
   return st;
 }
 
+// zero_header: clear the workspace header (status word, work counters) on the
+// stream right before the launches, once every argument has passed the checks
+// (the allocation-free entry point's shared scratch).
 static fpd_status attention_impl(const fpd_decode_args& a, void* workspace,
                                  size_t workspace_bytes, void* stream, void* ev0, void* ev1,
-                                 void* ev2) {
+                                 void* ev2, bool zero_header = false) {
   const int B = a.B, q_len = a.q_len, Hq = a.Hq, Hkv = a.Hkv, D = a.D, bt = a.block_tokens;
   const int max_blocks = a.max_blocks, num_blocks = a.num_blocks, window_left = a.window_left;
   fpd_status st = validate_shape(B, Hq, Hkv, D, bt, max_blocks, q_len);
@@ -789,6 +792,8 @@ static fpd_status attention_impl(const fpd_decode_args& a, void* workspace,
   p.adapt_chunk = plan.adapt_chunk_pages;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (zero_header && cudaMemsetAsync(workspace, 0, wl.zero_prefix, s) != cudaSuccess)
+    return FPD_ERR_CUDA;
   if (ev0 && cudaEventRecord(static_cast<cudaEvent_t>(ev0), s) != cudaSuccess) return FPD_ERR_CUDA;
   cudaError_t e;
   const int NT = n_tiles(plan.q_per_item * g);
@@ -986,15 +991,14 @@ fpd_status fp8_paged_decode_attention_noalloc(const void* q, const void* k_cache
   if (plan.workspace_bytes > FPD_NOALLOC_SCRATCH_BYTES) return FPD_ERR_WORKSPACE_TOO_SMALL;
   void* scratch = noalloc_scratch_address();
   if (!scratch) return FPD_ERR_CUDA;
-  // the status word and the work counters must start at zero; the partials
-  // are fully rewritten
-  const size_t zero = ws_layout(B, Hq, Hkv, D, plan.max_splits).zero_prefix;
-  if (cudaMemsetAsync(scratch, 0, zero, static_cast<cudaStream_t>(stream)) != cudaSuccess)
-    return FPD_ERR_CUDA;
+  // The status word and the work counters must start at zero (the partials
+  // are fully rewritten): the header is cleared on the stream after every
+  // argument check has passed, so a rejected call enqueues nothing.
   return attention_impl(plain_args(q, k_cache, v_cache, block_table, seq_lens, B, 1, Hq, Hkv, D,
                                    num_blocks, bt, max_blocks, k_scale, v_scale, sm_scale,
                                    window_left, sinks, out, lse, 0),
-                        scratch, FPD_NOALLOC_SCRATCH_BYTES, stream, nullptr, nullptr, nullptr);
+                        scratch, FPD_NOALLOC_SCRATCH_BYTES, stream, nullptr, nullptr, nullptr,
+                        true);
 }
 
 fpd_status fp8_paged_decode_cache_write_layout(const void* key, const void* value,

@@ -380,10 +380,15 @@ fpd_status fp8_paged_decode_attention_profiled(const void *q, const void *k_cach
  *  - Nothing is allocated or freed: no cudaMalloc/cudaFree and no allocating
  *    library routine on any call.
  *  - A shape whose plan needs more scratch than FPD_NOALLOC_SCRATCH_BYTES is
- *    rejected with FPD_ERR_WORKSPACE_TOO_SMALL before anything is launched.
+ *    rejected with FPD_ERR_WORKSPACE_TOO_SMALL, and every other argument error
+ *    with its status, before anything is enqueued on the stream.
  *  - The first call on each device looks up the array's device address on that
  *    device (cudaGetSymbolAddress); make that first call before any stream
  *    capture on the device.  A failed lookup returns FPD_ERR_CUDA.
+ *  - That address is kept for the life of the process.  Do not call this entry
+ *    point on a device after cudaDeviceReset, or after its primary context was
+ *    otherwise destroyed and created again: the library would write through
+ *    the old context's address.
  *  - Every call, on any stream, shares the one array, which keeps the previous
  *    call's contents; each call zeroes the part that must start at zero (the
  *    status word) on its own stream before its kernels.  Calls whose kernels
