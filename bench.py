@@ -616,7 +616,9 @@ def measure_native(args, lib, ws, rank, local, barrier):
     value = whole_job_value(ws, kv_bytes, K, max_total_ms)
 
     # One call captured in a CUDA graph, replayed with the L2 flushed before each
-    # replay (a write of 2x L2 bytes); median and p10/p90 of the replays.
+    # replay: a write of 2x L2 bytes, then a read of the same bytes, so that L2
+    # holds none of the call's data and the flush's dirty lines are written back
+    # before the replay starts, not during it; median and p10/p90 of the replays.
     graph = None
     if not args.no_graph:
         flush = torch.empty(2 * l2 // 4 + 1, dtype=torch.float32, device=dev)
@@ -637,9 +639,11 @@ def measure_native(args, lib, ws, rank, local, barrier):
         with torch.cuda.stream(gstream):
             for i in range(n_warm):
                 flush.fill_(float(i))
+                torch.amax(flush)
                 cg.replay()
             for i in range(n_rep):
                 flush.fill_(float(i))
+                torch.amax(flush)
                 e_a[i].record(gstream)
                 cg.replay()
                 e_b[i].record(gstream)
@@ -648,6 +652,7 @@ def measure_native(args, lib, ws, rank, local, barrier):
         graph = {"median_us": tr[n_rep // 2], "p10_us": tr[n_rep // 10],
                  "p90_us": tr[(9 * n_rep) // 10], "replays": n_rep, "warmup_replays": n_warm,
                  "l2_flush_bytes": int(flush.numel() * 4),
+                 "l2_flush": "write then read of l2_flush_bytes before each replay",
                  "kv_gbs_at_median": kv_bytes / tr[n_rep // 2] / 1e3}
         del cg
         assert fpd.fp8_paged_decode_check_status(wsp, clear=True) == 0
