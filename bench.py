@@ -404,7 +404,7 @@ def per_config_entry(line):
             "roofline_frac": rf["frac"], "roofline_traffic": rf["traffic"],
             "graph_replay_cold_l2": line["graph_replay_cold_l2"], "e2e": line["e2e"],
             "parity_guard": line["parity_guard"], "clocks": line["clocks"],
-            "steps": line["steps"], "plan": line["config"]["plan"]}
+            "steps": line["steps"], "warmup": line["warmup"], "plan": line["config"]["plan"]}
 
 
 def run_native(args):
@@ -429,12 +429,16 @@ def run_native(args):
     if line is not None and not args.kernels_only:
         others = per_config_names(args)
         if others:
-            # every other workload in the same run, the same way (no CPU
-            # baseline: that is quoted once, on the headline workload)
+            # every other workload in the same run, the same way, with at
+            # least 2000 timed calls after 50 warm-up calls (short workloads
+            # need that many to leave the launch ramp; the entries record
+            # their counts), and no CPU baseline (quoted once, on the headline)
             table = {args.config: per_config_entry(line)} if rank == 0 else None
             for name in others:
                 sub_args = argparse.Namespace(**{**vars(args), "config": name,
-                                                 "no_cpu_baseline": True})
+                                                 "no_cpu_baseline": True,
+                                                 "steps": max(args.steps, 2000),
+                                                 "warmup": max(args.warmup, 50)})
                 sub = measure_native(sub_args, lib, ws, rank, local, barrier)
                 if rank == 0:
                     table[name] = per_config_entry(sub)
