@@ -347,8 +347,8 @@ bool encode_nvfp4_map(CUtensorMap* map, const void* base, int num_blocks, int bt
 
 // Combine launch as a programmatic dependent of the split kernel: its CTAs may
 // start while the split kernel drains and wait for it on the device.
-template <int D, bool MQ>
-cudaError_t launch_combine(const fpd::CombineParams& c, cudaStream_t st) {
+template <int D, bool MQ, int NB>
+cudaError_t launch_combine_nb(const fpd::CombineParams& c, cudaStream_t st) {
   const int rows_per_cta = c.rows_per_cta;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)((c.B * c.q_len * c.Hq + rows_per_cta - 1) / rows_per_cta));
@@ -360,7 +360,23 @@ cudaError_t launch_combine(const fpd::CombineParams& c, cudaStream_t st) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, fpd::fpd_combine_kernel<D, MQ>, c);
+  return cudaLaunchKernelEx(&cfg, fpd::fpd_combine_kernel<D, MQ, NB>, c);
+}
+
+// The first-round batch: one warp per row loads min(max_splits, 8) partials.
+template <int D, bool MQ>
+cudaError_t launch_combine(const fpd::CombineParams& c, cudaStream_t st) {
+  if (c.wpr > 1) return launch_combine_nb<D, MQ, fpd::kCombineBatch>(c, st);
+  switch (c.max_splits) {
+    case 1: return launch_combine_nb<D, MQ, 1>(c, st);
+    case 2: return launch_combine_nb<D, MQ, 2>(c, st);
+    case 3: return launch_combine_nb<D, MQ, 3>(c, st);
+    case 4: return launch_combine_nb<D, MQ, 4>(c, st);
+    case 5: return launch_combine_nb<D, MQ, 5>(c, st);
+    case 6: return launch_combine_nb<D, MQ, 6>(c, st);
+    case 7: return launch_combine_nb<D, MQ, 7>(c, st);
+    default: return launch_combine_nb<D, MQ, fpd::kCombineBatch>(c, st);
+  }
 }
 
 // The split kernel is launched as a programmatic dependent of whatever ran

@@ -1454,8 +1454,17 @@ constexpr int kCombineBatch = 8;   // partials a warp loads before it reduces th
 // one round trip to memory.  Each warp reduces against its own maximum; the
 // row's warps are combined in shared memory.  MQ: several queries per
 // sequence, where a split may hold no key of a query (its lse is -inf).
-template <int D, bool MQ>
-__global__ void __launch_bounds__(kCombineMaxThreads) fpd_combine_kernel(const CombineParams p) {
+// NB: the partials each warp loads in its first round, min(max_splits, 8) for
+// one warp per row (256-thread CTAs; a call with few splits then holds fewer
+// registers and fits more CTAs per SM), kCombineBatch otherwise.
+template <int NB>
+struct CombineBounds {
+  static constexpr int threads = NB < kCombineBatch ? 256 : kCombineMaxThreads;
+  static constexpr int min_blocks = NB <= 4 ? 6 : (NB <= 6 ? 5 : 1);
+};
+template <int D, bool MQ, int NB = kCombineBatch>
+__global__ void __launch_bounds__(CombineBounds<NB>::threads, CombineBounds<NB>::min_blocks)
+fpd_combine_kernel(const CombineParams p) {
   constexpr int kMaxWarps = kCombineMaxThreads / 32;
   __shared__ float acc_sm[kMaxWarps][D];
   __shared__ float z_sm[kMaxWarps], m_sm[kMaxWarps];
@@ -1476,10 +1485,10 @@ __global__ void __launch_bounds__(kCombineMaxThreads) fpd_combine_kernel(const C
   const int L_raw = in_range ? p.seq_lens[row / (QL * p.Hq)] : 0;
   const int chunk = (int)*p.chunk_word;
   const float v_scale = p.v_scale_dev ? *p.v_scale_dev : p.v_scale;
-  float lv[kCombineBatch];
-  float x[kCombineBatch][PER];
+  float lv[NB];
+  float x[NB][PER];
 #pragma unroll
-  for (int u = 0; u < kCombineBatch; ++u) {
+  for (int u = 0; u < NB; ++u) {
     const int s = j + wpr * u;
     lv[u] = -INFINITY;
 #pragma unroll
@@ -1508,10 +1517,10 @@ __global__ void __launch_bounds__(kCombineMaxThreads) fpd_combine_kernel(const C
   for (int i = 0; i < PER; ++i) acc[i] = 0.f;
   if (active) {
 #pragma unroll
-    for (int u = 0; u < kCombineBatch; ++u)
+    for (int u = 0; u < NB; ++u)
       if (j + wpr * u < ns) m = fmaxf(m, lv[u]);
 #pragma unroll
-    for (int u = 0; u < kCombineBatch; ++u) {
+    for (int u = 0; u < NB; ++u) {
       // never touch unused (possibly stale) entries; -inf: no key of the query there
       if (j + wpr * u < ns && (!MQ || lv[u] != -INFINITY)) {
         const float w = fast_exp2(lv[u] - m);
@@ -1520,8 +1529,8 @@ __global__ void __launch_bounds__(kCombineMaxThreads) fpd_combine_kernel(const C
         for (int i = 0; i < PER; ++i) acc[i] = fmaf(w, x[u][i], acc[i]);
       }
     }
-    // splits beyond the first batch (more than wpr * kCombineBatch of them)
-    for (int s = j + wpr * kCombineBatch; s < ns; s += wpr) {
+    // splits beyond the first batch (more than wpr * NB of them)
+    for (int s = j + wpr * NB; s < ns; s += wpr) {
       const float l = pl[s];
       float v[PER];
       if constexpr (PER == 4) {

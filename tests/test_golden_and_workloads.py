@@ -76,3 +76,34 @@ def test_kernel_hash_ignores_comments_only():
     assert bench._code_lines(src) == 'int a = 1;\nasm("x // y");\nint b = 2;'
     assert bench._code_lines(src.replace("// one", "// uno")) == bench._code_lines(src)
     assert bench._code_lines(src.replace("b = 2", "b = 3")) != bench._code_lines(src)
+
+
+def test_bench_per_config_selection():
+    """The default E4M3 single-query run measures every other workload after the
+    headline; an explicit list or "none" overrides that; other runs measure the
+    headline alone."""
+    import argparse
+    import bench
+    base = dict(config=bench.DEFAULT_CONFIG, q_len=1, kv_format="e4m3", per_config="")
+    ns = lambda **kw: argparse.Namespace(**{**base, **kw})   # noqa: E731
+    others = bench.per_config_names(ns())
+    assert bench.DEFAULT_CONFIG == "large_mixed" and bench.DEFAULT_CONFIG not in others
+    assert sorted(others + [bench.DEFAULT_CONFIG]) == sorted(
+        ["tiny", "llama3_8b", "swa_sinks", "long_context", "large_mixed"])
+    assert bench.per_config_names(ns(per_config="none")) == []
+    assert bench.per_config_names(ns(per_config="tiny,large_mixed")) == ["tiny"]
+    assert bench.per_config_names(ns(q_len=4)) == []
+    assert bench.per_config_names(ns(kv_format="nvfp4")) == []
+    assert bench.per_config_names(ns(config="llama3_8b")) == []
+
+
+def test_bench_per_config_entry_keeps_both_timing_forms():
+    import bench
+    line = {"config": {"workload": "w", "kv_bytes_per_call": 10, "plan": {"ctas": 1}},
+            "us_per_call": 2.0, "value": 5.0, "pct_of_peak": 1.0, "split_kernel_us": 1.5,
+            "combine_kernel_us": 0.5, "roofline": {"frac": 0.5, "traffic": None},
+            "graph_replay_cold_l2": {"median_us": 3.0}, "e2e": {"value": 4.0},
+            "parity_guard": {"ok": True}, "clocks": {"sm_mhz": 1}, "steps": 20, "warmup": 5}
+    e = bench.per_config_entry(line)
+    assert e["us_per_call"] == 2.0 and e["graph_replay_cold_l2"]["median_us"] == 3.0
+    assert e["roofline_frac"] == 0.5 and e["e2e"]["value"] == 4.0 and e["steps"] == 20
