@@ -1460,7 +1460,7 @@ constexpr int kCombineBatch = 8;   // partials a warp loads before it reduces th
 template <int NB>
 struct CombineBounds {
   static constexpr int threads = NB < kCombineBatch ? 256 : kCombineMaxThreads;
-  static constexpr int min_blocks = NB <= 4 ? 6 : (NB <= 6 ? 5 : 1);
+  static constexpr int min_blocks = NB <= 4 ? 6 : (NB <= 6 ? 5 : (NB < kCombineBatch ? 4 : 1));
 };
 template <int D, bool MQ, int NB = kCombineBatch>
 __global__ void __launch_bounds__(CombineBounds<NB>::threads, CombineBounds<NB>::min_blocks)
