@@ -28,6 +28,16 @@ constexpr size_t kHeaderBytes = 256;    // status word, work counter, finished-C
 // larger items.
 constexpr int kTargetWaves1 = 8, kMinChunkRows1 = 256;    // one KV head per stage
 constexpr int kTargetWaves4 = 5, kMinChunkRows4 = 1024;   // four KV heads per stage
+// Four-head items over E4M3 pages of at least this many tokens at
+// kTargetWaves4 rounds take one round fewer: long items carry little fixed
+// cost per token, and fewer splits leave the combine kernel fewer partials to
+// merge (measured: large mixed batch 26 -> 33 pages 206.3 -> 202.5 us and
+// 213.0 -> 210.1 us on two boxes, long context 8 -> 10 pages 175.6 -> 173.7
+// us on one and equal on the other; the Llama-3-8B-shaped call, 256-token
+// items, keeps its 16 pages: 19 pages took 64.4 instead of 60.5 us).  NVFP4
+// pages keep kTargetWaves4: their kernel is bound by instruction issue, and
+// the larger items lengthened its tail (long context 155.3 -> 168.6 us).
+constexpr int kLongItemTokens4 = 512;
 constexpr int kMinItemTokens = 48;   // shortest split when a call cannot fill the machine
 constexpr int kOccCacheSize = 32;
 
@@ -470,9 +480,13 @@ void plan_shape(int B, int q_len, int Hq, int Hkv, int D, int bt, int max_blocks
   } else {
     const int waves = HB == 1 ? kTargetWaves1 : kTargetWaves4;
     const int min_rows = HB == 1 ? kMinChunkRows1 : kMinChunkRows4;
-    int64_t splits = (waves * slots + units - 1) / units;
-    if (splits < 1) splits = 1;
-    chunk = round_pps((pages_max + splits - 1) / splits);
+    const auto chunk_for = [&](int w) {
+      int64_t splits = (w * slots + units - 1) / units;
+      if (splits < 1) splits = 1;
+      return round_pps((int)((pages_max + splits - 1) / splits));
+    };
+    chunk = chunk_for(waves);
+    if (HB == 4 && !fp4 && (int64_t)chunk * bt >= kLongItemTokens4) chunk = chunk_for(waves - 1);
     const int min_chunk = round_pps(((int64_t)min_rows / HB + bt - 1) / bt);
     if (chunk < min_chunk) {
       // Too few pages for `waves` rounds of items of the minimum size.  Such

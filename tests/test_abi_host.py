@@ -62,8 +62,9 @@ def test_planner_fills_the_machine():
         assert p["heads_per_stage"] == 4 and p["stage_tokens"] == 16
         units = shape["B"] * shape["Hkv"] // 4
         assert p["ctas"] == min(296, units * p["max_splits"]) == 296
-        # enough work items for several per slot on long inputs
-        assert units * p["max_splits"] >= 4 * 296
+        # enough work items for several per slot on long inputs (about 4 rounds
+        # when the items are long, 5 otherwise)
+        assert units * p["max_splits"] >= 3 * 296
         # at least 256 (token, KV head) rows per work item
         assert p["chunk_pages"] * shape["block_tokens"] * 4 >= 256
 
