@@ -102,20 +102,16 @@ def test_unsupported_q_len():
     assert e.value.status == fpd.FPD_ERR_UNSUPPORTED
 
 
-def test_llama_shape_speculative():
-    """Llama-3-8B-shaped batch with 4 draft tokens per sequence, sampled rows."""
-    rng = np.random.default_rng(63)
-    lens = rng.integers(1024, 8193, 32)
-    wl = W.make_custom(B=32, Hq=32, Hkv=8, D=128, block_tokens=16, seq_lens=lens, seed=64,
-                       q_len=4, name="llama3_8b-q4")
-    rows = rng.choice(32 * 4 * 32, 48, replace=False)
-    ref_out, ref_lse = oracle.decode_workload(wl, rows=rows)
+@pytest.mark.parametrize("name,Q", [("llama3_8b", 4), ("large_mixed", 2)])
+def test_full_workload_speculative_every_row(name, Q):
+    """The full-size workloads with Q draft tokens per sequence (the bench's
+    `--q-len Q` calls): every (sequence, query, head) row against the oracle in
+    the default launch configuration."""
+    wl = W.make_workload(name, q_len=Q)
+    ref_out, ref_lse = oracle.decode_workload(wl)
     out, lse = run_cuda(wl)
-    B, Q = wl.B, wl.q_len
-    bi, rest = np.divmod(rows, Q * wl.Hq)
-    qi, hi = np.divmod(rest, wl.Hq)
-    assert_parity(out[bi, qi, hi][None], lse[bi, qi, hi][None], ref_out[bi, qi, hi][None],
-                  ref_lse[bi, qi, hi][None], what="llama shape q_len=4")
+    assert out.shape == ref_out.shape == (wl.B, Q, wl.Hq, wl.D)
+    assert_parity(out, lse, ref_out, ref_lse, what=f"{name} q_len={Q}, every row")
 
 
 @pytest.mark.parametrize("g,Hkv", [(1, 4), (16, 1)])

@@ -85,13 +85,13 @@ def test_no_sinks_and_empty_sequence():
     check(wl, chunk=1)
 
 
-def test_llama_shape_sampled():
-    """The Llama-3-8B-shaped workload over NVFP4 pages in the bench's launch
-    configuration; the oracle computes a sample of rows."""
-    wl = W.make_workload_nvfp4("llama3_8b")
-    rng = np.random.default_rng(612)
-    rows = rng.choice(wl.B * wl.Hq, 64, replace=False)
-    check(wl, rows=rows, what="llama3_8b NVFP4 sampled")
+@pytest.mark.parametrize("name", ["llama3_8b", "long_context", "large_mixed"])
+def test_full_workload_every_row(name):
+    """Every (sequence, head) row of the full-size workloads over NVFP4 pages
+    against the oracle, in the bench's launch configuration (the default plan),
+    with the block scales of every slot the decode must not read set to the
+    NaN code."""
+    check(W.make_workload_nvfp4(name), what=f"{name} NVFP4, every row")
 
 
 def test_invalid_page_flagged():
