@@ -98,6 +98,9 @@ int heads_per_stage(int Hkv) { return Hkv % 4 == 0 ? 4 : 1; }
 #ifndef FPD_STAGES_HB4_D64
 #define FPD_STAGES_HB4_D64 5
 #endif
+#ifndef FPD_STAGES_HB4_D128_NT2
+#define FPD_STAGES_HB4_D128_NT2 4
+#endif
 // NVFP4 stages are 72 D bytes instead of 128 D: the ring keeps about the same
 // bytes in flight with 16 / 9 as many stages.
 #ifndef FPD_FP4_STAGES_NUM
@@ -108,7 +111,8 @@ int heads_per_stage(int Hkv) { return Hkv % 4 == 0 ? 4 : 1; }
 #endif
 int ring_stages(int D, int NT, int HB, bool fp4 = false) {
   int s;
-  if (HB == 4) s = D == 128 ? FPD_STAGES_HB4_D128 : FPD_STAGES_HB4_D64;
+  if (HB == 4)
+    s = D == 128 ? (NT == 2 ? FPD_STAGES_HB4_D128_NT2 : FPD_STAGES_HB4_D128) : FPD_STAGES_HB4_D64;
   else if (D == 128) s = NT == 2 ? FPD_STAGES_D128_NT2 : FPD_STAGES_D128_NT1;
   else s = FPD_STAGES_D64;
   return fp4 ? s * FPD_FP4_STAGES_NUM / FPD_FP4_STAGES_DEN : s;

@@ -130,8 +130,20 @@ __host__ __device__ constexpr int hdr_slot_bytes(int D, int HB, int g) {
 // the host to size the launch and by the kernel to find its buffers.  Only
 // HB = 1 needs the merge buffer.
 struct SmemLayout {
-  int ring, merge, hdr, prefix, bars, total;
+  int ring, merge, qfrag, hdr, prefix, bars, total;
 };
+
+// Query fragments kept in shared memory instead of registers (D = 128 with two
+// n-tiles: their 32 registers per thread would otherwise spill at the 2-CTA
+// register cap).
+#ifndef FPD_QFRAG_SMEM
+#define FPD_QFRAG_SMEM 1
+#endif
+__host__ __device__ constexpr bool qfrag_in_smem(int D, int NT) {
+  return FPD_QFRAG_SMEM && D == 128 && NT == 2;
+}
+// Bytes of one consumer warp's query fragments: [NT][D/16 k-steps][32 lanes][2 words].
+__host__ __device__ constexpr int qfrag_warp_bytes(int D, int NT) { return NT * (D / 16) * 32 * 8; }
 
 __host__ __device__ constexpr int align_to(int x, int a) { return (x + a - 1) / a * a; }
 
@@ -168,7 +180,9 @@ __host__ __device__ inline SmemLayout smem_layout(int D, int NT, int HB, int sta
   L.merge = stages * stage_bytes(D, fp4);
   const int merge_bytes =
       HB == 1 ? kConsumerWarps * H * (D + 4) * 4 + kConsumerWarps * H * 2 * 4 : 0;
-  L.hdr = align_to(L.merge + merge_bytes, 128);
+  L.qfrag = align_to(L.merge + merge_bytes, 16);
+  const int qfrag_bytes = qfrag_in_smem(D, NT) ? kConsumerWarps * qfrag_warp_bytes(D, NT) : 0;
+  L.hdr = align_to(L.qfrag + qfrag_bytes, 128);
   L.prefix = align_to(L.hdr + hdr_slots * hdr_slot_bytes(D, HB, g), 16);
   L.bars = align_to(L.prefix + 4 * (B + 1), 16);
   L.total = align_to(L.bars + (2 * stages + 2 * kMaxHdrSlots + 1) * 8, 16) +
@@ -305,7 +319,11 @@ struct Consumer {
 
   uint32_t koff[D / 64];    // swizzled byte offsets of this thread's K reads (row n)
   uint32_t voff[2];         // swizzled byte offsets of its V reads (rows 2t, 2t + 1)
-  uint32_t qf[NT][KS][2];   // Q^T B fragments (f16x2), head = lane / 4 of n-tile
+  // Q^T B fragments (f16x2), head = lane / 4 of n-tile: in registers, or (QSM)
+  // in this warp's shared-memory area qs, [nt][ks][lane][2]
+  static constexpr bool QSM = qfrag_in_smem(D, NT);
+  uint32_t qf[QSM ? 1 : NT][QSM ? 1 : KS][2];
+  uint32_t* qs;
   float cs[NT][2];          // logit scale (log2) of this thread's C columns
   float m[NT][2];           // running max (log2 domain) of this thread's columns
   float thr[NT][2];         // raw-accumulator threshold that triggers a rescale
@@ -381,8 +399,14 @@ struct Consumer {
       const float fac = ldexpf(1.0f, sh);
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
-        qf[nt][ks][0] = pack_f16x2(vals[4 * ks] * fac, vals[4 * ks + 1] * fac);
-        qf[nt][ks][1] = pack_f16x2(vals[4 * ks + 2] * fac, vals[4 * ks + 3] * fac);
+        const uint32_t w0 = pack_f16x2(vals[4 * ks] * fac, vals[4 * ks + 1] * fac);
+        const uint32_t w1 = pack_f16x2(vals[4 * ks + 2] * fac, vals[4 * ks + 3] * fac);
+        if constexpr (QSM) {
+          *reinterpret_cast<uint2*>(qs + ((nt * KS + ks) * 32 + lane) * 2) = make_uint2(w0, w1);
+        } else {
+          qf[nt][ks][0] = w0;
+          qf[nt][ks][1] = w1;
+        }
       }
       // this thread's C columns are columns 2t and 2t+1 of the n-tile; the
       // prescale is a power of two, so undoing it is an exact multiply
@@ -547,7 +571,16 @@ struct Consumer {
       }
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
-        mma_16816(s[nt][ks & 1], a0, a1, a2, a3, qf[nt][ks][0], qf[nt][ks][1]);
+      {
+        uint32_t b0, b1;
+        if constexpr (QSM) {
+          const uint2 w = *reinterpret_cast<const uint2*>(qs + ((nt * KS + ks) * 32 + lane) * 2);
+          b0 = w.x, b1 = w.y;
+        } else {
+          b0 = qf[nt][ks][0], b1 = qf[nt][ks][1];
+        }
+        mma_16816(s[nt][ks & 1], a0, a1, a2, a3, b0, b1);
+      }
     }
     float acc[NT][4];
 #pragma unroll
@@ -1045,9 +1078,13 @@ __device__ __forceinline__ void producer_loop(const CUtensorMap* kmap, const CUt
 #ifndef FPD_MINB_D128_NT1
 #define FPD_MINB_D128_NT1 3
 #endif
+#ifndef FPD_MINB_D128_NT2
+#define FPD_MINB_D128_NT2 2
+#endif
 template <int D, int NT>
 struct MinBlocks {
-  static constexpr int value = (D == 128) ? (NT == 1 ? FPD_MINB_D128_NT1 : 2) : (NT == 1 ? 4 : 3);
+  static constexpr int value =
+      (D == 128) ? (NT == 1 ? FPD_MINB_D128_NT1 : FPD_MINB_D128_NT2) : (NT == 1 ? 4 : 3);
 };
 
 // The split kernel's body.  FP4: NVFP4 pages (kmap / vmap the E2M1 data,
@@ -1151,6 +1188,7 @@ __device__ __forceinline__ void split_body(const CUtensorMap* kmap, const CUtens
   uint32_t cpar = 0;
   bool alive = true;
   cw.setup(row0, lane);
+  cw.qs = reinterpret_cast<uint32_t*>(smem + L.qfrag + warp * qfrag_warp_bytes(D, NT));
   for (;;) {
     if (!__all_sync(0xffffffffu, mbar_wait_bounded(&hdr_full[hslot], hphase, kWaitLimitNs))) {
       alive = false;
