@@ -204,6 +204,12 @@ struct ItemHeader {
 };
 static_assert(sizeof(ItemHeader) == kHdrBytes, "header size");
 
+// x / d for x >= 0 and d >= 1 (both the same across the warp): a shift when d
+// is a power of two (page sizes, head groups), else the division.
+__device__ __forceinline__ int div_pos(int x, int d) {
+  return (d & (d - 1)) == 0 ? x >> (__ffs(d) - 1) : x / d;
+}
+
 // Attended page range of a sequence.
 struct SeqRange {
   int L, start, first_page, end_page, n_splits;
@@ -223,10 +229,10 @@ __device__ __forceinline__ SeqRange seq_range(int L_raw, int q_len, int bt, int 
   }
   r.L = L;
   r.start = (window_left >= 0) ? max(0, L - q_len - window_left) : 0;
-  r.first_page = r.start / bt;
-  r.end_page = (L + bt - 1) / bt;
+  r.first_page = div_pos(r.start, bt);
+  r.end_page = div_pos(L + bt - 1, bt);
   const int n_pages = r.end_page - r.first_page;
-  r.n_splits = (n_pages + chunk_pages - 1) / chunk_pages;
+  r.n_splits = div_pos(n_pages + chunk_pages - 1, chunk_pages);
   return r;
 }
 
@@ -237,47 +243,94 @@ __device__ __forceinline__ int groups_of(int L_raw, int q_len, const DecodeParam
   return r.n_splits > 0 ? r.n_splits : 1;
 }
 
-// Prefix over the sequences of their work groups at split size `chunk`
-// (every CTA builds its own: prefix[b] groups come before sequence b).  Every
-// thread of the block takes part.  MOST: also return the most groups of one
-// sequence.  AGAIN: an earlier pass may still be reading `red`.
-// red: 2 * kThreads / 32 ints of shared memory.
-template <bool MOST, bool AGAIN>
-__device__ __forceinline__ int build_prefix(const DecodeParams& p, int q_len, int chunk,
-                                            int* prefix, int* red) {
-  constexpr int kWarps = kThreads / 32;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int per = (p.B + kThreads - 1) / kThreads;
-  const int b0 = min(p.B, tid * per), b1 = min(p.B, b0 + per);
+// The producer warp builds the call's work list itself (no other warp needs
+// it): the prefix over sequences of their work groups, prefix[b] groups before
+// sequence b, in shared memory.  Every CTA builds the same one.
+struct WorkPrefix {
+  int total;       // work groups of the call
+  int first_b;     // sequence of the CTA's first work group (-1: none)
+  int first_len;   // its length
+};
+
+// Lane l of the producer warp owns sequences [l * per, (l + 1) * per) with
+// per = ceil(B / 32): it loads their lengths, sums their work groups and
+// writes their prefix entries; one warp scan joins the lanes.  Only the loads
+// are unrolled: the code runs once per call, often from cold caches.
+__device__ __forceinline__ void lane_range(const DecodeParams& p, int lane, int& b0, int& b1) {
+  const int per = (p.B + 31) / 32;
+  b0 = min(p.B, lane * per);
+  b1 = min(p.B, b0 + per);
+}
+
+// Stages the sequence lengths in prefix[1..B] (each lane's loads back to back).
+__device__ __forceinline__ void stage_lengths(const DecodeParams& p, int* prefix, int lane) {
+  int b0, b1;
+  lane_range(p, lane, b0, b1);
+#pragma unroll 8
+  for (int b = b0; b < b1; ++b) prefix[b + 1] = __ldg(p.seq_lens + b);
+}
+
+// From the staged lengths at split size `chunk`: all work groups, and the
+// most of one sequence.
+__device__ __forceinline__ void length_totals(const DecodeParams& p, int q_len, int chunk,
+                                              const int* prefix, int lane, int& total,
+                                              int& most) {
+  int b0, b1;
+  lane_range(p, lane, b0, b1);
   int sum = 0, mx = 0;
+#pragma unroll 1
   for (int b = b0; b < b1; ++b) {
-    const int g = groups_of(__ldg(p.seq_lens + b), q_len, p, chunk);
+    const int g = groups_of(prefix[b + 1], q_len, p, chunk);
     sum += g;
-    if (MOST) mx = max(mx, g);
+    mx = max(mx, g);
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  total = sum;
+  most = mx;
+}
+
+// Replaces the staged lengths by the prefix at split size `chunk` and finds
+// the sequence that holds work group `first_group`.
+__device__ __forceinline__ WorkPrefix build_prefix(const DecodeParams& p, int q_len, int chunk,
+                                                   int* prefix, int lane, int first_group) {
+  int b0, b1;
+  lane_range(p, lane, b0, b1);
+  int sum = 0;
+#pragma unroll 1
+  for (int b = b0; b < b1; ++b) sum += groups_of(prefix[b + 1], q_len, p, chunk);
   int incl = sum;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const int v = __shfl_up_sync(0xffffffffu, incl, o);
     if (lane >= o) incl += v;
-    if (MOST) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   }
-  if (AGAIN) __syncthreads();
-  if (lane == 31) red[warp] = incl;
-  if (MOST && lane == 0) red[kWarps + warp] = mx;
-  __syncthreads();
   int run = incl - sum;
-  for (int w = 0; w < warp; ++w) run += red[w];
-  if (tid == 0) prefix[0] = 0;
+  int fb = -1, fl = 0;
+#pragma unroll 1
   for (int b = b0; b < b1; ++b) {
-    run += groups_of(__ldg(p.seq_lens + b), q_len, p, chunk);
+    const int Lb = prefix[b + 1];
+    const int before = run;
+    run += groups_of(Lb, q_len, p, chunk);
+    if (before <= first_group && first_group < run) {
+      fb = b;
+      fl = Lb;
+    }
     prefix[b + 1] = run;
   }
-  int most = 0;
-  if (MOST)
-    for (int w = 0; w < kWarps; ++w) most = max(most, red[kWarps + w]);
-  __syncthreads();   // the prefix is complete
-  return most;
+  WorkPrefix w{__shfl_sync(0xffffffffu, incl, 31), -1, 0};
+  const unsigned own = __ballot_sync(0xffffffffu, fb >= 0);
+  if (own) {
+    const int src = __ffs(own) - 1;
+    w.first_b = __shfl_sync(0xffffffffu, fb, src);
+    w.first_len = __shfl_sync(0xffffffffu, fl, src);
+  }
+  if (lane == 0) prefix[0] = 0;
+  __syncwarp();   // the prefix is complete for the whole warp
+  return w;
 }
 
 // Byte offset inside a 1024-byte-aligned tile written by TMA with 128-byte
@@ -826,7 +879,8 @@ __device__ __forceinline__ void producer_loop(const CUtensorMap* kmap, const CUt
                                               const SmemLayout& L, const int* prefix,
                                               int chunk, int total_items, int hslot_bytes,
                                               uint64_t* full_bar, uint64_t* empty_bar,
-                                              uint64_t* hdr_full, uint64_t* hdr_empty, int lane) {
+                                              uint64_t* hdr_full, uint64_t* hdr_empty, int lane,
+                                              WorkPrefix first) {
   constexpr int kTileBytes = kTileTokens * D;
   constexpr int kStage = stage_bytes(D, FP4);
   constexpr int kDataBytes = fp4_data_bytes(D);   // NVFP4 regions of a stage
@@ -858,8 +912,6 @@ __device__ __forceinline__ void producer_loop(const CUtensorMap* kmap, const CUt
   uint32_t item = blockIdx.x;
   for (;;) {
     const bool done = item >= (uint32_t)total_items;
-    uint32_t next = 0;
-    if (!done && lane == 0) next = gridDim.x + atomicAdd(&p.sched[0], 1u);   // latency hidden below
     if (hs >= n_hslots) {
       const bool ok = mbar_wait_bounded(&hdr_empty[hslot], hphase ^ 1u, kWaitLimitNs);
       if (!__all_sync(0xffffffffu, ok)) {
@@ -879,19 +931,23 @@ __device__ __forceinline__ void producer_loop(const CUtensorMap* kmap, const CUt
     // item -> (group, kv head group, query chunk) -> (sequence, split) by
     // binary search.  The query chunks of one KV range are consecutive items,
     // so they run at about the same time and share the pages in L2.
-    const int unit = MQ ? (int)item / QC : (int)item;
+    const int unit = MQ ? div_pos((int)item, QC) : (int)item;
     const int qc = MQ ? (int)item - unit * QC : 0;
-    const int group = unit / groups;
-    const int kvh0 = (unit % groups) * HB;
-    int lo = 0, hi = p.B;   // largest b with prefix[b] <= group
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (prefix[mid] <= group) lo = mid; else hi = mid;
+    const int group = div_pos(unit, groups);
+    const int kvh0 = (unit - group * groups) * HB;
+    int b = first.first_b;   // the first item's sequence came with the prefix
+    if (hs > 0) {
+      int lo = 0, hi = p.B;   // largest b with prefix[b] <= group
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (prefix[mid] <= group) lo = mid; else hi = mid;
+      }
+      b = lo;
     }
-    const int b = lo;
     const int split = group - prefix[b];
-    const SeqRange R = seq_range(__ldg(p.seq_lens + b), QL, p.bt, p.max_blocks,
-                                 p.window_left, chunk, lane == 0 ? p.status : nullptr);
+    const SeqRange R = seq_range(hs > 0 ? __ldg(p.seq_lens + b) : first.first_len, QL, p.bt,
+                                 p.max_blocks, p.window_left, chunk,
+                                 lane == 0 ? p.status : nullptr);
     int pb = 0, pe = 0, tok_lo = 0, tok_hi = 0, t0 = 0, n_st = 0;
     if (R.n_splits > 0) {
       pb = R.first_page + split * chunk;
@@ -935,6 +991,11 @@ __device__ __forceinline__ void producer_loop(const CUtensorMap* kmap, const CUt
       hslot = 0;
       hphase ^= 1u;
     }
+
+    // the next item: fetched once this item's first loads are on their way
+    // (its latency is hidden behind the item's stages)
+    uint32_t next = 0;
+    bool fetched = false;
 
     // ---- stream the item's KV; block-table entries 32 at a time
     const int32_t* tbl = p.block_table + (size_t)b * p.max_blocks;
@@ -983,7 +1044,7 @@ __device__ __forceinline__ void producer_loop(const CUtensorMap* kmap, const CUt
         // NVFP4, 16 tokens of 4 heads: lanes 0..3 load K data, K scales, V
         // data, V scales of the block
         const int tok = t0 + s * kBoxTokens;
-        const int rel = tok / p.bt - pb;
+        const int rel = div_pos(tok, p.bt) - pb;
         if ((rel & ~31) != batch_base) {
           batch_base = rel & ~31;
           const int idx = pb + batch_base + lane;
@@ -1036,7 +1097,7 @@ __device__ __forceinline__ void producer_loop(const CUtensorMap* kmap, const CUt
       } else {
         // 16 tokens of HB heads: one box per tensor, lane 0 K and lane 1 V
         const int tok = t0 + s * kBoxTokens;
-        const int rel = tok / p.bt - pb;
+        const int rel = div_pos(tok, p.bt) - pb;
         if ((rel & ~31) != batch_base) {
           batch_base = rel & ~31;
           const int idx = pb + batch_base + lane;
@@ -1067,7 +1128,12 @@ __device__ __forceinline__ void producer_loop(const CUtensorMap* kmap, const CUt
         slot = 0;
         phase ^= 1u;
       }
+      if (!fetched) {
+        if (lane == 0) next = gridDim.x + atomicAdd(&p.sched[0], 1u);
+        fetched = true;
+      }
     }
+    if (!fetched && lane == 0) next = gridDim.x + atomicAdd(&p.sched[0], 1u);
     item = __shfl_sync(0xffffffffu, next, 0);
   }
 }
@@ -1094,7 +1160,6 @@ __device__ __forceinline__ void split_body(const CUtensorMap* kmap, const CUtens
                                            const CUtensorMap* ksmap, const CUtensorMap* vsmap,
                                            const DecodeParams& p) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ int warp_tot[2 * (kThreads / 32)];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   constexpr int kTileBytes = kTileTokens * D;
@@ -1121,8 +1186,8 @@ __device__ __forceinline__ void split_body(const CUtensorMap* kmap, const CUtens
   // The launch may be a programmatic dependent of the previous kernel in the
   // stream (so that this grid's CTAs are resident when it finishes): nothing
   // is read before that kernel has completed and its writes are visible.
-  pdl_wait_primary();
-
+  // (The barriers live in this CTA's shared memory: they are set up while that
+  // kernel may still run.)
   if (tid == 0) {
     for (int s = 0; s < stages; ++s) {
       mbar_init(&full_bar[s], 1);
@@ -1133,38 +1198,38 @@ __device__ __forceinline__ void split_body(const CUtensorMap* kmap, const CUtens
       mbar_init(&hdr_empty[s], kConsumerWarps);
     }
     mbar_init(cbar, kConsumerWarps);
-    fence_mbarrier_init();   // visible to the block after build_prefix's barriers
+    fence_mbarrier_init();
   }
-
-  // ---- the split size and the prefix over sequences of their work groups.
-  // The plan may offer a larger split size for calls of a few rounds of
-  // items: taken when the sequences are of about equal length (the longest
-  // one's groups times B within 4/3 of all groups), since then its items, one
-  // round of about two per SM, fill every SM alike; otherwise the plan's size
-  // runs over the grid, sized for the larger items.  Every CTA reaches the
-  // same choice from the same lengths.
-  const int G = (p.Hkv / HB) * (MQ ? p.q_chunks : 1);   // items per work group
-  int chunk = p.chunk_pages;
-  if (p.adapt_chunk > 0) {
-    const int most = build_prefix<true, false>(p, QL, chunk, prefix, warp_tot);
-    const int64_t groups = prefix[p.B];
-    if (groups * G > (int64_t)gridDim.x && 4 * groups >= 3 * (int64_t)p.B * most) {
-      chunk = p.adapt_chunk;
-      build_prefix<false, true>(p, QL, chunk, prefix, warp_tot);
-    }
-  } else {
-    build_prefix<false, false>(p, QL, chunk, prefix, warp_tot);
-  }
-  if (blockIdx.x == 0 && tid == 0) p.sched[2] = (uint32_t)chunk;
-  const int total_items = prefix[p.B] * (p.Hkv / HB) * (MQ ? p.q_chunks : 1);
-  pdl_launch_dependents();   // the combine kernel may be scheduled from now on
+  __syncthreads();   // the barriers are set up for every warp
+  pdl_wait_primary();
 
   if (warp == kConsumerWarps) {
+    // ---- the split size and the prefix over sequences of their work groups.
+    // The plan may offer a larger split size for calls of a few rounds of
+    // items: taken when the sequences are of about equal length (the longest
+    // one's groups times B within 4/3 of all groups), since then its items,
+    // one round of about two per SM, fill every SM alike; otherwise the
+    // plan's size runs over the grid, sized for the larger items.  Every CTA
+    // reaches the same choice from the same lengths.
+    const int G = (p.Hkv / HB) * (MQ ? p.q_chunks : 1);   // items per work group
+    int chunk = p.chunk_pages;
+    stage_lengths(p, prefix, lane);
+    if (p.adapt_chunk > 0) {
+      int groups = 0, most = 0;
+      length_totals(p, QL, chunk, prefix, lane, groups, most);
+      if ((int64_t)groups * G > (int64_t)gridDim.x &&
+          4 * (int64_t)groups >= 3 * (int64_t)p.B * most)
+        chunk = p.adapt_chunk;
+    }
+    const WorkPrefix w = build_prefix(p, QL, chunk, prefix, lane, (int)blockIdx.x / G);
+    if (blockIdx.x == 0 && lane == 0) p.sched[2] = (uint32_t)chunk;
+    pdl_launch_dependents();   // the combine kernel may be scheduled from now on
     producer_loop<D, HB, MQ, FP4>(kmap, vmap, ksmap, vsmap, p, smem, L, prefix, chunk,
-                                  total_items, hslot_bytes, full_bar, empty_bar, hdr_full,
-                                  hdr_empty, lane);
+                                  w.total * G, hslot_bytes, full_bar, empty_bar, hdr_full,
+                                  hdr_empty, lane, w);
     return;
   }
+  pdl_launch_dependents();
 
   // -------------------------------------------------------------- consumers
   // scales: host values, or device words (readable now: the grid dependency
