@@ -116,6 +116,30 @@ def test_page_permutation_bitwise():
     assert np.array_equal(out1, out2) and np.array_equal(lse1, lse2)
 
 
+# Each CTA's producer warp builds the call's work list with ceil(B / 32)
+# sequences per lane and one warp scan: batches that are not a multiple of 32,
+# lanes holding more sequences than the loads it issues back to back (8),
+# empty sequences among them, and several queries per sequence.
+MANY = [(33, 1, -1), (100, 1, 64), (1000, 1, -1), (300, 3, -1)]
+
+
+@pytest.mark.parametrize("B,Q,window", MANY, ids=[f"B{b}-q{q}-w{w}" for b, q, w in MANY])
+def test_many_sequences_per_producer_lane(B, Q, window):
+    rng = np.random.default_rng(900 + B + Q)
+    lens = rng.integers(1, 400, size=B)
+    if Q == 1:
+        lens[::7] = 0
+    wl = W.make_custom(B=B, Hq=16, Hkv=8, D=128, block_tokens=16, seq_lens=lens.tolist(),
+                       window_left=window, sinks=True, seed=910 + B, q_len=Q)
+    ref_out, ref_lse = oracle.decode_workload(wl)
+    n = B * Q
+    for chunk in (0, 3):
+        out, lse = run_cuda(wl, chunk_pages=chunk)
+        assert_parity(out.reshape(n, wl.Hq, wl.D), lse.reshape(n, wl.Hq),
+                      ref_out.reshape(n, wl.Hq, wl.D), ref_lse.reshape(n, wl.Hq),
+                      what=f"B={B} q_len={Q} window={window} chunk={chunk}")
+
+
 def test_deterministic_repeat():
     wl = W.make_workload("tiny")
     dev = to_device(wl)
