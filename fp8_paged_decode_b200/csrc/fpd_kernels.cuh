@@ -3,8 +3,10 @@
 // One persistent kernel.  Each CTA (one or more per SM) pulls work items from
 // a global counter; an item is (sequence b, group of HB KV heads, KV split)
 // and covers up to `chunk_pages` pages of that sequence's attended range.
-// Warp 4 is the producer: for every item it publishes a small header plus the
-// item's query rows (bulk copy) in a header ring, then streams the item's KV
+// Warp 4 is the producer: it first builds the call's work list alone (the
+// prefix over sequences of their splits, from seq_lens; the consumer warps
+// never wait for it), then for every item it publishes a small header plus the
+// item's query rows (bulk copy) in a header ring and streams the item's KV
 // with TMA tiled loads into a ring of shared-memory stages.  The stage ring
 // runs straight across item boundaries, so HBM reads never wait for an item to
 // start.  A stage holds 64 token rows of K and of V, in one of two shapes:
