@@ -292,9 +292,11 @@ def pin_multi_token_library(lib):
     """q_len queries per sequence against torch SDPA (float64, an explicit
     causal + window mask, the sink as an extra zero-valued key) and scipy
     logsumexp."""
-    for Q, window in ((3, -1), (4, 20), (2, 0)):
-        wl = W.make_custom(B=3, Hq=8, Hkv=2, D=64, block_tokens=16, seq_lens=[Q, 37, 90],
-                           sinks=True, window_left=window, seed=51 + Q, sm_scale=0.2,
+    # (a first sequence shorter than q_len: its earliest queries sit before the
+    # first key and see only the sink)
+    for Q, window, L0 in ((3, -1, 3), (4, 20, 4), (2, 0, 2), (5, -1, 2), (4, 1, 1)):
+        wl = W.make_custom(B=3, Hq=8, Hkv=2, D=64, block_tokens=16, seq_lens=[L0, 37, 90],
+                           sinks=True, window_left=window, seed=51 + Q + L0, sm_scale=0.2,
                            keep_dense=True, q_len=Q)
         q = wl.q
         out, lse = oracle.decode(q, wl.k_cache, wl.v_cache, wl.block_table, wl.seq_lens,
@@ -316,6 +318,8 @@ def pin_multi_token_library(lib):
             mask = torch.full((1, wl.Hq, Q, n + 1), -math.inf, dtype=torch.float64)
             for i in range(Q):
                 p = L - Q + i
+                if p < 0:
+                    continue   # no key at or before this query's position
                 lo = max(0, p - window) if window >= 0 else 0
                 mask[0, :, i, lo - s0:p + 1 - s0] = 0.0
             mask[0, :, :, n] = torch.from_numpy(sig)[:, None]
